@@ -1,0 +1,114 @@
+"""fp64 CPU oracle for Kimi Delta Attention (KDA) -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It is the plain token-by-token
+recurrence (KimiLinear article, section 2.3, KDA state-update rule) written in
+C (``kda_oracle.c``) and shares nothing with the CUDA library.
+
+Pins (tests/test_oracle_pins.py) tie it to facts other than itself: the
+gated/plain linear-attention closed form, dense brute-force products of the
+transition matrices on T <= 8, exact retrieval under the delta rule, the
+DeltaNet and Gated DeltaNet special cases, boundedness, and hand-derived
+worked examples under tests/golden/.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+
+MODE_DELTA = 0   # the KDA recurrence
+MODE_LINEAR = 1  # delta correction dropped: gated linear attention (pinning aid)
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE fp64, no fast-math) and return the .so path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, _SRC, "-lm"],
+                       check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def bind(path: str):
+    """Load an oracle shared object from ``path`` and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.kda_oracle_forward.argtypes = [dp, dp, dp, dp, dp, ctypes.c_double, dp, dp, dp] + [ctypes.c_int] * 7
+    lib.kda_oracle_forward.restype = ctypes.c_int
+    lib.kda_oracle_max_threads.argtypes = []
+    lib.kda_oracle_max_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = bind(build())
+    return _lib
+
+
+def _as_f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor (any dtype, any device): exact upcast to fp64
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def max_threads() -> int:
+    return int(_load().kda_oracle_max_threads())
+
+
+def kda_forward(q, k, v, g, beta, scale, initial_state=None, mode=MODE_DELTA, nthreads=0,
+                want_state=True, lib=None):
+    """Token-by-token fp64 KDA over [B,T,H,d] inputs.
+
+    Returns (o [B,T,H,dv] fp64, final_state [B,H,dk,dv] fp64 or None).
+    Inputs may be numpy arrays or torch tensors of any float dtype; they are
+    upcast exactly to fp64, so the oracle sees the values the GPU reads.
+    """
+    q, k, v, g, beta = (_as_f64(x) for x in (q, k, v, g, beta))
+    s0 = _as_f64(initial_state)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, T, H, dk) and g.shape == (B, T, H, dk)
+    assert v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    if s0 is not None:
+        assert s0.shape == (B, H, dk, dv)
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    sT = np.zeros((B, H, dk, dv), dtype=np.float64) if want_state else None
+    rc = (lib or _load()).kda_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                    _ptr(s0), _ptr(o), _ptr(sT), B, T, H, dk, dv, int(mode),
+                                    int(nthreads))
+    if rc != 0:
+        raise ValueError("kda_oracle_forward rejected its arguments")
+    return o, sT
+
+
+def kda_decode(q, k, v, g, beta, scale, state, nthreads=0):
+    """Decode steps: inputs [S,N,H,d] for S consecutive single-token steps.
+
+    The decode step is the same recurrence with one token per call, so it is
+    the forward pass with T = S on a [N,S,H,d] view (each sequence carries its
+    own state).  Returns (o [S,N,H,dv], final state [N,H,dk,dv]).
+    """
+    q, k, v, g, beta = (_as_f64(x) for x in (q, k, v, g, beta))
+    tr = lambda x: np.ascontiguousarray(np.swapaxes(x, 0, 1))
+    o, sT = kda_forward(tr(q), tr(k), tr(v), tr(g), tr(beta), scale, state, nthreads=nthreads)
+    return np.ascontiguousarray(np.swapaxes(o, 0, 1)), sT
