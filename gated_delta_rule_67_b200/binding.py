@@ -1,0 +1,168 @@
+"""Thin Python binding of libkda.so (include/kda.h): argument marshalling only.
+
+Every step of the operator runs in the library's CUDA kernels; this module
+checks tensor placement/dtype/contiguity, allocates outputs and workspace
+with torch when the caller did not pass them, and forwards raw device
+pointers plus the current CUDA stream.  There is no CPU fallback: without
+the compiled library or a CUDA device every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_F32, KDA_BF16 = 0, 1
+
+# Every symbol include/kda.h declares, with (restype, argtypes).
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "kda_status_string": (ctypes.c_char_p, [_i]),
+    "kda_version": (_i, []),
+    "kda_chunk_fwd_workspace_size": (_sz, [_i] * 7),
+    "kda_chunk_fwd": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp]),
+    "kda_chunk_fwd_check": (_i, [_vp, _sz, _vp]),
+    "kda_recurrent_step": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 5 + [_vp]),
+}
+
+_lib = None
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def load(path: str = LIB_PATH):
+    """Load libkda.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"libkda.so not built at {path}; run gated_delta_rule_67_b200.build.build()")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().kda_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(load().kda_version())
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return KDA_F32
+    if t == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError(f"unsupported dtype {t}; KDA takes float32 or bfloat16")
+
+
+def _check_dev(name, x, dtype=None):
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not x.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device (no CPU path exists)")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and x.dtype != dtype:
+        raise TypeError(f"{name} has dtype {x.dtype}, expected {dtype}")
+
+
+def _ptr(x):
+    return None if x is None else ctypes.c_void_p(x.data_ptr())
+
+
+def _stream(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    return int(load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, _dtype_code(dtype)))
+
+
+def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64, o=None, final_state=None,
+                  output_final_state=True, workspace=None, stream=None):
+    """Chunked KDA prefill.  q,k,g [B,T,H,dk], v [B,T,H,dv], beta [B,T,H] (fp32 or bf16, CUDA).
+
+    Returns (o [B,T,H,dv] in the input dtype, final_state [B,H,dk,dv] fp32 or None).
+    ``final_state`` may be ``initial_state`` itself for an in-place update.
+    """
+    lib = load()
+    for name, x in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
+        _check_dev(name, x, q.dtype)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != (B, T, H) or beta.shape != (B, T, H):
+        raise ValueError("shape mismatch among q, k, v, g, beta")
+    if scale is None:
+        scale = dk ** -0.5
+    code = _dtype_code(q.dtype)
+    if initial_state is not None:
+        _check_dev("initial_state", initial_state, torch.float32)
+        if initial_state.shape != (B, H, dk, dv):
+            raise ValueError("initial_state must be [B,H,dk,dv]")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _check_dev("o", o, q.dtype)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if final_state is not None:
+        _check_dev("final_state", final_state, torch.float32)
+    need = int(lib.kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
+                           _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk, code, _ptr(workspace), ws_bytes,
+                           _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd")
+    return o, final_state
+
+
+def kda_chunk_fwd_check(workspace, stream=None) -> int:
+    """Status word a bounded on-device wait may have left in ``workspace`` (synchronises)."""
+    if workspace is None:
+        return KDA_OK
+    return int(load().kda_chunk_fwd_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          _stream(stream, workspace.device)))
+
+
+def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=None):
+    """One decode step.  q,k,g [N,H,dk], v [N,H,dv], beta [N,H]; state [N,H,dk,dv] fp32 updated in place.
+
+    Returns o [N,H,dv] in the input dtype.
+    """
+    lib = load()
+    for name, x in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
+        _check_dev(name, x, q.dtype)
+    _check_dev("state", state, torch.float32)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:2] != (N, H) or beta.shape != (N, H):
+        raise ValueError("shape mismatch among q, k, v, g, beta")
+    if state.shape != (N, H, dk, dv):
+        raise ValueError("state must be [N,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    _check_dev("o", o, q.dtype)
+    st = lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(state),
+                                _ptr(o), N, H, dk, dv, _dtype_code(q.dtype), _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_recurrent_step")
+    return o

@@ -1,0 +1,159 @@
+// kda_api.cu -- the C ABI of libkda.so: host-side validation and dispatch.
+//
+// Every argument is checked here, before anything is enqueued; the kernels
+// themselves assume valid, aligned, non-overlapping buffers.
+#include <string.h>
+
+#include "kda_common.cuh"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  const char* lo;
+  size_t bytes;
+};
+
+bool overlaps(Range a, Range b) {
+  if (!a.lo || !b.lo || a.bytes == 0 || b.bytes == 0) return false;
+  return a.lo < b.lo + b.bytes && b.lo < a.lo + a.bytes;
+}
+
+size_t elem_bytes(int dtype) { return dtype == KDA_F32 ? 4 : 2; }
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+bool prefill_supported(int dk, int dv, int chunk, int dtype) {
+  if (dtype == KDA_F32)
+    return (dk == 64 || dk == 128) && (dv == 64 || dv == 128) &&
+           (chunk == 16 || chunk == 32 || chunk == 64);
+  return dk == 128 && dv == 128 && chunk == 64;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(int status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: null, misaligned, overlapping or out-of-range argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: valid arguments outside the implemented shapes/dtypes";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded on-device wait gave up";
+    default: return "KDA_ERR_UNKNOWN: not a kda_status value";
+  }
+}
+
+int kda_version(void) { return 100; }
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int dtype) {
+  if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || chunk < 1) return 0;
+  if (dtype != KDA_F32 && dtype != KDA_BF16) return 0;
+  if (!prefill_supported(dk, dv, chunk, dtype)) return 0;
+  if (dtype == KDA_BF16) return kda::prefill_bf16_workspace_bytes(B, T, H, dk, dv, chunk);
+  return 0;
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                         float scale, const float* initial_state, void* o, float* final_state, int B,
+                         int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || chunk < 1) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
+  const bool empty = (B == 0 || T == 0);
+  const size_t eb = elem_bytes(dtype);
+  const size_t ntok = (size_t)B * T * H;
+  const Range rq{(const char*)q, ntok * dk * eb}, rk{(const char*)k, ntok * dk * eb},
+      rg{(const char*)g, ntok * dk * eb}, rv{(const char*)v, ntok * dv * eb},
+      rb{(const char*)beta, ntok * eb}, ro{(const char*)o, ntok * dv * eb};
+  const size_t state_bytes = (size_t)B * H * dk * dv * sizeof(float);
+  const Range rs0{(const char*)initial_state, state_bytes}, rsT{(const char*)final_state, state_bytes};
+  if (!empty) {
+    const void* need[] = {q, k, v, g, beta, o};
+    for (const void* p : need)
+      if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    // o is written: it must not overlap any input.
+    for (Range r : {rq, rk, rg, rv, rb, rs0})
+      if (overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
+  }
+  if (initial_state && !aligned16(initial_state)) return KDA_ERR_INVALID_ARG;
+  if (final_state && !aligned16(final_state)) return KDA_ERR_INVALID_ARG;
+  if (final_state && !empty) {
+    for (Range r : {rq, rk, rg, rv, rb, ro})
+      if (overlaps(rsT, r)) return KDA_ERR_INVALID_ARG;
+    if (initial_state && (const void*)initial_state != (const void*)final_state && overlaps(rsT, rs0))
+      return KDA_ERR_INVALID_ARG;
+  }
+  if (!prefill_supported(dk, dv, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+  const size_t need_ws = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, dtype);
+  if (need_ws > 0 && !empty) {
+    if (!workspace || workspace_bytes < need_ws || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return KDA_ERR_INVALID_ARG;
+    const Range rw{(const char*)workspace, workspace_bytes};
+    for (Range r : {rq, rk, rg, rv, rb, ro, rs0, rsT})
+      if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
+  }
+
+  if (empty) {
+    // Nothing to run: the final state is the initial state (or zeros).
+    if (!final_state || state_bytes == 0) return KDA_OK;
+    if (initial_state == final_state) return KDA_OK;
+    cudaError_t e = initial_state
+                        ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, stream)
+                        : cudaMemsetAsync(final_state, 0, state_bytes, stream);
+    return from_cuda(e);
+  }
+
+  cudaError_t e;
+  if (dtype == KDA_F32) {
+    e = kda::launch_prefill_f32((const float*)q, (const float*)k, (const float*)v, (const float*)g,
+                                (const float*)beta, scale, initial_state, (float*)o, final_state, B, T,
+                                H, dk, dv, chunk, stream);
+  } else {
+    e = kda::launch_prefill_bf16((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                 (const __nv_bfloat16*)v, (const __nv_bfloat16*)g,
+                                 (const __nv_bfloat16*)beta, scale, initial_state, (__nv_bfloat16*)o,
+                                 final_state, B, T, H, dk, dv, chunk, workspace, workspace_bytes, stream);
+  }
+  return from_cuda(e);
+}
+
+kda_status kda_chunk_fwd_check(const void* workspace, size_t workspace_bytes, void* stream_) {
+  if (!workspace || workspace_bytes < sizeof(kda::WorkspaceHeader)) return KDA_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  kda::WorkspaceHeader h;
+  cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return KDA_ERR_CUDA;
+  return h.error ? KDA_ERR_TIMEOUT : KDA_OK;
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g,
+                              const void* beta, float scale, float* state, void* o, int N, int H,
+                              int dk, int dv, int dtype, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (N < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
+  if (N == 0) return KDA_OK;
+  const void* need[] = {q, k, v, g, beta, state, o};
+  for (const void* p : need)
+    if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  const size_t eb = elem_bytes(dtype);
+  const size_t nh = (size_t)N * H;
+  const Range rq{(const char*)q, nh * dk * eb}, rk{(const char*)k, nh * dk * eb},
+      rg{(const char*)g, nh * dk * eb}, rv{(const char*)v, nh * dv * eb}, rb{(const char*)beta, nh * eb},
+      ro{(const char*)o, nh * dv * eb}, rs{(const char*)state, nh * dk * dv * sizeof(float)};
+  for (Range r : {rq, rk, rg, rv, rb, rs})
+    if (overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
+  for (Range r : {rq, rk, rg, rv, rb})
+    if (overlaps(rs, r)) return KDA_ERR_INVALID_ARG;
+  if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+  return from_cuda(kda::launch_decode(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, stream));
+}
+
+}  // extern "C"

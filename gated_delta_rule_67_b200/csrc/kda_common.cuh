@@ -1,0 +1,51 @@
+// kda_common.cuh -- small helpers shared by the KDA kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Element loads/stores for the two supported I/O types.
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Launch entry points implemented in the individual .cu files.  Arguments
+// have been validated by the API layer.  Each returns the cudaError_t of its
+// launch(es).
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                          float scale, float* state, void* o, int N, int H, int dk, int dv, int dtype,
+                          cudaStream_t stream);
+
+cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* g,
+                               const float* beta, float scale, const float* s0, float* o, float* sT,
+                               int B, int T, int H, int dk, int dv, int chunk, cudaStream_t stream);
+
+// bf16 chunked prefill (tcgen05 path).  `ws` is the caller's workspace.
+size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk);
+cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                const __nv_bfloat16* g, const __nv_bfloat16* beta, float scale,
+                                const float* s0, __nv_bfloat16* o, float* sT, int B, int T, int H,
+                                int dk, int dv, int chunk, void* ws, size_t ws_bytes,
+                                cudaStream_t stream);
+
+// Every workspace starts with this header; kernels that wait on barriers with
+// an iteration limit record a give-up here instead of hanging.
+struct WorkspaceHeader {
+  unsigned int error;      // 0 = fine, nonzero = a bounded wait gave up
+  unsigned int where;      // which wait (kernel-specific code)
+  unsigned int pad[62];    // keeps the payload 256-byte aligned
+};
+static_assert(sizeof(WorkspaceHeader) == 256, "workspace header is 256 bytes");
+
+}  // namespace kda

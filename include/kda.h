@@ -1,0 +1,126 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention library, libkda.so.
+ *
+ * The operator (KimiLinear: A Next-Generation Linear Attention Architecture
+ * for Long-Context LLMs, section 2.3) is the per-head recurrence
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t
+ *
+ * with the state S a d_k x d_v fp32 matrix (row = key channel, column = value
+ * channel), g_t = log of the per-channel forget gate (acting on the rows of S;
+ * g_t <= 0 for a gate in (0, 1]), beta_t a scalar write strength per token
+ * and head, and o_t read from the state after token t has been written.
+ *
+ * Conventions shared by every call:
+ *  - All tensors are dense, contiguous, row-major device buffers owned by the
+ *    caller; the library allocates nothing and keeps no state between calls.
+ *  - Every pointer must be 16-byte aligned.
+ *  - `dtype` is the element type of q, k, v, g, beta and o (fp32 or bf16);
+ *    the state is always fp32.  bf16 results are rounded to nearest-even.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls only enqueue work on it; none synchronises the host.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call enqueues nothing.  No call raises an exception across the
+ *    ABI and no kernel uses device assertions.
+ *  - Results are deterministic: no atomics take part in any accumulation.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, aliasing not allowed */
+  KDA_ERR_UNSUPPORTED = 2, /* valid arguments outside what the kernels implement */
+  KDA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  KDA_ERR_TIMEOUT = 4      /* a bounded on-device wait gave up (reported by kda_chunk_fwd_check) */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+KDA_API const char* kda_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+KDA_API int kda_version(void);
+
+/*
+ * Bytes of device workspace kda_chunk_fwd needs for this problem (0 if none).
+ * Returns 0 as well for arguments kda_chunk_fwd would reject.
+ */
+KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int dtype);
+
+/*
+ * Chunked prefill: runs the recurrence over T tokens for B sequences x H heads.
+ *
+ * Defined by the KDA update (section 2.3) evaluated with the chunkwise
+ * parallel algorithm of the same article (section 3.1): the sequence is cut
+ * into chunks of `chunk` tokens; inside a chunk the token interactions are
+ * dense matrix products, across chunks the state is carried recursively.
+ * The chunk size does not change the result (up to rounding); a last partial
+ * chunk of T mod chunk tokens is handled.
+ *
+ *   q, k, g       : [B, T, H, dk]   (dtype)
+ *   v             : [B, T, H, dv]   (dtype)
+ *   beta          : [B, T, H]       (dtype)
+ *   scale         : output scale (commonly 1/sqrt(dk)); it does not touch the state
+ *   initial_state : [B, H, dk, dv] fp32, or NULL for a zero state
+ *   o             : [B, T, H, dv]   (dtype), written
+ *   final_state   : [B, H, dk, dv] fp32, or NULL to skip; may be the same
+ *                   buffer as initial_state (updated in place); must not
+ *                   overlap any other argument
+ *   workspace     : device buffer of at least kda_chunk_fwd_workspace_size()
+ *                   bytes (NULL allowed when that size is 0); its contents
+ *                   on entry do not matter; it must not be shared by two
+ *                   calls in flight at the same time
+ *
+ * Supported: dtype KDA_F32 with dk, dv in {64, 128} (any chunk in {16, 32, 64});
+ * dtype KDA_BF16 with dk = dv = 128 and chunk = 64.  Anything else with valid
+ * shapes returns KDA_ERR_UNSUPPORTED.  T = 0 or B = 0 is valid (the final state
+ * is the initial state).
+ */
+KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                         float scale, const float* initial_state, void* o, float* final_state, int B,
+                         int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * Reads the on-device error word that the last kda_chunk_fwd using this
+ * workspace left behind (synchronises `stream`).  Returns KDA_OK, or
+ * KDA_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the outputs of
+ * that call are then not valid).  A workspace of size 0 always reports KDA_OK.
+ */
+KDA_API kda_status kda_chunk_fwd_check(const void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Single-token decode (O(1) per token, constant-size state: same article,
+ * section 4.2): one step of the recurrence for N sequences x H heads, with
+ * the state updated in place.
+ *
+ *   q, k, g : [N, H, dk] (dtype)     v, o : [N, H, dv] (dtype)     beta : [N, H] (dtype)
+ *   state   : [N, H, dk, dv] fp32, read and overwritten with the new state
+ *
+ * Supported: dk, dv in {64, 128}, dtype KDA_F32 or KDA_BF16.
+ */
+KDA_API kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g,
+                              const void* beta, float scale, float* state, void* o, int N, int H,
+                              int dk, int dv, int dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

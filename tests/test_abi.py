@@ -1,0 +1,109 @@
+"""The C ABI on the host: the library loads, exports every declared symbol,
+and rejects bad arguments before touching the GPU (no device needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_67_b200 import binding
+from gated_delta_rule_67_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_symbols() == sorted(binding.SIGNATURES)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert binding.status_string(s).startswith("KDA_")
+    assert "UNKNOWN" in binding.status_string(99)
+    assert binding.version() >= 100
+
+
+def test_workspace_size_rejects_bad_args(lib):
+    f = lib.kda_chunk_fwd_workspace_size
+    assert f(1, 64, 1, 128, 128, 64, 9) == 0      # bad dtype
+    assert f(-1, 64, 1, 128, 128, 64, 1) == 0     # bad B
+    assert f(1, 64, 1, 96, 96, 64, 1) == 0        # unsupported d
+    assert f(1, 64, 1, 64, 64, 64, 0) == 0        # fp32 path needs none
+
+
+# Fake device addresses: validation must fail before any CUDA call is made.
+A = 1 << 40
+
+
+def _fwd(lib, q=A, k=A + (1 << 30), v=A + (2 << 30), g=A + (3 << 30), beta=A + (4 << 30), s0=None,
+         o=A + (5 << 30), sT=None, B=1, T=64, H=1, dk=128, dv=128, chunk=64, dtype=1, ws=None, wsb=0, scale=1.0):
+    return lib.kda_chunk_fwd(q, k, v, g, beta, scale, s0, o, sT, B, T, H, dk, dv, chunk, dtype, ws, wsb, None)
+
+
+def test_chunk_fwd_rejects_null_and_misaligned(lib):
+    assert _fwd(lib, q=None) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, o=None) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, k=A + 8) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, s0=A + (6 << 30) + 4) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, T=-1) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, H=0) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, dtype=5) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan")) == binding.KDA_ERR_INVALID_ARG
+
+
+def test_chunk_fwd_rejects_overlap(lib):
+    assert _fwd(lib, o=A + 64) == binding.KDA_ERR_INVALID_ARG                 # o overlaps q
+    assert _fwd(lib, sT=A + (2 << 30)) == binding.KDA_ERR_INVALID_ARG         # final state overlaps v
+
+
+def test_chunk_fwd_unsupported_shapes(lib):
+    assert _fwd(lib, dk=96, dv=96) == binding.KDA_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=0, chunk=48, dk=64, dv=64) == binding.KDA_ERR_UNSUPPORTED
+    assert _fwd(lib, dtype=0, dk=64, dv=32) == binding.KDA_ERR_UNSUPPORTED
+
+
+def test_chunk_fwd_workspace_checked(lib):
+    need = lib.kda_chunk_fwd_workspace_size(1, 64, 1, 128, 128, 64, 1)
+    if need == 0:
+        pytest.skip("bf16 path needs no workspace")
+    assert _fwd(lib, ws=None, wsb=0) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, ws=A + (7 << 30), wsb=need - 1) == binding.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, ws=A + (7 << 30) + 16, wsb=need) == binding.KDA_ERR_INVALID_ARG  # not 256-aligned
+
+
+def test_recurrent_step_validation(lib):
+    f = lib.kda_recurrent_step
+    args = [A, A + (1 << 30), A + (2 << 30), A + (3 << 30), A + (4 << 30), 1.0, A + (5 << 30), A + (6 << 30)]
+    assert f(*args, 0, 1, 128, 128, 1, None) == binding.KDA_OK          # N = 0: nothing to do
+    bad = list(args)
+    bad[0] = None
+    assert f(*bad, 4, 1, 128, 128, 1, None) == binding.KDA_ERR_INVALID_ARG
+    bad = list(args)
+    bad[7] = A + 32                                                        # o overlaps q
+    assert f(*bad, 4, 1, 128, 128, 1, None) == binding.KDA_ERR_INVALID_ARG
+    assert f(*args, 4, 1, 96, 128, 1, None) == binding.KDA_ERR_UNSUPPORTED
+    assert f(*args, 4, 1, 128, 128, 3, None) == binding.KDA_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
