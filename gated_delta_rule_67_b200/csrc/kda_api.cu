@@ -9,6 +9,7 @@
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 struct Range {
   const char* lo;
@@ -73,9 +74,10 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
   const size_t state_bytes = (size_t)B * H * dk * dv * sizeof(float);
   const Range rs0{(const char*)initial_state, state_bytes}, rsT{(const char*)final_state, state_bytes};
   if (!empty) {
-    const void* need[] = {q, k, v, g, beta, o};
+    const void* need[] = {q, k, v, g, o};
     for (const void* p : need)
       if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!beta || !aligned_to(beta, eb)) return KDA_ERR_INVALID_ARG;
     // o is written: it must not overlap any input.
     for (Range r : {rq, rk, rg, rv, rb, rs0})
       if (overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
@@ -140,10 +142,11 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
   if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
   if (N == 0) return KDA_OK;
-  const void* need[] = {q, k, v, g, beta, state, o};
+  const size_t eb = elem_bytes(dtype);
+  const void* need[] = {q, k, v, g, state, o};
   for (const void* p : need)
     if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
-  const size_t eb = elem_bytes(dtype);
+  if (!beta || !aligned_to(beta, eb)) return KDA_ERR_INVALID_ARG;
   const size_t nh = (size_t)N * H;
   const Range rq{(const char*)q, nh * dk * eb}, rk{(const char*)k, nh * dk * eb},
       rg{(const char*)g, nh * dk * eb}, rv{(const char*)v, nh * dv * eb}, rb{(const char*)beta, nh * eb},

@@ -15,7 +15,8 @@
  * Conventions shared by every call:
  *  - All tensors are dense, contiguous, row-major device buffers owned by the
  *    caller; the library allocates nothing and keeps no state between calls.
- *  - Every pointer must be 16-byte aligned.
+ *  - Every pointer must be 16-byte aligned, except beta, which needs only the
+ *    alignment of its element type (so a sequence may be cut at any token).
  *  - `dtype` is the element type of q, k, v, g, beta and o (fp32 or bf16);
  *    the state is always fp32.  bf16 results are rounded to nearest-even.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).

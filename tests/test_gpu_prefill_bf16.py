@@ -1,0 +1,129 @@
+"""bf16 chunked prefill (tcgen05 path) against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_67_b200 import kda_chunk_fwd, kda_chunk_fwd_check, kda_chunk_fwd_workspace_size
+from gated_delta_rule_67_b200.workloads import (LONG_BF16, PREFILL_BF16, TRAIN_BF16, make_config_inputs,
+                                                make_prefill_inputs)
+from tests.parity import TOL, cuda_or_skip, rel_err
+
+pytestmark = pytest.mark.gpu
+TOLB = TOL[torch.bfloat16]
+NAMES = ("q", "k", "v", "g", "beta")
+
+
+def _run(x, dev, scale=None, ws=None):
+    d = x["q"].shape[-1]
+    scale = d ** -0.5 if scale is None else scale
+    s0 = None if x["initial_state"] is None else x["initial_state"].to(dev)
+    o, sT = kda_chunk_fwd(*(x[n].to(dev) for n in NAMES), scale, s0, workspace=ws)
+    torch.cuda.synchronize()
+    return o, sT
+
+
+def _oracle(x, scale=None):
+    d = x["q"].shape[-1]
+    scale = d ** -0.5 if scale is None else scale
+    return oracle.kda_forward(*(x[n] for n in NAMES), scale, x["initial_state"])
+
+
+@pytest.mark.parametrize("B,T,H,s0", [(1, 64, 1, 0.1), (1, 64, 2, 0.0), (2, 200, 3, 0.1), (1, 1, 2, 0.1),
+                                      (1, 127, 2, 0.1), (3, 320, 2, 0.0)])
+def test_small_shapes(B, T, H, s0):
+    """One chunk, several chunks, a ragged tail, a single token, zero and random initial state."""
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(B, T, H, 128, 128, torch.bfloat16, s0, seed=41 + T, device="cpu")
+    o, sT = _run(x, dev)
+    ref_o, ref_s = _oracle(x)
+    assert rel_err(o, ref_o) < TOLB
+    assert rel_err(sT, ref_s) < TOLB
+
+
+def test_prefill_config_full():
+    """B=1, H=16, T=4096, d=128, random initial state: every output against the oracle."""
+    dev = cuda_or_skip()
+    x = make_config_inputs(PREFILL_BF16, device="cpu")
+    o, sT = _run(x, dev)
+    ref_o, ref_s = _oracle(x)
+    assert rel_err(o, ref_o) < TOLB
+    assert rel_err(sT, ref_s) < TOLB
+
+
+def _sampled(cfg, pairs, zero_state=False):
+    dev = cuda_or_skip()
+    x = make_config_inputs(cfg, device=dev)
+    if zero_state:
+        x["initial_state"] = None
+    o, sT = _run(x, dev)
+    for b, h in pairs:
+        sel = {n: x[n][b:b + 1, :, h:h + 1] for n in NAMES}
+        sel["initial_state"] = None if x["initial_state"] is None else x["initial_state"][b:b + 1, h:h + 1]
+        ref_o, ref_s = _oracle(sel)
+        assert rel_err(o[b:b + 1, :, h:h + 1], ref_o) < TOLB, (b, h)
+        assert rel_err(sT[b:b + 1, h:h + 1], ref_s) < TOLB, (b, h)
+
+
+def test_train_config_sampled_heads():
+    """B=8, H=32, T=8192 in one launch; the oracle checks a sample of (sequence, head) chains in full."""
+    rng = np.random.default_rng(7)
+    pairs = [(0, 0), (7, 31)] + [(int(b), int(h)) for b, h in zip(rng.integers(0, 8, 3), rng.integers(0, 32, 3))]
+    _sampled(TRAIN_BF16, pairs)
+
+
+def test_train_config_zero_state_sampled():
+    _sampled(TRAIN_BF16, [(3, 5), (6, 17)], zero_state=True)
+
+
+def test_long_context_sampled_head():
+    """T = 1,048,576 (16384 chunks carried in one chain); the oracle follows one head end to end."""
+    _sampled(LONG_BF16, [(0, 13)])
+
+
+def test_split_calls_and_in_place_state():
+    """Cutting the sequence (at a chunk boundary and inside a chunk) and carrying
+    final_state -> initial_state in place matches one call."""
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(2, 300, 2, 128, 128, torch.bfloat16, 0.1, seed=44, device=dev)
+    o_full, s_full = kda_chunk_fwd(*(x[n] for n in NAMES), None, x["initial_state"])
+    state = x["initial_state"].clone()
+    outs = []
+    for a, b in ((0, 64), (64, 101), (101, 300)):
+        part = [x[n][:, a:b].contiguous() for n in NAMES]
+        oo, _ = kda_chunk_fwd(*part, None, state, final_state=state)
+        outs.append(oo)
+    torch.cuda.synchronize()
+    ref_o, ref_s = _oracle({n: x[n] for n in NAMES} | {"initial_state": x["initial_state"]})
+    assert rel_err(torch.cat(outs, dim=1), ref_o) < TOLB
+    assert rel_err(state, ref_s) < TOLB
+    assert rel_err(o_full, ref_o) < TOLB
+
+
+def test_matches_decode_steps():
+    """A prefill over T tokens equals T single-token decode steps (GPU vs GPU)."""
+    from gated_delta_rule_67_b200 import kda_recurrent_step
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(2, 96, 4, 128, 128, torch.bfloat16, 0.1, seed=45, device=dev)
+    o_p, s_p = kda_chunk_fwd(*(x[n] for n in NAMES), None, x["initial_state"])
+    state = x["initial_state"].clone()
+    o_d = torch.stack([kda_recurrent_step(*(x[n][:, t].contiguous() for n in NAMES), state)
+                       for t in range(96)], dim=1)
+    torch.cuda.synchronize()
+    assert rel_err(o_p, o_d) < TOLB
+    assert rel_err(s_p, state) < TOLB
+
+
+def test_workspace_reuse_and_check():
+    """A caller-provided workspace can be reused; the on-device error word stays clear."""
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(1, 256, 2, 128, 128, torch.bfloat16, 0.1, seed=46, device="cpu")
+    need = kda_chunk_fwd_workspace_size(1, 256, 2, 128, 128)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws.fill_(0xAB)
+    o1, s1 = _run(x, dev, ws=ws)
+    assert kda_chunk_fwd_check(ws) == 0
+    o2, s2 = _run(x, dev, ws=ws)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)  # deterministic
+    ref_o, ref_s = _oracle(x)
+    assert rel_err(o1, ref_o) < TOLB and rel_err(s1, ref_s) < TOLB
