@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the B200 KDA library (kda_chunk_fwd / kda_recurrent_step).
+
+One step = one kda_chunk_fwd over the bf16 prefill workload (B=1, H=16,
+T=4096, d=128, chunk 64, random initial state): in-chunk gate cumsum and
+decay factors, the C x C score matrices, the triangular (UT/WY) solve, the
+W/U products, the sequential state pass and the outputs.  The single-token
+decode kernel is measured in the same run on its own workload (256
+sequences x 32 heads, d=128, 1000 consecutive steps) and reported under
+"decode".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs the same workload on
+its own seeded sequences: the units are independent, so there is no
+collective on the data path ("scaling": "weak"); timing is the device time
+of each rank, max over ranks.  `--impl reference` times the fp64 CPU oracle
+(the only reference this operator has) on the same workload and prints its
+line from rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s & TFLOP/s (% bf16 peak); decode GB/s (% HBM peak), 1×B200"
+DATA = ("synthetic, seeded: q,k ~N(0,1) L2-normalised per token; v ~N(0,1); beta=sigmoid(N(0,1)); "
+        "g=logsigmoid(N(3,1)) per channel; S0 ~N(0,0.1^2)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- accounting
+def prefill_flops_per_token_head(d: int, C: int = 64) -> float:
+    """Algorithmic FLOPs of the chunked method per token and head (triangle-aware):
+    A_kk, A_qk, the triangular inverse, W, U, A_qk V' and the three state-pass
+    products, divided by the chunk length."""
+    akk = 2 * C * (C - 1) / 2 * d
+    aqk = 2 * C * (C + 1) / 2 * d
+    tri = 3 * 2 * C * (C + 1) / 2 * d
+    inv = C * (C - 1) * (C - 2) / 3  # forward substitution of the unit triangle, 83,328 at C=64
+    state = 3 * 2 * C * d * d
+    return (akk + aqk + tri + inv + state) / C
+
+
+def prefill_bytes(B, T, H, dk, dv, elem=2, state_in=True, state_out=True) -> float:
+    """Algorithmic HBM bytes of one call: q,k,g,v,beta read, o written, the fp32 state read/written once."""
+    per_tok = (3 * dk + dv + 1 + dv) * elem
+    st = B * H * dk * dv * 4
+    return B * T * H * per_tok + st * (int(state_in) + int(state_out))
+
+
+def decode_bytes(N, H, dk, dv, elem=2) -> float:
+    return N * H * (2 * dk * dv * 4 + (3 * dk + 2 * dv + 1) * elem)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def weak_scaling_value(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max of a float over all ranks (no-op without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled in the background."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, interval_ms: int = 20):
+        self.path = tempfile.mktemp(prefix="kda_clocks_", suffix=".csv")
+        self.proc = None
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", f"-lms", str(interval_ms)],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- oracle leg
+def oracle_throughput(cfg, tokens: int, nthreads: int = 0):
+    """Times the fp64 oracle on all heads of the workload's first `tokens`
+    tokens; returns (tokens/s of the workload, seconds, threads)."""
+    import oracle
+    from gated_delta_rule_67_b200.workloads import make_config_inputs
+    x = make_config_inputs(cfg, device="cpu", T=tokens)
+    args = [x[n] for n in ("q", "k", "v", "g", "beta")]
+    import numpy as np
+    f64 = [np.ascontiguousarray(a.double().numpy()) for a in args]
+    s0 = None if x["initial_state"] is None else x["initial_state"].double().numpy()
+    t0 = time.perf_counter()
+    oracle.kda_forward(*f64, cfg.scale, s0, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return cfg.B * tokens / dt, dt, oracle.max_threads() if nthreads <= 0 else nthreads
+
+
+def run_reference(args, cfg):
+    """The reference arm: the fp64 oracle on the host cores, same workload/metric."""
+    import oracle
+    oracle.build()
+    # Size each step's sample so the whole --steps/--warmup run takes about a minute.
+    probe_tok = 64
+    _, dt_probe, cores = oracle_throughput(cfg, probe_tok)
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    tokens = int(max(16, min(cfg.T, probe_tok * budget / max(dt_probe, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_throughput(cfg, tokens)
+    times = []
+    for _ in range(args.steps):
+        _, dt, cores = oracle_throughput(cfg, tokens)
+        times.append(dt)
+    total = sum(times)
+    value = cfg.B * tokens * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv,
+                   "chunk": cfg.chunk},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"all {cfg.H} heads x first {tokens} of {cfg.T} tokens per step "
+                                   f"(fp64 token-by-token recurrence, OpenMP over heads x 16-column blocks)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- our arm
+def traffic_from_profile(kernel_sources):
+    """DRAM bytes per call from the committed ncu summary, if it was taken on
+    the kernel sources as they are now (else None)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None, None
+    with open(p) as f:
+        d = json.load(f)
+    h = hashlib.sha256()
+    for s in kernel_sources:
+        with open(os.path.join(ROOT, s), "rb") as fh:
+            h.update(fh.read())
+    if d.get("source_sha256") != h.hexdigest():
+        return None, d
+    return d, d
+
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+    from gated_delta_rule_67_b200 import (kda_chunk_fwd, kda_chunk_fwd_workspace_size, kda_recurrent_step)
+    from gated_delta_rule_67_b200.workloads import DECODE_BF16, make_decode_inputs, make_prefill_inputs
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    peaks, peaks_kind = load_peaks()
+
+    # ---- inputs (independent sequences per rank)
+    x = make_prefill_inputs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.torch_dtype, cfg.s0_std,
+                            seed=cfg.seed + 1000 * rank, device=dev)
+    names = ("q", "k", "v", "g", "beta")
+    ins = [x[n] for n in names]
+    s0 = x["initial_state"]
+    o = torch.empty_like(x["v"])
+    sT = torch.empty_like(s0)
+    ws = torch.empty(max(1, kda_chunk_fwd_workspace_size(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.chunk,
+                                                           cfg.torch_dtype)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB of L2
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        kda_chunk_fwd(*ins, cfg.scale, s0, chunk=cfg.chunk, o=o, final_state=sT, workspace=ws, events=evs)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for trip in evs:  # materialise the event handles
+        for e in trip:
+            e.record(stream)
+    torch.cuda.synchronize()
+
+    gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = gpu_id if gpu_id.startswith("GPU-") else "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()  # between timed iterations, outside the recorded events
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    clocks = sampler.summary()
+
+    step_ms = [a.elapsed_time(c) for a, _, c in evs]
+    prep_ms = [a.elapsed_time(b) for a, b, _ in evs]
+    state_ms = [b.elapsed_time(c) for _, b, c in evs]
+    total_s = reduce_max(sum(step_ms) / 1e3, dev)
+    tokens = cfg.B * cfg.T
+    value = weak_scaling_value(tokens * args.steps, world, total_s)
+    ms_per_step = 1e3 * total_s / args.steps
+    flops = prefill_flops_per_token_head(cfg.dk) * tokens * cfg.H
+    nbytes = prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, 2, s0 is not None, True)
+    mean_prep, mean_state = statistics.mean(prep_ms), statistics.mean(state_ms)
+    dom = "kda_state_pass" if mean_state >= mean_prep else "kda_chunk_prep"
+
+    # ---- roofline of the operator call (both kernels together)
+    call_s = ms_per_step / 1e3
+    achieved = nbytes / call_s / 1e9
+    prof, prof_any = traffic_from_profile(["gated_delta_rule_67_b200/csrc/kda_prefill_bf16.cu",
+                                           "gated_delta_rule_67_b200/csrc/sm100.cuh"])
+    traffic = None if prof is None else prof.get("bytes_per_call", {}).get(cfg.name)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "scope": "whole kda_chunk_fwd call (kda_chunk_prep + kda_state_pass), algorithmic bytes "
+                         f"{nbytes / 1e6:.2f} MB per call; peak = {peaks_kind} hbm_gbs",
+                "kernels": {"kda_chunk_prep": {"ms": mean_prep, "share": mean_prep / (mean_prep + mean_state)},
+                            "kda_state_pass": {"ms": mean_state, "share": mean_state / (mean_prep + mean_state)}},
+                "dominant": dom}
+    tflops = flops / call_s / 1e12
+
+    # ---- end to end through the public API with pinned host buffers
+    h_ins = [t.cpu().pin_memory() for t in ins]
+    h_s0 = s0.cpu().pin_memory()
+    h_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    h_sT = torch.empty(sT.shape, dtype=sT.dtype, pin_memory=True)
+    d_ins = [torch.empty_like(t) for t in ins]
+    d_s0 = torch.empty_like(s0)
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        for d, hsrc in zip(d_ins, h_ins):
+            d.copy_(hsrc, non_blocking=True)
+        d_s0.copy_(h_s0, non_blocking=True)
+        kda_chunk_fwd(*d_ins, cfg.scale, d_s0, chunk=cfg.chunk, o=o, final_state=sT, workspace=ws)
+        h_o.copy_(o, non_blocking=True)
+        h_sT.copy_(sT, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    eb.record()
+    torch.cuda.synchronize()
+    e2e_s = reduce_max(ea.elapsed_time(eb) / 1e3, dev)
+    h2d = sum(t.numel() * t.element_size() for t in h_ins) + h_s0.numel() * 4
+    d2h = h_o.numel() * h_o.element_size() + h_sT.numel() * 4
+    e2e = {"value": weak_scaling_value(tokens * e2e_steps, world, e2e_s), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+    del h_ins, d_ins
+
+    # ---- decode kernel on its own workload
+    decode = None
+    if not args.no_decode:
+        dc = DECODE_BF16
+        nsteps = args.decode_steps
+        y = make_decode_inputs(nsteps, dc.N, dc.H, dc.dk, dc.dv, dc.torch_dtype, dc.s0_std, dc.seed + rank, dev)
+        st = y["state"]
+        od = torch.empty((dc.N, dc.H, dc.dv), dtype=dc.torch_dtype, device=dev)
+        for t in range(min(5, nsteps)):
+            kda_recurrent_step(y["q"][t], y["k"][t], y["v"][t], y["g"][t], y["beta"][t], st, dc.scale, o=od)
+        torch.cuda.synchronize()
+        da, db = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        da.record()
+        for t in range(nsteps):
+            kda_recurrent_step(y["q"][t], y["k"][t], y["v"][t], y["g"][t], y["beta"][t], st, dc.scale, o=od)
+        db.record()
+        torch.cuda.synchronize()
+        d_s = reduce_max(da.elapsed_time(db) / 1e3, dev) / nsteps
+        gbs = decode_bytes(dc.N, dc.H, dc.dk, dc.dv) / d_s / 1e9
+        decode = {"workload": dc.name, "us_per_step": d_s * 1e6, "steps": nsteps,
+                  "value": gbs * world, "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                  "tokens_per_s": dc.N * world / d_s, "kernel": "decode_step_kernel (1 launch/step)",
+                  "bytes_per_step": decode_bytes(dc.N, dc.H, dc.dk, dc.dv)}
+        del y
+
+    # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ctoks = min(cfg.T, args.cpu_tokens)
+        v, dt, cores = oracle_throughput(cfg, ctoks)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"all {cfg.H} heads x first {ctoks} of {cfg.T} tokens, one pass ({dt:.2f} s), "
+                         f"fp64 token-by-token recurrence"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": DATA,
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv,
+                       "chunk": cfg.chunk, "l2": "flushed (256 MiB write) between timed steps",
+                       "parallelism": f"dp{world}: independent sequences per GPU, no collective"},
+            "tflops": tflops, "tflops_frac_bf16": tflops / peaks["bf16_tflops"],
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
+            "clocks": clocks, "decode": decode,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    from gated_delta_rule_67_b200.workloads import PREFILL_BF16, PREFILL_CONFIGS
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=PREFILL_BF16.name, choices=sorted(PREFILL_CONFIGS))
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=4096)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    cfg = PREFILL_CONFIGS[args.workload]
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", 0)) != 0:
+            return 0
+        run_reference(args, cfg)
+        return 0
+    run_ours(args, cfg)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -26,6 +26,7 @@ SIGNATURES = {
     "kda_version": (_i, []),
     "kda_chunk_fwd_workspace_size": (_sz, [_i] * 7),
     "kda_chunk_fwd": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp]),
+    "kda_chunk_fwd_profiled": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp, _vp]),
     "kda_chunk_fwd_check": (_i, [_vp, _sz, _vp]),
     "kda_recurrent_step": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 5 + [_vp]),
 }
@@ -94,11 +95,13 @@ def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16
 
 
 def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64, o=None, final_state=None,
-                  output_final_state=True, workspace=None, stream=None):
+                  output_final_state=True, workspace=None, stream=None, events=None):
     """Chunked KDA prefill.  q,k,g [B,T,H,dk], v [B,T,H,dv], beta [B,T,H] (fp32 or bf16, CUDA).
 
     Returns (o [B,T,H,dv] in the input dtype, final_state [B,H,dk,dv] fp32 or None).
     ``final_state`` may be ``initial_state`` itself for an in-place update.
+    ``events``: optional three recorded torch.cuda.Event objects; the library
+    records them before, between and after its kernels (kda_chunk_fwd_profiled).
     """
     lib = load()
     for name, x in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
@@ -125,9 +128,15 @@ def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64,
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
-                           _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk, code, _ptr(workspace), ws_bytes,
-                           _stream(stream, q.device))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state), _ptr(o),
+            _ptr(final_state), B, T, H, dk, dv, chunk, code, _ptr(workspace), ws_bytes, _stream(stream, q.device))
+    if events is None:
+        st = lib.kda_chunk_fwd(*args)
+    else:
+        if len(events) != 3:
+            raise ValueError("events must hold three torch.cuda.Event objects")
+        handles = (ctypes.c_void_p * 3)(*[ev.cuda_event for ev in events])
+        st = lib.kda_chunk_fwd_profiled(*args, handles)
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd")
     return o, final_state

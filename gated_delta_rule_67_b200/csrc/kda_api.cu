@@ -57,10 +57,10 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chu
   return 0;
 }
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                         float scale, const float* initial_state, void* o, float* final_state, int B,
-                         int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
-                         size_t workspace_bytes, void* stream_) {
+static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                 float scale, const float* initial_state, void* o, float* final_state, int B,
+                                 int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
+                                 size_t workspace_bytes, void* stream_, void* const* events) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || chunk < 1) return KDA_ERR_INVALID_ARG;
   if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
@@ -100,13 +100,16 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
       if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
   }
 
+  if (events)
+    for (int i = 0; i < 3; ++i)
+      if (!events[i]) return KDA_ERR_INVALID_ARG;
   if (empty) {
     // Nothing to run: the final state is the initial state (or zeros).
-    if (!final_state || state_bytes == 0) return KDA_OK;
-    if (initial_state == final_state) return KDA_OK;
-    cudaError_t e = initial_state
-                        ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, stream)
+    cudaError_t e = cudaSuccess;
+    if (final_state && state_bytes && initial_state != final_state)
+      e = initial_state ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, stream)
                         : cudaMemsetAsync(final_state, 0, state_bytes, stream);
+    for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = kda::mark(events, i, stream);
     return from_cuda(e);
   }
 
@@ -114,14 +117,32 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
   if (dtype == KDA_F32) {
     e = kda::launch_prefill_f32((const float*)q, (const float*)k, (const float*)v, (const float*)g,
                                 (const float*)beta, scale, initial_state, (float*)o, final_state, B, T,
-                                H, dk, dv, chunk, stream);
+                                H, dk, dv, chunk, stream, events);
   } else {
     e = kda::launch_prefill_bf16((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                  (const __nv_bfloat16*)v, (const __nv_bfloat16*)g,
                                  (const __nv_bfloat16*)beta, scale, initial_state, (__nv_bfloat16*)o,
-                                 final_state, B, T, H, dk, dv, chunk, workspace, workspace_bytes, stream);
+                                 final_state, B, T, H, dk, dv, chunk, workspace, workspace_bytes, stream,
+                                 events);
   }
   return from_cuda(e);
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                         float scale, const float* initial_state, void* o, float* final_state, int B,
+                         int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return chunk_fwd_impl(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
+                        workspace, workspace_bytes, stream, nullptr);
+}
+
+kda_status kda_chunk_fwd_profiled(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                  float scale, const float* initial_state, void* o, float* final_state, int B,
+                                  int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream, void* const* events) {
+  if (!events) return KDA_ERR_INVALID_ARG;
+  return chunk_fwd_impl(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
+                        workspace, workspace_bytes, stream, events);
 }
 
 kda_status kda_chunk_fwd_check(const void* workspace, size_t workspace_bytes, void* stream_) {

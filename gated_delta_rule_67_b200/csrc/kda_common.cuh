@@ -29,7 +29,8 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const voi
 
 cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* g,
                                const float* beta, float scale, const float* s0, float* o, float* sT,
-                               int B, int T, int H, int dk, int dv, int chunk, cudaStream_t stream);
+                               int B, int T, int H, int dk, int dv, int chunk, cudaStream_t stream,
+                               void* const* events);
 
 // bf16 chunked prefill (tcgen05 path).  `ws` is the caller's workspace.
 size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk);
@@ -37,7 +38,12 @@ cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, 
                                 const __nv_bfloat16* g, const __nv_bfloat16* beta, float scale,
                                 const float* s0, __nv_bfloat16* o, float* sT, int B, int T, int H,
                                 int dk, int dv, int chunk, void* ws, size_t ws_bytes,
-                                cudaStream_t stream);
+                                cudaStream_t stream, void* const* events);
+
+// Records events[i] on the stream when an events array was given.
+inline cudaError_t mark(void* const* events, int i, cudaStream_t stream) {
+  return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) : cudaSuccess;
+}
 
 // Every workspace starts with this header; kernels that wait on barriers with
 // an iteration limit record a give-up here instead of hanging.

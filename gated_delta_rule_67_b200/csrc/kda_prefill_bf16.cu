@@ -522,7 +522,8 @@ size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chu
 
 cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const bf16* beta,
                                 float scale, const float* s0, bf16* o, float* sT, int B, int T, int H, int dk,
-                                int dv, int chunk, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                                int dv, int chunk, void* ws, size_t ws_bytes, cudaStream_t stream,
+                                void* const* events) {
   (void)dk, (void)dv, (void)chunk, (void)ws_bytes;
   static bool attrs_set = false;
   if (!attrs_set) {
@@ -540,15 +541,19 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   const int NC = (T + kC - 1) / kC;
   WorkspaceHeader* hdr = static_cast<WorkspaceHeader*>(ws);
   uint8_t* records = static_cast<uint8_t*>(ws) + sizeof(WorkspaceHeader);
-  cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WorkspaceHeader), stream);
+  cudaError_t e = mark(events, 0, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(WorkspaceHeader), stream);
   if (e != cudaSuccess) return e;
   const unsigned tiles = (unsigned)((size_t)B * H * NC);
   kda_chunk_prep_kernel<<<tiles, 128, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records, hdr, T, H,
                                                                   NC);
   e = cudaGetLastError();
+  if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e != cudaSuccess) return e;
   kda_state_pass_kernel<<<(unsigned)(B * H), 128, kP2Bytes + 1024, stream>>>(records, hdr, s0, sT, o, T, H, NC);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = mark(events, 2, stream);
+  return e;
 }
 
 }  // namespace kda

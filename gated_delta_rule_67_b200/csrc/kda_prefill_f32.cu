@@ -91,14 +91,20 @@ __global__ void __launch_bounds__(kCols * kGroups)
 
 cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* g,
                                const float* beta, float scale, const float* s0, float* o, float* sT,
-                               int B, int T, int H, int dk, int dv, int chunk, cudaStream_t stream) {
+                               int B, int T, int H, int dk, int dv, int chunk, cudaStream_t stream,
+                               void* const* events) {
   (void)chunk;
   dim3 grid(dv / kCols, H, B);
+  cudaError_t e = mark(events, 0, stream);
+  if (e != cudaSuccess) return e;
   if (dk == 128)
     prefill_f32_kernel<128><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv);
   else
     prefill_f32_kernel<64><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = mark(events, 1, stream);
+  if (e == cudaSuccess) e = mark(events, 2, stream);
+  return e;
 }
 
 }  // namespace kda

@@ -99,6 +99,20 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
                          size_t workspace_bytes, void* stream);
 
 /*
+ * kda_chunk_fwd with timing marks for measurement: `events` points to three
+ * cudaEvent_t handles (created by the caller) which are recorded on `stream`
+ * before the first kernel, between the chunk-preparation kernel and the
+ * state-pass kernel, and after the last kernel (for the single-kernel fp32
+ * path the last two marks coincide).  Same arguments, checks and results as
+ * kda_chunk_fwd otherwise.
+ */
+KDA_API kda_status kda_chunk_fwd_profiled(const void* q, const void* k, const void* v, const void* g,
+                                          const void* beta, float scale, const float* initial_state, void* o,
+                                          float* final_state, int B, int T, int H, int dk, int dv, int chunk,
+                                          int dtype, void* workspace, size_t workspace_bytes, void* stream,
+                                          void* const* events);
+
+/*
  * Reads the on-device error word that the last kda_chunk_fwd using this
  * workspace left behind (synchronises `stream`).  Returns KDA_OK, or
  * KDA_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the outputs of
