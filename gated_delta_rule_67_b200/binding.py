@@ -27,6 +27,7 @@ SIGNATURES = {
     "kda_chunk_fwd_workspace_size": (_sz, [_i] * 7),
     "kda_chunk_fwd": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp]),
     "kda_chunk_fwd_profiled": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp, _vp]),
+    "kda_chunk_fwd_noalloc": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp]),
     "kda_chunk_fwd_check": (_i, [_vp, _sz, _vp]),
     "kda_recurrent_step": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 5 + [_vp]),
 }
@@ -139,6 +140,35 @@ def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64,
         st = lib.kda_chunk_fwd_profiled(*args, handles)
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd")
+    return o, final_state
+
+
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64, o=None,
+                          final_state=None, output_final_state=True, stream=None):
+    """kda_chunk_fwd using the library's static device scratch instead of a
+    workspace: for callers that cannot allocate device memory.  Fits
+    B*H*ceil(T/64) <= 903 chunk-heads (bf16); calls overlapping on the GPU race."""
+    lib = load()
+    for name, x in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
+        _check_dev(name, x, q.dtype)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != (B, T, H) or beta.shape != (B, T, H):
+        raise ValueError("shape mismatch among q, k, v, g, beta")
+    if scale is None:
+        scale = dk ** -0.5
+    if initial_state is not None:
+        _check_dev("initial_state", initial_state, torch.float32)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _check_dev("o", o, q.dtype)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                   _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk,
+                                   _dtype_code(q.dtype), _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd_noalloc")
     return o, final_state
 
 

@@ -113,6 +113,27 @@ KDA_API kda_status kda_chunk_fwd_profiled(const void* q, const void* k, const vo
                                           void* const* events);
 
 /*
+ * kda_chunk_fwd without a caller workspace, for callers that cannot allocate
+ * device memory (a host program with no allocator of its own, or a plugin in
+ * a framework that forbids further cudaMalloc calls).  The pages describe no
+ * such interface; it has no counterpart there.
+ *
+ * Same arguments and results as kda_chunk_fwd minus the workspace.  The
+ * scratch is a 64 MiB statically sized device array inside the library
+ * (present on every GPU that loads it, until the process exits), which fits
+ * B * H * ceil(T / 64) <= 903 for the bf16 path; larger problems return
+ * KDA_ERR_UNSUPPORTED before anything is launched.  The first call on a
+ * device looks up the array's device address (with that device current), so
+ * make it before any stream capture.  All calls share the array: calls whose
+ * work overlaps on the GPU race on it and must be serialised by the caller.
+ * It allocates nothing (no cudaMalloc, no cudaFree).
+ */
+KDA_API kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* g,
+                                         const void* beta, float scale, const float* initial_state, void* o,
+                                         float* final_state, int B, int T, int H, int dk, int dv, int chunk,
+                                         int dtype, void* stream);
+
+/*
  * Reads the on-device error word that the last kda_chunk_fwd using this
  * workspace left behind (synchronises `stream`).  Returns KDA_OK, or
  * KDA_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the outputs of

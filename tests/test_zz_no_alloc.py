@@ -1,0 +1,40 @@
+"""The allocation-free prefill entry point (kda_chunk_fwd_noalloc).
+
+Callers that cannot allocate device memory use the library's static device
+scratch instead of a workspace.  This checks, through the C ABI, that two
+calls in a row give the same results as the ordinary entry point with its
+own workspace (within the bf16 parity tolerance), and that a problem larger
+than the static scratch is refused.  It is collected last on purpose.
+"""
+import pytest
+import torch
+
+from gated_delta_rule_67_b200 import binding
+from gated_delta_rule_67_b200.workloads import make_prefill_inputs
+from tests.parity import TOL, cuda_or_skip, rel_err
+
+pytestmark = pytest.mark.gpu
+NAMES = ("q", "k", "v", "g", "beta")
+
+
+def test_noalloc_matches_workspace_entry_point_twice():
+    dev = cuda_or_skip()
+    binding.load()
+    for call, (B, T, H, seed) in enumerate([(2, 1000, 4, 61), (1, 333, 3, 62)]):
+        x = make_prefill_inputs(B, T, H, 128, 128, torch.bfloat16, 0.1, seed=seed, device=dev)
+        ins = [x[n] for n in NAMES]
+        o_ref, s_ref = binding.kda_chunk_fwd(*ins, None, x["initial_state"])
+        o_na, s_na = binding.kda_chunk_fwd_noalloc(*ins, None, x["initial_state"])
+        torch.cuda.synchronize()
+        assert rel_err(o_na, o_ref) < TOL[torch.bfloat16], call
+        assert rel_err(s_na, s_ref) < TOL[torch.bfloat16], call
+
+
+def test_noalloc_refuses_problems_beyond_the_scratch():
+    dev = cuda_or_skip()
+    lib = binding.load()
+    # 1 x 16 heads x ceil(4096/64)=64 chunks = 1024 chunk-heads > 903: refused before any launch.
+    x = make_prefill_inputs(1, 4096, 16, 128, 128, torch.bfloat16, 0.1, seed=63, device=dev)
+    with pytest.raises(binding.KDAError) as e:
+        binding.kda_chunk_fwd_noalloc(*(x[n] for n in NAMES), None, x["initial_state"])
+    assert e.value.status == binding.KDA_ERR_UNSUPPORTED
