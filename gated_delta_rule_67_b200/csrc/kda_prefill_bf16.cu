@@ -60,21 +60,30 @@ constexpr int kRefTok = 31;
 constexpr uint32_t kRecWQ = 0;          // [-W ; Q+]: K-major, 128 rows x 128 ch (32 KiB)
 constexpr uint32_t kRecAqk = 32768;     // A_qk: K-major, 64 rows (i) x 64 (j)  (8 KiB)
 constexpr uint32_t kRecKbar = 40960;    // Kbar: token-row 128B-swizzled tile 64 x 128 (16 KiB)
-constexpr uint32_t kRecU = 57344;       // U: plain row-major [64][128] bf16 (16 KiB)
+constexpr uint32_t kRecU = 57344;       // U^T: K-major, 128 rows (channel) x 64 (token) (16 KiB)
 constexpr uint32_t kRecGamma = 73728;   // gamma: 128 fp32
 constexpr uint32_t kRecBytes = 74240;
 
-// --- prep kernel shared memory (byte offsets from a 1024-aligned base) -----
-constexpr uint32_t kP1Q = 0;            // q tile (token rows), 16 KiB
-constexpr uint32_t kP1K = 16384;        // k tile, overwritten in place by K+ (start-decayed)
-constexpr uint32_t kP1V = 32768;        // v tile
-constexpr uint32_t kP1G = 49152;        // g tile; dead after the cumulative sum
-constexpr uint32_t kP1A1 = 49152;       // score A operand [K+_r ; Q+_r], 128 rows, 32 KiB (aliases g)
-constexpr uint32_t kP1Akk = 49152;      // fp32 A_kk [64][kAkkLd] for the solve (aliases A1)
-constexpr uint32_t kP1B1 = 81920;       // score B operand K-_r, 64 rows, 16 KiB
-constexpr uint32_t kP1B2 = 81920;       // (T diag beta)^T operand, 64 x 64, 8 KiB (aliases B1)
-constexpr uint32_t kP1Bytes = 98304;
-constexpr int kAkkLd = 68;              // padded fp32 row stride of A_kk
+// --- prep kernel: shared memory (byte offsets from a 1024-aligned base) ---
+// Region A (32 KiB) is a 128-row K-major tile: rows 0-63 first hold g and then
+// K+_r, rows 64-127 hold q and then Q+_r (both in place).  Once the score MMA
+// is done it holds the v tile [0,16K), the (T diag beta)^T operand [16K,24K)
+// and four T blocks [24K,28K).
+// Region K (16 KiB): the k tile, turned in place into K+ (start-decayed);
+// after the W/U MMAs the U^T staging tile.
+// Region B (16 KiB): K-_r (score B operand); then the 10 A_kk blocks [0,10K)
+// and six T blocks [10K,16K); finally the -W staging tile.
+constexpr uint32_t kP1A = 0;
+constexpr uint32_t kP1K = 32768;
+constexpr uint32_t kP1B = 49152;
+constexpr uint32_t kP1Bytes = 65536;
+constexpr uint32_t kP1V = kP1A;              // v tile, after the score MMA
+constexpr uint32_t kP1B2 = kP1A + 16384;     // (T diag beta)^T, K-major 64 x 64
+constexpr int kP1Threads = 256;
+// Per-chunk safe range of the factored form: every channel's cumulative
+// log-gate over the chunk must stay above -kSafeSpan, so that each factor
+// exp(+-(G_i - G_r)), exp(G_r), exp(G_C - G_r) lies in [e^-64, e^64].
+constexpr float kSafeSpan = 64.f;
 
 // --- state-pass kernel shared memory --------------------------------------
 constexpr uint32_t kStage = 74752;      // record rounded up to 1024
@@ -103,21 +112,6 @@ __device__ __forceinline__ void st_kmajor8(uint8_t* tile, uint32_t r, uint32_t k
   *reinterpret_cast<uint4*>(tile + kmajor_off(r, k0, rows)) = w;
 }
 
-__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y,
-                                            int32_t z, int32_t w) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
-      "[%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 __device__ __forceinline__ void wait_or_flag(uint64_t* bar, uint32_t parity, WorkspaceHeader* hdr, uint32_t where) {
   if (!mbar_wait(bar, parity, kWaitLimit)) {
     atomicOr(&hdr->error, 1u);
@@ -126,18 +120,42 @@ __device__ __forceinline__ void wait_or_flag(uint64_t* bar, uint32_t parity, Wor
 }
 
 // =============================================================== kernel 1
-__global__ void __launch_bounds__(128, 2)
+__device__ __forceinline__ float2 ld_bf2(const uint8_t* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ void st_bf2(uint8_t* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+// The lower-triangular 64 x 64 matrices A_kk and T are kept as 16 x 16 fp32
+// blocks (I, J), J <= I, numbered p = I(I+1)/2 + J; A blocks in region B,
+// T blocks 0-5 after them in region B and T blocks 6-9 at the end of region A.
+__device__ __forceinline__ int blk(int I, int J) { return I * (I + 1) / 2 + J; }
+__device__ __forceinline__ float* a_blk(uint8_t* sm, int p) { return reinterpret_cast<float*>(sm + kP1B) + p * 256; }
+__device__ __forceinline__ float* t_blk(uint8_t* sm, int p) {
+  return p < 6 ? reinterpret_cast<float*>(sm + kP1B + 10240) + p * 256
+               : reinterpret_cast<float*>(sm + kP1A + 24576) + (p - 6) * 256;
+}
+// 16x16x16 block product sum_m X[r][m] * Y[m][c].
+__device__ __forceinline__ float bdot(const float* X, const float* Y, int r, int c) {
+  float acc = 0.f;
+#pragma unroll
+  for (int m = 0; m < 16; ++m) acc = fmaf(X[r * 16 + m], Y[m * 16 + c], acc);
+  return acc;
+}
+
+__global__ void __launch_bounds__(kP1Threads, 3)
     kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                           const bf16* __restrict__ beta, float scale, uint8_t* __restrict__ records,
                           WorkspaceHeader* hdr, int T, int H, int NC) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  __shared__ uint64_t bar_tma, bar_mma;
+  __shared__ uint64_t bar_in, bar_v, bar_mma;
   __shared__ uint32_t tmem_base;
   __shared__ float sbeta[kC];
+  __shared__ float stot[4][kD];
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x % NC;
   const int bh = blockIdx.x / NC;
   const int h = bh % H, b = bh / H;
@@ -146,342 +164,549 @@ __global__ void __launch_bounds__(128, 2)
   uint8_t* rec = records + (size_t)blockIdx.x * kRecBytes;
 
   if (tid == 0) {
-    mbar_init(&bar_tma, 1);
+    mbar_init(&bar_in, 1);
+    mbar_init(&bar_v, 1);
     mbar_init(&bar_mma, 1);
     fence_mbar_init();
+    mbar_expect_tx(&bar_in, 3 * 16384);
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      tma_load_4d(sm + kP1A + kb * 16384, &tm_g, &bar_in, kb * 64, h, t0, b);         // rows 0-63
+      tma_load_4d(sm + kP1A + kb * 16384 + 8192, &tm_q, &bar_in, kb * 64, h, t0, b);  // rows 64-127
+      tma_load_4d(sm + kP1K + kb * 8192, &tm_k, &bar_in, kb * 64, h, t0, b);
+    }
   }
-  if (warp == 0) tmem_alloc(&tmem_base, 256);
+  if (warp == 0) tmem_alloc(&tmem_base, 128);
   if (tid < kC) sbeta[tid] = tid < L ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
+  wait_or_flag(&bar_in, 0, hdr, 1);
 
-  if (tid == 0) {
-    mbar_expect_tx(&bar_tma, 4 * 16384);
-    const CUtensorMap* maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
-    const uint32_t dst[4] = {kP1Q, kP1K, kP1V, kP1G};
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      tma_load_4d(sm + dst[m], maps[m], &bar_tma, 0, h, t0, b);
-      tma_load_4d(sm + dst[m] + 8192, maps[m], &bar_tma, 64, h, t0, b);
-    }
-  }
-  wait_or_flag(&bar_tma, 0, hdr, 1);
-
-  // ---- pass 1: in-chunk cumulative log-gate, one key channel per thread
-  const int ch = tid;
-  float G[kC];
+  // ---- pass 1: in-chunk cumulative log-gate.  Thread = (token quarter qt,
+  // channel pair c0, c0+1); each keeps its 16 x 2 values of G in registers.
+  const int qt = tid >> 6, c0 = 2 * (tid & 63);
+  float G0[16], G1[16];
   {
-    float run = 0.f;
+    float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-    for (int i = 0; i < kC; ++i) {
-      run += ldbf(sm + kP1G, kmajor_off(i, ch, kC));
-      G[i] = run;
+    for (int ii = 0; ii < 16; ++ii) {
+      const float2 f = ld_bf2(sm + kP1A + kmajor_off(qt * 16 + ii, c0, 128));
+      r0 += f.x;
+      r1 += f.y;
+      G0[ii] = r0;
+      G1[ii] = r1;
     }
+    stot[qt][c0] = r0;
+    stot[qt][c0 + 1] = r1;
   }
-  __syncthreads();  // the g tile is dead from here on (A1 aliases it)
-
-  // ---- pass 2: decayed operands
-  {
-    const float gref = G[kRefTok], gend = G[kC - 1];
-#pragma unroll
-    for (int i = 0; i < kC; ++i) {
-      const uint32_t o64 = kmajor_off(i, ch, kC);
-      const float kk = ldbf(sm + kP1K, o64);
-      const float qq = ldbf(sm + kP1Q, o64);
-      const float em = __expf(G[i] - gref);
-      const float ei = __expf(gref - G[i]);
-      const float e0 = __expf(G[i]);
-      const float eb = __expf(gend - G[i]);
-      stbf(sm + kP1A1, kmajor_off(i, ch, 128), kk * em);                 // K+_r
-      stbf(sm + kP1A1, kmajor_off(kC + i, ch, 128), scale * qq * em);    // Q+_r
-      stbf(sm + kP1B1, o64, kk * ei);                                    // K-_r
-      stbf(sm + kP1K, o64, kk * e0);                                     // K+ (chunk start), in place
-      stbf(rec + kRecWQ, kmajor_off(kC + i, ch, 128), scale * qq * e0);  // Q+ image rows 64..127
-      stbf(rec + kRecKbar, o64, kk * eb);                                // Kbar image
-    }
-    reinterpret_cast<float*>(rec + kRecGamma)[ch] = expf(gend);
-  }
-  fence_async_smem();
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-
-  // ---- score MMA: D[0:128, 0:64] = [K+_r ; Q+_r] (128 x 128) . K-_r^T
-  if (tid == 0) {
-    const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
-    const uint32_t a0 = smem_u32(sm + kP1A1), b0 = smem_u32(sm + kP1B1);
+  float off0 = 0.f, off1 = 0.f;
 #pragma unroll
-    for (int s = 0; s < kD / 16; ++s) {
-      const uint32_t a = a0 + (s / 4) * 16384 + (s % 4) * 32;
-      const uint32_t bb = b0 + (s / 4) * 8192 + (s % 4) * 32;
-      mma_bf16(tm, desc_sw128(a, 16, 1024), desc_sw128(bb, 16, 1024), idesc, s > 0);
+  for (int q4 = 0; q4 < 3; ++q4)
+    if (q4 < qt) {
+      off0 += stot[q4][c0];
+      off1 += stot[q4][c0 + 1];
     }
-    mma_commit(&bar_mma);
+  const float gref0 = stot[0][c0] + stot[1][c0], gref1 = stot[0][c0 + 1] + stot[1][c0 + 1];
+  const float gend0 = gref0 + stot[2][c0] + stot[3][c0], gend1 = gref1 + stot[2][c0 + 1] + stot[3][c0 + 1];
+#pragma unroll
+  for (int ii = 0; ii < 16; ++ii) {
+    G0[ii] += off0;
+    G1[ii] += off1;
   }
-  wait_or_flag(&bar_mma, 0, hdr, 2);
-  tc_fence_after();
+  if (qt == 0) {
+    reinterpret_cast<float*>(rec + kRecGamma)[c0] = expf(gend0);
+    reinterpret_cast<float*>(rec + kRecGamma)[c0 + 1] = expf(gend1);
+  }
+  // The g tile is dead after this barrier.
+  const int slow = __syncthreads_or((gend0 < -kSafeSpan) || (gend1 < -kSafeSpan));
 
-  // ---- masks: rows 0..63 -> A_kk (fp32, smem), rows 64..127 -> A_qk image
-  {
-    float* akk = reinterpret_cast<float*>(sm + kP1Akk);
-    const int r = tid & 63;
+  if (!slow) {
+    // ---- pass 2 (factored form): decayed operands relative to token kRefTok
+    const float egr0 = __expf(gref0), egr1 = __expf(gref1);
+    const float egb0 = __expf(gend0 - gref0), egb1 = __expf(gend1 - gref1);
 #pragma unroll
-    for (int cb = 0; cb < kC / 16; ++cb) {
-      float v[16];
-      tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + cb * 16, v);
-      tmem_wait_ld();
-      if (warp < 2) {
-        const float br = sbeta[r];
+    for (int ii = 0; ii < 16; ++ii) {
+      const int i = qt * 16 + ii;
+      const uint32_t oK = kmajor_off(i, c0, kC);        // 64-row tiles: k, K-_r, Kbar
+      const uint32_t oA = kmajor_off(i, c0, 128);       // row i of region A
+      const uint32_t oQ = kmajor_off(kC + i, c0, 128);  // row 64+i of region A and of the [-W;Q+] image
+      const float2 kk = ld_bf2(sm + kP1K + oK);
+      const float2 qq = ld_bf2(sm + kP1A + oQ);
+      const float ex0 = __expf(G0[ii] - gref0), ex1 = __expf(G1[ii] - gref1);
+      const float ei0 = __expf(gref0 - G0[ii]), ei1 = __expf(gref1 - G1[ii]);
+      const float e00 = ex0 * egr0, e01 = ex1 * egr1;  // exp(G_i)
+      st_bf2(sm + kP1A + oA, kk.x * ex0, kk.y * ex1);                          // K+_r
+      st_bf2(sm + kP1A + oQ, scale * qq.x * ex0, scale * qq.y * ex1);          // Q+_r
+      st_bf2(sm + kP1B + oK, kk.x * ei0, kk.y * ei1);                          // K-_r
+      st_bf2(sm + kP1K + oK, kk.x * e00, kk.y * e01);                          // K+
+      st_bf2(rec + kRecWQ + oQ, scale * qq.x * e00, scale * qq.y * e01);       // Q+ image
+      st_bf2(rec + kRecKbar + oK, kk.x * (ei0 * egb0), kk.y * (ei1 * egb1));   // Kbar image
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- score MMA: D[0:128, 0:64] = [K+_r ; Q+_r] (128 x 128) . K-_r^T
+    if (tid == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t a0 = smem_u32(sm + kP1A), b0 = smem_u32(sm + kP1B);
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int j = cb * 16 + jj;
-          akk[r * kAkkLd + j] = j < r ? br * v[jj] : 0.f;
+      for (int k = 0; k < kD / 16; ++k)
+        mma_bf16(tm, desc_sw128(a0 + (k / 4) * 16384 + (k % 4) * 32, 16, 1024),
+                 desc_sw128(b0 + (k / 4) * 8192 + (k % 4) * 32, 16, 1024), idesc, k > 0);
+      mma_commit(&bar_mma);
+    }
+    wait_or_flag(&bar_mma, 0, hdr, 2);
+    tc_fence_after();
+
+    // ---- rows 0-63 -> A_kk blocks (times beta_i, strictly lower); rows 64-127 -> A_qk image
+    {
+      const int row = (warp & 3) * 32 + lane;
+      const int col0 = (warp >> 2) * 32;
+      float v[32];
+      tmem_ld32(tm + ((uint32_t)((warp & 3) * 32) << 16) + col0, v);
+      if (row < kC) {
+        const int i = row, I = i >> 4;
+        const float bi = sbeta[i];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int j = col0 + jj, J = j >> 4;
+          if (J <= I) a_blk(sm, blk(I, J))[(i & 15) * 16 + (j & 15)] = j < i ? bi * v[jj] : 0.f;
         }
       } else {
-        float m[16];
+        const int i = row - kC;
+        float m[32];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) m[jj] = (cb * 16 + jj) <= r ? v[jj] : 0.f;
-        st_kmajor8(rec + kRecAqk, r, cb * 16, kC, m);
-        st_kmajor8(rec + kRecAqk, r, cb * 16 + 8, kC, m + 8);
+        for (int jj = 0; jj < 32; ++jj) m[jj] = (col0 + jj) <= i ? v[jj] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st_kmajor8(rec + kRecAqk, i, col0 + 8 * e, kC, m + 8 * e);
       }
+    }
+  } else {
+    // ---- exact path for chunks whose gates decay past e^-64: the score
+    // matrices straight from their definition, every decay factor
+    // exp(G_i - G_j) <= 1 formed per (pair, channel).
+    auto gp = [&](int i, int c) -> float* {
+      return c < 32 ? reinterpret_cast<float*>(sm + kP1A) + i * 32 + c
+                    : c < 64 ? reinterpret_cast<float*>(sm + kP1A + 16384) + i * 32 + (c - 32)
+                             : reinterpret_cast<float*>(sm + kP1B) + i * 64 + (c - 64);
+    };
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) {
+      *gp(qt * 16 + ii, c0) = G0[ii];
+      *gp(qt * 16 + ii, c0 + 1) = G1[ii];
+    }
+    __syncthreads();
+    constexpr int kPairs = kC * (kC + 1) / 2;  // (i, j) with j <= i
+    float akk[9], aqk[9];
+#pragma unroll 1
+    for (int t = 0; t < 9; ++t) {
+      const int p = tid + t * kP1Threads;
+      akk[t] = aqk[t] = 0.f;
+      if (p < kPairs) {
+        int i = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+        while (i * (i + 1) / 2 > p) --i;
+        while ((i + 1) * (i + 2) / 2 <= p) ++i;
+        const int j = p - i * (i + 1) / 2;
+        float sk = 0.f, sq = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < kD; c += 2) {
+          const float2 ki = ld_bf2(sm + kP1K + kmajor_off(i, c, kC));
+          const float2 kj = ld_bf2(sm + kP1K + kmajor_off(j, c, kC));
+          const float2 qi = ld_bf2(sm + kP1A + kmajor_off(kC + i, c, 128));
+          const float d0 = __expf(*gp(i, c) - *gp(j, c)), d1 = __expf(*gp(i, c + 1) - *gp(j, c + 1));
+          sk = fmaf(ki.x * kj.x, d0, fmaf(ki.y * kj.y, d1, sk));
+          sq = fmaf(qi.x * kj.x, d0, fmaf(qi.y * kj.y, d1, sq));
+        }
+        akk[t] = sk;
+        aqk[t] = sq;
+      }
+    }
+    __syncthreads();  // G (in regions A and B) is dead from here on
+#pragma unroll 1
+    for (int t = 0; t < 9; ++t) {
+      const int p = tid + t * kP1Threads;
+      if (p < kPairs) {
+        int i = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+        while (i * (i + 1) / 2 > p) --i;
+        while ((i + 1) * (i + 2) / 2 <= p) ++i;
+        const int j = p - i * (i + 1) / 2;
+        a_blk(sm, blk(i >> 4, j >> 4))[(i & 15) * 16 + (j & 15)] = j < i ? sbeta[i] * akk[t] : 0.f;
+        stbf(rec + kRecAqk, kmajor_off(i, j, kC), scale * aqk[t]);
+      }
+    }
+    for (int e = tid; e < kC * kC; e += kP1Threads) {
+      const int i = e / kC, j = e % kC;
+      if (j > i) stbf(rec + kRecAqk, kmajor_off(i, j, kC), 0.f);
+    }
+    // pass 2 (exact): start- and end-decayed operands, factors <= 1
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) {
+      const int i = qt * 16 + ii;
+      const uint32_t oK = kmajor_off(i, c0, kC);
+      const uint32_t oQ = kmajor_off(kC + i, c0, 128);
+      const float2 kk = ld_bf2(sm + kP1K + oK);
+      const float2 qq = ld_bf2(sm + kP1A + oQ);
+      const float e00 = __expf(G0[ii]), e01 = __expf(G1[ii]);
+      st_bf2(sm + kP1K + oK, kk.x * e00, kk.y * e01);
+      st_bf2(rec + kRecWQ + oQ, scale * qq.x * e00, scale * qq.y * e01);
+      st_bf2(rec + kRecKbar + oK, kk.x * __expf(gend0 - G0[ii]), kk.y * __expf(gend1 - G1[ii]));
     }
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
 
-  // ---- T = (I + A_kk)^-1, one column per thread (threads 0..63), fp32
-  if (tid < kC) {
-    const int j = tid;
-    const float* akk = reinterpret_cast<const float*>(sm + kP1Akk);
-    float t[kC];
+  // ---- region A is free: bring the v tile while the triangle is inverted
+  if (tid == 0) {
+    mbar_expect_tx(&bar_v, 16384);
+    tma_load_4d(sm + kP1V, &tm_v, &bar_v, 0, h, t0, b);
+    tma_load_4d(sm + kP1V + 8192, &tm_v, &bar_v, 64, h, t0, b);
+  }
+
+  // ---- T = (I + A_kk)^-1 by 16 x 16 blocks, fp32
+  if (tid < 64) {  // diagonal blocks by forward substitution, one column per thread
+    const int I = tid >> 4, jj = tid & 15;
+    const float* A = a_blk(sm, blk(I, I));
+    float t[16];
 #pragma unroll
-    for (int i = 0; i < kC; ++i) {
-      float acc0 = 0.f, acc1 = 0.f;
-      const float4* row = reinterpret_cast<const float4*>(akk + i * kAkkLd);
+    for (int r = 0; r < 16; ++r) {
+      float acc = 0.f;
 #pragma unroll
-      for (int m4 = 0; m4 < i / 4; ++m4) {
-        const float4 a = row[m4];
-        acc0 = fmaf(a.x, t[4 * m4 + 0], acc0);
-        acc1 = fmaf(a.y, t[4 * m4 + 1], acc1);
-        acc0 = fmaf(a.z, t[4 * m4 + 2], acc0);
-        acc1 = fmaf(a.w, t[4 * m4 + 3], acc1);
-      }
-#pragma unroll
-      for (int m = (i / 4) * 4; m < i; ++m) acc0 = fmaf(akk[i * kAkkLd + m], t[m], acc0);
-      t[i] = i < j ? 0.f : (i == j ? 1.f : -(acc0 + acc1));
+      for (int m = 0; m < r; ++m) acc = fmaf(A[r * 16 + m], t[m], acc);
+      t[r] = r < jj ? 0.f : (r == jj ? 1.f : -acc);
     }
-    // (T diag(beta))^T as the K-major B operand: row n = i, column k = j.
-    const float bj = sbeta[j];
+    float* Tb = t_blk(sm, blk(I, I));
 #pragma unroll
-    for (int i = 0; i < kC; ++i) stbf(sm + kP1B2, kmajor_off(i, j, kC), t[i] * bj);
+    for (int r = 0; r < 16; ++r) Tb[r * 16 + jj] = t[r];
+  }
+  __syncthreads();
+  // off-diagonal blocks, one sub-diagonal at a time:
+  //   T_IJ = -T_II * (sum_{K=J}^{I-1} A_IK T_KJ)
+#pragma unroll 1
+  for (int d = 1; d < 4; ++d) {
+    const int nb = 4 - d;  // blocks (J+d, J), J = 0..nb-1
+    float y[3];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int e = tid + q * kP1Threads;
+      if (q < nb) {
+        const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
+        float x = 0.f;
+        for (int K = J; K < I; ++K) x += bdot(a_blk(sm, blk(I, K)), t_blk(sm, blk(K, J)), r, c);
+        y[q] = x;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int e = tid + q * kP1Threads;
+      if (q < nb) t_blk(sm, blk((e >> 8) + d, e >> 8))[e & 255] = y[q];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int e = tid + q * kP1Threads;
+      if (q < nb) {
+        const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
+        y[q] = -bdot(t_blk(sm, blk(I, I)), t_blk(sm, blk(I, J)), r, c);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const int e = tid + q * kP1Threads;
+      if (q < nb) t_blk(sm, blk((e >> 8) + d, e >> 8))[e & 255] = y[q];
+    }
+    __syncthreads();
+  }
+  // (T diag(beta))^T as the K-major B operand of the W/U MMAs: row n = i, column k = j.
+  {
+    const int i = tid >> 2, j0 = (tid & 3) * 16, I = i >> 4, J = j0 >> 4;
+    float vals[16];
+    if (J <= I) {
+      const float* Tb = t_blk(sm, blk(I, J));
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) vals[jj] = (j0 + jj) <= i ? Tb[(i & 15) * 16 + jj] * sbeta[j0 + jj] : 0.f;
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) vals[jj] = 0.f;
+    }
+    st_kmajor8(sm + kP1B2, i, j0, kC, vals);
+    st_kmajor8(sm + kP1B2, i, j0 + 8, kC, vals + 8);
   }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
-  // ---- W^T = K+^T (T diag beta)^T and U^T = V^T (T diag beta)^T  (M=128, N=64, K=64)
+  // ---- W^T = K+^T (T diag beta)^T, U^T = V^T (T diag beta)^T  (M=128, N=64, K=64)
   if (tid == 0) {
+    wait_or_flag(&bar_v, 0, hdr, 3);
+    tc_fence_after();
     const uint32_t idesc = idesc_bf16_f32(128, 64, 1, 0);
     const uint32_t kb = smem_u32(sm + kP1K), vb = smem_u32(sm + kP1V), b2 = smem_u32(sm + kP1B2);
 #pragma unroll
-    for (int s = 0; s < kC / 16; ++s) {
-      const uint64_t bd = desc_sw128(b2 + s * 32, 16, 1024);
-      mma_bf16(tm + 64, desc_sw128(kb + 2 * s * 1024, 8192, 1024), bd, idesc, s > 0);
-      mma_bf16(tm + 128, desc_sw128(vb + 2 * s * 1024, 8192, 1024), bd, idesc, s > 0);
+    for (int k = 0; k < kC / 16; ++k) {
+      const uint64_t bd = desc_sw128(b2 + k * 32, 16, 1024);
+      mma_bf16(tm, desc_sw128(kb + 2 * k * 1024, 8192, 1024), bd, idesc, k > 0);
+      mma_bf16(tm + 64, desc_sw128(vb + 2 * k * 1024, 8192, 1024), bd, idesc, k > 0);
     }
     mma_commit(&bar_mma);
   }
-  wait_or_flag(&bar_mma, 1, hdr, 3);
+  wait_or_flag(&bar_mma, slow ? 0 : 1, hdr, 4);
   tc_fence_after();
 
-  // ---- -W into rows 0..63 of the [-W ; Q+] image, U as plain rows
+  // ---- -W (staged in region B as a 64-row K-major tile) and U^T (region K, 128-row K-major)
   {
-    const int c = tid;
-    bf16* uimg = reinterpret_cast<bf16*>(rec + kRecU);
+    const int c = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float v[32];
 #pragma unroll
-    for (int cb = 0; cb < kC / 16; ++cb) {
-      float w[16], u[16];
-      tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 64 + cb * 16, w);
-      tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 128 + cb * 16, u);
-      tmem_wait_ld();
+    for (int half = 0; half < 2; ++half) {
+      if (warp < 4) {
+        tmem_ld32(tm + lane_off + half * 32, v);
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) {
-        const int i = cb * 16 + ii;
-        stbf(rec + kRecWQ, kmajor_off(i, c, 128), -w[ii]);
-        uimg[i * kD + c] = __float2bfloat16_rn(u[ii]);
+        for (int ii = 0; ii < 32; ++ii) stbf(sm + kP1B, kmajor_off(half * 32 + ii, c, kC), -v[ii]);
+      } else {
+        tmem_ld32(tm + lane_off + 64 + half * 32, v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st_kmajor8(sm + kP1K, c, half * 32 + 8 * e, 128, v + 8 * e);
       }
     }
   }
+  fence_async_smem();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tm, 256);
+  if (tid == 0) {
+    bulk_store(rec + kRecWQ, sm + kP1B, 8192);                // -W rows, channels 0-63
+    bulk_store(rec + kRecWQ + 16384, sm + kP1B + 8192, 8192); // -W rows, channels 64-127
+    bulk_store(rec + kRecU, sm + kP1K, 16384);
+    bulk_commit();
+    bulk_wait_read();
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, 128);
 }
 
 // =============================================================== kernel 2
-__global__ void __launch_bounds__(128, 1)
+// Warp roles (256 threads):
+//   warps 0-3  "state":  the sequential chain.  Thread j owns TMEM lane j =
+//              value channel j (row j of S^T).  Thread 0 also issues the MMAs.
+//   warps 4-7  "output": read O^T of each chunk from TMEM and store o; thread
+//              128 also streams the per-chunk records into two stages (the
+//              stage of chunk n is free again once chunk n's last MMA, the
+//              one that completes O^T, has finished).
+// Tensor memory (512 columns): S^T [0,128), P = -(W S0)^T [128,192),
+// two O^T buffers [192,256) and [256,320).
+constexpr int kSPThreads = 256;
+constexpr uint32_t kNamedStateBar = 1;
+
+__global__ void __launch_bounds__(kSPThreads, 1)
     kda_state_pass_kernel(const uint8_t* __restrict__ records, WorkspaceHeader* hdr, const float* s0, float* sT,
                           bf16* __restrict__ o, int T, int H, int NC) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  __shared__ uint64_t bar_full[2], bar_mma;
+  __shared__ uint64_t bar_full[2], bar_o[2], bar_ofree[2], bar_p, bar_s;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int bh = blockIdx.x;
   const int h = bh % H, b = bh / H;
   const uint8_t* recs = records + (size_t)bh * NC * kRecBytes;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const size_t sbase = (size_t)bh * kD * kD;
 
   if (tid == 0) {
-    mbar_init(&bar_full[0], 1);
-    mbar_init(&bar_full[1], 1);
-    mbar_init(&bar_mma, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_o[i], 1);
+      mbar_init(&bar_ofree[i], 128);
+    }
+    mbar_init(&bar_p, 1);
+    mbar_init(&bar_s, 1);
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(&tmem_base, 256);
+  if (warp == 0) tmem_alloc(&tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tS = tmem_base, tD = tmem_base + 128;
+  const uint32_t tS = tmem_base, tP = tmem_base + 128, tO = tmem_base + 192;
 
-  if (tid == 0) {
-    mbar_expect_tx(&bar_full[0], kRecBytes);
-    bulk_load(sm, recs, kRecBytes, &bar_full[0]);
-  }
-  // S^T row j (= column j of S) into TMEM lane j.
-  const int j = tid;
-  const size_t sbase = (size_t)bh * kD * kD;
-#pragma unroll
-  for (int cb = 0; cb < kD / 16; ++cb) {
-    float v[16];
-#pragma unroll
-    for (int ii = 0; ii < 16; ++ii) v[ii] = s0 ? s0[sbase + (size_t)(cb * 16 + ii) * kD + j] : 0.f;
-    tmem_st16(tS + lane_off + cb * 16, v);
-  }
-  tmem_wait_st();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-
-  uint32_t mma_phase = 0;
-  for (int n = 0; n < NC; ++n) {
-    const int st = n & 1;
-    uint8_t* stage = sm + st * kStage;
-    if (tid == 0 && n + 1 < NC) {
-      mbar_expect_tx(&bar_full[st ^ 1], kRecBytes);
-      bulk_load(sm + (st ^ 1) * kStage, recs + (size_t)(n + 1) * kRecBytes, kRecBytes, &bar_full[st ^ 1]);
-    }
-    wait_or_flag(&bar_full[st], (n >> 1) & 1, hdr, 10);
-
-    // (A) S0^T -> bf16 operand; S^T <- S^T Diag(gamma) in place
-    {
-      const float* gam = reinterpret_cast<const float*>(stage + kRecGamma);
-#pragma unroll
-      for (int cb = 0; cb < kD / 16; ++cb) {
-        float v[16];
-        tmem_ld16(tS + lane_off + cb * 16, v);
-        tmem_wait_ld();
-        st_kmajor8(sm + kP2S, j, cb * 16, kD, v);
-        st_kmajor8(sm + kP2S, j, cb * 16 + 8, kD, v + 8);
-#pragma unroll
-        for (int ii = 0; ii < 16; ++ii) v[ii] *= gam[cb * 16 + ii];
-        tmem_st16(tS + lane_off + cb * 16, v);
-      }
-      tmem_wait_st();
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // (B) D = S0^T [-W ; Q+]^T : cols 0..63 = -(W S0)^T, cols 64..127 = (Q+ S0)^T
-    if (tid == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t a0 = smem_u32(sm + kP2S), b0 = smem_u32(stage + kRecWQ);
-#pragma unroll
-      for (int s = 0; s < kD / 16; ++s) {
-        const uint32_t off = (s / 4) * 16384 + (s % 4) * 32;
-        mma_bf16(tD, desc_sw128(a0 + off, 16, 1024), desc_sw128(b0 + off, 16, 1024), idesc, s > 0);
-      }
-      mma_commit(&bar_mma);
-    }
-    wait_or_flag(&bar_mma, mma_phase, hdr, 11);
-    mma_phase ^= 1;
-    tc_fence_after();
-
-    // (C) V'^T = U^T - (W S0)^T -> bf16 operand
-    {
-      const bf16* u = reinterpret_cast<const bf16*>(stage + kRecU);
-#pragma unroll
-      for (int cb = 0; cb < kC / 16; ++cb) {
-        float v[16];
-        tmem_ld16(tD + lane_off + cb * 16, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int ii = 0; ii < 16; ++ii) v[ii] += __bfloat162float(u[(cb * 16 + ii) * kD + j]);
-        st_kmajor8(sm + kP2Vp, j, cb * 16, kD, v);
-        st_kmajor8(sm + kP2Vp, j, cb * 16 + 8, kD, v + 8);
+  if (warp >= 4) {
+    // ------------------------------------------------------------ output + loads
+    const int j = tid - 128;
+    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    if (tid == 128) {
+      for (int n = 0; n < 2 && n < NC; ++n) {
+        mbar_expect_tx(&bar_full[n], kRecBytes);
+        bulk_load(sm + n * kStage, recs + (size_t)n * kRecBytes, kRecBytes, &bar_full[n]);
       }
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // (D) O^T += V'^T A_qk^T ;  S^T += V'^T Kbar
-    if (tid == 0) {
-      const uint32_t id_o = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
-      const uint32_t vp = smem_u32(sm + kP2Vp), aq = smem_u32(stage + kRecAqk), kbar = smem_u32(stage + kRecKbar);
-#pragma unroll
-      for (int s = 0; s < kC / 16; ++s) {
-        const uint64_t ad = desc_sw128(vp + s * 32, 16, 1024);
-        mma_bf16(tD + 64, ad, desc_sw128(aq + s * 32, 16, 1024), id_o, 1);
-        mma_bf16(tS, ad, desc_sw128(kbar + 2 * s * 1024, 8192, 1024), id_s, 1);
+    for (int n = 0; n < NC; ++n) {
+      const int s = n & 1;
+      wait_or_flag(&bar_o[s], (n >> 1) & 1, hdr, 21);
+      tc_fence_after();
+      if (tid == 128 && n + 2 < NC) {  // every reader of stage s is done with chunk n
+        mbar_expect_tx(&bar_full[s], kRecBytes);
+        bulk_load(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, kRecBytes, &bar_full[s]);
       }
-      mma_commit(&bar_mma);
-    }
-    wait_or_flag(&bar_mma, mma_phase, hdr, 12);
-    mma_phase ^= 1;
-    tc_fence_after();
-
-    // (E) output rows of this chunk
-    {
+      uint32_t r[64];
+      tmem_ld32_raw(tO + s * 64 + lane_off, r);
+      tmem_ld32_raw(tO + s * 64 + lane_off + 32, r + 32);
+      tmem_wait_ld();
+      reg_pin<64>(r);
+      tc_fence_before();
+      mbar_arrive(&bar_ofree[s]);
       const int t0 = n * kC;
       const int L = min(kC, T - t0);
       bf16* orow = o + (((size_t)b * T + t0) * H + h) * kD + j;
+      const size_t ostride = (size_t)H * kD;
 #pragma unroll
-      for (int cb = 0; cb < kC / 16; ++cb) {
-        float v[16];
-        tmem_ld16(tD + lane_off + 64 + cb * 16, v);
-        tmem_wait_ld();
+      for (int i = 0; i < kC; ++i)
+        if (i < L) orow[(size_t)i * ostride] = __float2bfloat16_rn(__uint_as_float(r[i]));
+    }
+  } else {
+    // ------------------------------------------------------------ state
+    const int j = tid;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    {
+      float v[32];
 #pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-          const int i = cb * 16 + ii;
-          if (i < L) orow[(size_t)i * H * kD] = __float2bfloat16_rn(v[ii]);
+      for (int cb = 0; cb < kD / 32; ++cb) {
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii) v[ii] = s0 ? s0[sbase + (size_t)(cb * 32 + ii) * kD + j] : 0.f;
+        tmem_st32(tS + lane_off + cb * 32, v);
+      }
+      tmem_wait_st();
+    }
+    for (int n = 0; n < NC; ++n) {
+      const int s = n & 1;
+      uint8_t* stage = sm + s * kStage;
+      if (n > 0) wait_or_flag(&bar_s, (n - 1) & 1, hdr, 22);
+      tc_fence_after();
+
+      // (1) S0^T -> bf16 operand (row j of a K-major 128 x 128 tile)
+      uint32_t sr[kD];
+#pragma unroll
+      for (int cb = 0; cb < kD / 32; ++cb) tmem_ld32_raw(tS + lane_off + cb * 32, sr + cb * 32);
+      tmem_wait_ld();
+      reg_pin<kD>(sr);
+#pragma unroll
+      for (int k8 = 0; k8 < kD / 8; ++k8) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(sr[k8 * 8 + e]);
+        st_kmajor8(sm + kP2S, j, k8 * 8, kD, f);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      named_bar_sync(kNamedStateBar, 128);
+      tc_fence_after();
+
+      // (2) P = S0^T (-W)^T (critical), then O^T = S0^T Q+^T into this chunk's O buffer
+      if (tid == 0) {
+        wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 23);
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
+        const uint32_t a0 = smem_u32(sm + kP2S), b0 = smem_u32(stage + kRecWQ);
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k) {
+          const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+          mma_bf16(tP, desc_sw128(a0 + off, 16, 1024), desc_sw128(b0 + off, 16, 1024), idesc, k > 0);
+        }
+        mma_commit(&bar_p);
+        if (n >= 2) wait_or_flag(&bar_ofree[s], ((n - 2) >> 1) & 1, hdr, 24);
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k) {
+          const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
+          mma_bf16(tO + s * 64, desc_sw128(a0 + off, 16, 1024), desc_sw128(b0 + 8192 + off, 16, 1024), idesc,
+                   k > 0);
         }
       }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  }
 
-  if (sT) {
+      // (3) S^T <- S^T Diag(gamma) while the MMAs run
+      wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 25);
+      {
+        const float4* gam = reinterpret_cast<const float4*>(stage + kRecGamma);
 #pragma unroll
-    for (int cb = 0; cb < kD / 16; ++cb) {
-      float v[16];
-      tmem_ld16(tS + lane_off + cb * 16, v);
-      tmem_wait_ld();
+        for (int cb = 0; cb < kD / 32; ++cb) {
+          float v[32];
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) sT[sbase + (size_t)(cb * 16 + ii) * kD + j] = v[ii];
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 gg = gam[cb * 8 + q4];
+            v[q4 * 4 + 0] = __uint_as_float(sr[cb * 32 + q4 * 4 + 0]) * gg.x;
+            v[q4 * 4 + 1] = __uint_as_float(sr[cb * 32 + q4 * 4 + 1]) * gg.y;
+            v[q4 * 4 + 2] = __uint_as_float(sr[cb * 32 + q4 * 4 + 2]) * gg.z;
+            v[q4 * 4 + 3] = __uint_as_float(sr[cb * 32 + q4 * 4 + 3]) * gg.w;
+          }
+          tmem_st32(tS + lane_off + cb * 32, v);
+        }
+        tmem_wait_st();
+      }
+
+      // (4) V'^T = U^T + P  -> bf16 operand (row j of a K-major 128 x 64 tile)
+      wait_or_flag(&bar_p, n & 1, hdr, 26);
+      tc_fence_after();
+      {
+        uint32_t pr[kC];
+        tmem_ld32_raw(tP + lane_off, pr);
+        tmem_ld32_raw(tP + lane_off + 32, pr + 32);
+        tmem_wait_ld();
+        reg_pin<kC>(pr);
+#pragma unroll
+        for (int k8 = 0; k8 < kC / 8; ++k8) {
+          const uint32_t off = kmajor_off(j, k8 * 8, kD);
+          const uint4 uu = *reinterpret_cast<const uint4*>(stage + kRecU + off);
+          const uint32_t uw[4] = {uu.x, uu.y, uu.z, uu.w};
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 u2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[e]));
+            f[2 * e] = u2.x + __uint_as_float(pr[k8 * 8 + 2 * e]);
+            f[2 * e + 1] = u2.y + __uint_as_float(pr[k8 * 8 + 2 * e + 1]);
+          }
+          st_kmajor8(sm + kP2Vp, j, k8 * 8, kD, f);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      named_bar_sync(kNamedStateBar, 128);
+      tc_fence_after();
+
+      // (5) S^T += V'^T Kbar (critical), then O^T += V'^T A_qk^T
+      if (tid == 0) {
+        const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
+        const uint32_t id_o = idesc_bf16_f32(128, 64, 0, 0);
+        const uint32_t vp = smem_u32(sm + kP2Vp), aq = smem_u32(stage + kRecAqk), kbar = smem_u32(stage + kRecKbar);
+#pragma unroll
+        for (int k = 0; k < kC / 16; ++k)
+          mma_bf16(tS, desc_sw128(vp + k * 32, 16, 1024), desc_sw128(kbar + 2 * k * 1024, 8192, 1024), id_s, 1);
+        mma_commit(&bar_s);
+#pragma unroll
+        for (int k = 0; k < kC / 16; ++k)
+          mma_bf16(tO + s * 64, desc_sw128(vp + k * 32, 16, 1024), desc_sw128(aq + k * 32, 16, 1024), id_o, 1);
+        mma_commit(&bar_o[s]);
+      }
+    }
+    wait_or_flag(&bar_s, (NC - 1) & 1, hdr, 27);
+    tc_fence_after();
+    if (sT) {
+#pragma unroll
+      for (int cb = 0; cb < kD / 32; ++cb) {
+        float v[32];
+        tmem_ld32(tS + lane_off + cb * 32, v);
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii) sT[sbase + (size_t)(cb * 32 + ii) * kD + j] = v[ii];
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem_base, 256);
+  if (warp == 0) tmem_dealloc(tmem_base, 512);
 }
 
 // ================================================================== host
@@ -545,12 +770,13 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(WorkspaceHeader), stream);
   if (e != cudaSuccess) return e;
   const unsigned tiles = (unsigned)((size_t)B * H * NC);
-  kda_chunk_prep_kernel<<<tiles, 128, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records, hdr, T, H,
+  kda_chunk_prep_kernel<<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records, hdr, T, H,
                                                                   NC);
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e != cudaSuccess) return e;
-  kda_state_pass_kernel<<<(unsigned)(B * H), 128, kP2Bytes + 1024, stream>>>(records, hdr, s0, sT, o, T, H, NC);
+  kda_state_pass_kernel<<<(unsigned)(B * H), kSPThreads, kP2Bytes + 1024, stream>>>(records, hdr, s0, sT, o, T,
+                                                                                     H, NC);
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 2, stream);
   return e;

@@ -127,3 +127,39 @@ def test_workspace_reuse_and_check():
     assert torch.equal(o1, o2) and torch.equal(s1, s2)  # deterministic
     ref_o, ref_s = _oracle(x)
     assert rel_err(o1, ref_o) < TOLB and rel_err(s1, ref_s) < TOLB
+
+
+@pytest.mark.parametrize("pattern", ["half_channels", "some_chunks", "all"])
+def test_extreme_gates(pattern):
+    """Gates of exp(-20) per token (cumulative decay far below e^-64 within a
+    chunk) next to gates of exactly 1: the chunks that need it take the exact
+    per-pair path; results stay finite and match the oracle."""
+    dev = cuda_or_skip()
+    B, T, H, d = 1, 300, 2, 128
+    x = make_prefill_inputs(B, T, H, d, d, torch.bfloat16, 0.1, seed=47, device="cpu")
+    g = x["g"].float()
+    if pattern == "half_channels":
+        g[..., : d // 2] = -20.0
+        g[..., d // 2:] = 0.0
+    elif pattern == "some_chunks":
+        g[:, 64:128, :, :5] = -20.0   # chunk 1 only, a few channels
+        g[:, 200:260, 1, :] = -3.0    # chunks 3-4 of head 1: -3 per token crosses -64 inside the chunk
+    else:
+        g[:] = -20.0
+    x["g"] = g.to(torch.bfloat16)
+    o, sT = _run(x, dev)
+    ref_o, ref_s = _oracle(x)
+    assert rel_err(o, ref_o) < TOLB
+    assert rel_err(sT, ref_s) < TOLB
+
+
+def test_gate_span_just_inside_fast_path():
+    """Per-token log-gate of -0.95: the chunk's cumulative decay (-60.8) stays
+    inside the factored form's safe range, with factors up to e^30 each way."""
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(1, 256, 2, 128, 128, torch.bfloat16, 0.1, seed=48, device="cpu")
+    x["g"] = torch.full_like(x["g"], -0.95)
+    o, sT = _run(x, dev)
+    ref_o, ref_s = _oracle(x)
+    assert rel_err(o, ref_o) < TOLB
+    assert rel_err(sT, ref_s) < TOLB
