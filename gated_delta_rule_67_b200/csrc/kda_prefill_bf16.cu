@@ -58,8 +58,9 @@ constexpr int kRefTok = 31;
 
 // --- per-chunk record in the workspace (byte offsets) -----------------------
 constexpr uint32_t kRecWQ = 0;          // [-W ; Q+]: K-major, 128 rows x 128 ch (32 KiB)
-constexpr uint32_t kRecAqk = 32768;     // A_qk: K-major, 64 rows (i) x 64 (j)  (8 KiB)
-constexpr uint32_t kRecKbar = 40960;    // Kbar: token-row 128B-swizzled tile 64 x 128 (16 KiB)
+constexpr uint32_t kRecAqk = 32768;     // A_qk^T: token-row tile, row j, column i (8 KiB)
+constexpr uint32_t kRecKbar = 40960;    // Kbar: token-row tile 64 x 128 (16 KiB)
+// [A_qk^T | Kbar] = 24 KiB read as one MN-major B operand (N = 64 + 128, LBO 8 KiB).
 constexpr uint32_t kRecU = 57344;       // U^T: K-major, 128 rows (channel) x 64 (token) (16 KiB)
 constexpr uint32_t kRecGamma = 73728;   // gamma: 128 fp32
 constexpr uint32_t kRecBytes = 74240;
@@ -87,9 +88,7 @@ constexpr float kSafeSpan = 64.f;
 
 // --- state-pass kernel shared memory --------------------------------------
 constexpr uint32_t kStage = 74752;      // record rounded up to 1024
-constexpr uint32_t kP2S = 2 * kStage;   // S0^T bf16, K-major 128 rows x 128 (32 KiB)
-constexpr uint32_t kP2Vp = kP2S + 32768;// V'^T bf16, K-major 128 rows x 64 (16 KiB)
-constexpr uint32_t kP2Bytes = kP2Vp + 16384;
+constexpr uint32_t kP2Bytes = 2 * kStage;
 
 constexpr uint32_t kWaitLimit = 1u << 24;
 
@@ -279,11 +278,8 @@ __global__ void __launch_bounds__(kP1Threads, 3)
         }
       } else {
         const int i = row - kC;
-        float m[32];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) m[jj] = (col0 + jj) <= i ? v[jj] : 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) st_kmajor8(rec + kRecAqk, i, col0 + 8 * e, kC, m + 8 * e);
+        for (int jj = 0; jj < 32; ++jj) stbf(rec + kRecAqk, kmajor_off(col0 + jj, i, kC), (col0 + jj) <= i ? v[jj] : 0.f);
       }
     }
   } else {
@@ -336,12 +332,12 @@ __global__ void __launch_bounds__(kP1Threads, 3)
         while ((i + 1) * (i + 2) / 2 <= p) ++i;
         const int j = p - i * (i + 1) / 2;
         a_blk(sm, blk(i >> 4, j >> 4))[(i & 15) * 16 + (j & 15)] = j < i ? sbeta[i] * akk[t] : 0.f;
-        stbf(rec + kRecAqk, kmajor_off(i, j, kC), scale * aqk[t]);
+        stbf(rec + kRecAqk, kmajor_off(j, i, kC), scale * aqk[t]);
       }
     }
     for (int e = tid; e < kC * kC; e += kP1Threads) {
       const int i = e / kC, j = e % kC;
-      if (j > i) stbf(rec + kRecAqk, kmajor_off(i, j, kC), 0.f);
+      if (j > i) stbf(rec + kRecAqk, kmajor_off(j, i, kC), 0.f);
     }
     // pass 2 (exact): start- and end-decayed operands, factors <= 1
 #pragma unroll
@@ -493,24 +489,30 @@ __global__ void __launch_bounds__(kP1Threads, 3)
 }
 
 // =============================================================== kernel 2
-// Warp roles (256 threads):
+// Warp roles (288 threads):
 //   warps 0-3  "state":  the sequential chain.  Thread j owns TMEM lane j =
-//              value channel j (row j of S^T).  Thread 0 also issues the MMAs.
+//              value channel j (row j of S^T); they convert S0^T and V'^T to
+//              bf16 MMA operands and decay S^T in place.
 //   warps 4-7  "output": read O^T of each chunk from TMEM and store o; thread
-//              128 also streams the per-chunk records into two stages (the
-//              stage of chunk n is free again once chunk n's last MMA, the
-//              one that completes O^T, has finished).
-// Tensor memory (512 columns): S^T [0,128), P = -(W S0)^T [128,192),
-// two O^T buffers [192,256) and [256,320).
-constexpr int kSPThreads = 256;
-constexpr uint32_t kNamedStateBar = 1;
+//              128 also streams the per-chunk records into two stages.
+//   warp  8    "mma":    one thread issues every tcgen05.mma (an issue costs
+//              tens of cycles, so the issuer gets a warp of its own).
+// Tensor memory (fp32 unless noted):
+//   [P | O^T | S^T] at [0,64) [64,128) [128,256)
+//   S0^T as bf16 A operand [256,320), V'^T as bf16 A operand [320,352)
+// Two MMA chains per chunk, both A operands read from tensor memory:
+//   [P | O^T]   = S0^T [-W ; Q+]^T          (N = 128, K = 128: 8 instructions)
+//   [O^T | S^T] += V'^T [A_qk^T | Kbar]      (N = 192, K = 64:  4 instructions)
+// with P = -(W S0)^T and V'^T = U^T + P formed in between on the CUDA cores.
+constexpr int kSPThreads = 288;
+constexpr uint32_t kTmP = 0, kTmO = 64, kTmS = 128, kTmAS = 256, kTmAV = 320;
 
 __global__ void __launch_bounds__(kSPThreads, 1)
     kda_state_pass_kernel(const uint8_t* __restrict__ records, WorkspaceHeader* hdr, const float* s0, float* sT,
                           bf16* __restrict__ o, int T, int H, int NC) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  __shared__ uint64_t bar_full[2], bar_o[2], bar_ofree[2], bar_p, bar_s;
+  __shared__ uint64_t bar_full[2], bar_o, bar_ofree, bar_p, bar_s, bar_as, bar_av;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -520,22 +522,54 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   const size_t sbase = (size_t)bh * kD * kD;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_o[i], 1);
-      mbar_init(&bar_ofree[i], 128);
-    }
+    mbar_init(&bar_full[0], 1);
+    mbar_init(&bar_full[1], 1);
+    mbar_init(&bar_o, 1);
+    mbar_init(&bar_ofree, 128);
     mbar_init(&bar_p, 1);
     mbar_init(&bar_s, 1);
+    mbar_init(&bar_as, 128);
+    mbar_init(&bar_av, 128);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tS = tmem_base, tP = tmem_base + 128, tO = tmem_base + 192;
+  const uint32_t tm = tmem_base;
 
-  if (warp >= 4) {
+  if (warp == 8) {
+    // ------------------------------------------------------------ mma
+    if ((tid & 31) == 0) {
+      const uint32_t id_1 = idesc_bf16_f32(128, 128, 0, 0);  // [P|O] = S0^T [-W;Q+]^T
+      const uint32_t id_2 = idesc_bf16_f32(128, 192, 0, 1);  // [O|S] += V'^T [A_qk^T|Kbar]
+      // first descriptors of each stage; later steps add address offsets (in 16-byte units)
+      const uint64_t d1s0 = desc_sw128(smem_u32(sm + kRecWQ), 16, 1024);
+      const uint64_t d1s1 = desc_sw128(smem_u32(sm + kStage + kRecWQ), 16, 1024);
+      const uint64_t d2s0 = desc_sw128(smem_u32(sm + kRecAqk), 8192, 1024);
+      const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStage + kRecAqk), 8192, 1024);
+      for (int n = 0; n < NC; ++n) {
+        const int s = n & 1;
+        wait_or_flag(&bar_as, n & 1, hdr, 30);
+        wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 31);
+        if (n >= 1) wait_or_flag(&bar_ofree, (n - 1) & 1, hdr, 32);  // O^T of chunk n-1 has been read
+        tc_fence_after();
+        const uint64_t d1 = s ? d1s1 : d1s0, d2 = s ? d2s1 : d2s0;
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k)  // K-major B: +32 B per step inside a 64-wide block, +16 KiB per block
+          mma_bf16_ts(tm + kTmP, tm + kTmAS + k * 8, d1 + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), id_1,
+                      k > 0);
+        mma_commit(&bar_p);
+        wait_or_flag(&bar_av, n & 1, hdr, 33);
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kC / 16; ++k)  // MN-major B: +2 KiB per 16 K-rows
+          mma_bf16_ts(tm + kTmO, tm + kTmAV + k * 8, d2 + (uint64_t)((2 * k * 1024) >> 4), id_2, 1);
+        mma_commit(&bar_s);
+        mma_commit(&bar_o);
+      }
+    }
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ output + loads
     const int j = tid - 128;
     const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
@@ -547,26 +581,31 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     }
     for (int n = 0; n < NC; ++n) {
       const int s = n & 1;
-      wait_or_flag(&bar_o[s], (n >> 1) & 1, hdr, 21);
+      wait_or_flag(&bar_o, n & 1, hdr, 21);
       tc_fence_after();
       if (tid == 128 && n + 2 < NC) {  // every reader of stage s is done with chunk n
         mbar_expect_tx(&bar_full[s], kRecBytes);
         bulk_load(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, kRecBytes, &bar_full[s]);
       }
       uint32_t r[64];
-      tmem_ld32_raw(tO + s * 64 + lane_off, r);
-      tmem_ld32_raw(tO + s * 64 + lane_off + 32, r + 32);
+      tmem_ld32_raw(tm + kTmO + lane_off, r);
+      tmem_ld32_raw(tm + kTmO + lane_off + 32, r + 32);
       tmem_wait_ld();
       reg_pin<64>(r);
       tc_fence_before();
-      mbar_arrive(&bar_ofree[s]);
+      mbar_arrive(&bar_ofree);
       const int t0 = n * kC;
       const int L = min(kC, T - t0);
       bf16* orow = o + (((size_t)b * T + t0) * H + h) * kD + j;
       const size_t ostride = (size_t)H * kD;
+      if (L == kC) {
 #pragma unroll
-      for (int i = 0; i < kC; ++i)
-        if (i < L) orow[(size_t)i * ostride] = __float2bfloat16_rn(__uint_as_float(r[i]));
+        for (int i = 0; i < kC; ++i, orow += ostride) *orow = __float2bfloat16_rn(__uint_as_float(r[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < kC; ++i, orow += ostride)
+          if (i < L) *orow = __float2bfloat16_rn(__uint_as_float(r[i]));
+      }
     }
   } else {
     // ------------------------------------------------------------ state
@@ -578,119 +617,90 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       for (int cb = 0; cb < kD / 32; ++cb) {
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii) v[ii] = s0 ? s0[sbase + (size_t)(cb * 32 + ii) * kD + j] : 0.f;
-        tmem_st32(tS + lane_off + cb * 32, v);
+        tmem_st32(tm + kTmS + lane_off + cb * 32, v);
       }
       tmem_wait_st();
     }
     for (int n = 0; n < NC; ++n) {
       const int s = n & 1;
-      uint8_t* stage = sm + s * kStage;
+      const uint8_t* stage = sm + s * kStage;
       if (n > 0) wait_or_flag(&bar_s, (n - 1) & 1, hdr, 22);
       tc_fence_after();
 
-      // (1) S0^T -> bf16 operand (row j of a K-major 128 x 128 tile)
-      uint32_t sr[kD];
+      // (1) S0^T -> bf16 A operand in tensor memory, 64 columns at a time
 #pragma unroll
-      for (int cb = 0; cb < kD / 32; ++cb) tmem_ld32_raw(tS + lane_off + cb * 32, sr + cb * 32);
-      tmem_wait_ld();
-      reg_pin<kD>(sr);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[64];
+        tmem_ld32_raw(tm + kTmS + lane_off + half * 64, sr);
+        tmem_ld32_raw(tm + kTmS + lane_off + half * 64 + 32, sr + 32);
+        tmem_wait_ld();
+        reg_pin<64>(sr);
+        uint32_t pk[32];
 #pragma unroll
-      for (int k8 = 0; k8 < kD / 8; ++k8) {
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(sr[k8 * 8 + e]);
-        st_kmajor8(sm + kP2S, j, k8 * 8, kD, f);
+        for (int e = 0; e < 32; ++e) pk[e] = pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
+        tmem_st32u(tm + kTmAS + lane_off + half * 32, pk);
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      named_bar_sync(kNamedStateBar, 128);
-      tc_fence_after();
+      mbar_arrive(&bar_as);
 
-      // (2) P = S0^T (-W)^T (critical), then O^T = S0^T Q+^T into this chunk's O buffer
-      if (tid == 0) {
-        wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 23);
-        tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
-        const uint32_t a0 = smem_u32(sm + kP2S), b0 = smem_u32(stage + kRecWQ);
-#pragma unroll
-        for (int k = 0; k < kD / 16; ++k) {
-          const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-          mma_bf16(tP, desc_sw128(a0 + off, 16, 1024), desc_sw128(b0 + off, 16, 1024), idesc, k > 0);
-        }
-        mma_commit(&bar_p);
-        if (n >= 2) wait_or_flag(&bar_ofree[s], ((n - 2) >> 1) & 1, hdr, 24);
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kD / 16; ++k) {
-          const uint32_t off = (k / 4) * 16384 + (k % 4) * 32;
-          mma_bf16(tO + s * 64, desc_sw128(a0 + off, 16, 1024), desc_sw128(b0 + 8192 + off, 16, 1024), idesc,
-                   k > 0);
-        }
-      }
-
-      // (3) S^T <- S^T Diag(gamma) while the MMAs run
+      // (2) S^T <- S^T Diag(gamma) while the MMAs run
       wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 25);
       {
         const float4* gam = reinterpret_cast<const float4*>(stage + kRecGamma);
 #pragma unroll
         for (int cb = 0; cb < kD / 32; ++cb) {
+          uint32_t sr[32];
+          tmem_ld32_raw(tm + kTmS + lane_off + cb * 32, sr);
+          tmem_wait_ld();
+          reg_pin<32>(sr);
           float v[32];
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             const float4 gg = gam[cb * 8 + q4];
-            v[q4 * 4 + 0] = __uint_as_float(sr[cb * 32 + q4 * 4 + 0]) * gg.x;
-            v[q4 * 4 + 1] = __uint_as_float(sr[cb * 32 + q4 * 4 + 1]) * gg.y;
-            v[q4 * 4 + 2] = __uint_as_float(sr[cb * 32 + q4 * 4 + 2]) * gg.z;
-            v[q4 * 4 + 3] = __uint_as_float(sr[cb * 32 + q4 * 4 + 3]) * gg.w;
+            v[q4 * 4 + 0] = __uint_as_float(sr[q4 * 4 + 0]) * gg.x;
+            v[q4 * 4 + 1] = __uint_as_float(sr[q4 * 4 + 1]) * gg.y;
+            v[q4 * 4 + 2] = __uint_as_float(sr[q4 * 4 + 2]) * gg.z;
+            v[q4 * 4 + 3] = __uint_as_float(sr[q4 * 4 + 3]) * gg.w;
           }
-          tmem_st32(tS + lane_off + cb * 32, v);
+          tmem_st32(tm + kTmS + lane_off + cb * 32, v);
         }
-        tmem_wait_st();
       }
 
-      // (4) V'^T = U^T + P  -> bf16 operand (row j of a K-major 128 x 64 tile)
+      // (3) V'^T = U^T + P -> bf16 A operand in tensor memory, 32 columns at a time
+      uint4 urow[4];
+#pragma unroll
+      for (int k8 = 0; k8 < 4; ++k8)
+        urow[k8] = *reinterpret_cast<const uint4*>(stage + kRecU + kmajor_off(j, k8 * 8, kD));
       wait_or_flag(&bar_p, n & 1, hdr, 26);
       tc_fence_after();
-      {
-        uint32_t pr[kC];
-        tmem_ld32_raw(tP + lane_off, pr);
-        tmem_ld32_raw(tP + lane_off + 32, pr + 32);
-        tmem_wait_ld();
-        reg_pin<kC>(pr);
 #pragma unroll
-        for (int k8 = 0; k8 < kC / 8; ++k8) {
-          const uint32_t off = kmajor_off(j, k8 * 8, kD);
-          const uint4 uu = *reinterpret_cast<const uint4*>(stage + kRecU + off);
-          const uint32_t uw[4] = {uu.x, uu.y, uu.z, uu.w};
-          float f[8];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pr[32];
+        tmem_ld32_raw(tm + kTmP + lane_off + half * 32, pr);
+        tmem_wait_ld();
+        reg_pin<32>(pr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+          const uint32_t uw[4] = {urow[k8].x, urow[k8].y, urow[k8].z, urow[k8].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 u2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[e]));
-            f[2 * e] = u2.x + __uint_as_float(pr[k8 * 8 + 2 * e]);
-            f[2 * e + 1] = u2.y + __uint_as_float(pr[k8 * 8 + 2 * e + 1]);
+            pk[k8 * 4 + e] = pack2(u2.x + __uint_as_float(pr[k8 * 8 + 2 * e]),
+                                   u2.y + __uint_as_float(pr[k8 * 8 + 2 * e + 1]));
           }
-          st_kmajor8(sm + kP2Vp, j, k8 * 8, kD, f);
         }
+        if (half == 0) {
+#pragma unroll
+          for (int k8 = 0; k8 < 4; ++k8)
+            urow[k8] = *reinterpret_cast<const uint4*>(stage + kRecU + kmajor_off(j, 32 + k8 * 8, kD));
+        }
+        tmem_st16u(tm + kTmAV + lane_off + half * 16, pk);
       }
-      fence_async_smem();
+      tmem_wait_st();  // also covers the decayed S^T
       tc_fence_before();
-      named_bar_sync(kNamedStateBar, 128);
-      tc_fence_after();
-
-      // (5) S^T += V'^T Kbar (critical), then O^T += V'^T A_qk^T
-      if (tid == 0) {
-        const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);
-        const uint32_t id_o = idesc_bf16_f32(128, 64, 0, 0);
-        const uint32_t vp = smem_u32(sm + kP2Vp), aq = smem_u32(stage + kRecAqk), kbar = smem_u32(stage + kRecKbar);
-#pragma unroll
-        for (int k = 0; k < kC / 16; ++k)
-          mma_bf16(tS, desc_sw128(vp + k * 32, 16, 1024), desc_sw128(kbar + 2 * k * 1024, 8192, 1024), id_s, 1);
-        mma_commit(&bar_s);
-#pragma unroll
-        for (int k = 0; k < kC / 16; ++k)
-          mma_bf16(tO + s * 64, desc_sw128(vp + k * 32, 16, 1024), desc_sw128(aq + k * 32, 16, 1024), id_o, 1);
-        mma_commit(&bar_o[s]);
-      }
+      mbar_arrive(&bar_av);
     }
     wait_or_flag(&bar_s, (NC - 1) & 1, hdr, 27);
     tc_fence_after();
@@ -698,7 +708,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
 #pragma unroll
       for (int cb = 0; cb < kD / 32; ++cb) {
         float v[32];
-        tmem_ld32(tS + lane_off + cb * 32, v);
+        tmem_ld32(tm + kTmS + lane_off + cb * 32, v);
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii) sT[sbase + (size_t)(cb * 32 + ii) * kD + j] = v[ii];
       }
