@@ -80,6 +80,7 @@ constexpr uint32_t kP1B = 49152;
 constexpr uint32_t kP1Bytes = 65536;
 constexpr uint32_t kP1V = kP1A;              // v tile, after the score MMA
 constexpr uint32_t kP1B2 = kP1A + 16384;     // (T diag beta)^T, K-major 64 x 64
+constexpr uint32_t kP1QT = kP1A + 16384;     // A_qk^T staging (bulk-stored before the B2 operand is built)
 constexpr int kP1Threads = 256;
 // Per-chunk safe range of the factored form: every channel's cumulative
 // log-gate over the chunk must stay above -kSafeSpan, so that each factor
@@ -125,6 +126,20 @@ __device__ __forceinline__ float2 ld_bf2(const uint8_t* p) {
 __device__ __forceinline__ void st_bf2(uint8_t* p, float a, float b) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
+// 8 bf16 (16 bytes, 16-byte aligned) <-> 8 floats.
+__device__ __forceinline__ void ld8(const uint8_t* p, float* f) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+    f[2 * e] = t.x;
+    f[2 * e + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void st8(uint8_t* p, const float* f) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
 // The lower-triangular 64 x 64 matrices A_kk and T are kept as 16 x 16 fp32
 // blocks (I, J), J <= I, numbered p = I(I+1)/2 + J; A blocks in region B,
 // T blocks 0-5 after them in region B and T blocks 6-9 at the end of region A.
@@ -134,12 +149,41 @@ __device__ __forceinline__ float* t_blk(uint8_t* sm, int p) {
   return p < 6 ? reinterpret_cast<float*>(sm + kP1B + 10240) + p * 256
                : reinterpret_cast<float*>(sm + kP1A + 24576) + (p - 6) * 256;
 }
-// 16x16x16 block product sum_m X[r][m] * Y[m][c].
-__device__ __forceinline__ float bdot(const float* X, const float* Y, int r, int c) {
-  float acc = 0.f;
+// Warp-level 16x16x16 product acc += P Q of row-major fp32 16x16 blocks, with
+// mma.sync m16n8k8 (tf32 operands rounded to nearest).  acc[nh] holds the
+// 16x8 accumulator fragment of columns 8nh..8nh+7: rows g and g+8, columns
+// 2t and 2t+1, where g = lane / 4 and t = lane % 4.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void block_mma_tf32(float (&acc)[2][4], const float* P, const float* Q, int lane) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int m = 0; m < 16; ++m) acc = fmaf(X[r * 16 + m], Y[m * 16 + c], acc);
-  return acc;
+  for (int kh = 0; kh < 2; ++kh) {
+    const uint32_t a0 = to_tf32(P[g * 16 + 8 * kh + t]), a1 = to_tf32(P[(g + 8) * 16 + 8 * kh + t]);
+    const uint32_t a2 = to_tf32(P[g * 16 + 8 * kh + t + 4]), a3 = to_tf32(P[(g + 8) * 16 + 8 * kh + t + 4]);
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+      const uint32_t b0 = to_tf32(Q[(8 * kh + t) * 16 + 8 * nh + g]), b1 = to_tf32(Q[(8 * kh + t + 4) * 16 + 8 * nh + g]);
+      asm volatile(
+          "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+          "{%0,%1,%2,%3};"
+          : "+f"(acc[nh][0]), "+f"(acc[nh][1]), "+f"(acc[nh][2]), "+f"(acc[nh][3])
+          : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+  }
+}
+__device__ __forceinline__ void store_block_frag(float* X, const float (&acc)[2][4], int lane, float sign) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nh = 0; nh < 2; ++nh) {
+    X[g * 16 + 8 * nh + 2 * t] = sign * acc[nh][0];
+    X[g * 16 + 8 * nh + 2 * t + 1] = sign * acc[nh][1];
+    X[(g + 8) * 16 + 8 * nh + 2 * t] = sign * acc[nh][2];
+    X[(g + 8) * 16 + 8 * nh + 2 * t + 1] = sign * acc[nh][3];
+  }
 }
 
 __global__ void __launch_bounds__(kP1Threads, 3)
@@ -152,7 +196,6 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   __shared__ uint64_t bar_in, bar_v, bar_mma;
   __shared__ uint32_t tmem_base;
   __shared__ float sbeta[kC];
-  __shared__ float stot[4][kD];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x % NC;
@@ -183,66 +226,89 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   const uint32_t tm = tmem_base;
   wait_or_flag(&bar_in, 0, hdr, 1);
 
-  // ---- pass 1: in-chunk cumulative log-gate.  Thread = (token quarter qt,
-  // channel pair c0, c0+1); each keeps its 16 x 2 values of G in registers.
-  const int qt = tid >> 6, c0 = 2 * (tid & 63);
-  float G0[16], G1[16];
+  // ---- pass 1: in-chunk cumulative log-gate.  Thread = (8-channel group cg,
+  // 4-token group tg); the 16 token groups of a channel group are the 16 lanes
+  // of one half-warp, so the scan across token groups is a shuffle scan.
+  const int cg = 2 * warp + (lane >> 4);
+  const int tg = lane & 15;
+  const int c8 = 8 * cg;
+  float excl[8], gref[8], gend[8];
   {
-    float r0 = 0.f, r1 = 0.f;
+    float tot[8];
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) {
-      const float2 f = ld_bf2(sm + kP1A + kmajor_off(qt * 16 + ii, c0, 128));
-      r0 += f.x;
-      r1 += f.y;
-      G0[ii] = r0;
-      G1[ii] = r1;
+    for (int e = 0; e < 8; ++e) tot[e] = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float g8[8];
+      ld8(sm + kP1A + kmajor_off(4 * tg + t, c8, 128), g8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tot[e] += g8[e];
     }
-    stot[qt][c0] = r0;
-    stot[qt][c0 + 1] = r1;
-  }
-  __syncthreads();
-  float off0 = 0.f, off1 = 0.f;
 #pragma unroll
-  for (int q4 = 0; q4 < 3; ++q4)
-    if (q4 < qt) {
-      off0 += stot[q4][c0];
-      off1 += stot[q4][c0 + 1];
+    for (int e = 0; e < 8; ++e) {
+      float x = tot[e];  // inclusive prefix over token groups 0..tg
+#pragma unroll
+      for (int d = 1; d < 16; d <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, d, 16);
+        if (tg >= d) x += y;
+      }
+      const float prev = __shfl_up_sync(0xffffffffu, x, 1, 16);
+      excl[e] = tg == 0 ? 0.f : prev;
+      gref[e] = __shfl_sync(0xffffffffu, x, 7, 16);   // G at token 31
+      gend[e] = __shfl_sync(0xffffffffu, x, 15, 16);  // G at token 63 (= G_C; padding has g = 0)
     }
-  const float gref0 = stot[0][c0] + stot[1][c0], gref1 = stot[0][c0 + 1] + stot[1][c0 + 1];
-  const float gend0 = gref0 + stot[2][c0] + stot[3][c0], gend1 = gref1 + stot[2][c0 + 1] + stot[3][c0 + 1];
+  }
+  bool unsafe = false;
 #pragma unroll
-  for (int ii = 0; ii < 16; ++ii) {
-    G0[ii] += off0;
-    G1[ii] += off1;
+  for (int e = 0; e < 8; ++e) unsafe |= gend[e] < -kSafeSpan;
+  if (tg == 0) {
+    float* gam = reinterpret_cast<float*>(rec + kRecGamma) + c8;
+    *reinterpret_cast<float4*>(gam) = make_float4(expf(gend[0]), expf(gend[1]), expf(gend[2]), expf(gend[3]));
+    *reinterpret_cast<float4*>(gam + 4) = make_float4(expf(gend[4]), expf(gend[5]), expf(gend[6]), expf(gend[7]));
   }
-  if (qt == 0) {
-    reinterpret_cast<float*>(rec + kRecGamma)[c0] = expf(gend0);
-    reinterpret_cast<float*>(rec + kRecGamma)[c0 + 1] = expf(gend1);
-  }
-  // The g tile is dead after this barrier.
-  const int slow = __syncthreads_or((gend0 < -kSafeSpan) || (gend1 < -kSafeSpan));
+  const int slow = __syncthreads_or(unsafe);
 
   if (!slow) {
-    // ---- pass 2 (factored form): decayed operands relative to token kRefTok
-    const float egr0 = __expf(gref0), egr1 = __expf(gref1);
-    const float egb0 = __expf(gend0 - gref0), egb1 = __expf(gend1 - gref1);
+    // ---- pass 2 (factored form): decayed operands relative to token kRefTok.
+    // G is re-accumulated token by token; g row i is read before K+_r
+    // overwrites it (same thread, same bytes).
+    float egr[8], egb[8], G[8];
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) {
-      const int i = qt * 16 + ii;
-      const uint32_t oK = kmajor_off(i, c0, kC);        // 64-row tiles: k, K-_r, Kbar
-      const uint32_t oA = kmajor_off(i, c0, 128);       // row i of region A
-      const uint32_t oQ = kmajor_off(kC + i, c0, 128);  // row 64+i of region A and of the [-W;Q+] image
-      const float2 kk = ld_bf2(sm + kP1K + oK);
-      const float2 qq = ld_bf2(sm + kP1A + oQ);
-      const float ex0 = __expf(G0[ii] - gref0), ex1 = __expf(G1[ii] - gref1);
-      const float ei0 = __expf(gref0 - G0[ii]), ei1 = __expf(gref1 - G1[ii]);
-      const float e00 = ex0 * egr0, e01 = ex1 * egr1;  // exp(G_i)
-      st_bf2(sm + kP1A + oA, kk.x * ex0, kk.y * ex1);                          // K+_r
-      st_bf2(sm + kP1A + oQ, scale * qq.x * ex0, scale * qq.y * ex1);          // Q+_r
-      st_bf2(sm + kP1B + oK, kk.x * ei0, kk.y * ei1);                          // K-_r
-      st_bf2(sm + kP1K + oK, kk.x * e00, kk.y * e01);                          // K+
-      st_bf2(rec + kRecWQ + oQ, scale * qq.x * e00, scale * qq.y * e01);       // Q+ image
-      st_bf2(rec + kRecKbar + oK, kk.x * (ei0 * egb0), kk.y * (ei1 * egb1));   // Kbar image
+    for (int e = 0; e < 8; ++e) {
+      egr[e] = __expf(gref[e]);
+      egb[e] = __expf(gend[e] - gref[e]);
+      G[e] = excl[e];
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int i = 4 * tg + t;
+      const uint32_t oK = kmajor_off(i, c8, kC);        // 64-row tiles: k, K-_r, Kbar
+      const uint32_t oA = kmajor_off(i, c8, 128);       // row i of region A
+      const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A and of the [-W;Q+] image
+      float g8[8], k8[8], q8[8];
+      ld8(sm + kP1A + oA, g8);
+      ld8(sm + kP1K + oK, k8);
+      ld8(sm + kP1A + oQ, q8);
+      float kr[8], qr[8], km[8], kp[8], qp[8], kb[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        G[e] += g8[e];
+        const float ex = __expf(G[e] - gref[e]), ei = __expf(gref[e] - G[e]);
+        const float e0 = ex * egr[e];  // exp(G_i)
+        const float sq = scale * q8[e];
+        kr[e] = k8[e] * ex;
+        qr[e] = sq * ex;
+        km[e] = k8[e] * ei;
+        kp[e] = k8[e] * e0;
+        qp[e] = sq * e0;
+        kb[e] = k8[e] * (ei * egb[e]);  // k exp(G_C - G_i)
+      }
+      st8(sm + kP1A + oA, kr);              // K+_r
+      st8(sm + kP1A + oQ, qr);              // Q+_r (in place of q)
+      st8(sm + kP1B + oK, km);              // K-_r
+      st8(sm + kP1K + oK, kp);              // K+ (chunk start), in place of k
+      st8(rec + kRecWQ + oQ, qp);           // Q+ image
+      st8(rec + kRecKbar + oK, kb);         // Kbar image
     }
     fence_async_smem();
     tc_fence_before();
@@ -252,17 +318,17 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     // ---- score MMA: D[0:128, 0:64] = [K+_r ; Q+_r] (128 x 128) . K-_r^T
     if (tid == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t a0 = smem_u32(sm + kP1A), b0 = smem_u32(sm + kP1B);
+      const uint64_t a0 = desc_sw128(smem_u32(sm + kP1A), 16, 1024), b0 = desc_sw128(smem_u32(sm + kP1B), 16, 1024);
 #pragma unroll
       for (int k = 0; k < kD / 16; ++k)
-        mma_bf16(tm, desc_sw128(a0 + (k / 4) * 16384 + (k % 4) * 32, 16, 1024),
-                 desc_sw128(b0 + (k / 4) * 8192 + (k % 4) * 32, 16, 1024), idesc, k > 0);
+        mma_bf16(tm, a0 + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4),
+                 b0 + (uint64_t)(((k / 4) * 8192 + (k % 4) * 32) >> 4), idesc, k > 0);
       mma_commit(&bar_mma);
     }
     wait_or_flag(&bar_mma, 0, hdr, 2);
     tc_fence_after();
 
-    // ---- rows 0-63 -> A_kk blocks (times beta_i, strictly lower); rows 64-127 -> A_qk image
+    // ---- rows 0-63 -> A_kk blocks (times beta_i, strictly lower); rows 64-127 -> A_qk^T staging
     {
       const int row = (warp & 3) * 32 + lane;
       const int col0 = (warp >> 2) * 32;
@@ -272,30 +338,58 @@ __global__ void __launch_bounds__(kP1Threads, 3)
         const int i = row, I = i >> 4;
         const float bi = sbeta[i];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int j = col0 + jj, J = j >> 4;
-          if (J <= I) a_blk(sm, blk(I, J))[(i & 15) * 16 + (j & 15)] = j < i ? bi * v[jj] : 0.f;
+        for (int half = 0; half < 2; ++half) {
+          const int J = (col0 >> 4) + half;
+          if (J <= I) {
+            float4* dst = reinterpret_cast<float4*>(a_blk(sm, blk(I, J)) + (i & 15) * 16);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              float w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int jj = half * 16 + q4 * 4 + e;
+                w[e] = (col0 + jj) < i ? bi * v[jj] : 0.f;
+              }
+              dst[q4] = make_float4(w[0], w[1], w[2], w[3]);
+            }
+          }
         }
       } else {
         const int i = row - kC;
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) stbf(rec + kRecAqk, kmajor_off(col0 + jj, i, kC), (col0 + jj) <= i ? v[jj] : 0.f);
+        for (int jj = 0; jj < 32; ++jj) stbf(sm + kP1QT, kmajor_off(col0 + jj, i, kC), (col0 + jj) <= i ? v[jj] : 0.f);
       }
     }
   } else {
     // ---- exact path for chunks whose gates decay past e^-64: the score
     // matrices straight from their definition, every decay factor
     // exp(G_i - G_j) <= 1 formed per (pair, channel).
+    float G[4][8];
+    {
+      float run[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) run[e] = excl[e];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float g8[8];
+        ld8(sm + kP1A + kmajor_off(4 * tg + t, c8, 128), g8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          run[e] += g8[e];
+          G[t][e] = run[e];
+        }
+      }
+    }
+    __syncthreads();  // every g read is done before G overwrites it
     auto gp = [&](int i, int c) -> float* {
       return c < 32 ? reinterpret_cast<float*>(sm + kP1A) + i * 32 + c
                     : c < 64 ? reinterpret_cast<float*>(sm + kP1A + 16384) + i * 32 + (c - 32)
                              : reinterpret_cast<float*>(sm + kP1B) + i * 64 + (c - 64);
     };
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) {
-      *gp(qt * 16 + ii, c0) = G0[ii];
-      *gp(qt * 16 + ii, c0 + 1) = G1[ii];
-    }
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) *gp(4 * tg + t, c8 + e) = G[t][e];
     __syncthreads();
     constexpr int kPairs = kC * (kC + 1) / 2;  // (i, j) with j <= i
     float akk[9], aqk[9];
@@ -332,30 +426,42 @@ __global__ void __launch_bounds__(kP1Threads, 3)
         while ((i + 1) * (i + 2) / 2 <= p) ++i;
         const int j = p - i * (i + 1) / 2;
         a_blk(sm, blk(i >> 4, j >> 4))[(i & 15) * 16 + (j & 15)] = j < i ? sbeta[i] * akk[t] : 0.f;
-        stbf(rec + kRecAqk, kmajor_off(j, i, kC), scale * aqk[t]);
+        stbf(sm + kP1QT, kmajor_off(j, i, kC), scale * aqk[t]);
       }
     }
     for (int e = tid; e < kC * kC; e += kP1Threads) {
       const int i = e / kC, j = e % kC;
-      if (j > i) stbf(rec + kRecAqk, kmajor_off(j, i, kC), 0.f);
+      if (j > i) stbf(sm + kP1QT, kmajor_off(j, i, kC), 0.f);
     }
     // pass 2 (exact): start- and end-decayed operands, factors <= 1
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) {
-      const int i = qt * 16 + ii;
-      const uint32_t oK = kmajor_off(i, c0, kC);
-      const uint32_t oQ = kmajor_off(kC + i, c0, 128);
-      const float2 kk = ld_bf2(sm + kP1K + oK);
-      const float2 qq = ld_bf2(sm + kP1A + oQ);
-      const float e00 = __expf(G0[ii]), e01 = __expf(G1[ii]);
-      st_bf2(sm + kP1K + oK, kk.x * e00, kk.y * e01);
-      st_bf2(rec + kRecWQ + oQ, scale * qq.x * e00, scale * qq.y * e01);
-      st_bf2(rec + kRecKbar + oK, kk.x * __expf(gend0 - G0[ii]), kk.y * __expf(gend1 - G1[ii]));
+    for (int t = 0; t < 4; ++t) {
+      const int i = 4 * tg + t;
+      const uint32_t oK = kmajor_off(i, c8, kC);
+      const uint32_t oQ = kmajor_off(kC + i, c8, 128);
+      float k8[8], q8[8], kp[8], qp[8], kb[8];
+      ld8(sm + kP1K + oK, k8);
+      ld8(sm + kP1A + oQ, q8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float e0 = __expf(G[t][e]);
+        kp[e] = k8[e] * e0;
+        qp[e] = scale * q8[e] * e0;
+        kb[e] = k8[e] * __expf(gend[e] - G[t][e]);
+      }
+      st8(sm + kP1K + oK, kp);
+      st8(rec + kRecWQ + oQ, qp);
+      st8(rec + kRecKbar + oK, kb);
     }
   }
+  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid == 0) {
+    bulk_store(rec + kRecAqk, sm + kP1QT, 8192);
+    bulk_commit();
+  }
 
   // ---- region A is free: bring the v tile while the triangle is inverted
   if (tid == 0) {
@@ -381,45 +487,30 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     for (int r = 0; r < 16; ++r) Tb[r * 16 + jj] = t[r];
   }
   __syncthreads();
-  // off-diagonal blocks, one sub-diagonal at a time:
-  //   T_IJ = -T_II * (sum_{K=J}^{I-1} A_IK T_KJ)
+  // off-diagonal blocks, one sub-diagonal at a time, one warp per block:
+  //   X = sum_{K=J}^{I-1} A_IK T_KJ,   T_IJ = -T_II X
+  // as 16x16x16 products on the warp-level tensor cores (tf32 in, fp32
+  // accumulate; the result is rounded to bf16 for the W/U MMAs afterwards).
 #pragma unroll 1
   for (int d = 1; d < 4; ++d) {
-    const int nb = 4 - d;  // blocks (J+d, J), J = 0..nb-1
-    float y[3];
-#pragma unroll
-    for (int q = 0; q < 3; ++q) {
-      const int e = tid + q * kP1Threads;
-      if (q < nb) {
-        const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
-        float x = 0.f;
-        for (int K = J; K < I; ++K) x += bdot(a_blk(sm, blk(I, K)), t_blk(sm, blk(K, J)), r, c);
-        y[q] = x;
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < 3; ++q) {
-      const int e = tid + q * kP1Threads;
-      if (q < nb) t_blk(sm, blk((e >> 8) + d, e >> 8))[e & 255] = y[q];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < 3; ++q) {
-      const int e = tid + q * kP1Threads;
-      if (q < nb) {
-        const int J = e >> 8, I = J + d, r = (e >> 4) & 15, c = e & 15;
-        y[q] = -bdot(t_blk(sm, blk(I, I)), t_blk(sm, blk(I, J)), r, c);
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < 3; ++q) {
-      const int e = tid + q * kP1Threads;
-      if (q < nb) t_blk(sm, blk((e >> 8) + d, e >> 8))[e & 255] = y[q];
+    if (warp < 4 - d) {
+      const int J = warp, I = J + d;
+      float* Tij = t_blk(sm, blk(I, J));
+      float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int K = J; K < I; ++K) block_mma_tf32(x, a_blk(sm, blk(I, K)), t_blk(sm, blk(K, J)), lane);
+      store_block_frag(Tij, x, lane, 1.f);  // X parked in the slot of T_IJ
+      __syncwarp();
+      float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      block_mma_tf32(y, t_blk(sm, blk(I, I)), Tij, lane);
+      __syncwarp();
+      store_block_frag(Tij, y, lane, -1.f);
     }
     __syncthreads();
   }
   // (T diag(beta))^T as the K-major B operand of the W/U MMAs: row n = i, column k = j.
+  // It reuses the A_qk^T staging bytes, so the bulk store must have read them.
+  if (tid == 0) bulk_wait_read();
+  __syncthreads();
   {
     const int i = tid >> 2, j0 = (tid & 3) * 16, I = i >> 4, J = j0 >> 4;
     float vals[16];
