@@ -144,6 +144,10 @@ __device__ __forceinline__ void st8(uint8_t* p, const float* f) {
 // blocks (I, J), J <= I, numbered p = I(I+1)/2 + J; A blocks in region B,
 // T blocks 0-5 after them in region B and T blocks 6-9 at the end of region A.
 __device__ __forceinline__ int blk(int I, int J) { return I * (I + 1) / 2 + J; }
+// Element (r, c) of a 16 x 16 block: rows of 16 floats with the float4 column
+// XOR-ed by (r/2)%4, so that 8 consecutive rows at one float4 column hit 8
+// different 16-byte bank groups.
+__device__ __forceinline__ int bidx(int r, int c) { return r * 16 + ((((c >> 2) ^ ((r >> 1) & 3)) << 2) | (c & 3)); }
 __device__ __forceinline__ float* a_blk(uint8_t* sm, int p) { return reinterpret_cast<float*>(sm + kP1B) + p * 256; }
 __device__ __forceinline__ float* t_blk(uint8_t* sm, int p) {
   return p < 6 ? reinterpret_cast<float*>(sm + kP1B + 10240) + p * 256
@@ -162,11 +166,11 @@ __device__ __forceinline__ void block_mma_tf32(float (&acc)[2][4], const float* 
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int kh = 0; kh < 2; ++kh) {
-    const uint32_t a0 = to_tf32(P[g * 16 + 8 * kh + t]), a1 = to_tf32(P[(g + 8) * 16 + 8 * kh + t]);
-    const uint32_t a2 = to_tf32(P[g * 16 + 8 * kh + t + 4]), a3 = to_tf32(P[(g + 8) * 16 + 8 * kh + t + 4]);
+    const uint32_t a0 = to_tf32(P[bidx(g, 8 * kh + t)]), a1 = to_tf32(P[bidx(g + 8, 8 * kh + t)]);
+    const uint32_t a2 = to_tf32(P[bidx(g, 8 * kh + t + 4)]), a3 = to_tf32(P[bidx(g + 8, 8 * kh + t + 4)]);
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh) {
-      const uint32_t b0 = to_tf32(Q[(8 * kh + t) * 16 + 8 * nh + g]), b1 = to_tf32(Q[(8 * kh + t + 4) * 16 + 8 * nh + g]);
+      const uint32_t b0 = to_tf32(Q[bidx(8 * kh + t, 8 * nh + g)]), b1 = to_tf32(Q[bidx(8 * kh + t + 4, 8 * nh + g)]);
       asm volatile(
           "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
           "{%0,%1,%2,%3};"
@@ -179,10 +183,10 @@ __device__ __forceinline__ void store_block_frag(float* X, const float (&acc)[2]
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int nh = 0; nh < 2; ++nh) {
-    X[g * 16 + 8 * nh + 2 * t] = sign * acc[nh][0];
-    X[g * 16 + 8 * nh + 2 * t + 1] = sign * acc[nh][1];
-    X[(g + 8) * 16 + 8 * nh + 2 * t] = sign * acc[nh][2];
-    X[(g + 8) * 16 + 8 * nh + 2 * t + 1] = sign * acc[nh][3];
+    X[bidx(g, 8 * nh + 2 * t)] = sign * acc[nh][0];
+    X[bidx(g, 8 * nh + 2 * t + 1)] = sign * acc[nh][1];
+    X[bidx(g + 8, 8 * nh + 2 * t)] = sign * acc[nh][2];
+    X[bidx(g + 8, 8 * nh + 2 * t + 1)] = sign * acc[nh][3];
   }
 }
 
@@ -227,36 +231,35 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   wait_or_flag(&bar_in, 0, hdr, 1);
 
   // ---- pass 1: in-chunk cumulative log-gate.  Thread = (8-channel group cg,
-  // 4-token group tg); the 16 token groups of a channel group are the 16 lanes
-  // of one half-warp, so the scan across token groups is a shuffle scan.
+  // token lane tg) owning tokens tg, tg+16, tg+32, tg+48: the 8 lanes of a
+  // quarter-warp then touch rows of 8 different swizzle phases (no bank
+  // conflicts).  Inclusive scans over the 16 lanes of each token stride,
+  // then the stride totals are added in order.
   const int cg = 2 * warp + (lane >> 4);
   const int tg = lane & 15;
   const int c8 = 8 * cg;
-  float excl[8], gref[8], gend[8];
-  {
-    float tot[8];
+  float G[4][8], gref[8], gend[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) tot[e] = 0.f;
+  for (int t = 0; t < 4; ++t) ld8(sm + kP1A + kmajor_off(tg + 16 * t, c8, 128), G[t]);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    float tot[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      float g8[8];
-      ld8(sm + kP1A + kmajor_off(4 * tg + t, c8, 128), g8);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) tot[e] += g8[e];
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float x = tot[e];  // inclusive prefix over token groups 0..tg
+      float x = G[t][e];
 #pragma unroll
       for (int d = 1; d < 16; d <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, x, d, 16);
         if (tg >= d) x += y;
       }
-      const float prev = __shfl_up_sync(0xffffffffu, x, 1, 16);
-      excl[e] = tg == 0 ? 0.f : prev;
-      gref[e] = __shfl_sync(0xffffffffu, x, 7, 16);   // G at token 31
-      gend[e] = __shfl_sync(0xffffffffu, x, 15, 16);  // G at token 63 (= G_C; padding has g = 0)
+      G[t][e] = x;
+      tot[t] = __shfl_sync(0xffffffffu, x, 15, 16);
     }
+    G[1][e] += tot[0];
+    G[2][e] += tot[0] + tot[1];
+    G[3][e] += (tot[0] + tot[1]) + tot[2];
+    gref[e] = tot[0] + tot[1];                 // G at token 31
+    gend[e] = ((tot[0] + tot[1]) + tot[2]) + tot[3];  // G at token 63 (= G_C; padding has g = 0)
   }
   bool unsafe = false;
 #pragma unroll
@@ -266,49 +269,50 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     *reinterpret_cast<float4*>(gam) = make_float4(expf(gend[0]), expf(gend[1]), expf(gend[2]), expf(gend[3]));
     *reinterpret_cast<float4*>(gam + 4) = make_float4(expf(gend[4]), expf(gend[5]), expf(gend[6]), expf(gend[7]));
   }
-  const int slow = __syncthreads_or(unsafe);
+  const int slow = __syncthreads_or(unsafe);  // the g tile is dead from here on
 
   if (!slow) {
-    // ---- pass 2 (factored form): decayed operands relative to token kRefTok.
-    // G is re-accumulated token by token; g row i is read before K+_r
-    // overwrites it (same thread, same bytes).
-    float egr[8], egb[8], G[8];
+    // ---- pass 2 (factored form): decayed operands relative to token kRefTok
+    float egr[8], egb[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       egr[e] = __expf(gref[e]);
       egb[e] = __expf(gend[e] - gref[e]);
-      G[e] = excl[e];
     }
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      const int i = 4 * tg + t;
+      const int i = tg + 16 * t;
       const uint32_t oK = kmajor_off(i, c8, kC);        // 64-row tiles: k, K-_r, Kbar
       const uint32_t oA = kmajor_off(i, c8, 128);       // row i of region A
       const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A and of the [-W;Q+] image
-      float g8[8], k8[8], q8[8];
-      ld8(sm + kP1A + oA, g8);
+      float k8[8], q8[8];
       ld8(sm + kP1K + oK, k8);
       ld8(sm + kP1A + oQ, q8);
-      float kr[8], qr[8], km[8], kp[8], qp[8], kb[8];
+      float ex[8], ei[8], w[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        G[e] += g8[e];
-        const float ex = __expf(G[e] - gref[e]), ei = __expf(gref[e] - G[e]);
-        const float e0 = ex * egr[e];  // exp(G_i)
-        const float sq = scale * q8[e];
-        kr[e] = k8[e] * ex;
-        qr[e] = sq * ex;
-        km[e] = k8[e] * ei;
-        kp[e] = k8[e] * e0;
-        qp[e] = sq * e0;
-        kb[e] = k8[e] * (ei * egb[e]);  // k exp(G_C - G_i)
+        ex[e] = __expf(G[t][e] - gref[e]);
+        ei[e] = __expf(gref[e] - G[t][e]);
+        q8[e] *= scale;
       }
-      st8(sm + kP1A + oA, kr);              // K+_r
-      st8(sm + kP1A + oQ, qr);              // Q+_r (in place of q)
-      st8(sm + kP1B + oK, km);              // K-_r
-      st8(sm + kP1K + oK, kp);              // K+ (chunk start), in place of k
-      st8(rec + kRecWQ + oQ, qp);           // Q+ image
-      st8(rec + kRecKbar + oK, kb);         // Kbar image
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = k8[e] * ex[e];
+      st8(sm + kP1A + oA, w);               // K+_r (over the dead g rows)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = q8[e] * ex[e];
+      st8(sm + kP1A + oQ, w);               // Q+_r (in place of q)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = k8[e] * ei[e];
+      st8(sm + kP1B + oK, w);               // K-_r
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ex[e] * egr[e]);
+      st8(sm + kP1K + oK, w);               // K+ = k exp(G_i), in place of k
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * egr[e]);
+      st8(rec + kRecWQ + oQ, w);            // Q+ image
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ei[e] * egb[e]);
+      st8(rec + kRecKbar + oK, w);          // Kbar image = k exp(G_C - G_i)
     }
     fence_async_smem();
     tc_fence_before();
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
         for (int half = 0; half < 2; ++half) {
           const int J = (col0 >> 4) + half;
           if (J <= I) {
-            float4* dst = reinterpret_cast<float4*>(a_blk(sm, blk(I, J)) + (i & 15) * 16);
+            float* dst = a_blk(sm, blk(I, J));
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               float w[4];
@@ -350,7 +354,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
                 const int jj = half * 16 + q4 * 4 + e;
                 w[e] = (col0 + jj) < i ? bi * v[jj] : 0.f;
               }
-              dst[q4] = make_float4(w[0], w[1], w[2], w[3]);
+              *reinterpret_cast<float4*>(dst + bidx(i & 15, q4 * 4)) = make_float4(w[0], w[1], w[2], w[3]);
             }
           }
         }
@@ -364,23 +368,6 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     // ---- exact path for chunks whose gates decay past e^-64: the score
     // matrices straight from their definition, every decay factor
     // exp(G_i - G_j) <= 1 formed per (pair, channel).
-    float G[4][8];
-    {
-      float run[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) run[e] = excl[e];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        float g8[8];
-        ld8(sm + kP1A + kmajor_off(4 * tg + t, c8, 128), g8);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          run[e] += g8[e];
-          G[t][e] = run[e];
-        }
-      }
-    }
-    __syncthreads();  // every g read is done before G overwrites it
     auto gp = [&](int i, int c) -> float* {
       return c < 32 ? reinterpret_cast<float*>(sm + kP1A) + i * 32 + c
                     : c < 64 ? reinterpret_cast<float*>(sm + kP1A + 16384) + i * 32 + (c - 32)
@@ -389,7 +376,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
 #pragma unroll
     for (int t = 0; t < 4; ++t)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) *gp(4 * tg + t, c8 + e) = G[t][e];
+      for (int e = 0; e < 8; ++e) *gp(tg + 16 * t, c8 + e) = G[t][e];
     __syncthreads();
     constexpr int kPairs = kC * (kC + 1) / 2;  // (i, j) with j <= i
     float akk[9], aqk[9];
@@ -425,7 +412,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
         while (i * (i + 1) / 2 > p) --i;
         while ((i + 1) * (i + 2) / 2 <= p) ++i;
         const int j = p - i * (i + 1) / 2;
-        a_blk(sm, blk(i >> 4, j >> 4))[(i & 15) * 16 + (j & 15)] = j < i ? sbeta[i] * akk[t] : 0.f;
+        a_blk(sm, blk(i >> 4, j >> 4))[bidx(i & 15, j & 15)] = j < i ? sbeta[i] * akk[t] : 0.f;
         stbf(sm + kP1QT, kmajor_off(j, i, kC), scale * aqk[t]);
       }
     }
@@ -436,7 +423,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     // pass 2 (exact): start- and end-decayed operands, factors <= 1
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      const int i = 4 * tg + t;
+      const int i = tg + 16 * t;
       const uint32_t oK = kmajor_off(i, c8, kC);
       const uint32_t oQ = kmajor_off(kC + i, c8, 128);
       float k8[8], q8[8], kp[8], qp[8], kb[8];
@@ -479,12 +466,12 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     for (int r = 0; r < 16; ++r) {
       float acc = 0.f;
 #pragma unroll
-      for (int m = 0; m < r; ++m) acc = fmaf(A[r * 16 + m], t[m], acc);
+      for (int m = 0; m < r; ++m) acc = fmaf(A[bidx(r, m)], t[m], acc);
       t[r] = r < jj ? 0.f : (r == jj ? 1.f : -acc);
     }
     float* Tb = t_blk(sm, blk(I, I));
 #pragma unroll
-    for (int r = 0; r < 16; ++r) Tb[r * 16 + jj] = t[r];
+    for (int r = 0; r < 16; ++r) Tb[bidx(r, jj)] = t[r];
   }
   __syncthreads();
   // off-diagonal blocks, one sub-diagonal at a time, one warp per block:
@@ -517,7 +504,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     if (J <= I) {
       const float* Tb = t_blk(sm, blk(I, J));
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) vals[jj] = (j0 + jj) <= i ? Tb[(i & 15) * 16 + jj] * sbeta[j0 + jj] : 0.f;
+      for (int jj = 0; jj < 16; ++jj) vals[jj] = (j0 + jj) <= i ? Tb[bidx(i & 15, jj)] * sbeta[j0 + jj] : 0.f;
     } else {
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) vals[jj] = 0.f;
