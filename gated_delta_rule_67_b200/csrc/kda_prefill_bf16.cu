@@ -89,9 +89,11 @@ constexpr float kSafeSpan = 64.f;
 
 // --- state-pass kernel shared memory --------------------------------------
 constexpr uint32_t kStage = 74752;      // record rounded up to 1024
-constexpr uint32_t kP2Bytes = 2 * kStage;
+constexpr uint32_t kP2Out = 2 * kStage;     // two 16 KiB output staging tiles [half][token][64 ch] bf16
+constexpr uint32_t kP2Bytes = kP2Out + 2 * 16384;
 
 constexpr uint32_t kWaitLimit = 1u << 24;
+constexpr uint32_t kSpinLimit = 1u << 30;  // ~seconds of test_wait probes
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -114,6 +116,13 @@ __device__ __forceinline__ void st_kmajor8(uint8_t* tile, uint32_t r, uint32_t k
 
 __device__ __forceinline__ void wait_or_flag(uint64_t* bar, uint32_t parity, WorkspaceHeader* hdr, uint32_t where) {
   if (!mbar_wait(bar, parity, kWaitLimit)) {
+    atomicOr(&hdr->error, 1u);
+    atomicExch(&hdr->where, where);
+  }
+}
+// Same, spinning (for the sequential chain, where wake-up latency is the cost).
+__device__ __forceinline__ void spin_or_flag(uint64_t* bar, uint32_t parity, WorkspaceHeader* hdr, uint32_t where) {
+  if (!mbar_spin(bar, parity, kSpinLimit)) {
     atomicOr(&hdr->error, 1u);
     atomicExch(&hdr->where, where);
   }
@@ -571,10 +580,15 @@ __global__ void __launch_bounds__(kP1Threads, 3)
 //   warps 0-3  "state":  the sequential chain.  Thread j owns TMEM lane j =
 //              value channel j (row j of S^T); they convert S0^T and V'^T to
 //              bf16 MMA operands and decay S^T in place.
-//   warps 4-7  "output": read O^T of each chunk from TMEM and store o; thread
-//              128 also streams the per-chunk records into two stages.
+//   warps 4-7  "output": read O^T of each chunk from TMEM, stage it in shared
+//              memory and store it with two TMA tile stores (scattered 2-byte
+//              global stores from these warps were found to slow the tensor
+//              pipe down by half).
 //   warp  8    "mma":    one thread issues every tcgen05.mma (an issue costs
 //              tens of cycles, so the issuer gets a warp of its own).
+//   Thread 128 also streams the per-chunk records into two stages; it issues
+//   each copy only after releasing O^T, since a bulk-copy issue holds up its
+//   warp and the MMA warp waits for that release.
 // Tensor memory (fp32 unless noted):
 //   [P | O^T | S^T] at [0,64) [64,128) [128,256)
 //   S0^T as bf16 A operand [256,320), V'^T as bf16 A operand [320,352)
@@ -586,8 +600,8 @@ constexpr int kSPThreads = 288;
 constexpr uint32_t kTmP = 0, kTmO = 64, kTmS = 128, kTmAS = 256, kTmAV = 320;
 
 __global__ void __launch_bounds__(kSPThreads, 1)
-    kda_state_pass_kernel(const uint8_t* __restrict__ records, WorkspaceHeader* hdr, const float* s0, float* sT,
-                          bf16* __restrict__ o, int T, int H, int NC) {
+    kda_state_pass_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* __restrict__ records,
+                          WorkspaceHeader* hdr, const float* s0, float* sT, int T, int H, int NC) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t bar_full[2], bar_o, bar_ofree, bar_p, bar_s, bar_as, bar_av;
@@ -661,10 +675,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       const int s = n & 1;
       wait_or_flag(&bar_o, n & 1, hdr, 21);
       tc_fence_after();
-      if (tid == 128 && n + 2 < NC) {  // every reader of stage s is done with chunk n
-        mbar_expect_tx(&bar_full[s], kRecBytes);
-        bulk_load(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, kRecBytes, &bar_full[s]);
-      }
       uint32_t r[64];
       tmem_ld32_raw(tm + kTmO + lane_off, r);
       tmem_ld32_raw(tm + kTmO + lane_off + 32, r + 32);
@@ -672,19 +682,27 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       reg_pin<64>(r);
       tc_fence_before();
       mbar_arrive(&bar_ofree);
-      const int t0 = n * kC;
-      const int L = min(kC, T - t0);
-      bf16* orow = o + (((size_t)b * T + t0) * H + h) * kD + j;
-      const size_t ostride = (size_t)H * kD;
-      if (L == kC) {
+      if (tid == 128 && n + 2 < NC) {  // every reader of stage s is done with chunk n
+        mbar_expect_tx(&bar_full[s], kRecBytes);
+        bulk_load(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, kRecBytes, &bar_full[s]);
+      }
+      // staging tile n%2 must no longer be read by the TMA store of chunk n-2
+      if (tid == 128) bulk_wait_read_n<1>();
+      named_bar_sync(2, 128);
+      uint8_t* stg = sm + kP2Out + (n & 1) * 16384 + (j >> 6) * 8192 + (j & 63) * 2;
 #pragma unroll
-        for (int i = 0; i < kC; ++i, orow += ostride) *orow = __float2bfloat16_rn(__uint_as_float(r[i]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < kC; ++i, orow += ostride)
-          if (i < L) *orow = __float2bfloat16_rn(__uint_as_float(r[i]));
+      for (int i = 0; i < kC; ++i)
+        *reinterpret_cast<bf16*>(stg + i * 128) = __float2bfloat16_rn(__uint_as_float(r[i]));
+      fence_async_smem();
+      named_bar_sync(2, 128);
+      if (tid == 128) {
+        const uint8_t* src = sm + kP2Out + (n & 1) * 16384;
+        tma_store_4d(&tm_o, src, 0, h, n * kC, b);
+        tma_store_4d(&tm_o, src + 8192, 64, h, n * kC, b);
+        bulk_commit();
       }
     }
+    if (tid == 128) bulk_wait_read_n<0>();
   } else {
     // ------------------------------------------------------------ state
     const int j = tid;
@@ -813,7 +831,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 // [B, T, H, 128] bf16 viewed as a 4-D tensor (channel, head, token, batch);
 // box = 64 channels x 1 head x 64 tokens, 128-byte swizzle; tokens past T
 // read as zeros.
-bool make_map(CUtensorMap* map, const void* base, int B, int T, int H) {
+bool make_map(CUtensorMap* map, const void* base, int B, int T, int H, bool swizzle = true) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -821,7 +839,8 @@ bool make_map(CUtensorMap* map, const void* base, int B, int T, int H) {
   cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -847,9 +866,9 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     if (e != cudaSuccess) return e;
     attrs_set = true;
   }
-  CUtensorMap mq, mk, mv, mg;
+  CUtensorMap mq, mk, mv, mg, mo;
   if (!make_map(&mq, q, B, T, H) || !make_map(&mk, k, B, T, H) || !make_map(&mv, v, B, T, H) ||
-      !make_map(&mg, g, B, T, H))
+      !make_map(&mg, g, B, T, H) || !make_map(&mo, o, B, T, H, false))
     return cudaErrorInvalidValue;
   const int NC = (T + kC - 1) / kC;
   WorkspaceHeader* hdr = static_cast<WorkspaceHeader*>(ws);
@@ -863,8 +882,8 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e != cudaSuccess) return e;
-  kda_state_pass_kernel<<<(unsigned)(B * H), kSPThreads, kP2Bytes + 1024, stream>>>(records, hdr, s0, sT, o, T,
-                                                                                     H, NC);
+  kda_state_pass_kernel<<<(unsigned)(B * H), kSPThreads, kP2Bytes + 1024, stream>>>(mo, records, hdr, s0, sT, T, H,
+                                                                                     NC);
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 2, stream);
   return e;
