@@ -227,7 +227,7 @@ def run_ours(args, cfg):
     ins = [x[n] for n in names]
     s0 = x["initial_state"]
     o = torch.empty_like(x["v"])
-    sT = torch.empty_like(s0)
+    sT = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
     ws = torch.empty(max(1, kda_chunk_fwd_workspace_size(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.chunk,
                                                            cfg.torch_dtype)), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB of L2
@@ -271,7 +271,7 @@ def run_ours(args, cfg):
     value = weak_scaling_value(tokens * args.steps, world, total_s)
     ms_per_step = 1e3 * total_s / args.steps
     flops = prefill_flops_per_token_head(cfg.dk) * tokens * cfg.H
-    nbytes = prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, 2, s0 is not None, True)
+    nbytes = prefill_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, 4 if cfg.dtype == "f32" else 2, s0 is not None, True)
     mean_prep, mean_state = statistics.mean(prep_ms), statistics.mean(state_ms)
     dom = "kda_state_pass" if mean_state >= mean_prep else "kda_chunk_prep"
 
@@ -292,17 +292,18 @@ def run_ours(args, cfg):
 
     # ---- end to end through the public API with pinned host buffers
     h_ins = [t.cpu().pin_memory() for t in ins]
-    h_s0 = s0.cpu().pin_memory()
+    h_s0 = None if s0 is None else s0.cpu().pin_memory()
     h_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     h_sT = torch.empty(sT.shape, dtype=sT.dtype, pin_memory=True)
     d_ins = [torch.empty_like(t) for t in ins]
-    d_s0 = torch.empty_like(s0)
+    d_s0 = None if s0 is None else torch.empty_like(s0)
     e2e_steps = max(3, min(args.steps, 50))
 
     def e2e_step():
         for d, hsrc in zip(d_ins, h_ins):
             d.copy_(hsrc, non_blocking=True)
-        d_s0.copy_(h_s0, non_blocking=True)
+        if d_s0 is not None:
+            d_s0.copy_(h_s0, non_blocking=True)
         kda_chunk_fwd(*d_ins, cfg.scale, d_s0, chunk=cfg.chunk, o=o, final_state=sT, workspace=ws)
         h_o.copy_(o, non_blocking=True)
         h_sT.copy_(sT, non_blocking=True)
@@ -317,7 +318,7 @@ def run_ours(args, cfg):
     eb.record()
     torch.cuda.synchronize()
     e2e_s = reduce_max(ea.elapsed_time(eb) / 1e3, dev)
-    h2d = sum(t.numel() * t.element_size() for t in h_ins) + h_s0.numel() * 4
+    h2d = sum(t.numel() * t.element_size() for t in h_ins) + (0 if h_s0 is None else h_s0.numel() * 4)
     d2h = h_o.numel() * h_o.element_size() + h_sT.numel() * 4
     e2e = {"value": weak_scaling_value(tokens * e2e_steps, world, e2e_s), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
@@ -361,7 +362,7 @@ def run_ours(args, cfg):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": DATA,
+            "vs_baseline": None, "dtype": cfg.dtype, "data": DATA,
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv,
                        "chunk": cfg.chunk, "l2": "flushed (256 MiB write) between timed steps",
                        "parallelism": f"dp{world}: independent sequences per GPU, no collective"},

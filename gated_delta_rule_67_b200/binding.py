@@ -29,6 +29,7 @@ SIGNATURES = {
     "kda_chunk_fwd_profiled": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp, _vp]),
     "kda_chunk_fwd_noalloc": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp]),
     "kda_chunk_fwd_check": (_i, [_vp, _sz, _vp]),
+    "kda_wait_selftest": (_i, [_vp, _sz, _vp]),
     "kda_recurrent_step": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 5 + [_vp]),
 }
 
@@ -178,6 +179,17 @@ def kda_chunk_fwd_check(workspace, stream=None) -> int:
         return KDA_OK
     return int(load().kda_chunk_fwd_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                           _stream(stream, workspace.device)))
+
+
+def kda_wait_selftest(workspace, stream=None) -> int:
+    """Runs the bounded-wait failure path on the device (see include/kda.h); returns the status
+    kda_chunk_fwd_check reads afterwards (KDA_ERR_TIMEOUT when the mechanism works)."""
+    lib = load()
+    nbytes = workspace.numel() * workspace.element_size()
+    st = lib.kda_wait_selftest(_ptr(workspace), nbytes, _stream(stream, workspace.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_wait_selftest")
+    return kda_chunk_fwd_check(workspace, stream)
 
 
 def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=None):

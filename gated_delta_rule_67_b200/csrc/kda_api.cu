@@ -155,6 +155,13 @@ kda_status kda_chunk_fwd_check(const void* workspace, size_t workspace_bytes, vo
   return h.error ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
+kda_status kda_wait_selftest(void* workspace, size_t workspace_bytes, void* stream_) {
+  if (!workspace || workspace_bytes < sizeof(kda::WorkspaceHeader) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return KDA_ERR_INVALID_ARG;
+  return from_cuda(kda::launch_wait_selftest(workspace, static_cast<cudaStream_t>(stream_)));
+}
+
 kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, float scale, float* state, void* o, int N, int H,
                               int dk, int dv, int dtype, void* stream_) {

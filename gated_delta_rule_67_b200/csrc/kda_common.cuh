@@ -40,6 +40,9 @@ cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, 
                                 int dk, int dv, int chunk, void* ws, size_t ws_bytes,
                                 cudaStream_t stream, void* const* events);
 
+// Launches a kernel whose only wait can never be satisfied (short limit).
+cudaError_t launch_wait_selftest(void* ws, cudaStream_t stream);
+
 // Records events[i] on the stream when an events array was given.
 inline cudaError_t mark(void* const* events, int i, cudaStream_t stream) {
   return events ? cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) : cudaSuccess;

@@ -815,6 +815,26 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   if (warp == 0) tmem_dealloc(tmem_base, 512);
 }
 
+// =============================================== bounded-wait self-test
+// Waits on an mbarrier that nothing ever completes, with a short limit, and
+// reports the give-up exactly as the prefill kernels do (error word in the
+// workspace header).  It lets a test exercise the failure path without
+// faulting or hanging the GPU.
+__global__ void kda_wait_selftest_kernel(WorkspaceHeader* hdr, uint32_t limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, limit)) {
+    atomicOr(&hdr->error, 1u);
+    atomicExch(&hdr->where, 99u);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_arrive(&bar);  // leave the barrier completed
+}
+
 // ================================================================== host
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -845,6 +865,14 @@ bool make_map(CUtensorMap* map, const void* base, int B, int T, int H, bool swiz
 }
 
 }  // namespace
+
+cudaError_t launch_wait_selftest(void* ws, cudaStream_t stream) {
+  WorkspaceHeader* hdr = static_cast<WorkspaceHeader*>(ws);
+  cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WorkspaceHeader), stream);
+  if (e != cudaSuccess) return e;
+  kda_wait_selftest_kernel<<<1, 32, 0, stream>>>(hdr, 1u << 12);
+  return cudaGetLastError();
+}
 
 size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk) {
   (void)dk, (void)dv, (void)chunk;

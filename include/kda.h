@@ -142,6 +142,16 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const voi
 KDA_API kda_status kda_chunk_fwd_check(const void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Failure-path self-test: enqueues a tiny kernel whose single mbarrier wait
+ * can never be satisfied; the wait gives up after a short bounded number of
+ * polls and records the give-up in the workspace header, exactly like a
+ * prefill kernel would.  A following kda_chunk_fwd_check on the same
+ * workspace then returns KDA_ERR_TIMEOUT.  `workspace` needs 256 bytes,
+ * 256-byte aligned.  Nothing faults and the GPU stays usable.
+ */
+KDA_API kda_status kda_wait_selftest(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Single-token decode (O(1) per token, constant-size state: same article,
  * section 4.2): one step of the recurrence for N sequences x H heads, with
  * the state updated in place.

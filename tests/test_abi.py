@@ -107,3 +107,9 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         binding.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+def test_wait_selftest_validation(lib):
+    assert lib.kda_wait_selftest(None, 256, None) == binding.KDA_ERR_INVALID_ARG
+    assert lib.kda_wait_selftest(A, 128, None) == binding.KDA_ERR_INVALID_ARG
+    assert lib.kda_wait_selftest(A + 16, 256, None) == binding.KDA_ERR_INVALID_ARG
