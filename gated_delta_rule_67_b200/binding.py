@@ -147,8 +147,9 @@ def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64,
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64, o=None,
                           final_state=None, output_final_state=True, stream=None):
     """kda_chunk_fwd using the library's static device scratch instead of a
-    workspace: for callers that cannot allocate device memory.  Fits
-    B*H*ceil(T/64) <= 903 chunk-heads (bf16); calls overlapping on the GPU race."""
+    workspace: for callers that cannot allocate device memory.  Fits problems
+    whose workspace is at most 64 MiB (about 900 chunk-heads, bf16); calls
+    overlapping on the GPU race."""
     lib = load()
     for name, x in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
         _check_dev(name, x, q.dtype)

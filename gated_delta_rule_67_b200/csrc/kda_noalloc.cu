@@ -11,9 +11,10 @@
 //
 // Facts a caller must know:
 //  * Size: kNoAllocScratchBytes (64 MiB) on every GPU that loads the library,
-//    held until the process exits.  It fits problems with
-//    B * H * ceil(T / 64) <= 903 (bf16, d = 128); bigger problems are
-//    rejected with KDA_ERR_UNSUPPORTED before anything is launched.
+//    held until the process exits.  Problems whose workspace
+//    (kda_chunk_fwd_workspace_size) is larger -- for bf16 at d = 128 about
+//    900 chunk-heads, B * H * ceil(T / 64) -- are rejected with
+//    KDA_ERR_UNSUPPORTED before anything is launched.
 //  * The array's host-side name is only a stand-in for the device symbol, so
 //    its device address is looked up once per device, with that device
 //    current, on the first call made on that device (cudaGetSymbolAddress).

@@ -43,6 +43,8 @@
 // one channel.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "kda_common.cuh"
 #include "sm100.cuh"
 
@@ -599,19 +601,76 @@ __global__ void __launch_bounds__(kP1Threads, 3)
 constexpr int kSPThreads = 288;
 constexpr uint32_t kTmP = 0, kTmO = 64, kTmS = 128, kTmAS = 256, kTmAV = 320;
 
+// What one state-pass CTA does.  Phase 0: a whole chain.  With the
+// chunk-parallel scan (few chains, long sequences) a chain is cut into G
+// groups of L chunks; phase 1 runs, per group, a zero-start pass whose final
+// state is R_g (group 0 starts from the true initial state instead) and an
+// identity-start pass with U = 0 whose final state is the group's transition
+// M_g (S_end = M_g S_start + R_g, the map is affine in S_start); phase 3 runs
+// every group again from its true start state S_g (computed in between by
+// kda_scan_combine_kernel) and writes the outputs.
+struct StatePassArgs {
+  const uint8_t* records;
+  WorkspaceHeader* hdr;
+  const float* s0;  // [B*H][128][128] or null (zero)
+  float* sT;        // [B*H][128][128] or null
+  float* rbuf;      // [B*H][G][128][128] scan buffers
+  float* mbuf;
+  const float* sbuf;
+  int T, H, NC, G, L, phase;
+};
+
 __global__ void __launch_bounds__(kSPThreads, 1)
-    kda_state_pass_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* __restrict__ records,
-                          WorkspaceHeader* hdr, const float* s0, float* sT, int T, int H, int NC) {
+    kda_state_pass_kernel(const __grid_constant__ CUtensorMap tm_o, const StatePassArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t bar_full[2], bar_o, bar_ofree, bar_p, bar_s, bar_as, bar_av;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int bh = blockIdx.x;
+  WorkspaceHeader* hdr = args.hdr;
+  const int T = args.T, H = args.H, NC = args.NC, G = args.G, L = args.L;
+  constexpr size_t kSt = (size_t)kD * kD;
+  // ---- role of this CTA
+  int bh, cb, ce;
+  const float* init = nullptr;  // null: zero start
+  bool ident = false, zero_u = false, out = true;
+  float* fin = nullptr;
+  if (args.phase == 0) {
+    bh = blockIdx.x;
+    cb = 0;
+    ce = NC;
+    init = args.s0 ? args.s0 + bh * kSt : nullptr;
+    fin = args.sT ? args.sT + bh * kSt : nullptr;
+  } else if (args.phase == 1) {
+    const int per = 2 * G - 3;
+    bh = blockIdx.x / per;
+    const int r = blockIdx.x % per;
+    out = false;
+    int g;
+    if (r < G - 1) {
+      g = r;
+      init = (g == 0 && args.s0) ? args.s0 + bh * kSt : nullptr;
+      fin = args.rbuf + ((size_t)bh * G + g) * kSt;
+    } else {
+      g = r - (G - 1) + 1;
+      ident = true;
+      zero_u = true;
+      fin = args.mbuf + ((size_t)bh * G + g) * kSt;
+    }
+    cb = g * L;
+    ce = min(NC, cb + L);
+  } else {
+    bh = blockIdx.x / G;
+    const int g = blockIdx.x % G;
+    cb = g * L;
+    ce = min(NC, cb + L);
+    init = args.sbuf + ((size_t)bh * G + g) * kSt;
+    fin = (g == G - 1 && args.sT) ? args.sT + bh * kSt : nullptr;
+  }
+  const int NCL = ce - cb;  // chunks this CTA walks
   const int h = bh % H, b = bh / H;
-  const uint8_t* recs = records + (size_t)bh * NC * kRecBytes;
-  const size_t sbase = (size_t)bh * kD * kD;
+  const uint8_t* recs = args.records + ((size_t)bh * NC + cb) * kRecBytes;
 
   if (tid == 0) {
     mbar_init(&bar_full[0], 1);
@@ -633,18 +692,22 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ mma
     if ((tid & 31) == 0) {
-      const uint32_t id_1 = idesc_bf16_f32(128, 128, 0, 0);  // [P|O] = S0^T [-W;Q+]^T
-      const uint32_t id_2 = idesc_bf16_f32(128, 192, 0, 1);  // [O|S] += V'^T [A_qk^T|Kbar]
+      // with outputs: [P|O] = S0^T [-W;Q+]^T (N=128) and [O|S] += V'^T [A_qk^T|Kbar] (N=192);
+      // without: P = S0^T (-W)^T (N=64) and S += V'^T Kbar (N=128)
+      const uint32_t id_1 = idesc_bf16_f32(128, out ? 128 : 64, 0, 0);
+      const uint32_t id_2 = idesc_bf16_f32(128, out ? 192 : 128, 0, 1);
+      const uint32_t d2_off = out ? 0 : (8192 >> 4);  // skip the A_qk^T block
+      const uint32_t t2 = out ? tm + kTmO : tm + kTmS;
       // first descriptors of each stage; later steps add address offsets (in 16-byte units)
       const uint64_t d1s0 = desc_sw128(smem_u32(sm + kRecWQ), 16, 1024);
       const uint64_t d1s1 = desc_sw128(smem_u32(sm + kStage + kRecWQ), 16, 1024);
-      const uint64_t d2s0 = desc_sw128(smem_u32(sm + kRecAqk), 8192, 1024);
-      const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStage + kRecAqk), 8192, 1024);
-      for (int n = 0; n < NC; ++n) {
+      const uint64_t d2s0 = desc_sw128(smem_u32(sm + kRecAqk), 8192, 1024) + d2_off;
+      const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStage + kRecAqk), 8192, 1024) + d2_off;
+      for (int n = 0; n < NCL; ++n) {
         const int s = n & 1;
         wait_or_flag(&bar_as, n & 1, hdr, 30);
         wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 31);
-        if (n >= 1) wait_or_flag(&bar_ofree, (n - 1) & 1, hdr, 32);  // O^T of chunk n-1 has been read
+        if (out && n >= 1) wait_or_flag(&bar_ofree, (n - 1) & 1, hdr, 32);  // O^T of chunk n-1 has been read
         tc_fence_after();
         const uint64_t d1 = s ? d1s1 : d1s0, d2 = s ? d2s1 : d2s0;
 #pragma unroll
@@ -656,7 +719,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kC / 16; ++k)  // MN-major B: +2 KiB per 16 K-rows
-          mma_bf16_ts(tm + kTmO, tm + kTmAV + k * 8, d2 + (uint64_t)((2 * k * 1024) >> 4), id_2, 1);
+          mma_bf16_ts(t2, tm + kTmAV + k * 8, d2 + (uint64_t)((2 * k * 1024) >> 4), id_2, 1);
         mma_commit(&bar_s);
         mma_commit(&bar_o);
       }
@@ -666,15 +729,22 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     const int j = tid - 128;
     const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
     if (tid == 128) {
-      for (int n = 0; n < 2 && n < NC; ++n) {
+      for (int n = 0; n < 2 && n < NCL; ++n) {
         mbar_expect_tx(&bar_full[n], kRecBytes);
         bulk_load(sm + n * kStage, recs + (size_t)n * kRecBytes, kRecBytes, &bar_full[n]);
       }
     }
-    for (int n = 0; n < NC; ++n) {
+    for (int n = 0; n < NCL; ++n) {
       const int s = n & 1;
       wait_or_flag(&bar_o, n & 1, hdr, 21);
       tc_fence_after();
+      if (!out) {
+        if (tid == 128 && n + 2 < NCL) {
+          mbar_expect_tx(&bar_full[s], kRecBytes);
+          bulk_load(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, kRecBytes, &bar_full[s]);
+        }
+        continue;
+      }
       uint32_t r[64];
       tmem_ld32_raw(tm + kTmO + lane_off, r);
       tmem_ld32_raw(tm + kTmO + lane_off + 32, r + 32);
@@ -682,7 +752,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       reg_pin<64>(r);
       tc_fence_before();
       mbar_arrive(&bar_ofree);
-      if (tid == 128 && n + 2 < NC) {  // every reader of stage s is done with chunk n
+      if (tid == 128 && n + 2 < NCL) {  // every reader of stage s is done with chunk n
         mbar_expect_tx(&bar_full[s], kRecBytes);
         bulk_load(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, kRecBytes, &bar_full[s]);
       }
@@ -697,8 +767,8 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       named_bar_sync(2, 128);
       if (tid == 128) {
         const uint8_t* src = sm + kP2Out + (n & 1) * 16384;
-        tma_store_4d(&tm_o, src, 0, h, n * kC, b);
-        tma_store_4d(&tm_o, src + 8192, 64, h, n * kC, b);
+        tma_store_4d(&tm_o, src, 0, h, (cb + n) * kC, b);
+        tma_store_4d(&tm_o, src + 8192, 64, h, (cb + n) * kC, b);
         bulk_commit();
       }
     }
@@ -710,14 +780,17 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     {
       float v[32];
 #pragma unroll
-      for (int cb = 0; cb < kD / 32; ++cb) {
+      for (int q = 0; q < kD / 32; ++q) {
 #pragma unroll
-        for (int ii = 0; ii < 32; ++ii) v[ii] = s0 ? s0[sbase + (size_t)(cb * 32 + ii) * kD + j] : 0.f;
-        tmem_st32(tm + kTmS + lane_off + cb * 32, v);
+        for (int ii = 0; ii < 32; ++ii) {
+          const int c = q * 32 + ii;
+          v[ii] = init ? init[(size_t)c * kD + j] : (ident && c == j ? 1.f : 0.f);
+        }
+        tmem_st32(tm + kTmS + lane_off + q * 32, v);
       }
       tmem_wait_st();
     }
-    for (int n = 0; n < NC; ++n) {
+    for (int n = 0; n < NCL; ++n) {
       const int s = n & 1;
       const uint8_t* stage = sm + s * kStage;
       if (n > 0) wait_or_flag(&bar_s, (n - 1) & 1, hdr, 22);
@@ -782,7 +855,8 @@ __global__ void __launch_bounds__(kSPThreads, 1)
           const uint32_t uw[4] = {urow[k8].x, urow[k8].y, urow[k8].z, urow[k8].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 u2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[e]));
+            float2 u2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[e]));
+            if (zero_u) u2 = make_float2(0.f, 0.f);
             pk[k8 * 4 + e] = pack2(u2.x + __uint_as_float(pr[k8 * 8 + 2 * e]),
                                    u2.y + __uint_as_float(pr[k8 * 8 + 2 * e + 1]));
           }
@@ -798,21 +872,82 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar_av);
     }
-    wait_or_flag(&bar_s, (NC - 1) & 1, hdr, 27);
+    wait_or_flag(&bar_s, (NCL - 1) & 1, hdr, 27);
     tc_fence_after();
-    if (sT) {
+    if (fin) {
 #pragma unroll
-      for (int cb = 0; cb < kD / 32; ++cb) {
+      for (int q = 0; q < kD / 32; ++q) {
         float v[32];
-        tmem_ld32(tm + kTmS + lane_off + cb * 32, v);
+        tmem_ld32(tm + kTmS + lane_off + q * 32, v);
 #pragma unroll
-        for (int ii = 0; ii < 32; ++ii) sT[sbase + (size_t)(cb * 32 + ii) * kD + j] = v[ii];
+        for (int ii = 0; ii < 32; ++ii) fin[(size_t)(q * 32 + ii) * kD + j] = v[ii];
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem_base, 512);
+}
+
+// ======================================================== scan combine
+// S_{g+1} = M_g S_g + R_g for g = 1 .. G-2 (S_0 = initial state, S_1 = R_0),
+// in fp32 on the CUDA cores.  The columns of S never mix, so each CTA owns 16
+// columns of one chain and walks the groups on its own.
+constexpr int kScanCols = 16;
+constexpr int kScanLd = 132;  // padded row stride of M in shared memory
+__global__ void __launch_bounds__(256) kda_scan_combine_kernel(const float* s0, float* sbuf, const float* rbuf,
+                                                               const float* mbuf, int G) {
+  extern __shared__ __align__(16) float scm[];
+  float* Ms = scm;                    // [128][kScanLd]
+  float* Sc = scm + kD * kScanLd;     // [128][kScanCols]
+  constexpr size_t kSt = (size_t)kD * kD;
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.x / (kD / kScanCols);
+  const int c0 = (blockIdx.x % (kD / kScanCols)) * kScanCols;
+  const int r = tid >> 1, cc = c0 + (tid & 1) * 8;  // this thread: row r, columns cc..cc+7
+  float* sb = sbuf + (size_t)bh * G * kSt;
+  const float* rb = rbuf + (size_t)bh * G * kSt;
+  const float* mb = mbuf + (size_t)bh * G * kSt;
+  // S_0 and S_1
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const size_t idx = (size_t)r * kD + cc + e;
+    sb[idx] = s0 ? s0[(size_t)bh * kSt + idx] : 0.f;
+    const float s1 = rb[idx];
+    sb[kSt + idx] = s1;
+    Sc[r * kScanCols + (tid & 1) * 8 + e] = s1;
+  }
+  for (int g = 1; g + 1 < G; ++g) {
+    const float4* mg4 = reinterpret_cast<const float4*>(mb + g * kSt);
+    for (int e = tid; e < kD * kD / 4; e += 256) {
+      const int rr = e / (kD / 4), q = e % (kD / 4);
+      *reinterpret_cast<float4*>(Ms + rr * kScanLd + q * 4) = mg4[e];
+    }
+    __syncthreads();
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = rb[g * kSt + (size_t)r * kD + cc + e];
+#pragma unroll 4
+    for (int k = 0; k < kD; ++k) {
+      const float m = Ms[r * kScanLd + k];
+      const float4 x0 = *reinterpret_cast<const float4*>(Sc + k * kScanCols + (tid & 1) * 8);
+      const float4 x1 = *reinterpret_cast<const float4*>(Sc + k * kScanCols + (tid & 1) * 8 + 4);
+      acc[0] = fmaf(m, x0.x, acc[0]);
+      acc[1] = fmaf(m, x0.y, acc[1]);
+      acc[2] = fmaf(m, x0.z, acc[2]);
+      acc[3] = fmaf(m, x0.w, acc[3]);
+      acc[4] = fmaf(m, x1.x, acc[4]);
+      acc[5] = fmaf(m, x1.y, acc[5]);
+      acc[6] = fmaf(m, x1.z, acc[6]);
+      acc[7] = fmaf(m, x1.w, acc[7]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      Sc[r * kScanCols + (tid & 1) * 8 + e] = acc[e];
+      sb[(g + 1) * kSt + (size_t)r * kD + cc + e] = acc[e];
+    }
+  }
 }
 
 // =============================================== bounded-wait self-test
@@ -874,10 +1009,34 @@ cudaError_t launch_wait_selftest(void* ws, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Groups of the chunk-parallel scan for B*H chains of NC chunks (1 = no scan).
+// Phase 1 runs 2G-3 CTAs per chain, sized to one wave of a 148-SM part; the
+// count is a fixed function of the shape so results do not depend on the GPU.
+constexpr int kScanSMs = 148;
+constexpr int kScanMinChunks = 4;
+void scan_groups(int BH, int NC, int* G_out, int* L_out) {
+  int G = 1;
+  if (BH > 0 && 3 * BH <= kScanSMs) G = std::min((kScanSMs / BH + 3) / 2, NC / kScanMinChunks);
+  if (G >= 3) {
+    const int L = (NC + G - 1) / G;
+    G = (NC + L - 1) / L;
+    if (G >= 3) {
+      *G_out = G;
+      *L_out = L;
+      return;
+    }
+  }
+  *G_out = 1;
+  *L_out = NC;
+}
+
 size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk) {
   (void)dk, (void)dv, (void)chunk;
-  const size_t nc = ((size_t)T + kC - 1) / kC;
-  return sizeof(WorkspaceHeader) + (size_t)B * H * nc * kRecBytes;
+  const int NC = (int)(((size_t)T + kC - 1) / kC);
+  int G, L;
+  scan_groups(B * H, NC, &G, &L);
+  const size_t scan = G > 1 ? 3 * (size_t)B * H * G * kD * kD * sizeof(float) : 0;
+  return sizeof(WorkspaceHeader) + (size_t)B * H * NC * kRecBytes + scan;
 }
 
 cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const bf16* beta,
@@ -891,6 +1050,9 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
                                          kP1Bytes + 1024);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kP2Bytes + 1024);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kda_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (kD * kScanLd + kD * kScanCols) * sizeof(float));
     if (e != cudaSuccess) return e;
     attrs_set = true;
   }
@@ -910,8 +1072,32 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e != cudaSuccess) return e;
-  kda_state_pass_kernel<<<(unsigned)(B * H), kSPThreads, kP2Bytes + 1024, stream>>>(mo, records, hdr, s0, sT, T, H,
-                                                                                     NC);
+  StatePassArgs a{records, hdr, s0, sT, nullptr, nullptr, nullptr, T, H, NC, 1, NC, 0};
+  const int BH = B * H;
+  int G, L;
+  scan_groups(BH, NC, &G, &L);
+  if (G == 1) {
+    kda_state_pass_kernel<<<(unsigned)BH, kSPThreads, kP2Bytes + 1024, stream>>>(mo, a);
+  } else {
+    float* scan = reinterpret_cast<float*>(records + (size_t)BH * NC * kRecBytes);
+    const size_t per = (size_t)BH * G * kD * kD;
+    a.rbuf = scan;
+    a.mbuf = scan + per;
+    a.sbuf = scan + 2 * per;
+    a.G = G;
+    a.L = L;
+    a.phase = 1;
+    kda_state_pass_kernel<<<(unsigned)(BH * (2 * G - 3)), kSPThreads, kP2Bytes + 1024, stream>>>(mo, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    kda_scan_combine_kernel<<<(unsigned)(BH * (kD / kScanCols)), 256,
+                              (kD * kScanLd + kD * kScanCols) * sizeof(float), stream>>>(s0, scan + 2 * per, scan,
+                                                                                           scan + per, G);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    a.phase = 3;
+    kda_state_pass_kernel<<<(unsigned)(BH * G), kSPThreads, kP2Bytes + 1024, stream>>>(mo, a);
+  }
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 2, stream);
   return e;

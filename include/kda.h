@@ -120,9 +120,10 @@ KDA_API kda_status kda_chunk_fwd_profiled(const void* q, const void* k, const vo
  *
  * Same arguments and results as kda_chunk_fwd minus the workspace.  The
  * scratch is a 64 MiB statically sized device array inside the library
- * (present on every GPU that loads it, until the process exits), which fits
- * B * H * ceil(T / 64) <= 903 for the bf16 path; larger problems return
- * KDA_ERR_UNSUPPORTED before anything is launched.  The first call on a
+ * (present on every GPU that loads it, until the process exits); problems
+ * whose kda_chunk_fwd_workspace_size exceeds it (for the bf16 path about 900
+ * chunk-heads, B * H * ceil(T / 64)) return KDA_ERR_UNSUPPORTED before
+ * anything is launched.  The first call on a
  * device looks up the array's device address (with that device current), so
  * make it before any stream capture.  All calls share the array: calls whose
  * work overlaps on the GPU race on it and must be serialised by the caller.

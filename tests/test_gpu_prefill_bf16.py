@@ -163,3 +163,34 @@ def test_gate_span_just_inside_fast_path():
     ref_o, ref_s = _oracle(x)
     assert rel_err(o, ref_o) < TOLB
     assert rel_err(sT, ref_s) < TOLB
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 64 * 13 + 5, 2), (1, 64 * 40, 1), (2, 64 * 24 + 63, 3)])
+def test_chunk_parallel_scan_shapes(B, T, H):
+    """Few chains over many chunks take the chunk-parallel scan (groups of
+    chunks, per-group transition and offset, fp32 combination, outputs per
+    group); a ragged tail and a random initial state, against the oracle."""
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(B, T, H, 128, 128, torch.bfloat16, 0.1, seed=50 + T, device="cpu")
+    o, sT = _run(x, dev)
+    ref_o, ref_s = _oracle(x)
+    assert rel_err(o, ref_o) < TOLB
+    assert rel_err(sT, ref_s) < TOLB
+
+
+def test_scan_with_extreme_gates_and_in_place_state():
+    """The scan path with exact-path chunks inside its groups, zero gate (no
+    decay) channels, and the final state written over the initial state."""
+    dev = cuda_or_skip()
+    B, T, H = 1, 64 * 30, 2
+    x = make_prefill_inputs(B, T, H, 128, 128, torch.bfloat16, 0.1, seed=77, device="cpu")
+    g = x["g"].float()
+    g[:, 600:700, 0, :8] = -20.0
+    g[:, :, 1, 100:] = 0.0
+    x["g"] = g.to(torch.bfloat16)
+    ref_o, ref_s = _oracle(x)
+    state = x["initial_state"].to(dev)
+    o, _ = kda_chunk_fwd(*(x[n].to(dev) for n in NAMES), None, state, final_state=state)
+    torch.cuda.synchronize()
+    assert rel_err(o, ref_o) < TOLB
+    assert rel_err(state, ref_s) < TOLB

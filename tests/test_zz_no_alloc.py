@@ -33,7 +33,8 @@ def test_noalloc_matches_workspace_entry_point_twice():
 def test_noalloc_refuses_problems_beyond_the_scratch():
     dev = cuda_or_skip()
     lib = binding.load()
-    # 1 x 16 heads x ceil(4096/64)=64 chunks = 1024 chunk-heads > 903: refused before any launch.
+    # 1 x 16 heads x ceil(4096/64)=64 chunks = 1024 chunk-heads: its workspace exceeds the 64 MiB
+    # scratch, so the call is refused before any launch.
     x = make_prefill_inputs(1, 4096, 16, 128, 128, torch.bfloat16, 0.1, seed=63, device=dev)
     with pytest.raises(binding.KDAError) as e:
         binding.kda_chunk_fwd_noalloc(*(x[n] for n in NAMES), None, x["initial_state"])
