@@ -594,12 +594,39 @@ __global__ void __launch_bounds__(kP1Threads, 3)
 // Tensor memory (fp32 unless noted):
 //   [P | O^T | S^T] at [0,64) [64,128) [128,256)
 //   S0^T as bf16 A operand [256,320), V'^T as bf16 A operand [320,352)
-// Two MMA chains per chunk, both A operands read from tensor memory:
-//   [P | O^T]   = S0^T [-W ; Q+]^T          (N = 128, K = 128: 8 instructions)
+// Three MMA groups per chunk, all A operands read from tensor memory:
+//   P           = S0^T (-W)^T               (N = 64,  K = 128: 8 instructions, committed alone)
+//   O^T         = S0^T Q+^T                 (N = 64,  K = 128: 8 instructions, while V' is formed)
 //   [O^T | S^T] += V'^T [A_qk^T | Kbar]      (N = 192, K = 64:  4 instructions)
-// with P = -(W S0)^T and V'^T = U^T + P formed in between on the CUDA cores.
+// with P = -(W S0)^T and V'^T = U^T + P formed on the CUDA cores.  Only P
+// and the last group are on the chain's critical path; the O^T group waits
+// for the output warps to release the previous chunk's O^T off that path.
 constexpr int kSPThreads = 288;
 constexpr uint32_t kTmP = 0, kTmO = 64, kTmS = 128, kTmAS = 256, kTmAV = 320;
+
+// Brings the record of one chunk into a stage.  A pass that writes outputs
+// needs all of it; a pass without outputs reads only -W (the first 64 rows
+// of each 64-column block of [-W; Q+]), Kbar, U and gamma; the transition
+// pass (U = 0) not even U.
+constexpr uint32_t kRecNoOutBytes = 2 * 8192 + (kRecBytes - kRecKbar);
+constexpr uint32_t kRecTransBytes = 2 * 8192 + (kRecU - kRecKbar) + (kRecBytes - kRecGamma);
+__device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, uint64_t* bar, bool out,
+                                            bool zero_u) {
+  if (out) {
+    mbar_expect_tx(bar, kRecBytes);
+    bulk_load(stage, rec, kRecBytes, bar);
+    return;
+  }
+  mbar_expect_tx(bar, zero_u ? kRecTransBytes : kRecNoOutBytes);
+  bulk_load(stage + kRecWQ, rec + kRecWQ, 8192, bar);
+  bulk_load(stage + kRecWQ + 16384, rec + kRecWQ + 16384, 8192, bar);
+  if (zero_u) {
+    bulk_load(stage + kRecKbar, rec + kRecKbar, kRecU - kRecKbar, bar);
+    bulk_load(stage + kRecGamma, rec + kRecGamma, kRecBytes - kRecGamma, bar);
+  } else {
+    bulk_load(stage + kRecKbar, rec + kRecKbar, kRecBytes - kRecKbar, bar);
+  }
+}
 
 // What one state-pass CTA does.  Phase 0: a whole chain.  With the
 // chunk-parallel scan (few chains, long sequences) a chain is cut into G
@@ -615,7 +642,7 @@ struct StatePassArgs {
   const float* s0;  // [B*H][128][128] or null (zero)
   float* sT;        // [B*H][128][128] or null
   float* rbuf;      // [B*H][G][128][128] scan buffers
-  float* mbuf;
+  float* mbuf;      // transition matrices, transposed: [B*H][G][k][r] = M_g[r][k]
   const float* sbuf;
   int T, H, NC, G, L, phase;
 };
@@ -624,7 +651,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     kda_state_pass_kernel(const __grid_constant__ CUtensorMap tm_o, const StatePassArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  __shared__ uint64_t bar_full[2], bar_o, bar_ofree, bar_p, bar_s, bar_as, bar_av;
+  __shared__ uint64_t bar_full[2], bar_o, bar_p, bar_s, bar_as, bar_av, bar_init;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -676,12 +703,18 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     mbar_init(&bar_full[0], 1);
     mbar_init(&bar_full[1], 1);
     mbar_init(&bar_o, 1);
-    mbar_init(&bar_ofree, 128);
     mbar_init(&bar_p, 1);
     mbar_init(&bar_s, 1);
-    mbar_init(&bar_as, 128);
+    mbar_init(&bar_as, out ? 256 : 128);  // with outputs the output warps release O^T through it too
     mbar_init(&bar_av, 128);
+    mbar_init(&bar_init, 1);
     fence_mbar_init();
+    if (init) {  // the start state, row-major fp32, into stage 1 (its record follows once it is read)
+      mbar_expect_tx(&bar_init, kD * kD * sizeof(float));
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        bulk_load(sm + kStage + p * 16384, init + p * 4096, 16384, &bar_init);
+    }
   }
   if (warp == 0) tmem_alloc(&tmem_base, 512);
   tc_fence_before();
@@ -692,9 +725,11 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ mma
     if ((tid & 31) == 0) {
-      // with outputs: [P|O] = S0^T [-W;Q+]^T (N=128) and [O|S] += V'^T [A_qk^T|Kbar] (N=192);
-      // without: P = S0^T (-W)^T (N=64) and S += V'^T Kbar (N=128)
-      const uint32_t id_1 = idesc_bf16_f32(128, out ? 128 : 64, 0, 0);
+      // P = S0^T (-W)^T (N=64) first, committed alone so that V' can be formed
+      // at once; with outputs, O^T = S0^T Q+^T (N=64) is issued next, while
+      // the state warps form V', and [O|S] += V'^T [A_qk^T|Kbar] (N=192)
+      // closes the chunk; without outputs S += V'^T Kbar (N=128).
+      const uint32_t id_1 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id_2 = idesc_bf16_f32(128, out ? 192 : 128, 0, 1);
       const uint32_t d2_off = out ? 0 : (8192 >> 4);  // skip the A_qk^T block
       const uint32_t t2 = out ? tm + kTmO : tm + kTmS;
@@ -703,11 +738,11 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       const uint64_t d1s1 = desc_sw128(smem_u32(sm + kStage + kRecWQ), 16, 1024);
       const uint64_t d2s0 = desc_sw128(smem_u32(sm + kRecAqk), 8192, 1024) + d2_off;
       const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStage + kRecAqk), 8192, 1024) + d2_off;
+      constexpr uint64_t kQoff = 8192 >> 4;  // rows 64-127 (Q+) of each 64-column block of [-W; Q+]
       for (int n = 0; n < NCL; ++n) {
         const int s = n & 1;
         wait_or_flag(&bar_as, n & 1, hdr, 30);
         wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 31);
-        if (out && n >= 1) wait_or_flag(&bar_ofree, (n - 1) & 1, hdr, 32);  // O^T of chunk n-1 has been read
         tc_fence_after();
         const uint64_t d1 = s ? d1s1 : d1s0, d2 = s ? d2s1 : d2s0;
 #pragma unroll
@@ -715,6 +750,12 @@ __global__ void __launch_bounds__(kSPThreads, 1)
           mma_bf16_ts(tm + kTmP, tm + kTmAS + k * 8, d1 + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), id_1,
                       k > 0);
         mma_commit(&bar_p);
+        if (out) {  // bar_as also covered the read of O^T of chunk n-1
+#pragma unroll
+          for (int k = 0; k < kD / 16; ++k)
+            mma_bf16_ts(tm + kTmO, tm + kTmAS + k * 8,
+                        d1 + kQoff + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), id_1, k > 0);
+        }
         wait_or_flag(&bar_av, n & 1, hdr, 33);
         tc_fence_after();
 #pragma unroll
@@ -729,20 +770,20 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     const int j = tid - 128;
     const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
     if (tid == 128) {
-      for (int n = 0; n < 2 && n < NCL; ++n) {
-        mbar_expect_tx(&bar_full[n], kRecBytes);
-        bulk_load(sm + n * kStage, recs + (size_t)n * kRecBytes, kRecBytes, &bar_full[n]);
-      }
+      for (int n = 0; n < 2 && n < NCL; ++n)
+        if (n == 0 || !init) load_record(sm + n * kStage, recs + (size_t)n * kRecBytes, &bar_full[n], out, zero_u);
     }
+    // With outputs, each chunk's bar_as phase also waits for these 128
+    // threads: the first has nothing to release, later ones the O^T of the
+    // chunk before (whose O^T group overwrites it).
+    if (out) mbar_arrive(&bar_as);
     for (int n = 0; n < NCL; ++n) {
       const int s = n & 1;
       wait_or_flag(&bar_o, n & 1, hdr, 21);
       tc_fence_after();
       if (!out) {
-        if (tid == 128 && n + 2 < NCL) {
-          mbar_expect_tx(&bar_full[s], kRecBytes);
-          bulk_load(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, kRecBytes, &bar_full[s]);
-        }
+        if (tid == 128 && n + 2 < NCL)
+          load_record(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, &bar_full[s], false, zero_u);
         continue;
       }
       uint32_t r[64];
@@ -751,7 +792,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       tmem_wait_ld();
       reg_pin<64>(r);
       tc_fence_before();
-      mbar_arrive(&bar_ofree);
+      if (n + 1 < NCL) mbar_arrive(&bar_as);
       if (tid == 128 && n + 2 < NCL) {  // every reader of stage s is done with chunk n
         mbar_expect_tx(&bar_full[s], kRecBytes);
         bulk_load(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, kRecBytes, &bar_full[s]);
@@ -778,17 +819,24 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     const int j = tid;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     {
+      // column j of the start state (row j of S^T) into lane j
+      const float* s0s = reinterpret_cast<const float*>(sm + kStage);
+      if (init) wait_or_flag(&bar_init, 0, hdr, 20);
       float v[32];
 #pragma unroll
       for (int q = 0; q < kD / 32; ++q) {
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii) {
           const int c = q * 32 + ii;
-          v[ii] = init ? init[(size_t)c * kD + j] : (ident && c == j ? 1.f : 0.f);
+          v[ii] = init ? s0s[c * kD + j] : (ident && c == j ? 1.f : 0.f);
         }
         tmem_st32(tm + kTmS + lane_off + q * 32, v);
       }
       tmem_wait_st();
+      if (init) {  // stage 1 is free again: bring the record of chunk 1
+        named_bar_sync(1, 128);
+        if (tid == 0 && NCL > 1) load_record(sm + kStage, recs + kRecBytes, &bar_full[1], out, zero_u);
+      }
     }
     for (int n = 0; n < NCL; ++n) {
       const int s = n & 1;
@@ -879,8 +927,17 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       for (int q = 0; q < kD / 32; ++q) {
         float v[32];
         tmem_ld32(tm + kTmS + lane_off + q * 32, v);
+        if (ident) {
+          // A transition matrix is stored transposed (row j of M^T = column j
+          // of M), the layout the combination kernel streams.
+          float4* dst = reinterpret_cast<float4*>(fin + (size_t)j * kD + q * 32);
 #pragma unroll
-        for (int ii = 0; ii < 32; ++ii) fin[(size_t)(q * 32 + ii) * kD + j] = v[ii];
+          for (int i4 = 0; i4 < 8; ++i4)
+            dst[i4] = make_float4(v[4 * i4], v[4 * i4 + 1], v[4 * i4 + 2], v[4 * i4 + 3]);
+        } else {
+#pragma unroll
+          for (int ii = 0; ii < 32; ++ii) fin[(size_t)(q * 32 + ii) * kD + j] = v[ii];
+        }
       }
     }
   }
@@ -892,61 +949,119 @@ __global__ void __launch_bounds__(kSPThreads, 1)
 // ======================================================== scan combine
 // S_{g+1} = M_g S_g + R_g for g = 1 .. G-2 (S_0 = initial state, S_1 = R_0),
 // in fp32 on the CUDA cores.  The columns of S never mix, so each CTA owns 16
-// columns of one chain and walks the groups on its own.
+// columns of one chain and walks the groups on its own.  Every M_g and R_g is
+// ready when the kernel starts, so the transposed transition matrices stream
+// through a ring of shared-memory stages by bulk copies while earlier steps
+// compute.  Thread (warp w, lane l) owns rows l + 32 i (i < 4), columns
+// 4 (w % 4) .. +3 of the CTA's block and half w / 4 of the k range: per k one
+// broadcast float4 of S_g and four conflict-free scalars of M_g^T feed 16
+// FMAs; the upper half's partial sums are added through shared memory.
 constexpr int kScanCols = 16;
-constexpr int kScanLd = 132;  // padded row stride of M in shared memory
-__global__ void __launch_bounds__(256) kda_scan_combine_kernel(const float* s0, float* sbuf, const float* rbuf,
-                                                               const float* mbuf, int G) {
+constexpr int kScanStages = 3;
+constexpr int kScanThreads = 256;
+constexpr int kScanLd = 20;  // padded row stride of the S_g blocks (conflict-free float4 stores)
+constexpr uint32_t kScanStageBytes = kD * kD * sizeof(float);
+constexpr size_t kScanSmem = kScanStages * (size_t)kScanStageBytes + 3 * (size_t)kD * kScanLd * sizeof(float);
+
+__global__ void __launch_bounds__(kScanThreads) kda_scan_combine_kernel(const float* s0, float* sbuf, const float* rbuf,
+                                                                        const float* mbuf_t, int G,
+                                                                        WorkspaceHeader* hdr) {
   extern __shared__ __align__(16) float scm[];
-  float* Ms = scm;                    // [128][kScanLd]
-  float* Sc = scm + kD * kScanLd;     // [128][kScanCols]
+  __shared__ uint64_t full[kScanStages];
   constexpr size_t kSt = (size_t)kD * kD;
-  const int tid = threadIdx.x;
+  float* Mt = scm;                              // [stage][k][r] = M_g[r][k]
+  float* Sc = scm + kScanStages * kSt;          // [2][128][kScanLd] S_g blocks
+  float* Pu = Sc + 2 * kD * kScanLd;            // [128][kScanLd] upper-half partial sums
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cw = 4 * (warp & 3), kh = warp >> 2;
   const int bh = blockIdx.x / (kD / kScanCols);
-  const int c0 = (blockIdx.x % (kD / kScanCols)) * kScanCols;
-  const int r = tid >> 1, cc = c0 + (tid & 1) * 8;  // this thread: row r, columns cc..cc+7
+  const int c0 = (blockIdx.x % (kD / kScanCols)) * kScanCols + cw;  // this thread's first global column
   float* sb = sbuf + (size_t)bh * G * kSt;
   const float* rb = rbuf + (size_t)bh * G * kSt;
-  const float* mb = mbuf + (size_t)bh * G * kSt;
-  // S_0 and S_1
+  const float* mb = mbuf_t + (size_t)bh * G * kSt;
+  const int nsteps = G - 2;
+  auto issue = [&](int stage, int g) {
+    mbar_expect_tx(&full[stage], kScanStageBytes);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const size_t idx = (size_t)r * kD + cc + e;
-    sb[idx] = s0 ? s0[(size_t)bh * kSt + idx] : 0.f;
-    const float s1 = rb[idx];
-    sb[kSt + idx] = s1;
-    Sc[r * kScanCols + (tid & 1) * 8 + e] = s1;
+    for (int p = 0; p < 4; ++p)
+      bulk_load(Mt + stage * kSt + p * (kSt / 4), mb + g * kSt + p * (kSt / 4), kScanStageBytes / 4, &full[stage]);
+  };
+  if (tid == 0) {
+    for (int s = 0; s < kScanStages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+    for (int s = 0; s < kScanStages && s < nsteps; ++s) issue(s, 1 + s);
   }
-  for (int g = 1; g + 1 < G; ++g) {
-    const float4* mg4 = reinterpret_cast<const float4*>(mb + g * kSt);
-    for (int e = tid; e < kD * kD / 4; e += 256) {
-      const int rr = e / (kD / 4), q = e % (kD / 4);
-      *reinterpret_cast<float4*>(Ms + rr * kScanLd + q * 4) = mg4[e];
-    }
-    __syncthreads();
-    float acc[8];
+  // S_0 (lower half of the threads) and S_1 = R_0 (upper half)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = rb[g * kSt + (size_t)r * kD + cc + e];
-#pragma unroll 4
-    for (int k = 0; k < kD; ++k) {
-      const float m = Ms[r * kScanLd + k];
-      const float4 x0 = *reinterpret_cast<const float4*>(Sc + k * kScanCols + (tid & 1) * 8);
-      const float4 x1 = *reinterpret_cast<const float4*>(Sc + k * kScanCols + (tid & 1) * 8 + 4);
-      acc[0] = fmaf(m, x0.x, acc[0]);
-      acc[1] = fmaf(m, x0.y, acc[1]);
-      acc[2] = fmaf(m, x0.z, acc[2]);
-      acc[3] = fmaf(m, x0.w, acc[3]);
-      acc[4] = fmaf(m, x1.x, acc[4]);
-      acc[5] = fmaf(m, x1.y, acc[5]);
-      acc[6] = fmaf(m, x1.z, acc[6]);
-      acc[7] = fmaf(m, x1.w, acc[7]);
+  for (int i = 0; i < 4; ++i) {
+    const int r = lane + 32 * i;
+    const size_t idx = (size_t)r * kD + c0;
+    if (kh == 0) {
+      const float4 a =
+          s0 ? *reinterpret_cast<const float4*>(s0 + (size_t)bh * kSt + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(sb + idx) = a;
+    } else {
+      const float4 s1 = *reinterpret_cast<const float4*>(rb + idx);
+      *reinterpret_cast<float4*>(sb + kSt + idx) = s1;
+      *reinterpret_cast<float4*>(Sc + r * kScanLd + cw) = s1;
     }
-    __syncthreads();
+  }
+  float4 rn[4];
+  if (kh == 0 && nsteps > 0) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      Sc[r * kScanCols + (tid & 1) * 8 + e] = acc[e];
-      sb[(g + 1) * kSt + (size_t)r * kD + cc + e] = acc[e];
+    for (int i = 0; i < 4; ++i) rn[i] = *reinterpret_cast<const float4*>(rb + kSt + (size_t)(lane + 32 * i) * kD + c0);
+  }
+  __syncthreads();
+  for (int step = 0; step < nsteps; ++step) {
+    const int g = step + 1, s = step % kScanStages;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[i][0] = kh ? 0.f : rn[i].x;
+      acc[i][1] = kh ? 0.f : rn[i].y;
+      acc[i][2] = kh ? 0.f : rn[i].z;
+      acc[i][3] = kh ? 0.f : rn[i].w;
     }
+    if (kh == 0 && step + 1 < nsteps) {  // R of the next step, in flight during this one
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        rn[i] = *reinterpret_cast<const float4*>(rb + (size_t)(g + 1) * kSt + (size_t)(lane + 32 * i) * kD + c0);
+    }
+    wait_or_flag(&full[s], (step / kScanStages) & 1, hdr, 40);
+    const float* M = Mt + s * kSt + kh * (kD / 2) * kD;
+    const float* X = Sc + (step & 1) * kD * kScanLd + kh * (kD / 2) * kScanLd;
+#pragma unroll 8
+    for (int k = 0; k < kD / 2; ++k) {
+      const float4 x = *reinterpret_cast<const float4*>(X + k * kScanLd + cw);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float m = M[k * kD + lane + 32 * i];
+        acc[i][0] = fmaf(m, x.x, acc[i][0]);
+        acc[i][1] = fmaf(m, x.y, acc[i][1]);
+        acc[i][2] = fmaf(m, x.z, acc[i][2]);
+        acc[i][3] = fmaf(m, x.w, acc[i][3]);
+      }
+    }
+    if (kh) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4*>(Pu + (lane + 32 * i) * kScanLd + cw) =
+            make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    }
+    __syncthreads();  // partial sums visible; stage s no longer read
+    if (tid == 0 && step + kScanStages < nsteps) issue(s, g + kScanStages);
+    if (kh == 0) {
+      float* Xn = Sc + ((step + 1) & 1) * kD * kScanLd;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane + 32 * i;
+        const float4 p = *reinterpret_cast<const float4*>(Pu + r * kScanLd + cw);
+        const float4 o = make_float4(acc[i][0] + p.x, acc[i][1] + p.y, acc[i][2] + p.z, acc[i][3] + p.w);
+        *reinterpret_cast<float4*>(Xn + r * kScanLd + cw) = o;
+        *reinterpret_cast<float4*>(sb + (size_t)(g + 1) * kSt + (size_t)r * kD + c0) = o;
+      }
+    }
+    __syncthreads();  // S_{g+1} block complete; partial-sum buffer free
   }
 }
 
@@ -1051,8 +1166,7 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kP2Bytes + 1024);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (kD * kScanLd + kD * kScanCols) * sizeof(float));
+    e = cudaFuncSetAttribute(kda_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
     if (e != cudaSuccess) return e;
     attrs_set = true;
   }
@@ -1090,9 +1204,8 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     kda_state_pass_kernel<<<(unsigned)(BH * (2 * G - 3)), kSPThreads, kP2Bytes + 1024, stream>>>(mo, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    kda_scan_combine_kernel<<<(unsigned)(BH * (kD / kScanCols)), 256,
-                              (kD * kScanLd + kD * kScanCols) * sizeof(float), stream>>>(s0, scan + 2 * per, scan,
-                                                                                           scan + per, G);
+    kda_scan_combine_kernel<<<(unsigned)(BH * (kD / kScanCols)), kScanThreads, kScanSmem, stream>>>(
+        s0, scan + 2 * per, scan, scan + per, G, hdr);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     a.phase = 3;
