@@ -238,6 +238,9 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The state pass may now be scheduled: it waits for this grid to finish
+  // before it reads anything, and this CTA already holds its tensor memory.
+  grid_dep_launch();
   const uint32_t tm = tmem_base;
   wait_or_flag(&bar_in, 0, hdr, 1);
 
@@ -699,6 +702,11 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   const int h = bh % H, b = bh / H;
   const uint8_t* recs = args.records + ((size_t)bh * NC + cb) * kRecBytes;
 
+  // Launched right behind the kernel that wrote its inputs: nothing global
+  // (and no tensor memory, which that kernel's CTAs may still be allocating)
+  // is touched before it has finished.
+  if (tid == 0) prefetch_tensormap(&tm_o);
+  grid_dep_wait();
   if (tid == 0) {
     mbar_init(&bar_full[0], 1);
     mbar_init(&bar_full[1], 1);
@@ -721,6 +729,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
+  if (args.phase == 1) grid_dep_launch();  // the combination kernel may be scheduled
 
   if (warp == 8) {
     // ------------------------------------------------------------ mma
@@ -986,6 +995,8 @@ __global__ void __launch_bounds__(kScanThreads) kda_scan_combine_kernel(const fl
     for (int p = 0; p < 4; ++p)
       bulk_load(Mt + stage * kSt + p * (kSt / 4), mb + g * kSt + p * (kSt / 4), kScanStageBytes / 4, &full[stage]);
   };
+  grid_dep_wait();    // the transition and offset passes have finished
+  grid_dep_launch();  // the output pass may be scheduled (it waits for this grid)
   if (tid == 0) {
     for (int s = 0; s < kScanStages; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
@@ -1145,6 +1156,25 @@ void scan_groups(int BH, int NC, int* G_out, int* L_out) {
   *L_out = NC;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the one before it in the stream still runs, and waits for it on the
+// device (grid_dep_wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk) {
   (void)dk, (void)dv, (void)chunk;
   const int NC = (int)(((size_t)T + kC - 1) / kC);
@@ -1191,7 +1221,7 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   int G, L;
   scan_groups(BH, NC, &G, &L);
   if (G == 1) {
-    kda_state_pass_kernel<<<(unsigned)BH, kSPThreads, kP2Bytes + 1024, stream>>>(mo, a);
+    e = launch_dependent(kda_state_pass_kernel, (unsigned)BH, kSPThreads, kP2Bytes + 1024, stream, mo, a);
   } else {
     float* scan = reinterpret_cast<float*>(records + (size_t)BH * NC * kRecBytes);
     const size_t per = (size_t)BH * G * kD * kD;
@@ -1201,17 +1231,16 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     a.G = G;
     a.L = L;
     a.phase = 1;
-    kda_state_pass_kernel<<<(unsigned)(BH * (2 * G - 3)), kSPThreads, kP2Bytes + 1024, stream>>>(mo, a);
-    e = cudaGetLastError();
+    e = launch_dependent(kda_state_pass_kernel, (unsigned)(BH * (2 * G - 3)), kSPThreads, kP2Bytes + 1024, stream,
+                         mo, a);
     if (e != cudaSuccess) return e;
-    kda_scan_combine_kernel<<<(unsigned)(BH * (kD / kScanCols)), kScanThreads, kScanSmem, stream>>>(
-        s0, scan + 2 * per, scan, scan + per, G, hdr);
-    e = cudaGetLastError();
+    e = launch_dependent(kda_scan_combine_kernel, (unsigned)(BH * (kD / kScanCols)), kScanThreads, kScanSmem, stream,
+                         s0, scan + 2 * per, (const float*)scan, (const float*)(scan + per), G, hdr);
     if (e != cudaSuccess) return e;
     a.phase = 3;
-    kda_state_pass_kernel<<<(unsigned)(BH * G), kSPThreads, kP2Bytes + 1024, stream>>>(mo, a);
+    e = launch_dependent(kda_state_pass_kernel, (unsigned)(BH * G), kSPThreads, kP2Bytes + 1024, stream, mo, a);
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 2, stream);
   return e;
 }

@@ -143,6 +143,15 @@ __device__ __forceinline__ void bulk_wait_read_n() { asm volatile("cp.async.bulk
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may be scheduled while the kernel before it still runs; it
+// must pass grid_dep_wait() before it touches any global memory the earlier
+// kernel reads or writes (the wait returns once that grid has completed and
+// its writes are visible; without the launch attribute it returns at once).
+// grid_dep_launch() lets the next such kernel be scheduled once every CTA of
+// this grid has issued it or exited.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 // Generic-proxy shared-memory writes -> visible to the async proxy (MMA/TMA).
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
