@@ -6,8 +6,8 @@
 The compiled library (libkda.so, built by ``build.build()``) does all the
 work; the binding only marshals arguments.  It is loaded on first use.
 """
-from .binding import (KDAError, kda_chunk_fwd, kda_chunk_fwd_check, kda_chunk_fwd_workspace_size,
-                      kda_recurrent_step, load, status_string, version)
+from .binding import (KDAError, kda_chunk_fwd, kda_chunk_fwd_check, kda_chunk_fwd_launch_count,
+                      kda_chunk_fwd_workspace_size, kda_recurrent_step, load, status_string, version)
 
-__all__ = ["KDAError", "kda_chunk_fwd", "kda_chunk_fwd_check", "kda_chunk_fwd_workspace_size",
-           "kda_recurrent_step", "load", "status_string", "version"]
+__all__ = ["KDAError", "kda_chunk_fwd", "kda_chunk_fwd_check", "kda_chunk_fwd_launch_count",
+           "kda_chunk_fwd_workspace_size", "kda_recurrent_step", "load", "status_string", "version"]

@@ -25,6 +25,7 @@ SIGNATURES = {
     "kda_status_string": (ctypes.c_char_p, [_i]),
     "kda_version": (_i, []),
     "kda_chunk_fwd_workspace_size": (_sz, [_i] * 7),
+    "kda_chunk_fwd_launch_count": (_i, [_i] * 7),
     "kda_chunk_fwd": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp]),
     "kda_chunk_fwd_profiled": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp, _vp]),
     "kda_chunk_fwd_noalloc": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp]),
@@ -94,6 +95,11 @@ def _stream(stream, device):
 
 def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
     return int(load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, _dtype_code(dtype)))
+
+
+def kda_chunk_fwd_launch_count(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
+    """Kernels one kda_chunk_fwd call with these arguments launches (-1: rejected)."""
+    return int(load().kda_chunk_fwd_launch_count(B, T, H, dk, dv, chunk, _dtype_code(dtype)))
 
 
 def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64, o=None, final_state=None,

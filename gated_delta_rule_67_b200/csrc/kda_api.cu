@@ -57,6 +57,14 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chu
   return 0;
 }
 
+int kda_chunk_fwd_launch_count(int B, int T, int H, int dk, int dv, int chunk, int dtype) {
+  if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || chunk < 1) return -1;
+  if (dtype != KDA_F32 && dtype != KDA_BF16) return -1;
+  if (!prefill_supported(dk, dv, chunk, dtype)) return -1;
+  if (B == 0 || T == 0) return 0;
+  return dtype == KDA_BF16 ? kda::prefill_bf16_launches(B, T, H) : 1;
+}
+
 static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
                                  float scale, const float* initial_state, void* o, float* final_state, int B,
                                  int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,

@@ -34,6 +34,7 @@ cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, c
 
 // bf16 chunked prefill (tcgen05 path).  `ws` is the caller's workspace.
 size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk);
+int prefill_bf16_launches(int B, int T, int H);
 cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                 const __nv_bfloat16* g, const __nv_bfloat16* beta, float scale,
                                 const float* s0, __nv_bfloat16* o, float* sT, int B, int T, int H,

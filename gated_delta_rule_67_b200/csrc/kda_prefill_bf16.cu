@@ -1184,6 +1184,13 @@ size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chu
   return sizeof(WorkspaceHeader) + (size_t)B * H * NC * kRecBytes + scan;
 }
 
+int prefill_bf16_launches(int B, int T, int H) {
+  const int NC = (int)(((size_t)T + kC - 1) / kC);
+  int G, L;
+  scan_groups(B * H, NC, &G, &L);
+  return G > 1 ? 4 : 2;
+}
+
 cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const bf16* beta,
                                 float scale, const float* s0, bf16* o, float* sT, int B, int T, int H, int dk,
                                 int dv, int chunk, void* ws, size_t ws_bytes, cudaStream_t stream,

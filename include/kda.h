@@ -65,6 +65,16 @@ KDA_API int kda_version(void);
 KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int dtype);
 
 /*
+ * Number of kernels one kda_chunk_fwd call with these arguments launches
+ * (the workspace-header clear, a memset, is not counted): 1 for the fp32
+ * path; for bf16 the chunk preparation plus either one state pass or, when
+ * few (sequence, head) chains cover many chunks, the three launches of the
+ * chunk-parallel scan.  0 when there is nothing to run (B or T zero), -1 for
+ * arguments kda_chunk_fwd would reject.  Pure host arithmetic.
+ */
+KDA_API int kda_chunk_fwd_launch_count(int B, int T, int H, int dk, int dv, int chunk, int dtype);
+
+/*
  * Chunked prefill: runs the recurrence over T tokens for B sequences x H heads.
  *
  * Defined by the KDA update (section 2.3) evaluated with the chunkwise

@@ -113,3 +113,14 @@ def test_wait_selftest_validation(lib):
     assert lib.kda_wait_selftest(None, 256, None) == binding.KDA_ERR_INVALID_ARG
     assert lib.kda_wait_selftest(A, 128, None) == binding.KDA_ERR_INVALID_ARG
     assert lib.kda_wait_selftest(A + 16, 256, None) == binding.KDA_ERR_INVALID_ARG
+
+
+def test_launch_count(lib):
+    f = lib.kda_chunk_fwd_launch_count
+    assert f(1, 64, 1, 128, 128, 64, 1) == 2        # prep + one state pass
+    assert f(1, 4096, 16, 128, 128, 64, 1) == 4     # few chains, many chunks: chunk-parallel scan
+    assert f(8, 8192, 32, 128, 128, 64, 1) == 2     # many chains: one state pass
+    assert f(1, 256, 2, 64, 64, 64, 0) == 1         # fp32 path
+    assert f(0, 64, 1, 128, 128, 64, 1) == 0
+    assert f(1, 64, 1, 96, 96, 64, 1) == -1
+    assert f(1, 64, 1, 128, 128, 64, 7) == -1
