@@ -32,7 +32,22 @@ SIGNATURES = {
     "kda_chunk_fwd_check": (_i, [_vp, _sz, _vp]),
     "kda_wait_selftest": (_i, [_vp, _sz, _vp]),
     "kda_recurrent_step": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 5 + [_vp]),
+    "kda_chunk_fwd_gate": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 8 + [_vp, _sz, _vp]),
+    "kda_recurrent_step_gate": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 6 + [_vp]),
 }
+
+# kda_gate: how the forget gate enters the update (see include/kda.h)
+KDA_GATE_CHANNEL, KDA_GATE_HEAD, KDA_GATE_NONE = 0, 1, 2
+
+
+def _gate_kind(g, lead):
+    """Gate kind from g's shape: per key channel [*lead, dk] (KDA), per head
+    [*lead] (Gated DeltaNet), or None (DeltaNet)."""
+    if g is None:
+        return KDA_GATE_NONE
+    if tuple(g.shape) == tuple(lead):
+        return KDA_GATE_HEAD
+    return KDA_GATE_CHANNEL
 
 _lib = None
 
@@ -104,19 +119,26 @@ def kda_chunk_fwd_launch_count(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) 
 
 def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64, o=None, final_state=None,
                   output_final_state=True, workspace=None, stream=None, events=None):
-    """Chunked KDA prefill.  q,k,g [B,T,H,dk], v [B,T,H,dv], beta [B,T,H] (fp32 or bf16, CUDA).
+    """Chunked KDA prefill.  q,k [B,T,H,dk], v [B,T,H,dv], beta [B,T,H] (fp32 or bf16, CUDA).
 
+    g selects the forget gate: [B,T,H,dk] per key channel (KDA), [B,T,H] one
+    per head (Gated DeltaNet), or None (DeltaNet, no forgetting).
     Returns (o [B,T,H,dv] in the input dtype, final_state [B,H,dk,dv] fp32 or None).
     ``final_state`` may be ``initial_state`` itself for an in-place update.
     ``events``: optional three recorded torch.cuda.Event objects; the library
-    records them before, between and after its kernels (kda_chunk_fwd_profiled).
+    records them before, between and after its kernels (kda_chunk_fwd_profiled,
+    per-channel gates only).
     """
     lib = load()
-    for name, x in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
+    for name, x in (("q", q), ("k", k), ("v", v), ("beta", beta)):
         _check_dev(name, x, q.dtype)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    if k.shape != q.shape or g.shape != q.shape or v.shape[:3] != (B, T, H) or beta.shape != (B, T, H):
+    gate = _gate_kind(g, (B, T, H))
+    if g is not None:
+        _check_dev("g", g, q.dtype)
+    if k.shape != q.shape or (gate == KDA_GATE_CHANNEL and g.shape != q.shape) or v.shape[:3] != (B, T, H) \
+            or beta.shape != (B, T, H):
         raise ValueError("shape mismatch among q, k, v, g, beta")
     if scale is None:
         scale = dk ** -0.5
@@ -138,7 +160,11 @@ def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64,
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state), _ptr(o),
             _ptr(final_state), B, T, H, dk, dv, chunk, code, _ptr(workspace), ws_bytes, _stream(stream, q.device))
-    if events is None:
+    if gate != KDA_GATE_CHANNEL:
+        if events is not None:
+            raise ValueError("events are recorded for per-channel gates only")
+        st = lib.kda_chunk_fwd_gate(*args[:16], gate, *args[16:])
+    elif events is None:
         st = lib.kda_chunk_fwd(*args)
     else:
         if len(events) != 3:
@@ -200,17 +226,22 @@ def kda_wait_selftest(workspace, stream=None) -> int:
 
 
 def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=None):
-    """One decode step.  q,k,g [N,H,dk], v [N,H,dv], beta [N,H]; state [N,H,dk,dv] fp32 updated in place.
+    """One decode step.  q,k [N,H,dk], v [N,H,dv], beta [N,H]; state [N,H,dk,dv] fp32 updated in place.
 
-    Returns o [N,H,dv] in the input dtype.
+    g selects the forget gate: [N,H,dk] per key channel (KDA), [N,H] one per
+    head (Gated DeltaNet), or None (DeltaNet).  Returns o [N,H,dv] in the input dtype.
     """
     lib = load()
-    for name, x in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
+    for name, x in (("q", q), ("k", k), ("v", v), ("beta", beta)):
         _check_dev(name, x, q.dtype)
     _check_dev("state", state, torch.float32)
     N, H, dk = q.shape
     dv = v.shape[-1]
-    if k.shape != q.shape or g.shape != q.shape or v.shape[:2] != (N, H) or beta.shape != (N, H):
+    gate = _gate_kind(g, (N, H))
+    if g is not None:
+        _check_dev("g", g, q.dtype)
+    if k.shape != q.shape or (gate == KDA_GATE_CHANNEL and g.shape != q.shape) or v.shape[:2] != (N, H) \
+            or beta.shape != (N, H):
         raise ValueError("shape mismatch among q, k, v, g, beta")
     if state.shape != (N, H, dk, dv):
         raise ValueError("state must be [N,H,dk,dv]")
@@ -219,8 +250,12 @@ def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=No
     if o is None:
         o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
     _check_dev("o", o, q.dtype)
-    st = lib.kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(state),
-                                _ptr(o), N, H, dk, dv, _dtype_code(q.dtype), _stream(stream, q.device))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(state), _ptr(o), N, H, dk, dv,
+            _dtype_code(q.dtype))
+    if gate == KDA_GATE_CHANNEL:
+        st = lib.kda_recurrent_step(*args, _stream(stream, q.device))
+    else:
+        st = lib.kda_recurrent_step_gate(*args, gate, _stream(stream, q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_recurrent_step")
     return o

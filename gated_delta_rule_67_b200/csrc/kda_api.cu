@@ -67,25 +67,29 @@ int kda_chunk_fwd_launch_count(int B, int T, int H, int dk, int dv, int chunk, i
 
 static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
                                  float scale, const float* initial_state, void* o, float* final_state, int B,
-                                 int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
+                                 int T, int H, int dk, int dv, int chunk, int dtype, int gate, void* workspace,
                                  size_t workspace_bytes, void* stream_, void* const* events) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || chunk < 1) return KDA_ERR_INVALID_ARG;
   if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
+  if (gate == KDA_GATE_NONE) g = nullptr;
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
   const bool empty = (B == 0 || T == 0);
   const size_t eb = elem_bytes(dtype);
   const size_t ntok = (size_t)B * T * H;
   const Range rq{(const char*)q, ntok * dk * eb}, rk{(const char*)k, ntok * dk * eb},
-      rg{(const char*)g, ntok * dk * eb}, rv{(const char*)v, ntok * dv * eb},
+      rg{(const char*)g, gate == KDA_GATE_CHANNEL ? ntok * dk * eb : ntok * eb}, rv{(const char*)v, ntok * dv * eb},
       rb{(const char*)beta, ntok * eb}, ro{(const char*)o, ntok * dv * eb};
   const size_t state_bytes = (size_t)B * H * dk * dv * sizeof(float);
   const Range rs0{(const char*)initial_state, state_bytes}, rsT{(const char*)final_state, state_bytes};
   if (!empty) {
-    const void* need[] = {q, k, v, g, o};
+    const void* need[] = {q, k, v, o};
     for (const void* p : need)
       if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
     if (!beta || !aligned_to(beta, eb)) return KDA_ERR_INVALID_ARG;
+    if (gate == KDA_GATE_CHANNEL && (!g || !aligned16(g))) return KDA_ERR_INVALID_ARG;
+    if (gate == KDA_GATE_HEAD && (!g || !aligned_to(g, eb))) return KDA_ERR_INVALID_ARG;
     // o is written: it must not overlap any input.
     for (Range r : {rq, rk, rg, rv, rb, rs0})
       if (overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
@@ -125,13 +129,13 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
   if (dtype == KDA_F32) {
     e = kda::launch_prefill_f32((const float*)q, (const float*)k, (const float*)v, (const float*)g,
                                 (const float*)beta, scale, initial_state, (float*)o, final_state, B, T,
-                                H, dk, dv, chunk, stream, events);
+                                H, dk, dv, chunk, gate, stream, events);
   } else {
     e = kda::launch_prefill_bf16((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                  (const __nv_bfloat16*)v, (const __nv_bfloat16*)g,
                                  (const __nv_bfloat16*)beta, scale, initial_state, (__nv_bfloat16*)o,
-                                 final_state, B, T, H, dk, dv, chunk, workspace, workspace_bytes, stream,
-                                 events);
+                                 final_state, B, T, H, dk, dv, chunk, gate, workspace, workspace_bytes,
+                                 stream, events);
   }
   return from_cuda(e);
 }
@@ -141,7 +145,15 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
                          int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream) {
   return chunk_fwd_impl(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
-                        workspace, workspace_bytes, stream, nullptr);
+                        KDA_GATE_CHANNEL, workspace, workspace_bytes, stream, nullptr);
+}
+
+kda_status kda_chunk_fwd_gate(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                              float scale, const float* initial_state, void* o, float* final_state, int B, int T,
+                              int H, int dk, int dv, int chunk, int dtype, int gate, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return chunk_fwd_impl(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
+                        gate, workspace, workspace_bytes, stream, nullptr);
 }
 
 kda_status kda_chunk_fwd_profiled(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -150,7 +162,7 @@ kda_status kda_chunk_fwd_profiled(const void* q, const void* k, const void* v, c
                                   size_t workspace_bytes, void* stream, void* const* events) {
   if (!events) return KDA_ERR_INVALID_ARG;
   return chunk_fwd_impl(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
-                        workspace, workspace_bytes, stream, events);
+                        KDA_GATE_CHANNEL, workspace, workspace_bytes, stream, events);
 }
 
 kda_status kda_chunk_fwd_check(const void* workspace, size_t workspace_bytes, void* stream_) {
@@ -170,29 +182,46 @@ kda_status kda_wait_selftest(void* workspace, size_t workspace_bytes, void* stre
   return from_cuda(kda::launch_wait_selftest(workspace, static_cast<cudaStream_t>(stream_)));
 }
 
-kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g,
-                              const void* beta, float scale, float* state, void* o, int N, int H,
-                              int dk, int dv, int dtype, void* stream_) {
+static kda_status recurrent_step_impl(const void* q, const void* k, const void* v, const void* g,
+                                      const void* beta, float scale, float* state, void* o, int N, int H, int dk,
+                                      int dv, int dtype, int gate, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (N < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
   if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
+  if (gate == KDA_GATE_NONE) g = nullptr;
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
   if (N == 0) return KDA_OK;
   const size_t eb = elem_bytes(dtype);
-  const void* need[] = {q, k, v, g, state, o};
+  const void* need[] = {q, k, v, state, o};
   for (const void* p : need)
     if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
   if (!beta || !aligned_to(beta, eb)) return KDA_ERR_INVALID_ARG;
+  if (gate == KDA_GATE_CHANNEL && (!g || !aligned16(g))) return KDA_ERR_INVALID_ARG;
+  if (gate == KDA_GATE_HEAD && (!g || !aligned_to(g, eb))) return KDA_ERR_INVALID_ARG;
   const size_t nh = (size_t)N * H;
   const Range rq{(const char*)q, nh * dk * eb}, rk{(const char*)k, nh * dk * eb},
-      rg{(const char*)g, nh * dk * eb}, rv{(const char*)v, nh * dv * eb}, rb{(const char*)beta, nh * eb},
-      ro{(const char*)o, nh * dv * eb}, rs{(const char*)state, nh * dk * dv * sizeof(float)};
+      rg{(const char*)g, gate == KDA_GATE_CHANNEL ? nh * dk * eb : nh * eb}, rv{(const char*)v, nh * dv * eb},
+      rb{(const char*)beta, nh * eb}, ro{(const char*)o, nh * dv * eb},
+      rs{(const char*)state, nh * dk * dv * sizeof(float)};
   for (Range r : {rq, rk, rg, rv, rb, rs})
     if (overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
   for (Range r : {rq, rk, rg, rv, rb})
     if (overlaps(rs, r)) return KDA_ERR_INVALID_ARG;
   if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
-  return from_cuda(kda::launch_decode(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, stream));
+  return from_cuda(kda::launch_decode(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, gate, stream));
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g,
+                              const void* beta, float scale, float* state, void* o, int N, int H,
+                              int dk, int dv, int dtype, void* stream) {
+  return recurrent_step_impl(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, KDA_GATE_CHANNEL, stream);
+}
+
+kda_status kda_recurrent_step_gate(const void* q, const void* k, const void* v, const void* g,
+                                   const void* beta, float scale, float* state, void* o, int N, int H,
+                                   int dk, int dv, int dtype, int gate, void* stream) {
+  return recurrent_step_impl(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, gate, stream);
 }
 
 }  // extern "C"

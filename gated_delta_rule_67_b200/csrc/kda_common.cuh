@@ -25,11 +25,11 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { retu
 // launch(es).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, const void* beta,
                           float scale, float* state, void* o, int N, int H, int dk, int dv, int dtype,
-                          cudaStream_t stream);
+                          int gate, cudaStream_t stream);
 
 cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* g,
                                const float* beta, float scale, const float* s0, float* o, float* sT,
-                               int B, int T, int H, int dk, int dv, int chunk, cudaStream_t stream,
+                               int B, int T, int H, int dk, int dv, int chunk, int gate, cudaStream_t stream,
                                void* const* events);
 
 // bf16 chunked prefill (tcgen05 path).  `ws` is the caller's workspace.
@@ -38,11 +38,21 @@ int prefill_bf16_launches(int B, int T, int H);
 cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                 const __nv_bfloat16* g, const __nv_bfloat16* beta, float scale,
                                 const float* s0, __nv_bfloat16* o, float* sT, int B, int T, int H,
-                                int dk, int dv, int chunk, void* ws, size_t ws_bytes,
+                                int dk, int dv, int chunk, int gate, void* ws, size_t ws_bytes,
                                 cudaStream_t stream, void* const* events);
 
 // Launches a kernel whose only wait can never be satisfied (short limit).
 cudaError_t launch_wait_selftest(void* ws, cudaStream_t stream);
+
+// Decay factor alpha = exp(g) of key channel c for one (token, head) whose
+// per-channel gates start at g_chan and whose per-head gate is g_head
+// (kda_gate: per channel, per head, or none).
+template <typename T>
+__device__ __forceinline__ float gate_alpha(int gate, const T* g_chan, const T* g_head, int c) {
+  if (gate == KDA_GATE_CHANNEL) return expf(to_f32(g_chan[c]));
+  if (gate == KDA_GATE_HEAD) return expf(to_f32(*g_head));
+  return 1.f;
+}
 
 // Records events[i] on the stream when an events array was given.
 inline cudaError_t mark(void* const* events, int i, cudaStream_t stream) {

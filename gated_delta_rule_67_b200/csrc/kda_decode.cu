@@ -49,7 +49,7 @@ template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
     decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                        const T* __restrict__ g, const T* __restrict__ beta, float scale,
-                       float* __restrict__ state, T* __restrict__ o) {
+                       float* __restrict__ state, T* __restrict__ o, int gate) {
   constexpr int NW = kDecodeWarps, RW = DK / NW, CL = DV / 32;
   __shared__ float sq[DK], sk[DK], sa[DK], sv[DV], su[DV];
   __shared__ __align__(16) float pk[NW][DV];
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   if (tid < DK) {
     sq[tid] = to_f32(q[head * DK + tid]);
     sk[tid] = to_f32(k[head * DK + tid]);
-    sa[tid] = expf(to_f32(g[head * DK + tid]));
+    sa[tid] = gate_alpha(gate, g + head * DK, g + head, tid);
   }
   if (tid < DV) sv[tid] = to_f32(v[head * DV + tid]);
   if (tid == 0) sbeta = to_f32(beta[head]);
@@ -133,31 +133,31 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 
 template <typename T, int DK, int DV>
 cudaError_t launch_typed(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                         float scale, float* state, void* o, int N, int H, cudaStream_t stream) {
+                         float scale, float* state, void* o, int N, int H, int gate, cudaStream_t stream) {
   const unsigned heads = (unsigned)N * (unsigned)H;
   decode_step_kernel<T, DK, DV><<<heads, kDecodeWarps * 32, 0, stream>>>(
-      (const T*)q, (const T*)k, (const T*)v, (const T*)g, (const T*)beta, scale, state, (T*)o);
+      (const T*)q, (const T*)k, (const T*)v, (const T*)g, (const T*)beta, scale, state, (T*)o, gate);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_dims(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                        float scale, float* state, void* o, int N, int H, int dk, int dv,
+                        float scale, float* state, void* o, int N, int H, int dk, int dv, int gate,
                         cudaStream_t stream) {
-  if (dk == 128 && dv == 128) return launch_typed<T, 128, 128>(q, k, v, g, beta, scale, state, o, N, H, stream);
-  if (dk == 128 && dv == 64) return launch_typed<T, 128, 64>(q, k, v, g, beta, scale, state, o, N, H, stream);
-  if (dk == 64 && dv == 128) return launch_typed<T, 64, 128>(q, k, v, g, beta, scale, state, o, N, H, stream);
-  return launch_typed<T, 64, 64>(q, k, v, g, beta, scale, state, o, N, H, stream);
+  if (dk == 128 && dv == 128) return launch_typed<T, 128, 128>(q, k, v, g, beta, scale, state, o, N, H, gate, stream);
+  if (dk == 128 && dv == 64) return launch_typed<T, 128, 64>(q, k, v, g, beta, scale, state, o, N, H, gate, stream);
+  if (dk == 64 && dv == 128) return launch_typed<T, 64, 128>(q, k, v, g, beta, scale, state, o, N, H, gate, stream);
+  return launch_typed<T, 64, 64>(q, k, v, g, beta, scale, state, o, N, H, gate, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, const void* beta,
                           float scale, float* state, void* o, int N, int H, int dk, int dv, int dtype,
-                          cudaStream_t stream) {
+                          int gate, cudaStream_t stream) {
   if (dtype == KDA_F32)
-    return launch_dims<float>(q, k, v, g, beta, scale, state, o, N, H, dk, dv, stream);
-  return launch_dims<__nv_bfloat16>(q, k, v, g, beta, scale, state, o, N, H, dk, dv, stream);
+    return launch_dims<float>(q, k, v, g, beta, scale, state, o, N, H, dk, dv, gate, stream);
+  return launch_dims<__nv_bfloat16>(q, k, v, g, beta, scale, state, o, N, H, dk, dv, gate, stream);
 }
 
 }  // namespace kda

@@ -201,16 +201,21 @@ __device__ __forceinline__ void store_block_frag(float* X, const float (&acc)[2]
   }
 }
 
+// kScalarGate: the forget gate is one log-gate per (token, head) read from
+// g_head (Gated DeltaNet), or none when g_head is null (DeltaNet); otherwise
+// the per-channel g tile comes in by TMA (KDA).
+template <bool kScalarGate>
 __global__ void __launch_bounds__(kP1Threads, 3)
     kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                           const bf16* __restrict__ beta, float scale, uint8_t* __restrict__ records,
-                          WorkspaceHeader* hdr, int T, int H, int NC) {
+                          WorkspaceHeader* hdr, int T, int H, int NC, const bf16* __restrict__ g_head) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t bar_in, bar_v, bar_mma;
   __shared__ uint32_t tmem_base;
   __shared__ float sbeta[kC];
+  __shared__ float sgh[kScalarGate ? kC : 1];  // per-head log-gates of the chunk (zeros without a gate)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x % NC;
@@ -225,16 +230,20 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     mbar_init(&bar_v, 1);
     mbar_init(&bar_mma, 1);
     fence_mbar_init();
-    mbar_expect_tx(&bar_in, 3 * 16384);
+    mbar_expect_tx(&bar_in, (kScalarGate ? 2 : 3) * 16384);
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) {
-      tma_load_4d(sm + kP1A + kb * 16384, &tm_g, &bar_in, kb * 64, h, t0, b);         // rows 0-63
-      tma_load_4d(sm + kP1A + kb * 16384 + 8192, &tm_q, &bar_in, kb * 64, h, t0, b);  // rows 64-127
+      if (!kScalarGate) tma_load_4d(sm + kP1A + kb * 16384, &tm_g, &bar_in, kb * 64, h, t0, b);  // rows 0-63
+      tma_load_4d(sm + kP1A + kb * 16384 + 8192, &tm_q, &bar_in, kb * 64, h, t0, b);     // rows 64-127
       tma_load_4d(sm + kP1K + kb * 8192, &tm_k, &bar_in, kb * 64, h, t0, b);
     }
   }
   if (warp == 0) tmem_alloc(&tmem_base, 128);
   if (tid < kC) sbeta[tid] = tid < L ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
+  if (kScalarGate && tid >= kC && tid < 2 * kC) {
+    const int i = tid - kC;
+    sgh[i] = (g_head && i < L) ? __bfloat162float(g_head[((size_t)b * T + t0 + i) * H + h]) : 0.f;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -253,8 +262,15 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   const int tg = lane & 15;
   const int c8 = 8 * cg;
   float G[4][8], gref[8], gend[8];
+  if (!kScalarGate) {
 #pragma unroll
-  for (int t = 0; t < 4; ++t) ld8(sm + kP1A + kmajor_off(tg + 16 * t, c8, 128), G[t]);
+    for (int t = 0; t < 4; ++t) ld8(sm + kP1A + kmajor_off(tg + 16 * t, c8, 128), G[t]);
+  } else {  // one log-gate per token for every channel (zero without a gate)
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) G[t][e] = sgh[tg + 16 * t];
+  }
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     float tot[4];
@@ -1193,13 +1209,16 @@ int prefill_bf16_launches(int B, int T, int H) {
 
 cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const bf16* beta,
                                 float scale, const float* s0, bf16* o, float* sT, int B, int T, int H, int dk,
-                                int dv, int chunk, void* ws, size_t ws_bytes, cudaStream_t stream,
+                                int dv, int chunk, int gate, void* ws, size_t ws_bytes, cudaStream_t stream,
                                 void* const* events) {
   (void)dk, (void)dv, (void)chunk, (void)ws_bytes;
   static bool attrs_set = false;
   if (!attrs_set) {
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_prep_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kP1Bytes + 1024);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kda_chunk_prep_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kP1Bytes + 1024);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kP2Bytes + 1024);
     if (e != cudaSuccess) return e;
@@ -1208,8 +1227,9 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     attrs_set = true;
   }
   CUtensorMap mq, mk, mv, mg, mo;
+  memset(&mg, 0, sizeof(mg));  // only the per-channel gate is read through a tensor map
   if (!make_map(&mq, q, B, T, H) || !make_map(&mk, k, B, T, H) || !make_map(&mv, v, B, T, H) ||
-      !make_map(&mg, g, B, T, H) || !make_map(&mo, o, B, T, H, false))
+      (gate == KDA_GATE_CHANNEL && !make_map(&mg, g, B, T, H)) || !make_map(&mo, o, B, T, H, false))
     return cudaErrorInvalidValue;
   const int NC = (T + kC - 1) / kC;
   WorkspaceHeader* hdr = static_cast<WorkspaceHeader*>(ws);
@@ -1218,8 +1238,12 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(WorkspaceHeader), stream);
   if (e != cudaSuccess) return e;
   const unsigned tiles = (unsigned)((size_t)B * H * NC);
-  kda_chunk_prep_kernel<<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records, hdr, T, H,
-                                                                  NC);
+  if (gate == KDA_GATE_CHANNEL)
+    kda_chunk_prep_kernel<false><<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records,
+                                                                               hdr, T, H, NC, nullptr);
+  else
+    kda_chunk_prep_kernel<true><<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(
+        mq, mk, mv, mg, beta, scale, records, hdr, T, H, NC, gate == KDA_GATE_HEAD ? g : nullptr);
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e != cudaSuccess) return e;

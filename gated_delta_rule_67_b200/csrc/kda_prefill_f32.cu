@@ -25,7 +25,7 @@ __global__ void __launch_bounds__(kCols * kGroups)
     prefill_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                        const float* __restrict__ v, const float* __restrict__ g,
                        const float* __restrict__ beta, float scale, const float* __restrict__ s0,
-                       float* __restrict__ o, float* sT, int T, int H, int DV) {
+                       float* __restrict__ o, float* sT, int T, int H, int DV, int gate) {
   constexpr int RW = DK / kGroups;
   __shared__ float sq[kTile][DK], sk[kTile][DK], sa[kTile][DK];
   __shared__ float sv[kTile][kCols], sb[kTile];
@@ -46,10 +46,10 @@ __global__ void __launch_bounds__(kCols * kGroups)
     __syncthreads();
     for (int e = tid; e < nt * DK; e += blockDim.x) {
       const int tt = e / DK, c = e % DK;
-      const size_t off = (((size_t)b * T + t0 + tt) * H + h) * DK + c;
+      const size_t tok = ((size_t)b * T + t0 + tt) * H + h, off = tok * DK + c;
       sq[tt][c] = q[off];
       sk[tt][c] = k[off];
-      sa[tt][c] = expf(g[off]);
+      sa[tt][c] = gate_alpha(gate, g + tok * DK, g + tok, c);
     }
     for (int e = tid; e < nt * kCols; e += blockDim.x) {
       const int tt = e / kCols, c = e % kCols;
@@ -91,16 +91,16 @@ __global__ void __launch_bounds__(kCols * kGroups)
 
 cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* g,
                                const float* beta, float scale, const float* s0, float* o, float* sT,
-                               int B, int T, int H, int dk, int dv, int chunk, cudaStream_t stream,
+                               int B, int T, int H, int dk, int dv, int chunk, int gate, cudaStream_t stream,
                                void* const* events) {
   (void)chunk;
   dim3 grid(dv / kCols, H, B);
   cudaError_t e = mark(events, 0, stream);
   if (e != cudaSuccess) return e;
   if (dk == 128)
-    prefill_f32_kernel<128><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv);
+    prefill_f32_kernel<128><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv, gate);
   else
-    prefill_f32_kernel<64><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv);
+    prefill_f32_kernel<64><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv, gate);
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e == cudaSuccess) e = mark(events, 2, stream);

@@ -144,3 +144,10 @@ def make_decode_inputs(steps, N, H, dk, dv, dtype=torch.bfloat16, s0_std=0.1, se
     g = _draw("gate", (steps, N, H, dk), 0, dtype, gen, device)
     state = torch.randn((N, H, dk, dv), generator=gen, device=device, dtype=torch.float32) * s0_std
     return dict(q=q, k=k, v=v, g=g, beta=beta, state=state)
+
+
+def make_head_gates(lead_shape, seq_axis, dtype=torch.bfloat16, seed=0, device="cpu"):
+    """Seeded per-head log-gates for the Gated DeltaNet form: one
+    logsigmoid(N(3, 1)) value per (token, head), shape ``lead_shape`` (e.g.
+    [B, T, H] or [steps, N, H]), drawn from its own generator."""
+    return _draw("gate", tuple(lead_shape), seq_axis, dtype, _gen(seed, device), device)

@@ -52,6 +52,22 @@ typedef enum {
 
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
 
+/*
+ * How the forget gate enters the state update (argument `gate` of the *_gate
+ * entry points; the plain entry points use KDA_GATE_CHANNEL):
+ *   KDA_GATE_CHANNEL  KDA ("KimiLinear: A Next-Generation Linear Attention
+ *                     Architecture for Long-Context LLMs", section 2.3): one
+ *                     log-gate per key channel, g [.., dk], alpha = exp(g)
+ *                     scales the rows of the state before the delta step.
+ *   KDA_GATE_HEAD     Gated DeltaNet (same page, section 2.2): one scalar
+ *                     log-gate per token and head, g [.., 1] (layout
+ *                     [B, T, H] / [N, H] like beta), alpha_t = exp(g) scales
+ *                     the whole state.
+ *   KDA_GATE_NONE     DeltaNet (same page, section 2.1): no forget gate,
+ *                     alpha = 1; g is ignored and may be NULL.
+ */
+typedef enum { KDA_GATE_CHANNEL = 0, KDA_GATE_HEAD = 1, KDA_GATE_NONE = 2 } kda_gate;
+
 /* Human-readable name of a status code (static storage, never NULL). */
 KDA_API const char* kda_status_string(int status);
 
@@ -107,6 +123,19 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
                          float scale, const float* initial_state, void* o, float* final_state, int B,
                          int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * kda_chunk_fwd with the forget gate of `gate` (kda_gate): KDA_GATE_CHANNEL
+ * is kda_chunk_fwd itself; KDA_GATE_HEAD takes g as [B, T, H] (dtype,
+ * element alignment like beta); KDA_GATE_NONE ignores g (NULL allowed).  The
+ * workspace size is the same for every gate.  Other arguments, supported
+ * shapes, checks and errors as kda_chunk_fwd; an unknown gate is
+ * KDA_ERR_INVALID_ARG.
+ */
+KDA_API kda_status kda_chunk_fwd_gate(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                      float scale, const float* initial_state, void* o, float* final_state, int B,
+                                      int T, int H, int dk, int dv, int chunk, int dtype, int gate, void* workspace,
+                                      size_t workspace_bytes, void* stream);
 
 /*
  * kda_chunk_fwd with timing marks for measurement: `events` points to three
@@ -175,6 +204,15 @@ KDA_API kda_status kda_wait_selftest(void* workspace, size_t workspace_bytes, vo
 KDA_API kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, float scale, float* state, void* o, int N, int H,
                               int dk, int dv, int dtype, void* stream);
+
+/*
+ * kda_recurrent_step with the forget gate of `gate` (kda_gate): g is [N, H, dk]
+ * for KDA_GATE_CHANNEL, [N, H] for KDA_GATE_HEAD (element alignment), and
+ * ignored (NULL allowed) for KDA_GATE_NONE.  Otherwise as kda_recurrent_step.
+ */
+KDA_API kda_status kda_recurrent_step_gate(const void* q, const void* k, const void* v, const void* g,
+                                           const void* beta, float scale, float* state, void* o, int N, int H,
+                                           int dk, int dv, int dtype, int gate, void* stream);
 
 #ifdef __cplusplus
 }
