@@ -32,12 +32,15 @@ SIGNATURES = {
     "kda_chunk_fwd_check": (_i, [_vp, _sz, _vp]),
     "kda_wait_selftest": (_i, [_vp, _sz, _vp]),
     "kda_recurrent_step": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 5 + [_vp]),
-    "kda_chunk_fwd_gate": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 8 + [_vp, _sz, _vp]),
-    "kda_recurrent_step_gate": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 6 + [_vp]),
+    "kda_chunk_fwd_ex": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 9 + [_vp, _sz, _vp]),
+    "kda_recurrent_step_ex": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 7 + [_vp]),
 }
 
 # kda_gate: how the forget gate enters the update (see include/kda.h)
 KDA_GATE_CHANNEL, KDA_GATE_HEAD, KDA_GATE_NONE = 0, 1, 2
+# kda_prep bits: raw inputs prepared inside the kernels (see include/kda.h)
+KDA_PREP_L2NORM_QK, KDA_PREP_GATE_LOGSIGMOID, KDA_PREP_BETA_SIGMOID = 1, 2, 4
+KDA_PREP_ALL = KDA_PREP_L2NORM_QK | KDA_PREP_GATE_LOGSIGMOID | KDA_PREP_BETA_SIGMOID
 
 
 def _gate_kind(g, lead):
@@ -118,11 +121,13 @@ def kda_chunk_fwd_launch_count(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) 
 
 
 def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64, o=None, final_state=None,
-                  output_final_state=True, workspace=None, stream=None, events=None):
+                  output_final_state=True, workspace=None, stream=None, events=None, prep=0):
     """Chunked KDA prefill.  q,k [B,T,H,dk], v [B,T,H,dv], beta [B,T,H] (fp32 or bf16, CUDA).
 
     g selects the forget gate: [B,T,H,dk] per key channel (KDA), [B,T,H] one
     per head (Gated DeltaNet), or None (DeltaNet, no forgetting).
+    ``prep``: KDA_PREP_* bits; the marked inputs are raw projections prepared
+    in the kernels (q, k to unit length; g = logsigmoid(g); beta = sigmoid(beta)).
     Returns (o [B,T,H,dv] in the input dtype, final_state [B,H,dk,dv] fp32 or None).
     ``final_state`` may be ``initial_state`` itself for an in-place update.
     ``events``: optional three recorded torch.cuda.Event objects; the library
@@ -160,10 +165,10 @@ def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64,
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state), _ptr(o),
             _ptr(final_state), B, T, H, dk, dv, chunk, code, _ptr(workspace), ws_bytes, _stream(stream, q.device))
-    if gate != KDA_GATE_CHANNEL:
+    if gate != KDA_GATE_CHANNEL or prep:
         if events is not None:
-            raise ValueError("events are recorded for per-channel gates only")
-        st = lib.kda_chunk_fwd_gate(*args[:16], gate, *args[16:])
+            raise ValueError("events are recorded for prepared per-channel-gate inputs only")
+        st = lib.kda_chunk_fwd_ex(*args[:16], gate, int(prep), *args[16:])
     elif events is None:
         st = lib.kda_chunk_fwd(*args)
     else:
@@ -225,11 +230,12 @@ def kda_wait_selftest(workspace, stream=None) -> int:
     return kda_chunk_fwd_check(workspace, stream)
 
 
-def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=None):
+def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=None, prep=0):
     """One decode step.  q,k [N,H,dk], v [N,H,dv], beta [N,H]; state [N,H,dk,dv] fp32 updated in place.
 
     g selects the forget gate: [N,H,dk] per key channel (KDA), [N,H] one per
-    head (Gated DeltaNet), or None (DeltaNet).  Returns o [N,H,dv] in the input dtype.
+    head (Gated DeltaNet), or None (DeltaNet).  ``prep``: KDA_PREP_* bits as for
+    kda_chunk_fwd.  Returns o [N,H,dv] in the input dtype.
     """
     lib = load()
     for name, x in (("q", q), ("k", k), ("v", v), ("beta", beta)):
@@ -252,10 +258,10 @@ def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=No
     _check_dev("o", o, q.dtype)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(state), _ptr(o), N, H, dk, dv,
             _dtype_code(q.dtype))
-    if gate == KDA_GATE_CHANNEL:
+    if gate == KDA_GATE_CHANNEL and not prep:
         st = lib.kda_recurrent_step(*args, _stream(stream, q.device))
     else:
-        st = lib.kda_recurrent_step_gate(*args, gate, _stream(stream, q.device))
+        st = lib.kda_recurrent_step_ex(*args, gate, int(prep), _stream(stream, q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_recurrent_step")
     return o

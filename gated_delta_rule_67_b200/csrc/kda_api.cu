@@ -67,12 +67,13 @@ int kda_chunk_fwd_launch_count(int B, int T, int H, int dk, int dv, int chunk, i
 
 static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
                                  float scale, const float* initial_state, void* o, float* final_state, int B,
-                                 int T, int H, int dk, int dv, int chunk, int dtype, int gate, void* workspace,
-                                 size_t workspace_bytes, void* stream_, void* const* events) {
+                                 int T, int H, int dk, int dv, int chunk, int dtype, int gate, int prep,
+                                 void* workspace, size_t workspace_bytes, void* stream_, void* const* events) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || chunk < 1) return KDA_ERR_INVALID_ARG;
   if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
+  if (prep & ~kda::kPrepMask) return KDA_ERR_INVALID_ARG;
   if (gate == KDA_GATE_NONE) g = nullptr;
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
   const bool empty = (B == 0 || T == 0);
@@ -129,12 +130,12 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
   if (dtype == KDA_F32) {
     e = kda::launch_prefill_f32((const float*)q, (const float*)k, (const float*)v, (const float*)g,
                                 (const float*)beta, scale, initial_state, (float*)o, final_state, B, T,
-                                H, dk, dv, chunk, gate, stream, events);
+                                H, dk, dv, chunk, gate, prep, stream, events);
   } else {
     e = kda::launch_prefill_bf16((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
                                  (const __nv_bfloat16*)v, (const __nv_bfloat16*)g,
                                  (const __nv_bfloat16*)beta, scale, initial_state, (__nv_bfloat16*)o,
-                                 final_state, B, T, H, dk, dv, chunk, gate, workspace, workspace_bytes,
+                                 final_state, B, T, H, dk, dv, chunk, gate, prep, workspace, workspace_bytes,
                                  stream, events);
   }
   return from_cuda(e);
@@ -145,15 +146,15 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
                          int T, int H, int dk, int dv, int chunk, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream) {
   return chunk_fwd_impl(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
-                        KDA_GATE_CHANNEL, workspace, workspace_bytes, stream, nullptr);
+                        KDA_GATE_CHANNEL, KDA_PREP_NONE, workspace, workspace_bytes, stream, nullptr);
 }
 
-kda_status kda_chunk_fwd_gate(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                              float scale, const float* initial_state, void* o, float* final_state, int B, int T,
-                              int H, int dk, int dv, int chunk, int dtype, int gate, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                            float scale, const float* initial_state, void* o, float* final_state, int B, int T,
+                            int H, int dk, int dv, int chunk, int dtype, int gate, int prep, void* workspace,
+                            size_t workspace_bytes, void* stream) {
   return chunk_fwd_impl(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
-                        gate, workspace, workspace_bytes, stream, nullptr);
+                        gate, prep, workspace, workspace_bytes, stream, nullptr);
 }
 
 kda_status kda_chunk_fwd_profiled(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -162,7 +163,7 @@ kda_status kda_chunk_fwd_profiled(const void* q, const void* k, const void* v, c
                                   size_t workspace_bytes, void* stream, void* const* events) {
   if (!events) return KDA_ERR_INVALID_ARG;
   return chunk_fwd_impl(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
-                        KDA_GATE_CHANNEL, workspace, workspace_bytes, stream, events);
+                        KDA_GATE_CHANNEL, KDA_PREP_NONE, workspace, workspace_bytes, stream, events);
 }
 
 kda_status kda_chunk_fwd_check(const void* workspace, size_t workspace_bytes, void* stream_) {
@@ -184,11 +185,12 @@ kda_status kda_wait_selftest(void* workspace, size_t workspace_bytes, void* stre
 
 static kda_status recurrent_step_impl(const void* q, const void* k, const void* v, const void* g,
                                       const void* beta, float scale, float* state, void* o, int N, int H, int dk,
-                                      int dv, int dtype, int gate, void* stream_) {
+                                      int dv, int dtype, int gate, int prep, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (N < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
   if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
+  if (prep & ~kda::kPrepMask) return KDA_ERR_INVALID_ARG;
   if (gate == KDA_GATE_NONE) g = nullptr;
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
   if (N == 0) return KDA_OK;
@@ -209,19 +211,20 @@ static kda_status recurrent_step_impl(const void* q, const void* k, const void* 
   for (Range r : {rq, rk, rg, rv, rb})
     if (overlaps(rs, r)) return KDA_ERR_INVALID_ARG;
   if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
-  return from_cuda(kda::launch_decode(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, gate, stream));
+  return from_cuda(kda::launch_decode(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, gate, prep, stream));
 }
 
 kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, float scale, float* state, void* o, int N, int H,
                               int dk, int dv, int dtype, void* stream) {
-  return recurrent_step_impl(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, KDA_GATE_CHANNEL, stream);
+  return recurrent_step_impl(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, KDA_GATE_CHANNEL,
+                             KDA_PREP_NONE, stream);
 }
 
-kda_status kda_recurrent_step_gate(const void* q, const void* k, const void* v, const void* g,
-                                   const void* beta, float scale, float* state, void* o, int N, int H,
-                                   int dk, int dv, int dtype, int gate, void* stream) {
-  return recurrent_step_impl(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, gate, stream);
+kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v, const void* g,
+                                 const void* beta, float scale, float* state, void* o, int N, int H,
+                                 int dk, int dv, int dtype, int gate, int prep, void* stream) {
+  return recurrent_step_impl(q, k, v, g, beta, scale, state, o, N, H, dk, dv, dtype, gate, prep, stream);
 }
 
 }  // extern "C"

@@ -25,12 +25,12 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { retu
 // launch(es).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, const void* beta,
                           float scale, float* state, void* o, int N, int H, int dk, int dv, int dtype,
-                          int gate, cudaStream_t stream);
+                          int gate, int prep, cudaStream_t stream);
 
 cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* g,
                                const float* beta, float scale, const float* s0, float* o, float* sT,
-                               int B, int T, int H, int dk, int dv, int chunk, int gate, cudaStream_t stream,
-                               void* const* events);
+                               int B, int T, int H, int dk, int dv, int chunk, int gate, int prep,
+                               cudaStream_t stream, void* const* events);
 
 // bf16 chunked prefill (tcgen05 path).  `ws` is the caller's workspace.
 size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk);
@@ -38,19 +38,29 @@ int prefill_bf16_launches(int B, int T, int H);
 cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                                 const __nv_bfloat16* g, const __nv_bfloat16* beta, float scale,
                                 const float* s0, __nv_bfloat16* o, float* sT, int B, int T, int H,
-                                int dk, int dv, int chunk, int gate, void* ws, size_t ws_bytes,
+                                int dk, int dv, int chunk, int gate, int prep, void* ws, size_t ws_bytes,
                                 cudaStream_t stream, void* const* events);
 
 // Launches a kernel whose only wait can never be satisfied (short limit).
 cudaError_t launch_wait_selftest(void* ws, cudaStream_t stream);
 
+// Fused input preparation (kda_prep).
+constexpr int kPrepMask = KDA_PREP_L2NORM_QK | KDA_PREP_GATE_LOGSIGMOID | KDA_PREP_BETA_SIGMOID;
+constexpr float kL2Eps = 1e-6f;  // q <- q (sum q^2 + kL2Eps)^-1/2
+__device__ __forceinline__ float log_sigmoid(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
+__device__ __forceinline__ float sigmoidf(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float prep_gate(int prep, float g) {
+  return (prep & KDA_PREP_GATE_LOGSIGMOID) ? log_sigmoid(g) : g;
+}
+__device__ __forceinline__ float prep_beta(int prep, float b) { return (prep & KDA_PREP_BETA_SIGMOID) ? sigmoidf(b) : b; }
+
 // Decay factor alpha = exp(g) of key channel c for one (token, head) whose
 // per-channel gates start at g_chan and whose per-head gate is g_head
-// (kda_gate: per channel, per head, or none).
+// (kda_gate: per channel, per head, or none); g prepared as `prep` says.
 template <typename T>
-__device__ __forceinline__ float gate_alpha(int gate, const T* g_chan, const T* g_head, int c) {
-  if (gate == KDA_GATE_CHANNEL) return expf(to_f32(g_chan[c]));
-  if (gate == KDA_GATE_HEAD) return expf(to_f32(*g_head));
+__device__ __forceinline__ float gate_alpha(int gate, int prep, const T* g_chan, const T* g_head, int c) {
+  if (gate == KDA_GATE_CHANNEL) return expf(prep_gate(prep, to_f32(g_chan[c])));
+  if (gate == KDA_GATE_HEAD) return expf(prep_gate(prep, to_f32(*g_head)));
   return 1.f;
 }
 

@@ -49,12 +49,12 @@ template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
     decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                        const T* __restrict__ g, const T* __restrict__ beta, float scale,
-                       float* __restrict__ state, T* __restrict__ o, int gate) {
+                       float* __restrict__ state, T* __restrict__ o, int gate, int prep) {
   constexpr int NW = kDecodeWarps, RW = DK / NW, CL = DV / 32;
   __shared__ float sq[DK], sk[DK], sa[DK], sv[DV], su[DV];
   __shared__ __align__(16) float pk[NW][DV];
   __shared__ __align__(16) float pq[NW][DV];
-  __shared__ float sqk, sbeta;
+  __shared__ float sqk, sbeta, snorm[2];
 
   const size_t head = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -69,11 +69,27 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   if (tid < DK) {
     sq[tid] = to_f32(q[head * DK + tid]);
     sk[tid] = to_f32(k[head * DK + tid]);
-    sa[tid] = gate_alpha(gate, g + head * DK, g + head, tid);
+    sa[tid] = gate_alpha(gate, prep, g + head * DK, g + head, tid);
   }
   if (tid < DV) sv[tid] = to_f32(v[head * DV + tid]);
-  if (tid == 0) sbeta = to_f32(beta[head]);
+  if (tid == 0) sbeta = prep_beta(prep, to_f32(beta[head]));
   __syncthreads();
+  if (prep & KDA_PREP_L2NORM_QK) {  // q, k to unit length (fused input preparation)
+    if (warp < 2) {
+      const float* x = warp == 0 ? sq : sk;
+      float ss = 0.f;
+      for (int i = lane; i < DK; i += 32) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (lane == 0) snorm[warp] = rsqrtf(ss + kL2Eps);
+    }
+    __syncthreads();
+    if (tid < DK) {
+      sq[tid] *= snorm[0];
+      sk[tid] *= snorm[1];
+    }
+    __syncthreads();
+  }
 
   // 3. decay rows; partial column sums of S'^T k and S'^T q over this warp's rows
   float ak[CL], aq[CL];
@@ -133,31 +149,32 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
 
 template <typename T, int DK, int DV>
 cudaError_t launch_typed(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                         float scale, float* state, void* o, int N, int H, int gate, cudaStream_t stream) {
+                         float scale, float* state, void* o, int N, int H, int gate, int prep,
+                         cudaStream_t stream) {
   const unsigned heads = (unsigned)N * (unsigned)H;
   decode_step_kernel<T, DK, DV><<<heads, kDecodeWarps * 32, 0, stream>>>(
-      (const T*)q, (const T*)k, (const T*)v, (const T*)g, (const T*)beta, scale, state, (T*)o, gate);
+      (const T*)q, (const T*)k, (const T*)v, (const T*)g, (const T*)beta, scale, state, (T*)o, gate, prep);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_dims(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                        float scale, float* state, void* o, int N, int H, int dk, int dv, int gate,
+                        float scale, float* state, void* o, int N, int H, int dk, int dv, int gate, int prep,
                         cudaStream_t stream) {
-  if (dk == 128 && dv == 128) return launch_typed<T, 128, 128>(q, k, v, g, beta, scale, state, o, N, H, gate, stream);
-  if (dk == 128 && dv == 64) return launch_typed<T, 128, 64>(q, k, v, g, beta, scale, state, o, N, H, gate, stream);
-  if (dk == 64 && dv == 128) return launch_typed<T, 64, 128>(q, k, v, g, beta, scale, state, o, N, H, gate, stream);
-  return launch_typed<T, 64, 64>(q, k, v, g, beta, scale, state, o, N, H, gate, stream);
+  if (dk == 128 && dv == 128) return launch_typed<T, 128, 128>(q, k, v, g, beta, scale, state, o, N, H, gate, prep, stream);
+  if (dk == 128 && dv == 64) return launch_typed<T, 128, 64>(q, k, v, g, beta, scale, state, o, N, H, gate, prep, stream);
+  if (dk == 64 && dv == 128) return launch_typed<T, 64, 128>(q, k, v, g, beta, scale, state, o, N, H, gate, prep, stream);
+  return launch_typed<T, 64, 64>(q, k, v, g, beta, scale, state, o, N, H, gate, prep, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const void* g, const void* beta,
                           float scale, float* state, void* o, int N, int H, int dk, int dv, int dtype,
-                          int gate, cudaStream_t stream) {
+                          int gate, int prep, cudaStream_t stream) {
   if (dtype == KDA_F32)
-    return launch_dims<float>(q, k, v, g, beta, scale, state, o, N, H, dk, dv, gate, stream);
-  return launch_dims<__nv_bfloat16>(q, k, v, g, beta, scale, state, o, N, H, dk, dv, gate, stream);
+    return launch_dims<float>(q, k, v, g, beta, scale, state, o, N, H, dk, dv, gate, prep, stream);
+  return launch_dims<__nv_bfloat16>(q, k, v, g, beta, scale, state, o, N, H, dk, dv, gate, prep, stream);
 }
 
 }  // namespace kda

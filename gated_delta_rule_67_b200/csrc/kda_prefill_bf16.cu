@@ -203,19 +203,24 @@ __device__ __forceinline__ void store_block_frag(float* X, const float (&acc)[2]
 
 // kScalarGate: the forget gate is one log-gate per (token, head) read from
 // g_head (Gated DeltaNet), or none when g_head is null (DeltaNet); otherwise
-// the per-channel g tile comes in by TMA (KDA).
-template <bool kScalarGate>
+// the per-channel g tile comes in by TMA (KDA).  kPrep: the inputs are raw
+// and `prep` (kda_prep bits) says which ones to prepare here: q, k scaled to
+// unit length per token (the per-token factors are applied wherever q and k
+// are read), log-sigmoid of g, sigmoid of beta.
+template <bool kScalarGate, bool kPrep>
 __global__ void __launch_bounds__(kP1Threads, 3)
     kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                           const bf16* __restrict__ beta, float scale, uint8_t* __restrict__ records,
-                          WorkspaceHeader* hdr, int T, int H, int NC, const bf16* __restrict__ g_head) {
+                          WorkspaceHeader* hdr, int T, int H, int NC, const bf16* __restrict__ g_head, int prep) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t bar_in, bar_v, bar_mma;
   __shared__ uint32_t tmem_base;
   __shared__ float sbeta[kC];
   __shared__ float sgh[kScalarGate ? kC : 1];  // per-head log-gates of the chunk (zeros without a gate)
+  __shared__ float snq[kPrep ? kC : 1], snk[kPrep ? kC : 1];  // per-token sums of q^2, k^2 (fused L2 norm)
+  const bool l2n = kPrep && (prep & KDA_PREP_L2NORM_QK);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x % NC;
@@ -239,10 +244,18 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     }
   }
   if (warp == 0) tmem_alloc(&tmem_base, 128);
-  if (tid < kC) sbeta[tid] = tid < L ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
+  if (tid < kC) {
+    const float x = tid < L ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
+    sbeta[tid] = (kPrep && tid < L) ? prep_beta(prep, x) : x;
+  }
   if (kScalarGate && tid >= kC && tid < 2 * kC) {
     const int i = tid - kC;
-    sgh[i] = (g_head && i < L) ? __bfloat162float(g_head[((size_t)b * T + t0 + i) * H + h]) : 0.f;
+    const float x = (g_head && i < L) ? __bfloat162float(g_head[((size_t)b * T + t0 + i) * H + h]) : 0.f;
+    sgh[i] = (kPrep && g_head && i < L) ? prep_gate(prep, x) : x;
+  }
+  if (kPrep && tid >= 2 * kC && tid < 3 * kC) {
+    snq[tid - 2 * kC] = 0.f;
+    snk[tid - 2 * kC] = 0.f;
   }
   tc_fence_before();
   __syncthreads();
@@ -262,9 +275,32 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   const int tg = lane & 15;
   const int c8 = 8 * cg;
   float G[4][8], gref[8], gend[8];
+  if (l2n) {  // per-token sums of squares of q and k over the 128 channels
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int i = tg + 16 * t;
+      float q8[8], k8[8];
+      ld8(sm + kP1A + kmajor_off(kC + i, c8, 128), q8);
+      ld8(sm + kP1K + kmajor_off(i, c8, kC), k8);
+      float sq2 = 0.f, sk2 = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sq2 = fmaf(q8[e], q8[e], sq2);
+        sk2 = fmaf(k8[e], k8[e], sk2);
+      }
+      atomicAdd(&snq[i], sq2);
+      atomicAdd(&snk[i], sk2);
+    }
+  }
   if (!kScalarGate) {
 #pragma unroll
     for (int t = 0; t < 4; ++t) ld8(sm + kP1A + kmajor_off(tg + 16 * t, c8, 128), G[t]);
+    if (kPrep && (prep & KDA_PREP_GATE_LOGSIGMOID)) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) G[t][e] = tg + 16 * t < L ? log_sigmoid(G[t][e]) : 0.f;  // padding: no decay
+    }
   } else {  // one log-gate per token for every channel (zero without a gate)
 #pragma unroll
     for (int t = 0; t < 4; ++t)
@@ -318,6 +354,14 @@ __global__ void __launch_bounds__(kP1Threads, 3)
       float k8[8], q8[8];
       ld8(sm + kP1K + oK, k8);
       ld8(sm + kP1A + oQ, q8);
+      if (l2n) {
+        const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          k8[e] *= rk;
+          q8[e] *= rq;
+        }
+      }
       float ex[8], ei[8], w[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -442,8 +486,14 @@ __global__ void __launch_bounds__(kP1Threads, 3)
         while (i * (i + 1) / 2 > p) --i;
         while ((i + 1) * (i + 2) / 2 <= p) ++i;
         const int j = p - i * (i + 1) / 2;
-        a_blk(sm, blk(i >> 4, j >> 4))[bidx(i & 15, j & 15)] = j < i ? sbeta[i] * akk[t] : 0.f;
-        stbf(sm + kP1QT, kmajor_off(j, i, kC), scale * aqk[t]);
+        float fk = 1.f, fq = 1.f;  // unit-length factors of k_i k_j and q_i k_j
+        if (l2n) {
+          const float rkj = rsqrtf(snk[j] + kL2Eps);
+          fk = rsqrtf(snk[i] + kL2Eps) * rkj;
+          fq = rsqrtf(snq[i] + kL2Eps) * rkj;
+        }
+        a_blk(sm, blk(i >> 4, j >> 4))[bidx(i & 15, j & 15)] = j < i ? sbeta[i] * (akk[t] * fk) : 0.f;
+        stbf(sm + kP1QT, kmajor_off(j, i, kC), scale * (aqk[t] * fq));
       }
     }
     for (int e = tid; e < kC * kC; e += kP1Threads) {
@@ -459,6 +509,14 @@ __global__ void __launch_bounds__(kP1Threads, 3)
       float k8[8], q8[8], kp[8], qp[8], kb[8];
       ld8(sm + kP1K + oK, k8);
       ld8(sm + kP1A + oQ, q8);
+      if (l2n) {
+        const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          k8[e] *= rk;
+          q8[e] *= rq;
+        }
+      }
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float e0 = __expf(G[t][e]);
@@ -1209,17 +1267,17 @@ int prefill_bf16_launches(int B, int T, int H) {
 
 cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const bf16* beta,
                                 float scale, const float* s0, bf16* o, float* sT, int B, int T, int H, int dk,
-                                int dv, int chunk, int gate, void* ws, size_t ws_bytes, cudaStream_t stream,
-                                void* const* events) {
+                                int dv, int chunk, int gate, int prep, void* ws, size_t ws_bytes,
+                                cudaStream_t stream, void* const* events) {
   (void)dk, (void)dv, (void)chunk, (void)ws_bytes;
   static bool attrs_set = false;
   if (!attrs_set) {
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_prep_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kP1Bytes + 1024);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_chunk_prep_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kP1Bytes + 1024);
-    if (e != cudaSuccess) return e;
+    for (auto kern : {kda_chunk_prep_kernel<false, false>, kda_chunk_prep_kernel<true, false>,
+                      kda_chunk_prep_kernel<false, true>, kda_chunk_prep_kernel<true, true>}) {
+      const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kP1Bytes + 1024);
+      if (e != cudaSuccess) return e;
+    }
+    cudaError_t e;
     e = cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kP2Bytes + 1024);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
@@ -1238,12 +1296,13 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   if (e == cudaSuccess) e = cudaMemsetAsync(hdr, 0, sizeof(WorkspaceHeader), stream);
   if (e != cudaSuccess) return e;
   const unsigned tiles = (unsigned)((size_t)B * H * NC);
-  if (gate == KDA_GATE_CHANNEL)
-    kda_chunk_prep_kernel<false><<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records,
-                                                                               hdr, T, H, NC, nullptr);
-  else
-    kda_chunk_prep_kernel<true><<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(
-        mq, mk, mv, mg, beta, scale, records, hdr, T, H, NC, gate == KDA_GATE_HEAD ? g : nullptr);
+  {
+    const bool scalar = gate != KDA_GATE_CHANNEL;
+    const bf16* gh = gate == KDA_GATE_HEAD ? g : nullptr;
+    auto kern = scalar ? (prep ? kda_chunk_prep_kernel<true, true> : kda_chunk_prep_kernel<true, false>)
+                       : (prep ? kda_chunk_prep_kernel<false, true> : kda_chunk_prep_kernel<false, false>);
+    kern<<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records, hdr, T, H, NC, gh, prep);
+  }
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e != cudaSuccess) return e;

@@ -25,7 +25,7 @@ __global__ void __launch_bounds__(kCols * kGroups)
     prefill_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                        const float* __restrict__ v, const float* __restrict__ g,
                        const float* __restrict__ beta, float scale, const float* __restrict__ s0,
-                       float* __restrict__ o, float* sT, int T, int H, int DV, int gate) {
+                       float* __restrict__ o, float* sT, int T, int H, int DV, int gate, int prep) {
   constexpr int RW = DK / kGroups;
   __shared__ float sq[kTile][DK], sk[kTile][DK], sa[kTile][DK];
   __shared__ float sv[kTile][kCols], sb[kTile];
@@ -49,14 +49,37 @@ __global__ void __launch_bounds__(kCols * kGroups)
       const size_t tok = ((size_t)b * T + t0 + tt) * H + h, off = tok * DK + c;
       sq[tt][c] = q[off];
       sk[tt][c] = k[off];
-      sa[tt][c] = gate_alpha(gate, g + tok * DK, g + tok, c);
+      sa[tt][c] = gate_alpha(gate, prep, g + tok * DK, g + tok, c);
     }
     for (int e = tid; e < nt * kCols; e += blockDim.x) {
       const int tt = e / kCols, c = e % kCols;
       sv[tt][c] = v[(((size_t)b * T + t0 + tt) * H + h) * DV + blockIdx.x * kCols + c];
     }
-    if (tid < nt) sb[tid] = beta[((size_t)b * T + t0 + tid) * H + h];
+    if (tid < nt) sb[tid] = prep_beta(prep, beta[((size_t)b * T + t0 + tid) * H + h]);
     __syncthreads();
+    if (prep & KDA_PREP_L2NORM_QK) {  // q, k of each staged token to unit length: 8 threads per token
+      static_assert(kCols * kGroups == 8 * kTile, "8 threads per staged token");
+      const int tt = tid >> 3, part = tid & 7;
+      constexpr int PW = DK / 8;
+      float qs = 0.f, ks = 0.f;
+#pragma unroll
+      for (int c = 0; c < PW; ++c) {
+        qs = fmaf(sq[tt][part * PW + c], sq[tt][part * PW + c], qs);
+        ks = fmaf(sk[tt][part * PW + c], sk[tt][part * PW + c], ks);
+      }
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1) {
+        qs += __shfl_xor_sync(0xffffffffu, qs, off);
+        ks += __shfl_xor_sync(0xffffffffu, ks, off);
+      }
+      const float rq = rsqrtf(qs + kL2Eps), rk = rsqrtf(ks + kL2Eps);
+#pragma unroll
+      for (int c = 0; c < PW; ++c) {
+        sq[tt][part * PW + c] *= rq;
+        sk[tt][part * PW + c] *= rk;
+      }
+      __syncthreads();
+    }
 
     for (int tt = 0; tt < nt; ++tt) {
       float pk = 0.f;
@@ -91,16 +114,16 @@ __global__ void __launch_bounds__(kCols * kGroups)
 
 cudaError_t launch_prefill_f32(const float* q, const float* k, const float* v, const float* g,
                                const float* beta, float scale, const float* s0, float* o, float* sT,
-                               int B, int T, int H, int dk, int dv, int chunk, int gate, cudaStream_t stream,
-                               void* const* events) {
+                               int B, int T, int H, int dk, int dv, int chunk, int gate, int prep,
+                               cudaStream_t stream, void* const* events) {
   (void)chunk;
   dim3 grid(dv / kCols, H, B);
   cudaError_t e = mark(events, 0, stream);
   if (e != cudaSuccess) return e;
   if (dk == 128)
-    prefill_f32_kernel<128><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv, gate);
+    prefill_f32_kernel<128><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv, gate, prep);
   else
-    prefill_f32_kernel<64><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv, gate);
+    prefill_f32_kernel<64><<<grid, kCols * kGroups, 0, stream>>>(q, k, v, g, beta, scale, s0, o, sT, T, H, dv, gate, prep);
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e == cudaSuccess) e = mark(events, 2, stream);

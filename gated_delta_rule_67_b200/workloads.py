@@ -110,6 +110,8 @@ def _draw(kind: str, shape, seq_axis: int, dtype, gen, device) -> torch.Tensor:
             x = torch.sigmoid(x)
         elif kind == "gate":
             x = F.logsigmoid(x + 3.0)
+        elif kind == "gate_raw":
+            x = x + 3.0
         out.narrow(seq_axis, r0, r1 - r0).copy_(x.to(dtype))
     return out
 
@@ -146,8 +148,26 @@ def make_decode_inputs(steps, N, H, dk, dv, dtype=torch.bfloat16, s0_std=0.1, se
     return dict(q=q, k=k, v=v, g=g, beta=beta, state=state)
 
 
-def make_head_gates(lead_shape, seq_axis, dtype=torch.bfloat16, seed=0, device="cpu"):
+def make_head_gates(lead_shape, seq_axis, dtype=torch.bfloat16, seed=0, device="cpu", raw=False):
     """Seeded per-head log-gates for the Gated DeltaNet form: one
-    logsigmoid(N(3, 1)) value per (token, head), shape ``lead_shape`` (e.g.
-    [B, T, H] or [steps, N, H]), drawn from its own generator."""
-    return _draw("gate", tuple(lead_shape), seq_axis, dtype, _gen(seed, device), device)
+    logsigmoid(N(3, 1)) value per (token, head) (``raw``: the N(3, 1) value
+    before its log-sigmoid), shape ``lead_shape`` (e.g. [B, T, H] or
+    [steps, N, H]), drawn from its own generator."""
+    return _draw("gate_raw" if raw else "gate", tuple(lead_shape), seq_axis, dtype, _gen(seed, device), device)
+
+
+def make_raw_prefill_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, s0_std=0.1, seed=0, device="cpu"):
+    """Seeded raw projections for the fused input preparation: q, k, v ~ N(0, 1)
+    (not normalised), beta ~ N(0, 1) before its sigmoid, g ~ N(3, 1) per key
+    channel before its log-sigmoid (so prepared, they follow the same
+    distributions as make_prefill_inputs)."""
+    gen = _gen(seed, device)
+    q = _draw("normal", (B, T, H, dk), 1, dtype, gen, device)
+    k = _draw("normal", (B, T, H, dk), 1, dtype, gen, device)
+    v = _draw("normal", (B, T, H, dv), 1, dtype, gen, device)
+    beta = _draw("normal", (B, T, H), 1, dtype, gen, device)
+    g = _draw("gate_raw", (B, T, H, dk), 1, dtype, gen, device)
+    s0 = None
+    if s0_std > 0:
+        s0 = torch.randn((B, H, dk, dv), generator=gen, device=device, dtype=torch.float32) * s0_std
+    return dict(q=q, k=k, v=v, g=g, beta=beta, initial_state=s0)

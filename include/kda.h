@@ -68,6 +68,23 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
  */
 typedef enum { KDA_GATE_CHANNEL = 0, KDA_GATE_HEAD = 1, KDA_GATE_NONE = 2 } kda_gate;
 
+/*
+ * Input preparation fused into the kernels (argument `prep` of the *_ex entry
+ * points, a bit set; 0 = inputs already prepared).  The pages give no formula
+ * for these steps; they are the transforms that turn raw projections into the
+ * operator's inputs (unit-norm keys and queries, a log-gate <= 0, a write
+ * strength in (0, 1)), evaluated in fp32 inside the kernels:
+ *   KDA_PREP_L2NORM_QK       q <- q (sum_c q_c^2 + 1e-6)^-1/2, same for k, per token and head
+ *   KDA_PREP_GATE_LOGSIGMOID g <- log sigmoid(g) = min(g, 0) - log(1 + exp(-|g|))
+ *   KDA_PREP_BETA_SIGMOID    beta <- 1 / (1 + exp(-beta))
+ */
+typedef enum {
+  KDA_PREP_NONE = 0,
+  KDA_PREP_L2NORM_QK = 1,
+  KDA_PREP_GATE_LOGSIGMOID = 2,
+  KDA_PREP_BETA_SIGMOID = 4
+} kda_prep;
+
 /* Human-readable name of a status code (static storage, never NULL). */
 KDA_API const char* kda_status_string(int status);
 
@@ -125,17 +142,20 @@ KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, co
                          size_t workspace_bytes, void* stream);
 
 /*
- * kda_chunk_fwd with the forget gate of `gate` (kda_gate): KDA_GATE_CHANNEL
- * is kda_chunk_fwd itself; KDA_GATE_HEAD takes g as [B, T, H] (dtype,
- * element alignment like beta); KDA_GATE_NONE ignores g (NULL allowed).  The
- * workspace size is the same for every gate.  Other arguments, supported
- * shapes, checks and errors as kda_chunk_fwd; an unknown gate is
- * KDA_ERR_INVALID_ARG.
+ * kda_chunk_fwd with a choice of forget gate and fused input preparation.
+ * `gate` (kda_gate): KDA_GATE_CHANNEL is kda_chunk_fwd's g [B, T, H, dk];
+ * KDA_GATE_HEAD takes g as [B, T, H] (dtype, element alignment like beta);
+ * KDA_GATE_NONE ignores g (NULL allowed).  `prep` (kda_prep bits): the
+ * inputs q, k, g, beta are raw and prepared in-kernel as listed there.  The
+ * workspace size is the same for every gate and prep.  Other arguments,
+ * supported shapes, checks and errors as kda_chunk_fwd; an unknown gate or
+ * prep bit is KDA_ERR_INVALID_ARG.  kda_chunk_fwd(...) equals
+ * kda_chunk_fwd_ex(..., KDA_GATE_CHANNEL, KDA_PREP_NONE, ...).
  */
-KDA_API kda_status kda_chunk_fwd_gate(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                                      float scale, const float* initial_state, void* o, float* final_state, int B,
-                                      int T, int H, int dk, int dv, int chunk, int dtype, int gate, void* workspace,
-                                      size_t workspace_bytes, void* stream);
+KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                    float scale, const float* initial_state, void* o, float* final_state, int B,
+                                    int T, int H, int dk, int dv, int chunk, int dtype, int gate, int prep,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * kda_chunk_fwd with timing marks for measurement: `events` points to three
@@ -206,13 +226,14 @@ KDA_API kda_status kda_recurrent_step(const void* q, const void* k, const void* 
                               int dk, int dv, int dtype, void* stream);
 
 /*
- * kda_recurrent_step with the forget gate of `gate` (kda_gate): g is [N, H, dk]
- * for KDA_GATE_CHANNEL, [N, H] for KDA_GATE_HEAD (element alignment), and
- * ignored (NULL allowed) for KDA_GATE_NONE.  Otherwise as kda_recurrent_step.
+ * kda_recurrent_step with a choice of forget gate (kda_gate: g is [N, H, dk]
+ * for KDA_GATE_CHANNEL, [N, H] for KDA_GATE_HEAD with element alignment, and
+ * ignored, NULL allowed, for KDA_GATE_NONE) and fused input preparation
+ * (kda_prep bits, as for kda_chunk_fwd_ex).  Otherwise as kda_recurrent_step.
  */
-KDA_API kda_status kda_recurrent_step_gate(const void* q, const void* k, const void* v, const void* g,
-                                           const void* beta, float scale, float* state, void* o, int N, int H,
-                                           int dk, int dv, int dtype, int gate, void* stream);
+KDA_API kda_status kda_recurrent_step_ex(const void* q, const void* k, const void* v, const void* g,
+                                         const void* beta, float scale, float* state, void* o, int N, int H,
+                                         int dk, int dv, int dtype, int gate, int prep, void* stream);
 
 #ifdef __cplusplus
 }

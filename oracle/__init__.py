@@ -9,7 +9,10 @@ Pins (tests/test_oracle_pins.py) tie it to facts other than itself: the
 gated/plain linear-attention closed form, dense brute-force products of the
 transition matrices on T <= 8, exact retrieval under the delta rule, the
 DeltaNet and Gated DeltaNet special cases, boundedness, and hand-derived
-worked examples under tests/golden/.
+worked examples under tests/golden/.  ``prepare_inputs`` (fused input
+preparation: unit-length q and k, log-sigmoid gates, sigmoid write
+strengths) is pinned in tests/test_oracle_prep.py against closed forms and
+a second formula for each step.
 """
 from __future__ import annotations
 
@@ -112,3 +115,28 @@ def kda_decode(q, k, v, g, beta, scale, state, nthreads=0):
     tr = lambda x: np.ascontiguousarray(np.swapaxes(x, 0, 1))
     o, sT = kda_forward(tr(q), tr(k), tr(v), tr(g), tr(beta), scale, state, nthreads=nthreads)
     return np.ascontiguousarray(np.swapaxes(o, 0, 1)), sT
+
+
+# Fused input preparation (kda_prep bits of the C ABI).  The pages give no
+# formula for these steps; they are the transforms that make raw projections
+# into the operator's inputs (unit-length q and k, log-gates <= 0, write
+# strengths in (0, 1)), written out in fp64 from their definitions.
+PREP_L2NORM_QK, PREP_GATE_LOGSIGMOID, PREP_BETA_SIGMOID = 1, 2, 4
+L2_EPS = 1e-6
+
+
+def prepare_inputs(q, k, g, beta, prep):
+    """(q, k, g, beta) in fp64 after the preparation steps selected by ``prep``:
+    q <- q / sqrt(sum_c q_c^2 + 1e-6) (same for k) per token and head,
+    g <- log sigmoid(g) = min(g, 0) - log(1 + exp(-|g|)), beta <- 1 / (1 + exp(-beta)).
+    g may be None (no gate)."""
+    q, k, beta = _as_f64(q), _as_f64(k), _as_f64(beta)
+    g = None if g is None else _as_f64(g)
+    if prep & PREP_L2NORM_QK:
+        q = q / np.sqrt(np.sum(q * q, axis=-1, keepdims=True) + L2_EPS)
+        k = k / np.sqrt(np.sum(k * k, axis=-1, keepdims=True) + L2_EPS)
+    if prep & PREP_GATE_LOGSIGMOID and g is not None:
+        g = np.minimum(g, 0.0) - np.log1p(np.exp(-np.abs(g)))
+    if prep & PREP_BETA_SIGMOID:
+        beta = 1.0 / (1.0 + np.exp(-beta))
+    return q, k, g, beta

@@ -126,16 +126,17 @@ def test_launch_count(lib):
     assert f(1, 64, 1, 128, 128, 64, 7) == -1
 
 
-def _fwd_gate(lib, gate, g=A + (3 << 30), dtype=1, **kw):
+def _fwd_gate(lib, gate, g=A + (3 << 30), dtype=1, prep=0, **kw):
     a = dict(q=A, k=A + (1 << 30), v=A + (2 << 30), beta=A + (4 << 30), o=A + (5 << 30), B=1, T=64, H=1, dk=128,
              dv=128, chunk=64)
     a.update(kw)
-    return lib.kda_chunk_fwd_gate(a["q"], a["k"], a["v"], g, a["beta"], 1.0, None, a["o"], None, a["B"], a["T"],
-                                  a["H"], a["dk"], a["dv"], a["chunk"], dtype, gate, None, 0, None)
+    return lib.kda_chunk_fwd_ex(a["q"], a["k"], a["v"], g, a["beta"], 1.0, None, a["o"], None, a["B"], a["T"],
+                                a["H"], a["dk"], a["dv"], a["chunk"], dtype, gate, prep, None, 0, None)
 
 
 def test_chunk_fwd_gate_validation(lib):
     assert _fwd_gate(lib, 3) == binding.KDA_ERR_INVALID_ARG                   # unknown gate
+    assert _fwd_gate(lib, 0, prep=8) == binding.KDA_ERR_INVALID_ARG           # unknown prep bit
     assert _fwd_gate(lib, 0, g=None) == binding.KDA_ERR_INVALID_ARG           # per-channel gate needs g
     assert _fwd_gate(lib, 1, g=None) == binding.KDA_ERR_INVALID_ARG           # per-head gate needs g
     assert _fwd_gate(lib, 0, g=A + (3 << 30) + 2) == binding.KDA_ERR_INVALID_ARG   # [.., dk] needs 16-B alignment
@@ -146,12 +147,13 @@ def test_chunk_fwd_gate_validation(lib):
 
 
 def test_recurrent_step_gate_validation(lib):
-    f = lib.kda_recurrent_step_gate
+    f = lib.kda_recurrent_step_ex
     args = [A, A + (1 << 30), A + (2 << 30)]
     rest = [A + (4 << 30), 1.0, A + (5 << 30), A + (6 << 30)]
-    assert f(*args, None, *rest, 4, 1, 128, 128, 1, 3, None) == binding.KDA_ERR_INVALID_ARG   # unknown gate
-    assert f(*args, None, *rest, 4, 1, 128, 128, 1, 1, None) == binding.KDA_ERR_INVALID_ARG   # per-head needs g
-    assert f(*args, None, *rest, 0, 1, 128, 128, 1, 2, None) == binding.KDA_OK                # N = 0
+    assert f(*args, None, *rest, 4, 1, 128, 128, 1, 3, 0, None) == binding.KDA_ERR_INVALID_ARG   # unknown gate
+    assert f(*args, None, *rest, 4, 1, 128, 128, 1, 2, 9, None) == binding.KDA_ERR_INVALID_ARG   # unknown prep bit
+    assert f(*args, None, *rest, 4, 1, 128, 128, 1, 1, 0, None) == binding.KDA_ERR_INVALID_ARG   # per-head needs g
+    assert f(*args, None, *rest, 0, 1, 128, 128, 1, 2, 7, None) == binding.KDA_OK                # N = 0
     bad_o = list(rest)
-    bad_o[3] = A + (3 << 30) + 8                                                           # o overlaps g [N,H]
-    assert f(*args, A + (3 << 30), *bad_o, 4, 1, 128, 128, 1, 1, None) == binding.KDA_ERR_INVALID_ARG
+    bad_o[3] = A + (3 << 30) + 8                                                              # o overlaps g [N,H]
+    assert f(*args, A + (3 << 30), *bad_o, 4, 1, 128, 128, 1, 1, 0, None) == binding.KDA_ERR_INVALID_ARG
