@@ -363,6 +363,54 @@ def run_ours(args, cfg):
                   "bytes_per_step": decode_bytes(dc.N, dc.H, dc.dk, dc.dv)}
         del y
 
+    # ---- the same workload through the scalar-gate forms and the fused input preparation
+    variants = None
+    if not args.no_variants:
+        import torch.nn.functional as F
+        from gated_delta_rule_67_b200.binding import KDA_PREP_ALL
+        from gated_delta_rule_67_b200.workloads import make_head_gates, make_raw_prefill_inputs
+        gh = make_head_gates((cfg.B, cfg.T, cfg.H), 1, cfg.torch_dtype, seed=cfg.seed + 7 + 1000 * rank, device=dev)
+        raw = make_raw_prefill_inputs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.torch_dtype, cfg.s0_std,
+                                      cfg.seed + 11 + 1000 * rank, dev)
+        rq, rk, rv, rg, rb = (raw[n] for n in names)
+        nvar = max(3, min(args.steps, 100))
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            ts = []
+            for _ in range(nvar):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+            us = 1e3 * reduce_max(statistics.median(ts), dev)
+            return {"us_per_call": us, "tokens_per_s": weak_scaling_value(tokens, world, us / 1e6), "calls": nvar}
+
+        def unfused():  # the same preparation as separate PyTorch ops ahead of the call (comparison only)
+            qn = (rq.float() * torch.rsqrt((rq.float() ** 2).sum(-1, keepdim=True) + 1e-6)).to(rq.dtype)
+            kn = (rk.float() * torch.rsqrt((rk.float() ** 2).sum(-1, keepdim=True) + 1e-6)).to(rk.dtype)
+            kda_chunk_fwd(qn, kn, rv, F.logsigmoid(rg.float()).to(rg.dtype), torch.sigmoid(rb.float()).to(rb.dtype),
+                          cfg.scale, s0, chunk=cfg.chunk, o=o, final_state=sT, workspace=ws)
+
+        variants = {
+            "gated_deltanet_head_gate": timed(lambda: kda_chunk_fwd(ins[0], ins[1], ins[2], gh, ins[4], cfg.scale, s0,
+                                                                    chunk=cfg.chunk, o=o, final_state=sT,
+                                                                    workspace=ws)),
+            "deltanet_no_gate": timed(lambda: kda_chunk_fwd(ins[0], ins[1], ins[2], None, ins[4], cfg.scale, s0,
+                                                            chunk=cfg.chunk, o=o, final_state=sT, workspace=ws)),
+            "fused_input_prep": timed(lambda: kda_chunk_fwd(rq, rk, rv, rg, rb, cfg.scale, s0, chunk=cfg.chunk, o=o,
+                                                            final_state=sT, workspace=ws, prep=KDA_PREP_ALL)),
+            "unfused_prep_torch_then_call": timed(unfused),
+            "note": "same workload and timing rules as the headline; raw inputs ~ N(0,1) (q, k, v, beta), "
+                    "N(3,1) (g) before preparation; the unfused line runs the preparation as PyTorch ops "
+                    "before the call, for comparison only",
+        }
+        del raw, gh
+
     # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -382,7 +430,7 @@ def run_ours(args, cfg):
                        "parallelism": f"dp{world}: independent sequences per GPU, no collective"},
             "tflops": tflops, "tflops_frac_bf16": tflops / peaks["bf16_tflops"],
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks, "decode": decode,
+            "clocks": clocks, "decode": decode, "variants": variants,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -401,6 +449,7 @@ def main(argv=None):
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true", help="skip the gate-variant / fused-prep timings")
     ap.add_argument("--cpu-tokens", type=int, default=4096)
     args = ap.parse_args(argv)
     if args.warmup < 3:

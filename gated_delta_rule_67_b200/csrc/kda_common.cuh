@@ -49,6 +49,8 @@ constexpr int kPrepMask = KDA_PREP_L2NORM_QK | KDA_PREP_GATE_LOGSIGMOID | KDA_PR
 constexpr float kL2Eps = 1e-6f;  // q <- q (sum q^2 + kL2Eps)^-1/2
 __device__ __forceinline__ float log_sigmoid(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
 __device__ __forceinline__ float sigmoidf(float x) { return 1.f / (1.f + expf(-x)); }
+// Same with the fast exp/log intrinsics (absolute error ~1e-7; for bf16 inputs).
+__device__ __forceinline__ float log_sigmoid_fast(float x) { return fminf(x, 0.f) - __logf(1.f + __expf(-fabsf(x))); }
 __device__ __forceinline__ float prep_gate(int prep, float g) {
   return (prep & KDA_PREP_GATE_LOGSIGMOID) ? log_sigmoid(g) : g;
 }

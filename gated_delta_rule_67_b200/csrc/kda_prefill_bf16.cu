@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
 #pragma unroll
       for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) G[t][e] = tg + 16 * t < L ? log_sigmoid(G[t][e]) : 0.f;  // padding: no decay
+        for (int e = 0; e < 8; ++e) G[t][e] = tg + 16 * t < L ? log_sigmoid_fast(G[t][e]) : 0.f;  // padding: no decay
     }
   } else {  // one log-gate per token for every channel (zero without a gate)
 #pragma unroll
