@@ -15,8 +15,9 @@
  *
  * with S_t a d_k x d_v matrix (row index = key channel, column index = value
  * channel), a_t = exp(g_t) the per-channel forget gate acting on the ROWS of
- * the state (same section: "different forgetting rates to different rows of
- * the state matrix"), and beta_t a scalar write strength per token and head.
+ * the state (the same section gives each row of the state, one latent
+ * feature per key channel, its own forgetting rate), and beta_t a scalar
+ * write strength per token and head.
  * Readings taken where the page is silent or garbled (each also listed in the
  * design notes):
  *   - orientation: the page writes the write term as v k^T but left-multiplies
