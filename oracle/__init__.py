@@ -50,6 +50,8 @@ def bind(path: str):
     lib.kda_oracle_forward.restype = ctypes.c_int
     lib.kda_oracle_max_threads.argtypes = []
     lib.kda_oracle_max_threads.restype = ctypes.c_int
+    lib.kda_oracle_backward.argtypes = [dp] * 5 + [ctypes.c_double] + [dp] * 9 + [ctypes.c_int] * 6
+    lib.kda_oracle_backward.restype = ctypes.c_int
     return lib
 
 
@@ -140,3 +142,25 @@ def prepare_inputs(q, k, g, beta, prep):
     if prep & PREP_BETA_SIGMOID:
         beta = 1.0 / (1.0 + np.exp(-beta))
     return q, k, g, beta
+
+
+def kda_backward(q, k, v, g, beta, scale, initial_state, d_o, d_final_state=None, nthreads=0, lib=None):
+    """fp64 gradients of a loss through kda_forward, given dL/do [B,T,H,dv] and
+    dL/dS_T [B,H,dk,dv] (None: zero).  Returns a dict with dq, dk, dv, dg
+    (per key channel), dbeta and dS0 (fp64 numpy arrays, the inputs' layouts).
+    Reverse-mode differentiation of the token-by-token recurrence, column by
+    column of the state (kda_oracle.c, kda_oracle_backward)."""
+    lib = lib or _load()
+    q, k, v, g, beta, d_o = (_as_f64(x) for x in (q, k, v, g, beta, d_o))
+    s0, dsT = _as_f64(initial_state), _as_f64(d_final_state)
+    B, T, H, nk = q.shape
+    nv = v.shape[-1]
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v), dg=np.zeros_like(g),
+               dbeta=np.zeros_like(beta), dS0=np.zeros((B, H, nk, nv)))
+    rc = lib.kda_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(s0),
+                                 _ptr(d_o), _ptr(dsT), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                 _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, nk, nv,
+                                 int(nthreads))
+    if rc != 0:
+        raise ValueError("kda_oracle_backward rejected its arguments")
+    return out

@@ -152,3 +152,107 @@ int kda_oracle_max_threads(void) {
   return 1;
 #endif
 }
+
+/*
+ * Backward pass: the gradients of a scalar loss L through the recurrence
+ * above, given dL/do (dO, [B,T,H,dv]) and dL/dS_T (dST, [B,H,dk,dv] or NULL
+ * for zero).  Outputs, in the layouts of the inputs: dq, dk, dg ([B,T,H,dk]),
+ * dv ([B,T,H,dv]), dbeta ([B,T,H]) and dS0 = dL/dS_0 ([B,H,dk,dv]).
+ *
+ * Reverse-mode differentiation of the sequential form, one state column j at
+ * a time (a column of S evolves on its own: s' = a_t .* s, w = v_t[j] - s'.k_t,
+ * u = beta_t w, s = s' + k_t u, o_t[j] = scale s.q_t).  With G = dL/dS_t[:, j],
+ * starting from dST[:, j], for t = T-1 .. 0:
+ *   G += scale q_t dO_t[j];   dq_t += scale s_t dO_t[j]          (o_t reads S_t)
+ *   du = G.k_t;   dk_t += G u;   dv_t[j] = beta_t du;   dbeta_t += du w
+ *   G -= beta_t k_t du;   dk_t -= beta_t s'_t du                   (G = dL/dS'_t)
+ *   dg_t += G .* s'_t                 (dL/da_t .* a_t, since s' = a_t .* s_{t-1})
+ *   G = a_t .* G                                                   (dL/dS_{t-1})
+ * and dS0[:, j] = G.  The per-token sums over j (dq, dk, dg, dbeta) collect
+ * over the columns of one (b, h) in column order.
+ */
+static void oracle_chain_bwd(const double* q, const double* k, const double* v, const double* g,
+                             const double* beta, double scale, const double* s0, const double* dO,
+                             const double* dST, double* dq, double* dk, double* dvv, double* dg,
+                             double* dbeta, double* dS0, int b, int h, int T, int H, int nk, int nv) {
+  double* sp = (double*)malloc(sizeof(double) * ((size_t)T * nk + 1));  /* s'_t, all t */
+  double* w = (double*)malloc(sizeof(double) * ((size_t)T + 1));
+  double* s = (double*)malloc(sizeof(double) * (size_t)nk);
+  double* G = (double*)malloc(sizeof(double) * (size_t)nk);
+  const size_t st0 = ((size_t)b * H + h) * nk * nv;
+  for (int t = 0; t < T; ++t) {  /* zero this (b, h)'s per-token sums */
+    const size_t tok = ((size_t)b * T + t) * H + h;
+    for (int i = 0; i < nk; ++i) dq[tok * nk + i] = dk[tok * nk + i] = dg[tok * nk + i] = 0.0;
+    dbeta[tok] = 0.0;
+  }
+  for (int j = 0; j < nv; ++j) {
+    /* forward over column j, keeping s'_t and w_t */
+    for (int i = 0; i < nk; ++i) s[i] = s0 ? s0[st0 + (size_t)i * nv + j] : 0.0;
+    for (int t = 0; t < T; ++t) {
+      const size_t tok = ((size_t)b * T + t) * H + h;
+      const double* kt = k + tok * nk;
+      const double* gt = g + tok * nk;
+      double* spt = sp + (size_t)t * nk;
+      double pred = 0.0;
+      for (int i = 0; i < nk; ++i) {
+        spt[i] = exp(gt[i]) * s[i];
+        pred += spt[i] * kt[i];
+      }
+      w[t] = v[tok * nv + j] - pred;
+      const double u = beta[tok] * w[t];
+      for (int i = 0; i < nk; ++i) s[i] = spt[i] + kt[i] * u;
+    }
+    /* reverse */
+    for (int i = 0; i < nk; ++i) G[i] = dST ? dST[st0 + (size_t)i * nv + j] : 0.0;
+    for (int t = T - 1; t >= 0; --t) {
+      const size_t tok = ((size_t)b * T + t) * H + h;
+      const double* qt = q + tok * nk;
+      const double* kt = k + tok * nk;
+      const double* gt = g + tok * nk;
+      const double* spt = sp + (size_t)t * nk;
+      const double bt = beta[tok], u = bt * w[t], dot = dO[tok * nv + j];
+      double du = 0.0;
+      for (int i = 0; i < nk; ++i) {
+        const double st = spt[i] + kt[i] * u;           /* S_t[i][j] */
+        G[i] += scale * qt[i] * dot;
+        dq[tok * nk + i] += scale * st * dot;
+        du += G[i] * kt[i];
+      }
+      dvv[tok * nv + j] = bt * du;
+      dbeta[tok] += du * w[t];
+      for (int i = 0; i < nk; ++i) {
+        dk[tok * nk + i] += G[i] * u - bt * spt[i] * du;
+        G[i] -= bt * kt[i] * du;
+        dg[tok * nk + i] += G[i] * spt[i];
+        G[i] *= exp(gt[i]);
+      }
+    }
+    if (dS0)
+      for (int i = 0; i < nk; ++i) dS0[st0 + (size_t)i * nv + j] = G[i];
+  }
+  free(sp);
+  free(w);
+  free(s);
+  free(G);
+}
+
+/* Backward over all (b, h) (OpenMP over them).  0 on success, -1 on a bad argument. */
+int kda_oracle_backward(const double* q, const double* k, const double* v, const double* g,
+                        const double* beta, double scale, const double* s0, const double* dO,
+                        const double* dST, double* dq, double* dk, double* dv_out, double* dg,
+                        double* dbeta, double* dS0, int B, int T, int H, int nk, int nv, int nthreads) {
+  if (B < 0 || T < 0 || H < 0 || nk <= 0 || nv <= 0) return -1;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !dO || !dq || !dk || !dv_out || !dg || !dbeta)) return -1;
+  const long total = (long)B * H;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long wk = 0; wk < total; ++wk) {
+    const int h = (int)(wk % H), b = (int)(wk / H);
+    oracle_chain_bwd(q, k, v, g, beta, scale, s0, dO, dST, dq, dk, dv_out, dg, dbeta, dS0, b, h, T, H, nk, nv);
+  }
+  return 0;
+}
