@@ -34,6 +34,8 @@ SIGNATURES = {
     "kda_recurrent_step": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 5 + [_vp]),
     "kda_chunk_fwd_ex": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 9 + [_vp, _sz, _vp]),
     "kda_recurrent_step_ex": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 7 + [_vp]),
+    "kda_backward_workspace_size": (_sz, [_i] * 6),
+    "kda_backward": (_i, [_vp] * 5 + [_f] + [_vp] * 9 + [_i] * 7 + [_vp, _sz, _vp]),
 }
 
 # kda_gate: how the forget gate enters the update (see include/kda.h)
@@ -265,3 +267,48 @@ def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=No
     if st != KDA_OK:
         raise KDAError(st, "kda_recurrent_step")
     return o
+
+
+def kda_backward(q, k, v, g, beta, grad_o, scale=None, initial_state=None, grad_final_state=None, *,
+                 workspace=None, stream=None, want_initial_state_grad=True):
+    """Gradients of a loss through kda_chunk_fwd (prepared inputs; g per key
+    channel [B,T,H,dk], per head [B,T,H] or None, as for the forward), given
+    grad_o = dL/do [B,T,H,dv] and grad_final_state = dL/dS_T [B,H,dk,dv] fp32 (or None).
+
+    Returns a dict: dq, dk, dv, dg (like g; None without a gate), dbeta (input
+    dtype) and dS0 = dL/dS_0 fp32 (None if not wanted).
+    """
+    lib = load()
+    for name, x in (("q", q), ("k", k), ("v", v), ("beta", beta), ("grad_o", grad_o)):
+        _check_dev(name, x, q.dtype)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    gate = _gate_kind(g, (B, T, H))
+    if g is not None:
+        _check_dev("g", g, q.dtype)
+    if k.shape != q.shape or (gate == KDA_GATE_CHANNEL and g.shape != q.shape) or v.shape[:3] != (B, T, H) \
+            or beta.shape != (B, T, H) or grad_o.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, g, beta, grad_o")
+    if scale is None:
+        scale = dk ** -0.5
+    for name, x in (("initial_state", initial_state), ("grad_final_state", grad_final_state)):
+        if x is not None:
+            _check_dev(name, x, torch.float32)
+            if x.shape != (B, H, dk, dv):
+                raise ValueError(f"{name} must be [B,H,dk,dv]")
+    code = _dtype_code(q.dtype)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dg=None if g is None else torch.empty_like(g), dbeta=torch.empty_like(beta),
+               dS0=torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_initial_state_grad
+               else None)
+    need = int(lib.kda_backward_workspace_size(B, T, H, dk, dv, code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
+                          _ptr(grad_o), _ptr(grad_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                          _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, dk, dv, code, gate,
+                          _ptr(workspace), ws_bytes, _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_backward")
+    return out

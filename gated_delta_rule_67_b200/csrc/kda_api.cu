@@ -183,6 +183,72 @@ kda_status kda_wait_selftest(void* workspace, size_t workspace_bytes, void* stre
   return from_cuda(kda::launch_wait_selftest(workspace, static_cast<cudaStream_t>(stream_)));
 }
 
+size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, int dtype) {
+  if (B < 0 || T < 0 || H < 1) return 0;
+  if (dtype != KDA_F32 && dtype != KDA_BF16) return 0;
+  if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return 0;
+  return kda::backward_workspace_bytes(B, T, H, dk, dv);
+}
+
+kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
+                        const float* initial_state, const void* grad_o, const float* grad_final_state, void* grad_q,
+                        void* grad_k, void* grad_v, void* grad_g, void* grad_beta, float* grad_initial_state, int B,
+                        int T, int H, int dk, int dv, int dtype, int gate, void* workspace, size_t workspace_bytes,
+                        void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
+  if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
+  if (gate == KDA_GATE_NONE) g = nullptr, grad_g = nullptr;
+  const bool empty = (B == 0 || T == 0);
+  const size_t eb = elem_bytes(dtype), ntok = (size_t)B * T * H, state_bytes = (size_t)B * H * dk * dv * 4;
+  const size_t gbytes = gate == KDA_GATE_CHANNEL ? ntok * dk * eb : ntok * eb;
+  const Range rq{(const char*)q, ntok * dk * eb}, rk{(const char*)k, ntok * dk * eb},
+      rv{(const char*)v, ntok * dv * eb}, rg{(const char*)g, gbytes}, rb{(const char*)beta, ntok * eb},
+      rs0{(const char*)initial_state, state_bytes}, rdo{(const char*)grad_o, ntok * dv * eb},
+      rdsT{(const char*)grad_final_state, state_bytes};
+  const Range wq{(const char*)grad_q, ntok * dk * eb}, wk{(const char*)grad_k, ntok * dk * eb},
+      wv{(const char*)grad_v, ntok * dv * eb}, wg{(const char*)grad_g, gbytes}, wb{(const char*)grad_beta, ntok * eb},
+      ws0{(const char*)grad_initial_state, state_bytes};
+  if (!empty) {
+    const void* need[] = {q, k, v, grad_o, grad_q, grad_k, grad_v};
+    for (const void* p : need)
+      if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    for (const void* p : {beta, (const void*)grad_beta})
+      if (!p || !aligned_to(p, eb)) return KDA_ERR_INVALID_ARG;
+    if (gate == KDA_GATE_CHANNEL && (!g || !grad_g || !aligned16(g) || !aligned16(grad_g))) return KDA_ERR_INVALID_ARG;
+    if (gate == KDA_GATE_HEAD && (!g || !grad_g || !aligned_to(g, eb) || !aligned_to(grad_g, eb)))
+      return KDA_ERR_INVALID_ARG;
+  }
+  for (const void* p : {(const void*)initial_state, (const void*)grad_final_state, (const void*)grad_initial_state})
+    if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  const Range outs[] = {wq, wk, wv, wg, wb, ws0};
+  for (int i = 0; i < 6; ++i) {
+    for (Range r : {rq, rk, rv, rg, rb, rs0, rdo, rdsT})
+      if (overlaps(outs[i], r)) return KDA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 6; ++j)
+      if (overlaps(outs[i], outs[j])) return KDA_ERR_INVALID_ARG;
+  }
+  if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+  if (empty) {  // dL/dS_0 = dL/dS_T
+    cudaError_t e = cudaSuccess;
+    if (grad_initial_state && state_bytes)
+      e = grad_final_state ? cudaMemcpyAsync(grad_initial_state, grad_final_state, state_bytes,
+                                             cudaMemcpyDeviceToDevice, stream)
+                           : cudaMemsetAsync(grad_initial_state, 0, state_bytes, stream);
+    return from_cuda(e);
+  }
+  const size_t need_ws = kda::backward_workspace_bytes(B, T, H, dk, dv);
+  if (!workspace || workspace_bytes < need_ws || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
+  const Range rw{(const char*)workspace, workspace_bytes};
+  for (Range r : {rq, rk, rv, rg, rb, rs0, rdo, rdsT, wq, wk, wv, wg, wb, ws0})
+    if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
+  return from_cuda(kda::launch_backward(q, k, v, g, beta, scale, initial_state, grad_o, grad_final_state, grad_q,
+                                        grad_k, grad_v, grad_g, grad_beta, grad_initial_state, B, T, H, dk, dv, dtype,
+                                        gate, workspace, stream));
+}
+
 static kda_status recurrent_step_impl(const void* q, const void* k, const void* v, const void* g,
                                       const void* beta, float scale, float* state, void* o, int N, int H, int dk,
                                       int dv, int dtype, int gate, int prep, void* stream_) {

@@ -171,3 +171,13 @@ def make_raw_prefill_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, s0_std=0.1, s
     if s0_std > 0:
         s0 = torch.randn((B, H, dk, dv), generator=gen, device=device, dtype=torch.float32) * s0_std
     return dict(q=q, k=k, v=v, g=g, beta=beta, initial_state=s0)
+
+
+def make_cotangents(B, T, H, dk, dv, dtype=torch.bfloat16, seed=0, device="cpu", final_state=True):
+    """Seeded upstream gradients for the backward pass: dL/do ~ N(0, 1)
+    [B, T, H, dv] (dtype) and, if ``final_state``, dL/dS_T ~ N(0, 0.1^2)
+    [B, H, dk, dv] fp32 (else None)."""
+    gen = _gen(seed, device)
+    d_o = _draw("normal", (B, T, H, dv), 1, dtype, gen, device)
+    d_s = torch.randn((B, H, dk, dv), generator=gen, device=device, dtype=torch.float32) * 0.1 if final_state else None
+    return d_o, d_s

@@ -158,6 +158,47 @@ KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Bytes of device workspace kda_backward needs for this problem (fp32 state
+ * checkpoints every 16 tokens plus a 16-state scratch per (sequence, head));
+ * 0 for arguments kda_backward would reject.
+ */
+KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
+
+/*
+ * Backward pass: gradients of a scalar loss L through the forward pass
+ * (kda_chunk_fwd, or kda_chunk_fwd_ex with `gate` and KDA_PREP_NONE), given
+ * dL/do and dL/dS_T.  Reverse-mode differentiation of the token-by-token
+ * recurrence of the KimiLinear article, section 2.3 (sections 2.1-2.2 for the
+ * scalar gates), evaluated in fp32 token by token (not chunkwise).
+ *
+ *   q, k, v, g, beta, scale, initial_state : the forward's inputs (layouts
+ *                      and gate kinds as for kda_chunk_fwd_ex)
+ *   grad_o           : [B, T, H, dv] (dtype), dL/do
+ *   grad_final_state : [B, H, dk, dv] fp32 dL/dS_T, or NULL for zero
+ *   grad_q, grad_k   : [B, T, H, dk] (dtype), written
+ *   grad_v           : [B, T, H, dv] (dtype), written
+ *   grad_g           : like g ([B, T, H, dk] per channel, [B, T, H] per
+ *                      head), written; ignored (NULL allowed) for KDA_GATE_NONE
+ *   grad_beta        : [B, T, H] (dtype), written
+ *   grad_initial_state : [B, H, dk, dv] fp32 dL/dS_0, or NULL to skip
+ *   workspace        : at least kda_backward_workspace_size() bytes, 16-byte
+ *                      aligned; contents on entry do not matter
+ *
+ * Supported: dtype KDA_F32 or KDA_BF16, dk and dv in {64, 128}.  Pointers
+ * 16-byte aligned (beta, grad_beta and per-head g / grad_g: element
+ * alignment); outputs must not overlap any input, each other or the
+ * workspace.  The per-token sums over value channels are added in a fixed
+ * order, so results are bit-reproducible.  T = 0 or B = 0 is valid
+ * (grad_initial_state = grad_final_state).
+ */
+KDA_API kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                float scale, const float* initial_state, const void* grad_o,
+                                const float* grad_final_state, void* grad_q, void* grad_k, void* grad_v,
+                                void* grad_g, void* grad_beta, float* grad_initial_state, int B, int T, int H,
+                                int dk, int dv, int dtype, int gate, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
  * kda_chunk_fwd with timing marks for measurement: `events` points to three
  * cudaEvent_t handles (created by the caller) which are recorded on `stream`
  * before the first kernel, between the chunk-preparation kernel and the

@@ -157,3 +157,31 @@ def test_recurrent_step_gate_validation(lib):
     bad_o = list(rest)
     bad_o[3] = A + (3 << 30) + 8                                                              # o overlaps g [N,H]
     assert f(*args, A + (3 << 30), *bad_o, 4, 1, 128, 128, 1, 1, 0, None) == binding.KDA_ERR_INVALID_ARG
+
+
+def test_backward_validation(lib):
+    f = lib.kda_backward
+    assert lib.kda_backward_workspace_size(1, 64, 1, 128, 128, 1) > 0
+    assert lib.kda_backward_workspace_size(1, 64, 1, 96, 128, 1) == 0
+    ins = [A, A + (1 << 30), A + (2 << 30), A + (3 << 30), A + (4 << 30)]   # q k v g beta
+    grads = [A + (10 << 30), A + (11 << 30), A + (12 << 30), A + (13 << 30), A + (14 << 30)]
+
+    def call(ins=ins, grads=grads, gate=0, dk=128, dv=128, ws=A + (20 << 30), wsb=1 << 40, grad_o=A + (5 << 30)):
+        return f(*ins, 1.0, None, grad_o, None, *grads, None, 1, 64, 1, dk, dv, 1, gate, ws, wsb, None)
+
+    assert call(gate=3) == binding.KDA_ERR_INVALID_ARG
+    assert call(dk=96) == binding.KDA_ERR_UNSUPPORTED
+    assert call(ws=None) == binding.KDA_ERR_INVALID_ARG
+    assert call(wsb=16) == binding.KDA_ERR_INVALID_ARG
+    bad = list(grads)
+    bad[0] = A + 64                                                   # grad_q overlaps q
+    assert call(grads=bad) == binding.KDA_ERR_INVALID_ARG
+    bad = list(grads)
+    bad[1] = A + (10 << 30) + 256                                     # grad_k overlaps grad_q
+    assert call(grads=bad) == binding.KDA_ERR_INVALID_ARG
+    bad = list(grads)
+    bad[3] = None                                                     # per-channel gate needs grad_g
+    assert call(grads=bad) == binding.KDA_ERR_INVALID_ARG
+    assert call(grad_o=None) == binding.KDA_ERR_INVALID_ARG
+    assert f(*ins, 1.0, None, A + (5 << 30), None, *grads, None, 0, 64, 1, 128, 128, 1, 0, None, 0, None) \
+        == binding.KDA_OK                                             # B = 0 with nothing to copy

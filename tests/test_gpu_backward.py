@@ -1,0 +1,77 @@
+"""Backward pass (kda_backward) against the fp64 oracle's gradients
+(oracle.kda_backward, pinned by finite differences and autograd)."""
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_67_b200 import kda_backward
+from gated_delta_rule_67_b200.workloads import make_cotangents, make_head_gates, make_prefill_inputs
+from tests.parity import TOL, cuda_or_skip, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(B, T, H, dk, dv, dtype, gate="channel", s0=0.1, final=True, seed=90):
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(B, T, H, dk, dv, dtype, s0, seed=seed)
+    d_o, d_s = make_cotangents(B, T, H, dk, dv, dtype, seed=seed + 1, final_state=final)
+    if gate == "head":
+        g = make_head_gates((B, T, H), 1, dtype, seed=seed + 2)
+        g_or = g.unsqueeze(-1).expand_as(x["q"]).contiguous()
+    elif gate == "none":
+        g, g_or = None, torch.zeros_like(x["q"])
+    else:
+        g = g_or = x["g"]
+    scale = dk ** -0.5
+    to = lambda t: None if t is None else t.to(dev)
+    got = kda_backward(to(x["q"]), to(x["k"]), to(x["v"]), to(g), to(x["beta"]), to(d_o), scale,
+                       to(x["initial_state"]), to(d_s))
+    torch.cuda.synchronize()
+    ref = oracle.kda_backward(x["q"], x["k"], x["v"], g_or, x["beta"], scale, x["initial_state"], d_o, d_s)
+    tol = TOL[dtype]
+    for name in ("dq", "dk", "dv", "dbeta", "dS0"):
+        assert rel_err(got[name], ref[name]) < tol, (name, rel_err(got[name], ref[name]))
+    if gate == "channel":
+        assert rel_err(got["dg"], ref["dg"]) < tol, ("dg", rel_err(got["dg"], ref["dg"]))
+    elif gate == "head":
+        dgh = ref["dg"].sum(axis=-1)   # the per-head gate is broadcast over the key channels
+        assert rel_err(got["dg"], dgh) < tol, ("dg", rel_err(got["dg"], dgh))
+    else:
+        assert got["dg"] is None
+    return got
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("B,T,H,dk,dv", [(1, 37, 2, 128, 128), (2, 100, 3, 64, 64), (1, 64, 1, 128, 64),
+                                         (1, 64, 1, 64, 128), (1, 1, 1, 128, 128), (1, 16, 2, 128, 128),
+                                         (1, 17, 2, 128, 128)])
+def test_backward_shapes(dtype, B, T, H, dk, dv):
+    """Several windows and ragged tails (16-token windows, 4-token reduction
+    steps), a single token, every supported (dk, dv)."""
+    _case(B, T, H, dk, dv, dtype, seed=91 + T)
+
+
+@pytest.mark.parametrize("gate", ["head", "none"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_backward_scalar_gates(gate, dtype):
+    _case(1, 150, 2, 128, 128, dtype, gate=gate, seed=92)
+
+
+def test_backward_zero_state_and_no_final_gradient():
+    _case(2, 70, 2, 128, 128, torch.float32, s0=0.0, final=False, seed=93)
+
+
+def test_backward_bench_shape():
+    """B=1, H=16, T=4096, d=128 (bf16), random initial state, every gradient."""
+    _case(1, 4096, 16, 128, 128, torch.bfloat16, seed=94)
+
+
+def test_backward_deterministic():
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(1, 200, 2, 128, 128, torch.bfloat16, 0.1, seed=95, device=dev)
+    d_o, d_s = make_cotangents(1, 200, 2, 128, 128, torch.bfloat16, seed=96, device=dev)
+    args = (x["q"], x["k"], x["v"], x["g"], x["beta"], d_o, None, x["initial_state"], d_s)
+    a, b = kda_backward(*args), kda_backward(*args)
+    torch.cuda.synchronize()
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
