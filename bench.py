@@ -60,6 +60,13 @@ def prefill_bytes(B, T, H, dk, dv, elem=2, state_in=True, state_out=True) -> flo
     return B * T * H * per_tok + st * (int(state_in) + int(state_out))
 
 
+def backward_bytes(B, T, H, dk, dv, elem=2) -> float:
+    """Algorithmic HBM bytes of one backward call: q, k, g, v, beta, dL/do read;
+    dq, dk, dg, dv, dbeta written; S0 and dL/dS_T read, dL/dS0 written (fp32)."""
+    per_tok = ((3 * dk + 2 * dv + 1) + (3 * dk + dv + 1)) * elem
+    return B * T * H * per_tok + 3 * B * H * dk * dv * 4
+
+
 def decode_bytes(N, H, dk, dv, elem=2) -> float:
     return N * H * (2 * dk * dv * 4 + (3 * dk + 2 * dv + 1) * elem)
 
@@ -411,6 +418,37 @@ def run_ours(args, cfg):
         }
         del raw, gh
 
+    # ---- backward pass on the same workload
+    backward = None
+    if not args.no_backward:
+        from gated_delta_rule_67_b200 import kda_backward
+        from gated_delta_rule_67_b200.binding import load as load_lib
+        from gated_delta_rule_67_b200.workloads import make_cotangents
+        d_o, d_s = make_cotangents(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, cfg.torch_dtype, seed=cfg.seed + 13 + 1000 * rank,
+                                   device=dev)
+        bws = torch.empty(max(1, int(load_lib().kda_backward_workspace_size(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv,
+                                                                             1 if cfg.dtype == "bf16" else 0))),
+                          dtype=torch.uint8, device=dev)
+        bargs = (ins[0], ins[1], ins[2], ins[3], ins[4], d_o, cfg.scale, s0, d_s)
+        kda_backward(*bargs, workspace=bws)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.backward_calls):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            kda_backward(*bargs, workspace=bws)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        bs = reduce_max(statistics.median(ts) / 1e3, dev)
+        bbytes = backward_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, 2 if cfg.dtype == "bf16" else 4)
+        backward = {"us_per_call": bs * 1e6, "tokens_per_s": weak_scaling_value(tokens, world, bs),
+                    "calls": args.backward_calls, "algorithmic_bytes": bbytes,
+                    "achieved_gbs": bbytes / bs / 1e9, "frac_hbm": bbytes / bs / 1e9 / peaks["hbm_gbs"],
+                    "kernel": "kda_backward_kernel (token-recurrent fp32; column-split partials + fixed-order sum)"}
+        del bws, d_o, d_s
+
     # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -430,7 +468,7 @@ def run_ours(args, cfg):
                        "parallelism": f"dp{world}: independent sequences per GPU, no collective"},
             "tflops": tflops, "tflops_frac_bf16": tflops / peaks["bf16_tflops"],
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks, "decode": decode, "variants": variants,
+            "clocks": clocks, "decode": decode, "variants": variants, "backward": backward,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -450,6 +488,8 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true", help="skip the gate-variant / fused-prep timings")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
+    ap.add_argument("--backward-calls", type=int, default=5)
     ap.add_argument("--cpu-tokens", type=int, default=4096)
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -80,16 +80,22 @@ struct BwdArgs {
   const float *s0, *dsT;
   void *dq, *dk, *dv, *dg, *dbeta;
   float* ds0;
-  float* ckpt;     // [B*H][NCK] states of DK*DV floats, in the per-warp layout of st_tile_ws
-  float* scratch;  // [B*H][kCk] decayed states, same layout
+  float* ckpt;     // [CTA][NCK] state tiles of the CTA's columns, in the per-warp layout of st_tile_ws
+  float* scratch;  // [CTA][kCk] decayed-state tiles, same layout
+  float* part;     // split CTAs: fp32 partial dq, dk, dg [3][nsplit][tokens][DK]
+  float* partb;    // split CTAs: fp32 partial dbeta, per-head dg [2][nsplit][tokens]
   float scale;
   int T, H, gate;
 };
 
-template <typename IO, int DK, int DV>
-__global__ void __launch_bounds__(DV / kColsW * 32, 1) kda_backward_kernel(const BwdArgs a) {
-  constexpr int RW = DK / 32, NW = DV / kColsW;
-  static_assert(RW * 32 == DK && NW * kColsW == DV, "shape");
+// NSPLIT CTAs share one (sequence, head), each with DV / 8 / NSPLIT warps of
+// 8 columns; with NSPLIT > 1 their per-token column sums go to fp32 partial
+// buffers that kda_backward_reduce_kernel adds up in split order.
+template <typename IO, int DK, int DV, int NSPLIT>
+__global__ void __launch_bounds__(DV / kColsW / NSPLIT * 32, 1) kda_backward_kernel(const BwdArgs a) {
+  constexpr int RW = DK / 32, NW = DV / kColsW / NSPLIT;
+  constexpr int TS = NW * kColsW * DK;  // floats per state tile of this CTA's columns
+  static_assert(RW * 32 == DK && NW * kColsW * NSPLIT == DV, "shape");
   // dynamic shared memory: per-warp partial dq, dk, dg of kRed tokens; partial
   // dbeta and per-head dg; u_t and w_t of the window
   extern __shared__ __align__(16) float bsm[];
@@ -107,13 +113,13 @@ __global__ void __launch_bounds__(DV / kColsW * 32, 1) kda_backward_kernel(const
   float* stb = stage + 3 * kCk * DK + 2 * kCk * DV;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x, h = bh % a.H, b = bh / a.H;
+  const int cta = blockIdx.x, bh = cta / NSPLIT, cs = cta % NSPLIT, h = bh % a.H, b = bh / a.H;
   const int T = a.T, H = a.H, gate = a.gate;
-  const int r0 = RW * lane, c0 = kColsW * warp;
+  const int r0 = RW * lane, c0 = kColsW * (cs * NW + warp);
   const int NCK = (T + kCk - 1) / kCk;
-  const size_t st0 = (size_t)bh * DK * DV;
-  float* ck = a.ckpt + (size_t)bh * NCK * DK * DV;
-  float* sc = a.scratch + (size_t)bh * kCk * DK * DV;
+  const size_t st0 = (size_t)bh * DK * DV, ntok = (size_t)(gridDim.x / NSPLIT) * T;  // B * H * T
+  float* ck = a.ckpt + (size_t)cta * NCK * TS;
+  float* sc = a.scratch + (size_t)cta * kCk * TS;
   const IO* q = static_cast<const IO*>(a.q);
   const IO* k = static_cast<const IO*>(a.k);
   const IO* v = static_cast<const IO*>(a.v);
@@ -225,7 +231,7 @@ __global__ void __launch_bounds__(DV / kColsW * 32, 1) kda_backward_kernel(const
     for (int j = 0; j < kColsW; ++j) S[i][j] = a.s0 ? a.s0[st0 + (size_t)(r0 + i) * DV + c0 + j] : 0.f;
   for (int t0 = 0; t0 < T; t0 += kCk) {
     const int t1 = min(T, t0 + kCk);
-    st_tile_ws(ck + (size_t)(t0 / kCk) * DK * DV, S);
+    st_tile_ws(ck + (size_t)(t0 / kCk) * TS, S);
     __syncthreads();  // the previous tile's inputs are no longer read
     stage_window(t0, t1, false);
     __syncthreads();
@@ -247,11 +253,11 @@ __global__ void __launch_bounds__(DV / kColsW * 32, 1) kda_backward_kernel(const
     __syncthreads();  // the previous window's inputs are no longer read
     stage_window(t0, t1, true);
     __syncthreads();
-    ld_tile_ws(ck + (size_t)m * DK * DV, S);
+    ld_tile_ws(ck + (size_t)m * TS, S);
     for (int t = t0; t < t1; ++t) {
       float sp[RW][kColsW], u[kColsW], w[kColsW];
       fwd_token(t - t0, S, sp, u, w);
-      st_tile_ws(sc + (size_t)(t - t0) * DK * DV, sp);
+      st_tile_ws(sc + (size_t)(t - t0) * TS, sp);
       if (lane < kColsW) {
         suw[t - t0][0][c0 + lane] = pick8(u, lane);
         suw[t - t0][1][c0 + lane] = pick8(w, lane);
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(DV / kColsW * 32, 1) kda_backward_kernel(const
           u[j] = suw[tw][0][c0 + j];
           w[j] = suw[tw][1][c0 + j];
         }
-        ld_tile_ws(sc + (size_t)tw * DK * DV, sp);
+        ld_tile_ws(sc + (size_t)tw * TS, sp);
         float pdq[RW], du[kColsW];
 #pragma unroll
         for (int j = 0; j < kColsW; ++j) du[j] = 0.f;
@@ -342,8 +348,12 @@ __global__ void __launch_bounds__(DV / kColsW * 32, 1) kda_backward_kernel(const
         float x = 0.f;
 #pragma unroll
         for (int ww = 0; ww < NW; ++ww) x += red[ww][tr][which][r];
-        IO* out = static_cast<IO*>(which == 0 ? a.dq : which == 1 ? a.dk : a.dg);
-        out[tok_of(s0 + tr) * DK + r] = from_f32<IO>(x);
+        if (NSPLIT == 1) {
+          IO* out = static_cast<IO*>(which == 0 ? a.dq : which == 1 ? a.dk : a.dg);
+          out[tok_of(s0 + tr) * DK + r] = from_f32<IO>(x);
+        } else {
+          a.part[((size_t)which * NSPLIT + cs) * ntok * DK + tok_of(s0 + tr) * DK + r] = x;
+        }
       }
       if (tid < nt) {
         float x = 0.f, y = 0.f;
@@ -352,8 +362,13 @@ __global__ void __launch_bounds__(DV / kColsW * 32, 1) kda_backward_kernel(const
           x += redb[ww][tid];
           y += redgh[ww][tid];
         }
-        static_cast<IO*>(a.dbeta)[tok_of(s0 + tid)] = from_f32<IO>(x);
-        if (gate == KDA_GATE_HEAD) static_cast<IO*>(a.dg)[tok_of(s0 + tid)] = from_f32<IO>(y);
+        if (NSPLIT == 1) {
+          static_cast<IO*>(a.dbeta)[tok_of(s0 + tid)] = from_f32<IO>(x);
+          if (gate == KDA_GATE_HEAD) static_cast<IO*>(a.dg)[tok_of(s0 + tid)] = from_f32<IO>(y);
+        } else {
+          a.partb[(size_t)cs * ntok + tok_of(s0 + tid)] = x;
+          a.partb[((size_t)NSPLIT + cs) * ntok + tok_of(s0 + tid)] = y;
+        }
       }
       __syncthreads();
     }
@@ -361,35 +376,81 @@ __global__ void __launch_bounds__(DV / kColsW * 32, 1) kda_backward_kernel(const
   if (a.ds0) st_tile(a.ds0 + st0, G);
 }
 
-template <int DK, int DV>
-constexpr size_t smem_bytes() {
-  return sizeof(float) * ((size_t)(DV / kColsW) * kRed * 3 * DK + 2 * (DV / kColsW) * kRed + (size_t)kCk * 2 * DV +
-                           (size_t)kCk * (3 * DK + 2 * DV + 1));
+// Sums the NSPLIT partials of dq, dk, dg (per channel) and dbeta, dg (per
+// head) in split order and writes them in the output type.
+template <typename IO>
+__global__ void kda_backward_reduce_kernel(const BwdArgs a, size_t ntok, int DK, int nsplit) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x, n = ntok * DK;
+  if (i < n) {
+    for (int which = 0; which < 3; ++which) {
+      if (which == 2 && a.gate != KDA_GATE_CHANNEL) continue;
+      float x = 0.f;
+      for (int s = 0; s < nsplit; ++s) x += a.part[((size_t)which * nsplit + s) * n + i];
+      static_cast<IO*>(which == 0 ? a.dq : which == 1 ? a.dk : a.dg)[i] = from_f32<IO>(x);
+    }
+  }
+  if (i < ntok) {
+    float x = 0.f, y = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+      x += a.partb[(size_t)s * ntok + i];
+      y += a.partb[((size_t)nsplit + s) * ntok + i];
+    }
+    static_cast<IO*>(a.dbeta)[i] = from_f32<IO>(x);
+    if (a.gate == KDA_GATE_HEAD) static_cast<IO*>(a.dg)[i] = from_f32<IO>(y);
+  }
 }
 
-template <typename T, int DK, int DV>
-cudaError_t launch_typed(const BwdArgs& a, int BH, cudaStream_t stream) {
-  constexpr size_t smem = smem_bytes<DK, DV>();
-  cudaError_t e = cudaFuncSetAttribute(kda_backward_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+template <int DK, int DV, int NSPLIT>
+constexpr size_t smem_bytes() {
+  constexpr int NW = DV / kColsW / NSPLIT;
+  return sizeof(float) * ((size_t)NW * kRed * 3 * DK + 2 * NW * kRed + (size_t)kCk * 2 * DV +
+                          (size_t)kCk * (3 * DK + 2 * DV + 1));
+}
+
+template <typename IO, int DK, int DV, int NSPLIT>
+cudaError_t launch_split(const BwdArgs& a, int BH, cudaStream_t stream) {
+  constexpr size_t smem = smem_bytes<DK, DV, NSPLIT>();
+  cudaError_t e = cudaFuncSetAttribute(kda_backward_kernel<IO, DK, DV, NSPLIT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kda_backward_kernel<T, DK, DV><<<BH, DV / kColsW * 32, smem, stream>>>(a);
+  kda_backward_kernel<IO, DK, DV, NSPLIT><<<BH * NSPLIT, DV / kColsW / NSPLIT * 32, smem, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || NSPLIT == 1) return e;
+  const size_t ntok = (size_t)BH * a.T, n = ntok * DK;
+  kda_backward_reduce_kernel<IO><<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(a, ntok, DK, NSPLIT);
   return cudaGetLastError();
 }
 
-template <typename T>
-cudaError_t launch_dims(const BwdArgs& a, int BH, int dk, int dv, cudaStream_t stream) {
-  if (dk == 128 && dv == 128) return launch_typed<T, 128, 128>(a, BH, stream);
-  if (dk == 128 && dv == 64) return launch_typed<T, 128, 64>(a, BH, stream);
-  if (dk == 64 && dv == 128) return launch_typed<T, 64, 128>(a, BH, stream);
-  return launch_typed<T, 64, 64>(a, BH, stream);
+template <typename IO, int DK, int DV>
+cudaError_t launch_typed(const BwdArgs& a, int BH, int nsplit, cudaStream_t stream) {
+  if (nsplit == 4) return launch_split<IO, DK, DV, 4>(a, BH, stream);
+  if (nsplit == 2) return launch_split<IO, DK, DV, 2>(a, BH, stream);
+  return launch_split<IO, DK, DV, 1>(a, BH, stream);
+}
+
+template <typename IO>
+cudaError_t launch_dims(const BwdArgs& a, int BH, int dk, int dv, int nsplit, cudaStream_t stream) {
+  if (dk == 128 && dv == 128) return launch_typed<IO, 128, 128>(a, BH, nsplit, stream);
+  if (dk == 128 && dv == 64) return launch_typed<IO, 128, 64>(a, BH, nsplit, stream);
+  if (dk == 64 && dv == 128) return launch_typed<IO, 64, 128>(a, BH, nsplit, stream);
+  return launch_typed<IO, 64, 64>(a, BH, nsplit, stream);
+}
+
+// CTAs per (sequence, head): more when few pairs would leave SMs idle (up to
+// 4 and one wave of a 148-SM part); a fixed function of the shape.
+int backward_split(int BH) {
+  int n = 1;
+  while (n < 4 && BH * n * 2 <= 148) n *= 2;
+  return n;
 }
 
 }  // namespace
 
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv) {
-  const size_t nck = ((size_t)T + kCk - 1) / kCk;
-  return (size_t)B * H * (nck + kCk) * dk * dv * sizeof(float);
+  const size_t nck = ((size_t)T + kCk - 1) / kCk, ntok = (size_t)B * T * H;
+  const int ns = backward_split(B * H);
+  const size_t part = ns > 1 ? (size_t)ns * ntok * (3 * (size_t)dk + 2) : 0;
+  return ((size_t)B * H * (nck + kCk) * dk * dv + part) * sizeof(float);
 }
 
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -401,11 +462,15 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
   a.q = q, a.k = k, a.v = v, a.g = g, a.beta = beta, a.d_o = d_o;
   a.s0 = s0, a.dsT = dsT;
   a.dq = dq, a.dk = dk_out, a.dv = dv_out, a.dg = dg, a.dbeta = dbeta, a.ds0 = ds0;
+  const int ns = backward_split(B * H);
+  const size_t ntok = (size_t)B * T * H;
   a.ckpt = static_cast<float*>(ws);
   a.scratch = a.ckpt + (size_t)B * H * nck * dk * dv;
+  a.part = a.scratch + (size_t)B * H * kCk * dk * dv;
+  a.partb = a.part + (size_t)ns * ntok * 3 * dk;
   a.scale = scale, a.T = T, a.H = H, a.gate = gate;
-  if (dtype == KDA_F32) return launch_dims<float>(a, B * H, dk, dv, stream);
-  return launch_dims<__nv_bfloat16>(a, B * H, dk, dv, stream);
+  if (dtype == KDA_F32) return launch_dims<float>(a, B * H, dk, dv, ns, stream);
+  return launch_dims<__nv_bfloat16>(a, B * H, dk, dv, ns, stream);
 }
 
 }  // namespace kda

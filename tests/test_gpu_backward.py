@@ -75,3 +75,10 @@ def test_backward_deterministic():
     torch.cuda.synchronize()
     for n in a:
         assert torch.equal(a[n], b[n]), n
+
+
+@pytest.mark.parametrize("B,H", [(5, 8), (10, 8)], ids=["2-way-split", "no-split"])
+def test_backward_column_splits(B, H):
+    """Few (sequence, head) pairs split each head's value columns over 4 CTAs
+    (covered above); 40 pairs split in 2, 80 pairs not at all."""
+    _case(B, 40, H, 128, 128, torch.float32, seed=97 + B)
