@@ -45,7 +45,9 @@ struct Vec<2> {
 
 constexpr int kDecodeWarps = 8;
 
-template <typename T, int DK, int DV>
+// kGeneric: a forget gate other than per channel, or fused input preparation
+// (run-time `gate` and `prep`); the default instance is the plain KDA step.
+template <typename T, int DK, int DV, bool kGeneric>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
     decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                        const T* __restrict__ g, const T* __restrict__ beta, float scale,
@@ -69,12 +71,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   if (tid < DK) {
     sq[tid] = to_f32(q[head * DK + tid]);
     sk[tid] = to_f32(k[head * DK + tid]);
-    sa[tid] = gate_alpha(gate, prep, g + head * DK, g + head, tid);
+    sa[tid] = kGeneric ? gate_alpha(gate, prep, g + head * DK, g + head, tid) : expf(to_f32(g[head * DK + tid]));
   }
   if (tid < DV) sv[tid] = to_f32(v[head * DV + tid]);
-  if (tid == 0) sbeta = prep_beta(prep, to_f32(beta[head]));
+  if (tid == 0) sbeta = kGeneric ? prep_beta(prep, to_f32(beta[head])) : to_f32(beta[head]);
   __syncthreads();
-  if (prep & KDA_PREP_L2NORM_QK) {  // q, k to unit length (fused input preparation)
+  if (kGeneric && (prep & KDA_PREP_L2NORM_QK)) {  // q, k to unit length (fused input preparation)
     if (warp < 2) {
       const float* x = warp == 0 ? sq : sk;
       float ss = 0.f;
@@ -152,8 +154,12 @@ cudaError_t launch_typed(const void* q, const void* k, const void* v, const void
                          float scale, float* state, void* o, int N, int H, int gate, int prep,
                          cudaStream_t stream) {
   const unsigned heads = (unsigned)N * (unsigned)H;
-  decode_step_kernel<T, DK, DV><<<heads, kDecodeWarps * 32, 0, stream>>>(
-      (const T*)q, (const T*)k, (const T*)v, (const T*)g, (const T*)beta, scale, state, (T*)o, gate, prep);
+  if (gate == KDA_GATE_CHANNEL && prep == 0)
+    decode_step_kernel<T, DK, DV, false><<<heads, kDecodeWarps * 32, 0, stream>>>(
+        (const T*)q, (const T*)k, (const T*)v, (const T*)g, (const T*)beta, scale, state, (T*)o, gate, prep);
+  else
+    decode_step_kernel<T, DK, DV, true><<<heads, kDecodeWarps * 32, 0, stream>>>(
+        (const T*)q, (const T*)k, (const T*)v, (const T*)g, (const T*)beta, scale, state, (T*)o, gate, prep);
   return cudaGetLastError();
 }
 
