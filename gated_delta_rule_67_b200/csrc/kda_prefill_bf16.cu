@@ -719,7 +719,7 @@ struct StatePassArgs {
   const float* s0;  // [B*H][128][128] or null (zero)
   float* sT;        // [B*H][128][128] or null
   float* rbuf;      // [B*H][G][128][128] scan buffers
-  float* mbuf;      // transition matrices, transposed: [B*H][G][k][r] = M_g[r][k]
+  float* mbuf;      // transition matrices: [B*H][G] slots of 64 KiB, each the 32 KiB bf16 K-major image of M_g
   const float* sbuf;
   int T, H, NC, G, L, phase;
 };
@@ -769,7 +769,10 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     const int g = blockIdx.x % G;
     cb = g * L;
     ce = min(NC, cb + L);
-    init = args.sbuf + ((size_t)bh * G + g) * kSt;
+    // group 0 starts from the initial state, group 1 from R_0; later ones from
+    // the combination kernel's output
+    init = g == 0 ? (args.s0 ? args.s0 + (size_t)bh * kSt : nullptr)
+                  : g == 1 ? args.rbuf + (size_t)bh * G * kSt : args.sbuf + ((size_t)bh * G + g) * kSt;
     fin = (g == G - 1 && args.sT) ? args.sT + bh * kSt : nullptr;
   }
   const int NCL = ce - cb;  // chunks this CTA walks
@@ -1011,12 +1014,12 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         float v[32];
         tmem_ld32(tm + kTmS + lane_off + q * 32, v);
         if (ident) {
-          // A transition matrix is stored transposed (row j of M^T = column j
-          // of M), the layout the combination kernel streams.
-          float4* dst = reinterpret_cast<float4*>(fin + (size_t)j * kD + q * 32);
+          // A transition matrix is stored as the bf16 K-major 128-row image of
+          // M (row r, column j at kmajor_off(r, j)), the B operand of the
+          // combination kernel; this thread holds column j.
+          uint8_t* img = reinterpret_cast<uint8_t*>(fin);
 #pragma unroll
-          for (int i4 = 0; i4 < 8; ++i4)
-            dst[i4] = make_float4(v[4 * i4], v[4 * i4 + 1], v[4 * i4 + 2], v[4 * i4 + 3]);
+          for (int ii = 0; ii < 32; ++ii) stbf(img, kmajor_off(q * 32 + ii, j, kD), v[ii]);
         } else {
 #pragma unroll
           for (int ii = 0; ii < 32; ++ii) fin[(size_t)(q * 32 + ii) * kD + j] = v[ii];
@@ -1030,124 +1033,122 @@ __global__ void __launch_bounds__(kSPThreads, 1)
 }
 
 // ======================================================== scan combine
-// S_{g+1} = M_g S_g + R_g for g = 1 .. G-2 (S_0 = initial state, S_1 = R_0),
-// in fp32 on the CUDA cores.  The columns of S never mix, so each CTA owns 16
-// columns of one chain and walks the groups on its own.  Every M_g and R_g is
-// ready when the kernel starts, so the transposed transition matrices stream
-// through a ring of shared-memory stages by bulk copies while earlier steps
-// compute.  Thread (warp w, lane l) owns rows l + 32 i (i < 4), columns
-// 4 (w % 4) .. +3 of the CTA's block and half w / 4 of the k range: per k one
-// broadcast float4 of S_g and four conflict-free scalars of M_g^T feed 16
-// FMAs; the upper half's partial sums are added through shared memory.
-constexpr int kScanCols = 16;
-constexpr int kScanStages = 3;
-constexpr int kScanThreads = 256;
-constexpr int kScanLd = 20;  // padded row stride of the S_g blocks (conflict-free float4 stores)
-constexpr uint32_t kScanStageBytes = kD * kD * sizeof(float);
-constexpr size_t kScanSmem = kScanStages * (size_t)kScanStageBytes + 3 * (size_t)kD * kScanLd * sizeof(float);
+// S_{g+1} = M_g S_g + R_g for g = 1 .. G-2 (S_1 = R_0; the output pass reads
+// S_0 and S_1 from the initial state and from R_0 itself), one CTA per chain,
+// on the tensor cores in the state pass's transposed form
+//   S_{g+1}^T = S_g^T M_g^T + R_g^T:
+// thread n owns TMEM lane n (value channel n); the accumulator starts as
+// R_g^T, A is S_g^T in bf16 (tensor memory), B the bf16 K-major image of M_g
+// written by the transition pass (rows = rows of M_g).  S and M are rounded
+// to bf16 with fp32 accumulation, as in one chunk step of the state pass.
+// M_g images and R_g (fp32, row-major) stream through two-stage rings.
+constexpr int kCbThreads = 128;
+constexpr uint32_t kCbImg = 32768;             // bytes of one M_g image
+constexpr uint32_t kCbR = 65536;               // bytes of one R_g
+constexpr uint32_t kCbTmS = 0, kCbTmA = 128;   // TMEM: S^T fp32 [0,128), S^T bf16 [128,192)
+constexpr size_t kCbSmem = 2 * kCbImg + 2 * kCbR + 1024;
 
-__global__ void __launch_bounds__(kScanThreads) kda_scan_combine_kernel(const float* s0, float* sbuf, const float* rbuf,
-                                                                        const float* mbuf_t, int G,
-                                                                        WorkspaceHeader* hdr) {
-  extern __shared__ __align__(16) float scm[];
-  __shared__ uint64_t full[kScanStages];
+__global__ void __launch_bounds__(kCbThreads) kda_scan_combine_kernel(float* sbuf, const float* rbuf,
+                                                                      const float* mbuf, int G, WorkspaceHeader* hdr) {
+  extern __shared__ uint8_t cb_raw[];
+  uint8_t* sm = align1024(cb_raw);  // [2 M images][2 R stages]
+  __shared__ uint64_t bar_m[2], bar_r[2], bar_mma;
+  __shared__ uint32_t tmem_base;
   constexpr size_t kSt = (size_t)kD * kD;
-  float* Mt = scm;                              // [stage][k][r] = M_g[r][k]
-  float* Sc = scm + kScanStages * kSt;          // [2][128][kScanLd] S_g blocks
-  float* Pu = Sc + 2 * kD * kScanLd;            // [128][kScanLd] upper-half partial sums
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int cw = 4 * (warp & 3), kh = warp >> 2;
-  const int bh = blockIdx.x / (kD / kScanCols);
-  const int c0 = (blockIdx.x % (kD / kScanCols)) * kScanCols + cw;  // this thread's first global column
-  float* sb = sbuf + (size_t)bh * G * kSt;
+  const int tid = threadIdx.x, warp = tid >> 5, n = tid;
+  const int bh = blockIdx.x;
   const float* rb = rbuf + (size_t)bh * G * kSt;
-  const float* mb = mbuf_t + (size_t)bh * G * kSt;
+  float* sb = sbuf + (size_t)bh * G * kSt;
+  const uint8_t* mb = reinterpret_cast<const uint8_t*>(mbuf + (size_t)bh * G * kSt);  // slot g at g * kSt floats
   const int nsteps = G - 2;
-  auto issue = [&](int stage, int g) {
-    mbar_expect_tx(&full[stage], kScanStageBytes);
+  auto m_img = [&](int st) { return sm + st * kCbImg; };
+  auto r_tile = [&](int st) { return reinterpret_cast<const float*>(sm + 2 * kCbImg + st * kCbR); };
+  auto load_m = [&](int st, int g) {
+    mbar_expect_tx(&bar_m[st], kCbImg);
+    bulk_load(sm + st * kCbImg, mb + (size_t)g * kSt * sizeof(float), kCbImg, &bar_m[st]);
+  };
+  auto load_r = [&](int st, int g) {
+    mbar_expect_tx(&bar_r[st], kCbR);
 #pragma unroll
     for (int p = 0; p < 4; ++p)
-      bulk_load(Mt + stage * kSt + p * (kSt / 4), mb + g * kSt + p * (kSt / 4), kScanStageBytes / 4, &full[stage]);
+      bulk_load(sm + 2 * kCbImg + st * kCbR + p * (kCbR / 4), rb + (size_t)g * kSt + p * (kSt / 4), kCbR / 4,
+                &bar_r[st]);
   };
-  grid_dep_wait();    // the transition and offset passes have finished
-  grid_dep_launch();  // the output pass may be scheduled (it waits for this grid)
+  grid_dep_wait();  // the transition and offset passes have finished
   if (tid == 0) {
-    for (int s = 0; s < kScanStages; ++s) mbar_init(&full[s], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_m[i], 1);
+      mbar_init(&bar_r[i], 1);
+    }
+    mbar_init(&bar_mma, 1);
     fence_mbar_init();
-    for (int s = 0; s < kScanStages && s < nsteps; ++s) issue(s, 1 + s);
+    load_r(0, 0);                        // R_0 = S_1, the first A operand
+    load_r(1, 1);
+    for (int st = 0; st < 2 && st < nsteps; ++st) load_m(st, 1 + st);
   }
-  // S_0 (lower half of the threads) and S_1 = R_0 (upper half)
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = lane + 32 * i;
-    const size_t idx = (size_t)r * kD + c0;
-    if (kh == 0) {
-      const float4 a =
-          s0 ? *reinterpret_cast<const float4*>(s0 + (size_t)bh * kSt + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4*>(sb + idx) = a;
-    } else {
-      const float4 s1 = *reinterpret_cast<const float4*>(rb + idx);
-      *reinterpret_cast<float4*>(sb + kSt + idx) = s1;
-      *reinterpret_cast<float4*>(Sc + r * kScanLd + cw) = s1;
-    }
-  }
-  float4 rn[4];
-  if (kh == 0 && nsteps > 0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) rn[i] = *reinterpret_cast<const float4*>(rb + kSt + (size_t)(lane + 32 * i) * kD + c0);
-  }
+  if (warp == 0) tmem_alloc(&tmem_base, 256);
+  tc_fence_before();
   __syncthreads();
-  for (int step = 0; step < nsteps; ++step) {
-    const int g = step + 1, s = step % kScanStages;
-    float acc[4][4];
+  tc_fence_after();
+  grid_dep_launch();  // the output pass may be scheduled (it waits for this grid)
+  const uint32_t tm = tmem_base, lane_off = (uint32_t)(warp * 32) << 16;
+
+  // A <- S_1^T = R_0^T in bf16 (row k of R_0 at k * 128 floats; thread n reads column n)
+  wait_or_flag(&bar_r[0], 0, hdr, 40);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[i][0] = kh ? 0.f : rn[i].x;
-      acc[i][1] = kh ? 0.f : rn[i].y;
-      acc[i][2] = kh ? 0.f : rn[i].z;
-      acc[i][3] = kh ? 0.f : rn[i].w;
-    }
-    if (kh == 0 && step + 1 < nsteps) {  // R of the next step, in flight during this one
+  for (int q = 0; q < kD / 32; ++q) {
+    const float* r = r_tile(0) + (size_t)q * 32 * kD + n;
+    uint32_t pk[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        rn[i] = *reinterpret_cast<const float4*>(rb + (size_t)(g + 1) * kSt + (size_t)(lane + 32 * i) * kD + c0);
-    }
-    wait_or_flag(&full[s], (step / kScanStages) & 1, hdr, 40);
-    const float* M = Mt + s * kSt + kh * (kD / 2) * kD;
-    const float* X = Sc + (step & 1) * kD * kScanLd + kh * (kD / 2) * kScanLd;
-#pragma unroll 8
-    for (int k = 0; k < kD / 2; ++k) {
-      const float4 x = *reinterpret_cast<const float4*>(X + k * kScanLd + cw);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float m = M[k * kD + lane + 32 * i];
-        acc[i][0] = fmaf(m, x.x, acc[i][0]);
-        acc[i][1] = fmaf(m, x.y, acc[i][1]);
-        acc[i][2] = fmaf(m, x.z, acc[i][2]);
-        acc[i][3] = fmaf(m, x.w, acc[i][3]);
-      }
-    }
-    if (kh) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4*>(Pu + (lane + 32 * i) * kScanLd + cw) =
-            make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-    }
-    __syncthreads();  // partial sums visible; stage s no longer read
-    if (tid == 0 && step + kScanStages < nsteps) issue(s, g + kScanStages);
-    if (kh == 0) {
-      float* Xn = Sc + ((step + 1) & 1) * kD * kScanLd;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = lane + 32 * i;
-        const float4 p = *reinterpret_cast<const float4*>(Pu + r * kScanLd + cw);
-        const float4 o = make_float4(acc[i][0] + p.x, acc[i][1] + p.y, acc[i][2] + p.z, acc[i][3] + p.w);
-        *reinterpret_cast<float4*>(Xn + r * kScanLd + cw) = o;
-        *reinterpret_cast<float4*>(sb + (size_t)(g + 1) * kSt + (size_t)r * kD + c0) = o;
-      }
-    }
-    __syncthreads();  // S_{g+1} block complete; partial-sum buffer free
+    for (int e = 0; e < 16; ++e) pk[e] = pack2(r[(2 * e) * kD], r[(2 * e + 1) * kD]);
+    tmem_st16u(tm + kCbTmA + lane_off + q * 16, pk);
   }
+  const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+  for (int step = 0; step < nsteps; ++step) {
+    const int g = step + 1, s = step & 1, rs = g & 1;  // R_g sits in stage g % 2
+    // accumulator <- R_g^T
+    wait_or_flag(&bar_r[rs], (g >> 1) & 1, hdr, 43);
+#pragma unroll
+    for (int q = 0; q < kD / 32; ++q) {
+      const float* r = r_tile(rs) + (size_t)q * 32 * kD + n;
+      float v[32];
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) v[ii] = r[ii * kD];
+      tmem_st32(tm + kCbTmS + lane_off + q * 32, v);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();  // R_g (and at the first step R_0) fully read from shared memory
+    if (tid == 0) {
+      tc_fence_after();
+      if (g + 1 <= nsteps) load_r(rs ^ 1, g + 1);  // the other stage held R_{g-1}, read by now
+      wait_or_flag(&bar_m[s], (step >> 1) & 1, hdr, 41);
+      const uint64_t b0 = desc_sw128(smem_u32(m_img(s)), 16, 1024);
+#pragma unroll
+      for (int k = 0; k < kD / 16; ++k)  // K-major B: +32 B per step inside a 64-wide block, +16 KiB per block
+        mma_bf16_ts(tm + kCbTmS, tm + kCbTmA + k * 8, b0 + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), idesc, 1);
+      mma_commit(&bar_mma);
+    }
+    wait_or_flag(&bar_mma, step & 1, hdr, 42);
+    tc_fence_after();
+    if (tid == 0 && step + 2 < nsteps) load_m(s, g + 2);  // stage s is free: bring M_{g+2}
+    // S_{g+1}: to the scan buffer and, as bf16, into the next A operand
+#pragma unroll
+    for (int q = 0; q < kD / 32; ++q) {
+      float v[32];
+      tmem_ld32(tm + kCbTmS + lane_off + q * 32, v);
+#pragma unroll
+      for (int ii = 0; ii < 32; ++ii) sb[(size_t)(g + 1) * kSt + (size_t)(q * 32 + ii) * kD + n] = v[ii];
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) pk[e] = pack2(v[2 * e], v[2 * e + 1]);
+      tmem_st16u(tm + kCbTmA + lane_off + q * 16, pk);
+    }
+  }
+  tmem_wait_st();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem_base, 256);
 }
 
 // =============================================== bounded-wait self-test
@@ -1280,7 +1281,7 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     cudaError_t e;
     e = cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kP2Bytes + 1024);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
+    e = cudaFuncSetAttribute(kda_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCbSmem);
     if (e != cudaSuccess) return e;
     attrs_set = true;
   }
@@ -1324,8 +1325,8 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     e = launch_dependent(kda_state_pass_kernel, (unsigned)(BH * (2 * G - 3)), kSPThreads, kP2Bytes + 1024, stream,
                          mo, a);
     if (e != cudaSuccess) return e;
-    e = launch_dependent(kda_scan_combine_kernel, (unsigned)(BH * (kD / kScanCols)), kScanThreads, kScanSmem, stream,
-                         s0, scan + 2 * per, (const float*)scan, (const float*)(scan + per), G, hdr);
+    e = launch_dependent(kda_scan_combine_kernel, (unsigned)BH, kCbThreads, kCbSmem, stream, scan + 2 * per,
+                         (const float*)scan, (const float*)(scan + per), G, hdr);
     if (e != cudaSuccess) return e;
     a.phase = 3;
     e = launch_dependent(kda_state_pass_kernel, (unsigned)(BH * G), kSPThreads, kP2Bytes + 1024, stream, mo, a);
