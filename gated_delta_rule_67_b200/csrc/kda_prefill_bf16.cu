@@ -56,7 +56,8 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kC = 64;    // chunk length
 constexpr int kD = 128;   // d_k = d_v
-constexpr int kRefTok = 31;
+constexpr int kRefTok = 31;  // reference token of the factored form: the end of the second 16-token stride
+static_assert(kRefTok == 2 * 16 - 1, "pass 1 takes G_r as the sum of the first two stride totals");
 
 // --- per-chunk record in the workspace (byte offsets) -----------------------
 constexpr uint32_t kRecWQ = 0;          // [-W ; Q+]: K-major, 128 rows x 128 ch (32 KiB)
@@ -95,13 +96,9 @@ constexpr uint32_t kP2Out = 2 * kStage;     // two 16 KiB output staging tiles [
 constexpr uint32_t kP2Bytes = kP2Out + 2 * 16384;
 
 constexpr uint32_t kWaitLimit = 1u << 24;
-constexpr uint32_t kSpinLimit = 1u << 30;  // ~seconds of test_wait probes
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-__device__ __forceinline__ float ldbf(const uint8_t* base, uint32_t off) {
-  return __bfloat162float(*reinterpret_cast<const bf16*>(base + off));
 }
 __device__ __forceinline__ void stbf(uint8_t* base, uint32_t off, float x) {
   *reinterpret_cast<bf16*>(base + off) = __float2bfloat16_rn(x);
@@ -122,20 +119,10 @@ __device__ __forceinline__ void wait_or_flag(uint64_t* bar, uint32_t parity, Wor
     atomicExch(&hdr->where, where);
   }
 }
-// Same, spinning (for the sequential chain, where wake-up latency is the cost).
-__device__ __forceinline__ void spin_or_flag(uint64_t* bar, uint32_t parity, WorkspaceHeader* hdr, uint32_t where) {
-  if (!mbar_spin(bar, parity, kSpinLimit)) {
-    atomicOr(&hdr->error, 1u);
-    atomicExch(&hdr->where, where);
-  }
-}
 
 // =============================================================== kernel 1
 __device__ __forceinline__ float2 ld_bf2(const uint8_t* p) {
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-}
-__device__ __forceinline__ void st_bf2(uint8_t* p, float a, float b) {
-  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
 // 8 bf16 (16 bytes, 16-byte aligned) <-> 8 floats.
 __device__ __forceinline__ void ld8(const uint8_t* p, float* f) {
@@ -733,7 +720,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5;
   WorkspaceHeader* hdr = args.hdr;
-  const int T = args.T, H = args.H, NC = args.NC, G = args.G, L = args.L;
+  const int H = args.H, NC = args.NC, G = args.G, L = args.L;
   constexpr size_t kSt = (size_t)kD * kD;
   // ---- role of this CTA
   int bh, cb, ce;
