@@ -1,0 +1,973 @@
+// kda_backward_chunk.cu -- gradients of the KDA forward pass in the chunkwise form.
+//
+// Differentiates the chunk equations of the forward (KimiLinear article,
+// section 2.3 for the recurrence, section 3.1 for the chunkwise algorithm and
+// section 3.2 for the per-chunk C x C score matrices).  One chunk of C = 64
+// tokens with entering state S0 (d_k x d_v), G_i the in-chunk inclusive
+// cumsum of the log-gates, Gamma_i = exp(G_i), gamma = Gamma_C:
+//
+//   Q+ = scale q . Gamma,  K+ = k . Gamma,  Kbar_j = k_j . Gamma_C / Gamma_j
+//   P  = strict_tril(K+ K-^T)  with K- = k / Gamma     (pairwise: sum_r k_ir k_jr exp(G_ir - G_jr))
+//   Aqk = tril(Q+ K-^T),  T = (I + diag(beta) P)^-1,  W = T diag(beta) K+,  U = T diag(beta) V
+//   V' = U - W S0,  O = Q+ S0 + Aqk V',  S1 = diag(gamma) S0 + Kbar^T V'
+//
+// Reverse mode, chunk by chunk from the last one, with dS = dL/dS1:
+//
+//   dV' = Aqk^T dO + Kbar dS                       dS0 = diag(gamma) dS + Q+^T dO - W^T dV'
+//   dAqk = tril(dO V'^T)   dQ+ = dO S0^T + dAqk K-   dKbar = V' dS^T   dgamma = rowsum(dS . S0)
+//   dW = -dV' S0^T   dU = dV'   dT = dU (beta V)^T + dW (beta K+)^T   dA = -T^T dT T^T (strictly lower)
+//   dv = beta . T^T dU,   dK+ = beta . T^T dW + (beta dA) K-,   dK- = dAqk^T Q+ + (beta dA)^T K+
+//   dbeta = rowsum(V . T^T dU) + rowsum(K+ . T^T dW) + rowsum(dA . P)
+//
+// and the factors are folded back into dq, dk and dG, whose reverse in-chunk
+// cumsum is dg.  The pairwise products use factored operands relative to the
+// chunk's token 31 (K+_r = k exp(G - G_31), K-_r = k exp(G_31 - G)); their
+// products are independent of that reference, so the reference is a constant
+// for differentiation.  A chunk whose cumulative gates leave +-kSpan of the
+// reference takes an exact per-element path instead (exp of each difference).
+//
+// Four launches:
+//   1. bwd_prep    (chunk, seq x head): W, U, Q+, Kbar, Aqk, P, T, gamma per chunk
+//   2. bwd_pass    (seq x head x column slice, 2 roles): the forward state
+//      replay (checkpoints S0 and V' per chunk) and the reverse dS sweep
+//      (dS and dV' per chunk, dL/dS_0); the columns of the state evolve
+//      independently in both
+//   3. bwd_local_a (chunk, seq x head): the products contracting over d_v:
+//      dAqk, dT (first part), dv, dbeta (first part), dO S0^T, dW, dKbar, dgamma
+//   4. bwd_local_b (chunk, seq x head): the rest, and dq, dk, dg, dbeta
+// Arithmetic: warp-level tensor-core products (mma.sync m16n8k8, tf32
+// operands, fp32 accumulation) on fp32 shared-memory tiles.  With fp32 I/O
+// every product uses the three-term tf32 split (a_hi b_hi + a_hi b_lo +
+// a_lo b_hi), which keeps fp32-level accuracy; with bf16 I/O one tf32 term.
+// Everything in the workspace is fp32.  No atomics: every sum runs in a fixed
+// order, so results are bit-reproducible.
+#include <type_traits>
+
+#include "kda_common.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kC = 64;          // tokens per chunk
+constexpr int kRef = 31;        // reference token of the factored pairwise operands
+constexpr float kSpan = 64.f;   // factored operands need |G_i - G_ref| <= kSpan in every channel
+constexpr int kThreads = 256;   // 8 warps in every kernel
+constexpr int kLC = kC + 4;     // leading dimension of the C x C shared tiles
+
+// ------------------------------------------------------------------ warp MMA
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// A strided fp32 matrix view in shared memory: element (i, j) at p[i*rs + j*cs].
+struct View {
+  const float* p;
+  int rs, cs;
+  __device__ __forceinline__ float at(int i, int j) const { return p[i * rs + j * cs]; }
+};
+__device__ __forceinline__ View rowm(const float* p, int ld) { return View{p, ld, 1}; }  // X
+__device__ __forceinline__ View colm(const float* p, int ld) { return View{p, 1, ld}; }  // X^T
+
+// acc[MT][NT] (a (16 MT) x (8 NT) tile at rows m0, columns n0) += A[m0.., 0:K] B[0:K, n0..].
+// Fragment layout of mma.m16n8k8: g = lane / 4, t = lane % 4; A holds (g, t),
+// (g+8, t), (g, t+4), (g+8, t+4); B holds (t, g), (t+4, g); the accumulator
+// holds rows g, g+8 and columns 2t, 2t+1.  X3: three-term tf32 split.
+template <int MT, int NT, bool X3>
+__device__ __forceinline__ void warp_mma(float (&acc)[MT][NT][4], View A, View B, int m0, int n0, int K) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    uint32_t ah[MT][4], al[MT][4], bh[NT][2], bl[NT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int r = m0 + 16 * mt + g;
+      const float x[4] = {A.at(r, k0 + t), A.at(r + 8, k0 + t), A.at(r, k0 + t + 4), A.at(r + 8, k0 + t + 4)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ah[mt][e] = tf32_rna(x[e]);
+        if (X3) al[mt][e] = tf32_rna(x[e] - __uint_as_float(ah[mt][e]));
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int c = n0 + 8 * nt + g;
+      const float y[2] = {B.at(k0 + t, c), B.at(k0 + t + 4, c)};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        bh[nt][e] = tf32_rna(y[e]);
+        if (X3) bl[nt][e] = tf32_rna(y[e] - __uint_as_float(bh[nt][e]));
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (X3) {
+          mma_tf32(acc[mt][nt], al[mt][0], al[mt][1], al[mt][2], al[mt][3], bh[nt][0], bh[nt][1]);
+          mma_tf32(acc[mt][nt], ah[mt][0], ah[mt][1], ah[mt][2], ah[mt][3], bl[nt][0], bl[nt][1]);
+        }
+        mma_tf32(acc[mt][nt], ah[mt][0], ah[mt][1], ah[mt][2], ah[mt][3], bh[nt][0], bh[nt][1]);
+      }
+  }
+}
+
+// Split of an R x N output over the 8 warps: WM x WN warps, each (16 MT) x (8 NT).
+template <int R, int N>
+struct Tiling {
+  static constexpr int WM = (R / 16 >= 8) ? 8 : R / 16;
+  static constexpr int WN = 8 / WM;
+  static constexpr int MT = R / 16 / WM;
+  static constexpr int NT = N / 8 / WN;
+  static_assert(WM * WN == 8 && MT * 16 * WM == R && NT * 8 * WN == N, "tiling");
+  __device__ static int m0(int warp) { return (warp % WM) * MT * 16; }
+  __device__ static int n0(int warp) { return (warp / WM) * NT * 8; }
+};
+
+template <int MT, int NT>
+__device__ __forceinline__ void zero(float (&acc)[MT][NT][4]) {
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+}
+// f(mt, nt, e, row, col) over the accumulator elements acc[mt][nt][e] of this lane.
+template <int MT, int NT, typename F>
+__device__ __forceinline__ void for_acc(int m0, int n0, F&& f) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f(mt, nt, e, m0 + 16 * mt + g + 8 * (e >> 1), n0 + 8 * nt + 2 * t + (e & 1));
+}
+
+// Per-row sums of a tile product: each lane adds to rp[mt][half] for its rows
+// m0 + 16 mt + g + 8 half; the 4 lanes of a row are then combined and lane
+// t = 0 writes the warp's row sums to out[row] (one slot per column group).
+template <int MT>
+__device__ __forceinline__ void row_sums_out(float (&rp)[MT][2], int m0, float* out) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float x = rp[mt][hh];
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      if (t == 0) out[m0 + 16 * mt + g + 8 * hh] = x;
+    }
+}
+
+// ------------------------------------------------------------------ tiles
+// Rows of one chunk of a [B, T, H, len] tensor: token i of chunk (b, t0) is
+// row ((b*T + t0 + i) * H + h).  Loads columns col0 .. col0+W-1 of its 64 rows
+// as fp32 into dst (leading dimension ld), rows >= nv as zeros, times mult[i]
+// when mult is given.
+template <typename IO, int W>
+__device__ __forceinline__ void load_rows(float* dst, int ld, const IO* src, size_t row0, int H, int nv, int len,
+                                          int col0, const float* mult = nullptr) {
+  constexpr int V = 16 / sizeof(IO);  // elements per 16-byte load
+  constexpr int PER_ROW = W / V;
+  for (int idx = threadIdx.x; idx < kC * PER_ROW; idx += kThreads) {
+    const int i = idx / PER_ROW, c = (idx % PER_ROW) * V;
+    float x[V];
+    if (i < nv) {
+      const uint4 w = *reinterpret_cast<const uint4*>(src + (row0 + (size_t)i * H) * len + col0 + c);
+      if constexpr (std::is_same<IO, float>::value) {
+        x[0] = __uint_as_float(w.x), x[1] = __uint_as_float(w.y), x[2] = __uint_as_float(w.z),
+        x[3] = __uint_as_float(w.w);
+      } else {
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+          x[2 * e] = f.x, x[2 * e + 1] = f.y;
+        }
+      }
+      if (mult) {
+        const float m = mult[i];
+#pragma unroll
+        for (int e = 0; e < V; ++e) x[e] *= m;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < V; ++e) x[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < V; e += 4)
+      *reinterpret_cast<float4*>(dst + i * ld + c + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+  }
+}
+// fp32 rows x cols block from global (leading dimension gld) into shared (ld); cols % 4 == 0.
+__device__ __forceinline__ void load_f32(float* dst, int ld, const float* src, int gld, int rows, int cols) {
+  const int per = cols / 4;
+  for (int idx = threadIdx.x; idx < rows * per; idx += kThreads) {
+    const int i = idx / per, c = (idx % per) * 4;
+    *reinterpret_cast<float4*>(dst + i * ld + c) = *reinterpret_cast<const float4*>(src + (size_t)i * gld + c);
+  }
+}
+__device__ __forceinline__ void store_f32(float* dst, int gld, const float* src, int ld, int rows, int cols) {
+  const int per = cols / 4;
+  for (int idx = threadIdx.x; idx < rows * per; idx += kThreads) {
+    const int i = idx / per, c = (idx % per) * 4;
+    *reinterpret_cast<float4*>(dst + (size_t)i * gld + c) = *reinterpret_cast<const float4*>(src + i * ld + c);
+  }
+}
+
+// Per-channel log-gates of one chunk into sG [64][ld] (zeros past nv): per
+// channel, per head (broadcast over the channels) or none; then the inclusive
+// cumsum over the tokens, in place.
+template <typename IO, int DK>
+__device__ __forceinline__ void load_gates_cumsum(float* sG, int ld, const IO* g, int gate, size_t row0, int H,
+                                                  int nv) {
+  if (gate == KDA_GATE_CHANNEL) {
+    load_rows<IO, DK>(sG, ld, g, row0, H, nv, DK, 0);
+  } else {
+    for (int idx = threadIdx.x; idx < kC * DK; idx += kThreads) {
+      const int i = idx / DK, r = idx % DK;
+      sG[i * ld + r] = (gate == KDA_GATE_HEAD && i < nv) ? to_f32(g[row0 + (size_t)i * H]) : 0.f;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < DK) {
+    float acc = 0.f;
+    for (int i = 0; i < kC; ++i) {
+      acc += sG[i * ld + threadIdx.x];
+      sG[i * ld + threadIdx.x] = acc;
+    }
+  }
+  __syncthreads();
+}
+
+// Whether the chunk needs the exact pairwise path (block-uniform).
+template <int DK>
+__device__ __forceinline__ bool chunk_unsafe(const float* sG, int ld) {
+  bool bad = false;
+  for (int idx = threadIdx.x; idx < kC * DK; idx += kThreads) {
+    const int i = idx / DK, r = idx % DK;
+    bad |= !(fabsf(sG[i * ld + r] - sG[kRef * ld + r]) <= kSpan);
+  }
+  return __syncthreads_or(bad) != 0;
+}
+
+// ------------------------------------------------------------------ arguments
+struct ChunkBwdArgs {
+  const void *q, *k, *v, *g, *beta, *d_o;
+  const float *s0, *dsT;
+  void *dq, *dk, *dv, *dg, *dbeta;
+  float* ds0;
+  float scale;
+  int T, H, NC, gate;
+  // workspace (fp32), record rec = (b * H + h) * NC + chunk
+  float *W, *U, *Qp, *Kb;  // [rec][64][d_k] (U: [64][d_v]): W, U, Q+, Kbar
+  float *Aqk, *Tm, *Pkk;   // [rec][64][64]: Aqk, T, P
+  float* gam;              // [rec][d_k]: gamma
+  float *S0c, *dSc;        // [rec][d_k][d_v]: state entering the chunk, dL/d(state leaving it)
+  float *Vp, *dVp;         // [rec][64][d_v]: V', dV'
+  float *dAqk, *dT1;       // [rec][64][64]: dAqk, dU (beta V)^T (strictly lower)
+  float *dQs, *dW, *dKb;   // [rec][64][d_k]: dO S0^T, dW, dKbar
+  float* dgam;             // [rec][d_k]: rowsum(dS . S0)
+  float* dbu;              // [rec][64]: rowsum(V . T^T dU)
+};
+
+__device__ __forceinline__ size_t row_of(const ChunkBwdArgs& a, int bh, int t0) {
+  return ((size_t)(bh / a.H) * a.T + t0) * a.H + bh % a.H;
+}
+
+// ------------------------------------------------------------------ kernel 1
+template <int DK, int DV>
+constexpr size_t prep_smem() {
+  constexpr int LK = DK + 4, LM = (DK > DV ? DK : DV) + 4;
+  return sizeof(float) * ((size_t)4 * kC * LK + (size_t)kC * LM + 3 * kC * kLC + kC + DK);
+}
+
+// Per chunk: G, the factored and absolute operands, P and Aqk, T, W and U.
+template <typename IO, int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArgs a) {
+  constexpr bool X3 = std::is_same<IO, float>::value;
+  constexpr int LK = DK + 4, LM = (DK > DV ? DK : DV) + 4;
+  extern __shared__ __align__(16) float sm[];
+  float* sG = sm;             // [64][LK] cumulative log-gates
+  float* sK = sG + kC * LK;   // [64][LK] k
+  float* sQ = sK + kC * LK;   // [64][LK] q, then Q+_r (fast path)
+  float* sX = sQ + kC * LK;   // [64][LK] K+_r (exact path: K+), then beta K+
+  float* sY = sX + kC * LK;   // [64][LM] K-_r, then beta v
+  float* sP = sY + kC * LM;   // [64][kLC] P
+  float* sA = sP + kC * kLC;  // [64][kLC] Aqk
+  float* sT = sA + kC * kLC;  // [64][kLC] T
+  float* sb = sT + kC * kLC;  // [64] beta
+  float* se = sb + kC;        // [DK] exp(G_ref)
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int n = blockIdx.x % a.NC, bh = blockIdx.x / a.NC, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)bh * a.NC + n;
+  const IO* q = static_cast<const IO*>(a.q);
+  const IO* k = static_cast<const IO*>(a.k);
+  const IO* beta = static_cast<const IO*>(a.beta);
+
+  load_rows<IO, DK>(sK, LK, k, row0, a.H, nv, DK, 0);
+  load_rows<IO, DK>(sQ, LK, q, row0, a.H, nv, DK, 0);
+  if (tid < kC) sb[tid] = tid < nv ? to_f32(beta[row0 + (size_t)tid * a.H]) : 0.f;
+  load_gates_cumsum<IO, DK>(sG, LK, static_cast<const IO*>(a.g), a.gate, row0, a.H, nv);
+  const bool slow = chunk_unsafe<DK>(sG, LK);
+  if (tid < DK) {
+    se[tid] = expf(sG[kRef * LK + tid]);
+    a.gam[rec * DK + tid] = expf(sG[(kC - 1) * LK + tid]);
+  }
+  float* Qp = a.Qp + rec * kC * DK;
+  float* Kb = a.Kb + rec * kC * DK;
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {
+    const int i = idx / DK, r = idx % DK;
+    const float G = sG[i * LK + r], kk = sK[i * LK + r], qq = a.scale * sQ[i * LK + r];
+    const float gm = expf(G);
+    Qp[i * DK + r] = qq * gm;
+    Kb[i * DK + r] = kk * expf(sG[(kC - 1) * LK + r] - G);
+    if (!slow) {
+      const float d = G - sG[kRef * LK + r];
+      const float ex = expf(d);
+      sX[i * LK + r] = kk * ex;
+      sY[i * LK + r] = kk * expf(-d);
+      sQ[i * LK + r] = qq * ex;
+    } else {
+      sX[i * LK + r] = kk * gm;
+    }
+  }
+  __syncthreads();
+
+  // P = strict_tril(K+ K-^T), Aqk = tril(Q+ K-^T)
+  if (!slow) {
+    using Tl = Tiling<kC, kC>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);
+    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sX, LK), colm(sY, LK), m0, n0, DK);
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
+      sP[i * kLC + j] = j < i ? acc[mt][nt][e] : 0.f;
+    });
+    zero(acc);
+    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sQ, LK), colm(sY, LK), m0, n0, DK);
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
+      sA[i * kLC + j] = j <= i ? acc[mt][nt][e] : 0.f;
+    });
+  } else {
+    for (int idx = tid; idx < kC * kC; idx += kThreads) {
+      const int i = idx / kC, j = idx % kC;
+      float p = 0.f, s = 0.f;
+      if (j <= i) {
+        for (int r = 0; r < DK; ++r) {
+          const float e = expf(sG[i * LK + r] - sG[j * LK + r]) * sK[j * LK + r];
+          p = fmaf(sK[i * LK + r], e, p);
+          s = fmaf(sQ[i * LK + r], e, s);
+        }
+      }
+      sP[i * kLC + j] = j < i ? p : 0.f;
+      sA[i * kLC + j] = j <= i ? a.scale * s : 0.f;
+    }
+  }
+  __syncthreads();
+  store_f32(a.Pkk + rec * kC * kC, kC, sP, kLC, kC, kC);
+  store_f32(a.Aqk + rec * kC * kC, kC, sA, kLC, kC, kC);
+
+  // T = (I + diag(beta) P)^-1 (unit lower triangular) by forward substitution
+  // down each column: column j = tid / 4, its 4 lanes split the dot products.
+  {
+    const int j = tid >> 2, s = tid & 3;
+    for (int i = s; i < kC; i += 4) sT[i * kLC + j] = i == j ? 1.f : 0.f;
+    __syncwarp();
+    for (int i = 1; i < kC; ++i) {
+      float part = 0.f;
+      if (i > j)
+        for (int m = j + s; m < i; m += 4) part = fmaf(sP[i * kLC + m], sT[m * kLC + j], part);
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      if (i > j && s == 0) sT[i * kLC + j] = -sb[i] * part;
+      __syncwarp();
+    }
+  }
+  // beta K+ and beta v as the right operands of W and U
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {
+    const int i = idx / DK, r = idx % DK;
+    sX[i * LK + r] *= sb[i] * (slow ? 1.f : se[r]);
+  }
+  load_rows<IO, DV>(sY, LM, static_cast<const IO*>(a.v), row0, a.H, nv, DV, 0, sb);
+  __syncthreads();
+  store_f32(a.Tm + rec * kC * kC, kC, sT, kLC, kC, kC);
+  {
+    using Tl = Tiling<kC, DK>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);
+    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sT, kLC), rowm(sX, LK), m0, n0, kC);
+    float* Wg = a.W + rec * kC * DK;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { Wg[i * DK + c] = acc[mt][nt][e]; });
+  }
+  {
+    using Tl = Tiling<kC, DV>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);
+    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sT, kLC), rowm(sY, LM), m0, n0, kC);
+    float* Ug = a.U + rec * kC * DV;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { Ug[i * DV + c] = acc[mt][nt][e]; });
+  }
+}
+
+
+// ------------------------------------------------------------------ kernel 2
+template <int DK, int DV, int SW>
+constexpr size_t pass_smem() {
+  constexpr int LK = DK + 4, LS = SW + 4;
+  constexpr size_t fwd = (size_t)DK * LS + 2 * kC * LS + 2 * kC * LK + DK;
+  constexpr size_t rev = (size_t)DK * LS + 2 * kC * LS + kC * kLC + 3 * kC * LK + DK;
+  return sizeof(float) * (fwd > rev ? fwd : rev);
+}
+
+// Accumulator tile of an R x SW state block initialised from / stored to a shared tile.
+template <int MT, int NT>
+__device__ __forceinline__ void acc_from(float (&acc)[MT][NT][4], const float* src, int ld, const float* rowf, int m0,
+                                         int n0) {
+  for_acc<MT, NT>(m0, n0, [&](int mt, int nt, int e, int r, int c) { acc[mt][nt][e] = rowf[r] * src[r * ld + c]; });
+}
+
+// One CTA per (sequence, head, SW-column slice of the state) and role:
+// role 0 replays the forward over the chunks from S_0 and stores each chunk's
+// entering state and V'; role 1 walks the chunks backwards from dL/dS_T and
+// stores dL/d(state leaving the chunk) and dV', and writes dL/dS_0.
+template <typename IO, int DK, int DV, int SW>
+__global__ void __launch_bounds__(kThreads, 1) bwd_pass_kernel(const ChunkBwdArgs a) {
+  constexpr bool X3 = std::is_same<IO, float>::value;
+  constexpr int LK = DK + 4, LS = SW + 4, NS = DV / SW;
+  using TV = Tiling<kC, SW>;  // 64 x SW products
+  using TS = Tiling<DK, SW>;  // DK x SW products
+  extern __shared__ __align__(16) float sm[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int cs = blockIdx.x % NS, bh = blockIdx.x / NS, c0 = cs * SW, NC = a.NC;
+  const size_t st0 = (size_t)bh * DK * DV;
+  const int vm0 = TV::m0(warp), vn0 = TV::n0(warp), sm0 = TS::m0(warp), sn0 = TS::n0(warp);
+
+  if (blockIdx.y == 0) {
+    float* sS = sm;              // [DK][LS] state columns
+    float* sV = sS + DK * LS;    // [64][LS] V'
+    float* sU = sV + kC * LS;    // [64][LS] U columns
+    float* sW = sU + kC * LS;    // [64][LK] W
+    float* sKb = sW + kC * LK;   // [64][LK] Kbar
+    float* sgm = sKb + kC * LK;  // [DK] gamma
+    for (int idx = tid; idx < DK * SW; idx += kThreads) {
+      const int r = idx / SW, c = idx % SW;
+      sS[r * LS + c] = a.s0 ? a.s0[st0 + (size_t)r * DV + c0 + c] : 0.f;
+    }
+    for (int n = 0; n < NC; ++n) {
+      const size_t rec = (size_t)bh * NC + n;
+      __syncthreads();
+      store_f32(a.S0c + rec * DK * DV + c0, DV, sS, LS, DK, SW);
+      load_f32(sW, LK, a.W + rec * kC * DK, DK, kC, DK);
+      load_f32(sKb, LK, a.Kb + rec * kC * DK, DK, kC, DK);
+      load_f32(sU, LS, a.U + rec * kC * DV + c0, DV, kC, SW);
+      if (tid < DK) sgm[tid] = a.gam[rec * DK + tid];
+      __syncthreads();
+      {  // V' = U - W S
+        float acc[TV::MT][TV::NT][4];
+        zero(acc);
+        warp_mma<TV::MT, TV::NT, X3>(acc, rowm(sW, LK), rowm(sS, LS), vm0, vn0, DK);
+        float* vp = a.Vp + rec * kC * DV + c0;
+        for_acc<TV::MT, TV::NT>(vm0, vn0, [&](int mt, int nt, int e, int i, int c) {
+          const float x = sU[i * LS + c] - acc[mt][nt][e];
+          sV[i * LS + c] = x;
+          vp[i * DV + c] = x;
+        });
+      }
+      __syncthreads();
+      {  // S = diag(gamma) S + Kbar^T V'
+        float acc[TS::MT][TS::NT][4];
+        acc_from(acc, sS, LS, sgm, sm0, sn0);
+        warp_mma<TS::MT, TS::NT, X3>(acc, colm(sKb, LK), rowm(sV, LS), sm0, sn0, kC);
+        for_acc<TS::MT, TS::NT>(sm0, sn0,
+                                [&](int mt, int nt, int e, int r, int c) { sS[r * LS + c] = acc[mt][nt][e]; });
+      }
+    }
+  } else {
+    float* sD = sm;               // [DK][LS] dS columns
+    float* sdV = sD + DK * LS;    // [64][LS] dV'
+    float* sO = sdV + kC * LS;    // [64][LS] dO columns
+    float* sA = sO + kC * LS;     // [64][kLC] Aqk
+    float* sKb = sA + kC * kLC;   // [64][LK] Kbar
+    float* sQp = sKb + kC * LK;   // [64][LK] Q+
+    float* sW = sQp + kC * LK;    // [64][LK] W
+    float* sgm = sW + kC * LK;    // [DK] gamma
+    for (int idx = tid; idx < DK * SW; idx += kThreads) {
+      const int r = idx / SW, c = idx % SW;
+      sD[r * LS + c] = a.dsT ? a.dsT[st0 + (size_t)r * DV + c0 + c] : 0.f;
+    }
+    for (int n = NC - 1; n >= 0; --n) {
+      const size_t rec = (size_t)bh * NC + n;
+      const int t0 = n * kC, nv = min(kC, a.T - t0);
+      __syncthreads();
+      store_f32(a.dSc + rec * DK * DV + c0, DV, sD, LS, DK, SW);
+      load_f32(sA, kLC, a.Aqk + rec * kC * kC, kC, kC, kC);
+      load_f32(sKb, LK, a.Kb + rec * kC * DK, DK, kC, DK);
+      load_f32(sQp, LK, a.Qp + rec * kC * DK, DK, kC, DK);
+      load_f32(sW, LK, a.W + rec * kC * DK, DK, kC, DK);
+      load_rows<IO, SW>(sO, LS, static_cast<const IO*>(a.d_o), row_of(a, bh, t0), a.H, nv, DV, c0);
+      if (tid < DK) sgm[tid] = a.gam[rec * DK + tid];
+      __syncthreads();
+      {  // dV' = Aqk^T dO + Kbar dS
+        float acc[TV::MT][TV::NT][4];
+        zero(acc);
+        warp_mma<TV::MT, TV::NT, X3>(acc, colm(sA, kLC), rowm(sO, LS), vm0, vn0, kC);
+        warp_mma<TV::MT, TV::NT, X3>(acc, rowm(sKb, LK), rowm(sD, LS), vm0, vn0, DK);
+        float* dvp = a.dVp + rec * kC * DV + c0;
+        for_acc<TV::MT, TV::NT>(vm0, vn0, [&](int mt, int nt, int e, int i, int c) {
+          sdV[i * LS + c] = acc[mt][nt][e];
+          dvp[i * DV + c] = acc[mt][nt][e];
+        });
+      }
+      __syncthreads();
+      {  // dS = diag(gamma) dS + Q+^T dO - W^T dV'
+        float acc[TS::MT][TS::NT][4], neg[TS::MT][TS::NT][4];
+        acc_from(acc, sD, LS, sgm, sm0, sn0);
+        warp_mma<TS::MT, TS::NT, X3>(acc, colm(sQp, LK), rowm(sO, LS), sm0, sn0, kC);
+        zero(neg);
+        warp_mma<TS::MT, TS::NT, X3>(neg, colm(sW, LK), rowm(sdV, LS), sm0, sn0, kC);
+        for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) {
+          sD[r * LS + c] = acc[mt][nt][e] - neg[mt][nt][e];
+        });
+      }
+    }
+    __syncthreads();
+    if (a.ds0) store_f32(a.ds0 + st0 + c0, DV, sD, LS, DK, SW);
+  }
+}
+
+
+// ------------------------------------------------------------------ kernel 3
+template <int DK, int DV>
+constexpr size_t local_a_smem() {
+  constexpr int LV = DV + 4;
+  return sizeof(float) * ((size_t)4 * kC * LV + kC * kLC + 2 * 32 * LV + kC + 2 * kC);
+}
+
+// Per chunk: the products that contract over the value channels.
+template <typename IO, int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwdArgs a) {
+  constexpr bool X3 = std::is_same<IO, float>::value;
+  constexpr int LV = DV + 4;
+  extern __shared__ __align__(16) float sm[];
+  float* sO = sm;              // [64][LV] dO
+  float* sVp = sO + kC * LV;   // [64][LV] V'
+  float* sdV = sVp + kC * LV;  // [64][LV] dV'
+  float* sv = sdV + kC * LV;   // [64][LV] v
+  float* sT = sv + kC * LV;    // [64][kLC] T
+  float* sS0 = sT + kC * kLC;  // [32][LV] rows of S0
+  float* sdS = sS0 + 32 * LV;  // [32][LV] rows of dS
+  float* sb = sdS + 32 * LV;   // [64] beta
+  float* red = sb + kC;        // [2][64] row sums per column group
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % a.NC, bh = blockIdx.x / a.NC, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)bh * a.NC + n;
+
+  load_rows<IO, DV>(sO, LV, static_cast<const IO*>(a.d_o), row0, a.H, nv, DV, 0);
+  load_rows<IO, DV>(sv, LV, static_cast<const IO*>(a.v), row0, a.H, nv, DV, 0);
+  load_f32(sVp, LV, a.Vp + rec * kC * DV, DV, kC, DV);
+  load_f32(sdV, LV, a.dVp + rec * kC * DV, DV, kC, DV);
+  load_f32(sT, kLC, a.Tm + rec * kC * kC, kC, kC, kC);
+  if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const IO*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
+  __syncthreads();
+  {
+    using Tl = Tiling<kC, kC>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);  // dAqk = tril(dO V'^T)
+    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sO, LV), colm(sVp, LV), m0, n0, DV);
+    float* out = a.dAqk + rec * kC * kC;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
+      out[i * kC + j] = j <= i ? acc[mt][nt][e] : 0.f;
+    });
+    zero(acc);  // dU (beta V)^T, strictly lower part
+    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sdV, LV), colm(sv, LV), m0, n0, DV);
+    out = a.dT1 + rec * kC * kC;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
+      out[i * kC + j] = j < i ? acc[mt][nt][e] * sb[j] : 0.f;
+    });
+  }
+  {  // X = T^T dU: dv = beta X, dbeta part = rowsum(V . X)
+    using Tl = Tiling<kC, DV>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4], rp[Tl::MT][2] = {};
+    zero(acc);
+    warp_mma<Tl::MT, Tl::NT, X3>(acc, colm(sT, kLC), rowm(sdV, LV), m0, n0, kC);
+    IO* dv = static_cast<IO*>(a.dv);
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
+      const float x = acc[mt][nt][e];
+      if (i < nv) dv[(row0 + (size_t)i * a.H) * DV + c] = from_f32<IO>(sb[i] * x);
+      rp[mt][e >> 1] = fmaf(x, sv[i * LV + c], rp[mt][e >> 1]);
+    });
+    row_sums_out<Tl::MT>(rp, m0, red + (warp / Tl::WM) * kC);
+  }
+  __syncthreads();
+  if (tid < kC) a.dbu[rec * kC + tid] = red[tid] + red[kC + tid];
+
+  // blocks of 32 key rows of S0 and dS: dO S0^T, -dV' S0^T, V' dS^T, rowsum(dS . S0)
+  using Tr = Tiling<kC, 32>;
+  const int m0 = Tr::m0(warp), n0 = Tr::n0(warp);
+  for (int rb = 0; rb < DK / 32; ++rb) {
+    __syncthreads();
+    load_f32(sS0, LV, a.S0c + rec * DK * DV + (size_t)rb * 32 * DV, DV, 32, DV);
+    load_f32(sdS, LV, a.dSc + rec * DK * DV + (size_t)rb * 32 * DV, DV, 32, DV);
+    __syncthreads();
+    float acc[Tr::MT][Tr::NT][4];
+    zero(acc);
+    warp_mma<Tr::MT, Tr::NT, X3>(acc, rowm(sO, LV), colm(sS0, LV), m0, n0, DV);
+    float* out = a.dQs + rec * kC * DK + rb * 32;
+    for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
+    zero(acc);
+    warp_mma<Tr::MT, Tr::NT, X3>(acc, rowm(sdV, LV), colm(sS0, LV), m0, n0, DV);
+    out = a.dW + rec * kC * DK + rb * 32;
+    for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = -acc[mt][nt][e]; });
+    zero(acc);
+    warp_mma<Tr::MT, Tr::NT, X3>(acc, rowm(sVp, LV), colm(sdS, LV), m0, n0, DV);
+    out = a.dKb + rec * kC * DK + rb * 32;
+    for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {  // warp w: rows 4w .. 4w+3 of the block
+      const int r = 4 * warp + rr;
+      float x = 0.f;
+      for (int c = lane; c < DV; c += 32) x = fmaf(sdS[r * LV + c], sS0[r * LV + c], x);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+      if (lane == 0) a.dgam[rec * DK + rb * 32 + r] = x;
+    }
+  }
+}
+
+
+// ------------------------------------------------------------------ kernel 4
+template <int DK, int DV>
+constexpr size_t local_b_smem() {
+  constexpr int LK = DK + 4;
+  return sizeof(float) * ((size_t)4 * kC * LK + 4 * kC * kLC + kC + 4 * kC + 4 * DK);
+}
+
+// Per chunk: dT, dA, the pairwise gradients and the fold into dq, dk, dg, dbeta.
+template <typename IO, int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwdArgs a) {
+  constexpr bool X3 = std::is_same<IO, float>::value;
+  constexpr int LK = DK + 4;
+  using TK = Tiling<kC, DK>;  // every 64 x d_k product: the same tile per warp
+  using TC = Tiling<kC, kC>;
+  extern __shared__ __align__(16) float sm[];
+  float* sG = sm;               // [64][LK] cumulative log-gates
+  float* sX = sG + kC * LK;     // [64][LK] K+, then K+_r (exact path: k), then dG
+  float* sY = sX + kC * LK;     // [64][LK] dW, then K-_r
+  float* sZ = sY + kC * LK;     // [64][LK] Q+_r (exact path: scale q)
+  float* sT = sZ + kC * LK;     // [64][kLC] T
+  float* sDT = sT + kC * kLC;   // [64][kLC] dT, then M = diag(beta) dA
+  float* sY2 = sDT + kC * kLC;  // [64][kLC] dT T^T
+  float* sQA = sY2 + kC * kLC;  // [64][kLC] dAqk
+  float* sb = sQA + kC * kLC;   // [64] beta
+  float* red = sb + kC;         // [4][64] row sums: K+ . T^T dW (slots 0, 1), dA . P (slots 2, 3)
+  float* colC = red + 4 * kC;   // [4][DK] column sums of dKbar . Kbar per row group
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % a.NC, bh = blockIdx.x / a.NC, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)bh * a.NC + n;
+  const IO* q = static_cast<const IO*>(a.q);
+  const IO* k = static_cast<const IO*>(a.k);
+  const int m0 = TK::m0(warp), n0 = TK::n0(warp), cm0 = TC::m0(warp), cn0 = TC::n0(warp);
+  float dk_acc[TK::MT][TK::NT][4], dG_acc[TK::MT][TK::NT][4];
+  zero(dk_acc);
+  zero(dG_acc);
+
+  if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const IO*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
+  load_gates_cumsum<IO, DK>(sG, LK, static_cast<const IO*>(a.g), a.gate, row0, a.H, nv);
+  const bool slow = chunk_unsafe<DK>(sG, LK);
+  load_rows<IO, DK>(sX, LK, k, row0, a.H, nv, DK, 0);
+  load_f32(sY, LK, a.dW + rec * kC * DK, DK, kC, DK);
+  load_f32(sT, kLC, a.Tm + rec * kC * kC, kC, kC, kC);
+  load_f32(sDT, kLC, a.dT1 + rec * kC * kC, kC, kC, kC);
+  __syncthreads();
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {
+    const int i = idx / DK, r = idx % DK;
+    sX[i * LK + r] *= expf(sG[i * LK + r]);
+  }
+  __syncthreads();
+  {  // dT += dW (beta K+)^T, strictly lower part
+    float acc[TC::MT][TC::NT][4];
+    zero(acc);
+    warp_mma<TC::MT, TC::NT, X3>(acc, rowm(sY, LK), colm(sX, LK), cm0, cn0, DK);
+    for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
+      if (j < i) sDT[i * kLC + j] += acc[mt][nt][e] * sb[j];
+    });
+  }
+  {  // X = T^T dW: dK+ = beta X; dbeta part rowsum(K+ . X)
+    float acc[TK::MT][TK::NT][4], rp[TK::MT][2] = {};
+    zero(acc);
+    warp_mma<TK::MT, TK::NT, X3>(acc, colm(sT, kLC), rowm(sY, LK), m0, n0, kC);
+    for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+      const float x = acc[mt][nt][e], kp = sX[i * LK + r], bx = sb[i] * x;
+      dk_acc[mt][nt][e] = fmaf(bx, expf(sG[i * LK + r]), dk_acc[mt][nt][e]);
+      dG_acc[mt][nt][e] = fmaf(bx, kp, dG_acc[mt][nt][e]);
+      rp[mt][e >> 1] = fmaf(x, kp, rp[mt][e >> 1]);
+    });
+    row_sums_out<TK::MT>(rp, m0, red + (warp / TK::WM) * kC);
+  }
+  __syncthreads();
+  {  // dT T^T
+    float acc[TC::MT][TC::NT][4];
+    zero(acc);
+    warp_mma<TC::MT, TC::NT, X3>(acc, rowm(sDT, kLC), colm(sT, kLC), cm0, cn0, kC);
+    for_acc<TC::MT, TC::NT>(cm0, cn0,
+                            [&](int mt, int nt, int e, int i, int j) { sY2[i * kLC + j] = acc[mt][nt][e]; });
+  }
+  __syncthreads();
+  {  // dA = -T^T (dT T^T), strictly lower; dbeta part rowsum(dA . P); M = diag(beta) dA
+    float acc[TC::MT][TC::NT][4], rp[TC::MT][2] = {};
+    zero(acc);
+    warp_mma<TC::MT, TC::NT, X3>(acc, colm(sT, kLC), rowm(sY2, kLC), cm0, cn0, kC);
+    const float* P = a.Pkk + rec * kC * kC;
+    for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
+      const float d = j < i ? -acc[mt][nt][e] : 0.f;
+      rp[mt][e >> 1] = fmaf(d, P[i * kC + j], rp[mt][e >> 1]);
+      sDT[i * kLC + j] = sb[i] * d;
+    });
+    row_sums_out<TC::MT>(rp, cm0, red + (2 + warp / TC::WM) * kC);
+  }
+  // operands of the pairwise gradients
+  load_f32(sQA, kLC, a.dAqk + rec * kC * kC, kC, kC, kC);
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {
+    const int i = idx / DK, r = idx % DK;
+    const size_t o = (row0 + (size_t)i * a.H) * DK + r;
+    const float kk = i < nv ? to_f32(k[o]) : 0.f, qq = i < nv ? a.scale * to_f32(q[o]) : 0.f;
+    if (!slow) {
+      const float d = sG[i * LK + r] - sG[kRef * LK + r], ex = expf(d);
+      sX[i * LK + r] = kk * ex;
+      sY[i * LK + r] = kk * expf(-d);
+      sZ[i * LK + r] = qq * ex;
+    } else {
+      sX[i * LK + r] = kk;
+      sZ[i * LK + r] = qq;
+    }
+  }
+  __syncthreads();
+  const float* dQs = a.dQs + rec * kC * DK;
+  const float* Qp = a.Qp + rec * kC * DK;
+  IO* dq = static_cast<IO*>(a.dq);
+  if (!slow) {
+    {  // dQ+_r = dAqk K-_r;  dq = scale (exp(G - G_ref) dQ+_r + Gamma dO S0^T)
+      float acc[TK::MT][TK::NT][4];
+      zero(acc);
+      warp_mma<TK::MT, TK::NT, X3>(acc, rowm(sQA, kLC), rowm(sY, LK), m0, n0, kC);
+      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+        const float x = acc[mt][nt][e], G = sG[i * LK + r];
+        const float ex = expf(G - sG[kRef * LK + r]), dqs = dQs[i * DK + r];
+        if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = from_f32<IO>(a.scale * fmaf(ex, x, expf(G) * dqs));
+        dG_acc[mt][nt][e] += fmaf(x, sZ[i * LK + r], dqs * Qp[i * DK + r]);
+      });
+    }
+    {  // dK-_r = dAqk^T Q+_r + M^T K+_r
+      float acc[TK::MT][TK::NT][4];
+      zero(acc);
+      warp_mma<TK::MT, TK::NT, X3>(acc, colm(sQA, kLC), rowm(sZ, LK), m0, n0, kC);
+      warp_mma<TK::MT, TK::NT, X3>(acc, colm(sDT, kLC), rowm(sX, LK), m0, n0, kC);
+      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+        const float x = acc[mt][nt][e];
+        dk_acc[mt][nt][e] = fmaf(expf(sG[kRef * LK + r] - sG[i * LK + r]), x, dk_acc[mt][nt][e]);
+        dG_acc[mt][nt][e] = fmaf(-x, sY[i * LK + r], dG_acc[mt][nt][e]);
+      });
+    }
+    {  // dK+_r = M K-_r
+      float acc[TK::MT][TK::NT][4];
+      zero(acc);
+      warp_mma<TK::MT, TK::NT, X3>(acc, rowm(sDT, kLC), rowm(sY, LK), m0, n0, kC);
+      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+        const float x = acc[mt][nt][e];
+        dk_acc[mt][nt][e] = fmaf(expf(sG[i * LK + r] - sG[kRef * LK + r]), x, dk_acc[mt][nt][e]);
+        dG_acc[mt][nt][e] = fmaf(x, sX[i * LK + r], dG_acc[mt][nt][e]);
+      });
+    }
+  } else {
+    // exact pairwise terms, E = exp(G_ir - G_jr) for j <= i:
+    //   Aqk_ij = sum_r (scale q_ir) k_jr E,  P_ij = sum_r k_ir k_jr E
+    for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+      const float Gi = sG[i * LK + r], ki = sX[i * LK + r], qi = sZ[i * LK + r];
+      float dqp = 0.f, dkp = 0.f, dgp = 0.f;
+      for (int j = 0; j <= i; ++j) {  // row i of dAqk and M: i is the left factor
+        const float kE = expf(Gi - sG[j * LK + r]) * sX[j * LK + r];
+        const float c = sQA[i * kLC + j], m = sDT[i * kLC + j];
+        dqp = fmaf(c, kE, dqp);
+        dkp = fmaf(m, kE, dkp);
+        dgp = fmaf(fmaf(c, qi, m * ki), kE, dgp);
+      }
+      for (int j = i; j < kC; ++j) {  // column i of dAqk and M: i is the right factor
+        const float w =
+            fmaf(sQA[j * kLC + i], sZ[j * LK + r], sDT[j * kLC + i] * sX[j * LK + r]) * expf(sG[j * LK + r] - Gi);
+        dkp += w;
+        dgp = fmaf(-w, ki, dgp);
+      }
+      const float dqs = dQs[i * DK + r];
+      if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = from_f32<IO>(a.scale * fmaf(expf(Gi), dqs, dqp));
+      dk_acc[mt][nt][e] += dkp;
+      dG_acc[mt][nt][e] += fmaf(dqs, Qp[i * DK + r], dgp);
+    });
+  }
+  {  // Kbar: dk += exp(G_C - G) dKbar, dG -= dKbar . Kbar, dG_C += column sums of the same
+    const float* dKb = a.dKb + rec * kC * DK;
+    const float* Kb = a.Kb + rec * kC * DK;
+    float cp[TK::MT][TK::NT][2] = {};
+    for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+      const float x = dKb[i * DK + r], y = x * Kb[i * DK + r];
+      dk_acc[mt][nt][e] = fmaf(expf(sG[(kC - 1) * LK + r] - sG[i * LK + r]), x, dk_acc[mt][nt][e]);
+      dG_acc[mt][nt][e] -= y;
+      cp[mt][nt][e & 1] += y;
+    });
+#pragma unroll
+    for (int nt = 0; nt < TK::NT; ++nt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float x = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < TK::MT; ++mt) x += cp[mt][nt][c];
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        x += __shfl_xor_sync(0xffffffffu, x, 8);
+        x += __shfl_xor_sync(0xffffffffu, x, 16);
+        if (lane < 4) colC[(warp % TK::WM) * DK + n0 + 8 * nt + 2 * lane + c] = x;
+      }
+  }
+  IO* dk = static_cast<IO*>(a.dk);
+  for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+    if (i < nv) dk[(row0 + (size_t)i * a.H) * DK + r] = from_f32<IO>(dk_acc[mt][nt][e]);
+  });
+  __syncthreads();  // sX is no longer read: it takes dG
+  for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) { sX[i * LK + r] = dG_acc[mt][nt][e]; });
+  __syncthreads();
+  if (tid < DK) {  // dG_C terms, then dg = reverse cumsum of dG over the chunk
+    const int r = tid;
+    float x = colC[r] + colC[DK + r] + colC[2 * DK + r] + colC[3 * DK + r];
+    x = fmaf(expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
+    float acc = x;
+    for (int i = kC - 1; i >= 0; --i) {
+      acc += sX[i * LK + r];
+      sX[i * LK + r] = acc;
+    }
+  }
+  __syncthreads();
+  if (a.gate == KDA_GATE_CHANNEL) {
+    IO* dg = static_cast<IO*>(a.dg);
+    for (int idx = tid; idx < nv * DK; idx += kThreads) {
+      const int i = idx / DK, r = idx % DK;
+      dg[(row0 + (size_t)i * a.H) * DK + r] = from_f32<IO>(sX[i * LK + r]);
+    }
+  } else if (a.gate == KDA_GATE_HEAD) {
+    IO* dg = static_cast<IO*>(a.dg);
+    for (int i = warp; i < nv; i += kThreads / 32) {
+      float x = 0.f;
+      for (int r = lane; r < DK; r += 32) x += sX[i * LK + r];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+      if (lane == 0) dg[row0 + (size_t)i * a.H] = from_f32<IO>(x);
+    }
+  }
+  if (tid < nv)
+    static_cast<IO*>(a.dbeta)[row0 + (size_t)tid * a.H] =
+        from_f32<IO>(((a.dbu[rec * kC + tid] + red[tid]) + red[kC + tid]) + (red[2 * kC + tid] + red[3 * kC + tid]));
+}
+
+
+// ------------------------------------------------------------------ host
+// Floats of each workspace array per chunk record, in layout order.
+struct WsPlan {
+  size_t W, U, Qp, Kb, Aqk, Tm, Pkk, gam, S0c, dSc, Vp, dVp, dAqk, dT1, dQs, dW, dKb, dgam, dbu;
+  explicit WsPlan(int dk, int dv)
+      : W((size_t)kC * dk), U((size_t)kC * dv), Qp((size_t)kC * dk), Kb((size_t)kC * dk), Aqk(kC * kC),
+        Tm(kC * kC), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv), dSc((size_t)dk * dv), Vp((size_t)kC * dv),
+        dVp((size_t)kC * dv), dAqk(kC * kC), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk),
+        dKb((size_t)kC * dk), dgam(dk), dbu(kC) {}
+  size_t per_rec() const {
+    return W + U + Qp + Kb + Aqk + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs + dW + dKb + dgam + dbu;
+  }
+};
+
+// State columns per pass CTA: 32 while the 2 x (B H) x (d_v / 32) CTAs fit
+// in one wave of the 148 SMs, else 64 (fewer CTAs reading the same operands).
+int pass_width(int BH, int dv) { return (size_t)2 * BH * (dv / 32) <= 148 ? 32 : 64; }
+
+template <typename Kern>
+cudaError_t launch_k(Kern kern, dim3 grid, size_t smem, const ChunkBwdArgs& a, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename IO, int DK, int DV>
+cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t stream) {
+  const dim3 grid((unsigned)a.NC * BH);  // chunk-major within each (sequence, head)
+  cudaError_t e = launch_k(bwd_prep_kernel<IO, DK, DV>, grid, prep_smem<DK, DV>(), a, stream);
+  if (e != cudaSuccess) return e;
+  if (pass_width(BH, DV) == 32)
+    e = launch_k(bwd_pass_kernel<IO, DK, DV, 32>, dim3(BH * (DV / 32), 2), pass_smem<DK, DV, 32>(), a, stream);
+  else
+    e = launch_k(bwd_pass_kernel<IO, DK, DV, 64>, dim3(BH * (DV / 64), 2), pass_smem<DK, DV, 64>(), a, stream);
+  if (e != cudaSuccess) return e;
+  e = launch_k(bwd_local_a_kernel<IO, DK, DV>, grid, local_a_smem<DK, DV>(), a, stream);
+  if (e != cudaSuccess) return e;
+  return launch_k(bwd_local_b_kernel<IO, DK, DV>, grid, local_b_smem<DK, DV>(), a, stream);
+}
+
+template <typename IO>
+cudaError_t launch_chunk_dims(const ChunkBwdArgs& a, int BH, int dk, int dv, cudaStream_t stream) {
+  if (dk == 128 && dv == 128) return launch_chunk_typed<IO, 128, 128>(a, BH, stream);
+  if (dk == 128 && dv == 64) return launch_chunk_typed<IO, 128, 64>(a, BH, stream);
+  if (dk == 64 && dv == 128) return launch_chunk_typed<IO, 64, 128>(a, BH, stream);
+  return launch_chunk_typed<IO, 64, 64>(a, BH, stream);
+}
+
+static_assert(prep_smem<128, 128>() <= 232448 && local_a_smem<128, 128>() <= 232448 &&
+                  local_b_smem<128, 128>() <= 232448 && pass_smem<128, 128, 64>() <= 232448,
+              "shared memory per CTA");
+
+}  // namespace
+
+size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  const size_t nrec = (size_t)B * H * (((size_t)T + kC - 1) / kC);
+  return nrec * WsPlan(dk, dv).per_rec() * sizeof(float);
+}
+
+int backward_launches() { return 4; }
+
+cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                            float scale, const float* s0, const void* d_o, const float* dsT, void* dq, void* dk_out,
+                            void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H, int dk, int dv,
+                            int dtype, int gate, void* ws, cudaStream_t stream) {
+  ChunkBwdArgs a;
+  a.q = q, a.k = k, a.v = v, a.g = g, a.beta = beta, a.d_o = d_o;
+  a.s0 = s0, a.dsT = dsT;
+  a.dq = dq, a.dk = dk_out, a.dv = dv_out, a.dg = dg, a.dbeta = dbeta, a.ds0 = ds0;
+  a.scale = scale, a.T = T, a.H = H, a.NC = (T + kC - 1) / kC, a.gate = gate;
+  const size_t nrec = (size_t)B * H * a.NC;
+  const WsPlan p(dk, dv);
+  float* w = static_cast<float*>(ws);
+  auto take = [&](size_t per) {
+    float* r = w;
+    w += nrec * per;
+    return r;
+  };
+  a.W = take(p.W), a.U = take(p.U), a.Qp = take(p.Qp), a.Kb = take(p.Kb);
+  a.Aqk = take(p.Aqk), a.Tm = take(p.Tm), a.Pkk = take(p.Pkk), a.gam = take(p.gam);
+  a.S0c = take(p.S0c), a.dSc = take(p.dSc), a.Vp = take(p.Vp), a.dVp = take(p.dVp);
+  a.dAqk = take(p.dAqk), a.dT1 = take(p.dT1), a.dQs = take(p.dQs), a.dW = take(p.dW), a.dKb = take(p.dKb);
+  a.dgam = take(p.dgam), a.dbu = take(p.dbu);
+  if (dtype == KDA_F32) return launch_chunk_dims<float>(a, B * H, dk, dv, stream);
+  return launch_chunk_dims<__nv_bfloat16>(a, B * H, dk, dv, stream);
+}
+
+}  // namespace kda

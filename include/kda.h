@@ -158,18 +158,25 @@ KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Bytes of device workspace kda_backward needs for this problem (fp32 state
- * checkpoints every 16 tokens plus a 16-state scratch per (sequence, head));
- * 0 for arguments kda_backward would reject.
+ * Bytes of device workspace kda_backward needs for this problem: fp32
+ * per-chunk records (per 64-token chunk and head: the chunk's operands, the
+ * state entering it and the state gradient leaving it, and intermediate
+ * gradients; about 0.5 MB at dk = dv = 128); 0 for arguments kda_backward
+ * would reject.
  */
 KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
 
 /*
  * Backward pass: gradients of a scalar loss L through the forward pass
  * (kda_chunk_fwd, or kda_chunk_fwd_ex with `gate` and KDA_PREP_NONE), given
- * dL/do and dL/dS_T.  Reverse-mode differentiation of the token-by-token
- * recurrence of the KimiLinear article, section 2.3 (sections 2.1-2.2 for the
- * scalar gates), evaluated in fp32 token by token (not chunkwise).
+ * dL/do and dL/dS_T.  Reverse-mode differentiation of the chunkwise form
+ * (KimiLinear article, section 2.3 for the recurrence, sections 3.1-3.2 for
+ * the chunks; sections 2.1-2.2 for the scalar gates): a per-chunk
+ * recomputation of the chunk operands, a forward replay of the chunk states
+ * and a reverse sweep of the state gradient (each column of the state on its
+ * own), then per-chunk local gradients.  Four kernel launches; fp32 storage
+ * and accumulation, tensor-core products with tf32 operands (three-term
+ * split, i.e. fp32-level accuracy, when dtype is KDA_F32).
  *
  *   q, k, v, g, beta, scale, initial_state : the forward's inputs (layouts
  *                      and gate kinds as for kda_chunk_fwd_ex)
@@ -187,8 +194,8 @@ KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, 
  * Supported: dtype KDA_F32 or KDA_BF16, dk and dv in {64, 128}.  Pointers
  * 16-byte aligned (beta, grad_beta and per-head g / grad_g: element
  * alignment); outputs must not overlap any input, each other or the
- * workspace.  The per-token sums over value channels are added in a fixed
- * order, so results are bit-reproducible.  T = 0 or B = 0 is valid
+ * workspace.  Every sum runs in a fixed order (no atomics), so results are
+ * bit-reproducible.  T = 0 or B = 0 is valid
  * (grad_initial_state = grad_final_state).
  */
 KDA_API kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,

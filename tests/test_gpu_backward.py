@@ -43,11 +43,11 @@ def _case(B, T, H, dk, dv, dtype, gate="channel", s0=0.1, final=True, seed=90):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
 @pytest.mark.parametrize("B,T,H,dk,dv", [(1, 37, 2, 128, 128), (2, 100, 3, 64, 64), (1, 64, 1, 128, 64),
-                                         (1, 64, 1, 64, 128), (1, 1, 1, 128, 128), (1, 16, 2, 128, 128),
-                                         (1, 17, 2, 128, 128)])
+                                         (1, 64, 1, 64, 128), (1, 1, 1, 128, 128), (1, 65, 2, 128, 128),
+                                         (1, 200, 2, 128, 128), (2, 130, 3, 64, 128), (1, 129, 2, 128, 64)])
 def test_backward_shapes(dtype, B, T, H, dk, dv):
-    """Several windows and ragged tails (16-token windows, 4-token reduction
-    steps), a single token, every supported (dk, dv)."""
+    """One and several 64-token chunks with ragged tails (65 tokens: a
+    one-token tail), a single token, every supported (dk, dv)."""
     _case(B, T, H, dk, dv, dtype, seed=91 + T)
 
 
@@ -77,8 +77,36 @@ def test_backward_deterministic():
         assert torch.equal(a[n], b[n]), n
 
 
-@pytest.mark.parametrize("B,H", [(5, 8), (10, 8)], ids=["2-way-split", "no-split"])
-def test_backward_column_splits(B, H):
-    """Few (sequence, head) pairs split each head's value columns over 4 CTAs
-    (covered above); 40 pairs split in 2, 80 pairs not at all."""
-    _case(B, 40, H, 128, 128, torch.float32, seed=97 + B)
+@pytest.mark.parametrize("B,H", [(2, 8), (5, 8)], ids=["32-columns", "64-columns"])
+def test_backward_pass_widths(B, H):
+    """The state passes give each CTA 32 value columns while 2 x B H x d_v/32
+    CTAs fit in one wave of 148 SMs (16 pairs), else 64 (40 pairs)."""
+    _case(B, 200, H, 128, 128, torch.float32, seed=97 + B)
+
+
+def _extreme_gates(x, dtype):
+    """Per-channel log-gates with chunks whose cumulative decay leaves the
+    factored operands' safe span (|G_i - G_31| > 64): -4 per token in half
+    of the channels of the second chunk, -80 at one token of the fourth."""
+    g = x["g"].clone().float()
+    g[:, 64:128, :, ::2] = -4.0
+    g[:, 200, :, 5] = -80.0
+    x["g"] = g.to(dtype)
+    return x
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_backward_exact_pairwise_path(dtype):
+    """Chunks past the factored form's span take the exact per-element path;
+    the others in the same call keep the tensor-core path."""
+    dev = cuda_or_skip()
+    B, T, H, dk, dv = 1, 230, 2, 128, 128
+    x = _extreme_gates(make_prefill_inputs(B, T, H, dk, dv, dtype, 0.1, seed=98), dtype)
+    d_o, d_s = make_cotangents(B, T, H, dk, dv, dtype, seed=99)
+    to = lambda t: t.to(dev)
+    got = kda_backward(to(x["q"]), to(x["k"]), to(x["v"]), to(x["g"]), to(x["beta"]), to(d_o), dk ** -0.5,
+                       to(x["initial_state"]), to(d_s))
+    torch.cuda.synchronize()
+    ref = oracle.kda_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dk ** -0.5, x["initial_state"], d_o, d_s)
+    for name in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        assert rel_err(got[name], ref[name]) < TOL[dtype], (name, rel_err(got[name], ref[name]))
