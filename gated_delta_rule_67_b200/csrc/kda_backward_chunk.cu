@@ -51,7 +51,9 @@ namespace {
 constexpr int kC = 64;          // tokens per chunk
 constexpr int kRef = 31;        // reference token of the factored pairwise operands
 constexpr float kSpan = 64.f;   // factored operands need |G_i - G_ref| <= kSpan in every channel
-constexpr int kThreads = 256;   // 8 warps in every kernel
+constexpr int kThreads = 512;   // 16 warps in the per-chunk kernels
+constexpr int kWarps = kThreads / 32;
+constexpr int kPassThreads = 256;  // 8 warps in the state passes (longer tiles, fewer loads per MMA)
 constexpr int kLC = kC + 4;     // leading dimension of the C x C shared tiles
 
 // ------------------------------------------------------------------ warp MMA
@@ -81,10 +83,10 @@ __device__ __forceinline__ View colm(const float* p, int ld) { return View{p, 1,
 // Fragment layout of mma.m16n8k8: g = lane / 4, t = lane % 4; A holds (g, t),
 // (g+8, t), (g, t+4), (g+8, t+4); B holds (t, g), (t+4, g); the accumulator
 // holds rows g, g+8 and columns 2t, 2t+1.  X3: three-term tf32 split.
-template <int MT, int NT, bool X3>
-__device__ __forceinline__ void warp_mma(float (&acc)[MT][NT][4], View A, View B, int m0, int n0, int K) {
+template <int MT, int NT, bool X3, int K>
+__device__ __forceinline__ void warp_mma(float (&acc)[MT][NT][4], View A, View B, int m0, int n0) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-#pragma unroll 2
+#pragma unroll
   for (int k0 = 0; k0 < K; k0 += 8) {
     uint32_t ah[MT][4], al[MT][4], bh[NT][2], bl[NT][2];
 #pragma unroll
@@ -120,14 +122,14 @@ __device__ __forceinline__ void warp_mma(float (&acc)[MT][NT][4], View A, View B
   }
 }
 
-// Split of an R x N output over the 8 warps: WM x WN warps, each (16 MT) x (8 NT).
-template <int R, int N>
+// Split of an R x N output over NW warps: WM x WN warps, each (16 MT) x (8 NT).
+template <int R, int N, int NW = kWarps>
 struct Tiling {
-  static constexpr int WM = (R / 16 >= 8) ? 8 : R / 16;
-  static constexpr int WN = 8 / WM;
+  static constexpr int WM = (R / 16 >= NW) ? NW : R / 16;
+  static constexpr int WN = NW / WM;
   static constexpr int MT = R / 16 / WM;
   static constexpr int NT = N / 8 / WN;
-  static_assert(WM * WN == 8 && MT * 16 * WM == R && NT * 8 * WN == N, "tiling");
+  static_assert(WM * WN == NW && MT * 16 * WM == R && NT * 8 * WN == N, "tiling");
   __device__ static int m0(int warp) { return (warp % WM) * MT * 16; }
   __device__ static int n0(int warp) { return (warp / WM) * NT * 8; }
 };
@@ -179,48 +181,62 @@ template <typename IO, int W>
 __device__ __forceinline__ void load_rows(float* dst, int ld, const IO* src, size_t row0, int H, int nv, int len,
                                           int col0, const float* mult = nullptr) {
   constexpr int V = 16 / sizeof(IO);  // elements per 16-byte load
-  constexpr int PER_ROW = W / V;
-  for (int idx = threadIdx.x; idx < kC * PER_ROW; idx += kThreads) {
-    const int i = idx / PER_ROW, c = (idx % PER_ROW) * V;
+  constexpr int PER_ROW = W / V, N = kC * PER_ROW, IT = (N + kThreads - 1) / kThreads;
+  uint4 w[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {  // all loads in flight before the first store
+    const int idx = threadIdx.x + it * kThreads, i = idx / PER_ROW, c = (idx % PER_ROW) * V;
+    w[it] = (idx < N && i < nv) ? __ldg(reinterpret_cast<const uint4*>(src + (row0 + (size_t)i * H) * len + col0 + c))
+                                : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int idx = threadIdx.x + it * kThreads, i = idx / PER_ROW, c = (idx % PER_ROW) * V;
+    if (idx >= N) break;
     float x[V];
-    if (i < nv) {
-      const uint4 w = *reinterpret_cast<const uint4*>(src + (row0 + (size_t)i * H) * len + col0 + c);
-      if constexpr (std::is_same<IO, float>::value) {
-        x[0] = __uint_as_float(w.x), x[1] = __uint_as_float(w.y), x[2] = __uint_as_float(w.z),
-        x[3] = __uint_as_float(w.w);
-      } else {
-        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
-          x[2 * e] = f.x, x[2 * e + 1] = f.y;
-        }
-      }
-      if (mult) {
-        const float m = mult[i];
-#pragma unroll
-        for (int e = 0; e < V; ++e) x[e] *= m;
-      }
+    if constexpr (std::is_same<IO, float>::value) {
+      x[0] = __uint_as_float(w[it].x), x[1] = __uint_as_float(w[it].y), x[2] = __uint_as_float(w[it].z),
+      x[3] = __uint_as_float(w[it].w);
     } else {
+      const uint32_t u[4] = {w[it].x, w[it].y, w[it].z, w[it].w};
 #pragma unroll
-      for (int e = 0; e < V; ++e) x[e] = 0.f;
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+        x[2 * e] = f.x, x[2 * e + 1] = f.y;
+      }
+    }
+    if (mult) {
+      const float m = mult[i];
+#pragma unroll
+      for (int e = 0; e < V; ++e) x[e] *= m;
     }
 #pragma unroll
     for (int e = 0; e < V; e += 4)
       *reinterpret_cast<float4*>(dst + i * ld + c + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
   }
 }
-// fp32 rows x cols block from global (leading dimension gld) into shared (ld); cols % 4 == 0.
+// Asynchronous 16-byte copies global -> shared (cp.async); cp_wait() waits
+// for all of this thread's copies, a barrier then publishes them.
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// fp32 rows x cols block from global (leading dimension gld) into shared (ld),
+// cols % 4 == 0, by cp.async: complete after cp_wait().
+template <int NTH = kThreads>
 __device__ __forceinline__ void load_f32(float* dst, int ld, const float* src, int gld, int rows, int cols) {
   const int per = cols / 4;
-  for (int idx = threadIdx.x; idx < rows * per; idx += kThreads) {
+  for (int idx = threadIdx.x; idx < rows * per; idx += NTH) {
     const int i = idx / per, c = (idx % per) * 4;
-    *reinterpret_cast<float4*>(dst + i * ld + c) = *reinterpret_cast<const float4*>(src + (size_t)i * gld + c);
+    cp_async16(dst + i * ld + c, src + (size_t)i * gld + c);
   }
 }
+template <int NTH = kThreads>
 __device__ __forceinline__ void store_f32(float* dst, int gld, const float* src, int ld, int rows, int cols) {
   const int per = cols / 4;
-  for (int idx = threadIdx.x; idx < rows * per; idx += kThreads) {
+  for (int idx = threadIdx.x; idx < rows * per; idx += NTH) {
     const int i = idx / per, c = (idx % per) * 4;
     *reinterpret_cast<float4*>(dst + (size_t)i * gld + c) = *reinterpret_cast<const float4*>(src + i * ld + c);
   }
@@ -242,11 +258,13 @@ __device__ __forceinline__ void load_gates_cumsum(float* sG, int ld, const IO* g
   }
   __syncthreads();
   if (threadIdx.x < DK) {
-    float acc = 0.f;
-    for (int i = 0; i < kC; ++i) {
-      acc += sG[i * ld + threadIdx.x];
-      sG[i * ld + threadIdx.x] = acc;
-    }
+    float x[kC];
+#pragma unroll
+    for (int i = 0; i < kC; ++i) x[i] = sG[i * ld + threadIdx.x];
+#pragma unroll
+    for (int i = 1; i < kC; ++i) x[i] += x[i - 1];
+#pragma unroll
+    for (int i = 0; i < kC; ++i) sG[i * ld + threadIdx.x] = x[i];
   }
   __syncthreads();
 }
@@ -351,12 +369,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);
-    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sX, LK), colm(sY, LK), m0, n0, DK);
+    warp_mma<Tl::MT, Tl::NT, X3, DK>(acc, rowm(sX, LK), colm(sY, LK), m0, n0);
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       sP[i * kLC + j] = j < i ? acc[mt][nt][e] : 0.f;
     });
     zero(acc);
-    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sQ, LK), colm(sY, LK), m0, n0, DK);
+    warp_mma<Tl::MT, Tl::NT, X3, DK>(acc, rowm(sQ, LK), colm(sY, LK), m0, n0);
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       sA[i * kLC + j] = j <= i ? acc[mt][nt][e] : 0.f;
     });
@@ -380,19 +398,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
   store_f32(a.Aqk + rec * kC * kC, kC, sA, kLC, kC, kC);
 
   // T = (I + diag(beta) P)^-1 (unit lower triangular) by forward substitution
-  // down each column: column j = tid / 4, its 4 lanes split the dot products.
-  {
-    const int j = tid >> 2, s = tid & 3;
-    for (int i = s; i < kC; i += 4) sT[i * kLC + j] = i == j ? 1.f : 0.f;
-    __syncwarp();
-    for (int i = 1; i < kC; ++i) {
-      float part = 0.f;
-      if (i > j)
-        for (int m = j + s; m < i; m += 4) part = fmaf(sP[i * kLC + m], sT[m * kLC + j], part);
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      part += __shfl_xor_sync(0xffffffffu, part, 2);
-      if (i > j && s == 0) sT[i * kLC + j] = -sb[i] * part;
-      __syncwarp();
+  // down each column: thread j < 64 keeps column j in registers; row i reads
+  // P[i][0..i) as broadcast 16-byte loads (fully unrolled: 2016 FMAs).
+  if (tid < kC) {
+    const int j = tid;
+    float tc[kC];
+#pragma unroll
+    for (int i = 0; i < kC; ++i) {
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int m = 0; m < i; m += 4) {
+        const float4 p = *reinterpret_cast<const float4*>(sP + i * kLC + m);
+        s4[0] = fmaf(p.x, tc[m], s4[0]);
+        if (m + 1 < i) s4[1] = fmaf(p.y, tc[m + 1], s4[1]);
+        if (m + 2 < i) s4[2] = fmaf(p.z, tc[m + 2], s4[2]);
+        if (m + 3 < i) s4[3] = fmaf(p.w, tc[m + 3], s4[3]);
+      }
+      tc[i] = i == j ? 1.f : (i < j ? 0.f : -sb[i] * ((s4[0] + s4[1]) + (s4[2] + s4[3])));
+      sT[i * kLC + j] = tc[i];
     }
   }
   // beta K+ and beta v as the right operands of W and U
@@ -408,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);
-    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sT, kLC), rowm(sX, LK), m0, n0, kC);
+    warp_mma<Tl::MT, Tl::NT, X3, kC>(acc, rowm(sT, kLC), rowm(sX, LK), m0, n0);
     float* Wg = a.W + rec * kC * DK;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { Wg[i * DK + c] = acc[mt][nt][e]; });
   }
@@ -417,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);
-    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sT, kLC), rowm(sY, LM), m0, n0, kC);
+    warp_mma<Tl::MT, Tl::NT, X3, kC>(acc, rowm(sT, kLC), rowm(sY, LM), m0, n0);
     float* Ug = a.U + rec * kC * DV;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { Ug[i * DV + c] = acc[mt][nt][e]; });
   }
@@ -425,15 +448,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
 
 
 // ------------------------------------------------------------------ kernel 2
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Shared-memory plan of the pass kernel (floats).  Role 0 keeps the state
+// columns and V' and NB0 buffers of {W, Kbar, U columns, gamma}; role 1 keeps
+// dS, dV', dO, Q+, W and NB1 buffers of {Aqk, Kbar, gamma, raw dO columns}.  Two buffers
+// (the next chunk's operands load while this one computes) where they fit.
+template <int DK, int DV, int SW>
+struct PassPlan {
+  static constexpr int LK = DK + 4, LS = SW + 4;
+  static constexpr size_t kMax = 232448 / sizeof(float);
+  static constexpr size_t fix0 = (size_t)DK * LS + kC * LS, buf0 = 2 * (size_t)kC * LK + kC * LS + DK;
+  static constexpr size_t fix1 = (size_t)DK * LS + 2 * kC * LS + 2 * (size_t)kC * LK;
+  static constexpr size_t stage1 = (size_t)kC * SW * 4 / sizeof(float);  // raw dO columns, up to 4 bytes each
+  static constexpr size_t buf1 = (size_t)kC * kLC + kC * LK + DK + stage1;
+  static constexpr int NB0 = fix0 + 2 * buf0 <= kMax ? 2 : 1;
+  static constexpr int NB1 = fix1 + 2 * buf1 <= kMax ? 2 : 1;
+  static constexpr size_t r0 = fix0 + NB0 * buf0, r1 = fix1 + NB1 * buf1;
+  static constexpr size_t bytes = sizeof(float) * (r0 > r1 ? r0 : r1);
+};
 template <int DK, int DV, int SW>
 constexpr size_t pass_smem() {
-  constexpr int LK = DK + 4, LS = SW + 4;
-  constexpr size_t fwd = (size_t)DK * LS + 2 * kC * LS + 2 * kC * LK + DK;
-  constexpr size_t rev = (size_t)DK * LS + 2 * kC * LS + kC * kLC + 3 * kC * LK + DK;
-  return sizeof(float) * (fwd > rev ? fwd : rev);
+  return PassPlan<DK, DV, SW>::bytes;
 }
 
-// Accumulator tile of an R x SW state block initialised from / stored to a shared tile.
+// Accumulator tile of an R x SW state block initialised from a shared tile, rows scaled.
 template <int MT, int NT>
 __device__ __forceinline__ void acc_from(float (&acc)[MT][NT][4], const float* src, int ld, const float* rowf, int m0,
                                          int n0) {
@@ -445,11 +486,13 @@ __device__ __forceinline__ void acc_from(float (&acc)[MT][NT][4], const float* s
 // entering state and V'; role 1 walks the chunks backwards from dL/dS_T and
 // stores dL/d(state leaving the chunk) and dV', and writes dL/dS_0.
 template <typename IO, int DK, int DV, int SW>
-__global__ void __launch_bounds__(kThreads, 1) bwd_pass_kernel(const ChunkBwdArgs a) {
+__global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBwdArgs a) {
   constexpr bool X3 = std::is_same<IO, float>::value;
-  constexpr int LK = DK + 4, LS = SW + 4, NS = DV / SW;
-  using TV = Tiling<kC, SW>;  // 64 x SW products
-  using TS = Tiling<DK, SW>;  // DK x SW products
+  using PP = PassPlan<DK, DV, SW>;
+  constexpr int LK = PP::LK, LS = PP::LS, NS = DV / SW;
+  constexpr int NTH = kPassThreads;
+  using TV = Tiling<kC, SW, NTH / 32>;  // 64 x SW products
+  using TS = Tiling<DK, SW, NTH / 32>;  // DK x SW products
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x, warp = tid >> 5;
   const int cs = blockIdx.x % NS, bh = blockIdx.x / NS, c0 = cs * SW, NC = a.NC;
@@ -457,32 +500,44 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_pass_kernel(const ChunkBwdArg
   const int vm0 = TV::m0(warp), vn0 = TV::n0(warp), sm0 = TS::m0(warp), sn0 = TS::n0(warp);
 
   if (blockIdx.y == 0) {
-    float* sS = sm;              // [DK][LS] state columns
-    float* sV = sS + DK * LS;    // [64][LS] V'
-    float* sU = sV + kC * LS;    // [64][LS] U columns
-    float* sW = sU + kC * LS;    // [64][LK] W
-    float* sKb = sW + kC * LK;   // [64][LK] Kbar
-    float* sgm = sKb + kC * LK;  // [DK] gamma
-    for (int idx = tid; idx < DK * SW; idx += kThreads) {
+    constexpr int NB = PP::NB0;
+    float* sS = sm;            // [DK][LS] state columns
+    float* sV = sS + DK * LS;  // [64][LS] V'
+    float* sbuf = sV + kC * LS;
+    auto sW = [&](int p) { return sbuf + p * PP::buf0; };                        // [64][LK] W
+    auto sKb = [&](int p) { return sbuf + p * PP::buf0 + kC * LK; };             // [64][LK] Kbar
+    auto sU = [&](int p) { return sbuf + p * PP::buf0 + 2 * kC * LK; };          // [64][LS] U columns
+    auto sgm = [&](int p) { return sbuf + p * PP::buf0 + 2 * kC * LK + kC * LS; };  // [DK] gamma
+    auto issue = [&](int n, int p) {
+      const size_t rec = (size_t)bh * NC + n;
+      load_f32<NTH>(sW(p), LK, a.W + rec * kC * DK, DK, kC, DK);
+      load_f32<NTH>(sKb(p), LK, a.Kb + rec * kC * DK, DK, kC, DK);
+      load_f32<NTH>(sU(p), LS, a.U + rec * kC * DV + c0, DV, kC, SW);
+      load_f32<NTH>(sgm(p), DK, a.gam + rec * DK, DK, 1, DK);
+      cp_commit();
+    };
+    for (int idx = tid; idx < DK * SW; idx += NTH) {
       const int r = idx / SW, c = idx % SW;
       sS[r * LS + c] = a.s0 ? a.s0[st0 + (size_t)r * DV + c0 + c] : 0.f;
     }
+    issue(0, 0);
     for (int n = 0; n < NC; ++n) {
       const size_t rec = (size_t)bh * NC + n;
+      const int p = NB == 2 ? (n & 1) : 0;
+      __syncthreads();  // the previous chunk's reads are done
+      if (NB == 1 && n > 0) issue(n, 0);
+      store_f32<NTH>(a.S0c + rec * DK * DV + c0, DV, sS, LS, DK, SW);
+      cp_wait_group<0>();
       __syncthreads();
-      store_f32(a.S0c + rec * DK * DV + c0, DV, sS, LS, DK, SW);
-      load_f32(sW, LK, a.W + rec * kC * DK, DK, kC, DK);
-      load_f32(sKb, LK, a.Kb + rec * kC * DK, DK, kC, DK);
-      load_f32(sU, LS, a.U + rec * kC * DV + c0, DV, kC, SW);
-      if (tid < DK) sgm[tid] = a.gam[rec * DK + tid];
-      __syncthreads();
+      if (NB == 2 && n + 1 < NC) issue(n + 1, p ^ 1);
       {  // V' = U - W S
         float acc[TV::MT][TV::NT][4];
         zero(acc);
-        warp_mma<TV::MT, TV::NT, X3>(acc, rowm(sW, LK), rowm(sS, LS), vm0, vn0, DK);
+        warp_mma<TV::MT, TV::NT, X3, DK>(acc, rowm(sW(p), LK), rowm(sS, LS), vm0, vn0);
         float* vp = a.Vp + rec * kC * DV + c0;
+        const float* u = sU(p);
         for_acc<TV::MT, TV::NT>(vm0, vn0, [&](int mt, int nt, int e, int i, int c) {
-          const float x = sU[i * LS + c] - acc[mt][nt][e];
+          const float x = u[i * LS + c] - acc[mt][nt][e];
           sV[i * LS + c] = x;
           vp[i * DV + c] = x;
         });
@@ -490,71 +545,105 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_pass_kernel(const ChunkBwdArg
       __syncthreads();
       {  // S = diag(gamma) S + Kbar^T V'
         float acc[TS::MT][TS::NT][4];
-        acc_from(acc, sS, LS, sgm, sm0, sn0);
-        warp_mma<TS::MT, TS::NT, X3>(acc, colm(sKb, LK), rowm(sV, LS), sm0, sn0, kC);
+        acc_from(acc, sS, LS, sgm(p), sm0, sn0);
+        warp_mma<TS::MT, TS::NT, X3, kC>(acc, colm(sKb(p), LK), rowm(sV, LS), sm0, sn0);
         for_acc<TS::MT, TS::NT>(sm0, sn0,
                                 [&](int mt, int nt, int e, int r, int c) { sS[r * LS + c] = acc[mt][nt][e]; });
       }
     }
   } else {
+    constexpr int NB = PP::NB1;
     float* sD = sm;               // [DK][LS] dS columns
     float* sdV = sD + DK * LS;    // [64][LS] dV'
     float* sO = sdV + kC * LS;    // [64][LS] dO columns
-    float* sA = sO + kC * LS;     // [64][kLC] Aqk
-    float* sKb = sA + kC * kLC;   // [64][LK] Kbar
-    float* sQp = sKb + kC * LK;   // [64][LK] Q+
+    float* sQp = sO + kC * LS;    // [64][LK] Q+
     float* sW = sQp + kC * LK;    // [64][LK] W
-    float* sgm = sW + kC * LK;    // [DK] gamma
-    for (int idx = tid; idx < DK * SW; idx += kThreads) {
+    float* sbuf = sW + kC * LK;
+    auto sA = [&](int p) { return sbuf + p * PP::buf1; };                        // [64][kLC] Aqk
+    auto sKb = [&](int p) { return sbuf + p * PP::buf1 + kC * kLC; };            // [64][LK] Kbar
+    auto sgm = [&](int p) { return sbuf + p * PP::buf1 + kC * kLC + kC * LK; };  // [DK] gamma
+    auto sraw = [&](int p) {  // [64][SW] dO columns as stored (IO)
+      return reinterpret_cast<IO*>(sbuf + p * PP::buf1 + kC * kLC + kC * LK + DK);
+    };
+    const IO* d_o = static_cast<const IO*>(a.d_o);
+    auto issue = [&](int n, int p) {
+      const size_t rec = (size_t)bh * NC + n;
+      load_f32<NTH>(sA(p), kLC, a.Aqk + rec * kC * kC, kC, kC, kC);
+      load_f32<NTH>(sKb(p), LK, a.Kb + rec * kC * DK, DK, kC, DK);
+      load_f32<NTH>(sgm(p), DK, a.gam + rec * DK, DK, 1, DK);
+      constexpr int V = 16 / sizeof(IO), PER = SW / V;  // 16-byte pieces per row
+      const int t0 = n * kC, nv = min(kC, a.T - t0);
+      const size_t r0 = row_of(a, bh, t0);
+      for (int idx = tid; idx < kC * PER; idx += NTH) {
+        const int i = idx / PER, c = (idx % PER) * V;
+        const IO* src = i < nv ? d_o + (r0 + (size_t)i * a.H) * DV + c0 + c : d_o;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                         (uint32_t)__cvta_generic_to_shared(sraw(p) + i * SW + c)),
+                     "l"(src), "r"(i < nv ? 16 : 0)
+                     : "memory");
+      }
+      cp_commit();
+    };
+    for (int idx = tid; idx < DK * SW; idx += NTH) {
       const int r = idx / SW, c = idx % SW;
       sD[r * LS + c] = a.dsT ? a.dsT[st0 + (size_t)r * DV + c0 + c] : 0.f;
     }
+    issue(NC - 1, NB == 2 ? ((NC - 1) & 1) : 0);
     for (int n = NC - 1; n >= 0; --n) {
       const size_t rec = (size_t)bh * NC + n;
-      const int t0 = n * kC, nv = min(kC, a.T - t0);
+      const int p = NB == 2 ? (n & 1) : 0;
+      __syncthreads();  // the previous chunk's reads are done
+      if (NB == 1 && n < NC - 1) issue(n, 0);
+      store_f32<NTH>(a.dSc + rec * DK * DV + c0, DV, sD, LS, DK, SW);
+      load_f32<NTH>(sQp, LK, a.Qp + rec * kC * DK, DK, kC, DK);
+      load_f32<NTH>(sW, LK, a.W + rec * kC * DK, DK, kC, DK);
+      cp_commit();
+      cp_wait_group<1>();  // this chunk's Aqk, Kbar, gamma, dO (Q+ and W may still be in flight)
       __syncthreads();
-      store_f32(a.dSc + rec * DK * DV + c0, DV, sD, LS, DK, SW);
-      load_f32(sA, kLC, a.Aqk + rec * kC * kC, kC, kC, kC);
-      load_f32(sKb, LK, a.Kb + rec * kC * DK, DK, kC, DK);
-      load_f32(sQp, LK, a.Qp + rec * kC * DK, DK, kC, DK);
-      load_f32(sW, LK, a.W + rec * kC * DK, DK, kC, DK);
-      load_rows<IO, SW>(sO, LS, static_cast<const IO*>(a.d_o), row_of(a, bh, t0), a.H, nv, DV, c0);
-      if (tid < DK) sgm[tid] = a.gam[rec * DK + tid];
+      for (int idx = tid; idx < kC * SW; idx += NTH) {  // dO columns to fp32 (zeros past the tail)
+        const int i = idx / SW, c = idx % SW;
+        sO[i * LS + c] = to_f32(sraw(p)[i * SW + c]);
+      }
       __syncthreads();
       {  // dV' = Aqk^T dO + Kbar dS
         float acc[TV::MT][TV::NT][4];
         zero(acc);
-        warp_mma<TV::MT, TV::NT, X3>(acc, colm(sA, kLC), rowm(sO, LS), vm0, vn0, kC);
-        warp_mma<TV::MT, TV::NT, X3>(acc, rowm(sKb, LK), rowm(sD, LS), vm0, vn0, DK);
+        warp_mma<TV::MT, TV::NT, X3, kC>(acc, colm(sA(p), kLC), rowm(sO, LS), vm0, vn0);
+        warp_mma<TV::MT, TV::NT, X3, DK>(acc, rowm(sKb(p), LK), rowm(sD, LS), vm0, vn0);
         float* dvp = a.dVp + rec * kC * DV + c0;
         for_acc<TV::MT, TV::NT>(vm0, vn0, [&](int mt, int nt, int e, int i, int c) {
           sdV[i * LS + c] = acc[mt][nt][e];
           dvp[i * DV + c] = acc[mt][nt][e];
         });
       }
+      if (NB == 2 && n > 0) {
+        issue(n - 1, p ^ 1);
+        cp_wait_group<1>();  // Q+ and W of this chunk
+      } else {
+        cp_wait_group<0>();
+      }
       __syncthreads();
       {  // dS = diag(gamma) dS + Q+^T dO - W^T dV'
         float acc[TS::MT][TS::NT][4], neg[TS::MT][TS::NT][4];
-        acc_from(acc, sD, LS, sgm, sm0, sn0);
-        warp_mma<TS::MT, TS::NT, X3>(acc, colm(sQp, LK), rowm(sO, LS), sm0, sn0, kC);
+        acc_from(acc, sD, LS, sgm(p), sm0, sn0);
+        warp_mma<TS::MT, TS::NT, X3, kC>(acc, colm(sQp, LK), rowm(sO, LS), sm0, sn0);
         zero(neg);
-        warp_mma<TS::MT, TS::NT, X3>(neg, colm(sW, LK), rowm(sdV, LS), sm0, sn0, kC);
+        warp_mma<TS::MT, TS::NT, X3, kC>(neg, colm(sW, LK), rowm(sdV, LS), sm0, sn0);
         for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) {
           sD[r * LS + c] = acc[mt][nt][e] - neg[mt][nt][e];
         });
       }
     }
     __syncthreads();
-    if (a.ds0) store_f32(a.ds0 + st0 + c0, DV, sD, LS, DK, SW);
+    if (a.ds0) store_f32<NTH>(a.ds0 + st0 + c0, DV, sD, LS, DK, SW);
   }
 }
-
 
 // ------------------------------------------------------------------ kernel 3
 template <int DK, int DV>
 constexpr size_t local_a_smem() {
   constexpr int LV = DV + 4;
-  return sizeof(float) * ((size_t)4 * kC * LV + kC * kLC + 2 * 32 * LV + kC + 2 * kC);
+  return sizeof(float) * ((size_t)4 * kC * LV + kC * kLC + 2 * 32 * LV + kC + 4 * kC);
 }
 
 // Per chunk: the products that contract over the value channels.
@@ -571,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
   float* sS0 = sT + kC * kLC;  // [32][LV] rows of S0
   float* sdS = sS0 + 32 * LV;  // [32][LV] rows of dS
   float* sb = sdS + 32 * LV;   // [64] beta
-  float* red = sb + kC;        // [2][64] row sums per column group
+  float* red = sb + kC;        // [4][64] row sums per column group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % a.NC, bh = blockIdx.x / a.NC, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)bh * a.NC + n;
@@ -582,19 +671,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
   load_f32(sdV, LV, a.dVp + rec * kC * DV, DV, kC, DV);
   load_f32(sT, kLC, a.Tm + rec * kC * kC, kC, kC, kC);
   if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const IO*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
+  cp_wait();
   __syncthreads();
   {
     using Tl = Tiling<kC, kC>;
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);  // dAqk = tril(dO V'^T)
-    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sO, LV), colm(sVp, LV), m0, n0, DV);
+    warp_mma<Tl::MT, Tl::NT, X3, DV>(acc, rowm(sO, LV), colm(sVp, LV), m0, n0);
     float* out = a.dAqk + rec * kC * kC;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       out[i * kC + j] = j <= i ? acc[mt][nt][e] : 0.f;
     });
     zero(acc);  // dU (beta V)^T, strictly lower part
-    warp_mma<Tl::MT, Tl::NT, X3>(acc, rowm(sdV, LV), colm(sv, LV), m0, n0, DV);
+    warp_mma<Tl::MT, Tl::NT, X3, DV>(acc, rowm(sdV, LV), colm(sv, LV), m0, n0);
     out = a.dT1 + rec * kC * kC;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       out[i * kC + j] = j < i ? acc[mt][nt][e] * sb[j] : 0.f;
@@ -605,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4], rp[Tl::MT][2] = {};
     zero(acc);
-    warp_mma<Tl::MT, Tl::NT, X3>(acc, colm(sT, kLC), rowm(sdV, LV), m0, n0, kC);
+    warp_mma<Tl::MT, Tl::NT, X3, kC>(acc, colm(sT, kLC), rowm(sdV, LV), m0, n0);
     IO* dv = static_cast<IO*>(a.dv);
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
       const float x = acc[mt][nt][e];
@@ -615,7 +705,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
     row_sums_out<Tl::MT>(rp, m0, red + (warp / Tl::WM) * kC);
   }
   __syncthreads();
-  if (tid < kC) a.dbu[rec * kC + tid] = red[tid] + red[kC + tid];
+  if (tid < kC) {
+    float x = 0.f;
+#pragma unroll
+    for (int w = 0; w < Tiling<kC, DV>::WN; ++w) x += red[w * kC + tid];
+    a.dbu[rec * kC + tid] = x;
+  }
 
   // blocks of 32 key rows of S0 and dS: dO S0^T, -dV' S0^T, V' dS^T, rowsum(dS . S0)
   using Tr = Tiling<kC, 32>;
@@ -624,23 +719,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
     __syncthreads();
     load_f32(sS0, LV, a.S0c + rec * DK * DV + (size_t)rb * 32 * DV, DV, 32, DV);
     load_f32(sdS, LV, a.dSc + rec * DK * DV + (size_t)rb * 32 * DV, DV, 32, DV);
+    cp_wait();
     __syncthreads();
     float acc[Tr::MT][Tr::NT][4];
     zero(acc);
-    warp_mma<Tr::MT, Tr::NT, X3>(acc, rowm(sO, LV), colm(sS0, LV), m0, n0, DV);
+    warp_mma<Tr::MT, Tr::NT, X3, DV>(acc, rowm(sO, LV), colm(sS0, LV), m0, n0);
     float* out = a.dQs + rec * kC * DK + rb * 32;
     for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
     zero(acc);
-    warp_mma<Tr::MT, Tr::NT, X3>(acc, rowm(sdV, LV), colm(sS0, LV), m0, n0, DV);
+    warp_mma<Tr::MT, Tr::NT, X3, DV>(acc, rowm(sdV, LV), colm(sS0, LV), m0, n0);
     out = a.dW + rec * kC * DK + rb * 32;
     for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = -acc[mt][nt][e]; });
     zero(acc);
-    warp_mma<Tr::MT, Tr::NT, X3>(acc, rowm(sVp, LV), colm(sdS, LV), m0, n0, DV);
+    warp_mma<Tr::MT, Tr::NT, X3, DV>(acc, rowm(sVp, LV), colm(sdS, LV), m0, n0);
     out = a.dKb + rec * kC * DK + rb * 32;
     for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
 #pragma unroll
-    for (int rr = 0; rr < 4; ++rr) {  // warp w: rows 4w .. 4w+3 of the block
-      const int r = 4 * warp + rr;
+    for (int rr = 0; rr < 32 / kWarps; ++rr) {  // each warp: 32 / kWarps rows of the block
+      const int r = (32 / kWarps) * warp + rr;
       float x = 0.f;
       for (int c = lane; c < DV; c += 32) x = fmaf(sdS[r * LV + c], sS0[r * LV + c], x);
 #pragma unroll
@@ -655,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
 template <int DK, int DV>
 constexpr size_t local_b_smem() {
   constexpr int LK = DK + 4;
-  return sizeof(float) * ((size_t)4 * kC * LK + 4 * kC * kLC + kC + 4 * kC + 4 * DK);
+  return sizeof(float) * ((size_t)4 * kC * LK + 4 * kC * kLC + kC + 8 * kC + 4 * DK);
 }
 
 // Per chunk: dT, dA, the pairwise gradients and the fold into dq, dk, dg, dbeta.
@@ -675,8 +771,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   float* sY2 = sDT + kC * kLC;  // [64][kLC] dT T^T
   float* sQA = sY2 + kC * kLC;  // [64][kLC] dAqk
   float* sb = sQA + kC * kLC;   // [64] beta
-  float* red = sb + kC;         // [4][64] row sums: K+ . T^T dW (slots 0, 1), dA . P (slots 2, 3)
-  float* colC = red + 4 * kC;   // [4][DK] column sums of dKbar . Kbar per row group
+  float* red = sb + kC;         // [8][64] row sums per column group: K+ . T^T dW (slots 0-3), dA . P (4-7)
+  float* colC = red + 8 * kC;   // [4][DK] column sums of dKbar . Kbar per row group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % a.NC, bh = blockIdx.x / a.NC, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)bh * a.NC + n;
@@ -694,6 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   load_f32(sY, LK, a.dW + rec * kC * DK, DK, kC, DK);
   load_f32(sT, kLC, a.Tm + rec * kC * kC, kC, kC, kC);
   load_f32(sDT, kLC, a.dT1 + rec * kC * kC, kC, kC, kC);
+  cp_wait();
   __syncthreads();
   for (int idx = tid; idx < kC * DK; idx += kThreads) {
     const int i = idx / DK, r = idx % DK;
@@ -703,7 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   {  // dT += dW (beta K+)^T, strictly lower part
     float acc[TC::MT][TC::NT][4];
     zero(acc);
-    warp_mma<TC::MT, TC::NT, X3>(acc, rowm(sY, LK), colm(sX, LK), cm0, cn0, DK);
+    warp_mma<TC::MT, TC::NT, X3, DK>(acc, rowm(sY, LK), colm(sX, LK), cm0, cn0);
     for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
       if (j < i) sDT[i * kLC + j] += acc[mt][nt][e] * sb[j];
     });
@@ -711,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   {  // X = T^T dW: dK+ = beta X; dbeta part rowsum(K+ . X)
     float acc[TK::MT][TK::NT][4], rp[TK::MT][2] = {};
     zero(acc);
-    warp_mma<TK::MT, TK::NT, X3>(acc, colm(sT, kLC), rowm(sY, LK), m0, n0, kC);
+    warp_mma<TK::MT, TK::NT, X3, kC>(acc, colm(sT, kLC), rowm(sY, LK), m0, n0);
     for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
       const float x = acc[mt][nt][e], kp = sX[i * LK + r], bx = sb[i] * x;
       dk_acc[mt][nt][e] = fmaf(bx, expf(sG[i * LK + r]), dk_acc[mt][nt][e]);
@@ -724,7 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   {  // dT T^T
     float acc[TC::MT][TC::NT][4];
     zero(acc);
-    warp_mma<TC::MT, TC::NT, X3>(acc, rowm(sDT, kLC), colm(sT, kLC), cm0, cn0, kC);
+    warp_mma<TC::MT, TC::NT, X3, kC>(acc, rowm(sDT, kLC), colm(sT, kLC), cm0, cn0);
     for_acc<TC::MT, TC::NT>(cm0, cn0,
                             [&](int mt, int nt, int e, int i, int j) { sY2[i * kLC + j] = acc[mt][nt][e]; });
   }
@@ -732,28 +829,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   {  // dA = -T^T (dT T^T), strictly lower; dbeta part rowsum(dA . P); M = diag(beta) dA
     float acc[TC::MT][TC::NT][4], rp[TC::MT][2] = {};
     zero(acc);
-    warp_mma<TC::MT, TC::NT, X3>(acc, colm(sT, kLC), rowm(sY2, kLC), cm0, cn0, kC);
+    warp_mma<TC::MT, TC::NT, X3, kC>(acc, colm(sT, kLC), rowm(sY2, kLC), cm0, cn0);
     const float* P = a.Pkk + rec * kC * kC;
     for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
       const float d = j < i ? -acc[mt][nt][e] : 0.f;
       rp[mt][e >> 1] = fmaf(d, P[i * kC + j], rp[mt][e >> 1]);
       sDT[i * kLC + j] = sb[i] * d;
     });
-    row_sums_out<TC::MT>(rp, cm0, red + (2 + warp / TC::WM) * kC);
+    row_sums_out<TC::MT>(rp, cm0, red + (4 + warp / TC::WM) * kC);
   }
   // operands of the pairwise gradients
   load_f32(sQA, kLC, a.dAqk + rec * kC * kC, kC, kC, kC);
+  load_rows<IO, DK>(sX, LK, k, row0, a.H, nv, DK, 0);
+  load_rows<IO, DK>(sZ, LK, q, row0, a.H, nv, DK, 0);
+  cp_wait();
+  __syncthreads();
   for (int idx = tid; idx < kC * DK; idx += kThreads) {
     const int i = idx / DK, r = idx % DK;
-    const size_t o = (row0 + (size_t)i * a.H) * DK + r;
-    const float kk = i < nv ? to_f32(k[o]) : 0.f, qq = i < nv ? a.scale * to_f32(q[o]) : 0.f;
+    const float kk = sX[i * LK + r], qq = a.scale * sZ[i * LK + r];
     if (!slow) {
       const float d = sG[i * LK + r] - sG[kRef * LK + r], ex = expf(d);
       sX[i * LK + r] = kk * ex;
       sY[i * LK + r] = kk * expf(-d);
       sZ[i * LK + r] = qq * ex;
     } else {
-      sX[i * LK + r] = kk;
       sZ[i * LK + r] = qq;
     }
   }
@@ -765,7 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
     {  // dQ+_r = dAqk K-_r;  dq = scale (exp(G - G_ref) dQ+_r + Gamma dO S0^T)
       float acc[TK::MT][TK::NT][4];
       zero(acc);
-      warp_mma<TK::MT, TK::NT, X3>(acc, rowm(sQA, kLC), rowm(sY, LK), m0, n0, kC);
+      warp_mma<TK::MT, TK::NT, X3, kC>(acc, rowm(sQA, kLC), rowm(sY, LK), m0, n0);
       for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
         const float x = acc[mt][nt][e], G = sG[i * LK + r];
         const float ex = expf(G - sG[kRef * LK + r]), dqs = dQs[i * DK + r];
@@ -776,8 +875,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
     {  // dK-_r = dAqk^T Q+_r + M^T K+_r
       float acc[TK::MT][TK::NT][4];
       zero(acc);
-      warp_mma<TK::MT, TK::NT, X3>(acc, colm(sQA, kLC), rowm(sZ, LK), m0, n0, kC);
-      warp_mma<TK::MT, TK::NT, X3>(acc, colm(sDT, kLC), rowm(sX, LK), m0, n0, kC);
+      warp_mma<TK::MT, TK::NT, X3, kC>(acc, colm(sQA, kLC), rowm(sZ, LK), m0, n0);
+      warp_mma<TK::MT, TK::NT, X3, kC>(acc, colm(sDT, kLC), rowm(sX, LK), m0, n0);
       for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
         const float x = acc[mt][nt][e];
         dk_acc[mt][nt][e] = fmaf(expf(sG[kRef * LK + r] - sG[i * LK + r]), x, dk_acc[mt][nt][e]);
@@ -787,7 +886,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
     {  // dK+_r = M K-_r
       float acc[TK::MT][TK::NT][4];
       zero(acc);
-      warp_mma<TK::MT, TK::NT, X3>(acc, rowm(sDT, kLC), rowm(sY, LK), m0, n0, kC);
+      warp_mma<TK::MT, TK::NT, X3, kC>(acc, rowm(sDT, kLC), rowm(sY, LK), m0, n0);
       for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
         const float x = acc[mt][nt][e];
         dk_acc[mt][nt][e] = fmaf(expf(sG[i * LK + r] - sG[kRef * LK + r]), x, dk_acc[mt][nt][e]);
@@ -851,7 +950,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   __syncthreads();
   if (tid < DK) {  // dG_C terms, then dg = reverse cumsum of dG over the chunk
     const int r = tid;
-    float x = colC[r] + colC[DK + r] + colC[2 * DK + r] + colC[3 * DK + r];
+    float x = 0.f;
+#pragma unroll
+    for (int w = 0; w < TK::WM; ++w) x += colC[w * DK + r];
     x = fmaf(expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
     float acc = x;
     for (int i = kC - 1; i >= 0; --i) {
@@ -876,9 +977,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
       if (lane == 0) dg[row0 + (size_t)i * a.H] = from_f32<IO>(x);
     }
   }
-  if (tid < nv)
-    static_cast<IO*>(a.dbeta)[row0 + (size_t)tid * a.H] =
-        from_f32<IO>(((a.dbu[rec * kC + tid] + red[tid]) + red[kC + tid]) + (red[2 * kC + tid] + red[3 * kC + tid]));
+  if (tid < nv) {
+    float x = a.dbu[rec * kC + tid], y = 0.f;
+#pragma unroll
+    for (int w = 0; w < TK::WN; ++w) x += red[w * kC + tid];
+#pragma unroll
+    for (int w = 0; w < TC::WN; ++w) y += red[(4 + w) * kC + tid];
+    static_cast<IO*>(a.dbeta)[row0 + (size_t)tid * a.H] = from_f32<IO>(x + y);
+  }
 }
 
 
@@ -901,10 +1007,11 @@ struct WsPlan {
 int pass_width(int BH, int dv) { return (size_t)2 * BH * (dv / 32) <= 148 ? 32 : 64; }
 
 template <typename Kern>
-cudaError_t launch_k(Kern kern, dim3 grid, size_t smem, const ChunkBwdArgs& a, cudaStream_t stream) {
+cudaError_t launch_k(Kern kern, dim3 grid, size_t smem, const ChunkBwdArgs& a, cudaStream_t stream,
+                     int nth = kThreads) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(a);
+  kern<<<grid, nth, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -914,9 +1021,11 @@ cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t strea
   cudaError_t e = launch_k(bwd_prep_kernel<IO, DK, DV>, grid, prep_smem<DK, DV>(), a, stream);
   if (e != cudaSuccess) return e;
   if (pass_width(BH, DV) == 32)
-    e = launch_k(bwd_pass_kernel<IO, DK, DV, 32>, dim3(BH * (DV / 32), 2), pass_smem<DK, DV, 32>(), a, stream);
+    e = launch_k(bwd_pass_kernel<IO, DK, DV, 32>, dim3(BH * (DV / 32), 2), pass_smem<DK, DV, 32>(), a, stream,
+                 kPassThreads);
   else
-    e = launch_k(bwd_pass_kernel<IO, DK, DV, 64>, dim3(BH * (DV / 64), 2), pass_smem<DK, DV, 64>(), a, stream);
+    e = launch_k(bwd_pass_kernel<IO, DK, DV, 64>, dim3(BH * (DV / 64), 2), pass_smem<DK, DV, 64>(), a, stream,
+                 kPassThreads);
   if (e != cudaSuccess) return e;
   e = launch_k(bwd_local_a_kernel<IO, DK, DV>, grid, local_a_smem<DK, DV>(), a, stream);
   if (e != cudaSuccess) return e;
