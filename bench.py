@@ -67,8 +67,24 @@ def backward_bytes(B, T, H, dk, dv, elem=2) -> float:
     return B * T * H * per_tok + 3 * B * H * dk * dv * 4
 
 
+def backward_macs(B, T, H, dk, dv, chunk=64) -> float:
+    """Tensor-core multiply-adds the chunkwise backward issues (full tiles):
+    the chunk operands (P, Aqk, W, U), the forward replay (V', S), the reverse
+    sweep (dV', dS), the d_v contractions (dAqk, dT, T^T dU, dO S0^T, dW,
+    dKbar) and the rest (dT, T^T dW, dA, dQ+, dK-, dK+), per chunk and head."""
+    c = chunk
+    per = (2 * c * c * dk + c * c * (dk + dv)) + 2 * c * dk * dv + (c * dv * (c + dk) + 2 * dk * dv * c) \
+        + (2 * c * c * dv + c * dv * c + 3 * c * dk * dv) + (2 * c * c * dk + 2 * c ** 3 + 4 * c * c * dk)
+    return B * H * -(-T // c) * per
+
+
 def decode_bytes(N, H, dk, dv, elem=2) -> float:
     return N * H * (2 * dk * dv * 4 + (3 * dk + 2 * dv + 1) * elem)
+
+
+# Dense tf32 / bf16 tensor throughput of the B200 (nominal 1.1 / 2.25 PFLOP/s),
+# applied to the measured bf16 peak to get a tf32 peak.
+TF32_PER_BF16 = 1.1 / 2.25
 
 
 def load_peaks():
@@ -443,10 +459,16 @@ def run_ours(args, cfg):
             ts.append(a.elapsed_time(b))
         bs = reduce_max(statistics.median(ts) / 1e3, dev)
         bbytes = backward_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, 2 if cfg.dtype == "bf16" else 4)
+        bflops = 2 * backward_macs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
+        tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
         backward = {"us_per_call": bs * 1e6, "tokens_per_s": weak_scaling_value(tokens, world, bs),
                     "calls": args.backward_calls, "algorithmic_bytes": bbytes,
                     "achieved_gbs": bbytes / bs / 1e9, "frac_hbm": bbytes / bs / 1e9 / peaks["hbm_gbs"],
-                    "kernel": "kda_backward_kernel (token-recurrent fp32; column-split partials + fixed-order sum)"}
+                    "issued_tflops": bflops / bs / 1e12, "tf32_peak_tflops": tf32_peak,
+                    "frac_tf32": bflops / bs / 1e12 / tf32_peak, "workspace_bytes": bws.numel(),
+                    "launches": 4,
+                    "kernel": "chunkwise: bwd_prep, bwd_pass (forward replay + reverse dS sweep), bwd_local_a, "
+                              "bwd_local_b (warp-level tf32 tensor-core products, fp32 workspace)"}
         del bws, d_o, d_s
 
     # ---- CPU baseline: the oracle on the host cores (rank 0, N = 1 only)
