@@ -122,6 +122,79 @@ __device__ __forceinline__ void warp_mma(float (&acc)[MT][NT][4], View A, View B
   }
 }
 
+// The same product for K-contiguous operands: A is [M][lda] and B^T is [N][ldb]
+// (element (k, n) of B at B[n*ldb + k]), both with k contiguous.  Fragments
+// come from ldmatrix (8 x 8 b16 matrices = 8 rows x 4 fp32): one x4 per A tile
+// and one x4 per pair of B tiles.  Row starts must be 16-byte aligned; ld = 4
+// (mod 32) floats keeps the 8 rows of each matrix in distinct bank groups.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const float* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const float* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+template <int MT, int NT, bool X3, int K>
+__device__ __forceinline__ void warp_mma_kk(float (&acc)[MT][NT][4], const float* A, int lda, const float* B, int ldb,
+                                            int m0, int n0) {
+  const int lane = threadIdx.x & 31, mat = lane >> 3, rr = lane & 7;
+  // odd NT: the last B tile by an x2 load (lanes 0-15 give its row addresses)
+  const float* pb1 = B + (n0 + 8 * (NT - 1) + rr) * ldb + 4 * (mat & 1);
+  // this lane's row address in each x4 load
+  const float* pa = A + (m0 + rr + 8 * (mat & 1)) * lda + 4 * (mat >> 1);
+  const float* pb = B + (n0 + rr + 8 * (mat >> 1)) * ldb + 4 * (mat & 1);
+#pragma unroll
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    uint32_t ah[MT][4], al[MT][4], bh[NT][2], bl[NT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      uint32_t r[4];
+      ldsm_x4(r, pa + 16 * mt * lda + k0);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x = __uint_as_float(r[e]);
+        ah[mt][e] = tf32_rna(x);
+        if (X3) al[mt][e] = tf32_rna(x - __uint_as_float(ah[mt][e]));
+      }
+    }
+#pragma unroll
+    for (int np = 0; np < NT / 2; ++np) {
+      uint32_t r[4];
+      ldsm_x4(r, pb + 16 * np * ldb + k0);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x = __uint_as_float(r[e]);
+        const int nt = 2 * np + (e >> 1), h = e & 1;
+        bh[nt][h] = tf32_rna(x);
+        if (X3) bl[nt][h] = tf32_rna(x - __uint_as_float(bh[nt][h]));
+      }
+    }
+    if constexpr (NT % 2 == 1) {
+      uint32_t r[2];
+      ldsm_x2(r, pb1 + k0);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float x = __uint_as_float(r[h]);
+        bh[NT - 1][h] = tf32_rna(x);
+        if (X3) bl[NT - 1][h] = tf32_rna(x - __uint_as_float(bh[NT - 1][h]));
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (X3) {
+          mma_tf32(acc[mt][nt], al[mt][0], al[mt][1], al[mt][2], al[mt][3], bh[nt][0], bh[nt][1]);
+          mma_tf32(acc[mt][nt], ah[mt][0], ah[mt][1], ah[mt][2], ah[mt][3], bl[nt][0], bl[nt][1]);
+        }
+        mma_tf32(acc[mt][nt], ah[mt][0], ah[mt][1], ah[mt][2], ah[mt][3], bh[nt][0], bh[nt][1]);
+      }
+  }
+}
+
 // Split of an R x N output over NW warps: WM x WN warps, each (16 MT) x (8 NT).
 template <int R, int N, int NW = kWarps>
 struct Tiling {
@@ -290,7 +363,8 @@ struct ChunkBwdArgs {
   int T, H, NC, gate;
   // workspace (fp32), record rec = (b * H + h) * NC + chunk
   float *W, *U, *Qp, *Kb;  // [rec][64][d_k] (U: [64][d_v]): W, U, Q+, Kbar
-  float *Aqk, *Tm, *Pkk;   // [rec][64][64]: Aqk, T, P
+  float *Wt, *Qpt, *Kbt;   // [rec][d_k][64]: their transposes for the state passes
+  float *Aqk, *Tm, *Pkk;   // [rec][64][64]: Aqk^T (transposed), T, P
   float* gam;              // [rec][d_k]: gamma
   float *S0c, *dSc;        // [rec][d_k][d_v]: state entering the chunk, dL/d(state leaving it)
   float *Vp, *dVp;         // [rec][64][d_v]: V', dV'
@@ -343,8 +417,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     se[tid] = expf(sG[kRef * LK + tid]);
     a.gam[rec * DK + tid] = expf(sG[(kC - 1) * LK + tid]);
   }
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+^T and Kbar^T (the same values as Q+, Kbar below)
+    const int r = idx / kC, i = idx % kC;
+    const float G = sG[i * LK + r], qq = a.scale * sQ[i * LK + r];
+    a.Qpt[rec * kC * DK + idx] = qq * expf(G);
+    a.Kbt[rec * kC * DK + idx] = sK[i * LK + r] * expf(sG[(kC - 1) * LK + r] - G);
+  }
   float* Qp = a.Qp + rec * kC * DK;
   float* Kb = a.Kb + rec * kC * DK;
+  __syncthreads();  // sQ is rewritten in place below
   for (int idx = tid; idx < kC * DK; idx += kThreads) {
     const int i = idx / DK, r = idx % DK;
     const float G = sG[i * LK + r], kk = sK[i * LK + r], qq = a.scale * sQ[i * LK + r];
@@ -369,12 +450,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);
-    warp_mma<Tl::MT, Tl::NT, X3, DK>(acc, rowm(sX, LK), colm(sY, LK), m0, n0);
+    warp_mma_kk<Tl::MT, Tl::NT, X3, DK>(acc, sX, LK, sY, LK, m0, n0);
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       sP[i * kLC + j] = j < i ? acc[mt][nt][e] : 0.f;
     });
     zero(acc);
-    warp_mma<Tl::MT, Tl::NT, X3, DK>(acc, rowm(sQ, LK), colm(sY, LK), m0, n0);
+    warp_mma_kk<Tl::MT, Tl::NT, X3, DK>(acc, sQ, LK, sY, LK, m0, n0);
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       sA[i * kLC + j] = j <= i ? acc[mt][nt][e] : 0.f;
     });
@@ -395,7 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
   }
   __syncthreads();
   store_f32(a.Pkk + rec * kC * kC, kC, sP, kLC, kC, kC);
-  store_f32(a.Aqk + rec * kC * kC, kC, sA, kLC, kC, kC);
+  for (int idx = tid; idx < kC * kC; idx += kThreads) {  // Aqk^T
+    const int j = idx / kC, i = idx % kC;
+    a.Aqk[rec * kC * kC + idx] = sA[i * kLC + j];
+  }
 
   // T = (I + diag(beta) P)^-1 (unit lower triangular) by forward substitution
   // down each column: thread j < 64 keeps column j in registers; row i reads
@@ -433,7 +517,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     zero(acc);
     warp_mma<Tl::MT, Tl::NT, X3, kC>(acc, rowm(sT, kLC), rowm(sX, LK), m0, n0);
     float* Wg = a.W + rec * kC * DK;
-    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { Wg[i * DK + c] = acc[mt][nt][e]; });
+    float* Wtg = a.Wt + rec * kC * DK;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
+      Wg[i * DK + c] = acc[mt][nt][e];
+      Wtg[c * kC + i] = acc[mt][nt][e];
+    });
   }
   {
     using Tl = Tiling<kC, DV>;
@@ -452,18 +540,23 @@ __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_grou
 template <int N>
 __device__ __forceinline__ void cp_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Shared-memory plan of the pass kernel (floats).  Role 0 keeps the state
-// columns and V' and NB0 buffers of {W, Kbar, U columns, gamma}; role 1 keeps
-// dS, dV', dO, Q+, W and NB1 buffers of {Aqk, Kbar, gamma, raw dO columns}.  Two buffers
-// (the next chunk's operands load while this one computes) where they fit.
+// Shared-memory plan of the pass kernel (floats).  Every product operand is
+// K-contiguous (ldmatrix fragments): the state columns, V', dS, dV' and dO are
+// kept transposed ([column][row]) and the chunk operands come transposed from
+// the prep kernel where the product needs it.  Role 0 keeps S^T and V'^T and
+// NB0 buffers of {W, Kbar^T, U columns, gamma}; role 1 keeps dS^T, dV'^T,
+// dO^T, Q+^T, W^T and NB1 buffers of {Aqk^T, Kbar, gamma, raw dO columns}.
+// Two buffers (the next chunk's operands load while this one computes) where
+// they fit.
 template <int DK, int DV, int SW>
 struct PassPlan {
   static constexpr int LK = DK + 4, LS = SW + 4;
   static constexpr size_t kMax = 232448 / sizeof(float);
-  static constexpr size_t fix0 = (size_t)DK * LS + kC * LS, buf0 = 2 * (size_t)kC * LK + kC * LS + DK;
-  static constexpr size_t fix1 = (size_t)DK * LS + 2 * kC * LS + 2 * (size_t)kC * LK;
+  static constexpr size_t fix0 = (size_t)SW * LK + SW * kLC;
+  static constexpr size_t buf0 = (size_t)kC * LK + (size_t)DK * kLC + kC * LS + DK;
+  static constexpr size_t fix1 = (size_t)SW * LK + 2 * SW * kLC + 2 * (size_t)DK * kLC;
   static constexpr size_t stage1 = (size_t)kC * SW * 4 / sizeof(float);  // raw dO columns, up to 4 bytes each
-  static constexpr size_t buf1 = (size_t)kC * kLC + kC * LK + DK + stage1;
+  static constexpr size_t buf1 = (size_t)kC * kLC + (size_t)kC * LK + DK + stage1;
   static constexpr int NB0 = fix0 + 2 * buf0 <= kMax ? 2 : 1;
   static constexpr int NB1 = fix1 + 2 * buf1 <= kMax ? 2 : 1;
   static constexpr size_t r0 = fix0 + NB0 * buf0, r1 = fix1 + NB1 * buf1;
@@ -474,11 +567,23 @@ constexpr size_t pass_smem() {
   return PassPlan<DK, DV, SW>::bytes;
 }
 
-// Accumulator tile of an R x SW state block initialised from a shared tile, rows scaled.
-template <int MT, int NT>
-__device__ __forceinline__ void acc_from(float (&acc)[MT][NT][4], const float* src, int ld, const float* rowf, int m0,
-                                         int n0) {
-  for_acc<MT, NT>(m0, n0, [&](int mt, int nt, int e, int r, int c) { acc[mt][nt][e] = rowf[r] * src[r * ld + c]; });
+// A DK x SW block of the state (rows r, columns c) held transposed in shared
+// memory (sT[c * ld + r]) to / from its place in a [DK][DV] fp32 array.
+template <int NTH, int DK, int SW>
+__device__ __forceinline__ void store_state_t(float* g, int DV, const float* sT, int ld) {
+  for (int idx = threadIdx.x; idx < DK * (SW / 4); idx += NTH) {
+    const int r = idx / (SW / 4), c = (idx % (SW / 4)) * 4;
+    *reinterpret_cast<float4*>(g + (size_t)r * DV + c) =
+        make_float4(sT[c * ld + r], sT[(c + 1) * ld + r], sT[(c + 2) * ld + r], sT[(c + 3) * ld + r]);
+  }
+}
+template <int NTH, int DK, int SW>
+__device__ __forceinline__ void load_state_t(float* sT, int ld, const float* g, int DV) {
+  for (int idx = threadIdx.x; idx < DK * (SW / 4); idx += NTH) {
+    const int r = idx / (SW / 4), c = (idx % (SW / 4)) * 4;
+    const float4 x = g ? *reinterpret_cast<const float4*>(g + (size_t)r * DV + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    sT[c * ld + r] = x.x, sT[(c + 1) * ld + r] = x.y, sT[(c + 2) * ld + r] = x.z, sT[(c + 3) * ld + r] = x.w;
+  }
 }
 
 // One CTA per (sequence, head, SW-column slice of the state) and role:
@@ -501,74 +606,74 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBw
 
   if (blockIdx.y == 0) {
     constexpr int NB = PP::NB0;
-    float* sS = sm;            // [DK][LS] state columns
-    float* sV = sS + DK * LS;  // [64][LS] V'
-    float* sbuf = sV + kC * LS;
-    auto sW = [&](int p) { return sbuf + p * PP::buf0; };                        // [64][LK] W
-    auto sKb = [&](int p) { return sbuf + p * PP::buf0 + kC * LK; };             // [64][LK] Kbar
-    auto sU = [&](int p) { return sbuf + p * PP::buf0 + 2 * kC * LK; };          // [64][LS] U columns
-    auto sgm = [&](int p) { return sbuf + p * PP::buf0 + 2 * kC * LK + kC * LS; };  // [DK] gamma
+    float* sSt = sm;             // [SW][LK] state columns, transposed
+    float* sVt = sSt + SW * LK;  // [SW][kLC] V', transposed
+    float* sbuf = sVt + SW * kLC;
+    auto sW = [&](int p) { return sbuf + p * PP::buf0; };                                   // [64][LK] W
+    auto sKbt = [&](int p) { return sbuf + p * PP::buf0 + kC * LK; };                       // [DK][kLC] Kbar^T
+    auto sU = [&](int p) { return sbuf + p * PP::buf0 + kC * LK + DK * kLC; };              // [64][LS] U columns
+    auto sgm = [&](int p) { return sbuf + p * PP::buf0 + kC * LK + DK * kLC + kC * LS; };   // [DK] gamma
     auto issue = [&](int n, int p) {
       const size_t rec = (size_t)bh * NC + n;
       load_f32<NTH>(sW(p), LK, a.W + rec * kC * DK, DK, kC, DK);
-      load_f32<NTH>(sKb(p), LK, a.Kb + rec * kC * DK, DK, kC, DK);
+      load_f32<NTH>(sKbt(p), kLC, a.Kbt + rec * kC * DK, kC, DK, kC);
       load_f32<NTH>(sU(p), LS, a.U + rec * kC * DV + c0, DV, kC, SW);
       load_f32<NTH>(sgm(p), DK, a.gam + rec * DK, DK, 1, DK);
       cp_commit();
     };
-    for (int idx = tid; idx < DK * SW; idx += NTH) {
-      const int r = idx / SW, c = idx % SW;
-      sS[r * LS + c] = a.s0 ? a.s0[st0 + (size_t)r * DV + c0 + c] : 0.f;
-    }
+    load_state_t<NTH, DK, SW>(sSt, LK, a.s0 ? a.s0 + st0 + c0 : nullptr, DV);
     issue(0, 0);
     for (int n = 0; n < NC; ++n) {
       const size_t rec = (size_t)bh * NC + n;
       const int p = NB == 2 ? (n & 1) : 0;
       __syncthreads();  // the previous chunk's reads are done
       if (NB == 1 && n > 0) issue(n, 0);
-      store_f32<NTH>(a.S0c + rec * DK * DV + c0, DV, sS, LS, DK, SW);
+      store_state_t<NTH, DK, SW>(a.S0c + rec * DK * DV + c0, DV, sSt, LK);
       cp_wait_group<0>();
       __syncthreads();
       if (NB == 2 && n + 1 < NC) issue(n + 1, p ^ 1);
       {  // V' = U - W S
         float acc[TV::MT][TV::NT][4];
         zero(acc);
-        warp_mma<TV::MT, TV::NT, X3, DK>(acc, rowm(sW(p), LK), rowm(sS, LS), vm0, vn0);
+        warp_mma_kk<TV::MT, TV::NT, X3, DK>(acc, sW(p), LK, sSt, LK, vm0, vn0);
         float* vp = a.Vp + rec * kC * DV + c0;
         const float* u = sU(p);
         for_acc<TV::MT, TV::NT>(vm0, vn0, [&](int mt, int nt, int e, int i, int c) {
           const float x = u[i * LS + c] - acc[mt][nt][e];
-          sV[i * LS + c] = x;
+          sVt[c * kLC + i] = x;
           vp[i * DV + c] = x;
         });
       }
       __syncthreads();
       {  // S = diag(gamma) S + Kbar^T V'
         float acc[TS::MT][TS::NT][4];
-        acc_from(acc, sS, LS, sgm(p), sm0, sn0);
-        warp_mma<TS::MT, TS::NT, X3, kC>(acc, colm(sKb(p), LK), rowm(sV, LS), sm0, sn0);
+        const float* gm = sgm(p);
+        for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) {
+          acc[mt][nt][e] = gm[r] * sSt[c * LK + r];
+        });
+        warp_mma_kk<TS::MT, TS::NT, X3, kC>(acc, sKbt(p), kLC, sVt, kLC, sm0, sn0);
         for_acc<TS::MT, TS::NT>(sm0, sn0,
-                                [&](int mt, int nt, int e, int r, int c) { sS[r * LS + c] = acc[mt][nt][e]; });
+                                [&](int mt, int nt, int e, int r, int c) { sSt[c * LK + r] = acc[mt][nt][e]; });
       }
     }
   } else {
     constexpr int NB = PP::NB1;
-    float* sD = sm;               // [DK][LS] dS columns
-    float* sdV = sD + DK * LS;    // [64][LS] dV'
-    float* sO = sdV + kC * LS;    // [64][LS] dO columns
-    float* sQp = sO + kC * LS;    // [64][LK] Q+
-    float* sW = sQp + kC * LK;    // [64][LK] W
-    float* sbuf = sW + kC * LK;
-    auto sA = [&](int p) { return sbuf + p * PP::buf1; };                        // [64][kLC] Aqk
-    auto sKb = [&](int p) { return sbuf + p * PP::buf1 + kC * kLC; };            // [64][LK] Kbar
-    auto sgm = [&](int p) { return sbuf + p * PP::buf1 + kC * kLC + kC * LK; };  // [DK] gamma
+    float* sDt = sm;                // [SW][LK] dS columns, transposed
+    float* sdVt = sDt + SW * LK;    // [SW][kLC] dV', transposed
+    float* sOt = sdVt + SW * kLC;   // [SW][kLC] dO columns, transposed
+    float* sQpt = sOt + SW * kLC;   // [DK][kLC] Q+^T
+    float* sWt = sQpt + DK * kLC;   // [DK][kLC] W^T
+    float* sbuf = sWt + DK * kLC;
+    auto sAt = [&](int p) { return sbuf + p * PP::buf1; };                        // [64][kLC] Aqk^T
+    auto sKb = [&](int p) { return sbuf + p * PP::buf1 + kC * kLC; };             // [64][LK] Kbar
+    auto sgm = [&](int p) { return sbuf + p * PP::buf1 + kC * kLC + kC * LK; };   // [DK] gamma
     auto sraw = [&](int p) {  // [64][SW] dO columns as stored (IO)
       return reinterpret_cast<IO*>(sbuf + p * PP::buf1 + kC * kLC + kC * LK + DK);
     };
     const IO* d_o = static_cast<const IO*>(a.d_o);
     auto issue = [&](int n, int p) {
       const size_t rec = (size_t)bh * NC + n;
-      load_f32<NTH>(sA(p), kLC, a.Aqk + rec * kC * kC, kC, kC, kC);
+      load_f32<NTH>(sAt(p), kLC, a.Aqk + rec * kC * kC, kC, kC, kC);
       load_f32<NTH>(sKb(p), LK, a.Kb + rec * kC * DK, DK, kC, DK);
       load_f32<NTH>(sgm(p), DK, a.gam + rec * DK, DK, 1, DK);
       constexpr int V = 16 / sizeof(IO), PER = SW / V;  // 16-byte pieces per row
@@ -584,58 +689,58 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBw
       }
       cp_commit();
     };
-    for (int idx = tid; idx < DK * SW; idx += NTH) {
-      const int r = idx / SW, c = idx % SW;
-      sD[r * LS + c] = a.dsT ? a.dsT[st0 + (size_t)r * DV + c0 + c] : 0.f;
-    }
+    load_state_t<NTH, DK, SW>(sDt, LK, a.dsT ? a.dsT + st0 + c0 : nullptr, DV);
     issue(NC - 1, NB == 2 ? ((NC - 1) & 1) : 0);
     for (int n = NC - 1; n >= 0; --n) {
       const size_t rec = (size_t)bh * NC + n;
       const int p = NB == 2 ? (n & 1) : 0;
       __syncthreads();  // the previous chunk's reads are done
       if (NB == 1 && n < NC - 1) issue(n, 0);
-      store_f32<NTH>(a.dSc + rec * DK * DV + c0, DV, sD, LS, DK, SW);
-      load_f32<NTH>(sQp, LK, a.Qp + rec * kC * DK, DK, kC, DK);
-      load_f32<NTH>(sW, LK, a.W + rec * kC * DK, DK, kC, DK);
+      store_state_t<NTH, DK, SW>(a.dSc + rec * DK * DV + c0, DV, sDt, LK);
+      load_f32<NTH>(sQpt, kLC, a.Qpt + rec * kC * DK, kC, DK, kC);
+      load_f32<NTH>(sWt, kLC, a.Wt + rec * kC * DK, kC, DK, kC);
       cp_commit();
-      cp_wait_group<1>();  // this chunk's Aqk, Kbar, gamma, dO (Q+ and W may still be in flight)
+      cp_wait_group<1>();  // this chunk's Aqk^T, Kbar, gamma, dO (Q+^T and W^T may still be in flight)
       __syncthreads();
-      for (int idx = tid; idx < kC * SW; idx += NTH) {  // dO columns to fp32 (zeros past the tail)
-        const int i = idx / SW, c = idx % SW;
-        sO[i * LS + c] = to_f32(sraw(p)[i * SW + c]);
+      for (int idx = tid; idx < kC * SW; idx += NTH) {  // dO columns to fp32, transposed (zeros past the tail)
+        const int c = idx / kC, i = idx % kC;
+        sOt[c * kLC + i] = to_f32(sraw(p)[i * SW + c]);
       }
       __syncthreads();
       {  // dV' = Aqk^T dO + Kbar dS
         float acc[TV::MT][TV::NT][4];
         zero(acc);
-        warp_mma<TV::MT, TV::NT, X3, kC>(acc, colm(sA(p), kLC), rowm(sO, LS), vm0, vn0);
-        warp_mma<TV::MT, TV::NT, X3, DK>(acc, rowm(sKb(p), LK), rowm(sD, LS), vm0, vn0);
+        warp_mma_kk<TV::MT, TV::NT, X3, kC>(acc, sAt(p), kLC, sOt, kLC, vm0, vn0);
+        warp_mma_kk<TV::MT, TV::NT, X3, DK>(acc, sKb(p), LK, sDt, LK, vm0, vn0);
         float* dvp = a.dVp + rec * kC * DV + c0;
         for_acc<TV::MT, TV::NT>(vm0, vn0, [&](int mt, int nt, int e, int i, int c) {
-          sdV[i * LS + c] = acc[mt][nt][e];
+          sdVt[c * kLC + i] = acc[mt][nt][e];
           dvp[i * DV + c] = acc[mt][nt][e];
         });
       }
       if (NB == 2 && n > 0) {
         issue(n - 1, p ^ 1);
-        cp_wait_group<1>();  // Q+ and W of this chunk
+        cp_wait_group<1>();  // Q+^T and W^T of this chunk
       } else {
         cp_wait_group<0>();
       }
       __syncthreads();
       {  // dS = diag(gamma) dS + Q+^T dO - W^T dV'
         float acc[TS::MT][TS::NT][4], neg[TS::MT][TS::NT][4];
-        acc_from(acc, sD, LS, sgm(p), sm0, sn0);
-        warp_mma<TS::MT, TS::NT, X3, kC>(acc, colm(sQp, LK), rowm(sO, LS), sm0, sn0);
-        zero(neg);
-        warp_mma<TS::MT, TS::NT, X3, kC>(neg, colm(sW, LK), rowm(sdV, LS), sm0, sn0);
+        const float* gm = sgm(p);
         for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) {
-          sD[r * LS + c] = acc[mt][nt][e] - neg[mt][nt][e];
+          acc[mt][nt][e] = gm[r] * sDt[c * LK + r];
+        });
+        warp_mma_kk<TS::MT, TS::NT, X3, kC>(acc, sQpt, kLC, sOt, kLC, sm0, sn0);
+        zero(neg);
+        warp_mma_kk<TS::MT, TS::NT, X3, kC>(neg, sWt, kLC, sdVt, kLC, sm0, sn0);
+        for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) {
+          sDt[c * LK + r] = acc[mt][nt][e] - neg[mt][nt][e];
         });
       }
     }
     __syncthreads();
-    if (a.ds0) store_f32<NTH>(a.ds0 + st0 + c0, DV, sD, LS, DK, SW);
+    if (a.ds0) store_state_t<NTH, DK, SW>(a.ds0 + st0 + c0, DV, sDt, LK);
   }
 }
 
@@ -678,13 +783,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);  // dAqk = tril(dO V'^T)
-    warp_mma<Tl::MT, Tl::NT, X3, DV>(acc, rowm(sO, LV), colm(sVp, LV), m0, n0);
+    warp_mma_kk<Tl::MT, Tl::NT, X3, DV>(acc, sO, LV, sVp, LV, m0, n0);
     float* out = a.dAqk + rec * kC * kC;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       out[i * kC + j] = j <= i ? acc[mt][nt][e] : 0.f;
     });
     zero(acc);  // dU (beta V)^T, strictly lower part
-    warp_mma<Tl::MT, Tl::NT, X3, DV>(acc, rowm(sdV, LV), colm(sv, LV), m0, n0);
+    warp_mma_kk<Tl::MT, Tl::NT, X3, DV>(acc, sdV, LV, sv, LV, m0, n0);
     out = a.dT1 + rec * kC * kC;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       out[i * kC + j] = j < i ? acc[mt][nt][e] * sb[j] : 0.f;
@@ -723,15 +828,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
     __syncthreads();
     float acc[Tr::MT][Tr::NT][4];
     zero(acc);
-    warp_mma<Tr::MT, Tr::NT, X3, DV>(acc, rowm(sO, LV), colm(sS0, LV), m0, n0);
+    warp_mma_kk<Tr::MT, Tr::NT, X3, DV>(acc, sO, LV, sS0, LV, m0, n0);
     float* out = a.dQs + rec * kC * DK + rb * 32;
     for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
     zero(acc);
-    warp_mma<Tr::MT, Tr::NT, X3, DV>(acc, rowm(sdV, LV), colm(sS0, LV), m0, n0);
+    warp_mma_kk<Tr::MT, Tr::NT, X3, DV>(acc, sdV, LV, sS0, LV, m0, n0);
     out = a.dW + rec * kC * DK + rb * 32;
     for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = -acc[mt][nt][e]; });
     zero(acc);
-    warp_mma<Tr::MT, Tr::NT, X3, DV>(acc, rowm(sVp, LV), colm(sdS, LV), m0, n0);
+    warp_mma_kk<Tr::MT, Tr::NT, X3, DV>(acc, sVp, LV, sdS, LV, m0, n0);
     out = a.dKb + rec * kC * DK + rb * 32;
     for_acc<Tr::MT, Tr::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
 #pragma unroll
@@ -800,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   {  // dT += dW (beta K+)^T, strictly lower part
     float acc[TC::MT][TC::NT][4];
     zero(acc);
-    warp_mma<TC::MT, TC::NT, X3, DK>(acc, rowm(sY, LK), colm(sX, LK), cm0, cn0);
+    warp_mma_kk<TC::MT, TC::NT, X3, DK>(acc, sY, LK, sX, LK, cm0, cn0);
     for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
       if (j < i) sDT[i * kLC + j] += acc[mt][nt][e] * sb[j];
     });
@@ -821,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   {  // dT T^T
     float acc[TC::MT][TC::NT][4];
     zero(acc);
-    warp_mma<TC::MT, TC::NT, X3, kC>(acc, rowm(sDT, kLC), colm(sT, kLC), cm0, cn0);
+    warp_mma_kk<TC::MT, TC::NT, X3, kC>(acc, sDT, kLC, sT, kLC, cm0, cn0);
     for_acc<TC::MT, TC::NT>(cm0, cn0,
                             [&](int mt, int nt, int e, int i, int j) { sY2[i * kLC + j] = acc[mt][nt][e]; });
   }
@@ -991,14 +1096,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
 // ------------------------------------------------------------------ host
 // Floats of each workspace array per chunk record, in layout order.
 struct WsPlan {
-  size_t W, U, Qp, Kb, Aqk, Tm, Pkk, gam, S0c, dSc, Vp, dVp, dAqk, dT1, dQs, dW, dKb, dgam, dbu;
+  size_t W, U, Qp, Kb, Wt, Qpt, Kbt, Aqk, Tm, Pkk, gam, S0c, dSc, Vp, dVp, dAqk, dT1, dQs, dW, dKb, dgam, dbu;
   explicit WsPlan(int dk, int dv)
-      : W((size_t)kC * dk), U((size_t)kC * dv), Qp((size_t)kC * dk), Kb((size_t)kC * dk), Aqk(kC * kC),
+      : W((size_t)kC * dk), U((size_t)kC * dv), Qp((size_t)kC * dk), Kb((size_t)kC * dk), Wt((size_t)kC * dk),
+        Qpt((size_t)kC * dk), Kbt((size_t)kC * dk), Aqk(kC * kC),
         Tm(kC * kC), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv), dSc((size_t)dk * dv), Vp((size_t)kC * dv),
         dVp((size_t)kC * dv), dAqk(kC * kC), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk),
         dKb((size_t)kC * dk), dgam(dk), dbu(kC) {}
   size_t per_rec() const {
-    return W + U + Qp + Kb + Aqk + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs + dW + dKb + dgam + dbu;
+    return W + U + Qp + Kb + Wt + Qpt + Kbt + Aqk + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs + dW +
+           dKb + dgam + dbu;
   }
 };
 
@@ -1071,6 +1178,7 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
     return r;
   };
   a.W = take(p.W), a.U = take(p.U), a.Qp = take(p.Qp), a.Kb = take(p.Kb);
+  a.Wt = take(p.Wt), a.Qpt = take(p.Qpt), a.Kbt = take(p.Kbt);
   a.Aqk = take(p.Aqk), a.Tm = take(p.Tm), a.Pkk = take(p.Pkk), a.gam = take(p.gam);
   a.S0c = take(p.S0c), a.dSc = take(p.dSc), a.Vp = take(p.Vp), a.dVp = take(p.dVp);
   a.dAqk = take(p.dAqk), a.dT1 = take(p.dT1), a.dQs = take(p.dQs), a.dW = take(p.dW), a.dKb = take(p.dKb);
