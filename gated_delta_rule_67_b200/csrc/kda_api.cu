@@ -239,14 +239,14 @@ kda_status kda_backward(const void* q, const void* k, const void* v, const void*
                            : cudaMemsetAsync(grad_initial_state, 0, state_bytes, stream);
     return from_cuda(e);
   }
-  const size_t need_ws = kda::backward_workspace_bytes(B, T, H, dk, dv);
+  const size_t need_ws = kda::backward_workspace_bytes(1, T, 1, dk, dv);  // one (sequence, head) at a time at least
   if (!workspace || workspace_bytes < need_ws || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
   const Range rw{(const char*)workspace, workspace_bytes};
   for (Range r : {rq, rk, rv, rg, rb, rs0, rdo, rdsT, wq, wk, wv, wg, wb, ws0})
     if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
   return from_cuda(kda::launch_backward(q, k, v, g, beta, scale, initial_state, grad_o, grad_final_state, grad_q,
                                         grad_k, grad_v, grad_g, grad_beta, grad_initial_state, B, T, H, dk, dv, dtype,
-                                        gate, workspace, stream));
+                                        gate, workspace, workspace_bytes, stream));
 }
 
 static kda_status recurrent_step_impl(const void* q, const void* k, const void* v, const void* g,

@@ -41,6 +41,7 @@
 // a_lo b_hi), which keeps fp32-level accuracy; with bf16 I/O one tf32 term.
 // Everything in the workspace is fp32.  No atomics: every sum runs in a fixed
 // order, so results are bit-reproducible.
+#include <algorithm>
 #include <type_traits>
 
 #include "kda_common.cuh"
@@ -361,7 +362,8 @@ struct ChunkBwdArgs {
   float* ds0;
   float scale;
   int T, H, NC, gate;
-  // workspace (fp32), record rec = (b * H + h) * NC + chunk
+  int bh0;  // first (sequence, head) of this launch group: bh = bh0 + local index
+  // workspace (fp32), record rec = (bh - bh0) * NC + chunk
   float *W, *U, *Qp, *Kb;  // [rec][64][d_k] (U: [64][d_v]): W, U, Q+, Kbar
   float *Wt, *Qpt, *Kbt;   // [rec][d_k][64]: their transposes for the state passes
   float *Aqk, *Tm, *Pkk;   // [rec][64][64]: Aqk^T (transposed), T, P
@@ -402,8 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
   float* sb = sT + kC * kLC;  // [64] beta
   float* se = sb + kC;        // [DK] exp(G_ref)
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int n = blockIdx.x % a.NC, bh = blockIdx.x / a.NC, t0 = n * kC, nv = min(kC, a.T - t0);
-  const size_t row0 = row_of(a, bh, t0), rec = (size_t)bh * a.NC + n;
+  const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
   const IO* q = static_cast<const IO*>(a.q);
   const IO* k = static_cast<const IO*>(a.k);
   const IO* beta = static_cast<const IO*>(a.beta);
@@ -600,7 +602,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBw
   using TS = Tiling<DK, SW, NTH / 32>;  // DK x SW products
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int cs = blockIdx.x % NS, bh = blockIdx.x / NS, c0 = cs * SW, NC = a.NC;
+  const int cs = blockIdx.x % NS, lb = blockIdx.x / NS, bh = a.bh0 + lb, c0 = cs * SW, NC = a.NC;
   const size_t st0 = (size_t)bh * DK * DV;
   const int vm0 = TV::m0(warp), vn0 = TV::n0(warp), sm0 = TS::m0(warp), sn0 = TS::n0(warp);
 
@@ -614,7 +616,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBw
     auto sU = [&](int p) { return sbuf + p * PP::buf0 + kC * LK + DK * kLC; };              // [64][LS] U columns
     auto sgm = [&](int p) { return sbuf + p * PP::buf0 + kC * LK + DK * kLC + kC * LS; };   // [DK] gamma
     auto issue = [&](int n, int p) {
-      const size_t rec = (size_t)bh * NC + n;
+      const size_t rec = (size_t)lb * NC + n;
       load_f32<NTH>(sW(p), LK, a.W + rec * kC * DK, DK, kC, DK);
       load_f32<NTH>(sKbt(p), kLC, a.Kbt + rec * kC * DK, kC, DK, kC);
       load_f32<NTH>(sU(p), LS, a.U + rec * kC * DV + c0, DV, kC, SW);
@@ -624,7 +626,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBw
     load_state_t<NTH, DK, SW>(sSt, LK, a.s0 ? a.s0 + st0 + c0 : nullptr, DV);
     issue(0, 0);
     for (int n = 0; n < NC; ++n) {
-      const size_t rec = (size_t)bh * NC + n;
+      const size_t rec = (size_t)lb * NC + n;
       const int p = NB == 2 ? (n & 1) : 0;
       __syncthreads();  // the previous chunk's reads are done
       if (NB == 1 && n > 0) issue(n, 0);
@@ -672,7 +674,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBw
     };
     const IO* d_o = static_cast<const IO*>(a.d_o);
     auto issue = [&](int n, int p) {
-      const size_t rec = (size_t)bh * NC + n;
+      const size_t rec = (size_t)lb * NC + n;
       load_f32<NTH>(sAt(p), kLC, a.Aqk + rec * kC * kC, kC, kC, kC);
       load_f32<NTH>(sKb(p), LK, a.Kb + rec * kC * DK, DK, kC, DK);
       load_f32<NTH>(sgm(p), DK, a.gam + rec * DK, DK, 1, DK);
@@ -692,7 +694,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBw
     load_state_t<NTH, DK, SW>(sDt, LK, a.dsT ? a.dsT + st0 + c0 : nullptr, DV);
     issue(NC - 1, NB == 2 ? ((NC - 1) & 1) : 0);
     for (int n = NC - 1; n >= 0; --n) {
-      const size_t rec = (size_t)bh * NC + n;
+      const size_t rec = (size_t)lb * NC + n;
       const int p = NB == 2 ? (n & 1) : 0;
       __syncthreads();  // the previous chunk's reads are done
       if (NB == 1 && n < NC - 1) issue(n, 0);
@@ -767,8 +769,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
   float* sb = sdS + 32 * LV;   // [64] beta
   float* red = sb + kC;        // [4][64] row sums per column group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = blockIdx.x % a.NC, bh = blockIdx.x / a.NC, t0 = n * kC, nv = min(kC, a.T - t0);
-  const size_t row0 = row_of(a, bh, t0), rec = (size_t)bh * a.NC + n;
+  const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
 
   load_rows<IO, DV>(sO, LV, static_cast<const IO*>(a.d_o), row0, a.H, nv, DV, 0);
   load_rows<IO, DV>(sv, LV, static_cast<const IO*>(a.v), row0, a.H, nv, DV, 0);
@@ -879,8 +881,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   float* red = sb + kC;         // [8][64] row sums per column group: K+ . T^T dW (slots 0-3), dA . P (4-7)
   float* colC = red + 8 * kC;   // [4][DK] column sums of dKbar . Kbar per row group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = blockIdx.x % a.NC, bh = blockIdx.x / a.NC, t0 = n * kC, nv = min(kC, a.T - t0);
-  const size_t row0 = row_of(a, bh, t0), rec = (size_t)bh * a.NC + n;
+  const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
   const IO* q = static_cast<const IO*>(a.q);
   const IO* k = static_cast<const IO*>(a.k);
   const int m0 = TK::m0(warp), n0 = TK::n0(warp), cm0 = TC::m0(warp), cn0 = TC::n0(warp);
@@ -1158,33 +1160,42 @@ size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv) {
   return nrec * WsPlan(dk, dv).per_rec() * sizeof(float);
 }
 
-int backward_launches() { return 4; }
-
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
                             float scale, const float* s0, const void* d_o, const float* dsT, void* dq, void* dk_out,
                             void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H, int dk, int dv,
-                            int dtype, int gate, void* ws, cudaStream_t stream) {
+                            int dtype, int gate, void* ws, size_t ws_bytes, cudaStream_t stream) {
   ChunkBwdArgs a;
   a.q = q, a.k = k, a.v = v, a.g = g, a.beta = beta, a.d_o = d_o;
   a.s0 = s0, a.dsT = dsT;
   a.dq = dq, a.dk = dk_out, a.dv = dv_out, a.dg = dg, a.dbeta = dbeta, a.ds0 = ds0;
   a.scale = scale, a.T = T, a.H = H, a.NC = (T + kC - 1) / kC, a.gate = gate;
-  const size_t nrec = (size_t)B * H * a.NC;
+  // (sequence, head) pairs per launch group: as many as the workspace holds
+  const int BH = B * H;
+  const size_t per_bh = backward_workspace_bytes(1, T, 1, dk, dv);
+  const int nfit = (int)std::min<size_t>((size_t)BH, ws_bytes / per_bh);
+  if (nfit < 1) return cudaErrorInvalidValue;
   const WsPlan p(dk, dv);
-  float* w = static_cast<float*>(ws);
-  auto take = [&](size_t per) {
-    float* r = w;
-    w += nrec * per;
-    return r;
-  };
-  a.W = take(p.W), a.U = take(p.U), a.Qp = take(p.Qp), a.Kb = take(p.Kb);
-  a.Wt = take(p.Wt), a.Qpt = take(p.Qpt), a.Kbt = take(p.Kbt);
-  a.Aqk = take(p.Aqk), a.Tm = take(p.Tm), a.Pkk = take(p.Pkk), a.gam = take(p.gam);
-  a.S0c = take(p.S0c), a.dSc = take(p.dSc), a.Vp = take(p.Vp), a.dVp = take(p.dVp);
-  a.dAqk = take(p.dAqk), a.dT1 = take(p.dT1), a.dQs = take(p.dQs), a.dW = take(p.dW), a.dKb = take(p.dKb);
-  a.dgam = take(p.dgam), a.dbu = take(p.dbu);
-  if (dtype == KDA_F32) return launch_chunk_dims<float>(a, B * H, dk, dv, stream);
-  return launch_chunk_dims<__nv_bfloat16>(a, B * H, dk, dv, stream);
+  for (int bh0 = 0; bh0 < BH; bh0 += nfit) {
+    const int nbh = std::min(nfit, BH - bh0);
+    const size_t nrec = (size_t)nbh * a.NC;
+    float* w = static_cast<float*>(ws);
+    auto take = [&](size_t per) {
+      float* r = w;
+      w += nrec * per;
+      return r;
+    };
+    a.bh0 = bh0;
+    a.W = take(p.W), a.U = take(p.U), a.Qp = take(p.Qp), a.Kb = take(p.Kb);
+    a.Wt = take(p.Wt), a.Qpt = take(p.Qpt), a.Kbt = take(p.Kbt);
+    a.Aqk = take(p.Aqk), a.Tm = take(p.Tm), a.Pkk = take(p.Pkk), a.gam = take(p.gam);
+    a.S0c = take(p.S0c), a.dSc = take(p.dSc), a.Vp = take(p.Vp), a.dVp = take(p.dVp);
+    a.dAqk = take(p.dAqk), a.dT1 = take(p.dT1), a.dQs = take(p.dQs), a.dW = take(p.dW), a.dKb = take(p.dKb);
+    a.dgam = take(p.dgam), a.dbu = take(p.dbu);
+    const cudaError_t e = dtype == KDA_F32 ? launch_chunk_dims<float>(a, nbh, dk, dv, stream)
+                                           : launch_chunk_dims<__nv_bfloat16>(a, nbh, dk, dv, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace kda

@@ -41,12 +41,14 @@ cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, 
                                 int dk, int dv, int chunk, int gate, int prep, void* ws, size_t ws_bytes,
                                 cudaStream_t stream, void* const* events);
 
-// Backward pass (kda_backward.cu).
+// Backward pass (kda_backward_chunk.cu).  The workspace holds the records of
+// one or more (sequence, head) pairs; the pairs are processed in groups of
+// as many as fit (at least backward_workspace_bytes(1, T, 1, dk, dv) bytes).
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
                             float scale, const float* s0, const void* d_o, const float* dsT, void* dq, void* dk_out,
                             void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H, int dk, int dv,
-                            int dtype, int gate, void* ws, cudaStream_t stream);
+                            int dtype, int gate, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // Launches a kernel whose only wait can never be satisfied (short limit).
 cudaError_t launch_wait_selftest(void* ws, cudaStream_t stream);

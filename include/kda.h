@@ -188,8 +188,13 @@ KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, 
  *                      head), written; ignored (NULL allowed) for KDA_GATE_NONE
  *   grad_beta        : [B, T, H] (dtype), written
  *   grad_initial_state : [B, H, dk, dv] fp32 dL/dS_0, or NULL to skip
- *   workspace        : at least kda_backward_workspace_size() bytes, 16-byte
- *                      aligned; contents on entry do not matter
+ *   workspace        : 16-byte aligned, contents on entry do not matter;
+ *                      kda_backward_workspace_size() bytes hold every
+ *                      (sequence, head) at once.  A smaller workspace works
+ *                      too, down to kda_backward_workspace_size(1, T, 1, ...)
+ *                      (one pair): the pairs are then processed in groups of
+ *                      as many as fit, four launches per group, in order on
+ *                      the stream (results identical)
  *
  * Supported: dtype KDA_F32 or KDA_BF16, dk and dv in {64, 128}.  Pointers
  * 16-byte aligned (beta, grad_beta and per-head g / grad_g: element

@@ -173,6 +173,9 @@ def test_backward_validation(lib):
     assert call(dk=96) == binding.KDA_ERR_UNSUPPORTED
     assert call(ws=None) == binding.KDA_ERR_INVALID_ARG
     assert call(wsb=16) == binding.KDA_ERR_INVALID_ARG
+    one = lib.kda_backward_workspace_size(1, 64, 1, 128, 128, 1)
+    assert call(wsb=one - 1) == binding.KDA_ERR_INVALID_ARG           # below one (sequence, head)'s records
+    assert lib.kda_backward_workspace_size(2, 64, 3, 128, 128, 1) == 6 * one
     bad = list(grads)
     bad[0] = A + 64                                                   # grad_q overlaps q
     assert call(grads=bad) == binding.KDA_ERR_INVALID_ARG

@@ -110,3 +110,21 @@ def test_backward_exact_pairwise_path(dtype):
     ref = oracle.kda_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dk ** -0.5, x["initial_state"], d_o, d_s)
     for name in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
         assert rel_err(got[name], ref[name]) < TOL[dtype], (name, rel_err(got[name], ref[name]))
+
+
+@pytest.mark.parametrize("fit", [1, 2, 4], ids=["one-pair", "two-pairs", "four-pairs"])
+def test_backward_small_workspace_groups(fit):
+    """A workspace for `fit` (sequence, head) pairs processes the 6 pairs in
+    groups; the result is bit-identical to the one-group call."""
+    dev = cuda_or_skip()
+    from gated_delta_rule_67_b200.binding import load
+    B, T, H = 2, 130, 3
+    x = make_prefill_inputs(B, T, H, 128, 128, torch.bfloat16, 0.1, seed=100, device=dev)
+    d_o, d_s = make_cotangents(B, T, H, 128, 128, torch.bfloat16, seed=101, device=dev)
+    args = (x["q"], x["k"], x["v"], x["g"], x["beta"], d_o, None, x["initial_state"], d_s)
+    one = int(load().kda_backward_workspace_size(1, T, 1, 128, 128, 1))
+    full = kda_backward(*args)
+    part = kda_backward(*args, workspace=torch.empty(fit * one + 8, dtype=torch.uint8, device=dev))
+    torch.cuda.synchronize()
+    for n in full:
+        assert torch.equal(full[n], part[n]), n
