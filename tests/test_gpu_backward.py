@@ -128,3 +128,36 @@ def test_backward_small_workspace_groups(fit):
     torch.cuda.synchronize()
     for n in full:
         assert torch.equal(full[n], part[n]), n
+
+
+@pytest.mark.parametrize("gate", ["channel", "head"])
+def test_backward_matches_gpu_forward_directional_derivative(gate):
+    """Independent of the oracle: for L = <dO, o> + <dS_T, S_T> computed from
+    the library's own fp32 forward, the central difference of L along a random
+    direction of (q, k, v, g, beta, S_0) equals the sum of the backward's
+    gradients times that direction."""
+    from gated_delta_rule_67_b200 import kda_chunk_fwd
+    dev = cuda_or_skip()
+    B, T, H, dk, dv = 1, 150, 2, 64, 64
+    x = make_prefill_inputs(B, T, H, dk, dv, torch.float32, 0.1, seed=102, device=dev)
+    if gate == "head":
+        x["g"] = make_head_gates((B, T, H), 1, torch.float32, seed=103, device=dev)
+    d_o, d_s = make_cotangents(B, T, H, dk, dv, torch.float32, seed=104, device=dev)
+    names = ("q", "k", "v", "g", "beta", "initial_state")
+    gen = torch.Generator(device="cpu").manual_seed(105)
+    direction = {n: (0.1 * torch.randn(x[n].shape, generator=gen)).to(dev) for n in names}
+    scale = dk ** -0.5
+
+    def loss(eps):
+        y = {n: x[n] + eps * direction[n] for n in names}
+        o, s = kda_chunk_fwd(y["q"], y["k"], y["v"], y["g"], y["beta"], scale, y["initial_state"])
+        torch.cuda.synchronize()
+        return float((o.double() * d_o.double()).sum() + (s.double() * d_s.double()).sum())
+
+    eps = 1e-2
+    fd = (loss(eps) - loss(-eps)) / (2 * eps)
+    gr = kda_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d_o, scale, x["initial_state"], d_s)
+    torch.cuda.synchronize()
+    key = dict(q="dq", k="dk", v="dv", g="dg", beta="dbeta", initial_state="dS0")
+    dot = sum(float((gr[key[n]].double() * direction[n].double()).sum()) for n in names)
+    assert abs(fd - dot) <= 1e-3 * abs(dot) + 1e-3, (fd, dot)
