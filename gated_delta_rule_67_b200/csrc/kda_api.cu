@@ -187,7 +187,7 @@ size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, int dtyp
   if (B < 0 || T < 0 || H < 1) return 0;
   if (dtype != KDA_F32 && dtype != KDA_BF16) return 0;
   if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return 0;
-  return kda::backward_workspace_bytes(B, T, H, dk, dv);
+  return kda::backward_workspace_bytes(B, T, H, dk, dv, dtype);
 }
 
 kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
@@ -239,7 +239,7 @@ kda_status kda_backward(const void* q, const void* k, const void* v, const void*
                            : cudaMemsetAsync(grad_initial_state, 0, state_bytes, stream);
     return from_cuda(e);
   }
-  const size_t need_ws = kda::backward_workspace_bytes(1, T, 1, dk, dv);  // one (sequence, head) at a time at least
+  const size_t need_ws = kda::backward_workspace_bytes(1, T, 1, dk, dv, dtype);  // one (sequence, head) at least
   if (!workspace || workspace_bytes < need_ws || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
   const Range rw{(const char*)workspace, workspace_bytes};
   for (Range r : {rq, rk, rv, rg, rb, rs0, rdo, rdsT, wq, wk, wv, wg, wb, ws0})

@@ -365,8 +365,9 @@ struct ChunkBwdArgs {
   int bh0;  // first (sequence, head) of this launch group: bh = bh0 + local index
   // workspace (fp32), record rec = (bh - bh0) * NC + chunk
   float *W, *U, *Qp, *Kb;  // [rec][64][d_k] (U: [64][d_v]): W, U, Q+, Kbar
-  float *Wt, *Qpt, *Kbt;   // [rec][d_k][64]: their transposes for the state passes
-  float *Aqk, *Tm, *Pkk;   // [rec][64][64]: Aqk^T (transposed), T, P
+  float *Wt, *Qpt, *Kbt;   // [rec][d_k][64]: their transposes for the state passes (fp32 inputs)
+  float *Aqk, *Tm, *Pkk;   // [rec][64][64]: Aqk^T (transposed; fp32 inputs), T, P
+  __nv_bfloat16* prec;     // bf16 inputs: [rec] bf16 pass record (W, W^T, Kbar, Kbar^T, Q+^T, Aqk^T)
   float* gam;              // [rec][d_k]: gamma
   float *S0c, *dSc;        // [rec][d_k][d_v]: state entering the chunk, dL/d(state leaving it)
   float *Vp, *dVp;         // [rec][64][d_v]: V', dV'
@@ -379,6 +380,25 @@ struct ChunkBwdArgs {
 __device__ __forceinline__ size_t row_of(const ChunkBwdArgs& a, int bh, int t0) {
   return ((size_t)(bh / a.H) * a.T + t0) * a.H + bh % a.H;
 }
+
+// Element offsets of the bf16 pass record of one chunk (bf16 inputs): the
+// state passes' operands in their shared-memory layout, rows padded by 16
+// bytes.  Part 1 (Aqk^T, Kbar, Q+^T, W^T) feeds the reverse sweep, part 0
+// (W, Kbar^T) the forward replay.
+using bf16 = __nv_bfloat16;
+template <int DK>
+struct PassRec {  // element offsets of the bf16 pass record of one chunk
+  static constexpr int LKb = DK + 8, LCb = kC + 8;
+  static constexpr int oAqkt = 0;                 // [64][LCb]  Aqk^T      (reverse sweep)
+  static constexpr int oKb = oAqkt + kC * LCb;    // [64][LKb]  Kbar
+  static constexpr int oQpt = oKb + kC * LKb;     // [DK][LCb]  Q+^T
+  static constexpr int oWt = oQpt + DK * LCb;     // [DK][LCb]  W^T
+  static constexpr int n1 = oWt + DK * LCb;       // end of the reverse sweep's part
+  static constexpr int oW = n1;                   // [64][LKb]  W          (forward replay)
+  static constexpr int oKbt = oW + kC * LKb;      // [DK][LCb]  Kbar^T
+  static constexpr int n = oKbt + DK * LCb;
+  static_assert(oKb % 8 == 0 && oQpt % 8 == 0 && oWt % 8 == 0 && n1 % 8 == 0 && oKbt % 8 == 0 && n % 8 == 0, "16 B");
+};
 
 // ------------------------------------------------------------------ kernel 1
 template <int DK, int DV>
@@ -422,8 +442,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
   for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+^T and Kbar^T (the same values as Q+, Kbar below)
     const int r = idx / kC, i = idx % kC;
     const float G = sG[i * LK + r], qq = a.scale * sQ[i * LK + r];
-    a.Qpt[rec * kC * DK + idx] = qq * expf(G);
-    a.Kbt[rec * kC * DK + idx] = sK[i * LK + r] * expf(sG[(kC - 1) * LK + r] - G);
+    const float qp = qq * expf(G), kb = sK[i * LK + r] * expf(sG[(kC - 1) * LK + r] - G);
+    if constexpr (X3) {
+      a.Qpt[rec * kC * DK + idx] = qp;
+      a.Kbt[rec * kC * DK + idx] = kb;
+    } else {
+      bf16* pr = a.prec + rec * PassRec<DK>::n;
+      pr[PassRec<DK>::oQpt + r * PassRec<DK>::LCb + i] = __float2bfloat16_rn(qp);
+      pr[PassRec<DK>::oKbt + r * PassRec<DK>::LCb + i] = __float2bfloat16_rn(kb);
+    }
   }
   float* Qp = a.Qp + rec * kC * DK;
   float* Kb = a.Kb + rec * kC * DK;
@@ -434,6 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     const float gm = expf(G);
     Qp[i * DK + r] = qq * gm;
     Kb[i * DK + r] = kk * expf(sG[(kC - 1) * LK + r] - G);
+    if constexpr (!X3)
+      a.prec[rec * PassRec<DK>::n + PassRec<DK>::oKb + i * PassRec<DK>::LKb + r] = __float2bfloat16_rn(Kb[i * DK + r]);
     if (!slow) {
       const float d = G - sG[kRef * LK + r];
       const float ex = expf(d);
@@ -480,7 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
   store_f32(a.Pkk + rec * kC * kC, kC, sP, kLC, kC, kC);
   for (int idx = tid; idx < kC * kC; idx += kThreads) {  // Aqk^T
     const int j = idx / kC, i = idx % kC;
-    a.Aqk[rec * kC * kC + idx] = sA[i * kLC + j];
+    if constexpr (X3)
+      a.Aqk[rec * kC * kC + idx] = sA[i * kLC + j];
+    else
+      a.prec[rec * PassRec<DK>::n + PassRec<DK>::oAqkt + j * PassRec<DK>::LCb + i] = __float2bfloat16_rn(sA[i * kLC + j]);
   }
 
   // T = (I + diag(beta) P)^-1 (unit lower triangular) by forward substitution
@@ -518,12 +550,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);
     warp_mma<Tl::MT, Tl::NT, X3, kC>(acc, rowm(sT, kLC), rowm(sX, LK), m0, n0);
-    float* Wg = a.W + rec * kC * DK;
-    float* Wtg = a.Wt + rec * kC * DK;
-    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
-      Wg[i * DK + c] = acc[mt][nt][e];
-      Wtg[c * kC + i] = acc[mt][nt][e];
-    });
+    if constexpr (X3) {
+      float* Wg = a.W + rec * kC * DK;
+      float* Wtg = a.Wt + rec * kC * DK;
+      for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
+        Wg[i * DK + c] = acc[mt][nt][e];
+        Wtg[c * kC + i] = acc[mt][nt][e];
+      });
+    } else {
+      using PR = PassRec<DK>;
+      bf16* pr = a.prec + rec * PR::n;
+      for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
+        const bf16 w = __float2bfloat16_rn(acc[mt][nt][e]);
+        pr[PR::oW + i * PR::LKb + c] = w;
+        pr[PR::oWt + c * PR::LCb + i] = w;
+      });
+    }
   }
   {
     using Tl = Tiling<kC, DV>;
@@ -743,6 +785,248 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBw
     }
     __syncthreads();
     if (a.ds0) store_state_t<NTH, DK, SW>(a.ds0 + st0 + c0, DV, sDt, LK);
+  }
+}
+
+// ------------------------------------------------------------------ kernel 2 (bf16 operands)
+// With bf16 inputs the state passes run on bf16 operand images and
+// mma.m16n8k16 (bf16 in, fp32 accumulation); the state itself stays in fp32
+// registers for the whole chain and is rounded only as an operand image.
+// The prep kernel writes each chunk's pass operands as one bf16 record in
+// the shared-memory layout (rows padded by 16 bytes), so a chunk's operands
+// arrive by one contiguous cp.async copy.
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4_b(uint32_t (&r)[4], const bf16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const bf16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], const bf16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+
+// acc[MT][NT] (rows m0.., columns n0..) += A[m0.., 0:K] B[0:K, n0..] with A
+// [M][lda] and B [K][ldb] bf16 row-major: A fragments by ldmatrix, B
+// fragments by ldmatrix.trans (k x n blocks read as their transposes).
+// Row starts 16-byte aligned; row strides = 16 (mod 128) bytes avoid conflicts.
+template <int MT, int NT, int K>
+__device__ __forceinline__ void warp_mma_bf16(float (&acc)[MT][NT][4], const bf16* A, int lda, const bf16* B, int ldb,
+                                              int m0, int n0) {
+  const int lane = threadIdx.x & 31, mat = lane >> 3, rr = lane & 7;
+  const bf16* pa = A + (m0 + rr + 8 * (mat & 1)) * lda + 8 * (mat >> 1);
+  const bf16* pb = B + (rr + 8 * (mat & 1)) * ldb + n0 + 8 * (mat >> 1);
+  const bf16* pb1 = B + (rr + 8 * (mat & 1)) * ldb + n0 + 8 * (NT - 1);  // odd NT: last tile (lanes 0-15)
+#pragma unroll
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    uint32_t af[MT][4], bfr[NT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) ldsm_x4_b(af[mt], pa + 16 * mt * lda + k0);
+#pragma unroll
+    for (int np = 0; np < NT / 2; ++np) {
+      uint32_t r[4];
+      ldsm_x4_t(r, pb + k0 * ldb + 16 * np);
+      bfr[2 * np][0] = r[0], bfr[2 * np][1] = r[1], bfr[2 * np + 1][0] = r[2], bfr[2 * np + 1][1] = r[3];
+    }
+    if constexpr (NT % 2 == 1) {
+      uint32_t r[2];
+      ldsm_x2_t(r, pb1 + k0 * ldb);
+      bfr[NT - 1][0] = r[0], bfr[NT - 1][1] = r[1];
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc[mt][nt], af[mt], bfr[nt][0], bfr[nt][1]);
+  }
+}
+
+// The accumulator tile as a bf16 image: rows and column pairs of this lane.
+template <int MT, int NT>
+__device__ __forceinline__ void acc_to_bf16(const float (&acc)[MT][NT][4], bf16* img, int ld, int m0, int n0) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = m0 + 16 * mt + g + 8 * hh, c = n0 + 8 * nt + 2 * t;
+        *reinterpret_cast<__nv_bfloat162*>(img + r * ld + c) =
+            __floats2bfloat162_rn(acc[mt][nt][2 * hh], acc[mt][nt][2 * hh + 1]);
+      }
+}
+// ... and as fp32 into a [rows][gld] global array (column pairs as float2).
+template <int MT, int NT>
+__device__ __forceinline__ void acc_to_global(const float (&acc)[MT][NT][4], float* g0, size_t gld, int m0, int n0) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = m0 + 16 * mt + g + 8 * hh, c = n0 + 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(g0 + r * gld + c) = make_float2(acc[mt][nt][2 * hh], acc[mt][nt][2 * hh + 1]);
+      }
+}
+
+template <int DK, int DV, int SW>
+struct PassPlanB {  // bytes
+  using R = PassRec<DK>;
+  static constexpr int LS = SW + 8;  // bf16 images of the state / V' / dV' / dO columns
+  static constexpr size_t img = (size_t)(DK + kC) * LS * 2;
+  static constexpr size_t buf0 = (size_t)(R::n - R::n1) * 2 + DK * 4 + (size_t)kC * SW * 4;  // W, Kbar^T, gamma, U
+  static constexpr size_t buf1 = (size_t)R::n1 * 2 + DK * 4 + (size_t)kC * LS * 2;          // part 1, gamma, dO
+  static constexpr size_t bytes = img + 2 * (buf0 > buf1 ? buf0 : buf1);
+  static_assert(img % 16 == 0 && buf0 % 16 == 0 && buf1 % 16 == 0, "16 B");
+};
+template <int DK, int DV, int SW>
+constexpr size_t pass_bf16_smem() {
+  return PassPlanB<DK, DV, SW>::bytes;
+}
+
+template <int DK, int DV, int SW>
+__global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const ChunkBwdArgs a) {
+  using PB = PassPlanB<DK, DV, SW>;
+  using R = PassRec<DK>;
+  constexpr int LS = PB::LS, NS = DV / SW, NTH = kPassThreads;
+  constexpr size_t BUF = PB::buf0 > PB::buf1 ? PB::buf0 : PB::buf1;
+  using TV = Tiling<kC, SW, NTH / 32>;  // 64 x SW products
+  using TS = Tiling<DK, SW, NTH / 32>;  // DK x SW products (the state, in registers)
+  extern __shared__ __align__(16) uint8_t smb[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int cs = blockIdx.x % NS, lb = blockIdx.x / NS, bh = a.bh0 + lb, c0 = cs * SW, NC = a.NC;
+  const size_t st0 = (size_t)bh * DK * DV;
+  const int vm0 = TV::m0(warp), vn0 = TV::n0(warp), sm0 = TS::m0(warp), sn0 = TS::n0(warp);
+  bf16* simg = reinterpret_cast<bf16*>(smb);      // [DK][LS] state (or dS) image
+  bf16* vimg = simg + DK * LS;                    // [64][LS] V' (or dV') image
+  uint8_t* bufs = smb + PB::img;
+  auto cp16 = [&](void* dst, const void* src, int bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(bytes)
+                 : "memory");
+  };
+  auto copy = [&](uint8_t* dst, const void* src, size_t bytes) {  // bytes % 16 == 0
+    const uint8_t* s = static_cast<const uint8_t*>(src);
+    for (size_t o = (size_t)tid * 16; o < bytes; o += (size_t)NTH * 16) cp16(dst + o, s + o, 16);
+  };
+  float st[TS::MT][TS::NT][4];  // the state (or dS) columns of this warp's tile
+  const float* init = blockIdx.y == 0 ? a.s0 : a.dsT;
+  for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) {
+    st[mt][nt][e] = init ? init[st0 + (size_t)r * DV + c0 + c] : 0.f;
+  });
+
+  if (blockIdx.y == 0) {
+    // buffer: W [64][LKb], Kbar^T [DK][LCb] (bf16), gamma [DK], U columns [64][SW] (fp32)
+    auto bW = [&](int p) { return reinterpret_cast<const bf16*>(bufs + p * BUF); };
+    auto bKbt = [&](int p) { return bW(p) + (R::oKbt - R::oW); };
+    auto bgm = [&](int p) { return reinterpret_cast<const float*>(bufs + p * BUF + (R::n - R::n1) * 2); };
+    auto bU = [&](int p) { return bgm(p) + DK; };
+    auto issue = [&](int n, int p) {
+      const size_t rec = (size_t)lb * NC + n;
+      uint8_t* b = bufs + p * BUF;
+      copy(b, a.prec + rec * R::n + R::n1, (size_t)(R::n - R::n1) * 2);
+      copy(b + (R::n - R::n1) * 2, a.gam + rec * DK, DK * 4);
+      float* u = const_cast<float*>(bU(p));
+      const float* ug = a.U + rec * kC * DV + c0;
+      for (int idx = tid; idx < kC * (SW / 4); idx += NTH) {
+        const int i = idx / (SW / 4), c = (idx % (SW / 4)) * 4;
+        cp16(u + i * SW + c, ug + (size_t)i * DV + c, 16);
+      }
+      cp_commit();
+    };
+    issue(0, 0);
+    for (int n = 0; n < NC; ++n) {
+      const size_t rec = (size_t)lb * NC + n;
+      const int p = n & 1;
+      acc_to_bf16(st, simg, LS, sm0, sn0);
+      acc_to_global(st, a.S0c + rec * DK * DV + c0, DV, sm0, sn0);
+      cp_wait_group<0>();
+      __syncthreads();
+      if (n + 1 < NC) issue(n + 1, p ^ 1);
+      {  // V' = U - W S
+        float acc[TV::MT][TV::NT][4];
+        zero(acc);
+        warp_mma_bf16<TV::MT, TV::NT, DK>(acc, bW(p), R::LKb, simg, LS, vm0, vn0);
+        const float* u = bU(p);
+        for_acc<TV::MT, TV::NT>(vm0, vn0,
+                                [&](int mt, int nt, int e, int i, int c) { acc[mt][nt][e] = u[i * SW + c] - acc[mt][nt][e]; });
+        acc_to_bf16(acc, vimg, LS, vm0, vn0);
+        acc_to_global(acc, a.Vp + rec * kC * DV + c0, DV, vm0, vn0);
+      }
+      __syncthreads();
+      {  // S = diag(gamma) S + Kbar^T V'
+        const float* gm = bgm(p);
+        for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) { st[mt][nt][e] *= gm[r]; });
+        warp_mma_bf16<TS::MT, TS::NT, kC>(st, bKbt(p), R::LCb, vimg, LS, sm0, sn0);
+      }
+    }
+  } else {
+    // buffer: record part 1 (Aqk^T, Kbar, Q+^T, W^T; bf16), gamma [DK], dO columns [64][LS] (bf16)
+    auto bR = [&](int p) { return reinterpret_cast<const bf16*>(bufs + p * BUF); };
+    auto bgm = [&](int p) { return reinterpret_cast<const float*>(bufs + p * BUF + R::n1 * 2); };
+    auto bO = [&](int p) { return reinterpret_cast<const bf16*>(bufs + p * BUF + R::n1 * 2 + DK * 4); };
+    const bf16* d_o = static_cast<const bf16*>(a.d_o);
+    auto issue = [&](int n, int p) {
+      const size_t rec = (size_t)lb * NC + n;
+      uint8_t* b = bufs + p * BUF;
+      copy(b, a.prec + rec * R::n, (size_t)R::n1 * 2);
+      copy(b + R::n1 * 2, a.gam + rec * DK, DK * 4);
+      constexpr int PER = SW / 8;  // 16-byte pieces per row
+      const int t0 = n * kC, nv = min(kC, a.T - t0);
+      const size_t r0 = row_of(a, bh, t0);
+      bf16* o = const_cast<bf16*>(bO(p));
+      for (int idx = tid; idx < kC * PER; idx += NTH) {
+        const int i = idx / PER, c = (idx % PER) * 8;
+        cp16(o + i * LS + c, i < nv ? d_o + (r0 + (size_t)i * a.H) * DV + c0 + c : d_o, i < nv ? 16 : 0);
+      }
+      cp_commit();
+    };
+    issue(NC - 1, (NC - 1) & 1);
+    for (int n = NC - 1; n >= 0; --n) {
+      const size_t rec = (size_t)lb * NC + n;
+      const int p = n & 1;
+      acc_to_bf16(st, simg, LS, sm0, sn0);
+      acc_to_global(st, a.dSc + rec * DK * DV + c0, DV, sm0, sn0);
+      cp_wait_group<0>();
+      __syncthreads();
+      if (n > 0) issue(n - 1, p ^ 1);
+      const bf16* rp = bR(p);
+      {  // dV' = Aqk^T dO + Kbar dS
+        float acc[TV::MT][TV::NT][4];
+        zero(acc);
+        warp_mma_bf16<TV::MT, TV::NT, kC>(acc, rp + R::oAqkt, R::LCb, bO(p), LS, vm0, vn0);
+        warp_mma_bf16<TV::MT, TV::NT, DK>(acc, rp + R::oKb, R::LKb, simg, LS, vm0, vn0);
+        acc_to_bf16(acc, vimg, LS, vm0, vn0);
+        acc_to_global(acc, a.dVp + rec * kC * DV + c0, DV, vm0, vn0);
+      }
+      __syncthreads();
+      {  // dS = diag(gamma) dS + Q+^T dO - W^T dV'
+        const float* gm = bgm(p);
+        float neg[TS::MT][TS::NT][4];
+        for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) { st[mt][nt][e] *= gm[r]; });
+        warp_mma_bf16<TS::MT, TS::NT, kC>(st, rp + R::oQpt, R::LCb, bO(p), LS, sm0, sn0);
+        zero(neg);
+        warp_mma_bf16<TS::MT, TS::NT, kC>(neg, rp + R::oWt, R::LCb, vimg, LS, sm0, sn0);
+        for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) { st[mt][nt][e] -= neg[mt][nt][e]; });
+      }
+    }
+    if (a.ds0)
+      for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) {
+        a.ds0[st0 + (size_t)r * DV + c0 + c] = st[mt][nt][e];
+      });
   }
 }
 
@@ -1098,16 +1382,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
 // ------------------------------------------------------------------ host
 // Floats of each workspace array per chunk record, in layout order.
 struct WsPlan {
-  size_t W, U, Qp, Kb, Wt, Qpt, Kbt, Aqk, Tm, Pkk, gam, S0c, dSc, Vp, dVp, dAqk, dT1, dQs, dW, dKb, dgam, dbu;
-  explicit WsPlan(int dk, int dv)
-      : W((size_t)kC * dk), U((size_t)kC * dv), Qp((size_t)kC * dk), Kb((size_t)kC * dk), Wt((size_t)kC * dk),
-        Qpt((size_t)kC * dk), Kbt((size_t)kC * dk), Aqk(kC * kC),
+  size_t W, U, Qp, Kb, Wt, Qpt, Kbt, Aqk, prec, Tm, Pkk, gam, S0c, dSc, Vp, dVp, dAqk, dT1, dQs, dW, dKb, dgam, dbu;
+  // fp32 inputs keep the passes' operands as fp32 arrays, bf16 inputs as one bf16 record per chunk
+  explicit WsPlan(int dk, int dv, bool f32)
+      : W(f32 ? (size_t)kC * dk : 0), U((size_t)kC * dv), Qp((size_t)kC * dk), Kb((size_t)kC * dk),
+        Wt(f32 ? (size_t)kC * dk : 0), Qpt(f32 ? (size_t)kC * dk : 0), Kbt(f32 ? (size_t)kC * dk : 0),
+        Aqk(f32 ? kC * kC : 0), prec(f32 ? 0 : (dk == 128 ? PassRec<128>::n : PassRec<64>::n) / 2),
         Tm(kC * kC), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv), dSc((size_t)dk * dv), Vp((size_t)kC * dv),
         dVp((size_t)kC * dv), dAqk(kC * kC), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk),
         dKb((size_t)kC * dk), dgam(dk), dbu(kC) {}
   size_t per_rec() const {
-    return W + U + Qp + Kb + Wt + Qpt + Kbt + Aqk + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs + dW +
-           dKb + dgam + dbu;
+    return W + U + Qp + Kb + Wt + Qpt + Kbt + Aqk + prec + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs +
+           dW + dKb + dgam + dbu;
   }
 };
 
@@ -1129,12 +1415,22 @@ cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t strea
   const dim3 grid((unsigned)a.NC * BH);  // chunk-major within each (sequence, head)
   cudaError_t e = launch_k(bwd_prep_kernel<IO, DK, DV>, grid, prep_smem<DK, DV>(), a, stream);
   if (e != cudaSuccess) return e;
-  if (pass_width(BH, DV) == 32)
-    e = launch_k(bwd_pass_kernel<IO, DK, DV, 32>, dim3(BH * (DV / 32), 2), pass_smem<DK, DV, 32>(), a, stream,
-                 kPassThreads);
-  else
-    e = launch_k(bwd_pass_kernel<IO, DK, DV, 64>, dim3(BH * (DV / 64), 2), pass_smem<DK, DV, 64>(), a, stream,
-                 kPassThreads);
+  const bool w32 = pass_width(BH, DV) == 32;
+  if constexpr (std::is_same<IO, float>::value) {
+    if (w32)
+      e = launch_k(bwd_pass_kernel<IO, DK, DV, 32>, dim3(BH * (DV / 32), 2), pass_smem<DK, DV, 32>(), a, stream,
+                   kPassThreads);
+    else
+      e = launch_k(bwd_pass_kernel<IO, DK, DV, 64>, dim3(BH * (DV / 64), 2), pass_smem<DK, DV, 64>(), a, stream,
+                   kPassThreads);
+  } else {
+    if (w32)
+      e = launch_k(bwd_pass_bf16_kernel<DK, DV, 32>, dim3(BH * (DV / 32), 2), pass_bf16_smem<DK, DV, 32>(), a,
+                   stream, kPassThreads);
+    else
+      e = launch_k(bwd_pass_bf16_kernel<DK, DV, 64>, dim3(BH * (DV / 64), 2), pass_bf16_smem<DK, DV, 64>(), a,
+                   stream, kPassThreads);
+  }
   if (e != cudaSuccess) return e;
   e = launch_k(bwd_local_a_kernel<IO, DK, DV>, grid, local_a_smem<DK, DV>(), a, stream);
   if (e != cudaSuccess) return e;
@@ -1155,9 +1451,9 @@ static_assert(prep_smem<128, 128>() <= 232448 && local_a_smem<128, 128>() <= 232
 
 }  // namespace
 
-size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv) {
+size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
   const size_t nrec = (size_t)B * H * (((size_t)T + kC - 1) / kC);
-  return nrec * WsPlan(dk, dv).per_rec() * sizeof(float);
+  return nrec * WsPlan(dk, dv, dtype == KDA_F32).per_rec() * sizeof(float);
 }
 
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -1171,10 +1467,10 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
   a.scale = scale, a.T = T, a.H = H, a.NC = (T + kC - 1) / kC, a.gate = gate;
   // (sequence, head) pairs per launch group: as many as the workspace holds
   const int BH = B * H;
-  const size_t per_bh = backward_workspace_bytes(1, T, 1, dk, dv);
+  const size_t per_bh = backward_workspace_bytes(1, T, 1, dk, dv, dtype);
   const int nfit = (int)std::min<size_t>((size_t)BH, ws_bytes / per_bh);
   if (nfit < 1) return cudaErrorInvalidValue;
-  const WsPlan p(dk, dv);
+  const WsPlan p(dk, dv, dtype == KDA_F32);
   for (int bh0 = 0; bh0 < BH; bh0 += nfit) {
     const int nbh = std::min(nfit, BH - bh0);
     const size_t nrec = (size_t)nbh * a.NC;
@@ -1187,7 +1483,8 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
     a.bh0 = bh0;
     a.W = take(p.W), a.U = take(p.U), a.Qp = take(p.Qp), a.Kb = take(p.Kb);
     a.Wt = take(p.Wt), a.Qpt = take(p.Qpt), a.Kbt = take(p.Kbt);
-    a.Aqk = take(p.Aqk), a.Tm = take(p.Tm), a.Pkk = take(p.Pkk), a.gam = take(p.gam);
+    a.Aqk = take(p.Aqk), a.prec = reinterpret_cast<bf16*>(take(p.prec));
+    a.Tm = take(p.Tm), a.Pkk = take(p.Pkk), a.gam = take(p.gam);
     a.S0c = take(p.S0c), a.dSc = take(p.dSc), a.Vp = take(p.Vp), a.dVp = take(p.dVp);
     a.dAqk = take(p.dAqk), a.dT1 = take(p.dT1), a.dQs = take(p.dQs), a.dW = take(p.dW), a.dKb = take(p.dKb);
     a.dgam = take(p.dgam), a.dbu = take(p.dbu);

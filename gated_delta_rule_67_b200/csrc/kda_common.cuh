@@ -43,8 +43,8 @@ cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, 
 
 // Backward pass (kda_backward_chunk.cu).  The workspace holds the records of
 // one or more (sequence, head) pairs; the pairs are processed in groups of
-// as many as fit (at least backward_workspace_bytes(1, T, 1, dk, dv) bytes).
-size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv);
+// as many as fit (at least backward_workspace_bytes(1, T, 1, dk, dv, dtype) bytes).
+size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
                             float scale, const float* s0, const void* d_o, const float* dsT, void* dq, void* dk_out,
                             void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H, int dk, int dv,
