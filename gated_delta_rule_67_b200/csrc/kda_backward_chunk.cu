@@ -812,37 +812,60 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const bf16* p) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"((uint32_t)__cvta_generic_to_shared(p)));
 }
+__device__ __forceinline__ void ldsm_x2_b(uint32_t (&r)[2], const bf16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
 __device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], const bf16* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
                : "=r"(r[0]), "=r"(r[1])
                : "r"((uint32_t)__cvta_generic_to_shared(p)));
 }
 
-// acc[MT][NT] (rows m0.., columns n0..) += A[m0.., 0:K] B[0:K, n0..] with A
-// [M][lda] and B [K][ldb] bf16 row-major: A fragments by ldmatrix, B
-// fragments by ldmatrix.trans (k x n blocks read as their transposes).
+// acc[MT][NT] (rows m0.., columns n0..) += A[m0.., 0:K] B[0:K, n0..], bf16
+// operands in shared memory.  A is [M][lda] (AT: stored transposed, [K][lda]),
+// B is [K][ldb] (BT: stored transposed, [N][ldb]).  Fragments come from
+// ldmatrix, with .trans where the stored rows run along the other index.
 // Row starts 16-byte aligned; row strides = 16 (mod 128) bytes avoid conflicts.
-template <int MT, int NT, int K>
+template <int MT, int NT, int K, bool AT = false, bool BT = false>
 __device__ __forceinline__ void warp_mma_bf16(float (&acc)[MT][NT][4], const bf16* A, int lda, const bf16* B, int ldb,
                                               int m0, int n0) {
   const int lane = threadIdx.x & 31, mat = lane >> 3, rr = lane & 7;
-  const bf16* pa = A + (m0 + rr + 8 * (mat & 1)) * lda + 8 * (mat >> 1);
-  const bf16* pb = B + (rr + 8 * (mat & 1)) * ldb + n0 + 8 * (mat >> 1);
-  const bf16* pb1 = B + (rr + 8 * (mat & 1)) * ldb + n0 + 8 * (NT - 1);  // odd NT: last tile (lanes 0-15)
+  // matrices of an A x4: (m 0-7, k 0-7), (m 8-15, k 0-7), (m 0-7, k 8-15), (m 8-15, k 8-15)
+  const bf16* pa = AT ? A + (rr + 8 * (mat >> 1)) * lda + m0 + 8 * (mat & 1)
+                      : A + (m0 + rr + 8 * (mat & 1)) * lda + 8 * (mat >> 1);
+  // matrices of a B x4: (k 0-7, n 0-7), (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15)
+  const bf16* pb = BT ? B + (n0 + rr + 8 * (mat >> 1)) * ldb + 8 * (mat & 1)
+                      : B + (rr + 8 * (mat & 1)) * ldb + n0 + 8 * (mat >> 1);
+  // odd NT: the last B tile by an x2 (lanes 0-15)
+  const bf16* pb1 = BT ? B + (n0 + 8 * (NT - 1) + rr) * ldb + 8 * (mat & 1)
+                       : B + (rr + 8 * (mat & 1)) * ldb + n0 + 8 * (NT - 1);
 #pragma unroll
   for (int k0 = 0; k0 < K; k0 += 16) {
     uint32_t af[MT][4], bfr[NT][2];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) ldsm_x4_b(af[mt], pa + 16 * mt * lda + k0);
+    for (int mt = 0; mt < MT; ++mt) {
+      if constexpr (AT)
+        ldsm_x4_t(af[mt], pa + k0 * lda + 16 * mt);
+      else
+        ldsm_x4_b(af[mt], pa + 16 * mt * lda + k0);
+    }
 #pragma unroll
     for (int np = 0; np < NT / 2; ++np) {
       uint32_t r[4];
-      ldsm_x4_t(r, pb + k0 * ldb + 16 * np);
+      if constexpr (BT)
+        ldsm_x4_b(r, pb + 16 * np * ldb + k0);
+      else
+        ldsm_x4_t(r, pb + k0 * ldb + 16 * np);
       bfr[2 * np][0] = r[0], bfr[2 * np][1] = r[1], bfr[2 * np + 1][0] = r[2], bfr[2 * np + 1][1] = r[3];
     }
     if constexpr (NT % 2 == 1) {
       uint32_t r[2];
-      ldsm_x2_t(r, pb1 + k0 * ldb);
+      if constexpr (BT)
+        ldsm_x2_b(r, pb1 + k0);
+      else
+        ldsm_x2_t(r, pb1 + k0 * ldb);
       bfr[NT - 1][0] = r[0], bfr[NT - 1][1] = r[1];
     }
 #pragma unroll
@@ -952,7 +975,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
       const size_t rec = (size_t)lb * NC + n;
       const int p = n & 1;
       acc_to_bf16(st, simg, LS, sm0, sn0);
-      acc_to_global(st, a.S0c + rec * DK * DV + c0, DV, sm0, sn0);
+      acc_to_bf16(st, reinterpret_cast<bf16*>(a.S0c) + rec * DK * DV + c0, DV, sm0, sn0);
       cp_wait_group<0>();
       __syncthreads();
       if (n + 1 < NC) issue(n + 1, p ^ 1);
@@ -964,7 +987,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
         for_acc<TV::MT, TV::NT>(vm0, vn0,
                                 [&](int mt, int nt, int e, int i, int c) { acc[mt][nt][e] = u[i * SW + c] - acc[mt][nt][e]; });
         acc_to_bf16(acc, vimg, LS, vm0, vn0);
-        acc_to_global(acc, a.Vp + rec * kC * DV + c0, DV, vm0, vn0);
+        acc_to_bf16(acc, reinterpret_cast<bf16*>(a.Vp) + rec * kC * DV + c0, DV, vm0, vn0);
       }
       __syncthreads();
       {  // S = diag(gamma) S + Kbar^T V'
@@ -999,7 +1022,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
       const size_t rec = (size_t)lb * NC + n;
       const int p = n & 1;
       acc_to_bf16(st, simg, LS, sm0, sn0);
-      acc_to_global(st, a.dSc + rec * DK * DV + c0, DV, sm0, sn0);
+      acc_to_bf16(st, reinterpret_cast<bf16*>(a.dSc) + rec * DK * DV + c0, DV, sm0, sn0);
       cp_wait_group<0>();
       __syncthreads();
       if (n > 0) issue(n - 1, p ^ 1);
@@ -1010,7 +1033,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
         warp_mma_bf16<TV::MT, TV::NT, kC>(acc, rp + R::oAqkt, R::LCb, bO(p), LS, vm0, vn0);
         warp_mma_bf16<TV::MT, TV::NT, DK>(acc, rp + R::oKb, R::LKb, simg, LS, vm0, vn0);
         acc_to_bf16(acc, vimg, LS, vm0, vn0);
-        acc_to_global(acc, a.dVp + rec * kC * DV + c0, DV, vm0, vn0);
+        acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dVp) + rec * kC * DV + c0, DV, vm0, vn0);
       }
       __syncthreads();
       {  // dS = diag(gamma) dS + Q+^T dO - W^T dV'
@@ -1137,6 +1160,134 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
   }
 }
 
+
+// ------------------------------------------------------------------ kernel 3 (bf16 operands)
+template <int DK, int DV>
+struct LocalAPlanB {  // bytes
+  static constexpr int LVb = DV + 8, LCb = kC + 8;
+  static constexpr size_t oO = 0, oVp = oO + (size_t)kC * LVb * 2, odV = oVp + (size_t)kC * LVb * 2,
+                          ov = odV + (size_t)kC * LVb * 2, oT = ov + (size_t)kC * LVb * 2,
+                          oS0 = oT + (size_t)kC * LCb * 2, odS = oS0 + (size_t)DK * LVb * 2,
+                          ob = odS + (size_t)DK * LVb * 2, ored = ob + kC * 4, bytes = ored + 4 * kC * 4;
+};
+
+// Per chunk, bf16 inputs: the products that contract over the value channels,
+// all operands bf16 images in shared memory (S0, dS, V', dV' and T come from
+// the state passes and the prep kernel as bf16).
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const ChunkBwdArgs a) {
+  using PL = LocalAPlanB<DK, DV>;
+  constexpr int LVb = PL::LVb, LCb = PL::LCb;
+  extern __shared__ __align__(16) uint8_t smb[];
+  bf16* sO = reinterpret_cast<bf16*>(smb + PL::oO);    // [64][LVb] dO
+  bf16* sVp = reinterpret_cast<bf16*>(smb + PL::oVp);  // [64][LVb] V'
+  bf16* sdV = reinterpret_cast<bf16*>(smb + PL::odV);  // [64][LVb] dV'
+  bf16* sv = reinterpret_cast<bf16*>(smb + PL::ov);    // [64][LVb] v
+  bf16* sT = reinterpret_cast<bf16*>(smb + PL::oT);    // [64][LCb] T
+  bf16* sS0 = reinterpret_cast<bf16*>(smb + PL::oS0);  // [DK][LVb] S0
+  bf16* sdS = reinterpret_cast<bf16*>(smb + PL::odS);  // [DK][LVb] dS
+  float* sb = reinterpret_cast<float*>(smb + PL::ob);  // [64] beta
+  float* red = reinterpret_cast<float*>(smb + PL::ored);  // [4][64] row sums per column group
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
+  auto cp16 = [&](void* dst, const void* src, int bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(bytes)
+                 : "memory");
+  };
+  // rows of 16-byte pieces: [rows][width] bf16 from global (row i at src_row(i)) into [rows][ld]
+  auto rows_in = [&](bf16* dst, int ld, int rows, int width, auto src_row, int valid) {
+    const int per = width / 8;
+    for (int idx = tid; idx < rows * per; idx += kThreads) {
+      const int i = idx / per, c = (idx % per) * 8;
+      cp16(dst + i * ld + c, i < valid ? src_row(i) + c : src_row(0), i < valid ? 16 : 0);
+    }
+  };
+  const bf16* d_o = static_cast<const bf16*>(a.d_o);
+  const bf16* vin = static_cast<const bf16*>(a.v);
+  const bf16* Vp = reinterpret_cast<const bf16*>(a.Vp) + rec * kC * DV;
+  const bf16* dVp = reinterpret_cast<const bf16*>(a.dVp) + rec * kC * DV;
+  const bf16* S0 = reinterpret_cast<const bf16*>(a.S0c) + rec * DK * DV;
+  const bf16* dS = reinterpret_cast<const bf16*>(a.dSc) + rec * DK * DV;
+  rows_in(sO, LVb, kC, DV, [&](int i) { return d_o + (row0 + (size_t)i * a.H) * DV; }, nv);
+  rows_in(sv, LVb, kC, DV, [&](int i) { return vin + (row0 + (size_t)i * a.H) * DV; }, nv);
+  rows_in(sVp, LVb, kC, DV, [&](int i) { return Vp + (size_t)i * DV; }, kC);
+  rows_in(sdV, LVb, kC, DV, [&](int i) { return dVp + (size_t)i * DV; }, kC);
+  rows_in(sS0, LVb, DK, DV, [&](int i) { return S0 + (size_t)i * DV; }, DK);
+  rows_in(sdS, LVb, DK, DV, [&](int i) { return dS + (size_t)i * DV; }, DK);
+  if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const bf16*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
+  for (int idx = tid; idx < kC * kC / 4; idx += kThreads) {  // T (fp32) as a bf16 image
+    const int i = idx / (kC / 4), j = (idx % (kC / 4)) * 4;
+    const float4 x = *reinterpret_cast<const float4*>(a.Tm + rec * kC * kC + i * kC + j);
+    *reinterpret_cast<__nv_bfloat162*>(sT + i * LCb + j) = __floats2bfloat162_rn(x.x, x.y);
+    *reinterpret_cast<__nv_bfloat162*>(sT + i * LCb + j + 2) = __floats2bfloat162_rn(x.z, x.w);
+  }
+  cp_wait();
+  __syncthreads();
+  {
+    using Tl = Tiling<kC, kC>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);  // dAqk = tril(dO V'^T)
+    warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sO, LVb, sVp, LVb, m0, n0);
+    float* out = a.dAqk + rec * kC * kC;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
+      out[i * kC + j] = j <= i ? acc[mt][nt][e] : 0.f;
+    });
+    zero(acc);  // dU (beta V)^T, strictly lower part
+    warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sdV, LVb, sv, LVb, m0, n0);
+    out = a.dT1 + rec * kC * kC;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
+      out[i * kC + j] = j < i ? acc[mt][nt][e] * sb[j] : 0.f;
+    });
+  }
+  {  // X = T^T dU: dv = beta X, dbeta part = rowsum(V . X)
+    using Tl = Tiling<kC, DV>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4], rp[Tl::MT][2] = {};
+    zero(acc);
+    warp_mma_bf16<Tl::MT, Tl::NT, kC, true, false>(acc, sT, LCb, sdV, LVb, m0, n0);
+    bf16* dv = static_cast<bf16*>(a.dv);
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
+      const float x = acc[mt][nt][e];
+      if (i < nv) dv[(row0 + (size_t)i * a.H) * DV + c] = __float2bfloat16_rn(sb[i] * x);
+      rp[mt][e >> 1] = fmaf(x, __bfloat162float(sv[i * LVb + c]), rp[mt][e >> 1]);
+    });
+    row_sums_out<Tl::MT>(rp, m0, red + (warp / Tl::WM) * kC);
+  }
+  {  // dO S0^T, -dV' S0^T, V' dS^T (64 x DK, contracting the value channels)
+    using Tl = Tiling<kC, DK>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);
+    warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sO, LVb, sS0, LVb, m0, n0);
+    float* out = a.dQs + rec * kC * DK;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
+    zero(acc);
+    warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sdV, LVb, sS0, LVb, m0, n0);
+    out = a.dW + rec * kC * DK;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = -acc[mt][nt][e]; });
+    zero(acc);
+    warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sVp, LVb, sdS, LVb, m0, n0);
+    out = a.dKb + rec * kC * DK;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
+  }
+  for (int r = warp; r < DK; r += kWarps) {  // rowsum(dS . S0)
+    float x = 0.f;
+    for (int c = lane; c < DV; c += 32) x = fmaf(__bfloat162float(sdS[r * LVb + c]), __bfloat162float(sS0[r * LVb + c]), x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if (lane == 0) a.dgam[rec * DK + r] = x;
+  }
+  __syncthreads();
+  if (tid < kC) {
+    float x = 0.f;
+#pragma unroll
+    for (int w = 0; w < Tiling<kC, DV>::WN; ++w) x += red[w * kC + tid];
+    a.dbu[rec * kC + tid] = x;
+  }
+}
 
 // ------------------------------------------------------------------ kernel 4
 template <int DK, int DV>
@@ -1388,8 +1539,9 @@ struct WsPlan {
       : W(f32 ? (size_t)kC * dk : 0), U((size_t)kC * dv), Qp((size_t)kC * dk), Kb((size_t)kC * dk),
         Wt(f32 ? (size_t)kC * dk : 0), Qpt(f32 ? (size_t)kC * dk : 0), Kbt(f32 ? (size_t)kC * dk : 0),
         Aqk(f32 ? kC * kC : 0), prec(f32 ? 0 : (dk == 128 ? PassRec<128>::n : PassRec<64>::n) / 2),
-        Tm(kC * kC), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv), dSc((size_t)dk * dv), Vp((size_t)kC * dv),
-        dVp((size_t)kC * dv), dAqk(kC * kC), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk),
+        // bf16 inputs: S0, dS, V', dV' are kept as bf16 (half the floats)
+        Tm(kC * kC), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv / (f32 ? 1 : 2)), dSc((size_t)dk * dv / (f32 ? 1 : 2)),
+        Vp((size_t)kC * dv / (f32 ? 1 : 2)), dVp((size_t)kC * dv / (f32 ? 1 : 2)), dAqk(kC * kC), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk),
         dKb((size_t)kC * dk), dgam(dk), dbu(kC) {}
   size_t per_rec() const {
     return W + U + Qp + Kb + Wt + Qpt + Kbt + Aqk + prec + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs +
@@ -1432,7 +1584,10 @@ cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t strea
                    stream, kPassThreads);
   }
   if (e != cudaSuccess) return e;
-  e = launch_k(bwd_local_a_kernel<IO, DK, DV>, grid, local_a_smem<DK, DV>(), a, stream);
+  if constexpr (std::is_same<IO, float>::value)
+    e = launch_k(bwd_local_a_kernel<IO, DK, DV>, grid, local_a_smem<DK, DV>(), a, stream);
+  else
+    e = launch_k(bwd_local_a_bf16_kernel<DK, DV>, grid, LocalAPlanB<DK, DV>::bytes, a, stream);
   if (e != cudaSuccess) return e;
   return launch_k(bwd_local_b_kernel<IO, DK, DV>, grid, local_b_smem<DK, DV>(), a, stream);
 }
