@@ -1530,6 +1530,275 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
 }
 
 
+// ------------------------------------------------------------------ kernel 4 (bf16 operands)
+template <int DK, int DV>
+struct LocalBPlanB {  // bytes
+  static constexpr int LK = DK + 4, LKb = DK + 8, LCb = kC + 8;
+  static constexpr size_t tk = (size_t)kC * LKb * 2, tc = (size_t)kC * LCb * 2;
+  static constexpr size_t oG = 0, ok = oG + (size_t)kC * LK * 4, oq = ok + tk, oA = oq + tk, oB = oA + tk,
+                          oC = oB + tk, oT = oC + tk, oDT = oT + tc, oY = oDT + tc, oQA = oY + tc, ob = oQA + tc,
+                          ored = ob + kC * 4, ocol = ored + 8 * kC * 4, bytes = ocol + 4 * DK * 4;
+  static_assert(tk % 16 == 0 && tc % 16 == 0 && ok % 16 == 0, "16 B");
+  static_assert(2 * tk >= (size_t)kC * LK * 4, "dG (fp32) fits over the k and q tiles");
+};
+
+// Per chunk, bf16 inputs: dT, T^T dW, dA, the pairwise gradients and the fold
+// into dq, dk, dg, dbeta.  Operands are bf16 images; G, the decay factors and
+// the fold run in fp32 (from the exact k, q inputs).
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const ChunkBwdArgs a) {
+  using PL = LocalBPlanB<DK, DV>;
+  constexpr int LK = PL::LK, LKb = PL::LKb, LCb = PL::LCb;
+  using TK = Tiling<kC, DK>;  // every 64 x d_k product: the same tile per warp
+  using TC = Tiling<kC, kC>;
+  extern __shared__ __align__(16) uint8_t smb[];
+  float* sG = reinterpret_cast<float*>(smb + PL::oG);   // [64][LK] cumulative log-gates
+  bf16* sk = reinterpret_cast<bf16*>(smb + PL::ok);     // [64][LKb] k (input)
+  bf16* sq = reinterpret_cast<bf16*>(smb + PL::oq);     // [64][LKb] q (input)
+  bf16* sA = reinterpret_cast<bf16*>(smb + PL::oA);     // [64][LKb] dW, then K-_r
+  bf16* sB = reinterpret_cast<bf16*>(smb + PL::oB);     // [64][LKb] K+, then K+_r
+  bf16* sC = reinterpret_cast<bf16*>(smb + PL::oC);     // [64][LKb] Q+_r
+  bf16* sT = reinterpret_cast<bf16*>(smb + PL::oT);     // [64][LCb] T
+  bf16* sDT = reinterpret_cast<bf16*>(smb + PL::oDT);   // [64][LCb] dT, then M = diag(beta) dA
+  bf16* sY = reinterpret_cast<bf16*>(smb + PL::oY);     // [64][LCb] dT T^T
+  bf16* sQA = reinterpret_cast<bf16*>(smb + PL::oQA);   // [64][LCb] dAqk
+  float* sb = reinterpret_cast<float*>(smb + PL::ob);   // [64] beta
+  float* red = reinterpret_cast<float*>(smb + PL::ored);  // [8][64] row sums per column group
+  float* colC = reinterpret_cast<float*>(smb + PL::ocol);  // [4][DK] column sums of dKbar . Kbar
+  float* sdG = reinterpret_cast<float*>(smb + PL::ok);  // [64][LK] dG (fp32), over the k and q tiles at the end
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
+  const bf16* q = static_cast<const bf16*>(a.q);
+  const bf16* k = static_cast<const bf16*>(a.k);
+  const int m0 = TK::m0(warp), n0 = TK::n0(warp), cm0 = TC::m0(warp), cn0 = TC::n0(warp);
+  float dk_acc[TK::MT][TK::NT][4], dG_acc[TK::MT][TK::NT][4];
+  zero(dk_acc);
+  zero(dG_acc);
+  auto cp16 = [&](void* dst, const void* src, int bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(bytes)
+                 : "memory");
+  };
+  auto rows_in = [&](bf16* dst, const bf16* src) {  // 64 input rows of DK (zeros past the tail)
+    constexpr int per = DK / 8;
+    for (int idx = tid; idx < kC * per; idx += kThreads) {
+      const int i = idx / per, c = (idx % per) * 8;
+      cp16(dst + i * LKb + c, i < nv ? src + (row0 + (size_t)i * a.H) * DK + c : src, i < nv ? 16 : 0);
+    }
+  };
+  auto f32_to_img = [&](bf16* dst, int ld, const float* src, int rows, int cols) {  // fp32 [rows][cols] -> bf16 image
+    for (int idx = tid; idx < rows * cols / 4; idx += kThreads) {
+      const int i = idx / (cols / 4), j = (idx % (cols / 4)) * 4;
+      const float4 x = *reinterpret_cast<const float4*>(src + (size_t)i * cols + j);
+      *reinterpret_cast<__nv_bfloat162*>(dst + i * ld + j) = __floats2bfloat162_rn(x.x, x.y);
+      *reinterpret_cast<__nv_bfloat162*>(dst + i * ld + j + 2) = __floats2bfloat162_rn(x.z, x.w);
+    }
+  };
+
+  if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const bf16*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
+  rows_in(sk, k);
+  rows_in(sq, q);
+  load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
+  const bool slow = chunk_unsafe<DK>(sG, LK);
+  f32_to_img(sA, LKb, a.dW + rec * kC * DK, kC, DK);
+  f32_to_img(sT, LCb, a.Tm + rec * kC * kC, kC, kC);
+  f32_to_img(sQA, LCb, a.dAqk + rec * kC * kC, kC, kC);
+  cp_wait();
+  __syncthreads();
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // K+ = k exp(G)
+    const int i = idx / DK, r = idx % DK;
+    sB[i * LKb + r] = __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * expf(sG[i * LK + r]));
+  }
+  __syncthreads();
+  {  // dT = dU (beta V)^T + dW (beta K+)^T, strictly lower, as a bf16 image
+    float acc[TC::MT][TC::NT][4];
+    zero(acc);
+    warp_mma_bf16<TC::MT, TC::NT, DK, false, true>(acc, sA, LKb, sB, LKb, cm0, cn0);
+    const float* dT1 = a.dT1 + rec * kC * kC;
+    for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
+      acc[mt][nt][e] = j < i ? fmaf(acc[mt][nt][e], sb[j], dT1[i * kC + j]) : 0.f;
+    });
+    acc_to_bf16(acc, sDT, LCb, cm0, cn0);
+  }
+  {  // X = T^T dW: dK+ = beta X; dbeta part rowsum(K+ . X)
+    float acc[TK::MT][TK::NT][4], rp[TK::MT][2] = {};
+    zero(acc);
+    warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(acc, sT, LCb, sA, LKb, m0, n0);
+    for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+      const float x = acc[mt][nt][e], gm = expf(sG[i * LK + r]);
+      const float kp = __bfloat162float(sk[i * LKb + r]) * gm, bx = sb[i] * x;
+      dk_acc[mt][nt][e] = fmaf(bx, gm, dk_acc[mt][nt][e]);
+      dG_acc[mt][nt][e] = fmaf(bx, kp, dG_acc[mt][nt][e]);
+      rp[mt][e >> 1] = fmaf(x, kp, rp[mt][e >> 1]);
+    });
+    row_sums_out<TK::MT>(rp, m0, red + (warp / TK::WM) * kC);
+  }
+  __syncthreads();
+  {  // dT T^T
+    float acc[TC::MT][TC::NT][4];
+    zero(acc);
+    warp_mma_bf16<TC::MT, TC::NT, kC, false, true>(acc, sDT, LCb, sT, LCb, cm0, cn0);
+    acc_to_bf16(acc, sY, LCb, cm0, cn0);
+  }
+  __syncthreads();
+  {  // dA = -T^T (dT T^T), strictly lower; dbeta part rowsum(dA . P); M = diag(beta) dA
+    float acc[TC::MT][TC::NT][4], rp[TC::MT][2] = {};
+    zero(acc);
+    warp_mma_bf16<TC::MT, TC::NT, kC, true, false>(acc, sT, LCb, sY, LCb, cm0, cn0);
+    const float* P = a.Pkk + rec * kC * kC;
+    for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
+      const float d = j < i ? -acc[mt][nt][e] : 0.f;
+      rp[mt][e >> 1] = fmaf(d, P[i * kC + j], rp[mt][e >> 1]);
+      acc[mt][nt][e] = sb[i] * d;
+    });
+    acc_to_bf16(acc, sDT, LCb, cm0, cn0);
+    row_sums_out<TC::MT>(rp, cm0, red + (4 + warp / TC::WM) * kC);
+  }
+  if (!slow) {  // factored operands K+_r, K-_r, Q+_r
+    for (int idx = tid; idx < kC * DK; idx += kThreads) {
+      const int i = idx / DK, r = idx % DK;
+      const float d = sG[i * LK + r] - sG[kRef * LK + r], ex = expf(d);
+      const float kk = __bfloat162float(sk[i * LKb + r]), qq = a.scale * __bfloat162float(sq[i * LKb + r]);
+      sB[i * LKb + r] = __float2bfloat16_rn(kk * ex);
+      sA[i * LKb + r] = __float2bfloat16_rn(kk * expf(-d));
+      sC[i * LKb + r] = __float2bfloat16_rn(qq * ex);
+    }
+  }
+  __syncthreads();
+  const float* dQs = a.dQs + rec * kC * DK;
+  const float* Qp = a.Qp + rec * kC * DK;
+  bf16* dq = static_cast<bf16*>(a.dq);
+  if (!slow) {
+    {  // dQ+_r = dAqk K-_r;  dq = scale (exp(G - G_ref) dQ+_r + Gamma dO S0^T)
+      float acc[TK::MT][TK::NT][4];
+      zero(acc);
+      warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(acc, sQA, LCb, sA, LKb, m0, n0);
+      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+        const float x = acc[mt][nt][e], G = sG[i * LK + r];
+        const float ex = expf(G - sG[kRef * LK + r]), dqs = dQs[i * DK + r];
+        const float qr = a.scale * __bfloat162float(sq[i * LKb + r]) * ex;  // Q+_r
+        if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(a.scale * fmaf(ex, x, expf(G) * dqs));
+        dG_acc[mt][nt][e] += fmaf(x, qr, dqs * Qp[i * DK + r]);
+      });
+    }
+    {  // dK-_r = dAqk^T Q+_r + M^T K+_r
+      float acc[TK::MT][TK::NT][4];
+      zero(acc);
+      warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(acc, sQA, LCb, sC, LKb, m0, n0);
+      warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(acc, sDT, LCb, sB, LKb, m0, n0);
+      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+        const float x = acc[mt][nt][e], ei = expf(sG[kRef * LK + r] - sG[i * LK + r]);
+        dk_acc[mt][nt][e] = fmaf(ei, x, dk_acc[mt][nt][e]);
+        dG_acc[mt][nt][e] = fmaf(-x, __bfloat162float(sk[i * LKb + r]) * ei, dG_acc[mt][nt][e]);
+      });
+    }
+    {  // dK+_r = M K-_r
+      float acc[TK::MT][TK::NT][4];
+      zero(acc);
+      warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(acc, sDT, LCb, sA, LKb, m0, n0);
+      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+        const float x = acc[mt][nt][e], ex = expf(sG[i * LK + r] - sG[kRef * LK + r]);
+        dk_acc[mt][nt][e] = fmaf(ex, x, dk_acc[mt][nt][e]);
+        dG_acc[mt][nt][e] = fmaf(x, __bfloat162float(sk[i * LKb + r]) * ex, dG_acc[mt][nt][e]);
+      });
+    }
+  } else {
+    // exact pairwise terms, E = exp(G_ir - G_jr) for j <= i (see the fp32 kernel)
+    auto K_ = [&](int i, int r) { return __bfloat162float(sk[i * LKb + r]); };
+    auto Q_ = [&](int i, int r) { return a.scale * __bfloat162float(sq[i * LKb + r]); };
+    auto QA = [&](int i, int j) { return __bfloat162float(sQA[i * LCb + j]); };
+    auto MM = [&](int i, int j) { return __bfloat162float(sDT[i * LCb + j]); };
+    for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+      const float Gi = sG[i * LK + r], ki = K_(i, r), qi = Q_(i, r);
+      float dqp = 0.f, dkp = 0.f, dgp = 0.f;
+      for (int j = 0; j <= i; ++j) {
+        const float kE = expf(Gi - sG[j * LK + r]) * K_(j, r);
+        const float c = QA(i, j), m = MM(i, j);
+        dqp = fmaf(c, kE, dqp);
+        dkp = fmaf(m, kE, dkp);
+        dgp = fmaf(fmaf(c, qi, m * ki), kE, dgp);
+      }
+      for (int j = i; j < kC; ++j) {
+        const float w = fmaf(QA(j, i), Q_(j, r), MM(j, i) * K_(j, r)) * expf(sG[j * LK + r] - Gi);
+        dkp += w;
+        dgp = fmaf(-w, ki, dgp);
+      }
+      const float dqs = dQs[i * DK + r];
+      if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(a.scale * fmaf(expf(Gi), dqs, dqp));
+      dk_acc[mt][nt][e] += dkp;
+      dG_acc[mt][nt][e] += fmaf(dqs, Qp[i * DK + r], dgp);
+    });
+  }
+  {  // Kbar: dk += exp(G_C - G) dKbar, dG -= dKbar . Kbar, dG_C += column sums of the same
+    const float* dKb = a.dKb + rec * kC * DK;
+    const float* Kb = a.Kb + rec * kC * DK;
+    float cp[TK::MT][TK::NT][2] = {};
+    for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+      const float x = dKb[i * DK + r], y = x * Kb[i * DK + r];
+      dk_acc[mt][nt][e] = fmaf(expf(sG[(kC - 1) * LK + r] - sG[i * LK + r]), x, dk_acc[mt][nt][e]);
+      dG_acc[mt][nt][e] -= y;
+      cp[mt][nt][e & 1] += y;
+    });
+#pragma unroll
+    for (int nt = 0; nt < TK::NT; ++nt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float x = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < TK::MT; ++mt) x += cp[mt][nt][c];
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        x += __shfl_xor_sync(0xffffffffu, x, 8);
+        x += __shfl_xor_sync(0xffffffffu, x, 16);
+        if (lane < 4) colC[(warp % TK::WM) * DK + n0 + 8 * nt + 2 * lane + c] = x;
+      }
+  }
+  bf16* dk = static_cast<bf16*>(a.dk);
+  for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+    if (i < nv) dk[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(dk_acc[mt][nt][e]);
+  });
+  __syncthreads();  // the k and q tiles are no longer read: they take dG
+  for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) { sdG[i * LK + r] = dG_acc[mt][nt][e]; });
+  __syncthreads();
+  if (tid < DK) {  // dG_C terms, then dg = reverse cumsum of dG over the chunk
+    const int r = tid;
+    float x = 0.f;
+#pragma unroll
+    for (int w = 0; w < TK::WM; ++w) x += colC[w * DK + r];
+    x = fmaf(expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
+    float acc = x;
+    for (int i = kC - 1; i >= 0; --i) {
+      acc += sdG[i * LK + r];
+      sdG[i * LK + r] = acc;
+    }
+  }
+  __syncthreads();
+  if (a.gate == KDA_GATE_CHANNEL) {
+    bf16* dg = static_cast<bf16*>(a.dg);
+    for (int idx = tid; idx < nv * DK; idx += kThreads) {
+      const int i = idx / DK, r = idx % DK;
+      dg[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(sdG[i * LK + r]);
+    }
+  } else if (a.gate == KDA_GATE_HEAD) {
+    bf16* dg = static_cast<bf16*>(a.dg);
+    for (int i = warp; i < nv; i += kWarps) {
+      float x = 0.f;
+      for (int r = lane; r < DK; r += 32) x += sdG[i * LK + r];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+      if (lane == 0) dg[row0 + (size_t)i * a.H] = __float2bfloat16_rn(x);
+    }
+  }
+  if (tid < nv) {
+    float x = a.dbu[rec * kC + tid], y = 0.f;
+#pragma unroll
+    for (int w = 0; w < TK::WN; ++w) x += red[w * kC + tid];
+#pragma unroll
+    for (int w = 0; w < TC::WN; ++w) y += red[(4 + w) * kC + tid];
+    static_cast<bf16*>(a.dbeta)[row0 + (size_t)tid * a.H] = __float2bfloat16_rn(x + y);
+  }
+}
+
 // ------------------------------------------------------------------ host
 // Floats of each workspace array per chunk record, in layout order.
 struct WsPlan {
@@ -1589,7 +1858,10 @@ cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t strea
   else
     e = launch_k(bwd_local_a_bf16_kernel<DK, DV>, grid, LocalAPlanB<DK, DV>::bytes, a, stream);
   if (e != cudaSuccess) return e;
-  return launch_k(bwd_local_b_kernel<IO, DK, DV>, grid, local_b_smem<DK, DV>(), a, stream);
+  if constexpr (std::is_same<IO, float>::value)
+    return launch_k(bwd_local_b_kernel<IO, DK, DV>, grid, local_b_smem<DK, DV>(), a, stream);
+  else
+    return launch_k(bwd_local_b_bf16_kernel<DK, DV>, grid, LocalBPlanB<DK, DV>::bytes, a, stream);
 }
 
 template <typename IO>
