@@ -1161,6 +1161,180 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwd
 }
 
 
+// ------------------------------------------------------------------ kernel 1 (bf16 operands)
+template <int DK, int DV>
+struct PrepPlanB {  // bytes
+  static constexpr int LK = DK + 4, LKb = DK + 8, LVb = DV + 8, LMb = (DK > DV ? DK : DV) + 8, LCb = kC + 8;
+  static constexpr size_t oG = 0, ok = oG + (size_t)kC * LK * 4, oq = ok + (size_t)kC * LKb * 2,
+                          ov = oq + (size_t)kC * LKb * 2, oX = ov + (size_t)kC * LVb * 2,
+                          oY = oX + (size_t)kC * LKb * 2, oQ = oY + (size_t)kC * LMb * 2,
+                          oP = oQ + (size_t)kC * LKb * 2, oT = oP + (size_t)kC * kLC * 4,
+                          ob = oT + (size_t)kC * LCb * 2, oe = ob + kC * 4, bytes = oe + DK * 4;
+  static_assert(ok % 16 == 0 && oq % 16 == 0 && ov % 16 == 0 && oX % 16 == 0 && oY % 16 == 0 && oQ % 16 == 0 &&
+                    oP % 16 == 0 && oT % 16 == 0 && ob % 16 == 0,
+                "16 B");
+};
+
+// Per chunk, bf16 inputs: G (fp32), the factored operands as bf16 images, P
+// (fp32, for the solve) and Aqk, T by forward substitution in fp32, W and U;
+// the state passes' operands go out as the chunk's bf16 pass record, T as bf16.
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkBwdArgs a) {
+  using PL = PrepPlanB<DK, DV>;
+  using PR = PassRec<DK>;
+  constexpr int LK = PL::LK, LKb = PL::LKb, LVb = PL::LVb, LMb = PL::LMb, LCb = PL::LCb;
+  extern __shared__ __align__(16) uint8_t smb[];
+  float* sG = reinterpret_cast<float*>(smb + PL::oG);  // [64][LK] cumulative log-gates
+  bf16* sk = reinterpret_cast<bf16*>(smb + PL::ok);    // [64][LKb] k (input)
+  bf16* sq = reinterpret_cast<bf16*>(smb + PL::oq);    // [64][LKb] q (input)
+  bf16* sv = reinterpret_cast<bf16*>(smb + PL::ov);    // [64][LVb] v (input)
+  bf16* sX = reinterpret_cast<bf16*>(smb + PL::oX);    // [64][LKb] K+_r, then beta K+
+  bf16* sY = reinterpret_cast<bf16*>(smb + PL::oY);    // [64][LMb] K-_r, then beta v
+  bf16* sQ = reinterpret_cast<bf16*>(smb + PL::oQ);    // [64][LKb] Q+_r
+  float* sP = reinterpret_cast<float*>(smb + PL::oP);  // [64][kLC] P
+  bf16* sT = reinterpret_cast<bf16*>(smb + PL::oT);    // [64][LCb] T
+  float* sb = reinterpret_cast<float*>(smb + PL::ob);  // [64] beta
+  float* se = reinterpret_cast<float*>(smb + PL::oe);  // [DK] exp(G_ref)
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
+  const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
+  bf16* pr = a.prec + rec * PR::n;
+  auto cp16 = [&](void* dst, const void* src, int bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src), "r"(bytes)
+                 : "memory");
+  };
+  auto rows_in = [&](bf16* dst, int ld, const bf16* src, int D) {  // 64 input rows of D (zeros past the tail)
+    const int per = D / 8;
+    for (int idx = tid; idx < kC * per; idx += kThreads) {
+      const int i = idx / per, c = (idx % per) * 8;
+      cp16(dst + i * ld + c, i < nv ? src + (row0 + (size_t)i * a.H) * D + c : src, i < nv ? 16 : 0);
+    }
+  };
+  rows_in(sk, LKb, static_cast<const bf16*>(a.k), DK);
+  rows_in(sq, LKb, static_cast<const bf16*>(a.q), DK);
+  rows_in(sv, LVb, static_cast<const bf16*>(a.v), DV);
+  if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const bf16*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
+  load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
+  const bool slow = chunk_unsafe<DK>(sG, LK);
+  if (tid < DK) {
+    se[tid] = expf(sG[kRef * LK + tid]);
+    a.gam[rec * DK + tid] = expf(sG[(kC - 1) * LK + tid]);
+  }
+  cp_wait();
+  __syncthreads();
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+^T, Kbar^T (record), token index fastest
+    const int r = idx / kC, i = idx % kC;
+    const float G = sG[i * LK + r];
+    pr[PR::oQpt + r * PR::LCb + i] = __float2bfloat16_rn(a.scale * __bfloat162float(sq[i * LKb + r]) * expf(G));
+    pr[PR::oKbt + r * PR::LCb + i] =
+        __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * expf(sG[(kC - 1) * LK + r] - G));
+  }
+  float* Qp = a.Qp + rec * kC * DK;
+  float* Kb = a.Kb + rec * kC * DK;
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+, Kbar (fp32, record) and the factored operands
+    const int i = idx / DK, r = idx % DK;
+    const float G = sG[i * LK + r], kk = __bfloat162float(sk[i * LKb + r]);
+    const float qq = a.scale * __bfloat162float(sq[i * LKb + r]);
+    const float kb = kk * expf(sG[(kC - 1) * LK + r] - G);
+    Qp[i * DK + r] = qq * expf(G);
+    Kb[i * DK + r] = kb;
+    pr[PR::oKb + i * PR::LKb + r] = __float2bfloat16_rn(kb);
+    if (!slow) {
+      const float d = G - sG[kRef * LK + r], ex = expf(d);
+      sX[i * LKb + r] = __float2bfloat16_rn(kk * ex);
+      sY[i * LMb + r] = __float2bfloat16_rn(kk * expf(-d));
+      sQ[i * LKb + r] = __float2bfloat16_rn(qq * ex);
+    }
+  }
+  __syncthreads();
+
+  // P = strict_tril(K+ K-^T) (fp32, shared), Aqk = tril(Q+ K-^T) (record, transposed)
+  if (!slow) {
+    using Tl = Tiling<kC, kC>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);
+    warp_mma_bf16<Tl::MT, Tl::NT, DK, false, true>(acc, sX, LKb, sY, LMb, m0, n0);
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
+      sP[i * kLC + j] = j < i ? acc[mt][nt][e] : 0.f;
+    });
+    zero(acc);
+    warp_mma_bf16<Tl::MT, Tl::NT, DK, false, true>(acc, sQ, LKb, sY, LMb, m0, n0);
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
+      pr[PR::oAqkt + j * PR::LCb + i] = __float2bfloat16_rn(j <= i ? acc[mt][nt][e] : 0.f);
+    });
+  } else {
+    for (int idx = tid; idx < kC * kC; idx += kThreads) {
+      const int i = idx / kC, j = idx % kC;
+      float p = 0.f, s = 0.f;
+      if (j <= i) {
+        for (int r = 0; r < DK; ++r) {
+          const float e = expf(sG[i * LK + r] - sG[j * LK + r]) * __bfloat162float(sk[j * LKb + r]);
+          p = fmaf(__bfloat162float(sk[i * LKb + r]), e, p);
+          s = fmaf(__bfloat162float(sq[i * LKb + r]), e, s);
+        }
+      }
+      sP[i * kLC + j] = j < i ? p : 0.f;
+      pr[PR::oAqkt + j * PR::LCb + i] = __float2bfloat16_rn(j <= i ? a.scale * s : 0.f);
+    }
+  }
+  __syncthreads();
+  store_f32(a.Pkk + rec * kC * kC, kC, sP, kLC, kC, kC);
+
+  // T = (I + diag(beta) P)^-1: thread j < 64 keeps column j in registers (see the fp32 kernel)
+  bf16* Tg = reinterpret_cast<bf16*>(a.Tm) + rec * kC * kC;
+  if (tid < kC) {
+    const int j = tid;
+    float tc[kC];
+#pragma unroll
+    for (int i = 0; i < kC; ++i) {
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int m = 0; m < i; m += 4) {
+        const float4 p = *reinterpret_cast<const float4*>(sP + i * kLC + m);
+        s4[0] = fmaf(p.x, tc[m], s4[0]);
+        if (m + 1 < i) s4[1] = fmaf(p.y, tc[m + 1], s4[1]);
+        if (m + 2 < i) s4[2] = fmaf(p.z, tc[m + 2], s4[2]);
+        if (m + 3 < i) s4[3] = fmaf(p.w, tc[m + 3], s4[3]);
+      }
+      tc[i] = i == j ? 1.f : (i < j ? 0.f : -sb[i] * ((s4[0] + s4[1]) + (s4[2] + s4[3])));
+      const bf16 tb = __float2bfloat16_rn(tc[i]);
+      sT[i * LCb + j] = tb;
+      Tg[i * kC + j] = tb;
+    }
+  }
+  // beta K+ and beta v as the right operands of W and U (the factored tiles are dead)
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {
+    const int i = idx / DK, r = idx % DK;
+    sX[i * LKb + r] = __float2bfloat16_rn(sb[i] * __bfloat162float(sk[i * LKb + r]) * expf(sG[i * LK + r]));
+  }
+  for (int idx = tid; idx < kC * DV; idx += kThreads) {
+    const int i = idx / DV, c = idx % DV;
+    sY[i * LMb + c] = __float2bfloat16_rn(sb[i] * __bfloat162float(sv[i * LVb + c]));
+  }
+  __syncthreads();
+  {  // W = T (beta K+): record W and W^T
+    using Tl = Tiling<kC, DK>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);
+    warp_mma_bf16<Tl::MT, Tl::NT, kC, false, false>(acc, sT, LCb, sX, LKb, m0, n0);
+    acc_to_bf16(acc, pr + PR::oW, PR::LKb, m0, n0);
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
+      pr[PR::oWt + c * PR::LCb + i] = __float2bfloat16_rn(acc[mt][nt][e]);
+    });
+  }
+  {  // U = T (beta v), fp32
+    using Tl = Tiling<kC, DV>;
+    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
+    float acc[Tl::MT][Tl::NT][4];
+    zero(acc);
+    warp_mma_bf16<Tl::MT, Tl::NT, kC, false, false>(acc, sT, LCb, sY, LMb, m0, n0);
+    acc_to_global(acc, a.U + rec * kC * DV, DV, m0, n0);
+  }
+}
+
 // ------------------------------------------------------------------ kernel 3 (bf16 operands)
 template <int DK, int DV>
 struct LocalAPlanB {  // bytes
@@ -1217,11 +1391,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const Chu
   rows_in(sS0, LVb, DK, DV, [&](int i) { return S0 + (size_t)i * DV; }, DK);
   rows_in(sdS, LVb, DK, DV, [&](int i) { return dS + (size_t)i * DV; }, DK);
   if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const bf16*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
-  for (int idx = tid; idx < kC * kC / 4; idx += kThreads) {  // T (fp32) as a bf16 image
-    const int i = idx / (kC / 4), j = (idx % (kC / 4)) * 4;
-    const float4 x = *reinterpret_cast<const float4*>(a.Tm + rec * kC * kC + i * kC + j);
-    *reinterpret_cast<__nv_bfloat162*>(sT + i * LCb + j) = __floats2bfloat162_rn(x.x, x.y);
-    *reinterpret_cast<__nv_bfloat162*>(sT + i * LCb + j + 2) = __floats2bfloat162_rn(x.z, x.w);
+  {
+    const bf16* Tg = reinterpret_cast<const bf16*>(a.Tm) + rec * kC * kC;
+    rows_in(sT, LCb, kC, kC, [&](int i) { return Tg + (size_t)i * kC; }, kC);
   }
   cp_wait();
   __syncthreads();
@@ -1602,7 +1774,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
   const bool slow = chunk_unsafe<DK>(sG, LK);
   f32_to_img(sA, LKb, a.dW + rec * kC * DK, kC, DK);
-  f32_to_img(sT, LCb, a.Tm + rec * kC * kC, kC, kC);
+  {
+    const bf16* Tg = reinterpret_cast<const bf16*>(a.Tm) + rec * kC * kC;
+    for (int idx = tid; idx < kC * (kC / 8); idx += kThreads) {
+      const int i = idx / (kC / 8), c = (idx % (kC / 8)) * 8;
+      cp16(sT + i * LCb + c, Tg + (size_t)i * kC + c, 16);
+    }
+  }
   f32_to_img(sQA, LCb, a.dAqk + rec * kC * kC, kC, kC);
   cp_wait();
   __syncthreads();
@@ -1808,8 +1986,8 @@ struct WsPlan {
       : W(f32 ? (size_t)kC * dk : 0), U((size_t)kC * dv), Qp((size_t)kC * dk), Kb((size_t)kC * dk),
         Wt(f32 ? (size_t)kC * dk : 0), Qpt(f32 ? (size_t)kC * dk : 0), Kbt(f32 ? (size_t)kC * dk : 0),
         Aqk(f32 ? kC * kC : 0), prec(f32 ? 0 : (dk == 128 ? PassRec<128>::n : PassRec<64>::n) / 2),
-        // bf16 inputs: S0, dS, V', dV' are kept as bf16 (half the floats)
-        Tm(kC * kC), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv / (f32 ? 1 : 2)), dSc((size_t)dk * dv / (f32 ? 1 : 2)),
+        // bf16 inputs: T, S0, dS, V', dV' are kept as bf16 (half the floats)
+        Tm(kC * kC / (f32 ? 1 : 2)), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv / (f32 ? 1 : 2)), dSc((size_t)dk * dv / (f32 ? 1 : 2)),
         Vp((size_t)kC * dv / (f32 ? 1 : 2)), dVp((size_t)kC * dv / (f32 ? 1 : 2)), dAqk(kC * kC), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk),
         dKb((size_t)kC * dk), dgam(dk), dbu(kC) {}
   size_t per_rec() const {
@@ -1834,7 +2012,9 @@ cudaError_t launch_k(Kern kern, dim3 grid, size_t smem, const ChunkBwdArgs& a, c
 template <typename IO, int DK, int DV>
 cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t stream) {
   const dim3 grid((unsigned)a.NC * BH);  // chunk-major within each (sequence, head)
-  cudaError_t e = launch_k(bwd_prep_kernel<IO, DK, DV>, grid, prep_smem<DK, DV>(), a, stream);
+  cudaError_t e = std::is_same<IO, float>::value
+                      ? launch_k(bwd_prep_kernel<float, DK, DV>, grid, prep_smem<DK, DV>(), a, stream)
+                      : launch_k(bwd_prep_bf16_kernel<DK, DV>, grid, PrepPlanB<DK, DV>::bytes, a, stream);
   if (e != cudaSuccess) return e;
   const bool w32 = pass_width(BH, DV) == 32;
   if constexpr (std::is_same<IO, float>::value) {
