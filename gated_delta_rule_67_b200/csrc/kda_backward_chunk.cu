@@ -35,11 +35,14 @@
 //   3. bwd_local_a (chunk, seq x head): the products contracting over d_v:
 //      dAqk, dT (first part), dv, dbeta (first part), dO S0^T, dW, dKbar, dgamma
 //   4. bwd_local_b (chunk, seq x head): the rest, and dq, dk, dg, dbeta
-// Arithmetic: warp-level tensor-core products (mma.sync m16n8k8, tf32
-// operands, fp32 accumulation) on fp32 shared-memory tiles.  With fp32 I/O
-// every product uses the three-term tf32 split (a_hi b_hi + a_hi b_lo +
-// a_lo b_hi), which keeps fp32-level accuracy; with bf16 I/O one tf32 term.
-// Everything in the workspace is fp32.  No atomics: every sum runs in a fixed
+// Arithmetic: warp-level tensor-core products (mma.sync), fp32 accumulation.
+// fp32 inputs: fp32 shared tiles, m16n8k8 with tf32 operands in the
+// three-term split (a_hi b_hi + a_hi b_lo + a_lo b_hi), which keeps fp32-level
+// accuracy; fp32 workspace.  bf16 inputs: bf16 operand images (ldmatrix, with
+// .trans where the stored rows run along the other index), m16n8k16 with bf16
+// operands; the state passes keep the state in fp32 registers and read each
+// chunk's operands as one bf16 record; the decay factors, the fold into the
+// gradients and every sum stay fp32.  No atomics: every sum runs in a fixed
 // order, so results are bit-reproducible.
 #include <algorithm>
 #include <type_traits>
@@ -407,7 +410,8 @@ constexpr size_t prep_smem() {
   return sizeof(float) * ((size_t)4 * kC * LK + (size_t)kC * LM + 3 * kC * kLC + kC + DK);
 }
 
-// Per chunk: G, the factored and absolute operands, P and Aqk, T, W and U.
+// Per chunk, fp32 inputs (IO = float; bf16 inputs take the kernels on bf16
+// operands below): G, the factored and absolute operands, P and Aqk, T, W and U.
 template <typename IO, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArgs a) {
   constexpr bool X3 = std::is_same<IO, float>::value;
@@ -443,14 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     const int r = idx / kC, i = idx % kC;
     const float G = sG[i * LK + r], qq = a.scale * sQ[i * LK + r];
     const float qp = qq * expf(G), kb = sK[i * LK + r] * expf(sG[(kC - 1) * LK + r] - G);
-    if constexpr (X3) {
-      a.Qpt[rec * kC * DK + idx] = qp;
-      a.Kbt[rec * kC * DK + idx] = kb;
-    } else {
-      bf16* pr = a.prec + rec * PassRec<DK>::n;
-      pr[PassRec<DK>::oQpt + r * PassRec<DK>::LCb + i] = __float2bfloat16_rn(qp);
-      pr[PassRec<DK>::oKbt + r * PassRec<DK>::LCb + i] = __float2bfloat16_rn(kb);
-    }
+    a.Qpt[rec * kC * DK + idx] = qp;
+    a.Kbt[rec * kC * DK + idx] = kb;
   }
   float* Qp = a.Qp + rec * kC * DK;
   float* Kb = a.Kb + rec * kC * DK;
@@ -461,8 +459,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     const float gm = expf(G);
     Qp[i * DK + r] = qq * gm;
     Kb[i * DK + r] = kk * expf(sG[(kC - 1) * LK + r] - G);
-    if constexpr (!X3)
-      a.prec[rec * PassRec<DK>::n + PassRec<DK>::oKb + i * PassRec<DK>::LKb + r] = __float2bfloat16_rn(Kb[i * DK + r]);
     if (!slow) {
       const float d = G - sG[kRef * LK + r];
       const float ex = expf(d);
@@ -509,10 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
   store_f32(a.Pkk + rec * kC * kC, kC, sP, kLC, kC, kC);
   for (int idx = tid; idx < kC * kC; idx += kThreads) {  // Aqk^T
     const int j = idx / kC, i = idx % kC;
-    if constexpr (X3)
-      a.Aqk[rec * kC * kC + idx] = sA[i * kLC + j];
-    else
-      a.prec[rec * PassRec<DK>::n + PassRec<DK>::oAqkt + j * PassRec<DK>::LCb + i] = __float2bfloat16_rn(sA[i * kLC + j]);
+    a.Aqk[rec * kC * kC + idx] = sA[i * kLC + j];
   }
 
   // T = (I + diag(beta) P)^-1 (unit lower triangular) by forward substitution
@@ -550,22 +543,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);
     warp_mma<Tl::MT, Tl::NT, X3, kC>(acc, rowm(sT, kLC), rowm(sX, LK), m0, n0);
-    if constexpr (X3) {
-      float* Wg = a.W + rec * kC * DK;
-      float* Wtg = a.Wt + rec * kC * DK;
-      for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
-        Wg[i * DK + c] = acc[mt][nt][e];
-        Wtg[c * kC + i] = acc[mt][nt][e];
-      });
-    } else {
-      using PR = PassRec<DK>;
-      bf16* pr = a.prec + rec * PR::n;
-      for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
-        const bf16 w = __float2bfloat16_rn(acc[mt][nt][e]);
-        pr[PR::oW + i * PR::LKb + c] = w;
-        pr[PR::oWt + c * PR::LCb + i] = w;
-      });
-    }
+    float* Wg = a.W + rec * kC * DK;
+    float* Wtg = a.Wt + rec * kC * DK;
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
+      Wg[i * DK + c] = acc[mt][nt][e];
+      Wtg[c * kC + i] = acc[mt][nt][e];
+    });
   }
   {
     using Tl = Tiling<kC, DV>;
