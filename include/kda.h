@@ -158,11 +158,11 @@ KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Bytes of device workspace kda_backward needs for this problem: fp32
- * per-chunk records (per 64-token chunk and head: the chunk's operands, the
- * state entering it and the state gradient leaving it, and intermediate
- * gradients; about 0.6 MB at dk = dv = 128); 0 for arguments kda_backward
- * would reject.
+ * Bytes of device workspace kda_backward needs for this problem: per-chunk
+ * records (per 64-token chunk and head: the chunk's operands, the state
+ * entering it and the state gradient leaving it, and intermediate gradients;
+ * about 0.45 MB for bf16 and 0.6 MB for fp32 at dk = dv = 128); 0 for
+ * arguments kda_backward would reject.
  */
 KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
 
@@ -174,9 +174,10 @@ KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, 
  * the chunks; sections 2.1-2.2 for the scalar gates): a per-chunk
  * recomputation of the chunk operands, a forward replay of the chunk states
  * and a reverse sweep of the state gradient (each column of the state on its
- * own), then per-chunk local gradients.  Four kernel launches; fp32 storage
- * and accumulation, tensor-core products with tf32 operands (three-term
- * split, i.e. fp32-level accuracy, when dtype is KDA_F32).
+ * own), then per-chunk local gradients.  Four kernel launches (per group of
+ * (sequence, head) pairs, see workspace); tensor-core products with fp32
+ * accumulation: bf16 operands when dtype is KDA_BF16, tf32 operands in a
+ * three-term split (fp32-level accuracy) when dtype is KDA_F32.
  *
  *   q, k, v, g, beta, scale, initial_state : the forward's inputs (layouts
  *                      and gate kinds as for kda_chunk_fwd_ex)
