@@ -1158,7 +1158,9 @@ struct PrepPlanB {  // bytes
                 "16 B");
 };
 
-// Per chunk, bf16 inputs: G (fp32), the factored operands as bf16 images, P
+// Per chunk, bf16 inputs (exponentials by the fast intrinsic: every exponent
+// here is bounded by the factored form's span or is <= 0, and the results
+// feed bf16 operands): G (fp32), the factored operands as bf16 images, P
 // (fp32, for the solve) and Aqk, T by forward substitution in fp32, W and U;
 // the state passes' operands go out as the chunk's bf16 pass record, T as bf16.
 template <int DK, int DV>
@@ -1201,32 +1203,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
   const bool slow = chunk_unsafe<DK>(sG, LK);
   if (tid < DK) {
-    se[tid] = expf(sG[kRef * LK + tid]);
-    a.gam[rec * DK + tid] = expf(sG[(kC - 1) * LK + tid]);
+    se[tid] = __expf(sG[kRef * LK + tid]);
+    a.gam[rec * DK + tid] = __expf(sG[(kC - 1) * LK + tid]);
   }
   cp_wait();
   __syncthreads();
   for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+^T, Kbar^T (record), token index fastest
     const int r = idx / kC, i = idx % kC;
     const float G = sG[i * LK + r];
-    pr[PR::oQpt + r * PR::LCb + i] = __float2bfloat16_rn(a.scale * __bfloat162float(sq[i * LKb + r]) * expf(G));
+    pr[PR::oQpt + r * PR::LCb + i] = __float2bfloat16_rn(a.scale * __bfloat162float(sq[i * LKb + r]) * __expf(G));
     pr[PR::oKbt + r * PR::LCb + i] =
-        __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * expf(sG[(kC - 1) * LK + r] - G));
+        __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * __expf(sG[(kC - 1) * LK + r] - G));
   }
-  float* Qp = a.Qp + rec * kC * DK;
-  float* Kb = a.Kb + rec * kC * DK;
-  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+, Kbar (fp32, record) and the factored operands
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Kbar (record) and the factored operands
     const int i = idx / DK, r = idx % DK;
     const float G = sG[i * LK + r], kk = __bfloat162float(sk[i * LKb + r]);
     const float qq = a.scale * __bfloat162float(sq[i * LKb + r]);
-    const float kb = kk * expf(sG[(kC - 1) * LK + r] - G);
-    Qp[i * DK + r] = qq * expf(G);
-    Kb[i * DK + r] = kb;
-    pr[PR::oKb + i * PR::LKb + r] = __float2bfloat16_rn(kb);
+    pr[PR::oKb + i * PR::LKb + r] = __float2bfloat16_rn(kk * __expf(sG[(kC - 1) * LK + r] - G));
     if (!slow) {
-      const float d = G - sG[kRef * LK + r], ex = expf(d);
+      const float d = G - sG[kRef * LK + r], ex = __expf(d);
       sX[i * LKb + r] = __float2bfloat16_rn(kk * ex);
-      sY[i * LMb + r] = __float2bfloat16_rn(kk * expf(-d));
+      sY[i * LMb + r] = __float2bfloat16_rn(kk * __expf(-d));
       sQ[i * LKb + r] = __float2bfloat16_rn(qq * ex);
     }
   }
@@ -1253,7 +1250,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
       float p = 0.f, s = 0.f;
       if (j <= i) {
         for (int r = 0; r < DK; ++r) {
-          const float e = expf(sG[i * LK + r] - sG[j * LK + r]) * __bfloat162float(sk[j * LKb + r]);
+          const float e = __expf(sG[i * LK + r] - sG[j * LK + r]) * __bfloat162float(sk[j * LKb + r]);
           p = fmaf(__bfloat162float(sk[i * LKb + r]), e, p);
           s = fmaf(__bfloat162float(sq[i * LKb + r]), e, s);
         }
@@ -1290,7 +1287,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   // beta K+ and beta v as the right operands of W and U (the factored tiles are dead)
   for (int idx = tid; idx < kC * DK; idx += kThreads) {
     const int i = idx / DK, r = idx % DK;
-    sX[i * LKb + r] = __float2bfloat16_rn(sb[i] * __bfloat162float(sk[i * LKb + r]) * expf(sG[i * LK + r]));
+    sX[i * LKb + r] = __float2bfloat16_rn(sb[i] * __bfloat162float(sk[i * LKb + r]) * __expf(sG[i * LK + r]));
   }
   for (int idx = tid; idx < kC * DV; idx += kThreads) {
     const int i = idx / DV, c = idx % DV;
@@ -1699,7 +1696,8 @@ struct LocalBPlanB {  // bytes
 
 // Per chunk, bf16 inputs: dT, T^T dW, dA, the pairwise gradients and the fold
 // into dq, dk, dg, dbeta.  Operands are bf16 images; G, the decay factors and
-// the fold run in fp32 (from the exact k, q inputs).
+// the fold run in fp32 (from the exact k, q inputs), exponentials by the fast
+// intrinsic (exponents bounded by the factored form's span, or <= 0).
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const ChunkBwdArgs a) {
   using PL = LocalBPlanB<DK, DV>;
@@ -1769,7 +1767,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   __syncthreads();
   for (int idx = tid; idx < kC * DK; idx += kThreads) {  // K+ = k exp(G)
     const int i = idx / DK, r = idx % DK;
-    sB[i * LKb + r] = __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * expf(sG[i * LK + r]));
+    sB[i * LKb + r] = __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * __expf(sG[i * LK + r]));
   }
   __syncthreads();
   {  // dT = dU (beta V)^T + dW (beta K+)^T, strictly lower, as a bf16 image
@@ -1787,7 +1785,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     zero(acc);
     warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(acc, sT, LCb, sA, LKb, m0, n0);
     for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-      const float x = acc[mt][nt][e], gm = expf(sG[i * LK + r]);
+      const float x = acc[mt][nt][e], gm = __expf(sG[i * LK + r]);
       const float kp = __bfloat162float(sk[i * LKb + r]) * gm, bx = sb[i] * x;
       dk_acc[mt][nt][e] = fmaf(bx, gm, dk_acc[mt][nt][e]);
       dG_acc[mt][nt][e] = fmaf(bx, kp, dG_acc[mt][nt][e]);
@@ -1819,16 +1817,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   if (!slow) {  // factored operands K+_r, K-_r, Q+_r
     for (int idx = tid; idx < kC * DK; idx += kThreads) {
       const int i = idx / DK, r = idx % DK;
-      const float d = sG[i * LK + r] - sG[kRef * LK + r], ex = expf(d);
+      const float d = sG[i * LK + r] - sG[kRef * LK + r], ex = __expf(d);
       const float kk = __bfloat162float(sk[i * LKb + r]), qq = a.scale * __bfloat162float(sq[i * LKb + r]);
       sB[i * LKb + r] = __float2bfloat16_rn(kk * ex);
-      sA[i * LKb + r] = __float2bfloat16_rn(kk * expf(-d));
+      sA[i * LKb + r] = __float2bfloat16_rn(kk * __expf(-d));
       sC[i * LKb + r] = __float2bfloat16_rn(qq * ex);
     }
   }
   __syncthreads();
   const float* dQs = a.dQs + rec * kC * DK;
-  const float* Qp = a.Qp + rec * kC * DK;
   bf16* dq = static_cast<bf16*>(a.dq);
   if (!slow) {
     {  // dQ+_r = dAqk K-_r;  dq = scale (exp(G - G_ref) dQ+_r + Gamma dO S0^T)
@@ -1837,10 +1834,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(acc, sQA, LCb, sA, LKb, m0, n0);
       for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
         const float x = acc[mt][nt][e], G = sG[i * LK + r];
-        const float ex = expf(G - sG[kRef * LK + r]), dqs = dQs[i * DK + r];
-        const float qr = a.scale * __bfloat162float(sq[i * LKb + r]) * ex;  // Q+_r
-        if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(a.scale * fmaf(ex, x, expf(G) * dqs));
-        dG_acc[mt][nt][e] += fmaf(x, qr, dqs * Qp[i * DK + r]);
+        const float ex = __expf(G - sG[kRef * LK + r]), gm = __expf(G), dqs = dQs[i * DK + r];
+        const float qs = a.scale * __bfloat162float(sq[i * LKb + r]);  // Q+_r = qs ex, Q+ = qs Gamma
+        if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(a.scale * fmaf(ex, x, gm * dqs));
+        dG_acc[mt][nt][e] += qs * fmaf(x, ex, dqs * gm);
       });
     }
     {  // dK-_r = dAqk^T Q+_r + M^T K+_r
@@ -1849,7 +1846,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(acc, sQA, LCb, sC, LKb, m0, n0);
       warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(acc, sDT, LCb, sB, LKb, m0, n0);
       for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-        const float x = acc[mt][nt][e], ei = expf(sG[kRef * LK + r] - sG[i * LK + r]);
+        const float x = acc[mt][nt][e], ei = __expf(sG[kRef * LK + r] - sG[i * LK + r]);
         dk_acc[mt][nt][e] = fmaf(ei, x, dk_acc[mt][nt][e]);
         dG_acc[mt][nt][e] = fmaf(-x, __bfloat162float(sk[i * LKb + r]) * ei, dG_acc[mt][nt][e]);
       });
@@ -1859,7 +1856,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       zero(acc);
       warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(acc, sDT, LCb, sA, LKb, m0, n0);
       for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-        const float x = acc[mt][nt][e], ex = expf(sG[i * LK + r] - sG[kRef * LK + r]);
+        const float x = acc[mt][nt][e], ex = __expf(sG[i * LK + r] - sG[kRef * LK + r]);
         dk_acc[mt][nt][e] = fmaf(ex, x, dk_acc[mt][nt][e]);
         dG_acc[mt][nt][e] = fmaf(x, __bfloat162float(sk[i * LKb + r]) * ex, dG_acc[mt][nt][e]);
       });
@@ -1874,30 +1871,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       const float Gi = sG[i * LK + r], ki = K_(i, r), qi = Q_(i, r);
       float dqp = 0.f, dkp = 0.f, dgp = 0.f;
       for (int j = 0; j <= i; ++j) {
-        const float kE = expf(Gi - sG[j * LK + r]) * K_(j, r);
+        const float kE = __expf(Gi - sG[j * LK + r]) * K_(j, r);
         const float c = QA(i, j), m = MM(i, j);
         dqp = fmaf(c, kE, dqp);
         dkp = fmaf(m, kE, dkp);
         dgp = fmaf(fmaf(c, qi, m * ki), kE, dgp);
       }
       for (int j = i; j < kC; ++j) {
-        const float w = fmaf(QA(j, i), Q_(j, r), MM(j, i) * K_(j, r)) * expf(sG[j * LK + r] - Gi);
+        const float w = fmaf(QA(j, i), Q_(j, r), MM(j, i) * K_(j, r)) * __expf(sG[j * LK + r] - Gi);
         dkp += w;
         dgp = fmaf(-w, ki, dgp);
       }
-      const float dqs = dQs[i * DK + r];
-      if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(a.scale * fmaf(expf(Gi), dqs, dqp));
+      const float dqs = dQs[i * DK + r], gm = __expf(Gi);
+      if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(a.scale * fmaf(gm, dqs, dqp));
       dk_acc[mt][nt][e] += dkp;
-      dG_acc[mt][nt][e] += fmaf(dqs, Qp[i * DK + r], dgp);
+      dG_acc[mt][nt][e] += fmaf(dqs, qi * gm, dgp);
     });
   }
   {  // Kbar: dk += exp(G_C - G) dKbar, dG -= dKbar . Kbar, dG_C += column sums of the same
     const float* dKb = a.dKb + rec * kC * DK;
-    const float* Kb = a.Kb + rec * kC * DK;
     float cp[TK::MT][TK::NT][2] = {};
     for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-      const float x = dKb[i * DK + r], y = x * Kb[i * DK + r];
-      dk_acc[mt][nt][e] = fmaf(expf(sG[(kC - 1) * LK + r] - sG[i * LK + r]), x, dk_acc[mt][nt][e]);
+      const float kbf = __expf(sG[(kC - 1) * LK + r] - sG[i * LK + r]);  // Kbar = k kbf
+      const float x = dKb[i * DK + r], y = x * __bfloat162float(sk[i * LKb + r]) * kbf;
+      dk_acc[mt][nt][e] = fmaf(kbf, x, dk_acc[mt][nt][e]);
       dG_acc[mt][nt][e] -= y;
       cp[mt][nt][e & 1] += y;
     });
@@ -1926,7 +1923,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     float x = 0.f;
 #pragma unroll
     for (int w = 0; w < TK::WM; ++w) x += colC[w * DK + r];
-    x = fmaf(expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
+    x = fmaf(__expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
     float acc = x;
     for (int i = kC - 1; i >= 0; --i) {
       acc += sdG[i * LK + r];
@@ -1966,7 +1963,7 @@ struct WsPlan {
   size_t W, U, Qp, Kb, Wt, Qpt, Kbt, Aqk, prec, Tm, Pkk, gam, S0c, dSc, Vp, dVp, dAqk, dT1, dQs, dW, dKb, dgam, dbu;
   // fp32 inputs keep the passes' operands as fp32 arrays, bf16 inputs as one bf16 record per chunk
   explicit WsPlan(int dk, int dv, bool f32)
-      : W(f32 ? (size_t)kC * dk : 0), U((size_t)kC * dv), Qp((size_t)kC * dk), Kb((size_t)kC * dk),
+      : W(f32 ? (size_t)kC * dk : 0), U((size_t)kC * dv), Qp(f32 ? (size_t)kC * dk : 0), Kb(f32 ? (size_t)kC * dk : 0),
         Wt(f32 ? (size_t)kC * dk : 0), Qpt(f32 ? (size_t)kC * dk : 0), Kbt(f32 ? (size_t)kC * dk : 0),
         Aqk(f32 ? kC * kC : 0), prec(f32 ? 0 : (dk == 128 ? PassRec<128>::n : PassRec<64>::n) / 2),
         // bf16 inputs: T, S0, dS, V', dV' are kept as bf16 (half the floats)
