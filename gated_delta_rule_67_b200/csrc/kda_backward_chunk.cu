@@ -1383,13 +1383,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const Chu
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);  // dAqk = tril(dO V'^T)
     warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sO, LVb, sVp, LVb, m0, n0);
-    float* out = a.dAqk + rec * kC * kC;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
-      out[i * kC + j] = j <= i ? acc[mt][nt][e] : 0.f;
+      if (j > i) acc[mt][nt][e] = 0.f;
     });
+    acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dAqk) + rec * kC * kC, kC, m0, n0);  // an operand only: bf16
     zero(acc);  // dU (beta V)^T, strictly lower part
     warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sdV, LVb, sv, LVb, m0, n0);
-    out = a.dT1 + rec * kC * kC;
+    float* out = a.dT1 + rec * kC * kC;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
       out[i * kC + j] = j < i ? acc[mt][nt][e] * sb[j] : 0.f;
     });
@@ -1418,8 +1418,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const Chu
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
     zero(acc);
     warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sdV, LVb, sS0, LVb, m0, n0);
-    out = a.dW + rec * kC * DK;
-    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = -acc[mt][nt][e]; });
+    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { acc[mt][nt][e] = -acc[mt][nt][e]; });
+    acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dW) + rec * kC * DK, DK, m0, n0);  // an operand only: bf16
     zero(acc);
     warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sVp, LVb, sdS, LVb, m0, n0);
     out = a.dKb + rec * kC * DK;
@@ -1740,21 +1740,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       cp16(dst + i * LKb + c, i < nv ? src + (row0 + (size_t)i * a.H) * DK + c : src, i < nv ? 16 : 0);
     }
   };
-  auto f32_to_img = [&](bf16* dst, int ld, const float* src, int rows, int cols) {  // fp32 [rows][cols] -> bf16 image
-    for (int idx = tid; idx < rows * cols / 4; idx += kThreads) {
-      const int i = idx / (cols / 4), j = (idx % (cols / 4)) * 4;
-      const float4 x = *reinterpret_cast<const float4*>(src + (size_t)i * cols + j);
-      *reinterpret_cast<__nv_bfloat162*>(dst + i * ld + j) = __floats2bfloat162_rn(x.x, x.y);
-      *reinterpret_cast<__nv_bfloat162*>(dst + i * ld + j + 2) = __floats2bfloat162_rn(x.z, x.w);
-    }
-  };
+
 
   if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const bf16*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
   rows_in(sk, k);
   rows_in(sq, q);
   load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
   const bool slow = chunk_unsafe<DK>(sG, LK);
-  f32_to_img(sA, LKb, a.dW + rec * kC * DK, kC, DK);
+  {  // dW and dAqk (bf16 from the d_v kernel)
+    const bf16* dWg = reinterpret_cast<const bf16*>(a.dW) + rec * kC * DK;
+    const bf16* dAg = reinterpret_cast<const bf16*>(a.dAqk) + rec * kC * kC;
+    for (int idx = tid; idx < kC * (DK / 8); idx += kThreads) {
+      const int i = idx / (DK / 8), c = (idx % (DK / 8)) * 8;
+      cp16(sA + i * LKb + c, dWg + (size_t)i * DK + c, 16);
+    }
+    for (int idx = tid; idx < kC * (kC / 8); idx += kThreads) {
+      const int i = idx / (kC / 8), c = (idx % (kC / 8)) * 8;
+      cp16(sQA + i * LCb + c, dAg + (size_t)i * kC + c, 16);
+    }
+  }
   {
     const bf16* Tg = reinterpret_cast<const bf16*>(a.Tm) + rec * kC * kC;
     for (int idx = tid; idx < kC * (kC / 8); idx += kThreads) {
@@ -1762,7 +1766,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       cp16(sT + i * LCb + c, Tg + (size_t)i * kC + c, 16);
     }
   }
-  f32_to_img(sQA, LCb, a.dAqk + rec * kC * kC, kC, kC);
   cp_wait();
   __syncthreads();
   for (int idx = tid; idx < kC * DK; idx += kThreads) {  // K+ = k exp(G)
@@ -1966,9 +1969,9 @@ struct WsPlan {
       : W(f32 ? (size_t)kC * dk : 0), U((size_t)kC * dv), Qp(f32 ? (size_t)kC * dk : 0), Kb(f32 ? (size_t)kC * dk : 0),
         Wt(f32 ? (size_t)kC * dk : 0), Qpt(f32 ? (size_t)kC * dk : 0), Kbt(f32 ? (size_t)kC * dk : 0),
         Aqk(f32 ? kC * kC : 0), prec(f32 ? 0 : (dk == 128 ? PassRec<128>::n : PassRec<64>::n) / 2),
-        // bf16 inputs: T, S0, dS, V', dV' are kept as bf16 (half the floats)
+        // bf16 inputs: T, S0, dS, V', dV', dAqk, dW are kept as bf16 (half the floats)
         Tm(kC * kC / (f32 ? 1 : 2)), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv / (f32 ? 1 : 2)), dSc((size_t)dk * dv / (f32 ? 1 : 2)),
-        Vp((size_t)kC * dv / (f32 ? 1 : 2)), dVp((size_t)kC * dv / (f32 ? 1 : 2)), dAqk(kC * kC), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk),
+        Vp((size_t)kC * dv / (f32 ? 1 : 2)), dVp((size_t)kC * dv / (f32 ? 1 : 2)), dAqk(kC * kC / (f32 ? 1 : 2)), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk / (f32 ? 1 : 2)),
         dKb((size_t)kC * dk), dgam(dk), dbu(kC) {}
   size_t per_rec() const {
     return W + U + Qp + Kb + Wt + Qpt + Kbt + Aqk + prec + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs +
