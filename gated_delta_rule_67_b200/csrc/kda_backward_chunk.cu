@@ -1208,13 +1208,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   }
   cp_wait();
   __syncthreads();
-  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+^T, Kbar^T (record), token index fastest
-    const int r = idx / kC, i = idx % kC;
-    const float G = sG[i * LK + r];
-    pr[PR::oQpt + r * PR::LCb + i] = __float2bfloat16_rn(a.scale * __bfloat162float(sq[i * LKb + r]) * __expf(G));
-    pr[PR::oKbt + r * PR::LCb + i] =
-        __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * __expf(sG[(kC - 1) * LK + r] - G));
-  }
   for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Kbar (record) and the factored operands
     const int i = idx / DK, r = idx % DK;
     const float G = sG[i * LK + r], kk = __bfloat162float(sk[i * LKb + r]);
@@ -1260,9 +1253,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
     }
   }
   __syncthreads();
-  store_f32(a.Pkk + rec * kC * kC, kC, sP, kLC, kC, kC);
 
-  // T = (I + diag(beta) P)^-1: thread j < 64 keeps column j in registers (see the fp32 kernel)
+  // Warps 0-1: T = (I + diag(beta) P)^-1, thread j < 64 keeping column j in
+  // registers (see the fp32 kernel).  The other warps meanwhile store P, the
+  // record's Q+^T and Kbar^T, and the right operands beta K+ and beta v of W
+  // and U (the factored tiles are dead).
   bf16* Tg = reinterpret_cast<bf16*>(a.Tm) + rec * kC * kC;
   if (tid < kC) {
     const int j = tid;
@@ -1283,15 +1278,28 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
       sT[i * LCb + j] = tb;
       Tg[i * kC + j] = tb;
     }
-  }
-  // beta K+ and beta v as the right operands of W and U (the factored tiles are dead)
-  for (int idx = tid; idx < kC * DK; idx += kThreads) {
-    const int i = idx / DK, r = idx % DK;
-    sX[i * LKb + r] = __float2bfloat16_rn(sb[i] * __bfloat162float(sk[i * LKb + r]) * __expf(sG[i * LK + r]));
-  }
-  for (int idx = tid; idx < kC * DV; idx += kThreads) {
-    const int i = idx / DV, c = idx % DV;
-    sY[i * LMb + c] = __float2bfloat16_rn(sb[i] * __bfloat162float(sv[i * LVb + c]));
+  } else {
+    const int t2 = tid - kC, n2 = kThreads - kC;
+    float* Pg = a.Pkk + rec * kC * kC;
+    for (int idx = t2; idx < kC * kC / 4; idx += n2) {
+      const int i = idx / (kC / 4), j = (idx % (kC / 4)) * 4;
+      *reinterpret_cast<float4*>(Pg + i * kC + j) = *reinterpret_cast<const float4*>(sP + i * kLC + j);
+    }
+    for (int idx = t2; idx < kC * DK; idx += n2) {  // Q+^T, Kbar^T (record), token index fastest
+      const int r = idx / kC, i = idx % kC;
+      const float G = sG[i * LK + r];
+      pr[PR::oQpt + r * PR::LCb + i] = __float2bfloat16_rn(a.scale * __bfloat162float(sq[i * LKb + r]) * __expf(G));
+      pr[PR::oKbt + r * PR::LCb + i] =
+          __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * __expf(sG[(kC - 1) * LK + r] - G));
+    }
+    for (int idx = t2; idx < kC * DK; idx += n2) {
+      const int i = idx / DK, r = idx % DK;
+      sX[i * LKb + r] = __float2bfloat16_rn(sb[i] * __bfloat162float(sk[i * LKb + r]) * __expf(sG[i * LK + r]));
+    }
+    for (int idx = t2; idx < kC * DV; idx += n2) {
+      const int i = idx / DV, c = idx % DV;
+      sY[i * LMb + c] = __float2bfloat16_rn(sb[i] * __bfloat162float(sv[i * LVb + c]));
+    }
   }
   __syncthreads();
   {  // W = T (beta K+): record W and W^T
