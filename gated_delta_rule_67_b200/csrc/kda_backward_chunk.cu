@@ -1433,9 +1433,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const Chu
     out = a.dKb + rec * kC * DK;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
   }
-  for (int r = warp; r < DK; r += kWarps) {  // rowsum(dS . S0)
+  for (int r = warp; r < DK; r += kWarps) {  // rowsum(dS . S0), two columns per load
     float x = 0.f;
-    for (int c = lane; c < DV; c += 32) x = fmaf(__bfloat162float(sdS[r * LVb + c]), __bfloat162float(sS0[r * LVb + c]), x);
+    for (int c = 2 * lane; c < DV; c += 64) {
+      const float2 d = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sdS + r * LVb + c));
+      const float2 s0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sS0 + r * LVb + c));
+      x = fmaf(d.x, s0.x, fmaf(d.y, s0.y, x));
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
     if (lane == 0) a.dgam[rec * DK + r] = x;
@@ -1697,7 +1701,8 @@ struct LocalBPlanB {  // bytes
   static constexpr size_t tk = (size_t)kC * LKb * 2, tc = (size_t)kC * LCb * 2;
   static constexpr size_t oG = 0, ok = oG + (size_t)kC * LK * 4, oq = ok + tk, oA = oq + tk, oB = oA + tk,
                           oC = oB + tk, oT = oC + tk, oDT = oT + tc, oY = oDT + tc, oQA = oY + tc, ob = oQA + tc,
-                          ored = ob + kC * 4, ocol = ored + 8 * kC * 4, bytes = ocol + 4 * DK * 4;
+                          ored = ob + kC * 4, ocol = ored + 8 * kC * 4, oQs = ocol + 4 * DK * 4,
+                          oKs = oQs + (size_t)kC * DK * 4, bytes = oKs + (size_t)kC * DK * 4;
   static_assert(tk % 16 == 0 && tc % 16 == 0 && ok % 16 == 0, "16 B");
   static_assert(2 * tk >= (size_t)kC * LK * 4, "dG (fp32) fits over the k and q tiles");
 };
@@ -1727,6 +1732,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   float* red = reinterpret_cast<float*>(smb + PL::ored);  // [8][64] row sums per column group
   float* colC = reinterpret_cast<float*>(smb + PL::ocol);  // [4][DK] column sums of dKbar . Kbar
   float* sdG = reinterpret_cast<float*>(smb + PL::ok);  // [64][LK] dG (fp32), over the k and q tiles at the end
+  float* sQs = reinterpret_cast<float*>(smb + PL::oQs);  // [64][DK] dO S0^T (fp32, from the d_v kernel)
+  float* sKs = reinterpret_cast<float*>(smb + PL::oKs);  // [64][DK] dKbar (fp32, from the d_v kernel)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
@@ -1772,6 +1779,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     for (int idx = tid; idx < kC * (kC / 8); idx += kThreads) {
       const int i = idx / (kC / 8), c = (idx % (kC / 8)) * 8;
       cp16(sT + i * LCb + c, Tg + (size_t)i * kC + c, 16);
+    }
+  }
+  {  // the fold's fp32 inputs, in flight while the products run
+    const float* qs = a.dQs + rec * kC * DK;
+    const float* ks = a.dKb + rec * kC * DK;
+    for (int idx = tid; idx < kC * DK / 4; idx += kThreads) {
+      cp16(sQs + 4 * idx, qs + 4 * idx, 16);
+      cp16(sKs + 4 * idx, ks + 4 * idx, 16);
     }
   }
   cp_wait();
@@ -1836,7 +1851,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     }
   }
   __syncthreads();
-  const float* dQs = a.dQs + rec * kC * DK;
+  const float* dQs = sQs;
   bf16* dq = static_cast<bf16*>(a.dq);
   if (!slow) {
     {  // dQ+_r = dAqk K-_r;  dq = scale (exp(G - G_ref) dQ+_r + Gamma dO S0^T)
@@ -1900,7 +1915,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     });
   }
   {  // Kbar: dk += exp(G_C - G) dKbar, dG -= dKbar . Kbar, dG_C += column sums of the same
-    const float* dKb = a.dKb + rec * kC * DK;
+    const float* dKb = sKs;
     float cp[TK::MT][TK::NT][2] = {};
     for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
       const float kbf = __expf(sG[(kC - 1) * LK + r] - sG[i * LK + r]);  // Kbar = k kbf
