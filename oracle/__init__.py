@@ -144,6 +144,32 @@ def prepare_inputs(q, k, g, beta, prep):
     return q, k, g, beta
 
 
+def prepare_backward(q, k, g, beta, prep, dq_hat, dk_hat, dg_hat, dbeta_hat):
+    """Gradients with respect to the raw inputs of prepare_inputs, given the
+    gradients (dq_hat, dk_hat, dg_hat, dbeta_hat) with respect to its
+    outputs (the chain rule of each preparation step, fp64):
+    q_hat = r q with r = (sum_c q_c^2 + 1e-6)^-1/2:  dq = r (dq_hat - q_hat (q_hat . dq_hat));
+    g_hat = log sigmoid(g):  dg = dg_hat sigmoid(-g);
+    beta_hat = sigmoid(beta):  dbeta = dbeta_hat sigmoid(beta) (1 - sigmoid(beta)).
+    Steps whose bit is not set pass their gradient through; g may be None."""
+    q, k, beta = _as_f64(q), _as_f64(k), _as_f64(beta)
+    dq, dk, dbeta = _as_f64(dq_hat), _as_f64(dk_hat), _as_f64(dbeta_hat)
+    dg = None if dg_hat is None else _as_f64(dg_hat)
+    if prep & PREP_L2NORM_QK:
+        out = []
+        for x, dx in ((q, dq), (k, dk)):
+            r = 1.0 / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + L2_EPS)
+            xh = x * r
+            out.append(r * (dx - xh * np.sum(xh * dx, axis=-1, keepdims=True)))
+        dq, dk = out
+    if prep & PREP_GATE_LOGSIGMOID and dg is not None:
+        dg = dg / (1.0 + np.exp(_as_f64(g)))            # sigmoid(-g)
+    if prep & PREP_BETA_SIGMOID:
+        sb = 1.0 / (1.0 + np.exp(-beta))
+        dbeta = dbeta * sb * (1.0 - sb)
+    return dq, dk, dg, dbeta
+
+
 def kda_backward(q, k, v, g, beta, scale, initial_state, d_o, d_final_state=None, nthreads=0, lib=None):
     """fp64 gradients of a loss through kda_forward, given dL/do [B,T,H,dv] and
     dL/dS_T [B,H,dk,dv] (None: zero).  Returns a dict with dq, dk, dv, dg
