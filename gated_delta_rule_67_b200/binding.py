@@ -36,6 +36,8 @@ SIGNATURES = {
     "kda_recurrent_step_ex": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 7 + [_vp]),
     "kda_backward_workspace_size": (_sz, [_i] * 6),
     "kda_backward": (_i, [_vp] * 5 + [_f] + [_vp] * 9 + [_i] * 7 + [_vp, _sz, _vp]),
+    "kda_backward_ex_workspace_size": (_sz, [_i] * 7),
+    "kda_backward_ex": (_i, [_vp] * 5 + [_f] + [_vp] * 9 + [_i] * 8 + [_vp, _sz, _vp]),
 }
 
 # kda_gate: how the forget gate enters the update (see include/kda.h)
@@ -270,10 +272,12 @@ def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=No
 
 
 def kda_backward(q, k, v, g, beta, grad_o, scale=None, initial_state=None, grad_final_state=None, *,
-                 workspace=None, stream=None, want_initial_state_grad=True):
-    """Gradients of a loss through kda_chunk_fwd (prepared inputs; g per key
-    channel [B,T,H,dk], per head [B,T,H] or None, as for the forward), given
-    grad_o = dL/do [B,T,H,dv] and grad_final_state = dL/dS_T [B,H,dk,dv] fp32 (or None).
+                 workspace=None, stream=None, want_initial_state_grad=True, prep=0):
+    """Gradients of a loss through kda_chunk_fwd (g per key channel [B,T,H,dk],
+    per head [B,T,H] or None, as for the forward), given grad_o = dL/do
+    [B,T,H,dv] and grad_final_state = dL/dS_T [B,H,dk,dv] fp32 (or None).
+    ``prep``: the forward's KDA_PREP_* bits; q, k, g, beta are then the raw
+    inputs and the gradients are taken with respect to them.
 
     Returns a dict: dq, dk, dv, dg (like g; None without a gate), dbeta (input
     dtype) and dS0 = dL/dS_0 fp32 (None if not wanted).
@@ -301,14 +305,14 @@ def kda_backward(q, k, v, g, beta, grad_o, scale=None, initial_state=None, grad_
                dg=None if g is None else torch.empty_like(g), dbeta=torch.empty_like(beta),
                dS0=torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_initial_state_grad
                else None)
-    need = int(lib.kda_backward_workspace_size(B, T, H, dk, dv, code))
+    need = int(lib.kda_backward_ex_workspace_size(B, T, H, dk, dv, code, int(prep)))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
-                          _ptr(grad_o), _ptr(grad_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
-                          _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, dk, dv, code, gate,
-                          _ptr(workspace), ws_bytes, _stream(stream, q.device))
+    st = lib.kda_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
+                             _ptr(grad_o), _ptr(grad_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                             _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, dk, dv, code, gate,
+                             int(prep), _ptr(workspace), ws_bytes, _stream(stream, q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_backward")
     return out

@@ -190,15 +190,32 @@ size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, int dtyp
   return kda::backward_workspace_bytes(B, T, H, dk, dv, dtype);
 }
 
+size_t kda_backward_ex_workspace_size(int B, int T, int H, int dk, int dv, int dtype, int prep) {
+  const size_t base = kda_backward_workspace_size(B, T, H, dk, dv, dtype);
+  if (base == 0 || (prep & ~kda::kPrepMask)) return 0;
+  return prep ? base + kda::backward_prep_bytes(B, T, H, dk, dtype) : base;
+}
+
 kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
                         const float* initial_state, const void* grad_o, const float* grad_final_state, void* grad_q,
                         void* grad_k, void* grad_v, void* grad_g, void* grad_beta, float* grad_initial_state, int B,
                         int T, int H, int dk, int dv, int dtype, int gate, void* workspace, size_t workspace_bytes,
                         void* stream_) {
+  return kda_backward_ex(q, k, v, g, beta, scale, initial_state, grad_o, grad_final_state, grad_q, grad_k, grad_v,
+                         grad_g, grad_beta, grad_initial_state, B, T, H, dk, dv, dtype, gate, KDA_PREP_NONE, workspace,
+                         workspace_bytes, stream_);
+}
+
+kda_status kda_backward_ex(const void* q, const void* k, const void* v, const void* g, const void* beta, float scale,
+                           const float* initial_state, const void* grad_o, const float* grad_final_state, void* grad_q,
+                           void* grad_k, void* grad_v, void* grad_g, void* grad_beta, float* grad_initial_state, int B,
+                           int T, int H, int dk, int dv, int dtype, int gate, int prep, void* workspace,
+                           size_t workspace_bytes, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1) return KDA_ERR_INVALID_ARG;
   if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE) return KDA_ERR_INVALID_ARG;
+  if (prep & ~kda::kPrepMask) return KDA_ERR_INVALID_ARG;
   if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return KDA_ERR_INVALID_ARG;
   if (gate == KDA_GATE_NONE) g = nullptr, grad_g = nullptr;
   const bool empty = (B == 0 || T == 0);
@@ -239,11 +256,18 @@ kda_status kda_backward(const void* q, const void* k, const void* v, const void*
                            : cudaMemsetAsync(grad_initial_state, 0, state_bytes, stream);
     return from_cuda(e);
   }
-  const size_t need_ws = kda::backward_workspace_bytes(1, T, 1, dk, dv, dtype);  // one (sequence, head) at least
+  // at least one (sequence, head)'s records, after the prepared inputs when `prep` is set
+  const size_t prep_ws = prep ? kda::backward_prep_bytes(B, T, H, dk, dtype) : 0;
+  const size_t need_ws = prep_ws + kda::backward_workspace_bytes(1, T, 1, dk, dv, dtype);
   if (!workspace || workspace_bytes < need_ws || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
   const Range rw{(const char*)workspace, workspace_bytes};
   for (Range r : {rq, rk, rv, rg, rb, rs0, rdo, rdsT, wq, wk, wv, wg, wb, ws0})
     if (overlaps(rw, r)) return KDA_ERR_INVALID_ARG;
+  if (prep)
+    return from_cuda(kda::launch_backward_prepared(q, k, v, g, beta, scale, initial_state, grad_o, grad_final_state,
+                                                   grad_q, grad_k, grad_v, grad_g, grad_beta, grad_initial_state, B,
+                                                   T, H, dk, dv, dtype, gate, prep, workspace, workspace_bytes,
+                                                   stream));
   return from_cuda(kda::launch_backward(q, k, v, g, beta, scale, initial_state, grad_o, grad_final_state, grad_q,
                                         grad_k, grad_v, grad_g, grad_beta, grad_initial_state, B, T, H, dk, dv, dtype,
                                         gate, workspace, workspace_bytes, stream));

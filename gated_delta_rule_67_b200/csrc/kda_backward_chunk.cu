@@ -363,6 +363,7 @@ struct ChunkBwdArgs {
   const float *s0, *dsT;
   void *dq, *dk, *dv, *dg, *dbeta;
   float* ds0;
+  float *dq32, *dk32;  // bf16 inputs: when set, dq and dk go here in fp32 instead (for a later chain rule)
   float scale;
   int T, H, NC, gate;
   int bh0;  // first (sequence, head) of this launch group: bh = bh0 + local index
@@ -1862,7 +1863,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
         const float x = acc[mt][nt][e], G = sG[i * LK + r];
         const float ex = __expf(G - sG[kRef * LK + r]), gm = __expf(G), dqs = dQs[i * DK + r];
         const float qs = a.scale * __bfloat162float(sq[i * LKb + r]);  // Q+_r = qs ex, Q+ = qs Gamma
-        if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(a.scale * fmaf(ex, x, gm * dqs));
+        if (i < nv) {
+          const float v = a.scale * fmaf(ex, x, gm * dqs);
+          const size_t o = (row0 + (size_t)i * a.H) * DK + r;
+          if (a.dq32) a.dq32[o] = v; else dq[o] = __float2bfloat16_rn(v);
+        }
         dG_acc[mt][nt][e] += qs * fmaf(x, ex, dqs * gm);
       });
     }
@@ -1909,7 +1914,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
         dgp = fmaf(-w, ki, dgp);
       }
       const float dqs = dQs[i * DK + r], gm = __expf(Gi);
-      if (i < nv) dq[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(a.scale * fmaf(gm, dqs, dqp));
+      if (i < nv) {
+        const float v = a.scale * fmaf(gm, dqs, dqp);
+        const size_t o = (row0 + (size_t)i * a.H) * DK + r;
+        if (a.dq32) a.dq32[o] = v; else dq[o] = __float2bfloat16_rn(v);
+      }
       dk_acc[mt][nt][e] += dkp;
       dG_acc[mt][nt][e] += fmaf(dqs, qi * gm, dgp);
     });
@@ -1939,7 +1948,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   }
   bf16* dk = static_cast<bf16*>(a.dk);
   for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-    if (i < nv) dk[(row0 + (size_t)i * a.H) * DK + r] = __float2bfloat16_rn(dk_acc[mt][nt][e]);
+    if (i < nv) {
+      const size_t o = (row0 + (size_t)i * a.H) * DK + r;
+      if (a.dk32) a.dk32[o] = dk_acc[mt][nt][e]; else dk[o] = __float2bfloat16_rn(dk_acc[mt][nt][e]);
+    }
   });
   __syncthreads();  // the k and q tiles are no longer read: they take dG
   for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) { sdG[i * LK + r] = dG_acc[mt][nt][e]; });
@@ -2072,8 +2084,10 @@ size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) 
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
                             float scale, const float* s0, const void* d_o, const float* dsT, void* dq, void* dk_out,
                             void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H, int dk, int dv,
-                            int dtype, int gate, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                            int dtype, int gate, void* ws, size_t ws_bytes, cudaStream_t stream, float* dq32,
+                            float* dk32) {
   ChunkBwdArgs a;
+  a.dq32 = dq32, a.dk32 = dk32;
   a.q = q, a.k = k, a.v = v, a.g = g, a.beta = beta, a.d_o = d_o;
   a.s0 = s0, a.dsT = dsT;
   a.dq = dq, a.dk = dk_out, a.dv = dv_out, a.dg = dg, a.dbeta = dbeta, a.ds0 = ds0;

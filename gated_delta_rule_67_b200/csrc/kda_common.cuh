@@ -48,7 +48,17 @@ size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
                             float scale, const float* s0, const void* d_o, const float* dsT, void* dq, void* dk_out,
                             void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H, int dk, int dv,
-                            int dtype, int gate, void* ws, size_t ws_bytes, cudaStream_t stream);
+                            int dtype, int gate, void* ws, size_t ws_bytes, cudaStream_t stream,
+                            float* dq32 = nullptr, float* dk32 = nullptr);
+
+// Backward through the fused input preparation (kda_backward_prep.cu): the
+// workspace holds backward_prep_bytes of prepared inputs, then the records.
+size_t backward_prep_bytes(int B, int T, int H, int dk, int dtype);
+cudaError_t launch_backward_prepared(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                     float scale, const float* s0, const void* d_o, const float* dsT, void* dq,
+                                     void* dk_out, void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H,
+                                     int dk, int dv, int dtype, int gate, int prep, void* ws, size_t ws_bytes,
+                                     cudaStream_t stream);
 
 // Launches a kernel whose only wait can never be satisfied (short limit).
 cudaError_t launch_wait_selftest(void* ws, cudaStream_t stream);

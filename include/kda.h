@@ -212,6 +212,33 @@ KDA_API kda_status kda_backward(const void* q, const void* k, const void* v, con
                                 void* stream);
 
 /*
+ * Workspace bytes of kda_backward_ex: kda_backward_workspace_size plus, when
+ * `prep` has bits set, room for the prepared inputs; 0 for arguments
+ * kda_backward_ex would reject.
+ */
+KDA_API size_t kda_backward_ex_workspace_size(int B, int T, int H, int dk, int dv, int dtype, int prep);
+
+/*
+ * kda_backward for a forward that prepared raw inputs in its kernels
+ * (kda_chunk_fwd_ex with the same `prep` bits): q, k, g, beta are the RAW
+ * inputs and grad_q, grad_k, grad_g, grad_beta the gradients with respect to
+ * them.  The library prepares the inputs into the workspace (input dtype,
+ * so bf16 inputs are prepared and then rounded to bf16), runs the backward on
+ * them, and applies the chain rule of each step in place (fp32):
+ * dq = r (dq^ - q^ (q^ . dq^)) with r = (sum q^2 + 1e-6)^-1/2 (same for k),
+ * dg = dg^ sigmoid(-g), dbeta = dbeta^ sigmoid(beta) (1 - sigmoid(beta)).
+ * workspace: kda_backward_ex_workspace_size() bytes hold everything; smaller
+ * works down to the prepared inputs plus one (sequence, head)'s records.
+ * prep = KDA_PREP_NONE is kda_backward.  Other arguments as kda_backward.
+ */
+KDA_API kda_status kda_backward_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                   float scale, const float* initial_state, const void* grad_o,
+                                   const float* grad_final_state, void* grad_q, void* grad_k, void* grad_v,
+                                   void* grad_g, void* grad_beta, float* grad_initial_state, int B, int T, int H,
+                                   int dk, int dv, int dtype, int gate, int prep, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
  * kda_chunk_fwd with timing marks for measurement: `events` points to three
  * cudaEvent_t handles (created by the caller) which are recorded on `stream`
  * before the first kernel, between the chunk-preparation kernel and the

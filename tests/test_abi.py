@@ -174,6 +174,14 @@ def test_backward_validation(lib):
     assert call(ws=None) == binding.KDA_ERR_INVALID_ARG
     assert call(wsb=16) == binding.KDA_ERR_INVALID_ARG
     one = lib.kda_backward_workspace_size(1, 64, 1, 128, 128, 1)
+    assert lib.kda_backward_ex_workspace_size(1, 64, 1, 128, 128, 1, 0) == one
+    assert lib.kda_backward_ex_workspace_size(1, 64, 1, 128, 128, 1, 7) > one
+    assert lib.kda_backward_ex_workspace_size(1, 64, 1, 128, 128, 1, 8) == 0   # unknown prep bit
+    fx = lib.kda_backward_ex
+    assert fx(*ins, 1.0, None, A + (5 << 30), None, *grads, None, 1, 64, 1, 128, 128, 1, 0, 8, A + (20 << 30),
+              1 << 40, None) == binding.KDA_ERR_INVALID_ARG                # unknown prep bit
+    assert fx(*ins, 1.0, None, A + (5 << 30), None, *grads, None, 1, 64, 1, 128, 128, 1, 0, 7, A + (20 << 30),
+              one, None) == binding.KDA_ERR_INVALID_ARG                    # no room for the prepared inputs
     assert call(wsb=one - 1) == binding.KDA_ERR_INVALID_ARG           # below one (sequence, head)'s records
     assert lib.kda_backward_workspace_size(2, 64, 3, 128, 128, 1) == 6 * one
     bad = list(grads)

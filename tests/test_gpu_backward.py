@@ -161,3 +161,57 @@ def test_backward_matches_gpu_forward_directional_derivative(gate):
     key = dict(q="dq", k="dk", v="dv", g="dg", beta="dbeta", initial_state="dS0")
     dot = sum(float((gr[key[n]].double() * direction[n].double()).sum()) for n in names)
     assert abs(fd - dot) <= 1e-3 * abs(dot) + 1e-3, (fd, dot)
+
+
+@pytest.mark.parametrize("prep", [7, 1, 2, 4], ids=["all", "l2norm", "logsigmoid", "sigmoid"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_backward_through_fused_preparation(prep, dtype):
+    """Raw inputs with KDA_PREP_* bits: the gradients with respect to the raw
+    q, k, g, beta equal the oracle's backward on the prepared inputs followed
+    by its chain rule through the preparation (oracle.prepare_backward)."""
+    from gated_delta_rule_67_b200.workloads import make_raw_prefill_inputs
+    dev = cuda_or_skip()
+    B, T, H, dk, dv = 1, 150, 2, 128, 128
+    x = make_raw_prefill_inputs(B, T, H, dk, dv, dtype, 0.1, seed=106)
+    ready = make_prefill_inputs(B, T, H, dk, dv, dtype, 0.1, seed=106)  # inputs whose step is not selected
+    if not prep & 1:
+        x["q"], x["k"] = ready["q"], ready["k"]
+    if not prep & 2:
+        x["g"] = ready["g"]
+    if not prep & 4:
+        x["beta"] = ready["beta"]
+    d_o, d_s = make_cotangents(B, T, H, dk, dv, dtype, seed=107)
+    scale = dk ** -0.5
+    to = lambda t: t.to(dev)
+    got = kda_backward(to(x["q"]), to(x["k"]), to(x["v"]), to(x["g"]), to(x["beta"]), to(d_o), scale,
+                       to(x["initial_state"]), to(d_s), prep=prep)
+    torch.cuda.synchronize()
+    qp, kp, gp, bp = oracle.prepare_inputs(x["q"], x["k"], x["g"], x["beta"], prep)
+    ref = oracle.kda_backward(qp, kp, x["v"], gp, bp, scale, x["initial_state"], d_o, d_s)
+    dq, dk_, dg, db = oracle.prepare_backward(x["q"], x["k"], x["g"], x["beta"], prep, ref["dq"], ref["dk"], ref["dg"],
+                                              ref["dbeta"])
+    want = dict(dq=dq, dk=dk_, dv=ref["dv"], dg=dg, dbeta=db, dS0=ref["dS0"])
+    for name, r in want.items():
+        assert rel_err(got[name], r) < TOL[dtype], (name, rel_err(got[name], r))
+
+
+def test_backward_through_preparation_head_gate():
+    """Per-head raw gates with the log-sigmoid bit (and the other two bits)."""
+    dev = cuda_or_skip()
+    from gated_delta_rule_67_b200.workloads import make_raw_prefill_inputs
+    B, T, H, dk, dv = 1, 100, 2, 64, 64
+    x = make_raw_prefill_inputs(B, T, H, dk, dv, torch.float32, 0.1, seed=108)
+    gh = make_head_gates((B, T, H), 1, torch.float32, seed=109, raw=True)
+    d_o, d_s = make_cotangents(B, T, H, dk, dv, torch.float32, seed=110)
+    to = lambda t: t.to(dev)
+    got = kda_backward(to(x["q"]), to(x["k"]), to(x["v"]), to(gh), to(x["beta"]), to(d_o), None,
+                       to(x["initial_state"]), to(d_s), prep=7)
+    torch.cuda.synchronize()
+    g_b = gh.unsqueeze(-1).expand_as(x["q"]).contiguous()
+    qp, kp, gp, bp = oracle.prepare_inputs(x["q"], x["k"], g_b, x["beta"], 7)
+    ref = oracle.kda_backward(qp, kp, x["v"], gp, bp, dk ** -0.5, x["initial_state"], d_o, d_s)
+    dq, dk_, dg, db = oracle.prepare_backward(x["q"], x["k"], g_b, x["beta"], 7, ref["dq"], ref["dk"], ref["dg"],
+                                              ref["dbeta"])
+    assert rel_err(got["dg"], dg.sum(axis=-1)) < TOL[torch.float32]
+    for name, r in dict(dq=dq, dk=dk_, dv=ref["dv"], dbeta=db, dS0=ref["dS0"]).items():
+        assert rel_err(got[name], r) < TOL[torch.float32], (name, rel_err(got[name], r))
