@@ -1325,32 +1325,38 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
 }
 
 // ------------------------------------------------------------------ kernel 3 (bf16 operands)
+// Two CTAs of 8 warps per SM: the tiles stay under half of the SM's shared
+// memory by taking S0 and dS in halves of 64 key rows (the S0 half over the
+// v tile once v is dead), so one CTA's barriers and loads overlap the other's
+// products.
+constexpr int kLaThreads = 256;
 template <int DK, int DV>
 struct LocalAPlanB {  // bytes
-  static constexpr int LVb = DV + 8, LCb = kC + 8;
-  static constexpr size_t oO = 0, oVp = oO + (size_t)kC * LVb * 2, odV = oVp + (size_t)kC * LVb * 2,
-                          ov = odV + (size_t)kC * LVb * 2, oT = ov + (size_t)kC * LVb * 2,
-                          oS0 = oT + (size_t)kC * LCb * 2, odS = oS0 + (size_t)DK * LVb * 2,
-                          ob = odS + (size_t)DK * LVb * 2, ored = ob + kC * 4, bytes = ored + 4 * kC * 4;
+  static constexpr int LVb = DV + 8, LCb = kC + 8, HR = 64;  // HR: key rows per half of S0 / dS
+  static constexpr size_t tv = (size_t)kC * LVb * 2;
+  static constexpr size_t oO = 0, oVp = oO + tv, odV = oVp + tv, ov = odV + tv, oT = ov + tv,
+                          odS = oT + (size_t)kC * LCb * 2, ob = odS + (size_t)HR * LVb * 2, ored = ob + kC * 4,
+                          bytes = ored + 2 * kC * 4;
+  static_assert((size_t)HR * LVb * 2 <= tv, "an S0 half fits over the v tile");
 };
 
 // Per chunk, bf16 inputs: the products that contract over the value channels,
 // all operands bf16 images in shared memory (S0, dS, V', dV' and T come from
 // the state passes and the prep kernel as bf16).
 template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const ChunkBwdArgs a) {
+__global__ void __launch_bounds__(kLaThreads, 2) bwd_local_a_bf16_kernel(const ChunkBwdArgs a) {
   using PL = LocalAPlanB<DK, DV>;
-  constexpr int LVb = PL::LVb, LCb = PL::LCb;
+  constexpr int LVb = PL::LVb, LCb = PL::LCb, HR = PL::HR, NTH = kLaThreads, NW = NTH / 32;
   extern __shared__ __align__(16) uint8_t smb[];
   bf16* sO = reinterpret_cast<bf16*>(smb + PL::oO);    // [64][LVb] dO
   bf16* sVp = reinterpret_cast<bf16*>(smb + PL::oVp);  // [64][LVb] V'
   bf16* sdV = reinterpret_cast<bf16*>(smb + PL::odV);  // [64][LVb] dV'
-  bf16* sv = reinterpret_cast<bf16*>(smb + PL::ov);    // [64][LVb] v
+  bf16* sv = reinterpret_cast<bf16*>(smb + PL::ov);    // [64][LVb] v, then [HR][LVb] rows of S0
+  bf16* sS0 = sv;
   bf16* sT = reinterpret_cast<bf16*>(smb + PL::oT);    // [64][LCb] T
-  bf16* sS0 = reinterpret_cast<bf16*>(smb + PL::oS0);  // [DK][LVb] S0
-  bf16* sdS = reinterpret_cast<bf16*>(smb + PL::odS);  // [DK][LVb] dS
+  bf16* sdS = reinterpret_cast<bf16*>(smb + PL::odS);  // [HR][LVb] rows of dS
   float* sb = reinterpret_cast<float*>(smb + PL::ob);  // [64] beta
-  float* red = reinterpret_cast<float*>(smb + PL::ored);  // [4][64] row sums per column group
+  float* red = reinterpret_cast<float*>(smb + PL::ored);  // [2][64] row sums per column group
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
@@ -1362,7 +1368,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const Chu
   // rows of 16-byte pieces: [rows][width] bf16 from global (row i at src_row(i)) into [rows][ld]
   auto rows_in = [&](bf16* dst, int ld, int rows, int width, auto src_row, int valid) {
     const int per = width / 8;
-    for (int idx = tid; idx < rows * per; idx += kThreads) {
+    for (int idx = tid; idx < rows * per; idx += NTH) {
       const int i = idx / per, c = (idx % per) * 8;
       cp16(dst + i * ld + c, i < valid ? src_row(i) + c : src_row(0), i < valid ? 16 : 0);
     }
@@ -1373,21 +1379,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const Chu
   const bf16* dVp = reinterpret_cast<const bf16*>(a.dVp) + rec * kC * DV;
   const bf16* S0 = reinterpret_cast<const bf16*>(a.S0c) + rec * DK * DV;
   const bf16* dS = reinterpret_cast<const bf16*>(a.dSc) + rec * DK * DV;
+  const bf16* Tg = reinterpret_cast<const bf16*>(a.Tm) + rec * kC * kC;
   rows_in(sO, LVb, kC, DV, [&](int i) { return d_o + (row0 + (size_t)i * a.H) * DV; }, nv);
   rows_in(sv, LVb, kC, DV, [&](int i) { return vin + (row0 + (size_t)i * a.H) * DV; }, nv);
   rows_in(sVp, LVb, kC, DV, [&](int i) { return Vp + (size_t)i * DV; }, kC);
   rows_in(sdV, LVb, kC, DV, [&](int i) { return dVp + (size_t)i * DV; }, kC);
-  rows_in(sS0, LVb, DK, DV, [&](int i) { return S0 + (size_t)i * DV; }, DK);
-  rows_in(sdS, LVb, DK, DV, [&](int i) { return dS + (size_t)i * DV; }, DK);
+  rows_in(sT, LCb, kC, kC, [&](int i) { return Tg + (size_t)i * kC; }, kC);
+  rows_in(sdS, LVb, HR, DV, [&](int i) { return dS + (size_t)i * DV; }, HR);  // first half of dS
   if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const bf16*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
-  {
-    const bf16* Tg = reinterpret_cast<const bf16*>(a.Tm) + rec * kC * kC;
-    rows_in(sT, LCb, kC, kC, [&](int i) { return Tg + (size_t)i * kC; }, kC);
-  }
   cp_wait();
   __syncthreads();
   {
-    using Tl = Tiling<kC, kC>;
+    using Tl = Tiling<kC, kC, NW>;
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);  // dAqk = tril(dO V'^T)
@@ -1404,7 +1407,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const Chu
     });
   }
   {  // X = T^T dU: dv = beta X, dbeta part = rowsum(V . X)
-    using Tl = Tiling<kC, DV>;
+    using Tl = Tiling<kC, DV, NW>;
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4], rp[Tl::MT][2] = {};
     zero(acc);
@@ -1417,39 +1420,46 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_bf16_kernel(const Chu
     });
     row_sums_out<Tl::MT>(rp, m0, red + (warp / Tl::WM) * kC);
   }
-  {  // dO S0^T, -dV' S0^T, V' dS^T (64 x DK, contracting the value channels)
-    using Tl = Tiling<kC, DK>;
-    const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
-    float acc[Tl::MT][Tl::NT][4];
+  // dO S0^T, -dV' S0^T, V' dS^T (64 x DK, contracting the value channels) and
+  // rowsum(dS . S0), by halves of HR key rows
+  using Th = Tiling<kC, HR, NW>;
+  const int hm0 = Th::m0(warp), hn0 = Th::n0(warp);
+  for (int half = 0; half < DK / HR; ++half) {
+    __syncthreads();  // v (or the previous halves) no longer read
+    rows_in(sS0, LVb, HR, DV, [&](int i) { return S0 + (size_t)(half * HR + i) * DV; }, HR);
+    if (half > 0) rows_in(sdS, LVb, HR, DV, [&](int i) { return dS + (size_t)(half * HR + i) * DV; }, HR);
+    cp_wait();
+    __syncthreads();
+    float acc[Th::MT][Th::NT][4];
     zero(acc);
-    warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sO, LVb, sS0, LVb, m0, n0);
-    float* out = a.dQs + rec * kC * DK;
-    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
+    warp_mma_bf16<Th::MT, Th::NT, DV, false, true>(acc, sO, LVb, sS0, LVb, hm0, hn0);
+    float* out = a.dQs + rec * kC * DK + half * HR;
+    for_acc<Th::MT, Th::NT>(hm0, hn0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
     zero(acc);
-    warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sdV, LVb, sS0, LVb, m0, n0);
-    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { acc[mt][nt][e] = -acc[mt][nt][e]; });
-    acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dW) + rec * kC * DK, DK, m0, n0);  // an operand only: bf16
+    warp_mma_bf16<Th::MT, Th::NT, DV, false, true>(acc, sdV, LVb, sS0, LVb, hm0, hn0);
+    for_acc<Th::MT, Th::NT>(hm0, hn0, [&](int mt, int nt, int e, int i, int c) { acc[mt][nt][e] = -acc[mt][nt][e]; });
+    acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dW) + rec * kC * DK + half * HR, DK, hm0, hn0);  // operand only
     zero(acc);
-    warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sVp, LVb, sdS, LVb, m0, n0);
-    out = a.dKb + rec * kC * DK;
-    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
-  }
-  for (int r = warp; r < DK; r += kWarps) {  // rowsum(dS . S0), two columns per load
-    float x = 0.f;
-    for (int c = 2 * lane; c < DV; c += 64) {
-      const float2 d = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sdS + r * LVb + c));
-      const float2 s0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sS0 + r * LVb + c));
-      x = fmaf(d.x, s0.x, fmaf(d.y, s0.y, x));
-    }
+    warp_mma_bf16<Th::MT, Th::NT, DV, false, true>(acc, sVp, LVb, sdS, LVb, hm0, hn0);
+    out = a.dKb + rec * kC * DK + half * HR;
+    for_acc<Th::MT, Th::NT>(hm0, hn0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
+    for (int r = warp; r < HR; r += NW) {  // rowsum(dS . S0), two columns per load
+      float x = 0.f;
+      for (int c = 2 * lane; c < DV; c += 64) {
+        const float2 d = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sdS + r * LVb + c));
+        const float2 s0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sS0 + r * LVb + c));
+        x = fmaf(d.x, s0.x, fmaf(d.y, s0.y, x));
+      }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-    if (lane == 0) a.dgam[rec * DK + r] = x;
+      for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+      if (lane == 0) a.dgam[rec * DK + half * HR + r] = x;
+    }
   }
   __syncthreads();
   if (tid < kC) {
     float x = 0.f;
 #pragma unroll
-    for (int w = 0; w < Tiling<kC, DV>::WN; ++w) x += red[w * kC + tid];
+    for (int w = 0; w < Tiling<kC, DV, NW>::WN; ++w) x += red[w * kC + tid];
     a.dbu[rec * kC + tid] = x;
   }
 }
@@ -2054,7 +2064,7 @@ cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t strea
   if constexpr (std::is_same<IO, float>::value)
     e = launch_k(bwd_local_a_kernel<IO, DK, DV>, grid, local_a_smem<DK, DV>(), a, stream);
   else
-    e = launch_k(bwd_local_a_bf16_kernel<DK, DV>, grid, LocalAPlanB<DK, DV>::bytes, a, stream);
+    e = launch_k(bwd_local_a_bf16_kernel<DK, DV>, grid, LocalAPlanB<DK, DV>::bytes, a, stream, kLaThreads);
   if (e != cudaSuccess) return e;
   if constexpr (std::is_same<IO, float>::value)
     return launch_k(bwd_local_b_kernel<IO, DK, DV>, grid, local_b_smem<DK, DV>(), a, stream);
