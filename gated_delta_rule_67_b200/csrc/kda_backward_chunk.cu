@@ -60,6 +60,15 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kPassThreads = 256;  // 8 warps in the state passes (longer tiles, fewer loads per MMA)
 constexpr int kLC = kC + 4;     // leading dimension of the C x C shared tiles
 
+// ------------------------------------------------------------------ launch chaining
+// The four kernels of a call are chained by programmatic dependent launch:
+// each kernel lets the next one be scheduled as soon as all of its CTAs have
+// started (so the next grid's CTAs fill the SMs its last wave frees), and the
+// next one waits for the whole previous grid, memory included, before its
+// first access.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ warp MMA
 __device__ __forceinline__ uint32_t tf32_rna(float x) {
   uint32_t r;
@@ -415,6 +424,7 @@ constexpr size_t prep_smem() {
 // operands below): G, the factored and absolute operands, P and Aqk, T, W and U.
 template <typename IO, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArgs a) {
+  pdl_trigger();
   constexpr bool X3 = std::is_same<IO, float>::value;
   constexpr int LK = DK + 4, LM = (DK > DV ? DK : DV) + 4;
   extern __shared__ __align__(16) float sm[];
@@ -620,6 +630,8 @@ __device__ __forceinline__ void load_state_t(float* sT, int ld, const float* g, 
 // stores dL/d(state leaving the chunk) and dV', and writes dL/dS_0.
 template <typename IO, int DK, int DV, int SW>
 __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_kernel(const ChunkBwdArgs a) {
+  pdl_wait();  // the previous kernel of the call has finished
+  pdl_trigger();
   constexpr bool X3 = std::is_same<IO, float>::value;
   using PP = PassPlan<DK, DV, SW>;
   constexpr int LK = PP::LK, LS = PP::LS, NS = DV / SW;
@@ -906,6 +918,8 @@ constexpr size_t pass_bf16_smem() {
 
 template <int DK, int DV, int SW>
 __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const ChunkBwdArgs a) {
+  pdl_wait();  // the previous kernel of the call has finished
+  pdl_trigger();
   using PB = PassPlanB<DK, DV, SW>;
   using R = PassRec<DK>;
   constexpr int LS = PB::LS, NS = DV / SW, NTH = kPassThreads;
@@ -1047,6 +1061,8 @@ constexpr size_t local_a_smem() {
 // Per chunk: the products that contract over the value channels.
 template <typename IO, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) bwd_local_a_kernel(const ChunkBwdArgs a) {
+  pdl_wait();  // the previous kernel of the call has finished
+  pdl_trigger();
   constexpr bool X3 = std::is_same<IO, float>::value;
   constexpr int LV = DV + 4;
   extern __shared__ __align__(16) float sm[];
@@ -1166,6 +1182,7 @@ struct PrepPlanB {  // bytes
 // the state passes' operands go out as the chunk's bf16 pass record, T as bf16.
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkBwdArgs a) {
+  pdl_trigger();
   using PL = PrepPlanB<DK, DV>;
   using PR = PassRec<DK>;
   constexpr int LK = PL::LK, LKb = PL::LKb, LVb = PL::LVb, LMb = PL::LMb, LCb = PL::LCb;
@@ -1345,6 +1362,8 @@ struct LocalAPlanB {  // bytes
 // the state passes and the prep kernel as bf16).
 template <int DK, int DV>
 __global__ void __launch_bounds__(kLaThreads, 2) bwd_local_a_bf16_kernel(const ChunkBwdArgs a) {
+  pdl_wait();  // the previous kernel of the call has finished
+  pdl_trigger();
   using PL = LocalAPlanB<DK, DV>;
   constexpr int LVb = PL::LVb, LCb = PL::LCb, HR = PL::HR, NTH = kLaThreads, NW = NTH / 32;
   extern __shared__ __align__(16) uint8_t smb[];
@@ -1474,6 +1493,8 @@ constexpr size_t local_b_smem() {
 // Per chunk: dT, dA, the pairwise gradients and the fold into dq, dk, dg, dbeta.
 template <typename IO, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwdArgs a) {
+  pdl_wait();  // the previous kernel of the call has finished
+  pdl_trigger();
   constexpr bool X3 = std::is_same<IO, float>::value;
   constexpr int LK = DK + 4;
   using TK = Tiling<kC, DK>;  // every 64 x d_k product: the same tile per warp
@@ -1724,6 +1745,8 @@ struct LocalBPlanB {  // bytes
 // intrinsic (exponents bounded by the factored form's span, or <= 0).
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const ChunkBwdArgs a) {
+  pdl_wait();  // the previous kernel of the call has finished
+  pdl_trigger();
   using PL = LocalBPlanB<DK, DV>;
   constexpr int LK = PL::LK, LKb = PL::LKb, LCb = PL::LCb;
   using TK = Tiling<kC, DK>;  // every 64 x d_k product: the same tile per warp
@@ -2028,21 +2051,33 @@ struct WsPlan {
 // in one wave of the 148 SMs, else 64 (fewer CTAs reading the same operands).
 int pass_width(int BH, int dv) { return (size_t)2 * BH * (dv / 32) <= 148 ? 32 : 64; }
 
+// The first kernel of a call launches plainly (it follows arbitrary work on
+// the stream); the others as programmatic dependents of the one before.
 template <typename Kern>
 cudaError_t launch_k(Kern kern, dim3 grid, size_t smem, const ChunkBwdArgs& a, cudaStream_t stream,
-                     int nth = kThreads) {
+                     int nth = kThreads, bool dependent = true) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, nth, smem, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(nth);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 template <typename IO, int DK, int DV>
 cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t stream) {
   const dim3 grid((unsigned)a.NC * BH);  // chunk-major within each (sequence, head)
-  cudaError_t e = std::is_same<IO, float>::value
-                      ? launch_k(bwd_prep_kernel<float, DK, DV>, grid, prep_smem<DK, DV>(), a, stream)
-                      : launch_k(bwd_prep_bf16_kernel<DK, DV>, grid, PrepPlanB<DK, DV>::bytes, a, stream);
+  cudaError_t e =
+      std::is_same<IO, float>::value
+          ? launch_k(bwd_prep_kernel<float, DK, DV>, grid, prep_smem<DK, DV>(), a, stream, kThreads, false)
+          : launch_k(bwd_prep_bf16_kernel<DK, DV>, grid, PrepPlanB<DK, DV>::bytes, a, stream, kThreads, false);
   if (e != cudaSuccess) return e;
   const bool w32 = pass_width(BH, DV) == 32;
   if constexpr (std::is_same<IO, float>::value) {
