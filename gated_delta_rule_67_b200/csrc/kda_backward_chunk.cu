@@ -26,7 +26,9 @@
 // for differentiation.  A chunk whose cumulative gates leave +-kSpan of the
 // reference takes an exact per-element path instead (exp of each difference).
 //
-// Four launches:
+// Four launches per group of (sequence, head) pairs (as many as the workspace
+// holds), the last three chained to the one before by programmatic dependent
+// launch:
 //   1. bwd_prep    (chunk, seq x head): W, U, Q+, Kbar, Aqk, P, T, gamma per chunk
 //   2. bwd_pass    (seq x head x column slice, 2 roles): the forward state
 //      replay (checkpoints S0 and V' per chunk) and the reverse dS sweep
