@@ -1,6 +1,7 @@
-"""The prefill and decode calls inside CUDA graphs: captured once, replayed
-on new inputs copied into the captured buffers, bit-identical to eager calls
-(the prefill chains its kernels with programmatic dependent launch)."""
+"""The prefill, decode and backward calls inside CUDA graphs: captured once,
+replayed on new inputs copied into the captured buffers, bit-identical to
+eager calls (the prefill and the backward chain their kernels with
+programmatic dependent launch)."""
 import pytest
 import torch
 
@@ -63,3 +64,49 @@ def test_decode_graph_of_steps():
     graph.replay()                         # steps 8-15
     torch.cuda.synchronize()
     assert torch.equal(st, st_eager)
+
+
+@pytest.mark.parametrize("dtype,prep", [(torch.bfloat16, 0), (torch.float32, 0), (torch.bfloat16, 7)],
+                         ids=["bf16", "f32", "bf16-prep"])
+def test_backward_graph_replay_matches_eager(dtype, prep):
+    """kda_backward captured once (its four kernels chained by programmatic
+    dependent launch; with preparation bits, six), replayed on new inputs:
+    every gradient bit-identical to an eager call."""
+    from gated_delta_rule_67_b200 import kda_backward
+    from gated_delta_rule_67_b200.binding import load
+    from gated_delta_rule_67_b200.workloads import make_cotangents
+    dev = cuda_or_skip()
+    B, T, H = 1, 300, 4
+    xs = []
+    for s in (123, 124):
+        x = make_prefill_inputs(B, T, H, 128, 128, dtype, 0.1, seed=s, device=dev)
+        x["d_o"], x["d_s"] = make_cotangents(B, T, H, 128, 128, dtype, seed=s + 10, device=dev)
+        xs.append(x)
+    keys = NAMES + ("d_o", "initial_state", "d_s")
+    buf = {n: xs[0][n].clone() for n in keys}
+    code = 1 if dtype == torch.bfloat16 else 0
+    ws = torch.empty(int(load().kda_backward_ex_workspace_size(B, T, H, 128, 128, code, prep)), dtype=torch.uint8,
+                     device=dev)
+
+    def call(src):
+        return kda_backward(*(src[n] for n in NAMES), src["d_o"], None, src["initial_state"], src["d_s"],
+                            workspace=ws, prep=prep)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):  # warm-up (library setup) outside the capture
+        call(buf)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        out = call(buf)
+    for x in xs:
+        for n in keys:
+            buf[n].copy_(x[n])
+        graph.replay()
+        torch.cuda.synchronize()
+        got = {n: t.clone() for n, t in out.items()}
+        ref = call(x)
+        torch.cuda.synchronize()
+        for n in ref:
+            assert torch.equal(got[n], ref[n]), n
