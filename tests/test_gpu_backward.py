@@ -215,3 +215,9 @@ def test_backward_through_preparation_head_gate():
     assert rel_err(got["dg"], dg.sum(axis=-1)) < TOL[torch.float32]
     for name, r in dict(dq=dq, dk=dk_, dv=ref["dv"], dbeta=db, dS0=ref["dS0"]).items():
         assert rel_err(got[name], r) < TOL[torch.float32], (name, rel_err(got[name], r))
+
+
+def test_backward_long_chain():
+    """One (sequence, head) over 65,536 tokens (1,024 chunks, bf16): the state
+    passes carry the state and its gradient through the whole chain."""
+    _case(1, 65536, 1, 128, 128, torch.bfloat16, seed=111)
