@@ -415,6 +415,56 @@ struct PassRec {  // element offsets of the bf16 pass record of one chunk
   static_assert(oKb % 8 == 0 && oQpt % 8 == 0 && oWt % 8 == 0 && n1 % 8 == 0 && oKbt % 8 == 0 && n % 8 == 0, "16 B");
 };
 
+// T = (I + diag(beta) P)^-1 for a strictly lower 64 x 64 P (fp32, leading
+// dimension kLC) by 16 x 16 blocks, on the 128 threads of warps 0-3 (named
+// barrier 1): the diagonal blocks by forward substitution (one thread per
+// block column, the column in registers), then the blocks below the diagonal
+// level by level, T_IJ = -T_II (sum_{K=J..I-1} A_IK T_KJ) with A = diag(beta) P.
+// T (fp32, leading dimension kLC) is unit lower triangular with zeros above;
+// X is a 3 x 16 x 16 fp32 scratch.
+__device__ __forceinline__ void bar128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void solve_T_blocked(const float* sP, const float* sb, float* T, float* X, int t) {
+  if (t < kC) {  // diagonal block I = t / 16, column jj = t % 16
+    const int I = t >> 4, jj = t & 15, r0 = 16 * I;
+    float tc[16];
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) {
+      float s = 0.f;
+#pragma unroll
+      for (int m = 0; m < ii; ++m) s = fmaf(sP[(r0 + ii) * kLC + r0 + m], tc[m], s);
+      tc[ii] = ii == jj ? 1.f : (ii < jj ? 0.f : -sb[r0 + ii] * s);
+      T[(r0 + ii) * kLC + r0 + jj] = tc[ii];
+    }
+  } else {  // the six blocks above the diagonal are zero
+    for (int e = t - kC; e < 6 * 256; e += 128 - kC) {
+      const int blk = e >> 8, a = (e >> 4) & 15, b = e & 15;
+      const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2), J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+      T[(16 * I + a) * kLC + 16 * J + b] = 0.f;
+    }
+  }
+  bar128();
+  for (int d = 1; d < 4; ++d) {
+    const int nb = 4 - d;  // blocks (I, J = I - d), J = 0 .. nb-1
+    for (int e = t; e < nb * 256; e += 128) {
+      const int J = e >> 8, I = J + d, a = (e >> 4) & 15, b = e & 15;
+      float s = 0.f;
+      for (int K = J; K < I; ++K)
+#pragma unroll
+        for (int m = 0; m < 16; ++m) s = fmaf(sP[(16 * I + a) * kLC + 16 * K + m], T[(16 * K + m) * kLC + 16 * J + b], s);
+      X[e] = sb[16 * I + a] * s;
+    }
+    bar128();
+    for (int e = t; e < nb * 256; e += 128) {
+      const int J = e >> 8, I = J + d, a = (e >> 4) & 15, b = e & 15;
+      float s = 0.f;
+#pragma unroll
+      for (int m = 0; m < 16; ++m) s = fmaf(T[(16 * I + a) * kLC + 16 * I + m], X[J * 256 + m * 16 + b], s);
+      T[(16 * I + a) * kLC + 16 * J + b] = -s;
+    }
+    bar128();
+  }
+}
+
 // ------------------------------------------------------------------ kernel 1
 template <int DK, int DV>
 constexpr size_t prep_smem() {
@@ -1171,9 +1221,10 @@ struct PrepPlanB {  // bytes
                           ov = oq + (size_t)kC * LKb * 2, oX = ov + (size_t)kC * LVb * 2,
                           oY = oX + (size_t)kC * LKb * 2, oQ = oY + (size_t)kC * LMb * 2,
                           oP = oQ + (size_t)kC * LKb * 2, oT = oP + (size_t)kC * kLC * 4,
-                          ob = oT + (size_t)kC * LCb * 2, oe = ob + kC * 4, bytes = oe + DK * 4;
+                          oTf = oT + (size_t)kC * LCb * 2, oXs = oTf + (size_t)kC * kLC * 4,
+                          ob = oXs + 3 * 256 * 4, oe = ob + kC * 4, bytes = oe + DK * 4;
   static_assert(ok % 16 == 0 && oq % 16 == 0 && ov % 16 == 0 && oX % 16 == 0 && oY % 16 == 0 && oQ % 16 == 0 &&
-                    oP % 16 == 0 && oT % 16 == 0 && ob % 16 == 0,
+                    oP % 16 == 0 && oT % 16 == 0 && oTf % 16 == 0 && oXs % 16 == 0 && ob % 16 == 0,
                 "16 B");
 };
 
@@ -1198,6 +1249,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   bf16* sQ = reinterpret_cast<bf16*>(smb + PL::oQ);    // [64][LKb] Q+_r
   float* sP = reinterpret_cast<float*>(smb + PL::oP);  // [64][kLC] P
   bf16* sT = reinterpret_cast<bf16*>(smb + PL::oT);    // [64][LCb] T
+  float* sTf = reinterpret_cast<float*>(smb + PL::oTf);  // [64][kLC] T (fp32)
+  float* sXs = reinterpret_cast<float*>(smb + PL::oXs);  // [3][16][16] solve scratch
   float* sb = reinterpret_cast<float*>(smb + PL::ob);  // [64] beta
   float* se = reinterpret_cast<float*>(smb + PL::oe);  // [DK] exp(G_ref)
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -1274,32 +1327,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   }
   __syncthreads();
 
-  // Warps 0-1: T = (I + diag(beta) P)^-1, thread j < 64 keeping column j in
-  // registers (see the fp32 kernel).  The other warps meanwhile store P, the
-  // record's Q+^T and Kbar^T, and the right operands beta K+ and beta v of W
-  // and U (the factored tiles are dead).
+  // Warps 0-3: T = (I + diag(beta) P)^-1 by blocks (fp32), then its bf16 image
+  // and the global copy.  The other warps meanwhile store P, the record's
+  // Q+^T and Kbar^T, and the right operands beta K+ and beta v of W and U
+  // (the factored tiles are dead).
   bf16* Tg = reinterpret_cast<bf16*>(a.Tm) + rec * kC * kC;
-  if (tid < kC) {
-    const int j = tid;
-    float tc[kC];
-#pragma unroll
-    for (int i = 0; i < kC; ++i) {
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int m = 0; m < i; m += 4) {
-        const float4 p = *reinterpret_cast<const float4*>(sP + i * kLC + m);
-        s4[0] = fmaf(p.x, tc[m], s4[0]);
-        if (m + 1 < i) s4[1] = fmaf(p.y, tc[m + 1], s4[1]);
-        if (m + 2 < i) s4[2] = fmaf(p.z, tc[m + 2], s4[2]);
-        if (m + 3 < i) s4[3] = fmaf(p.w, tc[m + 3], s4[3]);
-      }
-      tc[i] = i == j ? 1.f : (i < j ? 0.f : -sb[i] * ((s4[0] + s4[1]) + (s4[2] + s4[3])));
-      const bf16 tb = __float2bfloat16_rn(tc[i]);
-      sT[i * LCb + j] = tb;
-      Tg[i * kC + j] = tb;
+  if (tid < 128) {
+    solve_T_blocked(sP, sb, sTf, sXs, tid);
+    for (int idx = tid; idx < kC * kC / 2; idx += 128) {
+      const int i = idx / (kC / 2), j = (idx % (kC / 2)) * 2;
+      const __nv_bfloat162 t2 = __floats2bfloat162_rn(sTf[i * kLC + j], sTf[i * kLC + j + 1]);
+      *reinterpret_cast<__nv_bfloat162*>(sT + i * LCb + j) = t2;
+      *reinterpret_cast<__nv_bfloat162*>(Tg + i * kC + j) = t2;
     }
   } else {
-    const int t2 = tid - kC, n2 = kThreads - kC;
+    const int t2 = tid - 128, n2 = kThreads - 128;
     float* Pg = a.Pkk + rec * kC * kC;
     for (int idx = t2; idx < kC * kC / 4; idx += n2) {
       const int i = idx / (kC / 4), j = (idx % (kC / 4)) * 4;
