@@ -398,21 +398,18 @@ __device__ __forceinline__ size_t row_of(const ChunkBwdArgs& a, int bh, int t0) 
 
 // Element offsets of the bf16 pass record of one chunk (bf16 inputs): the
 // state passes' operands in their shared-memory layout, rows padded by 16
-// bytes.  Part 1 (Aqk^T, Kbar, Q+^T, W^T) feeds the reverse sweep, part 0
-// (W, Kbar^T) the forward replay.
+// bytes.  The passes read the operands they need transposed (Aqk^T, Q+^T,
+// W^T, Kbar^T) with ldmatrix.trans, so each is stored once, row-major.
 using bf16 = __nv_bfloat16;
 template <int DK>
-struct PassRec {  // element offsets of the bf16 pass record of one chunk
+struct PassRec {  // element offsets of the bf16 pass record of one chunk (all row-major)
   static constexpr int LKb = DK + 8, LCb = kC + 8;
-  static constexpr int oAqkt = 0;                 // [64][LCb]  Aqk^T      (reverse sweep)
-  static constexpr int oKb = oAqkt + kC * LCb;    // [64][LKb]  Kbar
-  static constexpr int oQpt = oKb + kC * LKb;     // [DK][LCb]  Q+^T
-  static constexpr int oWt = oQpt + DK * LCb;     // [DK][LCb]  W^T
-  static constexpr int n1 = oWt + DK * LCb;       // end of the reverse sweep's part
-  static constexpr int oW = n1;                   // [64][LKb]  W          (forward replay)
-  static constexpr int oKbt = oW + kC * LKb;      // [DK][LCb]  Kbar^T
-  static constexpr int n = oKbt + DK * LCb;
-  static_assert(oKb % 8 == 0 && oQpt % 8 == 0 && oWt % 8 == 0 && n1 % 8 == 0 && oKbt % 8 == 0 && n % 8 == 0, "16 B");
+  static constexpr int oAqk = 0;                 // [64][LCb]  Aqk        (reverse sweep, read transposed)
+  static constexpr int oQp = oAqk + kC * LCb;    // [64][LKb]  Q+         (reverse sweep, read transposed)
+  static constexpr int oW = oQp + kC * LKb;      // [64][LKb]  W          (both; transposed in the reverse sweep)
+  static constexpr int oKb = oW + kC * LKb;      // [64][LKb]  Kbar       (both; transposed in the forward replay)
+  static constexpr int n = oKb + kC * LKb;       // the reverse sweep reads [0, n), the forward replay [oW, n)
+  static_assert(oQp % 8 == 0 && oW % 8 == 0 && oKb % 8 == 0 && n % 8 == 0, "16 B");
 };
 
 // T = (I + diag(beta) P)^-1 for a strictly lower 64 x 64 P (fp32, leading
@@ -958,8 +955,8 @@ struct PassPlanB {  // bytes
   using R = PassRec<DK>;
   static constexpr int LS = SW + 8;  // bf16 images of the state / V' / dV' / dO columns
   static constexpr size_t img = (size_t)(DK + kC) * LS * 2;
-  static constexpr size_t buf0 = (size_t)(R::n - R::n1) * 2 + DK * 4 + (size_t)kC * SW * 4;  // W, Kbar^T, gamma, U
-  static constexpr size_t buf1 = (size_t)R::n1 * 2 + DK * 4 + (size_t)kC * LS * 2;          // part 1, gamma, dO
+  static constexpr size_t buf0 = (size_t)(R::n - R::oW) * 2 + DK * 4 + (size_t)kC * SW * 4;  // W, Kbar, gamma, U
+  static constexpr size_t buf1 = (size_t)R::n * 2 + DK * 4 + (size_t)kC * LS * 2;            // record, gamma, dO
   static constexpr size_t bytes = img + 2 * (buf0 > buf1 ? buf0 : buf1);
   static_assert(img % 16 == 0 && buf0 % 16 == 0 && buf1 % 16 == 0, "16 B");
 };
@@ -1002,16 +999,16 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
   });
 
   if (blockIdx.y == 0) {
-    // buffer: W [64][LKb], Kbar^T [DK][LCb] (bf16), gamma [DK], U columns [64][SW] (fp32)
+    // buffer: W, Kbar [64][LKb] (bf16), gamma [DK], U columns [64][SW] (fp32)
     auto bW = [&](int p) { return reinterpret_cast<const bf16*>(bufs + p * BUF); };
-    auto bKbt = [&](int p) { return bW(p) + (R::oKbt - R::oW); };
-    auto bgm = [&](int p) { return reinterpret_cast<const float*>(bufs + p * BUF + (R::n - R::n1) * 2); };
+    auto bKb = [&](int p) { return bW(p) + (R::oKb - R::oW); };
+    auto bgm = [&](int p) { return reinterpret_cast<const float*>(bufs + p * BUF + (R::n - R::oW) * 2); };
     auto bU = [&](int p) { return bgm(p) + DK; };
     auto issue = [&](int n, int p) {
       const size_t rec = (size_t)lb * NC + n;
       uint8_t* b = bufs + p * BUF;
-      copy(b, a.prec + rec * R::n + R::n1, (size_t)(R::n - R::n1) * 2);
-      copy(b + (R::n - R::n1) * 2, a.gam + rec * DK, DK * 4);
+      copy(b, a.prec + rec * R::n + R::oW, (size_t)(R::n - R::oW) * 2);
+      copy(b + (R::n - R::oW) * 2, a.gam + rec * DK, DK * 4);
       float* u = const_cast<float*>(bU(p));
       const float* ug = a.U + rec * kC * DV + c0;
       for (int idx = tid; idx < kC * (SW / 4); idx += NTH) {
@@ -1043,20 +1040,20 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
       {  // S = diag(gamma) S + Kbar^T V'
         const float* gm = bgm(p);
         for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) { st[mt][nt][e] *= gm[r]; });
-        warp_mma_bf16<TS::MT, TS::NT, kC>(st, bKbt(p), R::LCb, vimg, LS, sm0, sn0);
+        warp_mma_bf16<TS::MT, TS::NT, kC, true>(st, bKb(p), R::LKb, vimg, LS, sm0, sn0);
       }
     }
   } else {
-    // buffer: record part 1 (Aqk^T, Kbar, Q+^T, W^T; bf16), gamma [DK], dO columns [64][LS] (bf16)
+    // buffer: the record (Aqk, Q+, W, Kbar; bf16), gamma [DK], dO columns [64][LS] (bf16)
     auto bR = [&](int p) { return reinterpret_cast<const bf16*>(bufs + p * BUF); };
-    auto bgm = [&](int p) { return reinterpret_cast<const float*>(bufs + p * BUF + R::n1 * 2); };
-    auto bO = [&](int p) { return reinterpret_cast<const bf16*>(bufs + p * BUF + R::n1 * 2 + DK * 4); };
+    auto bgm = [&](int p) { return reinterpret_cast<const float*>(bufs + p * BUF + R::n * 2); };
+    auto bO = [&](int p) { return reinterpret_cast<const bf16*>(bufs + p * BUF + R::n * 2 + DK * 4); };
     const bf16* d_o = static_cast<const bf16*>(a.d_o);
     auto issue = [&](int n, int p) {
       const size_t rec = (size_t)lb * NC + n;
       uint8_t* b = bufs + p * BUF;
-      copy(b, a.prec + rec * R::n, (size_t)R::n1 * 2);
-      copy(b + R::n1 * 2, a.gam + rec * DK, DK * 4);
+      copy(b, a.prec + rec * R::n, (size_t)R::n * 2);
+      copy(b + R::n * 2, a.gam + rec * DK, DK * 4);
       constexpr int PER = SW / 8;  // 16-byte pieces per row
       const int t0 = n * kC, nv = min(kC, a.T - t0);
       const size_t r0 = row_of(a, bh, t0);
@@ -1080,7 +1077,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
       {  // dV' = Aqk^T dO + Kbar dS
         float acc[TV::MT][TV::NT][4];
         zero(acc);
-        warp_mma_bf16<TV::MT, TV::NT, kC>(acc, rp + R::oAqkt, R::LCb, bO(p), LS, vm0, vn0);
+        warp_mma_bf16<TV::MT, TV::NT, kC, true>(acc, rp + R::oAqk, R::LCb, bO(p), LS, vm0, vn0);
         warp_mma_bf16<TV::MT, TV::NT, DK>(acc, rp + R::oKb, R::LKb, simg, LS, vm0, vn0);
         acc_to_bf16(acc, vimg, LS, vm0, vn0);
         acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dVp) + rec * kC * DV + c0, DV, vm0, vn0);
@@ -1090,9 +1087,9 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
         const float* gm = bgm(p);
         float neg[TS::MT][TS::NT][4];
         for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) { st[mt][nt][e] *= gm[r]; });
-        warp_mma_bf16<TS::MT, TS::NT, kC>(st, rp + R::oQpt, R::LCb, bO(p), LS, sm0, sn0);
+        warp_mma_bf16<TS::MT, TS::NT, kC, true>(st, rp + R::oQp, R::LKb, bO(p), LS, sm0, sn0);
         zero(neg);
-        warp_mma_bf16<TS::MT, TS::NT, kC>(neg, rp + R::oWt, R::LCb, vimg, LS, sm0, sn0);
+        warp_mma_bf16<TS::MT, TS::NT, kC, true>(neg, rp + R::oW, R::LKb, vimg, LS, sm0, sn0);
         for_acc<TS::MT, TS::NT>(sm0, sn0, [&](int mt, int nt, int e, int r, int c) { st[mt][nt][e] -= neg[mt][nt][e]; });
       }
     }
@@ -1281,11 +1278,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   }
   cp_wait();
   __syncthreads();
-  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Kbar (record) and the factored operands
+  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+, Kbar (record) and the factored operands
     const int i = idx / DK, r = idx % DK;
     const float G = sG[i * LK + r], kk = __bfloat162float(sk[i * LKb + r]);
     const float qq = a.scale * __bfloat162float(sq[i * LKb + r]);
     pr[PR::oKb + i * PR::LKb + r] = __float2bfloat16_rn(kk * __expf(sG[(kC - 1) * LK + r] - G));
+    pr[PR::oQp + i * PR::LKb + r] = __float2bfloat16_rn(qq * __expf(G));
     if (!slow) {
       const float d = G - sG[kRef * LK + r], ex = __expf(d);
       sX[i * LKb + r] = __float2bfloat16_rn(kk * ex);
@@ -1308,7 +1306,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
     zero(acc);
     warp_mma_bf16<Tl::MT, Tl::NT, DK, false, true>(acc, sQ, LKb, sY, LMb, m0, n0);
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
-      pr[PR::oAqkt + j * PR::LCb + i] = __float2bfloat16_rn(j <= i ? acc[mt][nt][e] : 0.f);
+      pr[PR::oAqk + i * PR::LCb + j] = __float2bfloat16_rn(j <= i ? acc[mt][nt][e] : 0.f);
     });
   } else {
     for (int idx = tid; idx < kC * kC; idx += kThreads) {
@@ -1322,15 +1320,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
         }
       }
       sP[i * kLC + j] = j < i ? p : 0.f;
-      pr[PR::oAqkt + j * PR::LCb + i] = __float2bfloat16_rn(j <= i ? a.scale * s : 0.f);
+      pr[PR::oAqk + i * PR::LCb + j] = __float2bfloat16_rn(j <= i ? a.scale * s : 0.f);
     }
   }
   __syncthreads();
 
   // Warps 0-3: T = (I + diag(beta) P)^-1 by blocks (fp32), then its bf16 image
-  // and the global copy.  The other warps meanwhile store P, the record's
-  // Q+^T and Kbar^T, and the right operands beta K+ and beta v of W and U
-  // (the factored tiles are dead).
+  // and the global copy.  The other warps meanwhile store P and the right
+  // operands beta K+ and beta v of W and U (the factored tiles are dead).
   bf16* Tg = reinterpret_cast<bf16*>(a.Tm) + rec * kC * kC;
   if (tid < 128) {
     solve_T_blocked(sP, sb, sTf, sXs, tid);
@@ -1347,13 +1344,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
       const int i = idx / (kC / 4), j = (idx % (kC / 4)) * 4;
       *reinterpret_cast<float4*>(Pg + i * kC + j) = *reinterpret_cast<const float4*>(sP + i * kLC + j);
     }
-    for (int idx = t2; idx < kC * DK; idx += n2) {  // Q+^T, Kbar^T (record), token index fastest
-      const int r = idx / kC, i = idx % kC;
-      const float G = sG[i * LK + r];
-      pr[PR::oQpt + r * PR::LCb + i] = __float2bfloat16_rn(a.scale * __bfloat162float(sq[i * LKb + r]) * __expf(G));
-      pr[PR::oKbt + r * PR::LCb + i] =
-          __float2bfloat16_rn(__bfloat162float(sk[i * LKb + r]) * __expf(sG[(kC - 1) * LK + r] - G));
-    }
     for (int idx = t2; idx < kC * DK; idx += n2) {
       const int i = idx / DK, r = idx % DK;
       sX[i * LKb + r] = __float2bfloat16_rn(sb[i] * __bfloat162float(sk[i * LKb + r]) * __expf(sG[i * LK + r]));
@@ -1364,16 +1354,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
     }
   }
   __syncthreads();
-  {  // W = T (beta K+): record W and W^T
+  {  // W = T (beta K+): record
     using Tl = Tiling<kC, DK>;
     const int m0 = Tl::m0(warp), n0 = Tl::n0(warp);
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);
     warp_mma_bf16<Tl::MT, Tl::NT, kC, false, false>(acc, sT, LCb, sX, LKb, m0, n0);
     acc_to_bf16(acc, pr + PR::oW, PR::LKb, m0, n0);
-    for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int c) {
-      pr[PR::oWt + c * PR::LCb + i] = __float2bfloat16_rn(acc[mt][nt][e]);
-    });
   }
   {  // U = T (beta v), fp32
     using Tl = Tiling<kC, DV>;
