@@ -332,9 +332,11 @@ __device__ __forceinline__ void store_f32(float* dst, int gld, const float* src,
 
 // Per-channel log-gates of one chunk into sG [64][ld] (zeros past nv): per
 // channel, per head (broadcast over the channels) or none; then the inclusive
-// cumsum over the tokens, in place.
+// cumsum over the tokens, in place (one thread per channel, the column in
+// registers).  Returns (block-uniform) whether the chunk needs the exact
+// pairwise path: some |G_i - G_ref| above kSpan.
 template <typename IO, int DK>
-__device__ __forceinline__ void load_gates_cumsum(float* sG, int ld, const IO* g, int gate, size_t row0, int H,
+__device__ __forceinline__ bool load_gates_cumsum(float* sG, int ld, const IO* g, int gate, size_t row0, int H,
                                                   int nv) {
   if (gate == KDA_GATE_CHANNEL) {
     load_rows<IO, DK>(sG, ld, g, row0, H, nv, DK, 0);
@@ -345,6 +347,7 @@ __device__ __forceinline__ void load_gates_cumsum(float* sG, int ld, const IO* g
     }
   }
   __syncthreads();
+  bool bad = false;
   if (threadIdx.x < DK) {
     float x[kC];
 #pragma unroll
@@ -352,18 +355,10 @@ __device__ __forceinline__ void load_gates_cumsum(float* sG, int ld, const IO* g
 #pragma unroll
     for (int i = 1; i < kC; ++i) x[i] += x[i - 1];
 #pragma unroll
-    for (int i = 0; i < kC; ++i) sG[i * ld + threadIdx.x] = x[i];
-  }
-  __syncthreads();
-}
-
-// Whether the chunk needs the exact pairwise path (block-uniform).
-template <int DK>
-__device__ __forceinline__ bool chunk_unsafe(const float* sG, int ld) {
-  bool bad = false;
-  for (int idx = threadIdx.x; idx < kC * DK; idx += kThreads) {
-    const int i = idx / DK, r = idx % DK;
-    bad |= !(fabsf(sG[i * ld + r] - sG[kRef * ld + r]) <= kSpan);
+    for (int i = 0; i < kC; ++i) {
+      sG[i * ld + threadIdx.x] = x[i];
+      bad |= !(fabsf(x[i] - x[kRef]) <= kSpan);
+    }
   }
   return __syncthreads_or(bad) != 0;
 }
@@ -497,8 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
   load_rows<IO, DK>(sK, LK, k, row0, a.H, nv, DK, 0);
   load_rows<IO, DK>(sQ, LK, q, row0, a.H, nv, DK, 0);
   if (tid < kC) sb[tid] = tid < nv ? to_f32(beta[row0 + (size_t)tid * a.H]) : 0.f;
-  load_gates_cumsum<IO, DK>(sG, LK, static_cast<const IO*>(a.g), a.gate, row0, a.H, nv);
-  const bool slow = chunk_unsafe<DK>(sG, LK);
+  const bool slow = load_gates_cumsum<IO, DK>(sG, LK, static_cast<const IO*>(a.g), a.gate, row0, a.H, nv);
   if (tid < DK) {
     se[tid] = expf(sG[kRef * LK + tid]);
     a.gam[rec * DK + tid] = expf(sG[(kC - 1) * LK + tid]);
@@ -1270,8 +1264,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   rows_in(sq, LKb, static_cast<const bf16*>(a.q), DK);
   rows_in(sv, LVb, static_cast<const bf16*>(a.v), DV);
   if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const bf16*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
-  load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
-  const bool slow = chunk_unsafe<DK>(sG, LK);
+  const bool slow = load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
   if (tid < DK) {
     se[tid] = __expf(sG[kRef * LK + tid]);
     a.gam[rec * DK + tid] = __expf(sG[(kC - 1) * LK + tid]);
@@ -1553,8 +1546,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   zero(dG_acc);
 
   if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const IO*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
-  load_gates_cumsum<IO, DK>(sG, LK, static_cast<const IO*>(a.g), a.gate, row0, a.H, nv);
-  const bool slow = chunk_unsafe<DK>(sG, LK);
+  const bool slow = load_gates_cumsum<IO, DK>(sG, LK, static_cast<const IO*>(a.g), a.gate, row0, a.H, nv);
   load_rows<IO, DK>(sX, LK, k, row0, a.H, nv, DK, 0);
   load_f32(sY, LK, a.dW + rec * kC * DK, DK, kC, DK);
   load_f32(sT, kLC, a.Tm + rec * kC * kC, kC, kC, kC);
@@ -1717,16 +1709,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_kernel(const ChunkBwd
   __syncthreads();  // sX is no longer read: it takes dG
   for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) { sX[i * LK + r] = dG_acc[mt][nt][e]; });
   __syncthreads();
-  if (tid < DK) {  // dG_C terms, then dg = reverse cumsum of dG over the chunk
+  if (tid < DK) {  // the dG_C terms of channel r, into colC row 0
     const int r = tid;
     float x = 0.f;
 #pragma unroll
     for (int w = 0; w < TK::WM; ++w) x += colC[w * DK + r];
-    x = fmaf(expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
-    float acc = x;
+    colC[r] = fmaf(expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
+  }
+  __syncthreads();
+  if (tid < DK) {  // dg = reverse cumsum of dG over the chunk, plus the dG_C terms
+    float acc = colC[tid];
     for (int i = kC - 1; i >= 0; --i) {
-      acc += sX[i * LK + r];
-      sX[i * LK + r] = acc;
+      acc += sX[i * LK + tid];
+      sX[i * LK + tid] = acc;
     }
   }
   __syncthreads();
@@ -1825,8 +1820,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   if (tid < kC) sb[tid] = tid < nv ? to_f32(static_cast<const bf16*>(a.beta)[row0 + (size_t)tid * a.H]) : 0.f;
   rows_in(sk, k);
   rows_in(sq, q);
-  load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
-  const bool slow = chunk_unsafe<DK>(sG, LK);
+  const bool slow = load_gates_cumsum<bf16, DK>(sG, LK, static_cast<const bf16*>(a.g), a.gate, row0, a.H, nv);
   {  // dW and dAqk (bf16 from the d_v kernel)
     const bf16* dWg = reinterpret_cast<const bf16*>(a.dW) + rec * kC * DK;
     const bf16* dAg = reinterpret_cast<const bf16*>(a.dAqk) + rec * kC * kC;
@@ -2020,16 +2014,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   __syncthreads();  // the k and q tiles are no longer read: they take dG
   for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) { sdG[i * LK + r] = dG_acc[mt][nt][e]; });
   __syncthreads();
-  if (tid < DK) {  // dG_C terms, then dg = reverse cumsum of dG over the chunk
+  if (tid < DK) {  // the dG_C terms of channel r, into colC row 0
     const int r = tid;
     float x = 0.f;
 #pragma unroll
     for (int w = 0; w < TK::WM; ++w) x += colC[w * DK + r];
-    x = fmaf(__expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
-    float acc = x;
+    colC[r] = fmaf(__expf(sG[(kC - 1) * LK + r]), a.dgam[rec * DK + r], x);
+  }
+  __syncthreads();
+  if (tid < DK) {  // dg = reverse cumsum of dG over the chunk, plus the dG_C terms
+    float acc = colC[tid];
     for (int i = kC - 1; i >= 0; --i) {
-      acc += sdG[i * LK + r];
-      sdG[i * LK + r] = acc;
+      acc += sdG[i * LK + tid];
+      sdG[i * LK + tid] = acc;
     }
   }
   __syncthreads();
