@@ -461,7 +461,7 @@ __device__ __forceinline__ void solve_T_blocked(const float* sP, const float* sb
 template <int DK, int DV>
 constexpr size_t prep_smem() {
   constexpr int LK = DK + 4, LM = (DK > DV ? DK : DV) + 4;
-  return sizeof(float) * ((size_t)4 * kC * LK + (size_t)kC * LM + 3 * kC * kLC + kC + DK);
+  return sizeof(float) * ((size_t)4 * kC * LK + (size_t)kC * LM + 3 * kC * kLC + kC + DK + 3 * 256);
 }
 
 // Per chunk, fp32 inputs (IO = float; bf16 inputs take the kernels on bf16
@@ -482,6 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
   float* sT = sA + kC * kLC;  // [64][kLC] T
   float* sb = sT + kC * kLC;  // [64] beta
   float* se = sb + kC;        // [DK] exp(G_ref)
+  float* sXs = se + DK;       // [3][16][16] solve scratch
   const int tid = threadIdx.x, warp = tid >> 5;
   const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
@@ -562,33 +563,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     a.Aqk[rec * kC * kC + idx] = sA[i * kLC + j];
   }
 
-  // T = (I + diag(beta) P)^-1 (unit lower triangular) by forward substitution
-  // down each column: thread j < 64 keeps column j in registers; row i reads
-  // P[i][0..i) as broadcast 16-byte loads (fully unrolled: 2016 FMAs).
-  if (tid < kC) {
-    const int j = tid;
-    float tc[kC];
-#pragma unroll
-    for (int i = 0; i < kC; ++i) {
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int m = 0; m < i; m += 4) {
-        const float4 p = *reinterpret_cast<const float4*>(sP + i * kLC + m);
-        s4[0] = fmaf(p.x, tc[m], s4[0]);
-        if (m + 1 < i) s4[1] = fmaf(p.y, tc[m + 1], s4[1]);
-        if (m + 2 < i) s4[2] = fmaf(p.z, tc[m + 2], s4[2]);
-        if (m + 3 < i) s4[3] = fmaf(p.w, tc[m + 3], s4[3]);
-      }
-      tc[i] = i == j ? 1.f : (i < j ? 0.f : -sb[i] * ((s4[0] + s4[1]) + (s4[2] + s4[3])));
-      sT[i * kLC + j] = tc[i];
+  // Warps 0-3: T = (I + diag(beta) P)^-1 by 16 x 16 blocks; the other warps
+  // meanwhile build beta K+ and beta v, the right operands of W and U.
+  if (tid < 128) {
+    solve_T_blocked(sP, sb, sT, sXs, tid);
+  } else {
+    for (int idx = tid - 128; idx < kC * DK; idx += kThreads - 128) {
+      const int i = idx / DK, r = idx % DK;
+      sX[i * LK + r] *= sb[i] * (slow ? 1.f : se[r]);
+    }
+    for (int idx = tid - 128; idx < kC * DV; idx += kThreads - 128) {
+      const int i = idx / DV, c = idx % DV;
+      const IO* vr = static_cast<const IO*>(a.v) + (row0 + (size_t)i * a.H) * DV;
+      sY[i * LM + c] = i < nv ? sb[i] * to_f32(vr[c]) : 0.f;
     }
   }
-  // beta K+ and beta v as the right operands of W and U
-  for (int idx = tid; idx < kC * DK; idx += kThreads) {
-    const int i = idx / DK, r = idx % DK;
-    sX[i * LK + r] *= sb[i] * (slow ? 1.f : se[r]);
-  }
-  load_rows<IO, DV>(sY, LM, static_cast<const IO*>(a.v), row0, a.H, nv, DV, 0, sb);
   __syncthreads();
   store_f32(a.Tm + rec * kC * kC, kC, sT, kLC, kC, kC);
   {
