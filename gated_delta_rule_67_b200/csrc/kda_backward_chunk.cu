@@ -408,14 +408,17 @@ struct PassRec {  // element offsets of the bf16 pass record of one chunk (all r
 };
 
 // T = (I + diag(beta) P)^-1 for a strictly lower 64 x 64 P (fp32, leading
-// dimension kLC) by 16 x 16 blocks, on the 128 threads of warps 0-3 (named
-// barrier 1): the diagonal blocks by forward substitution (one thread per
-// block column, the column in registers), then the blocks below the diagonal
-// level by level, T_IJ = -T_II (sum_{K=J..I-1} A_IK T_KJ) with A = diag(beta) P.
-// T (fp32, leading dimension kLC) is unit lower triangular with zeros above;
-// X is a 3 x 16 x 16 fp32 scratch.
-__device__ __forceinline__ void bar128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// dimension kLC) by 16 x 16 blocks, on the NT first threads of the block
+// (named barrier 1): the diagonal blocks by forward substitution (one thread
+// per block column, the column in registers), then the blocks below the
+// diagonal level by level, T_IJ = -T_II (sum_{K=J..I-1} A_IK T_KJ) with
+// A = diag(beta) P.  T (fp32, leading dimension kLC) is unit lower triangular
+// with zeros above; X is a 3 x 16 x 16 fp32 scratch.
+template <int NT>
+__device__ __forceinline__ void bar_nt() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
+template <int NT>
 __device__ __forceinline__ void solve_T_blocked(const float* sP, const float* sb, float* T, float* X, int t) {
+  static_assert(NT > kC && NT % 32 == 0, "threads");
   if (t < kC) {  // diagonal block I = t / 16, column jj = t % 16
     const int I = t >> 4, jj = t & 15, r0 = 16 * I;
     float tc[16];
@@ -428,16 +431,16 @@ __device__ __forceinline__ void solve_T_blocked(const float* sP, const float* sb
       T[(r0 + ii) * kLC + r0 + jj] = tc[ii];
     }
   } else {  // the six blocks above the diagonal are zero
-    for (int e = t - kC; e < 6 * 256; e += 128 - kC) {
+    for (int e = t - kC; e < 6 * 256; e += NT - kC) {
       const int blk = e >> 8, a = (e >> 4) & 15, b = e & 15;
       const int I = blk < 3 ? 0 : (blk < 5 ? 1 : 2), J = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
       T[(16 * I + a) * kLC + 16 * J + b] = 0.f;
     }
   }
-  bar128();
+  bar_nt<NT>();
   for (int d = 1; d < 4; ++d) {
     const int nb = 4 - d;  // blocks (I, J = I - d), J = 0 .. nb-1
-    for (int e = t; e < nb * 256; e += 128) {
+    for (int e = t; e < nb * 256; e += NT) {
       const int J = e >> 8, I = J + d, a = (e >> 4) & 15, b = e & 15;
       float s = 0.f;
       for (int K = J; K < I; ++K)
@@ -445,17 +448,18 @@ __device__ __forceinline__ void solve_T_blocked(const float* sP, const float* sb
         for (int m = 0; m < 16; ++m) s = fmaf(sP[(16 * I + a) * kLC + 16 * K + m], T[(16 * K + m) * kLC + 16 * J + b], s);
       X[e] = sb[16 * I + a] * s;
     }
-    bar128();
-    for (int e = t; e < nb * 256; e += 128) {
+    bar_nt<NT>();
+    for (int e = t; e < nb * 256; e += NT) {
       const int J = e >> 8, I = J + d, a = (e >> 4) & 15, b = e & 15;
       float s = 0.f;
 #pragma unroll
       for (int m = 0; m < 16; ++m) s = fmaf(T[(16 * I + a) * kLC + 16 * I + m], X[J * 256 + m * 16 + b], s);
       T[(16 * I + a) * kLC + 16 * J + b] = -s;
     }
-    bar128();
+    bar_nt<NT>();
   }
 }
+constexpr int kSolveThreads = 256;  // 8 warps solve T while the others prepare the W/U operands
 
 // ------------------------------------------------------------------ kernel 1
 template <int DK, int DV>
@@ -563,16 +567,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_kernel(const ChunkBwdArg
     a.Aqk[rec * kC * kC + idx] = sA[i * kLC + j];
   }
 
-  // Warps 0-3: T = (I + diag(beta) P)^-1 by 16 x 16 blocks; the other warps
+  // Warps 0-7: T = (I + diag(beta) P)^-1 by 16 x 16 blocks; the other warps
   // meanwhile build beta K+ and beta v, the right operands of W and U.
-  if (tid < 128) {
-    solve_T_blocked(sP, sb, sT, sXs, tid);
+  if (tid < kSolveThreads) {
+    solve_T_blocked<kSolveThreads>(sP, sb, sT, sXs, tid);
   } else {
-    for (int idx = tid - 128; idx < kC * DK; idx += kThreads - 128) {
+    for (int idx = tid - kSolveThreads; idx < kC * DK; idx += kThreads - kSolveThreads) {
       const int i = idx / DK, r = idx % DK;
       sX[i * LK + r] *= sb[i] * (slow ? 1.f : se[r]);
     }
-    for (int idx = tid - 128; idx < kC * DV; idx += kThreads - 128) {
+    for (int idx = tid - kSolveThreads; idx < kC * DV; idx += kThreads - kSolveThreads) {
       const int i = idx / DV, c = idx % DV;
       const IO* vr = static_cast<const IO*>(a.v) + (row0 + (size_t)i * a.H) * DV;
       sY[i * LM + c] = i < nv ? sb[i] * to_f32(vr[c]) : 0.f;
@@ -1307,20 +1311,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   }
   __syncthreads();
 
-  // Warps 0-3: T = (I + diag(beta) P)^-1 by blocks (fp32), then its bf16 image
+  // Warps 0-7: T = (I + diag(beta) P)^-1 by blocks (fp32), then its bf16 image
   // and the global copy.  The other warps meanwhile store P and the right
   // operands beta K+ and beta v of W and U (the factored tiles are dead).
   bf16* Tg = reinterpret_cast<bf16*>(a.Tm) + rec * kC * kC;
-  if (tid < 128) {
-    solve_T_blocked(sP, sb, sTf, sXs, tid);
-    for (int idx = tid; idx < kC * kC / 2; idx += 128) {
+  if (tid < kSolveThreads) {
+    solve_T_blocked<kSolveThreads>(sP, sb, sTf, sXs, tid);
+    for (int idx = tid; idx < kC * kC / 2; idx += kSolveThreads) {
       const int i = idx / (kC / 2), j = (idx % (kC / 2)) * 2;
       const __nv_bfloat162 t2 = __floats2bfloat162_rn(sTf[i * kLC + j], sTf[i * kLC + j + 1]);
       *reinterpret_cast<__nv_bfloat162*>(sT + i * LCb + j) = t2;
       *reinterpret_cast<__nv_bfloat162*>(Tg + i * kC + j) = t2;
     }
   } else {
-    const int t2 = tid - 128, n2 = kThreads - 128;
+    const int t2 = tid - kSolveThreads, n2 = kThreads - kSolveThreads;
     float* Pg = a.Pkk + rec * kC * kC;
     for (int idx = t2; idx < kC * kC / 4; idx += n2) {
       const int i = idx / (kC / 4), j = (idx % (kC / 4)) * 4;
