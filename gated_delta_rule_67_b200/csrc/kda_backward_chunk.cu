@@ -1906,43 +1906,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   const float* dQs = sQs;
   bf16* dq = static_cast<bf16*>(a.dq);
   if (!slow) {
-    {  // dQ+_r = dAqk K-_r;  dq = scale (exp(G - G_ref) dQ+_r + Gamma dO S0^T)
-      float acc[TK::MT][TK::NT][4];
-      zero(acc);
-      warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(acc, sQA, LCb, sA, LKb, m0, n0);
-      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-        const float x = acc[mt][nt][e], G = sG[i * LK + r];
-        const float ex = __expf(G - sG[kRef * LK + r]), gm = __expf(G), dqs = dQs[i * DK + r];
-        const float qs = a.scale * __bfloat162float(sq[i * LKb + r]);  // Q+_r = qs ex, Q+ = qs Gamma
-        if (i < nv) {
-          const float v = a.scale * fmaf(ex, x, gm * dqs);
-          const size_t o = (row0 + (size_t)i * a.H) * DK + r;
-          if (a.dq32) a.dq32[o] = v; else dq[o] = __float2bfloat16_rn(v);
-        }
-        dG_acc[mt][nt][e] += qs * fmaf(x, ex, dqs * gm);
-      });
-    }
-    {  // dK-_r = dAqk^T Q+_r + M^T K+_r
-      float acc[TK::MT][TK::NT][4];
-      zero(acc);
-      warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(acc, sQA, LCb, sC, LKb, m0, n0);
-      warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(acc, sDT, LCb, sB, LKb, m0, n0);
-      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-        const float x = acc[mt][nt][e], ei = __expf(sG[kRef * LK + r] - sG[i * LK + r]);
-        dk_acc[mt][nt][e] = fmaf(ei, x, dk_acc[mt][nt][e]);
-        dG_acc[mt][nt][e] = fmaf(-x, __bfloat162float(sk[i * LKb + r]) * ei, dG_acc[mt][nt][e]);
-      });
-    }
-    {  // dK+_r = M K-_r
-      float acc[TK::MT][TK::NT][4];
-      zero(acc);
-      warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(acc, sDT, LCb, sA, LKb, m0, n0);
-      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-        const float x = acc[mt][nt][e], ex = __expf(sG[i * LK + r] - sG[kRef * LK + r]);
-        dk_acc[mt][nt][e] = fmaf(ex, x, dk_acc[mt][nt][e]);
-        dG_acc[mt][nt][e] = fmaf(x, __bfloat162float(sk[i * LKb + r]) * ex, dG_acc[mt][nt][e]);
-      });
-    }
+    // the three pairwise products first, then one pass over the elements with
+    // the decay factors taken once: ex = exp(G - G_ref), 1/ex, Gamma = exp(G)
+    float aq[TK::MT][TK::NT][4], am[TK::MT][TK::NT][4], ap[TK::MT][TK::NT][4];
+    zero(aq);  // dQ+_r = dAqk K-_r
+    warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(aq, sQA, LCb, sA, LKb, m0, n0);
+    zero(am);  // dK-_r = dAqk^T Q+_r + M^T K+_r
+    warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(am, sQA, LCb, sC, LKb, m0, n0);
+    warp_mma_bf16<TK::MT, TK::NT, kC, true, false>(am, sDT, LCb, sB, LKb, m0, n0);
+    zero(ap);  // dK+_r = M K-_r
+    warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(ap, sDT, LCb, sA, LKb, m0, n0);
+    for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+      const float G = sG[i * LK + r], d = G - sG[kRef * LK + r];
+      const float ex = __expf(d), ei = __expf(-d), gm = __expf(G), dqs = dQs[i * DK + r];
+      const float kk = __bfloat162float(sk[i * LKb + r]);
+      const float qs = a.scale * __bfloat162float(sq[i * LKb + r]);  // Q+_r = qs ex, Q+ = qs Gamma
+      const float xq = aq[mt][nt][e], xm = am[mt][nt][e], xp = ap[mt][nt][e];
+      if (i < nv) {  // dq = scale (exp(G - G_ref) dQ+_r + Gamma dO S0^T)
+        const float v = a.scale * fmaf(ex, xq, gm * dqs);
+        const size_t o = (row0 + (size_t)i * a.H) * DK + r;
+        if (a.dq32) a.dq32[o] = v; else dq[o] = __float2bfloat16_rn(v);
+      }
+      dk_acc[mt][nt][e] = fmaf(ei, xm, fmaf(ex, xp, dk_acc[mt][nt][e]));
+      dG_acc[mt][nt][e] += fmaf(qs, fmaf(xq, ex, dqs * gm), kk * fmaf(xp, ex, -xm * ei));
+    });
   } else {
     // exact pairwise terms, E = exp(G_ir - G_jr) for j <= i (see the fp32 kernel)
     auto K_ = [&](int i, int r) { return __bfloat162float(sk[i * LKb + r]); };
