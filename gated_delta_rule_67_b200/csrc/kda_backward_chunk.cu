@@ -1833,7 +1833,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       cp16(sT + i * LCb + c, Tg + (size_t)i * kC + c, 16);
     }
   }
-  {  // the fold's fp32 inputs, in flight while the products run
+  cp_commit();  // group 1: everything the products need
+  {  // group 2: the fold's fp32 inputs, in flight while the products run
     const float* qs = a.dQs + rec * kC * DK;
     const float* ks = a.dKb + rec * kC * DK;
     for (int idx = tid; idx < kC * DK / 4; idx += kThreads) {
@@ -1841,7 +1842,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       cp16(sKs + 4 * idx, ks + 4 * idx, 16);
     }
   }
-  cp_wait();
+  cp_commit();
+  cp_wait_group<1>();
   __syncthreads();
   for (int idx = tid; idx < kC * DK; idx += kThreads) {  // K+ = k exp(G)
     const int i = idx / DK, r = idx % DK;
@@ -1902,6 +1904,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
       sC[i * LKb + r] = __float2bfloat16_rn(qq * ex);
     }
   }
+  cp_wait_group<0>();  // the fold's inputs
   __syncthreads();
   const float* dQs = sQs;
   bf16* dq = static_cast<bf16*>(a.dq);
