@@ -1264,17 +1264,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   }
   cp_wait();
   __syncthreads();
-  for (int idx = tid; idx < kC * DK; idx += kThreads) {  // Q+, Kbar (record) and the factored operands
-    const int i = idx / DK, r = idx % DK;
-    const float G = sG[i * LK + r], kk = __bfloat162float(sk[i * LKb + r]);
-    const float qq = a.scale * __bfloat162float(sq[i * LKb + r]);
-    pr[PR::oKb + i * PR::LKb + r] = __float2bfloat16_rn(kk * __expf(sG[(kC - 1) * LK + r] - G));
-    pr[PR::oQp + i * PR::LKb + r] = __float2bfloat16_rn(qq * __expf(G));
+  for (int idx = tid; idx < kC * DK / 2; idx += kThreads) {  // Q+, Kbar (record) and the factored operands
+    const int i = idx / (DK / 2), r = (idx % (DK / 2)) * 2;     // two channels per thread
+    const float2 G = *reinterpret_cast<const float2*>(sG + i * LK + r);
+    const float2 GC = *reinterpret_cast<const float2*>(sG + (kC - 1) * LK + r);
+    const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sk + i * LKb + r));
+    float2 qq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sq + i * LKb + r));
+    qq.x *= a.scale, qq.y *= a.scale;
+    *reinterpret_cast<__nv_bfloat162*>(pr + PR::oKb + i * PR::LKb + r) =
+        __floats2bfloat162_rn(kk.x * __expf(GC.x - G.x), kk.y * __expf(GC.y - G.y));
+    *reinterpret_cast<__nv_bfloat162*>(pr + PR::oQp + i * PR::LKb + r) =
+        __floats2bfloat162_rn(qq.x * __expf(G.x), qq.y * __expf(G.y));
     if (!slow) {
-      const float d = G - sG[kRef * LK + r], ex = __expf(d);
-      sX[i * LKb + r] = __float2bfloat16_rn(kk * ex);
-      sY[i * LMb + r] = __float2bfloat16_rn(kk * __expf(-d));
-      sQ[i * LKb + r] = __float2bfloat16_rn(qq * ex);
+      const float2 Gr = *reinterpret_cast<const float2*>(sG + kRef * LK + r);
+      const float dx = G.x - Gr.x, dy = G.y - Gr.y, ex = __expf(dx), ey = __expf(dy);
+      *reinterpret_cast<__nv_bfloat162*>(sX + i * LKb + r) = __floats2bfloat162_rn(kk.x * ex, kk.y * ey);
+      *reinterpret_cast<__nv_bfloat162*>(sY + i * LMb + r) =
+          __floats2bfloat162_rn(kk.x * __expf(-dx), kk.y * __expf(-dy));
+      *reinterpret_cast<__nv_bfloat162*>(sQ + i * LKb + r) = __floats2bfloat162_rn(qq.x * ex, qq.y * ey);
     }
   }
   __syncthreads();
@@ -1330,13 +1337,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
       const int i = idx / (kC / 4), j = (idx % (kC / 4)) * 4;
       *reinterpret_cast<float4*>(Pg + i * kC + j) = *reinterpret_cast<const float4*>(sP + i * kLC + j);
     }
-    for (int idx = t2; idx < kC * DK; idx += n2) {
-      const int i = idx / DK, r = idx % DK;
-      sX[i * LKb + r] = __float2bfloat16_rn(sb[i] * __bfloat162float(sk[i * LKb + r]) * __expf(sG[i * LK + r]));
+    for (int idx = t2; idx < kC * DK / 2; idx += n2) {
+      const int i = idx / (DK / 2), r = (idx % (DK / 2)) * 2;
+      const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sk + i * LKb + r));
+      const float2 G = *reinterpret_cast<const float2*>(sG + i * LK + r);
+      *reinterpret_cast<__nv_bfloat162*>(sX + i * LKb + r) =
+          __floats2bfloat162_rn(sb[i] * kk.x * __expf(G.x), sb[i] * kk.y * __expf(G.y));
     }
-    for (int idx = t2; idx < kC * DV; idx += n2) {
-      const int i = idx / DV, c = idx % DV;
-      sY[i * LMb + c] = __float2bfloat16_rn(sb[i] * __bfloat162float(sv[i * LVb + c]));
+    for (int idx = t2; idx < kC * DV / 2; idx += n2) {
+      const int i = idx / (DV / 2), c = (idx % (DV / 2)) * 2;
+      const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sv + i * LVb + c));
+      *reinterpret_cast<__nv_bfloat162*>(sY + i * LMb + c) = __floats2bfloat162_rn(sb[i] * v.x, sb[i] * v.y);
     }
   }
   __syncthreads();
