@@ -1918,6 +1918,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   cp_wait_group<0>();  // the fold's inputs
   __syncthreads();
   const float* dQs = sQs;
+  const float* dKb = sKs;
+  float cp[TK::MT][TK::NT][2] = {};  // column partial sums of dKbar . Kbar (for dG_C)
   bf16* dq = static_cast<bf16*>(a.dq);
   if (!slow) {
     // the three pairwise products first, then one pass over the elements with
@@ -1933,6 +1935,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
       const float G = sG[i * LK + r], d = G - sG[kRef * LK + r];
       const float ex = __expf(d), ei = __expf(-d), gm = __expf(G), dqs = dQs[i * DK + r];
+      const float kbf = __expf(sG[(kC - 1) * LK + r] - G);  // Kbar = k kbf
       const float kk = __bfloat162float(sk[i * LKb + r]);
       const float qs = a.scale * __bfloat162float(sq[i * LKb + r]);  // Q+_r = qs ex, Q+ = qs Gamma
       const float xq = aq[mt][nt][e], xm = am[mt][nt][e], xp = ap[mt][nt][e];
@@ -1941,8 +1944,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
         const size_t o = (row0 + (size_t)i * a.H) * DK + r;
         if (a.dq32) a.dq32[o] = v; else dq[o] = __float2bfloat16_rn(v);
       }
-      dk_acc[mt][nt][e] = fmaf(ei, xm, fmaf(ex, xp, dk_acc[mt][nt][e]));
-      dG_acc[mt][nt][e] += fmaf(qs, fmaf(xq, ex, dqs * gm), kk * fmaf(xp, ex, -xm * ei));
+      const float xb = dKb[i * DK + r], yb = xb * kk * kbf;  // the Kbar terms
+      dk_acc[mt][nt][e] = fmaf(kbf, xb, fmaf(ei, xm, fmaf(ex, xp, dk_acc[mt][nt][e])));
+      dG_acc[mt][nt][e] += fmaf(qs, fmaf(xq, ex, dqs * gm), kk * fmaf(xp, ex, -xm * ei)) - yb;
+      cp[mt][nt][e & 1] += yb;
     });
   } else {
     // exact pairwise terms, E = exp(G_ir - G_jr) for j <= i (see the fp32 kernel)
@@ -1976,15 +1981,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     });
   }
   {  // Kbar: dk += exp(G_C - G) dKbar, dG -= dKbar . Kbar, dG_C += column sums of the same
-    const float* dKb = sKs;
-    float cp[TK::MT][TK::NT][2] = {};
-    for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
-      const float kbf = __expf(sG[(kC - 1) * LK + r] - sG[i * LK + r]);  // Kbar = k kbf
-      const float x = dKb[i * DK + r], y = x * __bfloat162float(sk[i * LKb + r]) * kbf;
-      dk_acc[mt][nt][e] = fmaf(kbf, x, dk_acc[mt][nt][e]);
-      dG_acc[mt][nt][e] -= y;
-      cp[mt][nt][e & 1] += y;
-    });
+    if (slow)  // (the fast path folded these into its epilogue)
+      for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
+        const float kbf = __expf(sG[(kC - 1) * LK + r] - sG[i * LK + r]);  // Kbar = k kbf
+        const float x = dKb[i * DK + r], y = x * __bfloat162float(sk[i * LKb + r]) * kbf;
+        dk_acc[mt][nt][e] = fmaf(kbf, x, dk_acc[mt][nt][e]);
+        dG_acc[mt][nt][e] -= y;
+        cp[mt][nt][e & 1] += y;
+      });
 #pragma unroll
     for (int nt = 0; nt < TK::NT; ++nt)
 #pragma unroll
