@@ -311,6 +311,12 @@ __device__ __forceinline__ void cp_async16(float* dst, const float* src) {
                : "memory");
 }
 __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// 16-byte cp.async of which the first `bytes` (0 or 16) come from src, the rest zero-filled.
+__device__ __forceinline__ void cp16(void* dst, const void* src, int bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(bytes)
+               : "memory");
+}
 // fp32 rows x cols block from global (leading dimension gld) into shared (ld),
 // cols % 4 == 0, by cp.async: complete after cp_wait().
 template <int NTH = kThreads>
@@ -970,11 +976,6 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
   bf16* simg = reinterpret_cast<bf16*>(smb);      // [DK][LS] state (or dS) image
   bf16* vimg = simg + DK * LS;                    // [64][LS] V' (or dV') image
   uint8_t* bufs = smb + PB::img;
-  auto cp16 = [&](void* dst, const void* src, int bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src), "r"(bytes)
-                 : "memory");
-  };
   auto copy = [&](uint8_t* dst, const void* src, size_t bytes) {  // bytes % 16 == 0
     const uint8_t* s = static_cast<const uint8_t*>(src);
     for (size_t o = (size_t)tid * 16; o < bytes; o += (size_t)NTH * 16) cp16(dst + o, s + o, 16);
@@ -1241,11 +1242,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
   bf16* pr = a.prec + rec * PR::n;
-  auto cp16 = [&](void* dst, const void* src, int bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src), "r"(bytes)
-                 : "memory");
-  };
   auto rows_in = [&](bf16* dst, int ld, const bf16* src, int D) {  // 64 input rows of D (zeros past the tail)
     const int per = D / 8;
     for (int idx = tid; idx < kC * per; idx += kThreads) {
@@ -1407,11 +1403,6 @@ __global__ void __launch_bounds__(kLaThreads, 2) bwd_local_a_bf16_kernel(const C
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
-  auto cp16 = [&](void* dst, const void* src, int bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src), "r"(bytes)
-                 : "memory");
-  };
   // rows of 16-byte pieces: [rows][width] bf16 from global (row i at src_row(i)) into [rows][ld]
   auto rows_in = [&](bf16* dst, int ld, int rows, int width, auto src_row, int valid) {
     const int per = width / 8;
@@ -1807,11 +1798,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   float dk_acc[TK::MT][TK::NT][4], dG_acc[TK::MT][TK::NT][4];
   zero(dk_acc);
   zero(dG_acc);
-  auto cp16 = [&](void* dst, const void* src, int bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src), "r"(bytes)
-                 : "memory");
-  };
   auto rows_in = [&](bf16* dst, const bf16* src) {  // 64 input rows of DK (zeros past the tail)
     constexpr int per = DK / 8;
     for (int idx = tid; idx < kC * per; idx += kThreads) {
