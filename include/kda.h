@@ -161,7 +161,7 @@ KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
  * Bytes of device workspace kda_backward needs for this problem: per-chunk
  * records (per 64-token chunk and head: the chunk's operands, the state
  * entering it and the state gradient leaving it, and intermediate gradients;
- * about 0.45 MB for bf16 and 0.6 MB for fp32 at dk = dv = 128); 0 for
+ * about 0.33 MB for bf16 and 0.6 MB for fp32 at dk = dv = 128); 0 for
  * arguments kda_backward would reject.
  */
 KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, int dtype);

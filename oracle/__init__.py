@@ -12,7 +12,12 @@ DeltaNet and Gated DeltaNet special cases, boundedness, and hand-derived
 worked examples under tests/golden/.  ``prepare_inputs`` (fused input
 preparation: unit-length q and k, log-sigmoid gates, sigmoid write
 strengths) is pinned in tests/test_oracle_prep.py against closed forms and
-a second formula for each step.
+a second formula for each step.  ``kda_backward`` (reverse-mode gradients of
+the recurrence) is pinned in tests/test_oracle_backward.py by central
+differences of ``kda_forward`` and by torch autograd through a plain fp64
+loop; ``prepare_backward`` (the chain rule through the preparation) in
+tests/test_oracle_prep_backward.py by central differences of
+``prepare_inputs`` and of the prepared forward.
 """
 from __future__ import annotations
 
