@@ -69,22 +69,27 @@ constexpr uint32_t kRecGamma = 73728;   // gamma: 128 fp32
 constexpr uint32_t kRecBytes = 74240;
 
 // --- prep kernel: shared memory (byte offsets from a 1024-aligned base) ---
-// Region A (32 KiB) is a 128-row K-major tile: rows 0-63 first hold g and then
-// K+_r, rows 64-127 hold q and then Q+_r (both in place).  Once the score MMA
-// is done it holds the v tile [0,16K), the (T diag beta)^T operand [16K,24K)
-// and four T blocks [24K,28K).
-// Region K (16 KiB): the k tile, turned in place into K+ (start-decayed);
-// after the W/U MMAs the U^T staging tile.
-// Region B (16 KiB): K-_r (score B operand); then the 10 A_kk blocks [0,10K)
-// and six T blocks [10K,16K); finally the -W staging tile.
+// 52 KiB, so that four CTAs share an SM.
+// Region A (32 KiB) is a 128-row K-major tile in two 64-channel halves of
+// 16 KiB.  Rows 0-63 of each half ([0,8K) and [16K,24K)) first hold g, then
+// K+_r, which stays for the W product and is finally overwritten by the -W
+// staging tile; rows 64-127 ([8K,16K) and [24K,32K)) hold q, then Q+_r.
+// Once the score MMA is done, the v tile takes [8K,16K) and [24K,32K) (a
+// 64-row tile whose channel halves lie 16 KiB apart); its second half comes
+// after the A_qk^T staging tile at [24K,32K) has been bulk-stored.
+// Region B (16 KiB): the k tile, turned in place into K-_r (score B operand);
+// then the 10 A_kk blocks [0,10K) and six T blocks [10K,16K); after the
+// solve the (T diag beta)^T operand [0,8K); finally the U^T staging tile.
+// Region T (4 KiB): the last four T blocks.
 constexpr uint32_t kP1A = 0;
-constexpr uint32_t kP1K = 32768;
-constexpr uint32_t kP1B = 49152;
-constexpr uint32_t kP1Bytes = 65536;
-constexpr uint32_t kP1V = kP1A;              // v tile, after the score MMA
-constexpr uint32_t kP1B2 = kP1A + 16384;     // (T diag beta)^T, K-major 64 x 64
-constexpr uint32_t kP1QT = kP1A + 16384;     // A_qk^T staging (bulk-stored before the B2 operand is built)
+constexpr uint32_t kP1B = 32768;
+constexpr uint32_t kP1T = 49152;
+constexpr uint32_t kP1Bytes = 53248;
+constexpr uint32_t kP1V = kP1A + 8192;       // v tile (half stride 16 KiB), after the score MMA
+constexpr uint32_t kP1B2 = kP1B;             // (T diag beta)^T, K-major 64 x 64, after the solve
+constexpr uint32_t kP1QT = kP1A + 24576;     // A_qk^T staging (bulk-stored before v's second half lands)
 constexpr int kP1Threads = 256;
+constexpr int kP1Blocks = 4;                 // CTAs per SM: 4 x 128 TMEM columns, 4 x ~55 KiB shared memory
 // Per-chunk safe range of the factored form: every channel's cumulative
 // log-gate over the chunk must stay above -kSafeSpan, so that each factor
 // exp(+-(G_i - G_r)), exp(G_r), exp(G_C - G_r) lies in [e^-64, e^64].
@@ -140,7 +145,7 @@ __device__ __forceinline__ void st8(uint8_t* p, const float* f) {
 }
 // The lower-triangular 64 x 64 matrices A_kk and T are kept as 16 x 16 fp32
 // blocks (I, J), J <= I, numbered p = I(I+1)/2 + J; A blocks in region B,
-// T blocks 0-5 after them in region B and T blocks 6-9 at the end of region A.
+// T blocks 0-5 after them in region B and T blocks 6-9 in region T.
 __device__ __forceinline__ int blk(int I, int J) { return I * (I + 1) / 2 + J; }
 // Element (r, c) of a 16 x 16 block: rows of 16 floats with the float4 column
 // XOR-ed by (r/2)%4, so that 8 consecutive rows at one float4 column hit 8
@@ -149,7 +154,7 @@ __device__ __forceinline__ int bidx(int r, int c) { return r * 16 + ((((c >> 2) 
 __device__ __forceinline__ float* a_blk(uint8_t* sm, int p) { return reinterpret_cast<float*>(sm + kP1B) + p * 256; }
 __device__ __forceinline__ float* t_blk(uint8_t* sm, int p) {
   return p < 6 ? reinterpret_cast<float*>(sm + kP1B + 10240) + p * 256
-               : reinterpret_cast<float*>(sm + kP1A + 24576) + (p - 6) * 256;
+               : reinterpret_cast<float*>(sm + kP1T) + (p - 6) * 256;
 }
 // Warp-level 16x16x16 product acc += P Q of row-major fp32 16x16 blocks, with
 // mma.sync m16n8k8 (tf32 operands rounded to nearest).  acc[nh] holds the
@@ -195,7 +200,7 @@ __device__ __forceinline__ void store_block_frag(float* X, const float (&acc)[2]
 // unit length per token (the per-token factors are applied wherever q and k
 // are read), log-sigmoid of g, sigmoid of beta.
 template <bool kScalarGate, bool kPrep>
-__global__ void __launch_bounds__(kP1Threads, 3)
+__global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                           const bf16* __restrict__ beta, float scale, uint8_t* __restrict__ records,
@@ -207,6 +212,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   __shared__ float sbeta[kC];
   __shared__ float sgh[kScalarGate ? kC : 1];  // per-head log-gates of the chunk (zeros without a gate)
   __shared__ float snq[kPrep ? kC : 1], snk[kPrep ? kC : 1];  // per-token sums of q^2, k^2 (fused L2 norm)
+  __shared__ float segr[kD];  // per channel: exp(G_r) (factored form) or 1 (exact path); scales W in its extraction
   const bool l2n = kPrep && (prep & KDA_PREP_L2NORM_QK);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     for (int kb = 0; kb < 2; ++kb) {
       if (!kScalarGate) tma_load_4d(sm + kP1A + kb * 16384, &tm_g, &bar_in, kb * 64, h, t0, b);  // rows 0-63
       tma_load_4d(sm + kP1A + kb * 16384 + 8192, &tm_q, &bar_in, kb * 64, h, t0, b);     // rows 64-127
-      tma_load_4d(sm + kP1K + kb * 8192, &tm_k, &bar_in, kb * 64, h, t0, b);
+      tma_load_4d(sm + kP1B + kb * 8192, &tm_k, &bar_in, kb * 64, h, t0, b);
     }
   }
   if (warp == 0) tmem_alloc(&tmem_base, 128);
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
       const int i = tg + 16 * t;
       float q8[8], k8[8];
       ld8(sm + kP1A + kmajor_off(kC + i, c8, 128), q8);
-      ld8(sm + kP1K + kmajor_off(i, c8, kC), k8);
+      ld8(sm + kP1B + kmajor_off(i, c8, kC), k8);
       float sq2 = 0.f, sk2 = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -332,6 +338,10 @@ __global__ void __launch_bounds__(kP1Threads, 3)
       egr[e] = __expf(gref[e]);
       egb[e] = __expf(gend[e] - gref[e]);
     }
+    if (tg == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) segr[c8 + e] = egr[e];
+    }
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const int i = tg + 16 * t;
@@ -339,7 +349,7 @@ __global__ void __launch_bounds__(kP1Threads, 3)
       const uint32_t oA = kmajor_off(i, c8, 128);       // row i of region A
       const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A and of the [-W;Q+] image
       float k8[8], q8[8];
-      ld8(sm + kP1K + oK, k8);
+      ld8(sm + kP1B + oK, k8);
       ld8(sm + kP1A + oQ, q8);
       if (l2n) {
         const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
@@ -349,31 +359,37 @@ __global__ void __launch_bounds__(kP1Threads, 3)
           q8[e] *= rq;
         }
       }
-      float ex[8], ei[8], w[8];
+      // the start-decayed operands first, then the end-decayed ones, so that
+      // fewer values are live at once (64 registers at 4 CTAs per SM)
+      float w[8];
+      {
+        float ex[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        ex[e] = __expf(G[t][e] - gref[e]);
-        ei[e] = __expf(gref[e] - G[t][e]);
-        q8[e] *= scale;
+        for (int e = 0; e < 8; ++e) {
+          ex[e] = __expf(G[t][e] - gref[e]);
+          q8[e] *= scale;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = k8[e] * ex[e];
+        st8(sm + kP1A + oA, w);               // K+_r (over the dead g rows)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = q8[e] * ex[e];
+        st8(sm + kP1A + oQ, w);               // Q+_r (in place of q)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * egr[e]);
+        st8(rec + kRecWQ + oQ, w);            // Q+ image
       }
+      {
+        float ei[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = k8[e] * ex[e];
-      st8(sm + kP1A + oA, w);               // K+_r (over the dead g rows)
+        for (int e = 0; e < 8; ++e) ei[e] = __expf(gref[e] - G[t][e]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = q8[e] * ex[e];
-      st8(sm + kP1A + oQ, w);               // Q+_r (in place of q)
+        for (int e = 0; e < 8; ++e) w[e] = k8[e] * ei[e];
+        st8(sm + kP1B + oK, w);               // K-_r, in place of k
 #pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = k8[e] * ei[e];
-      st8(sm + kP1B + oK, w);               // K-_r
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ex[e] * egr[e]);
-      st8(sm + kP1K + oK, w);               // K+ = k exp(G_i), in place of k
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * egr[e]);
-      st8(rec + kRecWQ + oQ, w);            // Q+ image
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ei[e] * egb[e]);
-      st8(rec + kRecKbar + oK, w);          // Kbar image = k exp(G_C - G_i)
+        for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ei[e] * egb[e]);
+        st8(rec + kRecKbar + oK, w);          // Kbar image = k exp(G_C - G_i)
+      }
     }
     fence_async_smem();
     tc_fence_before();
@@ -428,43 +444,85 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   } else {
     // ---- exact path for chunks whose gates decay past e^-64: the score
     // matrices straight from their definition, every decay factor
-    // exp(G_i - G_j) <= 1 formed per (pair, channel).
-    auto gp = [&](int i, int c) -> float* {
+    // exp(G_i - G_j) <= 1 formed per (pair, channel).  G is staged in fp32
+    // one 64-channel half at a time over the dead g rows of region A.
+    auto gp = [&](int i, int c) -> float* {  // c in [0, 64): channel of the staged half
       return c < 32 ? reinterpret_cast<float*>(sm + kP1A) + i * 32 + c
-                    : c < 64 ? reinterpret_cast<float*>(sm + kP1A + 16384) + i * 32 + (c - 32)
-                             : reinterpret_cast<float*>(sm + kP1B) + i * 64 + (c - 64);
+                    : reinterpret_cast<float*>(sm + kP1A + 16384) + i * 32 + (c - 32);
     };
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) *gp(tg + 16 * t, c8 + e) = G[t][e];
-    __syncthreads();
     constexpr int kPairs = kC * (kC + 1) / 2;  // (i, j) with j <= i
     float akk[9], aqk[9];
+#pragma unroll
+    for (int t = 0; t < 9; ++t) akk[t] = aqk[t] = 0.f;
 #pragma unroll 1
-    for (int t = 0; t < 9; ++t) {
-      const int p = tid + t * kP1Threads;
-      akk[t] = aqk[t] = 0.f;
-      if (p < kPairs) {
-        int i = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
-        while (i * (i + 1) / 2 > p) --i;
-        while ((i + 1) * (i + 2) / 2 <= p) ++i;
-        const int j = p - i * (i + 1) / 2;
-        float sk = 0.f, sq = 0.f;
-#pragma unroll 4
-        for (int c = 0; c < kD; c += 2) {
-          const float2 ki = ld_bf2(sm + kP1K + kmajor_off(i, c, kC));
-          const float2 kj = ld_bf2(sm + kP1K + kmajor_off(j, c, kC));
-          const float2 qi = ld_bf2(sm + kP1A + kmajor_off(kC + i, c, 128));
-          const float d0 = __expf(*gp(i, c) - *gp(j, c)), d1 = __expf(*gp(i, c + 1) - *gp(j, c + 1));
-          sk = fmaf(ki.x * kj.x, d0, fmaf(ki.y * kj.y, d1, sk));
-          sq = fmaf(qi.x * kj.x, d0, fmaf(qi.y * kj.y, d1, sq));
-        }
-        akk[t] = sk;
-        aqk[t] = sq;
+    for (int hf = 0; hf < 2; ++hf) {
+      if ((c8 >> 6) == hf) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) *gp(tg + 16 * t, c8 - 64 * hf + e) = G[t][e];
       }
+      __syncthreads();
+#pragma unroll 1
+      for (int t = 0; t < 9; ++t) {
+        const int p = tid + t * kP1Threads;
+        if (p < kPairs) {
+          int i = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+          while (i * (i + 1) / 2 > p) --i;
+          while ((i + 1) * (i + 2) / 2 <= p) ++i;
+          const int j = p - i * (i + 1) / 2;
+          float sk = akk[t], sq = aqk[t];
+#pragma unroll 4
+          for (int c = 0; c < 64; c += 2) {
+            const int ch = 64 * hf + c;
+            const float2 ki = ld_bf2(sm + kP1B + kmajor_off(i, ch, kC));
+            const float2 kj = ld_bf2(sm + kP1B + kmajor_off(j, ch, kC));
+            const float2 qi = ld_bf2(sm + kP1A + kmajor_off(kC + i, ch, 128));
+            const float d0 = __expf(*gp(i, c) - *gp(j, c)), d1 = __expf(*gp(i, c + 1) - *gp(j, c + 1));
+            sk = fmaf(ki.x * kj.x, d0, fmaf(ki.y * kj.y, d1, sk));
+            sq = fmaf(qi.x * kj.x, d0, fmaf(qi.y * kj.y, d1, sq));
+          }
+          akk[t] = sk;
+          aqk[t] = sq;
+        }
+      }
+      __syncthreads();  // this half of G is read
     }
-    __syncthreads();  // G (in regions A and B) is dead from here on
+    // pass 2 (exact): start- and end-decayed operands, factors <= 1; K+ goes
+    // over the dead g rows of region A (where the factored form keeps K+_r),
+    // with a unit W scale
+    if (tg == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) segr[c8 + e] = 1.f;
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int i = tg + 16 * t;
+      const uint32_t oK = kmajor_off(i, c8, kC);
+      const uint32_t oQ = kmajor_off(kC + i, c8, 128);
+      float k8[8], q8[8], kp[8], qp[8], kb[8];
+      ld8(sm + kP1B + oK, k8);
+      ld8(sm + kP1A + oQ, q8);
+      if (l2n) {
+        const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          k8[e] *= rk;
+          q8[e] *= rq;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float e0 = __expf(G[t][e]);
+        kp[e] = k8[e] * e0;
+        qp[e] = scale * q8[e] * e0;
+        kb[e] = k8[e] * __expf(gend[e] - G[t][e]);
+      }
+      st8(sm + kP1A + kmajor_off(i, c8, 128), kp);
+      st8(rec + kRecWQ + oQ, qp);
+      st8(rec + kRecKbar + oK, kb);
+    }
+    __syncthreads();  // k and q are read: region B takes the A_kk blocks, [24K,32K) of region A the A_qk^T staging
 #pragma unroll 1
     for (int t = 0; t < 9; ++t) {
       const int p = tid + t * kP1Threads;
@@ -487,34 +545,6 @@ __global__ void __launch_bounds__(kP1Threads, 3)
       const int i = e / kC, j = e % kC;
       if (j > i) stbf(sm + kP1QT, kmajor_off(j, i, kC), 0.f);
     }
-    // pass 2 (exact): start- and end-decayed operands, factors <= 1
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int i = tg + 16 * t;
-      const uint32_t oK = kmajor_off(i, c8, kC);
-      const uint32_t oQ = kmajor_off(kC + i, c8, 128);
-      float k8[8], q8[8], kp[8], qp[8], kb[8];
-      ld8(sm + kP1K + oK, k8);
-      ld8(sm + kP1A + oQ, q8);
-      if (l2n) {
-        const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          k8[e] *= rk;
-          q8[e] *= rq;
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float e0 = __expf(G[t][e]);
-        kp[e] = k8[e] * e0;
-        qp[e] = scale * q8[e] * e0;
-        kb[e] = k8[e] * __expf(gend[e] - G[t][e]);
-      }
-      st8(sm + kP1K + oK, kp);
-      st8(rec + kRecWQ + oQ, qp);
-      st8(rec + kRecKbar + oK, kb);
-    }
   }
   fence_async_smem();
   tc_fence_before();
@@ -523,13 +553,10 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   if (tid == 0) {
     bulk_store(rec + kRecAqk, sm + kP1QT, 8192);
     bulk_commit();
-  }
-
-  // ---- region A is free: bring the v tile while the triangle is inverted
-  if (tid == 0) {
+    // Q+_r is dead: bring v while the triangle is inverted, its first
+    // channel half now, the second once the A_qk^T store has read its bytes
     mbar_expect_tx(&bar_v, 16384);
     tma_load_4d(sm + kP1V, &tm_v, &bar_v, 0, h, t0, b);
-    tma_load_4d(sm + kP1V + 8192, &tm_v, &bar_v, 64, h, t0, b);
   }
 
   // ---- T = (I + A_kk)^-1 by 16 x 16 blocks, fp32
@@ -549,6 +576,10 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     for (int r = 0; r < 16; ++r) Tb[bidx(r, jj)] = t[r];
   }
   __syncthreads();
+  if (tid == 0) {
+    bulk_wait_read();
+    tma_load_4d(sm + kP1V + 16384, &tm_v, &bar_v, 64, h, t0, b);
+  }
   // off-diagonal blocks, one sub-diagonal at a time, one warp per block:
   //   X = sum_{K=J}^{I-1} A_IK T_KJ,   T_IJ = -T_II X
   // as 16x16x16 products on the warp-level tensor cores (tf32 in, fp32
@@ -569,10 +600,8 @@ __global__ void __launch_bounds__(kP1Threads, 3)
     }
     __syncthreads();
   }
-  // (T diag(beta))^T as the K-major B operand of the W/U MMAs: row n = i, column k = j.
-  // It reuses the A_qk^T staging bytes, so the bulk store must have read them.
-  if (tid == 0) bulk_wait_read();
-  __syncthreads();
+  // (T diag(beta))^T as the K-major B operand of the W/U MMAs: row n = i, column k = j
+  // (over the A_kk blocks, read by now).
   {
     const int i = tid >> 2, j0 = (tid & 3) * 16, I = i >> 4, J = j0 >> 4;
     float vals[16];
@@ -592,38 +621,42 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   __syncthreads();
   tc_fence_after();
 
-  // ---- W^T = K+^T (T diag beta)^T, U^T = V^T (T diag beta)^T  (M=128, N=64, K=64)
+  // ---- W^T / segr = K+_r^T (T diag beta)^T, U^T = V^T (T diag beta)^T  (M=128, N=64, K=64).
+  // K+_r = K+ / exp(G_r) per channel (rows 0-63 of region A, channel halves
+  // 16 KiB apart; K+ itself on the exact path, segr = 1), so the extraction
+  // scales row c of the first product by segr[c]; v's halves are 16 KiB apart too.
   if (tid == 0) {
     wait_or_flag(&bar_v, 0, hdr, 3);
     tc_fence_after();
     const uint32_t idesc = idesc_bf16_f32(128, 64, 1, 0);
-    const uint32_t kb = smem_u32(sm + kP1K), vb = smem_u32(sm + kP1V), b2 = smem_u32(sm + kP1B2);
+    const uint32_t kb = smem_u32(sm + kP1A), vb = smem_u32(sm + kP1V), b2 = smem_u32(sm + kP1B2);
 #pragma unroll
     for (int k = 0; k < kC / 16; ++k) {
       const uint64_t bd = desc_sw128(b2 + k * 32, 16, 1024);
-      mma_bf16(tm, desc_sw128(kb + 2 * k * 1024, 8192, 1024), bd, idesc, k > 0);
-      mma_bf16(tm + 64, desc_sw128(vb + 2 * k * 1024, 8192, 1024), bd, idesc, k > 0);
+      mma_bf16(tm, desc_sw128(kb + 2 * k * 1024, 16384, 1024), bd, idesc, k > 0);
+      mma_bf16(tm + 64, desc_sw128(vb + 2 * k * 1024, 16384, 1024), bd, idesc, k > 0);
     }
     mma_commit(&bar_mma);
   }
   wait_or_flag(&bar_mma, slow ? 0 : 1, hdr, 4);
   tc_fence_after();
 
-  // ---- -W (staged in region B as a 64-row K-major tile) and U^T (region K, 128-row K-major)
+  // ---- -W (staged over K+_r: rows 0-63 of region A) and U^T (region B, 128-row K-major)
   {
     const int c = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const float wsc = warp < 4 ? -segr[c] : 0.f;
     float v[32];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       if (warp < 4) {
         tmem_ld32(tm + lane_off + half * 32, v);
 #pragma unroll
-        for (int ii = 0; ii < 32; ++ii) stbf(sm + kP1B, kmajor_off(half * 32 + ii, c, kC), -v[ii]);
+        for (int ii = 0; ii < 32; ++ii) stbf(sm + kP1A, kmajor_off(half * 32 + ii, c, 128), wsc * v[ii]);
       } else {
         tmem_ld32(tm + lane_off + 64 + half * 32, v);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) st_kmajor8(sm + kP1K, c, half * 32 + 8 * e, 128, v + 8 * e);
+        for (int e = 0; e < 4; ++e) st_kmajor8(sm + kP1B, c, half * 32 + 8 * e, 128, v + 8 * e);
       }
     }
   }
@@ -631,9 +664,9 @@ __global__ void __launch_bounds__(kP1Threads, 3)
   tc_fence_before();
   __syncthreads();
   if (tid == 0) {
-    bulk_store(rec + kRecWQ, sm + kP1B, 8192);                // -W rows, channels 0-63
-    bulk_store(rec + kRecWQ + 16384, sm + kP1B + 8192, 8192); // -W rows, channels 64-127
-    bulk_store(rec + kRecU, sm + kP1K, 16384);
+    bulk_store(rec + kRecWQ, sm + kP1A, 8192);                 // -W rows, channels 0-63
+    bulk_store(rec + kRecWQ + 16384, sm + kP1A + 16384, 8192); // -W rows, channels 64-127
+    bulk_store(rec + kRecU, sm + kP1B, 16384);
     bulk_commit();
     bulk_wait_read();
   }
@@ -1262,7 +1295,10 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   if (!attrs_set) {
     for (auto kern : {kda_chunk_prep_kernel<false, false>, kda_chunk_prep_kernel<true, false>,
                       kda_chunk_prep_kernel<false, true>, kda_chunk_prep_kernel<true, true>}) {
-      const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kP1Bytes + 1024);
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kP1Bytes + 1024);
+      if (e != cudaSuccess) return e;
+      // kP1Blocks CTAs per SM need nearly all of the SM's shared memory
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
       if (e != cudaSuccess) return e;
     }
     cudaError_t e;
