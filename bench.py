@@ -513,7 +513,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true", help="skip the gate-variant / fused-prep timings")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
-    ap.add_argument("--backward-calls", type=int, default=5)
+    ap.add_argument("--backward-calls", type=int, default=20)
     ap.add_argument("--cpu-tokens", type=int, default=4096)
     args = ap.parse_args(argv)
     if args.warmup < 3:
