@@ -44,6 +44,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "kda_common.cuh"
 #include "sm100.cuh"
@@ -1291,8 +1292,14 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
                                 int dv, int chunk, int gate, int prep, void* ws, size_t ws_bytes,
                                 cudaStream_t stream, void* const* events) {
   (void)dk, (void)dv, (void)chunk, (void)ws_bytes;
-  static bool attrs_set = false;
-  if (!attrs_set) {
+  // Function attributes belong to each device's context: set them once per
+  // device (one bit per device ordinal; ordinals past 63 set them every call).
+  static std::atomic<unsigned long long> attrs_done{0};
+  int dev = 0;
+  const cudaError_t dev_err = cudaGetDevice(&dev);
+  if (dev_err != cudaSuccess) return dev_err;
+  const unsigned long long dev_bit = dev < 64 ? 1ull << dev : 0ull;
+  if (!(attrs_done.load(std::memory_order_acquire) & dev_bit) || !dev_bit) {
     for (auto kern : {kda_chunk_prep_kernel<false, false>, kda_chunk_prep_kernel<true, false>,
                       kda_chunk_prep_kernel<false, true>, kda_chunk_prep_kernel<true, true>}) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kP1Bytes + 1024);
@@ -1306,7 +1313,7 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCbSmem);
     if (e != cudaSuccess) return e;
-    attrs_set = true;
+    attrs_done.fetch_or(dev_bit, std::memory_order_release);
   }
   CUtensorMap mq, mk, mv, mg, mo;
   memset(&mg, 0, sizeof(mg));  // only the per-channel gate is read through a tensor map
