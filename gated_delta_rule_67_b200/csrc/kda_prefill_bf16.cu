@@ -21,22 +21,29 @@
 // G_r is a reference point inside the chunk (token 31): the products are
 // independent of it, and centring keeps both exponential factors near 1.
 //
-// Two kernels:
-//  1. kda_chunk_prep: one CTA per (sequence, head, chunk), fully parallel.
-//     TMA brings q, k, v, g (64 x 128 bf16 tiles, 128-byte swizzle); the CTA
-//     computes G and the decayed operands, the two score matrices with one
-//     tcgen05 MMA (M=128: rows 0-63 give A_kk, rows 64-127 give A_qk), the
-//     triangular inverse on the CUDA cores in fp32, and W^T, U^T with two
-//     more MMAs.  It writes, per chunk, a record of ready-to-use operand
-//     images (already in the swizzled shared-memory layout the MMA reads):
-//     [-W ; Q+] (128 x 128), A_qk (64 x 64), Kbar (64 x 128), U (64 x 128
-//     plain) and gamma = exp(G_C) (128 fp32).
-//  2. kda_state_pass: one CTA per (sequence, head); walks the chunks in
-//     order with the state S^T (d_v x d_k, fp32) resident in tensor memory.
-//     Per chunk: S0^T -> bf16 operand, S <- gamma*S in place; one MMA gives
-//     [-S0^T W^T | S0^T Q+^T]; V'^T = U^T + first half; then O^T += V'^T A_qk^T
-//     and S^T += V'^T Kbar.  The next chunk's record is prefetched with a
-//     bulk copy while the current one is processed.
+// Kernels:
+//  1. kda_chunk_prep: one CTA per (sequence, head, chunk), fully parallel,
+//     four CTAs per SM.  TMA brings q, k, v, g (64 x 128 bf16 tiles, 128-byte
+//     swizzle); the CTA computes G and the decayed operands, the two score
+//     matrices with one tcgen05 MMA (M=128: rows 0-63 give A_kk, rows 64-127
+//     give A_qk), the triangular inverse in fp32 by 16 x 16 blocks (diagonal
+//     blocks by forward substitution, the others with warp-level tf32
+//     products), and W^T, U^T with two more MMAs.  It writes, per chunk, a
+//     record of ready-to-use operand images (already in the swizzled
+//     shared-memory layout the MMAs read): [-W ; Q+] (128 x 128), A_qk^T
+//     (64 x 64), Kbar (64 x 128), U^T (128 x 64) and gamma = exp(G_C)
+//     (128 fp32).
+//  2. kda_state_pass: walks chunks in order with the state S^T (d_v x d_k,
+//     fp32) resident in tensor memory.  Per chunk: S0^T -> bf16 operand;
+//     P = S0^T (-W)^T; V'^T = U^T + P while S^T is decayed by gamma and
+//     O^T = S0^T Q+^T is formed; then [O^T | S^T] += V'^T [A_qk^T | Kbar].
+//     The next chunk's record is prefetched with bulk copies while the
+//     current one is processed.  One CTA per (sequence, head), or, when few
+//     chains cover many chunks, the chunk-parallel scan: one CTA per group
+//     of chunks and pass (phase 1: offsets and transitions; phase 3: the
+//     outputs from each group's true start state).
+//  3. kda_scan_combine_kernel: chains the groups' affine state maps of the
+//     scan on the tensor cores (one CTA per chain).
 //
 // Everything is transposed relative to the token-major notation above so
 // that every MMA has M = 128 (the d_v or d_k dimension) and each TMEM lane is
