@@ -211,3 +211,30 @@ def test_chunk_backward_with_strong_decay():
     got = chunk_backward(q, k, v, g, beta, 0.25, s0, d_o, d_sT)
     for n in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
         assert _rel(got[n], ref[n]) < 1e-9, n
+
+
+@pytest.mark.parametrize("gate", ["head", "none"])
+def test_scalar_gate_forms(gate):
+    """Gated DeltaNet (one log-gate per token and head, broadcast over the key
+    channels) and DeltaNet (no forgetting, g = 0) through the same chunk
+    equations."""
+    q, k, v, g, beta, s0 = _inputs(9, T=130)
+    g = np.repeat(g[..., :1], g.shape[-1], axis=-1) if gate == "head" else np.zeros_like(g)
+    o_ref, s_ref = oracle.kda_forward(q, k, v, g, beta, 0.25, s0)
+    o, s = chunk_forward(q, k, v, g, beta, 0.25, s0)
+    assert _rel(o, o_ref) < 1e-12 and _rel(s, s_ref) < 1e-12
+
+
+def test_exact_pairwise_form_equals_the_factored_one():
+    """The kernels' exact path forms every decay factor e^{G_i - G_j} (<= 1
+    for j <= i) per pair and channel instead of factoring it around G_r."""
+    q, k, v, g, beta, _ = _inputs(10, strong=True)
+    K, Q, V = _chunk(k[0, :, 0], 0, C, 16), _chunk(q[0, :, 0], 0, C, 16), _chunk(v[0, :, 0], 0, C, 8)
+    bt = beta[0, :C, 0]
+    c = _chunk_operands(K, Q, V, g[0, :C, 0], bt, 0.25, 31)
+    G = c["G"]
+    E = np.exp(G[:, None, :] - G[None, :, :])  # [i, j, channel]
+    Akk = bt[:, None] * np.tril(np.einsum("ic,jc,ijc->ij", K, K, E), -1)
+    Aqk = np.tril(0.25 * np.einsum("ic,jc,ijc->ij", Q, K, E))
+    assert np.all(np.tril(E.max(axis=2)) <= 1.0 + 1e-15)
+    assert _rel(Akk, c["Akk"]) < 1e-12 and _rel(Aqk, c["Aqk"]) < 1e-12
