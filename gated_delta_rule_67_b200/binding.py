@@ -30,6 +30,7 @@ SIGNATURES = {
     "kda_chunk_fwd_profiled": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp, _sz, _vp, _vp]),
     "kda_chunk_fwd_noalloc": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 7 + [_vp]),
     "kda_chunk_fwd_check": (_i, [_vp, _sz, _vp]),
+    "kda_chunk_fwd_noalloc_check": (_i, [_vp]),
     "kda_wait_selftest": (_i, [_vp, _sz, _vp]),
     "kda_recurrent_step": (_i, [_vp] * 5 + [_f, _vp, _vp] + [_i] * 5 + [_vp]),
     "kda_chunk_fwd_ex": (_i, [_vp] * 5 + [_f, _vp, _vp, _vp] + [_i] * 9 + [_vp, _sz, _vp]),
@@ -115,6 +116,13 @@ def _stream(stream, device):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _on(device):
+    """Makes the tensors' device current for the C call: the library keys its
+    per-device set-up (function attributes, the static scratch) by the
+    current device, which must own the buffers and the stream."""
+    return torch.cuda.device(device)
+
+
 def kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16) -> int:
     return int(load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, chunk, _dtype_code(dtype)))
 
@@ -172,14 +180,17 @@ def kda_chunk_fwd(q, k, v, g, beta, scale=None, initial_state=None, *, chunk=64,
     if gate != KDA_GATE_CHANNEL or prep:
         if events is not None:
             raise ValueError("events are recorded for prepared per-channel-gate inputs only")
-        st = lib.kda_chunk_fwd_ex(*args[:16], gate, int(prep), *args[16:])
+        with _on(q.device):
+            st = lib.kda_chunk_fwd_ex(*args[:16], gate, int(prep), *args[16:])
     elif events is None:
-        st = lib.kda_chunk_fwd(*args)
+        with _on(q.device):
+            st = lib.kda_chunk_fwd(*args)
     else:
         if len(events) != 3:
             raise ValueError("events must hold three torch.cuda.Event objects")
         handles = (ctypes.c_void_p * 3)(*[ev.cuda_event for ev in events])
-        st = lib.kda_chunk_fwd_profiled(*args, handles)
+        with _on(q.device):
+            st = lib.kda_chunk_fwd_profiled(*args, handles)
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd")
     return o, final_state
@@ -207,9 +218,10 @@ def kda_chunk_fwd_noalloc(q, k, v, g, beta, scale=None, initial_state=None, *, c
     _check_dev("o", o, q.dtype)
     if final_state is None and output_final_state:
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
-    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
-                                   _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk,
-                                   _dtype_code(q.dtype), _stream(stream, q.device))
+    with _on(q.device):
+        st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                       _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv, chunk,
+                                       _dtype_code(q.dtype), _stream(stream, q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd_noalloc")
     return o, final_state
@@ -219,8 +231,18 @@ def kda_chunk_fwd_check(workspace, stream=None) -> int:
     """Status word a bounded on-device wait may have left in ``workspace`` (synchronises)."""
     if workspace is None:
         return KDA_OK
-    return int(load().kda_chunk_fwd_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
-                                          _stream(stream, workspace.device)))
+    with _on(workspace.device):
+        return int(load().kda_chunk_fwd_check(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                              _stream(stream, workspace.device)))
+
+
+def kda_chunk_fwd_noalloc_check(device=None, stream=None) -> int:
+    """Status word of the static scratch after kda_chunk_fwd_noalloc calls on
+    ``device`` (default: the current device); synchronises.  KDA_OK, or
+    KDA_ERR_TIMEOUT if a bounded on-device wait of the last call gave up."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with _on(device):
+        return int(load().kda_chunk_fwd_noalloc_check(_stream(stream, device)))
 
 
 def kda_wait_selftest(workspace, stream=None) -> int:
@@ -228,7 +250,8 @@ def kda_wait_selftest(workspace, stream=None) -> int:
     kda_chunk_fwd_check reads afterwards (KDA_ERR_TIMEOUT when the mechanism works)."""
     lib = load()
     nbytes = workspace.numel() * workspace.element_size()
-    st = lib.kda_wait_selftest(_ptr(workspace), nbytes, _stream(stream, workspace.device))
+    with _on(workspace.device):
+        st = lib.kda_wait_selftest(_ptr(workspace), nbytes, _stream(stream, workspace.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_wait_selftest")
     return kda_chunk_fwd_check(workspace, stream)
@@ -262,10 +285,11 @@ def kda_recurrent_step(q, k, v, g, beta, state, scale=None, *, o=None, stream=No
     _check_dev("o", o, q.dtype)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(state), _ptr(o), N, H, dk, dv,
             _dtype_code(q.dtype))
-    if gate == KDA_GATE_CHANNEL and not prep:
-        st = lib.kda_recurrent_step(*args, _stream(stream, q.device))
-    else:
-        st = lib.kda_recurrent_step_ex(*args, gate, int(prep), _stream(stream, q.device))
+    with _on(q.device):
+        if gate == KDA_GATE_CHANNEL and not prep:
+            st = lib.kda_recurrent_step(*args, _stream(stream, q.device))
+        else:
+            st = lib.kda_recurrent_step_ex(*args, gate, int(prep), _stream(stream, q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_recurrent_step")
     return o
@@ -309,10 +333,11 @@ def kda_backward(q, k, v, g, beta, grad_o, scale=None, initial_state=None, grad_
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.kda_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
-                             _ptr(grad_o), _ptr(grad_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
-                             _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, dk, dv, code, gate,
-                             int(prep), _ptr(workspace), ws_bytes, _stream(stream, q.device))
+    with _on(q.device):
+        st = lib.kda_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(initial_state),
+                                 _ptr(grad_o), _ptr(grad_final_state), _ptr(out["dq"]), _ptr(out["dk"]),
+                                 _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, dk,
+                                 dv, code, gate, int(prep), _ptr(workspace), ws_bytes, _stream(stream, q.device))
     if st != KDA_OK:
         raise KDAError(st, "kda_backward")
     return out

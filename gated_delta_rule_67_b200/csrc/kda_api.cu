@@ -29,7 +29,7 @@ bool prefill_supported(int dk, int dv, int chunk, int dtype) {
   if (dtype == KDA_F32)
     return (dk == 64 || dk == 128) && (dv == 64 || dv == 128) &&
            (chunk == 16 || chunk == 32 || chunk == 64);
-  return dk == 128 && dv == 128 && chunk == 64;
+  return (dk == 64 || dk == 128) && (dv == 64 || dv == 128) && chunk == 64;
 }
 
 }  // namespace

@@ -24,6 +24,9 @@
 //    on it and must be serialised by the caller.  The parts that must start
 //    at zero (the error word) are cleared on every call; everything else is
 //    fully rewritten before it is read.
+//  * A bounded wait that gave up inside a kernel is recorded in the error
+//    word at the start of the scratch; kda_chunk_fwd_noalloc_check reads it
+//    (the caller has no other way to reach the array).
 #include <mutex>
 
 #include "kda_common.cuh"
@@ -68,4 +71,10 @@ extern "C" KDA_API kda_status kda_chunk_fwd_noalloc(const void* q, const void* k
   if (scratch_address(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
   return kda_chunk_fwd(q, k, v, g, beta, scale, initial_state, o, final_state, B, T, H, dk, dv, chunk, dtype,
                        scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" KDA_API kda_status kda_chunk_fwd_noalloc_check(void* stream) {
+  void* scratch = nullptr;
+  if (scratch_address(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+  return kda_chunk_fwd_check(scratch, kNoAllocScratchBytes, stream);
 }

@@ -741,15 +741,21 @@ __device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, 
 // M_g (S_end = M_g S_start + R_g, the map is affine in S_start); phase 3 runs
 // every group again from its true start state S_g (computed in between by
 // kda_scan_combine_kernel) and writes the outputs.
+// The caller's states are [B*H][dk][dv] (dk, dv in {64, 128}); inside the
+// kernels every state is 128 x 128, the channels past dk (dv) being zero.
+// The scan buffers use that internal layout: R_g in rbuf, the transitions
+// in mbuf, and in sbuf the start state of group 0 (slot 0, copied there by
+// phase 1, so that phase 3 never reads the caller's initial state, which
+// the caller's final state may overwrite) and of groups 2..G-1.
 struct StatePassArgs {
   const uint8_t* records;
   WorkspaceHeader* hdr;
-  const float* s0;  // [B*H][128][128] or null (zero)
-  float* sT;        // [B*H][128][128] or null
+  const float* s0;  // [B*H][dk][dv] or null (zero)
+  float* sT;        // [B*H][dk][dv] or null
   float* rbuf;      // [B*H][G][128][128] scan buffers
   float* mbuf;      // transition matrices: [B*H][G] slots of 64 KiB, each the 32 KiB bf16 K-major image of M_g
-  const float* sbuf;
-  int T, H, NC, G, L, phase;
+  float* sbuf;
+  int T, H, NC, G, L, phase, dk, dv;
 };
 
 __global__ void __launch_bounds__(kSPThreads, 1)
@@ -764,16 +770,21 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   const int H = args.H, NC = args.NC, G = args.G, L = args.L;
   constexpr size_t kSt = (size_t)kD * kD;
   // ---- role of this CTA
+  const int dk = args.dk, dv = args.dv;
+  const size_t kUserSt = (size_t)dk * dv;
   int bh, cb, ce;
   const float* init = nullptr;  // null: zero start
   bool ident = false, zero_u = false, out = true;
+  bool init_user = false, fin_user = false;  // caller's [dk][dv] layout (else the internal 128 x 128)
   float* fin = nullptr;
+  float* init_copy = nullptr;  // phase 1, group 0: the start state is also kept in sbuf slot 0
   if (args.phase == 0) {
     bh = blockIdx.x;
     cb = 0;
     ce = NC;
-    init = args.s0 ? args.s0 + bh * kSt : nullptr;
-    fin = args.sT ? args.sT + bh * kSt : nullptr;
+    init = args.s0 ? args.s0 + bh * kUserSt : nullptr;
+    fin = args.sT ? args.sT + bh * kUserSt : nullptr;
+    init_user = fin_user = true;
   } else if (args.phase == 1) {
     const int per = 2 * G - 3;
     bh = blockIdx.x / per;
@@ -782,7 +793,9 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     int g;
     if (r < G - 1) {
       g = r;
-      init = (g == 0 && args.s0) ? args.s0 + bh * kSt : nullptr;
+      init = (g == 0 && args.s0) ? args.s0 + bh * kUserSt : nullptr;
+      init_user = true;
+      if (g == 0 && args.s0) init_copy = args.sbuf + (size_t)bh * G * kSt;
       fin = args.rbuf + ((size_t)bh * G + g) * kSt;
     } else {
       g = r - (G - 1) + 1;
@@ -797,11 +810,12 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     const int g = blockIdx.x % G;
     cb = g * L;
     ce = min(NC, cb + L);
-    // group 0 starts from the initial state, group 1 from R_0; later ones from
-    // the combination kernel's output
-    init = g == 0 ? (args.s0 ? args.s0 + (size_t)bh * kSt : nullptr)
+    // group 0 starts from the initial state (its copy in sbuf slot 0), group 1
+    // from R_0; later ones from the combination kernel's output
+    init = g == 0 ? (args.s0 ? args.sbuf + (size_t)bh * G * kSt : nullptr)
                   : g == 1 ? args.rbuf + (size_t)bh * G * kSt : args.sbuf + ((size_t)bh * G + g) * kSt;
-    fin = (g == G - 1 && args.sT) ? args.sT + bh * kSt : nullptr;
+    fin = (g == G - 1 && args.sT) ? args.sT + bh * kUserSt : nullptr;
+    fin_user = true;
   }
   const int NCL = ce - cb;  // chunks this CTA walks
   const int h = bh % H, b = bh / H;
@@ -823,9 +837,9 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     mbar_init(&bar_init, 1);
     fence_mbar_init();
     if (init) {  // the start state, row-major fp32, into stage 1 (its record follows once it is read)
-      mbar_expect_tx(&bar_init, kD * kD * sizeof(float));
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
+      const uint32_t bytes = (uint32_t)((init_user ? kUserSt : kSt) * sizeof(float));  // 16, 32 or 64 KiB
+      mbar_expect_tx(&bar_init, bytes);
+      for (uint32_t p = 0; p < bytes / 16384; ++p)
         bulk_load(sm + kStage + p * 16384, init + p * 4096, 16384, &bar_init);
     }
   }
@@ -923,7 +937,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       if (tid == 128) {
         const uint8_t* src = sm + kP2Out + (n & 1) * 16384;
         tma_store_4d(&tm_o, src, 0, h, (cb + n) * kC, b);
-        tma_store_4d(&tm_o, src + 8192, 64, h, (cb + n) * kC, b);
+        if (dv > 64) tma_store_4d(&tm_o, src + 8192, 64, h, (cb + n) * kC, b);
         bulk_commit();
       }
     }
@@ -942,7 +956,13 @@ __global__ void __launch_bounds__(kSPThreads, 1)
 #pragma unroll
         for (int ii = 0; ii < 32; ++ii) {
           const int c = q * 32 + ii;
-          v[ii] = init ? s0s[c * kD + j] : (ident && c == j ? 1.f : 0.f);
+          if (!init)
+            v[ii] = ident && c == j ? 1.f : 0.f;
+          else if (init_user)
+            v[ii] = (c < dk && j < dv) ? s0s[c * dv + j] : 0.f;
+          else
+            v[ii] = s0s[c * kD + j];
+          if (init_copy) init_copy[(size_t)c * kD + j] = v[ii];
         }
         tmem_st32(tm + kTmS + lane_off + q * 32, v);
       }
@@ -1048,6 +1068,12 @@ __global__ void __launch_bounds__(kSPThreads, 1)
           uint8_t* img = reinterpret_cast<uint8_t*>(fin);
 #pragma unroll
           for (int ii = 0; ii < 32; ++ii) stbf(img, kmajor_off(q * 32 + ii, j, kD), v[ii]);
+        } else if (fin_user) {
+          if (j < dv) {
+#pragma unroll
+            for (int ii = 0; ii < 32; ++ii)
+              if (q * 32 + ii < dk) fin[(size_t)(q * 32 + ii) * dv + j] = v[ii];
+          }
         } else {
 #pragma unroll
           for (int ii = 0; ii < 32; ++ii) fin[(size_t)(q * 32 + ii) * kD + j] = v[ii];
@@ -1215,11 +1241,14 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 // [B, T, H, 128] bf16 viewed as a 4-D tensor (channel, head, token, batch);
 // box = 64 channels x 1 head x 64 tokens, 128-byte swizzle; tokens past T
 // read as zeros.
-bool make_map(CUtensorMap* map, const void* base, int B, int T, int H, bool swizzle = true) {
+// With d = 64 the box at channel 64 lies wholly outside the tensor and reads
+// as zeros: the kernels then run on 128 channels of which the last 64 are
+// zero (a zero key, query or value channel and a zero log-gate add nothing).
+bool make_map(CUtensorMap* map, const void* base, int B, int T, int H, int d, bool swizzle = true) {
   auto enc = get_encode();
   if (!enc) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)T * H * kD * 2};
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
   cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
@@ -1298,7 +1327,7 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
                                 float scale, const float* s0, bf16* o, float* sT, int B, int T, int H, int dk,
                                 int dv, int chunk, int gate, int prep, void* ws, size_t ws_bytes,
                                 cudaStream_t stream, void* const* events) {
-  (void)dk, (void)dv, (void)chunk, (void)ws_bytes;
+  (void)chunk, (void)ws_bytes;
   // Function attributes belong to each device's context: set them once per
   // device (one bit per device ordinal; ordinals past 63 set them every call).
   static std::atomic<unsigned long long> attrs_done{0};
@@ -1324,8 +1353,8 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   }
   CUtensorMap mq, mk, mv, mg, mo;
   memset(&mg, 0, sizeof(mg));  // only the per-channel gate is read through a tensor map
-  if (!make_map(&mq, q, B, T, H) || !make_map(&mk, k, B, T, H) || !make_map(&mv, v, B, T, H) ||
-      (gate == KDA_GATE_CHANNEL && !make_map(&mg, g, B, T, H)) || !make_map(&mo, o, B, T, H, false))
+  if (!make_map(&mq, q, B, T, H, dk) || !make_map(&mk, k, B, T, H, dk) || !make_map(&mv, v, B, T, H, dv) ||
+      (gate == KDA_GATE_CHANNEL && !make_map(&mg, g, B, T, H, dk)) || !make_map(&mo, o, B, T, H, dv, false))
     return cudaErrorInvalidValue;
   const int NC = (T + kC - 1) / kC;
   WorkspaceHeader* hdr = static_cast<WorkspaceHeader*>(ws);
@@ -1344,7 +1373,7 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e != cudaSuccess) return e;
-  StatePassArgs a{records, hdr, s0, sT, nullptr, nullptr, nullptr, T, H, NC, 1, NC, 0};
+  StatePassArgs a{records, hdr, s0, sT, nullptr, nullptr, nullptr, T, H, NC, 1, NC, 0, dk, dv};
   const int BH = B * H;
   int G, L;
   scan_groups(BH, NC, &G, &L);

@@ -20,7 +20,9 @@
  *  - `dtype` is the element type of q, k, v, g, beta and o (fp32 or bf16);
  *    the state is always fp32.  bf16 results are rounded to nearest-even.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
- *    Calls only enqueue work on it; none synchronises the host.
+ *    Calls only enqueue work on it; none synchronises the host.  The device
+ *    that owns the buffers and the stream must be the current device of the
+ *    calling thread (per-device set-up is keyed by cudaGetDevice).
  *  - Arguments are validated on the host before anything is launched; a
  *    rejected call enqueues nothing.  No call raises an exception across the
  *    ABI and no kernel uses device assertions.
@@ -131,8 +133,9 @@ KDA_API int kda_chunk_fwd_launch_count(int B, int T, int H, int dk, int dv, int 
  *                   on entry do not matter; it must not be shared by two
  *                   calls in flight at the same time
  *
- * Supported: dtype KDA_F32 with dk, dv in {64, 128} (any chunk in {16, 32, 64});
- * dtype KDA_BF16 with dk = dv = 128 and chunk = 64.  Anything else with valid
+ * Supported: dk, dv in {64, 128}; dtype KDA_F32 with any chunk in {16, 32,
+ * 64}, dtype KDA_BF16 with chunk = 64 (the bf16 kernels run 128 channels, a
+ * 64-channel input being zero-padded on the fly).  Anything else with valid
  * shapes returns KDA_ERR_UNSUPPORTED.  T = 0 or B = 0 is valid (the final state
  * is the initial state).
  */
@@ -273,6 +276,16 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const voi
                                          const void* beta, float scale, const float* initial_state, void* o,
                                          float* final_state, int B, int T, int H, int dk, int dv, int chunk,
                                          int dtype, void* stream);
+
+/*
+ * The on-device error word of the static scratch used by
+ * kda_chunk_fwd_noalloc (synchronises `stream`): KDA_OK, or KDA_ERR_TIMEOUT
+ * if a bounded wait inside a kernel of the last kda_chunk_fwd_noalloc call on
+ * the current device gave up (that call's outputs are then not valid).  It is
+ * the kda_chunk_fwd_check of that path, whose scratch the caller cannot name.
+ * No counterpart on the pages.  Allocates nothing.
+ */
+KDA_API kda_status kda_chunk_fwd_noalloc_check(void* stream);
 
 /*
  * Reads the on-device error word that the last kda_chunk_fwd using this

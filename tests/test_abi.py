@@ -46,6 +46,9 @@ def test_workspace_size_rejects_bad_args(lib):
     assert f(-1, 64, 1, 128, 128, 64, 1) == 0     # bad B
     assert f(1, 64, 1, 96, 96, 64, 1) == 0        # unsupported d
     assert f(1, 64, 1, 64, 64, 64, 0) == 0        # fp32 path needs none
+    # bf16 takes d in {64, 128} (64 channels zero-padded inside the kernels): the same workspace
+    assert f(1, 64, 1, 64, 64, 64, 1) == f(1, 64, 1, 128, 128, 64, 1) > 0
+    assert f(1, 64, 1, 64, 128, 64, 1) > 0
 
 
 # Fake device addresses: validation must fail before any CUDA call is made.

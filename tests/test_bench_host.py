@@ -74,3 +74,19 @@ def test_reference_arm_silent_on_other_ranks(monkeypatch):
 def test_warmup_floor():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2"])
+
+
+def test_reference_arm_config_keys_match_ours():
+    """Both arms describe the workload with the same config keys."""
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3", "--workload", TINY_F32.name])
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["config"] == bench.bench_config(TINY_F32, 1)
+    assert {"workload", "l2", "parallelism"} <= set(line["config"])
+
+
+def test_hbm_fractions_flag_readings_above_the_measured_copy():
+    peaks = {"hbm_gbs": 6000.0}
+    assert bench.hbm_fracs(3000.0, peaks) == {"frac": 0.5, "frac_nominal": 3000.0 / bench.NOMINAL_HBM_GBS}
+    assert bench.hbm_fracs(6500.0, peaks)["above_measured_peak"] is True
