@@ -341,6 +341,10 @@ def run_ours(args, cfg):
     # between two kernels would hold the second one back until the first has
     # drained); the prep / state-pass split comes from separate profiled calls.
     split_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(min(args.steps, 10))]
+    for trip in split_evs:  # materialise the event handles before the library records them
+        for e in trip:
+            e.record(stream)
+    torch.cuda.synchronize()
     for trip in split_evs:
         flush.zero_()
         case.call(trip)
