@@ -46,8 +46,9 @@ def test_in_place_state_and_split_calls():
     o1, _ = kda_chunk_fwd(*(part(n, 0, cut) for n in ("q", "k", "v", "g", "beta")), None, state, final_state=state)
     o2, _ = kda_chunk_fwd(*(part(n, cut, 150) for n in ("q", "k", "v", "g", "beta")), None, state, final_state=state)
     torch.cuda.synchronize()
-    assert rel_err(torch.cat([o1, o2], dim=1), o_full) < 1e-6
-    assert rel_err(state, s_full) < 1e-6
+    # the cut at token 61 moves every later chunk boundary, so the two runs round differently (fp32)
+    assert rel_err(torch.cat([o1, o2], dim=1), o_full) < 1e-5
+    assert rel_err(state, s_full) < 1e-5
 
 
 def test_empty_sequence_copies_state():
@@ -60,3 +61,36 @@ def test_empty_sequence_copies_state():
     o, sT = kda_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, None)
     torch.cuda.synchronize()
     assert torch.count_nonzero(sT) == 0
+
+
+@pytest.mark.parametrize("dk", [64, 128])
+def test_chunk_size_changes_the_arithmetic_not_the_result(dk):
+    """The fp32 path evaluates the chunk form with the caller's chunk size:
+    C in {16, 32, 64} must agree with one another far inside the tolerance,
+    each must meet the oracle, and they must not be bit-identical (the chunk
+    size really selects a different evaluation)."""
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(1, 200, 2, dk, dk, torch.float32, 0.1, seed=34 + dk, device="cpu")
+    res = {c: _check(x, dev, chunk=c) for c in (16, 32, 64)}
+    for c in (16, 32):
+        assert rel_err(res[c][0], res[64][0]) < 1e-5 and rel_err(res[c][1], res[64][1]) < 1e-5
+    assert not torch.equal(res[16][0], res[64][0])
+
+
+@pytest.mark.parametrize("gate", ["head", "none"])
+def test_scalar_gates_chunked(gate):
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(1, 100, 2, 64, 64, torch.float32, 0.1, seed=36, device="cpu")
+    if gate == "head":
+        x["g"] = x["g"][..., 0].contiguous()
+        ref = dict(x, g=x["g"].unsqueeze(-1).expand(-1, -1, -1, 64).contiguous())
+    else:
+        x["g"] = None
+        ref = dict(x, g=torch.zeros(1, 100, 2, 64))
+    ref_o, ref_s = oracle.kda_forward(ref["q"], ref["k"], ref["v"], ref["g"], ref["beta"], 64 ** -0.5,
+                                      ref["initial_state"])
+    for c in (16, 64):
+        o, sT = kda_chunk_fwd(*(None if x[n] is None else x[n].to(dev) for n in ("q", "k", "v", "g", "beta")), None,
+                              x["initial_state"].to(dev), chunk=c)
+        torch.cuda.synchronize()
+        assert rel_err(o, ref_o) < TOL[torch.float32] and rel_err(sT, ref_s) < TOL[torch.float32]
