@@ -63,43 +63,41 @@ using namespace sm100;
 using bf16 = __nv_bfloat16;
 
 constexpr int kC = 64;    // chunk length
-constexpr int kD = 128;   // channels inside the kernels (d_k = d_v = 64 inputs are zero-padded)
-constexpr int kRefTok = 31;  // reference token of the factored form: the last token of the second 16-token quarter
-static_assert(kRefTok == 2 * 16 - 1, "the prep kernel takes G_r as the sum of the first two quarter totals");
+constexpr int kD = 128;   // d_k = d_v
+constexpr int kRefTok = 31;  // reference token of the factored form: the end of the second 16-token stride
+static_assert(kRefTok == 2 * 16 - 1, "pass 1 takes G_r as the sum of the first two stride totals");
 
 // --- per-chunk record in the workspace (byte offsets) -----------------------
-// Every image is a stack of 128-byte rows of 64 bf16 tokens in the canonical
-// 128-byte swizzle: element (row r, token t) at r*128 + ((t/8 ^ r%8) << 4) +
-// (t%8)*2.  The rows are key channels, value channels or query tokens, so the
-// preparation kernel writes each row as four contiguous 16-byte pieces.
-constexpr uint32_t kRecW = 0;           // -W^T: row = key channel; MN-major B of P = S0^T (-W)^T (16 KiB)
-constexpr uint32_t kRecQ = 16384;       // Q+^T: row = key channel; MN-major B of O^T = S0^T Q+^T (16 KiB)
-constexpr uint32_t kRecAqk = 32768;     // A_qk: row = query token i, column = key token j (8 KiB)
-constexpr uint32_t kRecKbar = 40960;    // Kbar^T: row = key channel (16 KiB)
-// [A_qk | Kbar^T] = 192 rows read as one K-major B operand (N = 64 + 128, K = 64 tokens).
-constexpr uint32_t kRecU = 57344;       // U^T: row = value channel (16 KiB)
-constexpr uint32_t kRecGamma = 73728;   // gamma = exp(G_C): 128 fp32
+constexpr uint32_t kRecWQ = 0;          // [-W ; Q+]: K-major, 128 rows x 128 ch (32 KiB)
+constexpr uint32_t kRecAqk = 32768;     // A_qk^T: token-row tile, row j, column i (8 KiB)
+constexpr uint32_t kRecKbar = 40960;    // Kbar: token-row tile 64 x 128 (16 KiB)
+// [A_qk^T | Kbar] = 24 KiB read as one MN-major B operand (N = 64 + 128, LBO 8 KiB).
+constexpr uint32_t kRecU = 57344;       // U^T: K-major, 128 rows (channel) x 64 (token) (16 KiB)
+constexpr uint32_t kRecGamma = 73728;   // gamma: 128 fp32
 constexpr uint32_t kRecBytes = 74240;
 
-// --- prep kernel: shared memory (byte offsets from a 1024-aligned base), 64 KiB
-// R1, R2, R3 first hold the g, k, q tiles as TMA lands them (token rows: 64
-// tokens x 64 channels per 8 KiB half).  Once every thread has read its
-// channels of them into registers, they are overwritten by the channel-row
-// images K+_r^T (R1), K-_r^T (R2) and Q+_r^T (R3): [R1 | R3] is the score
-// product's MN-major A operand (M = 2 x 64 tokens, LBO 32 KiB), R2 its B
-// operand, and R1 later the K-major A operand of the W product.  After the
-// score product, R2 and R3 hold the A_kk and T blocks and (T diag beta)^T.
-// On the exact path R1 stages G in fp32 (one 64-channel half at a time)
-// before it takes K+^T.
-constexpr uint32_t kP1R1 = 0;
-constexpr uint32_t kP1R2 = 16384;
-constexpr uint32_t kP1R3 = 32768;
-constexpr uint32_t kP1V = 49152;     // v tile: MN-major A of U^T = V^T (T diag beta)^T (LBO 8 KiB)
-constexpr uint32_t kP1Blk = 16384;   // A_kk blocks [16K, 26K), T blocks [26K, 36K) (fp32 16 x 16)
-constexpr uint32_t kP1B2 = 36864;    // (T diag beta)^T: K-major 64 x 64 (8 KiB)
-constexpr uint32_t kP1Bytes = 65536;
+// --- prep kernel: shared memory (byte offsets from a 1024-aligned base) ---
+// 52 KiB, so that four CTAs share an SM.
+// Region A (32 KiB) is a 128-row K-major tile in two 64-channel halves of
+// 16 KiB.  Rows 0-63 of each half ([0,8K) and [16K,24K)) first hold g, then
+// K+_r, which stays for the W product and is finally overwritten by the -W
+// staging tile; rows 64-127 ([8K,16K) and [24K,32K)) hold q, then Q+_r.
+// Once the score MMA is done, the v tile takes [8K,16K) and [24K,32K) (a
+// 64-row tile whose channel halves lie 16 KiB apart); its second half comes
+// after the A_qk^T staging tile at [24K,32K) has been bulk-stored.
+// Region B (16 KiB): the k tile, turned in place into K-_r (score B operand);
+// then the 10 A_kk blocks [0,10K) and six T blocks [10K,16K); after the
+// solve the (T diag beta)^T operand [0,8K); finally the U^T staging tile.
+// Region T (4 KiB): the last four T blocks.
+constexpr uint32_t kP1A = 0;
+constexpr uint32_t kP1B = 32768;
+constexpr uint32_t kP1T = 49152;
+constexpr uint32_t kP1Bytes = 53248;
+constexpr uint32_t kP1V = kP1A + 8192;       // v tile (half stride 16 KiB), after the score MMA
+constexpr uint32_t kP1B2 = kP1B;             // (T diag beta)^T, K-major 64 x 64, after the solve
+constexpr uint32_t kP1QT = kP1A + 24576;     // A_qk^T staging (bulk-stored before v's second half lands)
 constexpr int kP1Threads = 256;
-constexpr int kP1Blocks = 3;         // CTAs per SM: 3 x 128 TMEM columns, 3 x ~68 KiB shared memory
+constexpr int kP1Blocks = 4;                 // CTAs per SM: 4 x 128 TMEM columns, 4 x ~55 KiB shared memory
 // Per-chunk safe range of the factored form: every channel's cumulative
 // log-gate over the chunk must stay above -kSafeSpan, so that each factor
 // exp(+-(G_i - G_r)), exp(G_r), exp(G_C - G_r) lies in [e^-64, e^64].
@@ -122,11 +120,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
 }
-__device__ __forceinline__ float2 unpack2(uint32_t w) {
-  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
-}
-// Byte offset of the 16-byte piece holding tokens 8p .. 8p+7 of row r of an image.
-__device__ __forceinline__ uint32_t row_piece(uint32_t r, uint32_t p) { return r * 128 + ((p ^ (r & 7)) << 4); }
 // 8 consecutive K elements (k0 % 8 == 0) of row r of a K-major tile: one 16-byte store.
 __device__ __forceinline__ void st_kmajor8(uint8_t* tile, uint32_t r, uint32_t k0, uint32_t rows, const float* v) {
   uint4 w = make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
@@ -144,17 +137,32 @@ __device__ __forceinline__ void wait_or_flag(uint64_t* bar, uint32_t parity, Wor
 __device__ __forceinline__ float2 ld_bf2(const uint8_t* p) {
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
 }
+// 8 bf16 (16 bytes, 16-byte aligned) <-> 8 floats.
+__device__ __forceinline__ void ld8(const uint8_t* p, float* f) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+    f[2 * e] = t.x;
+    f[2 * e + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void st8(uint8_t* p, const float* f) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+}
 // The lower-triangular 64 x 64 matrices A_kk and T are kept as 16 x 16 fp32
-// blocks (I, J), J <= I, numbered p = I(I+1)/2 + J; A blocks at kP1Blk, T
-// blocks 10 KiB after them.
+// blocks (I, J), J <= I, numbered p = I(I+1)/2 + J; A blocks in region B,
+// T blocks 0-5 after them in region B and T blocks 6-9 in region T.
 __device__ __forceinline__ int blk(int I, int J) { return I * (I + 1) / 2 + J; }
 // Element (r, c) of a 16 x 16 block: rows of 16 floats with the float4 column
 // XOR-ed by (r/2)%4, so that 8 consecutive rows at one float4 column hit 8
 // different 16-byte bank groups.
 __device__ __forceinline__ int bidx(int r, int c) { return r * 16 + ((((c >> 2) ^ ((r >> 1) & 3)) << 2) | (c & 3)); }
-__device__ __forceinline__ float* a_blk(uint8_t* sm, int p) { return reinterpret_cast<float*>(sm + kP1Blk) + p * 256; }
+__device__ __forceinline__ float* a_blk(uint8_t* sm, int p) { return reinterpret_cast<float*>(sm + kP1B) + p * 256; }
 __device__ __forceinline__ float* t_blk(uint8_t* sm, int p) {
-  return reinterpret_cast<float*>(sm + kP1Blk + 10240) + p * 256;
+  return p < 6 ? reinterpret_cast<float*>(sm + kP1B + 10240) + p * 256
+               : reinterpret_cast<float*>(sm + kP1T) + (p - 6) * 256;
 }
 // Warp-level 16x16x16 product acc += P Q of row-major fp32 16x16 blocks, with
 // mma.sync m16n8k8 (tf32 operands rounded to nearest).  acc[nh] holds the
@@ -193,20 +201,12 @@ __device__ __forceinline__ void store_block_frag(float* X, const float (&acc)[2]
   }
 }
 
-// One chunk of one (sequence, head) per CTA.  kScalarGate: the forget gate
-// is one log-gate per (token, head) read from g_head (Gated DeltaNet), or none
-// when g_head is null (DeltaNet); otherwise the per-channel g tile comes in
-// by TMA (KDA).  kPrep: the inputs are raw and `prep` (kda_prep bits) says
-// which ones to prepare here: q, k scaled to unit length per token,
-// log-sigmoid of g, sigmoid of beta.
-//
-// The elementwise work runs channel by channel: thread (warp w, lane l) owns
-// key channels c0 = 64 (w % 2) + 2 l and c0 + 1 over the 16 tokens of
-// quarter w / 2.  It reads them from the token-row tiles (one 32-bit word per
-// token), forms the cumulative log-gate G in registers (a running sum over its
-// quarter plus the totals of the quarters before it), and writes its two
-// channel rows of every image as 16-byte pieces.  The products (scores, W, U)
-// run on the tensor cores; the triangular inverse by 16 x 16 blocks.
+// kScalarGate: the forget gate is one log-gate per (token, head) read from
+// g_head (Gated DeltaNet), or none when g_head is null (DeltaNet); otherwise
+// the per-channel g tile comes in by TMA (KDA).  kPrep: the inputs are raw
+// and `prep` (kda_prep bits) says which ones to prepare here: q, k scaled to
+// unit length per token (the per-token factors are applied wherever q and k
+// are read), log-sigmoid of g, sigmoid of beta.
 template <bool kScalarGate, bool kPrep>
 __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -220,8 +220,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   __shared__ float sbeta[kC];
   __shared__ float sgh[kScalarGate ? kC : 1];  // per-head log-gates of the chunk (zeros without a gate)
   __shared__ float snq[kPrep ? kC : 1], snk[kPrep ? kC : 1];  // per-token sums of q^2, k^2 (fused L2 norm)
-  __shared__ __align__(16) float segr[kD];  // per channel: exp(G_r) (factored form) or 1 (exact path); scales W in its extraction
-  __shared__ __align__(16) float stot[4][kD];  // per token quarter and channel: the quarter's sum of log-gates
+  __shared__ float segr[kD];  // per channel: exp(G_r) (factored form) or 1 (exact path); scales W in its extraction
   const bool l2n = kPrep && (prep & KDA_PREP_L2NORM_QK);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -240,13 +239,10 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     mbar_expect_tx(&bar_in, (kScalarGate ? 2 : 3) * 16384);
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb) {
-      if (!kScalarGate) tma_load_4d(sm + kP1R1 + kb * 8192, &tm_g, &bar_in, kb * 64, h, t0, b);
-      tma_load_4d(sm + kP1R2 + kb * 8192, &tm_k, &bar_in, kb * 64, h, t0, b);
-      tma_load_4d(sm + kP1R3 + kb * 8192, &tm_q, &bar_in, kb * 64, h, t0, b);
+      if (!kScalarGate) tma_load_4d(sm + kP1A + kb * 16384, &tm_g, &bar_in, kb * 64, h, t0, b);  // rows 0-63
+      tma_load_4d(sm + kP1A + kb * 16384 + 8192, &tm_q, &bar_in, kb * 64, h, t0, b);     // rows 64-127
+      tma_load_4d(sm + kP1B + kb * 8192, &tm_k, &bar_in, kb * 64, h, t0, b);
     }
-    mbar_expect_tx(&bar_v, 16384);
-#pragma unroll
-    for (int kb = 0; kb < 2; ++kb) tma_load_4d(sm + kP1V + kb * 8192, &tm_v, &bar_v, kb * 64, h, t0, b);
   }
   if (warp == 0) tmem_alloc(&tmem_base, 128);
   if (tid < kC) {
@@ -271,129 +267,136 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   const uint32_t tm = tmem_base;
   wait_or_flag(&bar_in, 0, hdr, 1);
 
-  // ---- read: channels c0, c0+1 of this thread's 16 tokens, and the cumulative log-gate
-  const int hf = warp & 1, tq = warp >> 1, c0 = 64 * hf + 2 * lane;
-  // byte offset of the word (channels c0, c0+1) of token t inside a 64 x 128 token-row tile
-  auto word_off = [&](int t) -> uint32_t {
-    return (uint32_t)(hf * 8192 + t * 128 + ((((lane >> 2) ^ (t & 7))) << 4) + 4 * (lane & 3));
-  };
-  float G[16][2];
-  uint32_t kw[16], qw[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int t = 16 * tq + i;
-    const uint32_t o = word_off(t);
-    kw[i] = *reinterpret_cast<const uint32_t*>(sm + kP1R2 + o);
-    qw[i] = *reinterpret_cast<const uint32_t*>(sm + kP1R3 + o);
-    if (!kScalarGate) {
-      const float2 gg = unpack2(*reinterpret_cast<const uint32_t*>(sm + kP1R1 + o));
-      G[i][0] = gg.x;
-      G[i][1] = gg.y;
-      if (kPrep && (prep & KDA_PREP_GATE_LOGSIGMOID)) {  // padding keeps g = 0 (no decay)
-        G[i][0] = t < L ? log_sigmoid_fast(G[i][0]) : 0.f;
-        G[i][1] = t < L ? log_sigmoid_fast(G[i][1]) : 0.f;
-      }
-    } else {  // one log-gate per token for every channel (zero without a gate)
-      G[i][0] = G[i][1] = sgh[t];
-    }
-  }
-#pragma unroll
-  for (int i = 1; i < 16; ++i) {
-    G[i][0] += G[i - 1][0];
-    G[i][1] += G[i - 1][1];
-  }
-  *reinterpret_cast<float2*>(&stot[tq][c0]) = make_float2(G[15][0], G[15][1]);
+  // ---- pass 1: in-chunk cumulative log-gate.  Thread = (8-channel group cg,
+  // token lane tg) owning tokens tg, tg+16, tg+32, tg+48: the 8 lanes of a
+  // quarter-warp then touch rows of 8 different swizzle phases (no bank
+  // conflicts).  Inclusive scans over the 16 lanes of each token stride,
+  // then the stride totals are added in order.
+  const int cg = 2 * warp + (lane >> 4);
+  const int tg = lane & 15;
+  const int c8 = 8 * cg;
+  float G[4][8], gref[8], gend[8];
   if (l2n) {  // per-token sums of squares of q and k over the 128 channels
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float2 k2 = unpack2(kw[i]), q2 = unpack2(qw[i]);
-      atomicAdd(&snk[16 * tq + i], fmaf(k2.x, k2.x, k2.y * k2.y));
-      atomicAdd(&snq[16 * tq + i], fmaf(q2.x, q2.x, q2.y * q2.y));
-    }
-  }
-  __syncthreads();
-  float gr[2], gc[2];
-  {
-    const float2 s0 = *reinterpret_cast<const float2*>(&stot[0][c0]);
-    const float2 s1 = *reinterpret_cast<const float2*>(&stot[1][c0]);
-    const float2 s2 = *reinterpret_cast<const float2*>(&stot[2][c0]);
-    const float2 s3 = *reinterpret_cast<const float2*>(&stot[3][c0]);
-    // offsets added in the order that makes G_r and G_C equal the values at tokens 31 and 63
-    const float o1[2] = {s0.x, s0.y};
-    const float o2[2] = {s1.x + s0.x, s1.y + s0.y};
-    const float o3[2] = {(s0.x + s1.x) + s2.x, (s0.y + s1.y) + s2.y};
-    gr[0] = o2[0];
-    gr[1] = o2[1];
-    gc[0] = s3.x + o3[0];
-    gc[1] = s3.y + o3[1];
-    if (tq > 0) {
-      const float a0 = tq == 1 ? o1[0] : (tq == 2 ? o2[0] : o3[0]);
-      const float a1 = tq == 1 ? o1[1] : (tq == 2 ? o2[1] : o3[1]);
+    for (int t = 0; t < 4; ++t) {
+      const int i = tg + 16 * t;
+      float q8[8], k8[8];
+      ld8(sm + kP1A + kmajor_off(kC + i, c8, 128), q8);
+      ld8(sm + kP1B + kmajor_off(i, c8, kC), k8);
+      float sq2 = 0.f, sk2 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        G[i][0] += a0;
-        G[i][1] += a1;
+      for (int e = 0; e < 8; ++e) {
+        sq2 = fmaf(q8[e], q8[e], sq2);
+        sk2 = fmaf(k8[e], k8[e], sk2);
       }
+      atomicAdd(&snq[i], sq2);
+      atomicAdd(&snk[i], sk2);
     }
   }
-  if (tq == 3) {
-    *reinterpret_cast<float2*>(rec + kRecGamma + 4 * c0) = make_float2(expf(gc[0]), expf(gc[1]));
+  if (!kScalarGate) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) ld8(sm + kP1A + kmajor_off(tg + 16 * t, c8, 128), G[t]);
+    if (kPrep && (prep & KDA_PREP_GATE_LOGSIGMOID)) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) G[t][e] = tg + 16 * t < L ? log_sigmoid_fast(G[t][e]) : 0.f;  // padding: no decay
+    }
+  } else {  // one log-gate per token for every channel (zero without a gate)
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) G[t][e] = sgh[tg + 16 * t];
   }
-  if (l2n && tid < kC) {  // the sums of squares become the per-token unit-length factors (read after the vote)
-    snk[tid] = rsqrtf(snk[tid] + kL2Eps);
-    snq[tid] = rsqrtf(snq[tid] + kL2Eps);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    float tot[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float x = G[t][e];
+#pragma unroll
+      for (int d = 1; d < 16; d <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, d, 16);
+        if (tg >= d) x += y;
+      }
+      G[t][e] = x;
+      tot[t] = __shfl_sync(0xffffffffu, x, 15, 16);
+    }
+    G[1][e] += tot[0];
+    G[2][e] += tot[0] + tot[1];
+    G[3][e] += (tot[0] + tot[1]) + tot[2];
+    gref[e] = tot[0] + tot[1];                 // G at token 31
+    gend[e] = ((tot[0] + tot[1]) + tot[2]) + tot[3];  // G at token 63 (= G_C; padding has g = 0)
   }
-  const bool unsafe = gc[0] < -kSafeSpan || gc[1] < -kSafeSpan;
-  const int slow = __syncthreads_or(unsafe);  // every tile is read: R1-R3 are free for the images
+  bool unsafe = false;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) unsafe |= gend[e] < -kSafeSpan;
+  if (tg == 0) {
+    float* gam = reinterpret_cast<float*>(rec + kRecGamma) + c8;
+    *reinterpret_cast<float4*>(gam) = make_float4(expf(gend[0]), expf(gend[1]), expf(gend[2]), expf(gend[3]));
+    *reinterpret_cast<float4*>(gam + 4) = make_float4(expf(gend[4]), expf(gend[5]), expf(gend[6]), expf(gend[7]));
+  }
+  const int slow = __syncthreads_or(unsafe);  // the g tile is dead from here on
 
   if (!slow) {
-    // ---- factored form: images relative to token kRefTok
-    float egr[2], rho[2];
+    // ---- pass 2 (factored form): decayed operands relative to token kRefTok
+    float egr[8], egb[8];
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      egr[e] = __expf(gr[e]);
-      rho[e] = __expf(gc[e] - gr[e]);
+    for (int e = 0; e < 8; ++e) {
+      egr[e] = __expf(gref[e]);
+      egb[e] = __expf(gend[e] - gref[e]);
     }
-    if (tq == 0) *reinterpret_cast<float2*>(&segr[c0]) = make_float2(egr[0], egr[1]);
+    if (tg == 0) {
 #pragma unroll
-    for (int pc = 0; pc < 2; ++pc) {  // the two 8-token pieces of this quarter
-      uint32_t kp[2][4], km[2][4], qr[2][4], qa[2][4], kb[2][4];
+      for (int e = 0; e < 8; ++e) segr[c8 + e] = egr[e];
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {  // token pair (i, i+1)
-        const int i = 8 * pc + 2 * u;
-        const float2 ka = unpack2(kw[i]), kc = unpack2(kw[i + 1]);
-        const float2 qa2 = unpack2(qw[i]), qc = unpack2(qw[i + 1]);
-        const float rk0 = l2n ? snk[16 * tq + i] : 1.f, rk1 = l2n ? snk[16 * tq + i + 1] : 1.f;
-        const float rq0 = l2n ? snq[16 * tq + i] : 1.f, rq1 = l2n ? snq[16 * tq + i + 1] : 1.f;
-        const float kv[2][2] = {{ka.x * rk0, kc.x * rk1}, {ka.y * rk0, kc.y * rk1}};  // [channel][token]
-        const float qv[2][2] = {{qa2.x * rq0, qc.x * rq1}, {qa2.y * rq0, qc.y * rq1}};
+    for (int t = 0; t < 4; ++t) {
+      const int i = tg + 16 * t;
+      const uint32_t oK = kmajor_off(i, c8, kC);        // 64-row tiles: k, K-_r, Kbar
+      const uint32_t oA = kmajor_off(i, c8, 128);       // row i of region A
+      const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A and of the [-W;Q+] image
+      float k8[8], q8[8];
+      ld8(sm + kP1B + oK, k8);
+      ld8(sm + kP1A + oQ, q8);
+      if (l2n) {
+        const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float fp[2], fm[2], fq[2], fa[2], fb[2];
-#pragma unroll
-          for (int s = 0; s < 2; ++s) {
-            const float e1 = __expf(G[i + s][e] - gr[e]), e2 = __expf(gr[e] - G[i + s][e]);
-            fp[s] = kv[e][s] * e1;
-            fm[s] = kv[e][s] * e2;
-            fq[s] = qv[e][s] * (scale * e1);
-            fa[s] = fq[s] * egr[e];
-            fb[s] = fm[s] * rho[e];
-          }
-          kp[e][u] = pack2(fp[0], fp[1]);
-          km[e][u] = pack2(fm[0], fm[1]);
-          qr[e][u] = pack2(fq[0], fq[1]);
-          qa[e][u] = pack2(fa[0], fa[1]);
-          kb[e][u] = pack2(fb[0], fb[1]);
+        for (int e = 0; e < 8; ++e) {
+          k8[e] *= rk;
+          q8[e] *= rq;
         }
       }
+      // the start-decayed operands first, then the end-decayed ones, so that
+      // fewer values are live at once (64 registers at 4 CTAs per SM)
+      float w[8];
+      {
+        float ex[8];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const uint32_t o = row_piece(c0 + e, 2 * tq + pc);
-        *reinterpret_cast<uint4*>(sm + kP1R1 + o) = make_uint4(kp[e][0], kp[e][1], kp[e][2], kp[e][3]);
-        *reinterpret_cast<uint4*>(sm + kP1R2 + o) = make_uint4(km[e][0], km[e][1], km[e][2], km[e][3]);
-        *reinterpret_cast<uint4*>(sm + kP1R3 + o) = make_uint4(qr[e][0], qr[e][1], qr[e][2], qr[e][3]);
-        *reinterpret_cast<uint4*>(rec + kRecQ + o) = make_uint4(qa[e][0], qa[e][1], qa[e][2], qa[e][3]);
-        *reinterpret_cast<uint4*>(rec + kRecKbar + o) = make_uint4(kb[e][0], kb[e][1], kb[e][2], kb[e][3]);
+        for (int e = 0; e < 8; ++e) {
+          ex[e] = __expf(G[t][e] - gref[e]);
+          q8[e] *= scale;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = k8[e] * ex[e];
+        st8(sm + kP1A + oA, w);               // K+_r (over the dead g rows)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = q8[e] * ex[e];
+        st8(sm + kP1A + oQ, w);               // Q+_r (in place of q)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * egr[e]);
+        st8(rec + kRecWQ + oQ, w);            // Q+ image
+      }
+      {
+        float ei[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ei[e] = __expf(gref[e] - G[t][e]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = k8[e] * ei[e];
+        st8(sm + kP1B + oK, w);               // K-_r, in place of k
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ei[e] * egb[e]);
+        st8(rec + kRecKbar + oK, w);          // Kbar image = k exp(G_C - G_i)
       }
     }
     fence_async_smem();
@@ -401,20 +404,20 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     __syncthreads();
     tc_fence_after();
 
-    // ---- score MMA: D[0:128, 0:64] = [K+_r ; Q+_r] (M = tokens, K = channels) . K-_r^T
+    // ---- score MMA: D[0:128, 0:64] = [K+_r ; Q+_r] (128 x 128) . K-_r^T
     if (tid == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
-      const uint64_t a0 = desc_sw128(smem_u32(sm + kP1R1), kP1R3 - kP1R1, 1024);
-      const uint64_t b0 = desc_sw128(smem_u32(sm + kP1R2), 16384, 1024);
+      const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
+      const uint64_t a0 = desc_sw128(smem_u32(sm + kP1A), 16, 1024), b0 = desc_sw128(smem_u32(sm + kP1B), 16, 1024);
 #pragma unroll
-      for (int s = 0; s < kD / 16; ++s)  // 16 channels = 2 rows of 8-channel atoms per step
-        mma_bf16(tm, a0 + (uint64_t)((s * 2048) >> 4), b0 + (uint64_t)((s * 2048) >> 4), idesc, s > 0);
+      for (int k = 0; k < kD / 16; ++k)
+        mma_bf16(tm, a0 + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4),
+                 b0 + (uint64_t)(((k / 4) * 8192 + (k % 4) * 32) >> 4), idesc, k > 0);
       mma_commit(&bar_mma);
     }
     wait_or_flag(&bar_mma, 0, hdr, 2);
     tc_fence_after();
 
-    // ---- rows 0-63 -> A_kk blocks (times beta_i, strictly lower); rows 64-127 -> A_qk rows of the record
+    // ---- rows 0-63 -> A_kk blocks (times beta_i, strictly lower); rows 64-127 -> A_qk^T staging
     {
       const int row = (warp & 3) * 32 + lane;
       const int col0 = (warp >> 2) * 32;
@@ -443,35 +446,29 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       } else {
         const int i = row - kC;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j0 = col0 + 8 * p + 2 * e;
-            w[e] = pack2(j0 <= i ? v[8 * p + 2 * e] : 0.f, j0 + 1 <= i ? v[8 * p + 2 * e + 1] : 0.f);
-          }
-          *reinterpret_cast<uint4*>(rec + kRecAqk + row_piece(i, (col0 >> 3) + p)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        for (int jj = 0; jj < 32; ++jj) stbf(sm + kP1QT, kmajor_off(col0 + jj, i, kC), (col0 + jj) <= i ? v[jj] : 0.f);
       }
     }
   } else {
     // ---- exact path for chunks whose gates decay past e^-64: the score
     // matrices straight from their definition, every decay factor
     // exp(G_i - G_j) <= 1 formed per (pair, channel).  G is staged in fp32
-    // one 64-channel half at a time in R1 (the g tile is read); k and q are
-    // read from their token-row tiles, which stay until both halves are done.
-    if (tq == 0) *reinterpret_cast<float2*>(&segr[c0]) = make_float2(1.f, 1.f);
-    float* gst = reinterpret_cast<float*>(sm + kP1R1);  // [64 tokens][64 channels]
+    // one 64-channel half at a time over the dead g rows of region A.
+    auto gp = [&](int i, int c) -> float* {  // c in [0, 64): channel of the staged half
+      return c < 32 ? reinterpret_cast<float*>(sm + kP1A) + i * 32 + c
+                    : reinterpret_cast<float*>(sm + kP1A + 16384) + i * 32 + (c - 32);
+    };
     constexpr int kPairs = kC * (kC + 1) / 2;  // (i, j) with j <= i
     float akk[9], aqk[9];
 #pragma unroll
     for (int t = 0; t < 9; ++t) akk[t] = aqk[t] = 0.f;
 #pragma unroll 1
-    for (int hr = 0; hr < 2; ++hr) {
-      if (hf == hr) {
+    for (int hf = 0; hf < 2; ++hf) {
+      if ((c8 >> 6) == hf) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          *reinterpret_cast<float2*>(gst + (16 * tq + i) * 64 + 2 * lane) = make_float2(G[i][0], G[i][1]);
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) *gp(tg + 16 * t, c8 - 64 * hf + e) = G[t][e];
       }
       __syncthreads();
 #pragma unroll 1
@@ -485,12 +482,11 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
           float sk = akk[t], sq = aqk[t];
 #pragma unroll 4
           for (int c = 0; c < 64; c += 2) {
-            const int ch = 64 * hr + c;
-            const float2 ki = ld_bf2(sm + kP1R2 + kmajor_off(i, ch, kC));
-            const float2 kj = ld_bf2(sm + kP1R2 + kmajor_off(j, ch, kC));
-            const float2 qi = ld_bf2(sm + kP1R3 + kmajor_off(i, ch, kC));
-            const float d0 = __expf(gst[i * 64 + c] - gst[j * 64 + c]);
-            const float d1 = __expf(gst[i * 64 + c + 1] - gst[j * 64 + c + 1]);
+            const int ch = 64 * hf + c;
+            const float2 ki = ld_bf2(sm + kP1B + kmajor_off(i, ch, kC));
+            const float2 kj = ld_bf2(sm + kP1B + kmajor_off(j, ch, kC));
+            const float2 qi = ld_bf2(sm + kP1A + kmajor_off(kC + i, ch, 128));
+            const float d0 = __expf(*gp(i, c) - *gp(j, c)), d1 = __expf(*gp(i, c + 1) - *gp(j, c + 1));
             sk = fmaf(ki.x * kj.x, d0, fmaf(ki.y * kj.y, d1, sk));
             sq = fmaf(qi.x * kj.x, d0, fmaf(qi.y * kj.y, d1, sq));
           }
@@ -498,9 +494,43 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
           aqk[t] = sq;
         }
       }
-      __syncthreads();  // this half of G (and, after the second, the k and q tiles) is read
+      __syncthreads();  // this half of G is read
     }
-    // A_kk blocks (over the k and q tiles) and the A_qk rows of the record
+    // pass 2 (exact): start- and end-decayed operands, factors <= 1; K+ goes
+    // over the dead g rows of region A (where the factored form keeps K+_r),
+    // with a unit W scale
+    if (tg == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) segr[c8 + e] = 1.f;
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int i = tg + 16 * t;
+      const uint32_t oK = kmajor_off(i, c8, kC);
+      const uint32_t oQ = kmajor_off(kC + i, c8, 128);
+      float k8[8], q8[8], kp[8], qp[8], kb[8];
+      ld8(sm + kP1B + oK, k8);
+      ld8(sm + kP1A + oQ, q8);
+      if (l2n) {
+        const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          k8[e] *= rk;
+          q8[e] *= rq;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float e0 = __expf(G[t][e]);
+        kp[e] = k8[e] * e0;
+        qp[e] = scale * q8[e] * e0;
+        kb[e] = k8[e] * __expf(gend[e] - G[t][e]);
+      }
+      st8(sm + kP1A + kmajor_off(i, c8, 128), kp);
+      st8(rec + kRecWQ + oQ, qp);
+      st8(rec + kRecKbar + oK, kb);
+    }
+    __syncthreads();  // k and q are read: region B takes the A_kk blocks, [24K,32K) of region A the A_qk^T staging
 #pragma unroll 1
     for (int t = 0; t < 9; ++t) {
       const int p = tid + t * kP1Threads;
@@ -511,57 +541,31 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
         const int j = p - i * (i + 1) / 2;
         float fk = 1.f, fq = 1.f;  // unit-length factors of k_i k_j and q_i k_j
         if (l2n) {
-          fk = snk[i] * snk[j];
-          fq = snq[i] * snk[j];
+          const float rkj = rsqrtf(snk[j] + kL2Eps);
+          fk = rsqrtf(snk[i] + kL2Eps) * rkj;
+          fq = rsqrtf(snq[i] + kL2Eps) * rkj;
         }
         a_blk(sm, blk(i >> 4, j >> 4))[bidx(i & 15, j & 15)] = j < i ? sbeta[i] * (akk[t] * fk) : 0.f;
-        stbf(rec + kRecAqk, kmajor_off(i, j, kC), scale * (aqk[t] * fq));
+        stbf(sm + kP1QT, kmajor_off(j, i, kC), scale * (aqk[t] * fq));
       }
     }
     for (int e = tid; e < kC * kC; e += kP1Threads) {
       const int i = e / kC, j = e % kC;
-      if (j > i) stbf(rec + kRecAqk, kmajor_off(i, j, kC), 0.f);
-    }
-    // start- and end-decayed images with factors <= 1: K+^T over R1 (the W
-    // product's operand, with a unit W scale), Q+^T and Kbar^T into the record
-#pragma unroll
-    for (int pc = 0; pc < 2; ++pc) {
-      uint32_t kp[2][4], qa[2][4], kb[2][4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = 8 * pc + 2 * u;
-        const float2 ka = unpack2(kw[i]), kc = unpack2(kw[i + 1]);
-        const float2 qa2 = unpack2(qw[i]), qc = unpack2(qw[i + 1]);
-        const float rk0 = l2n ? snk[16 * tq + i] : 1.f, rk1 = l2n ? snk[16 * tq + i + 1] : 1.f;
-        const float rq0 = l2n ? snq[16 * tq + i] : 1.f, rq1 = l2n ? snq[16 * tq + i + 1] : 1.f;
-        const float kv[2][2] = {{ka.x * rk0, kc.x * rk1}, {ka.y * rk0, kc.y * rk1}};
-        const float qv[2][2] = {{qa2.x * rq0, qc.x * rq1}, {qa2.y * rq0, qc.y * rq1}};
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float fp[2], fa[2], fb[2];
-#pragma unroll
-          for (int s = 0; s < 2; ++s) {
-            const float e0 = __expf(G[i + s][e]);
-            fp[s] = kv[e][s] * e0;
-            fa[s] = scale * qv[e][s] * e0;
-            fb[s] = kv[e][s] * __expf(gc[e] - G[i + s][e]);
-          }
-          kp[e][u] = pack2(fp[0], fp[1]);
-          qa[e][u] = pack2(fa[0], fa[1]);
-          kb[e][u] = pack2(fb[0], fb[1]);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const uint32_t o = row_piece(c0 + e, 2 * tq + pc);
-        *reinterpret_cast<uint4*>(sm + kP1R1 + o) = make_uint4(kp[e][0], kp[e][1], kp[e][2], kp[e][3]);
-        *reinterpret_cast<uint4*>(rec + kRecQ + o) = make_uint4(qa[e][0], qa[e][1], qa[e][2], qa[e][3]);
-        *reinterpret_cast<uint4*>(rec + kRecKbar + o) = make_uint4(kb[e][0], kb[e][1], kb[e][2], kb[e][3]);
-      }
+      if (j > i) stbf(sm + kP1QT, kmajor_off(j, i, kC), 0.f);
     }
   }
   fence_async_smem();
-  __syncthreads();  // the A_kk blocks are complete
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0) {
+    bulk_store(rec + kRecAqk, sm + kP1QT, 8192);
+    bulk_commit();
+    // Q+_r is dead: bring v while the triangle is inverted, its first
+    // channel half now, the second once the A_qk^T store has read its bytes
+    mbar_expect_tx(&bar_v, 16384);
+    tma_load_4d(sm + kP1V, &tm_v, &bar_v, 0, h, t0, b);
+  }
 
   // ---- T = (I + A_kk)^-1 by 16 x 16 blocks, fp32
   if (tid < 64) {  // diagonal blocks by forward substitution, one column per thread
@@ -580,6 +584,10 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     for (int r = 0; r < 16; ++r) Tb[bidx(r, jj)] = t[r];
   }
   __syncthreads();
+  if (tid == 0) {
+    bulk_wait_read();
+    tma_load_4d(sm + kP1V + 16384, &tm_v, &bar_v, 64, h, t0, b);
+  }
   // off-diagonal blocks, one sub-diagonal at a time, one warp per block:
   //   X = sum_{K=J}^{I-1} A_IK T_KJ,   T_IJ = -T_II X
   // as 16x16x16 products on the warp-level tensor cores (tf32 in, fp32
@@ -600,7 +608,8 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     }
     __syncthreads();
   }
-  // (T diag(beta))^T as the K-major B operand of the W/U MMAs: row n = i, column k = j.
+  // (T diag(beta))^T as the K-major B operand of the W/U MMAs: row n = i, column k = j
+  // (over the A_kk blocks, read by now).
   {
     const int i = tid >> 2, j0 = (tid & 3) * 16, I = i >> 4, J = j0 >> 4;
     float vals[16];
@@ -620,49 +629,55 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   __syncthreads();
   tc_fence_after();
 
-  // ---- W^T / segr = K+_r^T (T diag beta)^T (A K-major: the channel rows of R1),
-  //      U^T = V^T (T diag beta)^T (A MN-major: the v tile), M = 128, N = 64, K = 64.
-  // K+_r = K+ / exp(G_r) per channel (K+ itself on the exact path, segr = 1), so
-  // the extraction scales row c of the first product by segr[c].
+  // ---- W^T / segr = K+_r^T (T diag beta)^T, U^T = V^T (T diag beta)^T  (M=128, N=64, K=64).
+  // K+_r = K+ / exp(G_r) per channel (rows 0-63 of region A, channel halves
+  // 16 KiB apart; K+ itself on the exact path, segr = 1), so the extraction
+  // scales row c of the first product by segr[c]; v's halves are 16 KiB apart too.
   if (tid == 0) {
     wait_or_flag(&bar_v, 0, hdr, 3);
     tc_fence_after();
-    const uint32_t idw = idesc_bf16_f32(128, 64, 0, 0), idu = idesc_bf16_f32(128, 64, 1, 0);
-    const uint32_t kb = smem_u32(sm + kP1R1), vb = smem_u32(sm + kP1V), b2 = smem_u32(sm + kP1B2);
+    const uint32_t idesc = idesc_bf16_f32(128, 64, 1, 0);
+    const uint32_t kb = smem_u32(sm + kP1A), vb = smem_u32(sm + kP1V), b2 = smem_u32(sm + kP1B2);
 #pragma unroll
-    for (int s = 0; s < kC / 16; ++s) {
-      const uint64_t bd = desc_sw128(b2 + s * 32, 16, 1024);
-      mma_bf16(tm, desc_sw128(kb + s * 32, 16, 1024), bd, idw, s > 0);
-      mma_bf16(tm + 64, desc_sw128(vb + 2 * s * 1024, 8192, 1024), bd, idu, s > 0);
+    for (int k = 0; k < kC / 16; ++k) {
+      const uint64_t bd = desc_sw128(b2 + k * 32, 16, 1024);
+      mma_bf16(tm, desc_sw128(kb + 2 * k * 1024, 16384, 1024), bd, idesc, k > 0);
+      mma_bf16(tm + 64, desc_sw128(vb + 2 * k * 1024, 16384, 1024), bd, idesc, k > 0);
     }
     mma_commit(&bar_mma);
   }
   wait_or_flag(&bar_mma, slow ? 0 : 1, hdr, 4);
   tc_fence_after();
 
-  // ---- -W^T (row = key channel c) and U^T (row = value channel) into the record
+  // ---- -W (staged over K+_r: rows 0-63 of region A) and U^T (region B, 128-row K-major)
   {
-    const int r = (warp & 3) * 32 + lane, col0 = (warp >> 2) * 32;
+    const int c = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const float wsc = -segr[r];
+    const float wsc = warp < 4 ? -segr[c] : 0.f;
     float v[32];
-    tmem_ld32(tm + lane_off + col0, v);
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float* x = v + 8 * p;
-      *reinterpret_cast<uint4*>(rec + kRecW + row_piece(r, (col0 >> 3) + p)) =
-          make_uint4(pack2(wsc * x[0], wsc * x[1]), pack2(wsc * x[2], wsc * x[3]), pack2(wsc * x[4], wsc * x[5]),
-                     pack2(wsc * x[6], wsc * x[7]));
-    }
-    tmem_ld32(tm + lane_off + 64 + col0, v);
+    for (int half = 0; half < 2; ++half) {
+      if (warp < 4) {
+        tmem_ld32(tm + lane_off + half * 32, v);
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float* x = v + 8 * p;
-      *reinterpret_cast<uint4*>(rec + kRecU + row_piece(r, (col0 >> 3) + p)) =
-          make_uint4(pack2(x[0], x[1]), pack2(x[2], x[3]), pack2(x[4], x[5]), pack2(x[6], x[7]));
+        for (int ii = 0; ii < 32; ++ii) stbf(sm + kP1A, kmajor_off(half * 32 + ii, c, 128), wsc * v[ii]);
+      } else {
+        tmem_ld32(tm + lane_off + 64 + half * 32, v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st_kmajor8(sm + kP1B, c, half * 32 + 8 * e, 128, v + 8 * e);
+      }
     }
   }
+  fence_async_smem();
   tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {
+    bulk_store(rec + kRecWQ, sm + kP1A, 8192);                 // -W rows, channels 0-63
+    bulk_store(rec + kRecWQ + 16384, sm + kP1A + 16384, 8192); // -W rows, channels 64-127
+    bulk_store(rec + kRecU, sm + kP1B, 16384);
+    bulk_commit();
+    bulk_wait_read();
+  }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tm, 128);
 }
@@ -688,9 +703,6 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
 //   P           = S0^T (-W)^T               (N = 64,  K = 128: 8 instructions, committed alone)
 //   O^T         = S0^T Q+^T                 (N = 64,  K = 128: 8 instructions, while V' is formed)
 //   [O^T | S^T] += V'^T [A_qk^T | Kbar]      (N = 192, K = 64:  4 instructions)
-// The B operands are the record's channel-row images: -W^T and Q+^T read
-// MN-major (N = tokens contiguous), [A_qk | Kbar^T] K-major (rows = the N
-// index, K = tokens contiguous).
 // with P = -(W S0)^T and V'^T = U^T + P formed on the CUDA cores.  Only P
 // and the last group are on the chain's critical path; the O^T group waits
 // for the output warps to release the previous chunk's O^T off that path.
@@ -698,10 +710,11 @@ constexpr int kSPThreads = 288;
 constexpr uint32_t kTmP = 0, kTmO = 64, kTmS = 128, kTmAS = 256, kTmAV = 320;
 
 // Brings the record of one chunk into a stage.  A pass that writes outputs
-// needs all of it; a pass without outputs reads only -W^T, Kbar^T, U^T and
-// gamma; the transition pass (U = 0) not even U^T.
-constexpr uint32_t kRecNoOutBytes = (kRecQ - kRecW) + (kRecBytes - kRecKbar);
-constexpr uint32_t kRecTransBytes = (kRecQ - kRecW) + (kRecU - kRecKbar) + (kRecBytes - kRecGamma);
+// needs all of it; a pass without outputs reads only -W (the first 64 rows
+// of each 64-column block of [-W; Q+]), Kbar, U and gamma; the transition
+// pass (U = 0) not even U.
+constexpr uint32_t kRecNoOutBytes = 2 * 8192 + (kRecBytes - kRecKbar);
+constexpr uint32_t kRecTransBytes = 2 * 8192 + (kRecU - kRecKbar) + (kRecBytes - kRecGamma);
 __device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, uint64_t* bar, bool out,
                                             bool zero_u) {
   if (out) {
@@ -710,7 +723,8 @@ __device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, 
     return;
   }
   mbar_expect_tx(bar, zero_u ? kRecTransBytes : kRecNoOutBytes);
-  bulk_load(stage + kRecW, rec + kRecW, kRecQ - kRecW, bar);
+  bulk_load(stage + kRecWQ, rec + kRecWQ, 8192, bar);
+  bulk_load(stage + kRecWQ + 16384, rec + kRecWQ + 16384, 8192, bar);
   if (zero_u) {
     bulk_load(stage + kRecKbar, rec + kRecKbar, kRecU - kRecKbar, bar);
     bulk_load(stage + kRecGamma, rec + kRecGamma, kRecBytes - kRecGamma, bar);
@@ -843,16 +857,16 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       // at once; with outputs, O^T = S0^T Q+^T (N=64) is issued next, while
       // the state warps form V', and [O|S] += V'^T [A_qk^T|Kbar] (N=192)
       // closes the chunk; without outputs S += V'^T Kbar (N=128).
-      const uint32_t id_1 = idesc_bf16_f32(128, 64, 0, 1);
-      const uint32_t id_2 = idesc_bf16_f32(128, out ? 192 : 128, 0, 0);
-      const uint32_t d2_off = out ? 0 : ((kRecKbar - kRecAqk) >> 4);  // skip the A_qk rows
+      const uint32_t id_1 = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t id_2 = idesc_bf16_f32(128, out ? 192 : 128, 0, 1);
+      const uint32_t d2_off = out ? 0 : (8192 >> 4);  // skip the A_qk^T block
       const uint32_t t2 = out ? tm + kTmO : tm + kTmS;
       // first descriptors of each stage; later steps add address offsets (in 16-byte units)
-      const uint64_t d1s0 = desc_sw128(smem_u32(sm + kRecW), 16384, 1024);
-      const uint64_t d1s1 = desc_sw128(smem_u32(sm + kStage + kRecW), 16384, 1024);
-      const uint64_t d2s0 = desc_sw128(smem_u32(sm + kRecAqk), 16, 1024) + d2_off;
-      const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStage + kRecAqk), 16, 1024) + d2_off;
-      constexpr uint64_t kQoff = (kRecQ - kRecW) >> 4;  // the Q+^T image follows -W^T
+      const uint64_t d1s0 = desc_sw128(smem_u32(sm + kRecWQ), 16, 1024);
+      const uint64_t d1s1 = desc_sw128(smem_u32(sm + kStage + kRecWQ), 16, 1024);
+      const uint64_t d2s0 = desc_sw128(smem_u32(sm + kRecAqk), 8192, 1024) + d2_off;
+      const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStage + kRecAqk), 8192, 1024) + d2_off;
+      constexpr uint64_t kQoff = 8192 >> 4;  // rows 64-127 (Q+) of each 64-column block of [-W; Q+]
       for (int n = 0; n < NCL; ++n) {
         const int s = n & 1;
         wait_or_flag(&bar_as, n & 1, hdr, 30);
@@ -860,19 +874,21 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         tc_fence_after();
         const uint64_t d1 = s ? d1s1 : d1s0, d2 = s ? d2s1 : d2s0;
 #pragma unroll
-        for (int k = 0; k < kD / 16; ++k)  // MN-major B: 16 channel rows (2 KiB) per step
-          mma_bf16_ts(tm + kTmP, tm + kTmAS + k * 8, d1 + (uint64_t)((k * 2048) >> 4), id_1, k > 0);
+        for (int k = 0; k < kD / 16; ++k)  // K-major B: +32 B per step inside a 64-wide block, +16 KiB per block
+          mma_bf16_ts(tm + kTmP, tm + kTmAS + k * 8, d1 + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), id_1,
+                      k > 0);
         mma_commit(&bar_p);
         if (out) {  // bar_as also covered the read of O^T of chunk n-1
 #pragma unroll
           for (int k = 0; k < kD / 16; ++k)
-            mma_bf16_ts(tm + kTmO, tm + kTmAS + k * 8, d1 + kQoff + (uint64_t)((k * 2048) >> 4), id_1, k > 0);
+            mma_bf16_ts(tm + kTmO, tm + kTmAS + k * 8,
+                        d1 + kQoff + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), id_1, k > 0);
         }
         wait_or_flag(&bar_av, n & 1, hdr, 33);
         tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < kC / 16; ++k)  // K-major B: 16 tokens = 32 bytes of each row per step
-          mma_bf16_ts(t2, tm + kTmAV + k * 8, d2 + (uint64_t)((k * 32) >> 4), id_2, 1);
+        for (int k = 0; k < kC / 16; ++k)  // MN-major B: +2 KiB per 16 K-rows
+          mma_bf16_ts(t2, tm + kTmAV + k * 8, d2 + (uint64_t)((2 * k * 1024) >> 4), id_2, 1);
         mma_commit(&bar_s);
         mma_commit(&bar_o);
       }
