@@ -46,10 +46,13 @@
 // chunk's operands as one bf16 record; the decay factors, the fold into the
 // gradients and every sum stay fp32.  No atomics: every sum runs in a fixed
 // order, so results are bit-reproducible.
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <type_traits>
 
 #include "kda_common.cuh"
+#include "sm100.cuh"
 
 namespace kda {
 namespace {
@@ -379,6 +382,7 @@ struct ChunkBwdArgs {
   float scale;
   int T, H, NC, gate;
   int bh0;  // first (sequence, head) of this launch group: bh = bh0 + local index
+  int tc_rec;  // bf16, d_k = d_v = 128: the pass record in the tensor-core passes' layout (TcRec)
   // workspace (fp32), record rec = (bh - bh0) * NC + chunk
   float *W, *U, *Qp, *Kb;  // [rec][64][d_k] (U: [64][d_v]): W, U, Q+, Kbar
   float *Wt, *Qpt, *Kbt;   // [rec][d_k][64]: their transposes for the state passes (fp32 inputs)
@@ -412,6 +416,26 @@ struct PassRec {  // element offsets of the bf16 pass record of one chunk (all r
   static constexpr int n = oKb + kC * LKb;       // the reverse sweep reads [0, n), the forward replay [oW, n)
   static_assert(oQp % 8 == 0 && oW % 8 == 0 && oKb % 8 == 0 && n % 8 == 0, "16 B");
 };
+
+// With d_k = d_v = 128 the state passes run on the tcgen05 tensor cores and
+// read the record as the canonical 128-byte-swizzled token-row tiles of
+// their MMA operands (the layout a TMA tile load of [64 tokens][64 channels]
+// produces): element (token i, channel c) of a 64 x 128 tile at byte
+// (c / 64) * 8192 + i * 128 + (((c % 64) / 8) ^ (i % 8)) * 16 + (c % 8) * 2.
+// Byte offsets inside the record (the record keeps PassRec's stride):
+struct TcRec {
+  static constexpr uint32_t oW = 0;         // W    [64 tokens][128 channels]
+  static constexpr uint32_t oQp = 16384;    // Q+   [64 tokens][128 channels]
+  static constexpr uint32_t oKb = 32768;    // Kbar [64 tokens][128 channels]
+  static constexpr uint32_t oAqk = 49152;   // Aqk  [64 query tokens i][64 key tokens j]
+  static constexpr uint32_t bytes = 57344;
+};
+static_assert(TcRec::bytes <= PassRec<128>::n * 2, "the tensor-core record fits the record stride");
+template <int DK, int DV>
+constexpr bool kTcPass = DK == 128 && DV == 128;
+__device__ __forceinline__ uint32_t tile_off(int i, int c) {  // byte offset of (token i, channel c) in a 64-row tile
+  return (uint32_t)((c >> 6) * 8192 + i * 128 + ((((c & 63) >> 3) ^ (i & 7)) << 4) + (c & 7) * 2);
+}
 
 // T = (I + diag(beta) P)^-1 for a strictly lower 64 x 64 P (fp32, leading
 // dimension kLC) by 16 x 16 blocks, on the NT first threads of the block
@@ -1088,6 +1112,298 @@ __global__ void __launch_bounds__(kPassThreads, 1) bwd_pass_bf16_kernel(const Ch
   }
 }
 
+// ------------------------------------------------------------------ kernel 2, tensor-core form
+// The two state passes for bf16 inputs at d_k = d_v = 128 on the tcgen05
+// tensor cores, one CTA per (sequence, head) and role, with the state kept
+// transposed in tensor memory (lane j = value channel j, 128 fp32 columns =
+// key channels) for the whole chain, as in the forward's state pass:
+//   role 0 (replay, chunks in order):   P = S0^T W^T;  V'^T = U^T - P;
+//                                       S^T <- S^T diag(gamma) + V'^T Kbar
+//   role 1 (reverse sweep, backwards):  dV'^T = dO^T Aqk + dS^T Kbar^T;
+//                                       dS^T <- dS^T diag(gamma) + dO^T Q+ - dV'^T W
+// Every product has M = 128 (the value channels): A is the state (or V'^T,
+// dV'^T) in bf16 from tensor memory, or dO^T read MN-major from the TMA
+// tile of dO; B is a token-row tile of the record (W, Kbar as K-major or
+// MN-major views, Q+, Aqk).  Warps 0-3 own the state rows: they convert the
+// state and V' to bf16 operands, decay the state by gamma, form V'^T = U^T - P,
+// and write the bf16 checkpoints (S0 or dS entering the chunk's step, V' or
+// dV') in the row-major layouts the per-chunk kernels read.  Warp 4 issues
+// the MMAs, warp 5 streams each chunk's operands into one of two stages.
+// Every mbarrier wait is bounded; a give-up sets the workspace error word.
+namespace tcpass {
+using namespace sm100;
+constexpr int kThreads = 192;
+constexpr uint32_t kStage = 83968;                                   // bytes per stage (82 KiB)
+constexpr uint32_t kStW = 0, kStQ = 16384, kStKb = 32768, kStAqk = 49152;  // record tiles (as in TcRec)
+constexpr uint32_t kStO = 57344;   // role 1: the dO tile, [64 tokens][2 x 64 value channels]
+constexpr uint32_t kStU = 49152;   // role 0: U (fp32 [64][128])
+constexpr uint32_t kStGam = 81920; // gamma (fp32 [128])
+constexpr size_t kSmem = 2 * (size_t)kStage + 1024;
+constexpr uint32_t kTmAcc = 0, kTmS = 64, kTmAS = 192, kTmAV = 256;  // tensor-memory columns
+constexpr uint32_t kWait = 1u << 24;
+static_assert(kStU + 32768 <= kStGam && kStO + 16384 <= kStGam && kStGam + 512 <= kStage, "stage layout");
+
+__device__ __forceinline__ void wait_or_flag(uint64_t* bar, uint32_t parity, WorkspaceHeader* hdr, uint32_t where) {
+  if (!mbar_wait(bar, parity, kWait)) {
+    atomicOr(&hdr->error, 1u);
+    atomicExch(&hdr->where, where);
+  }
+}
+__device__ __forceinline__ uint32_t pk2(float a, float b) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_pass_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const ChunkBwdArgs a, WorkspaceHeader* hdr) {
+  constexpr int DK = 128, DV = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t bar_full[2], bar_free[2], bar_as, bar_p, bar_av, bar_s;
+  __shared__ uint32_t tmem_base;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int role = blockIdx.y, lb = blockIdx.x, bh = a.bh0 + lb, NC = a.NC;
+  const int h = bh % a.H, b = bh / a.H;
+  const size_t st0 = (size_t)bh * DK * DV;
+  const uint8_t* recs = reinterpret_cast<const uint8_t*>(a.prec) + (size_t)lb * NC * (PassRec<DK>::n * 2);
+  if (tid == 0) prefetch_tensormap(&tm_do);
+  pdl_wait();  // the preparation kernel has finished
+  pdl_trigger();
+  if (tid == 0) {
+    mbar_init(&bar_full[0], 1);
+    mbar_init(&bar_full[1], 1);
+    mbar_init(&bar_free[0], 1);
+    mbar_init(&bar_free[1], 1);
+    mbar_init(&bar_as, 128);
+    mbar_init(&bar_p, 1);
+    mbar_init(&bar_av, 128);
+    mbar_init(&bar_s, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = tmem_base;
+  auto chunk_of = [&](int it) { return role ? NC - 1 - it : it; };
+
+  if (warp == 5) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0) {
+      auto load = [&](int it) {
+        const int n = chunk_of(it), s = it & 1;
+        uint8_t* st = sm + s * kStage;
+        const size_t rec = (size_t)lb * NC + n;
+        const uint8_t* rp = recs + (size_t)n * (PassRec<DK>::n * 2);
+        if (role == 0) {
+          mbar_expect_tx(&bar_full[s], 2 * 16384 + 32768 + 512);
+          bulk_load(st + kStW, rp + TcRec::oW, 16384, &bar_full[s]);
+          bulk_load(st + kStKb, rp + TcRec::oKb, 16384, &bar_full[s]);
+          bulk_load(st + kStU, a.U + rec * kC * DV, 32768, &bar_full[s]);
+        } else {
+          mbar_expect_tx(&bar_full[s], TcRec::bytes + 16384 + 512);
+          bulk_load(st, rp, TcRec::bytes, &bar_full[s]);
+          tma_load_4d(st + kStO, &tm_do, &bar_full[s], 0, h, n * kC, b);
+          tma_load_4d(st + kStO + 8192, &tm_do, &bar_full[s], 64, h, n * kC, b);
+        }
+        bulk_load(st + kStGam, a.gam + rec * DK, 512, &bar_full[s]);
+      };
+      for (int it = 0; it < 2 && it < NC; ++it) load(it);
+      // A stage is refilled once the products of the chunk it held are done
+      // (every read of it by the state rows precedes their last arrival).
+      for (int it = 0; it + 2 < NC; ++it) {
+        wait_or_flag(&bar_free[it & 1], (it >> 1) & 1, hdr, 60);
+        load(it + 2);
+      }
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t id_k64 = idesc_bf16_f32(128, 64, 0, 0);    // A tensor memory, B K-major, N = 64 tokens
+      const uint32_t id_m128 = idesc_bf16_f32(128, 128, 0, 1);  // A tensor memory, B MN-major, N = 128 channels
+      const uint32_t id_o64 = idesc_bf16_f32(128, 64, 1, 1);    // A = dO^T (MN-major), B MN-major, N = 64
+      const uint32_t id_o128 = idesc_bf16_f32(128, 128, 1, 1);  // A = dO^T, B MN-major, N = 128
+      for (int it = 0; it < NC; ++it) {
+        const int s = it & 1;
+        const uint32_t st = smem_u32(sm + s * kStage);
+        wait_or_flag(&bar_full[s], (it >> 1) & 1, hdr, 61);
+        wait_or_flag(&bar_as, it & 1, hdr, 62);
+        tc_fence_after();
+        // K-major view of a token-row tile: 16 channels per step, +8 KiB per 64-channel block
+        auto kview = [&](uint32_t off, int k) {
+          return desc_sw128(st + off, 16, 1024) + (uint64_t)((((k >> 2) * 8192) + (k & 3) * 32) >> 4);
+        };
+        // MN-major view (N or M = channels, two 64-wide blocks 8 KiB apart): 16 tokens per step
+        auto mview = [&](uint32_t off, int k) { return desc_sw128(st + off, 8192, 1024) + (uint64_t)((2 * k * 1024) >> 4); };
+        if (role == 0) {
+#pragma unroll
+          for (int k = 0; k < DK / 16; ++k)  // P = S0^T W^T
+            mma_bf16_ts(tm + kTmAcc, tm + kTmAS + k * 8, kview(kStW, k), id_k64, k > 0);
+        } else {
+#pragma unroll
+          for (int k = 0; k < kC / 16; ++k)  // dV'^T = dO^T Aqk ...
+            mma_bf16(tm + kTmAcc, mview(kStO, k), mview(kStAqk, k), id_o64, k > 0);
+#pragma unroll
+          for (int k = 0; k < DK / 16; ++k)  // ... + dS^T Kbar^T
+            mma_bf16_ts(tm + kTmAcc, tm + kTmAS + k * 8, kview(kStKb, k), id_k64, 1);
+        }
+        mma_commit(&bar_p);
+        wait_or_flag(&bar_av, it & 1, hdr, 63);
+        tc_fence_after();
+        if (role == 0) {
+#pragma unroll
+          for (int k = 0; k < kC / 16; ++k)  // S^T += V'^T Kbar
+            mma_bf16_ts(tm + kTmS, tm + kTmAV + k * 8, mview(kStKb, k), id_m128, 1);
+        } else {
+#pragma unroll
+          for (int k = 0; k < kC / 16; ++k)  // dS^T += dO^T Q+ ...
+            mma_bf16(tm + kTmS, mview(kStO, k), mview(kStQ, k), id_o128, 1);
+#pragma unroll
+          for (int k = 0; k < kC / 16; ++k)  // ... + (-dV'^T) W
+            mma_bf16_ts(tm + kTmS, tm + kTmAV + k * 8, mview(kStW, k), id_m128, 1);
+        }
+        mma_commit(&bar_s);
+        mma_commit(&bar_free[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ state rows
+    const int j = tid;  // value channel = tensor-memory lane
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    {
+      const float* init = role == 0 ? a.s0 : a.dsT;
+#pragma unroll
+      for (int q = 0; q < DK / 32; ++q) {
+        float v[32];
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii) v[ii] = init ? init[st0 + (size_t)(q * 32 + ii) * DV + j] : 0.f;
+        tmem_st32(tm + kTmS + lane_off + q * 32, v);
+      }
+      tmem_wait_st();
+    }
+    bf16* ck_state = reinterpret_cast<bf16*>(role == 0 ? a.S0c : a.dSc);
+    bf16* ck_v = reinterpret_cast<bf16*>(role == 0 ? a.Vp : a.dVp);
+    // The checkpoints are written after the arrivals the MMA warp waits for,
+    // so that their stores stay off the chain's critical path.
+    for (int it = 0; it < NC; ++it) {
+      const int n = chunk_of(it), s = it & 1;
+      const size_t rec = (size_t)lb * NC + n;
+      const uint8_t* st = sm + s * kStage;
+      if (it > 0) wait_or_flag(&bar_s, (it - 1) & 1, hdr, 64);
+      tc_fence_after();
+      // (1) the state as a bf16 operand (the MMA warp waits for it)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[64];
+        tmem_ld32_raw(tm + kTmS + lane_off + half * 64, r);
+        tmem_ld32_raw(tm + kTmS + lane_off + half * 64 + 32, r + 32);
+        tmem_wait_ld();
+        reg_pin<64>(r);
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pk2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+        tmem_st32u(tm + kTmAS + lane_off + half * 32, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_as);
+      // (2) the state times diag(gamma), while the first products run
+      wait_or_flag(&bar_full[s], (it >> 1) & 1, hdr, 65);
+      {
+        const float4* gam = reinterpret_cast<const float4*>(st + kStGam);
+#pragma unroll
+        for (int cb = 0; cb < DK / 32; ++cb) {
+          uint32_t r[32];
+          tmem_ld32_raw(tm + kTmS + lane_off + cb * 32, r);
+          tmem_wait_ld();
+          reg_pin<32>(r);
+          float v[32];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 gg = gam[cb * 8 + q4];
+            v[q4 * 4 + 0] = __uint_as_float(r[q4 * 4 + 0]) * gg.x;
+            v[q4 * 4 + 1] = __uint_as_float(r[q4 * 4 + 1]) * gg.y;
+            v[q4 * 4 + 2] = __uint_as_float(r[q4 * 4 + 2]) * gg.z;
+            v[q4 * 4 + 3] = __uint_as_float(r[q4 * 4 + 3]) * gg.w;
+          }
+          tmem_st32(tm + kTmS + lane_off + cb * 32, v);
+        }
+      }
+      // (3) checkpoint of the state (S0 entering the chunk, or dS leaving it), [DK][DV] bf16,
+      // from its bf16 operand image, still while the first products run
+      {
+        bf16* cs = ck_state + rec * DK * DV + j;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+          tmem_ld32_raw(tm + kTmAS + lane_off + half * 32, pk);
+          tmem_wait_ld();
+          reg_pin<32>(pk);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const __nv_bfloat162 two = *reinterpret_cast<const __nv_bfloat162*>(&pk[e]);
+            cs[(size_t)(half * 64 + 2 * e) * DV] = two.x;
+            cs[(size_t)(half * 64 + 2 * e + 1) * DV] = two.y;
+          }
+        }
+      }
+      // (4) V'^T = U^T - P (replay) or dV'^T (reverse sweep) as the operand (-dV'^T for the sweep)
+      wait_or_flag(&bar_p, it & 1, hdr, 66);
+      tc_fence_after();
+      const float* u = reinterpret_cast<const float*>(st + kStU) + j;
+      uint32_t vk[32];  // V' (or dV') packed, for the checkpoint
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+        tmem_ld32_raw(tm + kTmAcc + lane_off + half * 32, r);
+        tmem_wait_ld();
+        reg_pin<32>(r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int t = half * 32 + 2 * e;
+          float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+          if (role == 0) {
+            x0 = u[t * DV] - x0;
+            x1 = u[(t + 1) * DV] - x1;
+          }
+          vk[half * 16 + e] = pk2(x0, x1);
+          pk[e] = role == 0 ? vk[half * 16 + e] : (vk[half * 16 + e] ^ 0x80008000u);  // the sweep subtracts dV'^T W
+        }
+        tmem_st16u(tm + kTmAV + lane_off + half * 16, pk);
+      }
+      tmem_wait_st();  // also covers the decayed state
+      tc_fence_before();
+      mbar_arrive(&bar_av);
+      // (5) checkpoint of V' (or dV'), [64][DV] bf16, while the second products run
+      {
+        bf16* cv = ck_v + rec * kC * DV + j;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const __nv_bfloat162 two = *reinterpret_cast<const __nv_bfloat162*>(&vk[e]);
+          cv[(size_t)(2 * e) * DV] = two.x;
+          cv[(size_t)(2 * e + 1) * DV] = two.y;
+        }
+      }
+    }
+    wait_or_flag(&bar_s, (NC - 1) & 1, hdr, 67);
+    tc_fence_after();
+    if (role == 1 && a.ds0) {
+#pragma unroll
+      for (int q = 0; q < DK / 32; ++q) {
+        float v[32];
+        tmem_ld32(tm + kTmS + lane_off + q * 32, v);
+#pragma unroll
+        for (int ii = 0; ii < 32; ++ii) a.ds0[st0 + (size_t)(q * 32 + ii) * DV + j] = v[ii];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, 512);
+}
+}  // namespace tcpass
+
 // ------------------------------------------------------------------ kernel 3
 template <int DK, int DV>
 constexpr size_t local_a_smem() {
@@ -1242,6 +1558,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
   const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
   bf16* pr = a.prec + rec * PR::n;
+  uint8_t* prb = reinterpret_cast<uint8_t*>(pr);
+  const bool tcr = kTcPass<DK, DV> && a.tc_rec;  // record layout of the pass kernel that will read it
+  auto aqk_at = [&](int i, int j) -> bf16* {
+    return tcr ? reinterpret_cast<bf16*>(prb + TcRec::oAqk + tile_off(i, j)) : pr + PR::oAqk + i * PR::LCb + j;
+  };
   auto rows_in = [&](bf16* dst, int ld, const bf16* src, int D) {  // 64 input rows of D (zeros past the tail)
     const int per = D / 8;
     for (int idx = tid; idx < kC * per; idx += kThreads) {
@@ -1267,10 +1588,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
     const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sk + i * LKb + r));
     float2 qq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sq + i * LKb + r));
     qq.x *= a.scale, qq.y *= a.scale;
-    *reinterpret_cast<__nv_bfloat162*>(pr + PR::oKb + i * PR::LKb + r) =
-        __floats2bfloat162_rn(kk.x * __expf(GC.x - G.x), kk.y * __expf(GC.y - G.y));
-    *reinterpret_cast<__nv_bfloat162*>(pr + PR::oQp + i * PR::LKb + r) =
-        __floats2bfloat162_rn(qq.x * __expf(G.x), qq.y * __expf(G.y));
+    __nv_bfloat162* kb_dst = tcr
+                                 ? reinterpret_cast<__nv_bfloat162*>(prb + TcRec::oKb + tile_off(i, r))
+                                 : reinterpret_cast<__nv_bfloat162*>(pr + PR::oKb + i * PR::LKb + r);
+    __nv_bfloat162* qp_dst = tcr
+                                 ? reinterpret_cast<__nv_bfloat162*>(prb + TcRec::oQp + tile_off(i, r))
+                                 : reinterpret_cast<__nv_bfloat162*>(pr + PR::oQp + i * PR::LKb + r);
+    *kb_dst = __floats2bfloat162_rn(kk.x * __expf(GC.x - G.x), kk.y * __expf(GC.y - G.y));
+    *qp_dst = __floats2bfloat162_rn(qq.x * __expf(G.x), qq.y * __expf(G.y));
     if (!slow) {
       const float2 Gr = *reinterpret_cast<const float2*>(sG + kRef * LK + r);
       const float dx = G.x - Gr.x, dy = G.y - Gr.y, ex = __expf(dx), ey = __expf(dy);
@@ -1295,7 +1620,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
     zero(acc);
     warp_mma_bf16<Tl::MT, Tl::NT, DK, false, true>(acc, sQ, LKb, sY, LMb, m0, n0);
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
-      pr[PR::oAqk + i * PR::LCb + j] = __float2bfloat16_rn(j <= i ? acc[mt][nt][e] : 0.f);
+      *aqk_at(i, j) = __float2bfloat16_rn(j <= i ? acc[mt][nt][e] : 0.f);
     });
   } else {
     for (int idx = tid; idx < kC * kC; idx += kThreads) {
@@ -1309,7 +1634,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
         }
       }
       sP[i * kLC + j] = j < i ? p : 0.f;
-      pr[PR::oAqk + i * PR::LCb + j] = __float2bfloat16_rn(j <= i ? a.scale * s : 0.f);
+      *aqk_at(i, j) = __float2bfloat16_rn(j <= i ? a.scale * s : 0.f);
     }
   }
   __syncthreads();
@@ -1353,7 +1678,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_prep_bf16_kernel(const ChunkB
     float acc[Tl::MT][Tl::NT][4];
     zero(acc);
     warp_mma_bf16<Tl::MT, Tl::NT, kC, false, false>(acc, sT, LCb, sX, LKb, m0, n0);
-    acc_to_bf16(acc, pr + PR::oW, PR::LKb, m0, n0);
+    if (tcr) {  // token-row tile of the tensor-core pass
+      const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+      for (int mt = 0; mt < Tl::MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < Tl::NT; ++nt)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = m0 + 16 * mt + g + 8 * hh, c = n0 + 8 * nt + 2 * t;
+            *reinterpret_cast<__nv_bfloat162*>(prb + TcRec::oW + tile_off(r, c)) =
+                __floats2bfloat162_rn(acc[mt][nt][2 * hh], acc[mt][nt][2 * hh + 1]);
+          }
+    } else {
+      acc_to_bf16(acc, pr + PR::oW, PR::LKb, m0, n0);
+    }
   }
   {  // U = T (beta v), fp32
     using Tl = Tiling<kC, DV>;
@@ -2083,8 +2422,65 @@ cudaError_t launch_k(Kern kern, dim3 grid, size_t smem, const ChunkBwdArgs& a, c
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+// dO [B, T, H, d_v] bf16 as a 4-D tensor map (channel, head, token, batch),
+// box 64 channels x 64 tokens, 128-byte swizzle; tokens past T read as zeros.
+PFN_cuTensorMapEncodeTiled_v12000 bwd_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+bool bwd_map_bf16(CUtensorMap* map, const void* base, int B, int T, int H, int d) {
+  auto enc = bwd_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tensor-core state passes (bf16, d_k = d_v = 128): one CTA per
+// (sequence, head) of the group and role, a programmatic dependent of the
+// preparation kernel.
+cudaError_t launch_pass_tc(const ChunkBwdArgs& a, int BH, int B, WorkspaceHeader* hdr, cudaStream_t stream) {
+  CUtensorMap mo;
+  if (!bwd_map_bf16(&mo, a.d_o, B, a.T, a.H, 128)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(tcpass::bwd_pass_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)tcpass::kSmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)BH, 2);
+  cfg.blockDim = dim3(tcpass::kThreads);
+  cfg.dynamicSmemBytes = tcpass::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tcpass::bwd_pass_tc_kernel, mo, a, hdr);
+}
+
+// The tensor-core passes run one CTA per (sequence, head) and role, with all
+// 128 value channels in one tensor-memory accumulator; the warp-level passes
+// split the value channels over 4 CTAs.  With fewer than a wave of
+// tensor-core pass CTAs the split keeps more SMs busy and is faster
+// (measured: 492 vs 517 us per call at B1 H16 T4096; 13.4 vs 12.2 ms at
+// B8 H32 T8192 in favour of the tensor cores), so they take over from 148 CTAs on.
+bool tc_pass_pays(int BH) { return 2 * BH >= 148; }
+
 template <typename IO, int DK, int DV>
-cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t stream) {
+cudaError_t launch_chunk_typed(const ChunkBwdArgs& a_in, int BH, int B, WorkspaceHeader* hdr, cudaStream_t stream) {
+  ChunkBwdArgs a = a_in;
+  a.tc_rec = !std::is_same<IO, float>::value && kTcPass<DK, DV> && tc_pass_pays(BH);
   const dim3 grid((unsigned)a.NC * BH);  // chunk-major within each (sequence, head)
   cudaError_t e =
       std::is_same<IO, float>::value
@@ -2099,7 +2495,10 @@ cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t strea
     else
       e = launch_k(bwd_pass_kernel<IO, DK, DV, 64>, dim3(BH * (DV / 64), 2), pass_smem<DK, DV, 64>(), a, stream,
                    kPassThreads);
+  } else if (a.tc_rec) {
+    e = launch_pass_tc(a, BH, B, hdr, stream);
   } else {
+    (void)hdr;
     if (w32)
       e = launch_k(bwd_pass_bf16_kernel<DK, DV, 32>, dim3(BH * (DV / 32), 2), pass_bf16_smem<DK, DV, 32>(), a,
                    stream, kPassThreads);
@@ -2120,11 +2519,12 @@ cudaError_t launch_chunk_typed(const ChunkBwdArgs& a, int BH, cudaStream_t strea
 }
 
 template <typename IO>
-cudaError_t launch_chunk_dims(const ChunkBwdArgs& a, int BH, int dk, int dv, cudaStream_t stream) {
-  if (dk == 128 && dv == 128) return launch_chunk_typed<IO, 128, 128>(a, BH, stream);
-  if (dk == 128 && dv == 64) return launch_chunk_typed<IO, 128, 64>(a, BH, stream);
-  if (dk == 64 && dv == 128) return launch_chunk_typed<IO, 64, 128>(a, BH, stream);
-  return launch_chunk_typed<IO, 64, 64>(a, BH, stream);
+cudaError_t launch_chunk_dims(const ChunkBwdArgs& a, int BH, int B, WorkspaceHeader* hdr, int dk, int dv,
+                              cudaStream_t stream) {
+  if (dk == 128 && dv == 128) return launch_chunk_typed<IO, 128, 128>(a, BH, B, hdr, stream);
+  if (dk == 128 && dv == 64) return launch_chunk_typed<IO, 128, 64>(a, BH, B, hdr, stream);
+  if (dk == 64 && dv == 128) return launch_chunk_typed<IO, 64, 128>(a, BH, B, hdr, stream);
+  return launch_chunk_typed<IO, 64, 64>(a, BH, B, hdr, stream);
 }
 
 static_assert(prep_smem<128, 128>() <= 232448 && local_a_smem<128, 128>() <= 232448 &&
@@ -2133,17 +2533,30 @@ static_assert(prep_smem<128, 128>() <= 232448 && local_a_smem<128, 128>() <= 232
 
 }  // namespace
 
+// The workspace starts with a WorkspaceHeader (the error word of the bounded
+// waits of the tensor-core passes), then the per-chunk records.
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
   const size_t nrec = (size_t)B * H * (((size_t)T + kC - 1) / kC);
-  return nrec * WsPlan(dk, dv, dtype == KDA_F32).per_rec() * sizeof(float);
+  return sizeof(WorkspaceHeader) + nrec * WsPlan(dk, dv, dtype == KDA_F32).per_rec() * sizeof(float);
 }
 
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
                             float scale, const float* s0, const void* d_o, const float* dsT, void* dq, void* dk_out,
                             void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H, int dk, int dv,
                             int dtype, int gate, void* ws, size_t ws_bytes, cudaStream_t stream, float* dq32,
-                            float* dk32) {
+                            float* dk32, WorkspaceHeader* hdr) {
+  if (!hdr) {  // the header leads the caller's workspace
+    if (ws_bytes < sizeof(WorkspaceHeader)) return cudaErrorInvalidValue;
+    hdr = static_cast<WorkspaceHeader*>(ws);
+    ws = static_cast<uint8_t*>(ws) + sizeof(WorkspaceHeader);
+    ws_bytes -= sizeof(WorkspaceHeader);
+  }
+  {
+    const cudaError_t e0 = cudaMemsetAsync(hdr, 0, sizeof(WorkspaceHeader), stream);
+    if (e0 != cudaSuccess) return e0;
+  }
   ChunkBwdArgs a;
+  a.tc_rec = 0;
   a.dq32 = dq32, a.dk32 = dk32;
   a.q = q, a.k = k, a.v = v, a.g = g, a.beta = beta, a.d_o = d_o;
   a.s0 = s0, a.dsT = dsT;
@@ -2151,7 +2564,7 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
   a.scale = scale, a.T = T, a.H = H, a.NC = (T + kC - 1) / kC, a.gate = gate;
   // (sequence, head) pairs per launch group: as many as the workspace holds
   const int BH = B * H;
-  const size_t per_bh = backward_workspace_bytes(1, T, 1, dk, dv, dtype);
+  const size_t per_bh = backward_workspace_bytes(1, T, 1, dk, dv, dtype) - sizeof(WorkspaceHeader);
   const int nfit = (int)std::min<size_t>((size_t)BH, ws_bytes / per_bh);
   if (nfit < 1) return cudaErrorInvalidValue;
   const WsPlan p(dk, dv, dtype == KDA_F32);
@@ -2172,8 +2585,8 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
     a.S0c = take(p.S0c), a.dSc = take(p.dSc), a.Vp = take(p.Vp), a.dVp = take(p.dVp);
     a.dAqk = take(p.dAqk), a.dT1 = take(p.dT1), a.dQs = take(p.dQs), a.dW = take(p.dW), a.dKb = take(p.dKb);
     a.dgam = take(p.dgam), a.dbu = take(p.dbu);
-    const cudaError_t e = dtype == KDA_F32 ? launch_chunk_dims<float>(a, nbh, dk, dv, stream)
-                                           : launch_chunk_dims<__nv_bfloat16>(a, nbh, dk, dv, stream);
+    const cudaError_t e = dtype == KDA_F32 ? launch_chunk_dims<float>(a, nbh, B, hdr, dk, dv, stream)
+                                           : launch_chunk_dims<__nv_bfloat16>(a, nbh, B, hdr, dk, dv, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

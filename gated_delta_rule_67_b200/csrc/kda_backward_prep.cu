@@ -141,7 +141,9 @@ cudaError_t launch_backward_prepared(const void* q, const void* k, const void* v
                                      int dk, int dv, int dtype, int gate, int prep, void* ws, size_t ws_bytes,
                                      cudaStream_t stream) {
   const size_t rows = (size_t)B * T * H, eb = dtype == KDA_F32 ? 4 : 2;
-  uint8_t* w = static_cast<uint8_t*>(ws);
+  // the error word of the backward's bounded waits leads the workspace, then the prepared inputs
+  WorkspaceHeader* hdr = static_cast<WorkspaceHeader*>(ws);
+  uint8_t* w = static_cast<uint8_t*>(ws) + sizeof(WorkspaceHeader);
   PrepArgs a;
   a.q = q, a.k = k, a.g = g, a.beta = beta;
   a.qh = w, w += align256(rows * dk * eb);
@@ -162,7 +164,8 @@ cudaError_t launch_backward_prepared(const void* q, const void* k, const void* v
                                    : launch_pair<__nv_bfloat16>(false, a, dk, stream);
   if (e != cudaSuccess) return e;
   e = launch_backward(a.qh, a.kh, v, gate == KDA_GATE_NONE ? nullptr : a.gh, a.bh, scale, s0, d_o, dsT, dq, dk_out,
-                      dv_out, dg, dbeta, ds0, B, T, H, dk, dv, dtype, gate, w, ws_bytes - used, stream, a.dq32, a.dk32);
+                      dv_out, dg, dbeta, ds0, B, T, H, dk, dv, dtype, gate, w, ws_bytes - used, stream, a.dq32, a.dk32,
+                      hdr);
   if (e != cudaSuccess) return e;
   return dtype == KDA_F32 ? launch_pair<float>(true, a, dk, stream) : launch_pair<__nv_bfloat16>(true, a, dk, stream);
 }

@@ -20,6 +20,8 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+struct WorkspaceHeader;
+
 // Launch entry points implemented in the individual .cu files.  Arguments
 // have been validated by the API layer.  Each returns the cudaError_t of its
 // launch(es).
@@ -41,15 +43,17 @@ cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, 
                                 int dk, int dv, int chunk, int gate, int prep, void* ws, size_t ws_bytes,
                                 cudaStream_t stream, void* const* events);
 
-// Backward pass (kda_backward_chunk.cu).  The workspace holds the records of
-// one or more (sequence, head) pairs; the pairs are processed in groups of
-// as many as fit (at least backward_workspace_bytes(1, T, 1, dk, dv, dtype) bytes).
+// Backward pass (kda_backward_chunk.cu).  The workspace holds a
+// WorkspaceHeader (error word of the bounded waits; at the start of `ws`
+// unless `hdr` points elsewhere) and the records of one or more (sequence,
+// head) pairs; the pairs are processed in groups of as many as fit (at least
+// backward_workspace_bytes(1, T, 1, dk, dv, dtype) bytes, header included).
 size_t backward_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
                             float scale, const float* s0, const void* d_o, const float* dsT, void* dq, void* dk_out,
                             void* dv_out, void* dg, void* dbeta, float* ds0, int B, int T, int H, int dk, int dv,
                             int dtype, int gate, void* ws, size_t ws_bytes, cudaStream_t stream,
-                            float* dq32 = nullptr, float* dk32 = nullptr);
+                            float* dq32 = nullptr, float* dk32 = nullptr, struct WorkspaceHeader* hdr = nullptr);
 
 // Backward through the fused input preparation (kda_backward_prep.cu): the
 // workspace holds backward_prep_bytes of prepared inputs, then the records.

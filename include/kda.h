@@ -161,11 +161,13 @@ KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Bytes of device workspace kda_backward needs for this problem: per-chunk
- * records (per 64-token chunk and head: the chunk's operands, the state
- * entering it and the state gradient leaving it, and intermediate gradients;
- * about 0.33 MB for bf16 and 0.6 MB for fp32 at dk = dv = 128); 0 for
- * arguments kda_backward would reject.
+ * Bytes of device workspace kda_backward needs for this problem: a 256-byte
+ * header holding the error word of the bounded on-device waits (the same
+ * header kda_chunk_fwd_check reads), then per-chunk records (per 64-token
+ * chunk and head: the chunk's operands, the state entering it and the state
+ * gradient leaving it, and intermediate gradients; about 0.33 MB for bf16
+ * and 0.6 MB for fp32 at dk = dv = 128); 0 for arguments kda_backward would
+ * reject.
  */
 KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, int dtype);
 
@@ -205,7 +207,10 @@ KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, 
  * alignment); outputs must not overlap any input, each other or the
  * workspace.  Every sum runs in a fixed order (no atomics), so results are
  * bit-reproducible.  T = 0 or B = 0 is valid
- * (grad_initial_state = grad_final_state).
+ * (grad_initial_state = grad_final_state).  For bf16 at dk = dv = 128 the
+ * state passes run on the tcgen05 tensor cores with bounded mbarrier waits;
+ * kda_chunk_fwd_check(workspace, ...) afterwards returns KDA_ERR_TIMEOUT if
+ * one gave up (the gradients are then not valid), KDA_OK otherwise.
  */
 KDA_API kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
                                 float scale, const float* initial_state, const void* grad_o,
@@ -231,7 +236,8 @@ KDA_API size_t kda_backward_ex_workspace_size(int B, int T, int H, int dk, int d
  * dq = r (dq^ - q^ (q^ . dq^)) with r = (sum q^2 + 1e-6)^-1/2 (same for k),
  * dg = dg^ sigmoid(-g), dbeta = dbeta^ sigmoid(beta) (1 - sigmoid(beta)).
  * workspace: kda_backward_ex_workspace_size() bytes hold everything; smaller
- * works down to the prepared inputs plus one (sequence, head)'s records.
+ * works down to the prepared inputs plus one (sequence, head)'s records.  It
+ * starts with the same 256-byte error-word header as kda_backward's.
  * prep = KDA_PREP_NONE is kda_backward.  Other arguments as kda_backward.
  */
 KDA_API kda_status kda_backward_ex(const void* q, const void* k, const void* v, const void* g, const void* beta,
@@ -288,10 +294,11 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const voi
 KDA_API kda_status kda_chunk_fwd_noalloc_check(void* stream);
 
 /*
- * Reads the on-device error word that the last kda_chunk_fwd using this
- * workspace left behind (synchronises `stream`).  Returns KDA_OK, or
- * KDA_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the outputs of
- * that call are then not valid).  A workspace of size 0 always reports KDA_OK.
+ * Reads the on-device error word that the last kda_chunk_fwd (or
+ * kda_backward / kda_backward_ex) using this workspace left behind
+ * (synchronises `stream`).  Returns KDA_OK, or KDA_ERR_TIMEOUT if a bounded
+ * wait inside a kernel gave up (the outputs of that call are then not
+ * valid).  A workspace of size 0 always reports KDA_OK.
  */
 KDA_API kda_status kda_chunk_fwd_check(const void* workspace, size_t workspace_bytes, void* stream);
 

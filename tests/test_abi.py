@@ -186,7 +186,8 @@ def test_backward_validation(lib):
     assert fx(*ins, 1.0, None, A + (5 << 30), None, *grads, None, 1, 64, 1, 128, 128, 1, 0, 7, A + (20 << 30),
               one, None) == binding.KDA_ERR_INVALID_ARG                    # no room for the prepared inputs
     assert call(wsb=one - 1) == binding.KDA_ERR_INVALID_ARG           # below one (sequence, head)'s records
-    assert lib.kda_backward_workspace_size(2, 64, 3, 128, 128, 1) == 6 * one
+    # a 256-byte error-word header, then the records of every (sequence, head)
+    assert lib.kda_backward_workspace_size(2, 64, 3, 128, 128, 1) == 256 + 6 * (one - 256)
     bad = list(grads)
     bad[0] = A + 64                                                   # grad_q overlaps q
     assert call(grads=bad) == binding.KDA_ERR_INVALID_ARG

@@ -221,3 +221,51 @@ def test_backward_long_chain():
     """One (sequence, head) over 65,536 tokens (1,024 chunks, bf16): the state
     passes carry the state and its gradient through the whole chain."""
     _case(1, 65536, 1, 128, 128, torch.bfloat16, seed=111)
+
+
+def test_backward_error_word_and_many_waves():
+    """bf16, d = 128 (the tensor-core state passes): 160 (sequence, head)
+    chains x 2 roles = 320 pass CTAs (more than one wave of SMs); every
+    gradient against the oracle, and the workspace's error word reads clear."""
+    from gated_delta_rule_67_b200 import binding, kda_chunk_fwd_check
+    dev = cuda_or_skip()
+    B, T, H, d = 4, 150, 40, 128
+    x = make_prefill_inputs(B, T, H, d, d, torch.bfloat16, 0.1, seed=97)
+    d_o, d_s = make_cotangents(B, T, H, d, d, torch.bfloat16, seed=98)
+    ws = torch.empty(int(binding.load().kda_backward_workspace_size(B, T, H, d, d, 1)), dtype=torch.uint8, device=dev)
+    ws.fill_(0xCD)
+    to = lambda t: t.to(dev)
+    got = kda_backward(to(x["q"]), to(x["k"]), to(x["v"]), to(x["g"]), to(x["beta"]), to(d_o), None,
+                       to(x["initial_state"]), to(d_s), workspace=ws)
+    assert kda_chunk_fwd_check(ws) == binding.KDA_OK
+    ref = oracle.kda_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d ** -0.5, x["initial_state"], d_o, d_s)
+    for name in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        assert rel_err(got[name], ref[name]) < TOL[torch.bfloat16], name
+
+
+@pytest.mark.parametrize("T,gate,s0,final", [(100, "channel", 0.1, True), (64 * 3 + 7, "head", 0.1, True),
+                                             (70, "none", 0.1, True), (1, "channel", 0.1, True),
+                                             (130, "channel", 0.0, False)])
+def test_backward_tensor_core_passes(T, gate, s0, final):
+    """bf16, d = 128 with at least a wave of pass CTAs (2 x 40 heads x 2 sequences):
+    the state passes run on the tcgen05 tensor cores.  Gate kinds, chunk tails,
+    a single token, zero initial state without a final-state gradient."""
+    _case(2, T, 40, 128, 128, torch.bfloat16, gate=gate, s0=s0, final=final, seed=120 + T)
+
+
+def test_backward_tensor_core_passes_exact_path():
+    """The exact pairwise path of the preparation (gates of exp(-20)) feeding the tensor-core passes."""
+    dev = cuda_or_skip()
+    B, T, H, d = 2, 150, 40, 128
+    x = make_prefill_inputs(B, T, H, d, d, torch.bfloat16, 0.1, seed=131)
+    g = x["g"].float()
+    g[:, 64:128, :5, :8] = -20.0
+    x["g"] = g.to(torch.bfloat16)
+    d_o, d_s = make_cotangents(B, T, H, d, d, torch.bfloat16, seed=132)
+    to = lambda t: t.to(dev)
+    got = kda_backward(*(to(x[n]) for n in ("q", "k", "v", "g", "beta")), to(d_o), None, to(x["initial_state"]),
+                       to(d_s))
+    torch.cuda.synchronize()
+    ref = oracle.kda_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d ** -0.5, x["initial_state"], d_o, d_s)
+    for name in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
+        assert rel_err(got[name], ref[name]) < TOL[torch.bfloat16], name
