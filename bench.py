@@ -589,7 +589,7 @@ def time_backward(cfg, calls, rank, world, dev, flush, stream, peaks):
 
 
 def main(argv=None):
-    from gated_delta_rule_67_b200.workloads import LONG_BF16, PREFILL_BF16, PREFILL_CONFIGS, TRAIN_BF16
+    from gated_delta_rule_67_b200.workloads import LONG_BF16, PREFILL_BF16, PREFILL_CONFIGS, TINY_F32, TRAIN_BF16
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
@@ -597,7 +597,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=LONG_BF16.name, choices=sorted(PREFILL_CONFIGS),
                     help="headline prefill workload (default: the largest single-GPU one, T = 1,048,576)")
-    ap.add_argument("--also", nargs="*", default=[TRAIN_BF16.name, PREFILL_BF16.name],
+    ap.add_argument("--also", nargs="*", default=[TRAIN_BF16.name, PREFILL_BF16.name, TINY_F32.name],
                     help="further prefill workloads timed under the same rules (extra keys)")
     ap.add_argument("--backward-workloads", nargs="*", default=[PREFILL_BF16.name, TRAIN_BF16.name])
     ap.add_argument("--e2e-steps", type=int, default=5)

@@ -78,7 +78,12 @@ TRAIN_BF16 = PrefillConfig("train_bf16_B8_H32_T8192_d128", 8, 32, 8192, 128, 128
 LONG_BF16 = PrefillConfig("long_bf16_B1_H32_T1048576_d128", 1, 32, 1 << 20, 128, 128, 64, "bf16", 0.1, 3)
 DECODE_BF16 = DecodeConfig("decode_bf16_N256_H32_d128_1000steps", 256, 32, 128, 128, 1000, "bf16", 0.1, 4)
 
-PREFILL_CONFIGS = {c.name: c for c in (TINY_F32, PREFILL_BF16, TRAIN_BF16, LONG_BF16)}
+# The first 65,536 tokens of the long-context workload (same seed, same
+# recipe): the same chunk-parallel scan structure (3 groups per chain) at a
+# size whose DRAM traffic a profiler can capture; per-call traffic scales with T.
+LONG_PREFIX_BF16 = PrefillConfig("long_prefix_bf16_B1_H32_T65536_d128", 1, 32, 1 << 16, 128, 128, 64, "bf16", 0.1, 3)
+
+PREFILL_CONFIGS = {c.name: c for c in (TINY_F32, PREFILL_BF16, TRAIN_BF16, LONG_BF16, LONG_PREFIX_BF16)}
 
 _SLAB_ELEMS = 1 << 27  # fp32 elements drawn per slab (512 MB), bounds temporaries
 
