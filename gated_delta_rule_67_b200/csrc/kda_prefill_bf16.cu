@@ -709,6 +709,20 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
 constexpr int kSPThreads = 288;
 constexpr uint32_t kTmP = 0, kTmO = 64, kTmS = 128, kTmAS = 256, kTmAV = 320;
 
+// The passes without outputs (the scan's offset and transition passes) run
+// a lighter instance of the same kernel, two CTAs per SM: 192 threads (state
+// warps 0-3, warp 4 streams the records, warp 5 issues the MMAs), 256 columns
+// of tensor memory ([P | S^T | S0^T bf16], V'^T in bf16 written over the P
+// columns it was formed from), compact stages holding only -W (its two
+// 64-channel halves 8 KiB apart), Kbar, U and gamma, and the start state
+// read straight from global memory.
+constexpr int kSPThreadsNoOut = 192;
+constexpr uint32_t kTmSNo = 64, kTmASNo = 192;  // P at 0, V'^T bf16 over P's first 32 columns
+constexpr uint32_t kCW = 0, kCKbar = 16384, kCU = 32768, kCGamma = 49152;  // compact stage offsets
+constexpr uint32_t kStageNoOut = 50176;      // 49 KiB
+constexpr uint32_t kP2BytesNoOut = 2 * kStageNoOut;
+static_assert(kCGamma + 512 <= kStageNoOut, "compact stage");
+
 // Brings the record of one chunk into a stage.  A pass that writes outputs
 // needs all of it; a pass without outputs reads only -W (the first 64 rows
 // of each 64-column block of [-W; Q+]), Kbar, U and gamma; the transition
@@ -732,6 +746,22 @@ __device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, 
     bulk_load(stage + kRecKbar, rec + kRecKbar, kRecBytes - kRecKbar, bar);
   }
 }
+
+// The same parts into a compact stage: -W's halves (rows 0-63 of each
+// 64-column block) to [0, 16K), then Kbar, U and gamma, contiguous in the
+// record, to [16K, 48.5K) (U skipped for the transition pass).
+__device__ __forceinline__ void load_record_compact(uint8_t* stage, const uint8_t* rec, uint64_t* bar, bool zero_u) {
+  mbar_expect_tx(bar, zero_u ? kRecTransBytes : kRecNoOutBytes);
+  bulk_load(stage + kCW, rec + kRecWQ, 8192, bar);
+  bulk_load(stage + kCW + 8192, rec + kRecWQ + 16384, 8192, bar);
+  if (zero_u) {
+    bulk_load(stage + kCKbar, rec + kRecKbar, kRecU - kRecKbar, bar);
+    bulk_load(stage + kCGamma, rec + kRecGamma, kRecBytes - kRecGamma, bar);
+  } else {
+    bulk_load(stage + kCKbar, rec + kRecKbar, kRecBytes - kRecKbar, bar);
+  }
+}
+static_assert(kCU - kCKbar == kRecU - kRecKbar && kCGamma - kCKbar == kRecGamma - kRecKbar, "compact = record order");
 
 // What one state-pass CTA does.  Phase 0: a whole chain.  With the
 // chunk-parallel scan (few chains, long sequences) a chain is cut into G
@@ -758,7 +788,8 @@ struct StatePassArgs {
   int T, H, NC, G, L, phase, dk, dv;
 };
 
-__global__ void __launch_bounds__(kSPThreads, 1)
+template <bool kOut>
+__global__ void __launch_bounds__(kOut ? kSPThreads : kSPThreadsNoOut, kOut ? 1 : 2)
     kda_state_pass_kernel(const __grid_constant__ CUtensorMap tm_o, const StatePassArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -774,7 +805,13 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   const size_t kUserSt = (size_t)dk * dv;
   int bh, cb, ce;
   const float* init = nullptr;  // null: zero start
-  bool ident = false, zero_u = false, out = true;
+  bool ident = false, zero_u = false;
+  // Phases 0 and 3 write outputs (full instance).  Phase 1 writes none: the
+  // light instance for long chains, the full one otherwise.
+  const bool out = kOut && args.phase != 1;
+  constexpr uint32_t kStg = kOut ? kStage : kStageNoOut;
+  constexpr int kMmaWarp = kOut ? 8 : 5;
+  constexpr uint32_t tP = kTmP, tS = kOut ? kTmS : kTmSNo, tAS = kOut ? kTmAS : kTmASNo, tAV = kOut ? kTmAV : kTmP;
   bool init_user = false, fin_user = false;  // caller's [dk][dv] layout (else the internal 128 x 128)
   float* fin = nullptr;
   float* init_copy = nullptr;  // phase 1, group 0: the start state is also kept in sbuf slot 0
@@ -789,7 +826,6 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     const int per = 2 * G - 3;
     bh = blockIdx.x / per;
     const int r = blockIdx.x % per;
-    out = false;
     int g;
     if (r < G - 1) {
       g = r;
@@ -836,21 +872,21 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     mbar_init(&bar_av, 128);
     mbar_init(&bar_init, 1);
     fence_mbar_init();
-    if (init) {  // the start state, row-major fp32, into stage 1 (its record follows once it is read)
+    if (kOut && init) {  // the start state, row-major fp32, into stage 1 (its record follows once it is read)
       const uint32_t bytes = (uint32_t)((init_user ? kUserSt : kSt) * sizeof(float));  // 16, 32 or 64 KiB
       mbar_expect_tx(&bar_init, bytes);
       for (uint32_t p = 0; p < bytes / 16384; ++p)
         bulk_load(sm + kStage + p * 16384, init + p * 4096, 16384, &bar_init);
     }
   }
-  if (warp == 0) tmem_alloc(&tmem_base, 512);
+  if (warp == 0) tmem_alloc(&tmem_base, kOut ? 512 : 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
   if (args.phase == 1) grid_dep_launch();  // the combination kernel may be scheduled
 
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     // ------------------------------------------------------------ mma
     if ((tid & 31) == 0) {
       // P = S0^T (-W)^T (N=64) first, committed alone so that V' can be formed
@@ -859,13 +895,14 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       // closes the chunk; without outputs S += V'^T Kbar (N=128).
       const uint32_t id_1 = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id_2 = idesc_bf16_f32(128, out ? 192 : 128, 0, 1);
-      const uint32_t d2_off = out ? 0 : (8192 >> 4);  // skip the A_qk^T block
-      const uint32_t t2 = out ? tm + kTmO : tm + kTmS;
+      const uint32_t t2 = out ? tm + kTmO : tm + tS;
       // first descriptors of each stage; later steps add address offsets (in 16-byte units)
-      const uint64_t d1s0 = desc_sw128(smem_u32(sm + kRecWQ), 16, 1024);
-      const uint64_t d1s1 = desc_sw128(smem_u32(sm + kStage + kRecWQ), 16, 1024);
-      const uint64_t d2s0 = desc_sw128(smem_u32(sm + kRecAqk), 8192, 1024) + d2_off;
-      const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStage + kRecAqk), 8192, 1024) + d2_off;
+      const uint32_t oW = kOut ? kRecWQ : kCW, oB = kOut ? (out ? kRecAqk : kRecKbar) : kCKbar;
+      constexpr uint32_t kWBlk = kOut ? 16384 : 8192;  // bytes between the 64-channel blocks of -W
+      const uint64_t d1s0 = desc_sw128(smem_u32(sm + oW), 16, 1024);
+      const uint64_t d1s1 = desc_sw128(smem_u32(sm + kStg + oW), 16, 1024);
+      const uint64_t d2s0 = desc_sw128(smem_u32(sm + oB), 8192, 1024);
+      const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStg + oB), 8192, 1024);
       constexpr uint64_t kQoff = 8192 >> 4;  // rows 64-127 (Q+) of each 64-column block of [-W; Q+]
       for (int n = 0; n < NCL; ++n) {
         const int s = n & 1;
@@ -874,21 +911,21 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         tc_fence_after();
         const uint64_t d1 = s ? d1s1 : d1s0, d2 = s ? d2s1 : d2s0;
 #pragma unroll
-        for (int k = 0; k < kD / 16; ++k)  // K-major B: +32 B per step inside a 64-wide block, +16 KiB per block
-          mma_bf16_ts(tm + kTmP, tm + kTmAS + k * 8, d1 + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), id_1,
+        for (int k = 0; k < kD / 16; ++k)  // K-major B: +32 B per step inside a 64-wide block
+          mma_bf16_ts(tm + tP, tm + tAS + k * 8, d1 + (uint64_t)(((k / 4) * kWBlk + (k % 4) * 32) >> 4), id_1,
                       k > 0);
         mma_commit(&bar_p);
         if (out) {  // bar_as also covered the read of O^T of chunk n-1
 #pragma unroll
           for (int k = 0; k < kD / 16; ++k)
-            mma_bf16_ts(tm + kTmO, tm + kTmAS + k * 8,
+            mma_bf16_ts(tm + kTmO, tm + tAS + k * 8,
                         d1 + kQoff + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), id_1, k > 0);
         }
         wait_or_flag(&bar_av, n & 1, hdr, 33);
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kC / 16; ++k)  // MN-major B: +2 KiB per 16 K-rows
-          mma_bf16_ts(t2, tm + kTmAV + k * 8, d2 + (uint64_t)((2 * k * 1024) >> 4), id_2, 1);
+          mma_bf16_ts(t2, tm + tAV + k * 8, d2 + (uint64_t)((2 * k * 1024) >> 4), id_2, 1);
         mma_commit(&bar_s);
         mma_commit(&bar_o);
       }
@@ -898,8 +935,12 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     const int j = tid - 128;
     const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
     if (tid == 128) {
-      for (int n = 0; n < 2 && n < NCL; ++n)
-        if (n == 0 || !init) load_record(sm + n * kStage, recs + (size_t)n * kRecBytes, &bar_full[n], out, zero_u);
+      for (int n = 0; n < 2 && n < NCL; ++n) {
+        if (!kOut)
+          load_record_compact(sm + n * kStg, recs + (size_t)n * kRecBytes, &bar_full[n], zero_u);
+        else if (n == 0 || !init)
+          load_record(sm + n * kStage, recs + (size_t)n * kRecBytes, &bar_full[n], out, zero_u);
+      }
     }
     // With outputs, each chunk's bar_as phase also waits for these 128
     // threads: the first has nothing to release, later ones the O^T of the
@@ -910,8 +951,12 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       wait_or_flag(&bar_o, n & 1, hdr, 21);
       tc_fence_after();
       if (!out) {
-        if (tid == 128 && n + 2 < NCL)
-          load_record(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, &bar_full[s], false, zero_u);
+        if (tid == 128 && n + 2 < NCL) {
+          if (kOut)
+            load_record(sm + s * kStage, recs + (size_t)(n + 2) * kRecBytes, &bar_full[s], false, zero_u);
+          else
+            load_record_compact(sm + s * kStg, recs + (size_t)(n + 2) * kRecBytes, &bar_full[s], zero_u);
+        }
         continue;
       }
       uint32_t r[64];
@@ -947,9 +992,10 @@ __global__ void __launch_bounds__(kSPThreads, 1)
     const int j = tid;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     {
-      // column j of the start state (row j of S^T) into lane j
-      const float* s0s = reinterpret_cast<const float*>(sm + kStage);
-      if (init) wait_or_flag(&bar_init, 0, hdr, 20);
+      // column j of the start state (row j of S^T) into lane j: from stage 1
+      // (with outputs) or straight from global memory (without)
+      const float* s0s = kOut ? reinterpret_cast<const float*>(sm + kStage) : init;
+      if (kOut && init) wait_or_flag(&bar_init, 0, hdr, 20);
       float v[32];
 #pragma unroll
       for (int q = 0; q < kD / 32; ++q) {
@@ -964,17 +1010,18 @@ __global__ void __launch_bounds__(kSPThreads, 1)
             v[ii] = s0s[c * kD + j];
           if (init_copy) init_copy[(size_t)c * kD + j] = v[ii];
         }
-        tmem_st32(tm + kTmS + lane_off + q * 32, v);
+        tmem_st32(tm + tS + lane_off + q * 32, v);
       }
       tmem_wait_st();
-      if (init) {  // stage 1 is free again: bring the record of chunk 1
+      if (kOut && init) {  // stage 1 is free again: bring the record of chunk 1
         named_bar_sync(1, 128);
         if (tid == 0 && NCL > 1) load_record(sm + kStage, recs + kRecBytes, &bar_full[1], out, zero_u);
       }
     }
+    constexpr uint32_t oU = kOut ? kRecU : kCU, oGam = kOut ? kRecGamma : kCGamma;
     for (int n = 0; n < NCL; ++n) {
       const int s = n & 1;
-      const uint8_t* stage = sm + s * kStage;
+      const uint8_t* stage = sm + s * kStg;
       if (n > 0) wait_or_flag(&bar_s, (n - 1) & 1, hdr, 22);
       tc_fence_after();
 
@@ -982,14 +1029,14 @@ __global__ void __launch_bounds__(kSPThreads, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t sr[64];
-        tmem_ld32_raw(tm + kTmS + lane_off + half * 64, sr);
-        tmem_ld32_raw(tm + kTmS + lane_off + half * 64 + 32, sr + 32);
+        tmem_ld32_raw(tm + tS + lane_off + half * 64, sr);
+        tmem_ld32_raw(tm + tS + lane_off + half * 64 + 32, sr + 32);
         tmem_wait_ld();
         reg_pin<64>(sr);
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
-        tmem_st32u(tm + kTmAS + lane_off + half * 32, pk);
+        tmem_st32u(tm + tAS + lane_off + half * 32, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -998,11 +1045,11 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       // (2) S^T <- S^T Diag(gamma) while the MMAs run
       wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 25);
       {
-        const float4* gam = reinterpret_cast<const float4*>(stage + kRecGamma);
+        const float4* gam = reinterpret_cast<const float4*>(stage + oGam);
 #pragma unroll
         for (int cb = 0; cb < kD / 32; ++cb) {
           uint32_t sr[32];
-          tmem_ld32_raw(tm + kTmS + lane_off + cb * 32, sr);
+          tmem_ld32_raw(tm + tS + lane_off + cb * 32, sr);
           tmem_wait_ld();
           reg_pin<32>(sr);
           float v[32];
@@ -1014,7 +1061,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
             v[q4 * 4 + 2] = __uint_as_float(sr[q4 * 4 + 2]) * gg.z;
             v[q4 * 4 + 3] = __uint_as_float(sr[q4 * 4 + 3]) * gg.w;
           }
-          tmem_st32(tm + kTmS + lane_off + cb * 32, v);
+          tmem_st32(tm + tS + lane_off + cb * 32, v);
         }
       }
 
@@ -1022,13 +1069,13 @@ __global__ void __launch_bounds__(kSPThreads, 1)
       uint4 urow[4];
 #pragma unroll
       for (int k8 = 0; k8 < 4; ++k8)
-        urow[k8] = *reinterpret_cast<const uint4*>(stage + kRecU + kmajor_off(j, k8 * 8, kD));
+        urow[k8] = *reinterpret_cast<const uint4*>(stage + oU + kmajor_off(j, k8 * 8, kD));
       wait_or_flag(&bar_p, n & 1, hdr, 26);
       tc_fence_after();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pr[32];
-        tmem_ld32_raw(tm + kTmP + lane_off + half * 32, pr);
+        tmem_ld32_raw(tm + tP + lane_off + half * 32, pr);
         tmem_wait_ld();
         reg_pin<32>(pr);
         uint32_t pk[16];
@@ -1046,9 +1093,10 @@ __global__ void __launch_bounds__(kSPThreads, 1)
         if (half == 0) {
 #pragma unroll
           for (int k8 = 0; k8 < 4; ++k8)
-            urow[k8] = *reinterpret_cast<const uint4*>(stage + kRecU + kmajor_off(j, 32 + k8 * 8, kD));
+            urow[k8] = *reinterpret_cast<const uint4*>(stage + oU + kmajor_off(j, 32 + k8 * 8, kD));
         }
-        tmem_st16u(tm + kTmAV + lane_off + half * 16, pk);
+        // without outputs V'^T goes over the P columns this thread has just read
+        tmem_st16u(tm + tAV + lane_off + half * 16, pk);
       }
       tmem_wait_st();  // also covers the decayed S^T
       tc_fence_before();
@@ -1060,7 +1108,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
 #pragma unroll
       for (int q = 0; q < kD / 32; ++q) {
         float v[32];
-        tmem_ld32(tm + kTmS + lane_off + q * 32, v);
+        tmem_ld32(tm + tS + lane_off + q * 32, v);
         if (ident) {
           // A transition matrix is stored as the bf16 K-major 128-row image of
           // M (row r, column j at kmajor_off(r, j)), the B operand of the
@@ -1083,7 +1131,7 @@ __global__ void __launch_bounds__(kSPThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem_base, 512);
+  if (warp == 0) tmem_dealloc(tmem_base, kOut ? 512 : 256);
 }
 
 // ======================================================== scan combine
@@ -1268,13 +1316,29 @@ cudaError_t launch_wait_selftest(void* ws, cudaStream_t stream) {
 }
 
 // Groups of the chunk-parallel scan for B*H chains of NC chunks (1 = no scan).
-// Phase 1 runs 2G-3 CTAs per chain, sized to one wave of a 148-SM part; the
-// count is a fixed function of the shape so results do not depend on the GPU.
+// Phase 3 runs G CTAs per chain, one per SM of a 148-SM part; phase 1 runs
+// 2G-3 lighter CTAs per chain (two fit an SM).  The count is a fixed function
+// of the shape so results do not depend on the GPU.
 constexpr int kScanSMs = 148;
 constexpr int kScanMinChunks = 4;
-void scan_groups(int BH, int NC, int* G_out, int* L_out) {
+// With long chains (at least kScanLongChunks chunks per group at one phase-1
+// CTA per SM) the group count is as large as the light phase-1 CTAs allow
+// (two per SM, phase 3 still one wave): every group is shorter, which is what
+// the sequential passes cost.  Otherwise more groups only add combination
+// steps and launches (measured: 134 vs 77 us of state passes at B1 H16
+// T4096 with 8 groups of 8 chunks instead of 6 of 11).
+constexpr int kScanLongChunks = 256;
+void scan_groups(int BH, int NC, int* G_out, int* L_out, bool* light = nullptr) {
   int G = 1;
-  if (BH > 0 && 3 * BH <= kScanSMs) G = std::min((kScanSMs / BH + 3) / 2, NC / kScanMinChunks);
+  bool lt = false;
+  if (BH > 0 && 3 * BH <= kScanSMs) {
+    G = std::min((kScanSMs / BH + 3) / 2, NC / kScanMinChunks);
+    if (G >= 3 && NC / G >= kScanLongChunks) {
+      G = std::min(std::min(kScanSMs / BH, (2 * kScanSMs / BH + 3) / 2), NC / kScanMinChunks);
+      lt = true;
+    }
+  }
+  if (light) *light = lt;
   if (G >= 3) {
     const int L = (NC + G - 1) / G;
     G = (NC + L - 1) / L;
@@ -1345,7 +1409,14 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
       if (e != cudaSuccess) return e;
     }
     cudaError_t e;
-    e = cudaFuncSetAttribute(kda_state_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kP2Bytes + 1024);
+    e = cudaFuncSetAttribute(kda_state_pass_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kP2Bytes + 1024);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kda_state_pass_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kP2BytesNoOut + 1024);
+    if (e != cudaSuccess) return e;
+    // two of them share an SM
+    e = cudaFuncSetAttribute(kda_state_pass_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCbSmem);
     if (e != cudaSuccess) return e;
@@ -1376,9 +1447,10 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   StatePassArgs a{records, hdr, s0, sT, nullptr, nullptr, nullptr, T, H, NC, 1, NC, 0, dk, dv};
   const int BH = B * H;
   int G, L;
-  scan_groups(BH, NC, &G, &L);
+  bool light = false;
+  scan_groups(BH, NC, &G, &L, &light);
   if (G == 1) {
-    e = launch_dependent(kda_state_pass_kernel, (unsigned)BH, kSPThreads, kP2Bytes + 1024, stream, mo, a);
+    e = launch_dependent(kda_state_pass_kernel<true>, (unsigned)BH, kSPThreads, kP2Bytes + 1024, stream, mo, a);
   } else {
     float* scan = reinterpret_cast<float*>(records + (size_t)BH * NC * kRecBytes);
     const size_t per = (size_t)BH * G * kD * kD;
@@ -1388,14 +1460,16 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     a.G = G;
     a.L = L;
     a.phase = 1;
-    e = launch_dependent(kda_state_pass_kernel, (unsigned)(BH * (2 * G - 3)), kSPThreads, kP2Bytes + 1024, stream,
-                         mo, a);
+    e = light ? launch_dependent(kda_state_pass_kernel<false>, (unsigned)(BH * (2 * G - 3)), kSPThreadsNoOut,
+                                 kP2BytesNoOut + 1024, stream, mo, a)
+              : launch_dependent(kda_state_pass_kernel<true>, (unsigned)(BH * (2 * G - 3)), kSPThreads,
+                                 kP2Bytes + 1024, stream, mo, a);
     if (e != cudaSuccess) return e;
     e = launch_dependent(kda_scan_combine_kernel, (unsigned)BH, kCbThreads, kCbSmem, stream, scan + 2 * per,
                          (const float*)scan, (const float*)(scan + per), G, hdr);
     if (e != cudaSuccess) return e;
     a.phase = 3;
-    e = launch_dependent(kda_state_pass_kernel, (unsigned)(BH * G), kSPThreads, kP2Bytes + 1024, stream, mo, a);
+    e = launch_dependent(kda_state_pass_kernel<true>, (unsigned)(BH * G), kSPThreads, kP2Bytes + 1024, stream, mo, a);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 2, stream);

@@ -241,3 +241,20 @@ def test_scan_with_extreme_gates_and_in_place_state():
     torch.cuda.synchronize()
     assert rel_err(o, ref_o) < TOLB
     assert rel_err(state, ref_s) < TOLB
+
+
+@pytest.mark.parametrize("d,in_place", [(128, False), (64, True)])
+def test_long_chains_light_offset_passes(d, in_place):
+    """Few chains of many chunks (8 heads x 2600 chunks and a ragged tail):
+    the scan's offset and transition passes run two per SM on the light
+    instance of the state pass, with more groups; against the oracle (with
+    d = 64 and the final state written over the initial state as well)."""
+    dev = cuda_or_skip()
+    B, T, H = 1, 64 * 2600 + 17, 8
+    x = make_prefill_inputs(B, T, H, d, d, torch.bfloat16, 0.1, seed=150 + d, device="cpu")
+    ref_o, ref_s = _oracle(x)
+    state = x["initial_state"].to(dev)
+    o, sT = kda_chunk_fwd(*(x[n].to(dev) for n in NAMES), None, state, final_state=state if in_place else None)
+    torch.cuda.synchronize()
+    assert rel_err(o, ref_o) < TOLB
+    assert rel_err(state if in_place else sT, ref_s) < TOLB
