@@ -68,10 +68,10 @@ constexpr int kRefTok = 31;  // reference token of the factored form: the end of
 static_assert(kRefTok == 2 * 16 - 1, "pass 1 takes G_r as the sum of the first two stride totals");
 
 // --- per-chunk record in the workspace (byte offsets) -----------------------
-constexpr uint32_t kRecWQ = 0;          // [-W ; Q+]: K-major, 128 rows x 128 ch (32 KiB)
-constexpr uint32_t kRecAqk = 32768;     // A_qk^T: token-row tile, row j, column i (8 KiB)
+constexpr uint32_t kRecW = 0;           // -W^T: 128 key-channel rows x 64 tokens (MN-major B of P; 16 KiB)
+constexpr uint32_t kRecQ = 16384;       // Q+: 64 token rows x 128 channels (K-major B of O^T = S0^T Q+^T; 16 KiB)
+constexpr uint32_t kRecAqk = 32768;     // A_qk: 64 rows i x 64 columns j (K-major B of O^T += V'^T A_qk^T; 8 KiB)
 constexpr uint32_t kRecKbar = 40960;    // Kbar: token-row tile 64 x 128 (16 KiB)
-// [A_qk^T | Kbar] = 24 KiB read as one MN-major B operand (N = 64 + 128, LBO 8 KiB).
 constexpr uint32_t kRecU = 57344;       // U^T: K-major, 128 rows (channel) x 64 (token) (16 KiB)
 constexpr uint32_t kRecGamma = 73728;   // gamma: 128 fp32
 constexpr uint32_t kRecBytes = 74240;
@@ -95,7 +95,7 @@ constexpr uint32_t kP1T = 49152;
 constexpr uint32_t kP1Bytes = 53248;
 constexpr uint32_t kP1V = kP1A + 8192;       // v tile (half stride 16 KiB), after the score MMA
 constexpr uint32_t kP1B2 = kP1B;             // (T diag beta)^T, K-major 64 x 64, after the solve
-constexpr uint32_t kP1QT = kP1A + 24576;     // A_qk^T staging (bulk-stored before v's second half lands)
+constexpr uint32_t kP1QT = kP1A + 24576;     // A_qk staging (bulk-stored before v's second half lands)
 constexpr int kP1Threads = 256;
 constexpr int kP1Blocks = 4;                 // CTAs per SM: 4 x 128 TMEM columns, 4 x ~55 KiB shared memory
 // Per-chunk safe range of the factored form: every channel's cumulative
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
         st8(sm + kP1A + oQ, w);               // Q+_r (in place of q)
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * egr[e]);
-        st8(rec + kRecWQ + oQ, w);            // Q+ image
+        st8(rec + kRecQ + oK, w);             // Q+ image (64 token rows, the layout of the k tile)
       }
       {
         float ei[8];
@@ -446,7 +446,13 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       } else {
         const int i = row - kC;
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) stbf(sm + kP1QT, kmajor_off(col0 + jj, i, kC), (col0 + jj) <= i ? v[jj] : 0.f);
+#pragma unroll
+        for (int p8 = 0; p8 < 4; ++p8) {  // row i of A_qk, 8 columns per 16-byte store
+          float w8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w8[e] = (col0 + 8 * p8 + e) <= i ? v[8 * p8 + e] : 0.f;
+          st_kmajor8(sm + kP1QT, i, col0 + 8 * p8, kC, w8);
+        }
       }
     }
   } else {
@@ -527,7 +533,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
         kb[e] = k8[e] * __expf(gend[e] - G[t][e]);
       }
       st8(sm + kP1A + kmajor_off(i, c8, 128), kp);
-      st8(rec + kRecWQ + oQ, qp);
+      st8(rec + kRecQ + oK, qp);
       st8(rec + kRecKbar + oK, kb);
     }
     __syncthreads();  // k and q are read: region B takes the A_kk blocks, [24K,32K) of region A the A_qk^T staging
@@ -546,12 +552,12 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
           fq = rsqrtf(snq[i] + kL2Eps) * rkj;
         }
         a_blk(sm, blk(i >> 4, j >> 4))[bidx(i & 15, j & 15)] = j < i ? sbeta[i] * (akk[t] * fk) : 0.f;
-        stbf(sm + kP1QT, kmajor_off(j, i, kC), scale * (aqk[t] * fq));
+        stbf(sm + kP1QT, kmajor_off(i, j, kC), scale * (aqk[t] * fq));
       }
     }
     for (int e = tid; e < kC * kC; e += kP1Threads) {
       const int i = e / kC, j = e % kC;
-      if (j > i) stbf(sm + kP1QT, kmajor_off(j, i, kC), 0.f);
+      if (j > i) stbf(sm + kP1QT, kmajor_off(i, j, kC), 0.f);
     }
   }
   fence_async_smem();
@@ -649,7 +655,8 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   wait_or_flag(&bar_mma, slow ? 0 : 1, hdr, 4);
   tc_fence_after();
 
-  // ---- -W (staged over K+_r: rows 0-63 of region A) and U^T (region B, 128-row K-major)
+  // ---- -W^T (channel rows over the first 16 KiB of region A, dead once the
+  // W/U products are done: row c, 64 tokens) and U^T (region B, 128-row K-major)
   {
     const int c = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -660,7 +667,12 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       if (warp < 4) {
         tmem_ld32(tm + lane_off + half * 32, v);
 #pragma unroll
-        for (int ii = 0; ii < 32; ++ii) stbf(sm + kP1A, kmajor_off(half * 32 + ii, c, 128), wsc * v[ii]);
+        for (int p8 = 0; p8 < 4; ++p8) {
+          float w8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w8[e] = wsc * v[8 * p8 + e];
+          st_kmajor8(sm + kP1A, c, half * 32 + 8 * p8, 128, w8);
+        }
       } else {
         tmem_ld32(tm + lane_off + 64 + half * 32, v);
 #pragma unroll
@@ -672,8 +684,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   tc_fence_before();
   __syncthreads();
   if (tid == 0) {
-    bulk_store(rec + kRecWQ, sm + kP1A, 8192);                 // -W rows, channels 0-63
-    bulk_store(rec + kRecWQ + 16384, sm + kP1A + 16384, 8192); // -W rows, channels 64-127
+    bulk_store(rec + kRecW, sm + kP1A, 16384);
     bulk_store(rec + kRecU, sm + kP1B, 16384);
     bulk_commit();
     bulk_wait_read();
@@ -737,8 +748,7 @@ __device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, 
     return;
   }
   mbar_expect_tx(bar, zero_u ? kRecTransBytes : kRecNoOutBytes);
-  bulk_load(stage + kRecWQ, rec + kRecWQ, 8192, bar);
-  bulk_load(stage + kRecWQ + 16384, rec + kRecWQ + 16384, 8192, bar);
+  bulk_load(stage + kRecW, rec + kRecW, kRecQ - kRecW, bar);
   if (zero_u) {
     bulk_load(stage + kRecKbar, rec + kRecKbar, kRecU - kRecKbar, bar);
     bulk_load(stage + kRecGamma, rec + kRecGamma, kRecBytes - kRecGamma, bar);
@@ -752,8 +762,7 @@ __device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, 
 // record, to [16K, 48.5K) (U skipped for the transition pass).
 __device__ __forceinline__ void load_record_compact(uint8_t* stage, const uint8_t* rec, uint64_t* bar, bool zero_u) {
   mbar_expect_tx(bar, zero_u ? kRecTransBytes : kRecNoOutBytes);
-  bulk_load(stage + kCW, rec + kRecWQ, 8192, bar);
-  bulk_load(stage + kCW + 8192, rec + kRecWQ + 16384, 8192, bar);
+  bulk_load(stage + kCW, rec + kRecW, kRecQ - kRecW, bar);
   if (zero_u) {
     bulk_load(stage + kCKbar, rec + kRecKbar, kRecU - kRecKbar, bar);
     bulk_load(stage + kCGamma, rec + kRecGamma, kRecBytes - kRecGamma, bar);
@@ -891,41 +900,44 @@ __global__ void __launch_bounds__(kOut ? kSPThreads : kSPThreadsNoOut, kOut ? 1 
     if ((tid & 31) == 0) {
       // P = S0^T (-W)^T (N=64) first, committed alone so that V' can be formed
       // at once; with outputs, O^T = S0^T Q+^T (N=64) is issued next, while
-      // the state warps form V', and [O|S] += V'^T [A_qk^T|Kbar] (N=192)
-      // closes the chunk; without outputs S += V'^T Kbar (N=128).
-      const uint32_t id_1 = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t id_2 = idesc_bf16_f32(128, out ? 192 : 128, 0, 1);
-      const uint32_t t2 = out ? tm + kTmO : tm + tS;
+      // the state warps form V'; then O^T += V'^T A_qk^T (N=64) and
+      // S^T += V'^T Kbar (N=128) close the chunk (without outputs only the last).
+      const uint32_t id_w = idesc_bf16_f32(128, 64, 0, 1);    // B = -W^T, MN-major (N = tokens)
+      const uint32_t id_k = idesc_bf16_f32(128, 64, 0, 0);    // B = Q+ or A_qk rows, K-major
+      const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 1);   // B = Kbar, MN-major (N = channels)
       // first descriptors of each stage; later steps add address offsets (in 16-byte units)
-      const uint32_t oW = kOut ? kRecWQ : kCW, oB = kOut ? (out ? kRecAqk : kRecKbar) : kCKbar;
-      constexpr uint32_t kWBlk = kOut ? 16384 : 8192;  // bytes between the 64-channel blocks of -W
-      const uint64_t d1s0 = desc_sw128(smem_u32(sm + oW), 16, 1024);
-      const uint64_t d1s1 = desc_sw128(smem_u32(sm + kStg + oW), 16, 1024);
-      const uint64_t d2s0 = desc_sw128(smem_u32(sm + oB), 8192, 1024);
-      const uint64_t d2s1 = desc_sw128(smem_u32(sm + kStg + oB), 8192, 1024);
-      constexpr uint64_t kQoff = 8192 >> 4;  // rows 64-127 (Q+) of each 64-column block of [-W; Q+]
+      const uint32_t oW = kOut ? kRecW : kCW, oK = kOut ? kRecKbar : kCKbar;
+      auto desc_at = [&](int s, uint32_t off, uint32_t lbo) { return desc_sw128(smem_u32(sm + s * kStg + off), lbo, 1024); };
+      const uint64_t dw0 = desc_at(0, oW, 8192), dw1 = desc_at(1, oW, 8192);
+      const uint64_t dk0 = desc_at(0, oK, 8192), dk1 = desc_at(1, oK, 8192);
+      const uint64_t dq0 = desc_at(0, kRecQ, 16), dq1 = desc_at(1, kRecQ, 16);      // with outputs only
+      const uint64_t da0 = desc_at(0, kRecAqk, 16), da1 = desc_at(1, kRecAqk, 16);  // with outputs only
       for (int n = 0; n < NCL; ++n) {
         const int s = n & 1;
+        const uint64_t dws = s ? dw1 : dw0, dks = s ? dk1 : dk0, dqs = s ? dq1 : dq0, das = s ? da1 : da0;
         wait_or_flag(&bar_as, n & 1, hdr, 30);
         wait_or_flag(&bar_full[s], (n >> 1) & 1, hdr, 31);
         tc_fence_after();
-        const uint64_t d1 = s ? d1s1 : d1s0, d2 = s ? d2s1 : d2s0;
 #pragma unroll
-        for (int k = 0; k < kD / 16; ++k)  // K-major B: +32 B per step inside a 64-wide block
-          mma_bf16_ts(tm + tP, tm + tAS + k * 8, d1 + (uint64_t)(((k / 4) * kWBlk + (k % 4) * 32) >> 4), id_1,
-                      k > 0);
+        for (int k = 0; k < kD / 16; ++k)  // MN-major B: 16 channel rows (2 KiB) per step
+          mma_bf16_ts(tm + tP, tm + tAS + k * 8, dws + (uint64_t)((k * 2048) >> 4), id_w, k > 0);
         mma_commit(&bar_p);
         if (out) {  // bar_as also covered the read of O^T of chunk n-1
 #pragma unroll
-          for (int k = 0; k < kD / 16; ++k)
-            mma_bf16_ts(tm + kTmO, tm + tAS + k * 8,
-                        d1 + kQoff + (uint64_t)(((k / 4) * 16384 + (k % 4) * 32) >> 4), id_1, k > 0);
+          for (int k = 0; k < kD / 16; ++k)  // K-major B (64 token rows): +32 B per step, +8 KiB per 64-channel block
+            mma_bf16_ts(tm + kTmO, tm + tAS + k * 8, dqs + (uint64_t)(((k / 4) * 8192 + (k % 4) * 32) >> 4), id_k,
+                        k > 0);
         }
         wait_or_flag(&bar_av, n & 1, hdr, 33);
         tc_fence_after();
+        if (out) {
+#pragma unroll
+          for (int k = 0; k < kC / 16; ++k)  // K-major B (rows i): 16 tokens j = 32 B per step
+            mma_bf16_ts(tm + kTmO, tm + tAV + k * 8, das + (uint64_t)((k * 32) >> 4), id_k, 1);
+        }
 #pragma unroll
         for (int k = 0; k < kC / 16; ++k)  // MN-major B: +2 KiB per 16 K-rows
-          mma_bf16_ts(t2, tm + tAV + k * 8, d2 + (uint64_t)((2 * k * 1024) >> 4), id_2, 1);
+          mma_bf16_ts(tm + tS, tm + tAV + k * 8, dks + (uint64_t)((2 * k * 1024) >> 4), id_s, 1);
         mma_commit(&bar_s);
         mma_commit(&bar_o);
       }
