@@ -328,6 +328,13 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     gref[e] = tot[0] + tot[1];                 // G at token 31
     gend[e] = ((tot[0] + tot[1]) + tot[2]) + tot[3];  // G at token 63 (= G_C; padding has g = 0)
   }
+  // G goes to tensor memory until the decayed operands are formed (held in
+  // registers across that stretch it would spill to local memory): thread
+  // (warp, lane) keeps its 32 values in its own lane (warp % 4) * 32 + lane,
+  // columns (warp / 4) * 32 + 8t + e.  The score MMA overwrites them later.
+  const uint32_t g_tm = tm + ((uint32_t)((warp & 3) * 32) << 16) + (warp >> 2) * 32;
+  tmem_st32(g_tm, &G[0][0]);
+  tmem_wait_st();
   bool unsafe = false;
 #pragma unroll
   for (int e = 0; e < 8; ++e) unsafe |= gend[e] < -kSafeSpan;
@@ -356,7 +363,8 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       const uint32_t oK = kmajor_off(i, c8, kC);        // 64-row tiles: k, K-_r, Kbar
       const uint32_t oA = kmajor_off(i, c8, 128);       // row i of region A
       const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A and of the [-W;Q+] image
-      float k8[8], q8[8];
+      float k8[8], q8[8], Gt[8];
+      tmem_ld8(g_tm + 8 * t, Gt);
       ld8(sm + kP1B + oK, k8);
       ld8(sm + kP1A + oQ, q8);
       if (l2n) {
@@ -374,7 +382,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
         float ex[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          ex[e] = __expf(G[t][e] - gref[e]);
+          ex[e] = __expf(Gt[e] - gref[e]);
           q8[e] *= scale;
         }
 #pragma unroll
@@ -390,7 +398,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       {
         float ei[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ei[e] = __expf(gref[e] - G[t][e]);
+        for (int e = 0; e < 8; ++e) ei[e] = __expf(gref[e] - Gt[e]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = k8[e] * ei[e];
         st8(sm + kP1B + oK, w);               // K-_r, in place of k
@@ -472,9 +480,12 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     for (int hf = 0; hf < 2; ++hf) {
       if ((c8 >> 6) == hf) {
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
+        for (int t = 0; t < 4; ++t) {
+          float Gt[8];
+          tmem_ld8(g_tm + 8 * t, Gt);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) *gp(tg + 16 * t, c8 - 64 * hf + e) = G[t][e];
+          for (int e = 0; e < 8; ++e) *gp(tg + 16 * t, c8 - 64 * hf + e) = Gt[e];
+        }
       }
       __syncthreads();
 #pragma unroll 1
@@ -514,7 +525,8 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       const int i = tg + 16 * t;
       const uint32_t oK = kmajor_off(i, c8, kC);
       const uint32_t oQ = kmajor_off(kC + i, c8, 128);
-      float k8[8], q8[8], kp[8], qp[8], kb[8];
+      float k8[8], q8[8], kp[8], qp[8], kb[8], Gt[8];
+      tmem_ld8(g_tm + 8 * t, Gt);
       ld8(sm + kP1B + oK, k8);
       ld8(sm + kP1A + oQ, q8);
       if (l2n) {
@@ -527,10 +539,10 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float e0 = __expf(G[t][e]);
+        const float e0 = __expf(Gt[e]);
         kp[e] = k8[e] * e0;
         qp[e] = scale * q8[e] * e0;
-        kb[e] = k8[e] * __expf(gend[e] - G[t][e]);
+        kb[e] = k8[e] * __expf(gend[e] - Gt[e]);
       }
       st8(sm + kP1A + kmajor_off(i, c8, 128), kp);
       st8(rec + kRecQ + oK, qp);
