@@ -245,10 +245,9 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     }
   }
   if (warp == 0) tmem_alloc(&tmem_base, 128);
-  if (tid < kC) {
-    const float x = tid < L ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
-    sbeta[tid] = (kPrep && tid < L) ? prep_beta(prep, x) : x;
-  }
+  // beta is a strided gather (one 2-byte value per token): read it now, park
+  // it in shared memory only after the gate scan, off the first barrier's path
+  const float beta_x = (tid < L) ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
   if (kScalarGate && tid >= kC && tid < 2 * kC) {
     const int i = tid - kC;
     const float x = (g_head && i < L) ? __bfloat162float(g_head[((size_t)b * T + t0 + i) * H + h]) : 0.f;
@@ -335,6 +334,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   const uint32_t g_tm = tm + ((uint32_t)((warp & 3) * 32) << 16) + (warp >> 2) * 32;
   tmem_st32(g_tm, &G[0][0]);
   tmem_wait_st();
+  if (tid < kC) sbeta[tid] = (kPrep && tid < L) ? prep_beta(prep, beta_x) : beta_x;
   bool unsafe = false;
 #pragma unroll
   for (int e = 0; e < 8; ++e) unsafe |= gend[e] < -kSafeSpan;
