@@ -424,11 +424,11 @@ struct PassRec {  // element offsets of the bf16 pass record of one chunk (all r
 // (c / 64) * 8192 + i * 128 + (((c % 64) / 8) ^ (i % 8)) * 16 + (c % 8) * 2.
 // Byte offsets inside the record (the record keeps PassRec's stride):
 struct TcRec {
-  static constexpr uint32_t oW = 0;         // W    [64 tokens][128 channels]
-  static constexpr uint32_t oQp = 16384;    // Q+   [64 tokens][128 channels]
-  static constexpr uint32_t oKb = 32768;    // Kbar [64 tokens][128 channels]
-  static constexpr uint32_t oAqk = 49152;   // Aqk  [64 query tokens i][64 key tokens j]
-  static constexpr uint32_t bytes = 57344;
+  static constexpr uint32_t oW = kTcRecW;      // W    [64 tokens][128 channels]
+  static constexpr uint32_t oQp = kTcRecQp;    // Q+   [64 tokens][128 channels]
+  static constexpr uint32_t oKb = kTcRecKb;    // Kbar [64 tokens][128 channels]
+  static constexpr uint32_t oAqk = kTcRecAqk;  // Aqk  [64 query tokens i][64 key tokens j]
+  static constexpr uint32_t bytes = kTcRecBytes;
 };
 static_assert(TcRec::bytes <= PassRec<128>::n * 2, "the tensor-core record fits the record stride");
 template <int DK, int DV>
@@ -2482,10 +2482,20 @@ cudaError_t launch_chunk_typed(const ChunkBwdArgs& a_in, int BH, int B, Workspac
   ChunkBwdArgs a = a_in;
   a.tc_rec = !std::is_same<IO, float>::value && kTcPass<DK, DV> && tc_pass_pays(BH);
   const dim3 grid((unsigned)a.NC * BH);  // chunk-major within each (sequence, head)
-  cudaError_t e =
-      std::is_same<IO, float>::value
-          ? launch_k(bwd_prep_kernel<float, DK, DV>, grid, prep_smem<DK, DV>(), a, stream, kThreads, false)
-          : launch_k(bwd_prep_bf16_kernel<DK, DV>, grid, PrepPlanB<DK, DV>::bytes, a, stream, kThreads, false);
+  cudaError_t e;
+  if (std::is_same<IO, float>::value) {
+    e = launch_k(bwd_prep_kernel<float, DK, DV>, grid, prep_smem<DK, DV>(), a, stream, kThreads, false);
+  } else if (a.tc_rec) {
+    // the forward's preparation kernel (tcgen05, four tiles per SM) in its
+    // backward mode writes the same operands in the same layouts
+    const PrepBwdOut out{reinterpret_cast<uint8_t*>(a.prec), (size_t)PassRec<DK>::n * 2, a.Pkk,
+                         reinterpret_cast<bf16*>(a.Tm), a.U, a.gam, a.bh0, BH};
+    e = launch_prep_for_backward(static_cast<const bf16*>(a.q), static_cast<const bf16*>(a.k),
+                                 static_cast<const bf16*>(a.v), static_cast<const bf16*>(a.g),
+                                 static_cast<const bf16*>(a.beta), a.scale, B, a.T, a.H, a.gate, out, hdr, stream);
+  } else {
+    e = launch_k(bwd_prep_bf16_kernel<DK, DV>, grid, PrepPlanB<DK, DV>::bytes, a, stream, kThreads, false);
+  }
   if (e != cudaSuccess) return e;
   const bool w32 = pass_width(BH, DV) == 32;
   if constexpr (std::is_same<IO, float>::value) {

@@ -43,6 +43,30 @@ cudaError_t launch_prefill_bf16(const __nv_bfloat16* q, const __nv_bfloat16* k, 
                                 int dk, int dv, int chunk, int gate, int prep, void* ws, size_t ws_bytes,
                                 cudaStream_t stream, void* const* events);
 
+// The backward's tensor-core pass record (d_k = d_v = 128): 128-byte-swizzled
+// token-row tiles, element (token i, channel c) of a [64][128] tile at byte
+// (c / 64) * 8192 + i * 128 + (((c % 64) / 8) ^ (i % 8)) * 16 + (c % 8) * 2
+// (A_qk: [64 query tokens][64 key tokens], one 8 KiB half).
+constexpr uint32_t kTcRecW = 0, kTcRecQp = 16384, kTcRecKb = 32768, kTcRecAqk = 49152, kTcRecBytes = 57344;
+
+// The per-chunk operands of the backward (bf16, d_k = d_v = 128, tensor-core
+// state passes), written by the prefill's preparation kernel in its backward
+// mode: record = (sequence, head) index within the launch group * NC + chunk.
+struct PrepBwdOut {
+  uint8_t* rec;       // pass records: W, Q+, Kbar, A_qk at the kTcRec* offsets
+  size_t rec_stride;  // bytes between consecutive records
+  float* P;           // [rec][64][64] strict_tril(K+ K-^T), fp32
+  __nv_bfloat16* T;   // [rec][64][64] (I + diag(beta) P)^-1, bf16, row-major
+  float* U;           // [rec][64][128] T diag(beta) V, fp32
+  float* gam;         // [rec][128] exp(G_C)
+  int bh0;            // (sequence, head) of the launch's first record
+  int nbh;            // (sequence, head) pairs in the launch
+};
+cudaError_t launch_prep_for_backward(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                                     const __nv_bfloat16* g, const __nv_bfloat16* beta, float scale, int B, int T,
+                                     int H, int gate, const PrepBwdOut& out, struct WorkspaceHeader* hdr,
+                                     cudaStream_t stream);
+
 // Backward pass (kda_backward_chunk.cu).  The workspace holds a
 // WorkspaceHeader (error word of the bounded waits; at the start of `ws`
 // unless `hdr` points elsewhere) and the records of one or more (sequence,

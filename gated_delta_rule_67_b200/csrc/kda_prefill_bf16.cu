@@ -206,13 +206,17 @@ __device__ __forceinline__ void store_block_frag(float* X, const float (&acc)[2]
 // the per-channel g tile comes in by TMA (KDA).  kPrep: the inputs are raw
 // and `prep` (kda_prep bits) says which ones to prepare here: q, k scaled to
 // unit length per token (the per-token factors are applied wherever q and k
-// are read), log-sigmoid of g, sigmoid of beta.
-template <bool kScalarGate, bool kPrep>
+// are read), log-sigmoid of g, sigmoid of beta.  kBwd: the operands go to the
+// backward instead (`bo`: W, Q+, Kbar, A_qk as token-row tiles, P and U in
+// fp32, T in bf16, gamma) for the (sequence, head) pairs bo.bh0 onwards; the
+// forward record is not written.
+template <bool kScalarGate, bool kPrep, bool kBwd = false>
 __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                           const bf16* __restrict__ beta, float scale, uint8_t* __restrict__ records,
-                          WorkspaceHeader* hdr, int T, int H, int NC, const bf16* __restrict__ g_head, int prep) {
+                          WorkspaceHeader* hdr, int T, int H, int NC, const bf16* __restrict__ g_head, int prep,
+                          const PrepBwdOut bo) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ uint64_t bar_in, bar_v, bar_mma;
@@ -225,11 +229,15 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x % NC;
-  const int bh = blockIdx.x / NC;
+  const int bh = (kBwd ? bo.bh0 : 0) + (int)(blockIdx.x / NC);
   const int h = bh % H, b = bh / H;
   const int t0 = chunk * kC;
   const int L = min(kC, T - t0);
-  uint8_t* rec = records + (size_t)blockIdx.x * kRecBytes;
+  // the record of this chunk and the offsets of its images in it
+  const size_t ri = blockIdx.x;  // backward: the index of its per-chunk arrays too
+  uint8_t* rec = kBwd ? bo.rec + ri * bo.rec_stride : records + ri * kRecBytes;
+  constexpr uint32_t oRecQ = kBwd ? kTcRecQp : kRecQ, oRecKbar = kBwd ? kTcRecKb : kRecKbar;
+  constexpr uint32_t oRecAqk = kBwd ? kTcRecAqk : kRecAqk;
 
   if (tid == 0) {
     mbar_init(&bar_in, 1);
@@ -339,7 +347,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
 #pragma unroll
   for (int e = 0; e < 8; ++e) unsafe |= gend[e] < -kSafeSpan;
   if (tg == 0) {
-    float* gam = reinterpret_cast<float*>(rec + kRecGamma) + c8;
+    float* gam = (kBwd ? bo.gam + ri * kD : reinterpret_cast<float*>(rec + kRecGamma)) + c8;
     *reinterpret_cast<float4*>(gam) = make_float4(expf(gend[0]), expf(gend[1]), expf(gend[2]), expf(gend[3]));
     *reinterpret_cast<float4*>(gam + 4) = make_float4(expf(gend[4]), expf(gend[5]), expf(gend[6]), expf(gend[7]));
   }
@@ -393,7 +401,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
         st8(sm + kP1A + oQ, w);               // Q+_r (in place of q)
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * egr[e]);
-        st8(rec + kRecQ + oK, w);             // Q+ image (64 token rows, the layout of the k tile)
+        st8(rec + oRecQ + oK, w);             // Q+ image (64 token rows, the layout of the k tile)
       }
       {
         float ei[8];
@@ -404,7 +412,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
         st8(sm + kP1B + oK, w);               // K-_r, in place of k
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ei[e] * egb[e]);
-        st8(rec + kRecKbar + oK, w);          // Kbar image = k exp(G_C - G_i)
+        st8(rec + oRecKbar + oK, w);          // Kbar image = k exp(G_C - G_i)
       }
     }
     fence_async_smem();
@@ -434,6 +442,16 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       if (row < kC) {
         const int i = row, I = i >> 4;
         const float bi = sbeta[i];
+        if (kBwd) {  // P row i, columns col0 .. col0 + 31 (zero on and above the diagonal)
+          float4* Pr = reinterpret_cast<float4*>(bo.P + ri * (kC * kC) + i * kC + col0);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            float w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w[e] = (col0 + 4 * q4 + e) < i ? v[4 * q4 + e] : 0.f;
+            Pr[q4] = make_float4(w[0], w[1], w[2], w[3]);
+          }
+        }
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           const int J = (col0 >> 4) + half;
@@ -453,7 +471,6 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
         }
       } else {
         const int i = row - kC;
-#pragma unroll
 #pragma unroll
         for (int p8 = 0; p8 < 4; ++p8) {  // row i of A_qk, 8 columns per 16-byte store
           float w8[8];
@@ -545,8 +562,8 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
         kb[e] = k8[e] * __expf(gend[e] - Gt[e]);
       }
       st8(sm + kP1A + kmajor_off(i, c8, 128), kp);
-      st8(rec + kRecQ + oK, qp);
-      st8(rec + kRecKbar + oK, kb);
+      st8(rec + oRecQ + oK, qp);
+      st8(rec + oRecKbar + oK, kb);
     }
     __syncthreads();  // k and q are read: region B takes the A_kk blocks, [24K,32K) of region A the A_qk^T staging
 #pragma unroll 1
@@ -564,12 +581,16 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
           fq = rsqrtf(snq[i] + kL2Eps) * rkj;
         }
         a_blk(sm, blk(i >> 4, j >> 4))[bidx(i & 15, j & 15)] = j < i ? sbeta[i] * (akk[t] * fk) : 0.f;
+        if (kBwd) bo.P[ri * (kC * kC) + i * kC + j] = j < i ? akk[t] * fk : 0.f;
         stbf(sm + kP1QT, kmajor_off(i, j, kC), scale * (aqk[t] * fq));
       }
     }
     for (int e = tid; e < kC * kC; e += kP1Threads) {
       const int i = e / kC, j = e % kC;
-      if (j > i) stbf(sm + kP1QT, kmajor_off(i, j, kC), 0.f);
+      if (j > i) {
+        stbf(sm + kP1QT, kmajor_off(i, j, kC), 0.f);
+        if (kBwd) bo.P[ri * (kC * kC) + e] = 0.f;
+      }
     }
   }
   fence_async_smem();
@@ -577,7 +598,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   __syncthreads();
   tc_fence_after();
   if (tid == 0) {
-    bulk_store(rec + kRecAqk, sm + kP1QT, 8192);
+    bulk_store(rec + oRecAqk, sm + kP1QT, 8192);
     bulk_commit();
     // Q+_r is dead: bring v while the triangle is inverted, its first
     // channel half now, the second once the A_qk^T store has read its bytes
@@ -633,11 +654,24 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     float vals[16];
     if (J <= I) {
       const float* Tb = t_blk(sm, blk(I, J));
+      if (kBwd) {  // T itself, row i, columns j0 .. j0 + 15, bf16
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) vals[jj] = (j0 + jj) <= i ? Tb[bidx(i & 15, jj)] : 0.f;
+        uint4* Tr = reinterpret_cast<uint4*>(bo.T + ri * (kC * kC) + i * kC + j0);
+        Tr[0] = make_uint4(pack2(vals[0], vals[1]), pack2(vals[2], vals[3]), pack2(vals[4], vals[5]),
+                           pack2(vals[6], vals[7]));
+        Tr[1] = make_uint4(pack2(vals[8], vals[9]), pack2(vals[10], vals[11]), pack2(vals[12], vals[13]),
+                           pack2(vals[14], vals[15]));
+      }
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) vals[jj] = (j0 + jj) <= i ? Tb[bidx(i & 15, jj)] * sbeta[j0 + jj] : 0.f;
     } else {
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) vals[jj] = 0.f;
+      if (kBwd) {
+        uint4* Tr = reinterpret_cast<uint4*>(bo.T + ri * (kC * kC) + i * kC + j0);
+        Tr[0] = Tr[1] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
     st_kmajor8(sm + kP1B2, i, j0, kC, vals);
     st_kmajor8(sm + kP1B2, i, j0 + 8, kC, vals + 8);
@@ -672,23 +706,34 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   {
     const int c = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const float wsc = warp < 4 ? -segr[c] : 0.f;
+    const float wsc = warp < 4 ? (kBwd ? segr[c] : -segr[c]) : 0.f;
     float v[32];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       if (warp < 4) {
         tmem_ld32(tm + lane_off + half * 32, v);
+        if (kBwd) {  // W as token rows: element (token, channel c) of the 64 x 128 tile
 #pragma unroll
-        for (int p8 = 0; p8 < 4; ++p8) {
-          float w8[8];
+          for (int e = 0; e < 32; ++e) stbf(sm + kP1A, kmajor_off(half * 32 + e, c, kC), wsc * v[e]);
+        } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) w8[e] = wsc * v[8 * p8 + e];
-          st_kmajor8(sm + kP1A, c, half * 32 + 8 * p8, 128, w8);
+          for (int p8 = 0; p8 < 4; ++p8) {
+            float w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w8[e] = wsc * v[8 * p8 + e];
+            st_kmajor8(sm + kP1A, c, half * 32 + 8 * p8, 128, w8);
+          }
         }
       } else {
         tmem_ld32(tm + lane_off + 64 + half * 32, v);
+        if (kBwd) {  // U[token][c], fp32: a warp writes 32 consecutive channels of a token row
+          float* Ur = bo.U + ri * (kC * kD) + (size_t)(half * 32) * kD + c;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) st_kmajor8(sm + kP1B, c, half * 32 + 8 * e, 128, v + 8 * e);
+          for (int e = 0; e < 32; ++e) Ur[e * kD] = v[e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) st_kmajor8(sm + kP1B, c, half * 32 + 8 * e, 128, v + 8 * e);
+        }
       }
     }
   }
@@ -696,8 +741,12 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   tc_fence_before();
   __syncthreads();
   if (tid == 0) {
-    bulk_store(rec + kRecW, sm + kP1A, 16384);
-    bulk_store(rec + kRecU, sm + kP1B, 16384);
+    if (kBwd) {
+      bulk_store(rec + kTcRecW, sm + kP1A, 16384);
+    } else {
+      bulk_store(rec + kRecW, sm + kP1A, 16384);
+      bulk_store(rec + kRecU, sm + kP1B, 16384);
+    }
     bulk_commit();
     bulk_wait_read();
   }
@@ -1404,6 +1453,42 @@ size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chu
   return sizeof(WorkspaceHeader) + (size_t)B * H * NC * kRecBytes + scan;
 }
 
+// The preparation kernel in its backward mode (bf16, d_k = d_v = 128): the
+// per-chunk operands of the backward's tensor-core state passes and local
+// kernels for the (sequence, head) pairs out.bh0 .. out.bh0 + out.nbh - 1.
+cudaError_t launch_prep_for_backward(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const bf16* beta,
+                                     float scale, int B, int T, int H, int gate, const PrepBwdOut& out,
+                                     WorkspaceHeader* hdr, cudaStream_t stream) {
+  static std::atomic<unsigned long long> attrs_done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long dev_bit = dev < 64 ? 1ull << dev : 0ull;
+  if (!(attrs_done.load(std::memory_order_acquire) & dev_bit) || !dev_bit) {
+    for (auto kern : {kda_chunk_prep_kernel<false, false, true>, kda_chunk_prep_kernel<true, false, true>}) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kP1Bytes + 1024);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return e;
+    }
+    attrs_done.fetch_or(dev_bit, std::memory_order_release);
+  }
+  CUtensorMap mq, mk, mv, mg;
+  memset(&mg, 0, sizeof(mg));
+  if (!make_map(&mq, q, B, T, H, kD) || !make_map(&mk, k, B, T, H, kD) || !make_map(&mv, v, B, T, H, kD) ||
+      (gate == KDA_GATE_CHANNEL && !make_map(&mg, g, B, T, H, kD)))
+    return cudaErrorInvalidValue;
+  const int NC = (T + kC - 1) / kC;
+  const unsigned tiles = (unsigned)((size_t)out.nbh * NC);
+  if (gate == KDA_GATE_CHANNEL)
+    kda_chunk_prep_kernel<false, false, true><<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(
+        mq, mk, mv, mg, beta, scale, nullptr, hdr, T, H, NC, nullptr, 0, out);
+  else
+    kda_chunk_prep_kernel<true, false, true><<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(
+        mq, mk, mv, mg, beta, scale, nullptr, hdr, T, H, NC, gate == KDA_GATE_HEAD ? g : nullptr, 0, out);
+  return cudaGetLastError();
+}
+
 int prefill_bf16_launches(int B, int T, int H) {
   const int NC = (int)(((size_t)T + kC - 1) / kC);
   int G, L;
@@ -1463,7 +1548,8 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     const bf16* gh = gate == KDA_GATE_HEAD ? g : nullptr;
     auto kern = scalar ? (prep ? kda_chunk_prep_kernel<true, true> : kda_chunk_prep_kernel<true, false>)
                        : (prep ? kda_chunk_prep_kernel<false, true> : kda_chunk_prep_kernel<false, false>);
-    kern<<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records, hdr, T, H, NC, gh, prep);
+    kern<<<tiles, kP1Threads, kP1Bytes + 1024, stream>>>(mq, mk, mv, mg, beta, scale, records, hdr, T, H, NC, gh, prep,
+                                                         PrepBwdOut{});
   }
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
