@@ -2471,11 +2471,13 @@ cudaError_t launch_pass_tc(const ChunkBwdArgs& a, int BH, int B, WorkspaceHeader
 
 // The tensor-core passes run one CTA per (sequence, head) and role, with all
 // 128 value channels in one tensor-memory accumulator; the warp-level passes
-// split the value channels over 4 CTAs.  With fewer than a wave of
-// tensor-core pass CTAs the split keeps more SMs busy and is faster
-// (measured: 492 vs 517 us per call at B1 H16 T4096; 13.4 vs 12.2 ms at
-// B8 H32 T8192 in favour of the tensor cores), so they take over from 148 CTAs on.
-bool tc_pass_pays(int BH) { return 2 * BH >= 148; }
+// split the value channels over 4 CTAs, which keeps more SMs busy when the
+// chains are few.  The tensor-core path also takes its operands from the
+// forward's preparation kernel (four tiles per SM) instead of the one-tile-
+// per-SM preparation of the warp-level path.  Measured per call: 466 vs 493
+// us at B1 H16 T4096 and 10.1 vs 12.2 ms at B8 H32 T8192 in favour of the
+// tensor-core path; it is taken from 16 (sequence, head) chains on.
+bool tc_pass_pays(int BH) { return BH >= 16; }
 
 template <typename IO, int DK, int DV>
 cudaError_t launch_chunk_typed(const ChunkBwdArgs& a_in, int BH, int B, WorkspaceHeader* hdr, cudaStream_t stream) {

@@ -130,6 +130,24 @@ def test_backward_small_workspace_groups(fit):
         assert torch.equal(full[n], part[n]), n
 
 
+def test_backward_tensor_core_workspace_groups():
+    """40 (sequence, head) pairs through a workspace for 20: two groups, each
+    on the tensor-core path, whose preparation starts the second group at pair
+    20 of the inputs; bit-identical to the one-group call."""
+    dev = cuda_or_skip()
+    from gated_delta_rule_67_b200.binding import load
+    B, T, H = 2, 130, 20
+    x = make_prefill_inputs(B, T, H, 128, 128, torch.bfloat16, 0.1, seed=102, device=dev)
+    d_o, d_s = make_cotangents(B, T, H, 128, 128, torch.bfloat16, seed=103, device=dev)
+    args = (x["q"], x["k"], x["v"], x["g"], x["beta"], d_o, None, x["initial_state"], d_s)
+    one = int(load().kda_backward_workspace_size(1, T, 1, 128, 128, 1))
+    full = kda_backward(*args)
+    part = kda_backward(*args, workspace=torch.empty(20 * one + 8, dtype=torch.uint8, device=dev))
+    torch.cuda.synchronize()
+    for n in full:
+        assert torch.equal(full[n], part[n]), n
+
+
 @pytest.mark.parametrize("gate", ["channel", "head"])
 def test_backward_matches_gpu_forward_directional_derivative(gate):
     """Independent of the oracle: for L = <dO, o> + <dS_T, S_T> computed from
