@@ -1810,16 +1810,14 @@ __global__ void __launch_bounds__(kLaThreads, 2) bwd_local_a_bf16_kernel(const C
     float acc[Th::MT][Th::NT][4];
     zero(acc);
     warp_mma_bf16<Th::MT, Th::NT, DV, false, true>(acc, sO, LVb, sS0, LVb, hm0, hn0);
-    float* out = a.dQs + rec * kC * DK + half * HR;
-    for_acc<Th::MT, Th::NT>(hm0, hn0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
+    acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dQs) + rec * kC * DK + half * HR, DK, hm0, hn0);  // bf16 for the fold
     zero(acc);
     warp_mma_bf16<Th::MT, Th::NT, DV, false, true>(acc, sdV, LVb, sS0, LVb, hm0, hn0);
     for_acc<Th::MT, Th::NT>(hm0, hn0, [&](int mt, int nt, int e, int i, int c) { acc[mt][nt][e] = -acc[mt][nt][e]; });
     acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dW) + rec * kC * DK + half * HR, DK, hm0, hn0);  // operand only
     zero(acc);
     warp_mma_bf16<Th::MT, Th::NT, DV, false, true>(acc, sVp, LVb, sdS, LVb, hm0, hn0);
-    out = a.dKb + rec * kC * DK + half * HR;
-    for_acc<Th::MT, Th::NT>(hm0, hn0, [&](int mt, int nt, int e, int i, int c) { out[i * DK + c] = acc[mt][nt][e]; });
+    acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dKb) + rec * kC * DK + half * HR, DK, hm0, hn0);  // bf16 for the fold
     for (int r = warp; r < HR; r += NW) {  // rowsum(dS . S0), two columns per load
       float x = 0.f;
       for (int c = 2 * lane; c < DV; c += 64) {
@@ -2094,7 +2092,7 @@ struct LocalBPlanB {  // bytes
   static constexpr size_t oG = 0, ok = oG + (size_t)kC * LK * 4, oq = ok + tk, oA = oq + tk, oB = oA + tk,
                           oC = oB + tk, oT = oC + tk, oDT = oT + tc, oY = oDT + tc, oQA = oY + tc, ob = oQA + tc,
                           ored = ob + kC * 4, ocol = ored + 8 * kC * 4, oQs = ocol + 4 * DK * 4,
-                          oKs = oQs + (size_t)kC * DK * 4, bytes = oKs + (size_t)kC * DK * 4;
+                          oKs = oQs + tk, bytes = oKs + tk;
   static_assert(tk % 16 == 0 && tc % 16 == 0 && ok % 16 == 0, "16 B");
   static_assert(2 * tk >= (size_t)kC * LK * 4, "dG (fp32) fits over the k and q tiles");
 };
@@ -2126,8 +2124,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   float* red = reinterpret_cast<float*>(smb + PL::ored);  // [8][64] row sums per column group
   float* colC = reinterpret_cast<float*>(smb + PL::ocol);  // [4][DK] column sums of dKbar . Kbar
   float* sdG = reinterpret_cast<float*>(smb + PL::ok);  // [64][LK] dG (fp32), over the k and q tiles at the end
-  float* sQs = reinterpret_cast<float*>(smb + PL::oQs);  // [64][DK] dO S0^T (fp32, from the d_v kernel)
-  float* sKs = reinterpret_cast<float*>(smb + PL::oKs);  // [64][DK] dKbar (fp32, from the d_v kernel)
+  bf16* sQs = reinterpret_cast<bf16*>(smb + PL::oQs);  // [64][LKb] dO S0^T (bf16, from the d_v kernel)
+  bf16* sKs = reinterpret_cast<bf16*>(smb + PL::oKs);  // [64][LKb] dKbar (bf16, from the d_v kernel)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
@@ -2170,12 +2168,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     }
   }
   cp_commit();  // group 1: everything the products need
-  {  // group 2: the fold's fp32 inputs, in flight while the products run
-    const float* qs = a.dQs + rec * kC * DK;
-    const float* ks = a.dKb + rec * kC * DK;
-    for (int idx = tid; idx < kC * DK / 4; idx += kThreads) {
-      cp16(sQs + 4 * idx, qs + 4 * idx, 16);
-      cp16(sKs + 4 * idx, ks + 4 * idx, 16);
+  {  // group 2: the fold's inputs, in flight while the products run (rows padded against bank conflicts)
+    const bf16* qs = reinterpret_cast<const bf16*>(a.dQs) + rec * kC * DK;
+    const bf16* ks = reinterpret_cast<const bf16*>(a.dKb) + rec * kC * DK;
+    for (int idx = tid; idx < kC * (DK / 8); idx += kThreads) {
+      const int i = idx / (DK / 8), c = (idx % (DK / 8)) * 8;
+      cp16(sQs + i * LKb + c, qs + (size_t)i * DK + c, 16);
+      cp16(sKs + i * LKb + c, ks + (size_t)i * DK + c, 16);
     }
   }
   cp_commit();
@@ -2242,8 +2241,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   }
   cp_wait_group<0>();  // the fold's inputs
   __syncthreads();
-  const float* dQs = sQs;
-  const float* dKb = sKs;
+  auto dqs_at = [&](int i, int r) { return __bfloat162float(sQs[i * LKb + r]); };
+  auto dkb_at = [&](int i, int r) { return __bfloat162float(sKs[i * LKb + r]); };
   float cp[TK::MT][TK::NT][2] = {};  // column partial sums of dKbar . Kbar (for dG_C)
   bf16* dq = static_cast<bf16*>(a.dq);
   if (!slow) {
@@ -2259,7 +2258,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     warp_mma_bf16<TK::MT, TK::NT, kC, false, false>(ap, sDT, LCb, sA, LKb, m0, n0);
     for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
       const float G = sG[i * LK + r], d = G - sG[kRef * LK + r];
-      const float ex = __expf(d), ei = __expf(-d), gm = __expf(G), dqs = dQs[i * DK + r];
+      const float ex = __expf(d), ei = __expf(-d), gm = __expf(G), dqs = dqs_at(i, r);
       const float kbf = __expf(sG[(kC - 1) * LK + r] - G);  // Kbar = k kbf
       const float kk = __bfloat162float(sk[i * LKb + r]);
       const float qs = a.scale * __bfloat162float(sq[i * LKb + r]);  // Q+_r = qs ex, Q+ = qs Gamma
@@ -2269,7 +2268,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
         const size_t o = (row0 + (size_t)i * a.H) * DK + r;
         if (a.dq32) a.dq32[o] = v; else dq[o] = __float2bfloat16_rn(v);
       }
-      const float xb = dKb[i * DK + r], yb = xb * kk * kbf;  // the Kbar terms
+      const float xb = dkb_at(i, r), yb = xb * kk * kbf;  // the Kbar terms
       dk_acc[mt][nt][e] = fmaf(kbf, xb, fmaf(ei, xm, fmaf(ex, xp, dk_acc[mt][nt][e])));
       dG_acc[mt][nt][e] += fmaf(qs, fmaf(xq, ex, dqs * gm), kk * fmaf(xp, ex, -xm * ei)) - yb;
       cp[mt][nt][e & 1] += yb;
@@ -2295,7 +2294,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
         dkp += w;
         dgp = fmaf(-w, ki, dgp);
       }
-      const float dqs = dQs[i * DK + r], gm = __expf(Gi);
+      const float dqs = dqs_at(i, r), gm = __expf(Gi);
       if (i < nv) {
         const float v = a.scale * fmaf(gm, dqs, dqp);
         const size_t o = (row0 + (size_t)i * a.H) * DK + r;
@@ -2309,7 +2308,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     if (slow)  // (the fast path folded these into its epilogue)
       for_acc<TK::MT, TK::NT>(m0, n0, [&](int mt, int nt, int e, int i, int r) {
         const float kbf = __expf(sG[(kC - 1) * LK + r] - sG[i * LK + r]);  // Kbar = k kbf
-        const float x = dKb[i * DK + r], y = x * __bfloat162float(sk[i * LKb + r]) * kbf;
+        const float x = dkb_at(i, r), y = x * __bfloat162float(sk[i * LKb + r]) * kbf;
         dk_acc[mt][nt][e] = fmaf(kbf, x, dk_acc[mt][nt][e]);
         dG_acc[mt][nt][e] -= y;
         cp[mt][nt][e & 1] += y;
@@ -2388,10 +2387,10 @@ struct WsPlan {
       : W(f32 ? (size_t)kC * dk : 0), U((size_t)kC * dv), Qp(f32 ? (size_t)kC * dk : 0), Kb(f32 ? (size_t)kC * dk : 0),
         Wt(f32 ? (size_t)kC * dk : 0), Qpt(f32 ? (size_t)kC * dk : 0), Kbt(f32 ? (size_t)kC * dk : 0),
         Aqk(f32 ? kC * kC : 0), prec(f32 ? 0 : (dk == 128 ? PassRec<128>::n : PassRec<64>::n) / 2),
-        // bf16 inputs: T, S0, dS, V', dV', dAqk, dW are kept as bf16 (half the floats)
+        // bf16 inputs: T, S0, dS, V', dV', dAqk, dW, dO S0^T and dKbar are kept as bf16 (half the floats)
         Tm(kC * kC / (f32 ? 1 : 2)), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv / (f32 ? 1 : 2)), dSc((size_t)dk * dv / (f32 ? 1 : 2)),
-        Vp((size_t)kC * dv / (f32 ? 1 : 2)), dVp((size_t)kC * dv / (f32 ? 1 : 2)), dAqk(kC * kC / (f32 ? 1 : 2)), dT1(kC * kC), dQs((size_t)kC * dk), dW((size_t)kC * dk / (f32 ? 1 : 2)),
-        dKb((size_t)kC * dk), dgam(dk), dbu(kC) {}
+        Vp((size_t)kC * dv / (f32 ? 1 : 2)), dVp((size_t)kC * dv / (f32 ? 1 : 2)), dAqk(kC * kC / (f32 ? 1 : 2)), dT1(kC * kC), dQs((size_t)kC * dk / (f32 ? 1 : 2)), dW((size_t)kC * dk / (f32 ? 1 : 2)),
+        dKb((size_t)kC * dk / (f32 ? 1 : 2)), dgam(dk), dbu(kC) {}
   size_t per_rec() const {
     return W + U + Qp + Kb + Wt + Qpt + Kbt + Aqk + prec + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs +
            dW + dKb + dgam + dbu;
