@@ -1776,12 +1776,12 @@ __global__ void __launch_bounds__(kLaThreads, 2) bwd_local_a_bf16_kernel(const C
       if (j > i) acc[mt][nt][e] = 0.f;
     });
     acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dAqk) + rec * kC * kC, kC, m0, n0);  // an operand only: bf16
-    zero(acc);  // dU (beta V)^T, strictly lower part
+    zero(acc);  // dU (beta V)^T, strictly lower part (bf16: the sum it enters is rounded to bf16 at once)
     warp_mma_bf16<Tl::MT, Tl::NT, DV, false, true>(acc, sdV, LVb, sv, LVb, m0, n0);
-    float* out = a.dT1 + rec * kC * kC;
     for_acc<Tl::MT, Tl::NT>(m0, n0, [&](int mt, int nt, int e, int i, int j) {
-      out[i * kC + j] = j < i ? acc[mt][nt][e] * sb[j] : 0.f;
+      acc[mt][nt][e] = j < i ? acc[mt][nt][e] * sb[j] : 0.f;
     });
+    acc_to_bf16(acc, reinterpret_cast<bf16*>(a.dT1) + rec * kC * kC, kC, m0, n0);
   }
   {  // X = T^T dU: dv = beta X, dbeta part = rowsum(V . X)
     using Tl = Tiling<kC, DV, NW>;
@@ -2092,7 +2092,7 @@ struct LocalBPlanB {  // bytes
   static constexpr size_t oG = 0, ok = oG + (size_t)kC * LK * 4, oq = ok + tk, oA = oq + tk, oB = oA + tk,
                           oC = oB + tk, oT = oC + tk, oDT = oT + tc, oY = oDT + tc, oQA = oY + tc, ob = oQA + tc,
                           ored = ob + kC * 4, ocol = ored + 8 * kC * 4, oQs = ocol + 4 * DK * 4,
-                          oKs = oQs + tk, bytes = oKs + tk;
+                          oKs = oQs + tk, oD1 = oKs + tk, oPk = oD1 + tc, bytes = oPk + (size_t)kC * kLC * 4;
   static_assert(tk % 16 == 0 && tc % 16 == 0 && ok % 16 == 0, "16 B");
   static_assert(2 * tk >= (size_t)kC * LK * 4, "dG (fp32) fits over the k and q tiles");
 };
@@ -2126,6 +2126,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   float* sdG = reinterpret_cast<float*>(smb + PL::ok);  // [64][LK] dG (fp32), over the k and q tiles at the end
   bf16* sQs = reinterpret_cast<bf16*>(smb + PL::oQs);  // [64][LKb] dO S0^T (bf16, from the d_v kernel)
   bf16* sKs = reinterpret_cast<bf16*>(smb + PL::oKs);  // [64][LKb] dKbar (bf16, from the d_v kernel)
+  bf16* sD1 = reinterpret_cast<bf16*>(smb + PL::oD1);  // [64][LCb] dU (beta V)^T (bf16, from the d_v kernel)
+  float* sPk = reinterpret_cast<float*>(smb + PL::oPk);  // [64][kLC] P (fp32, from the preparation)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x % a.NC, lb = blockIdx.x / a.NC, bh = a.bh0 + lb, t0 = n * kC, nv = min(kC, a.T - t0);
   const size_t row0 = row_of(a, bh, t0), rec = (size_t)lb * a.NC + n;
@@ -2162,12 +2164,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
   }
   {
     const bf16* Tg = reinterpret_cast<const bf16*>(a.Tm) + rec * kC * kC;
+    const bf16* D1g = reinterpret_cast<const bf16*>(a.dT1) + rec * kC * kC;
     for (int idx = tid; idx < kC * (kC / 8); idx += kThreads) {
       const int i = idx / (kC / 8), c = (idx % (kC / 8)) * 8;
       cp16(sT + i * LCb + c, Tg + (size_t)i * kC + c, 16);
+      cp16(sD1 + i * LCb + c, D1g + (size_t)i * kC + c, 16);
+    }
+    const float* Pg = a.Pkk + rec * kC * kC;
+    for (int idx = tid; idx < kC * (kC / 4); idx += kThreads) {
+      const int i = idx / (kC / 4), c = (idx % (kC / 4)) * 4;
+      cp16(sPk + i * kLC + c, Pg + (size_t)i * kC + c, 16);
     }
   }
-  cp_commit();  // group 1: everything the products need
+  cp_commit();  // group 1: everything the products and their epilogues need
   {  // group 2: the fold's inputs, in flight while the products run (rows padded against bank conflicts)
     const bf16* qs = reinterpret_cast<const bf16*>(a.dQs) + rec * kC * DK;
     const bf16* ks = reinterpret_cast<const bf16*>(a.dKb) + rec * kC * DK;
@@ -2189,9 +2198,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     float acc[TC::MT][TC::NT][4];
     zero(acc);
     warp_mma_bf16<TC::MT, TC::NT, DK, false, true>(acc, sA, LKb, sB, LKb, cm0, cn0);
-    const float* dT1 = a.dT1 + rec * kC * kC;
     for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
-      acc[mt][nt][e] = j < i ? fmaf(acc[mt][nt][e], sb[j], dT1[i * kC + j]) : 0.f;
+      acc[mt][nt][e] = j < i ? fmaf(acc[mt][nt][e], sb[j], __bfloat162float(sD1[i * LCb + j])) : 0.f;
     });
     acc_to_bf16(acc, sDT, LCb, cm0, cn0);
   }
@@ -2220,10 +2228,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_local_b_bf16_kernel(const Chu
     float acc[TC::MT][TC::NT][4], rp[TC::MT][2] = {};
     zero(acc);
     warp_mma_bf16<TC::MT, TC::NT, kC, true, false>(acc, sT, LCb, sY, LCb, cm0, cn0);
-    const float* P = a.Pkk + rec * kC * kC;
     for_acc<TC::MT, TC::NT>(cm0, cn0, [&](int mt, int nt, int e, int i, int j) {
       const float d = j < i ? -acc[mt][nt][e] : 0.f;
-      rp[mt][e >> 1] = fmaf(d, P[i * kC + j], rp[mt][e >> 1]);
+      rp[mt][e >> 1] = fmaf(d, sPk[i * kLC + j], rp[mt][e >> 1]);
       acc[mt][nt][e] = sb[i] * d;
     });
     acc_to_bf16(acc, sDT, LCb, cm0, cn0);
@@ -2387,9 +2394,9 @@ struct WsPlan {
       : W(f32 ? (size_t)kC * dk : 0), U((size_t)kC * dv), Qp(f32 ? (size_t)kC * dk : 0), Kb(f32 ? (size_t)kC * dk : 0),
         Wt(f32 ? (size_t)kC * dk : 0), Qpt(f32 ? (size_t)kC * dk : 0), Kbt(f32 ? (size_t)kC * dk : 0),
         Aqk(f32 ? kC * kC : 0), prec(f32 ? 0 : (dk == 128 ? PassRec<128>::n : PassRec<64>::n) / 2),
-        // bf16 inputs: T, S0, dS, V', dV', dAqk, dW, dO S0^T and dKbar are kept as bf16 (half the floats)
+        // bf16 inputs: T, S0, dS, V', dV', dAqk, dU (beta V)^T, dW, dO S0^T and dKbar are kept as bf16 (half the floats)
         Tm(kC * kC / (f32 ? 1 : 2)), Pkk(kC * kC), gam(dk), S0c((size_t)dk * dv / (f32 ? 1 : 2)), dSc((size_t)dk * dv / (f32 ? 1 : 2)),
-        Vp((size_t)kC * dv / (f32 ? 1 : 2)), dVp((size_t)kC * dv / (f32 ? 1 : 2)), dAqk(kC * kC / (f32 ? 1 : 2)), dT1(kC * kC), dQs((size_t)kC * dk / (f32 ? 1 : 2)), dW((size_t)kC * dk / (f32 ? 1 : 2)),
+        Vp((size_t)kC * dv / (f32 ? 1 : 2)), dVp((size_t)kC * dv / (f32 ? 1 : 2)), dAqk(kC * kC / (f32 ? 1 : 2)), dT1(kC * kC / (f32 ? 1 : 2)), dQs((size_t)kC * dk / (f32 ? 1 : 2)), dW((size_t)kC * dk / (f32 ? 1 : 2)),
         dKb((size_t)kC * dk / (f32 ? 1 : 2)), dgam(dk), dbu(kC) {}
   size_t per_rec() const {
     return W + U + Qp + Kb + Wt + Qpt + Kbt + Aqk + prec + Tm + Pkk + gam + S0c + dSc + Vp + dVp + dAqk + dT1 + dQs +
@@ -2538,6 +2545,7 @@ cudaError_t launch_chunk_dims(const ChunkBwdArgs& a, int BH, int B, WorkspaceHea
   return launch_chunk_typed<IO, 64, 64>(a, BH, B, hdr, stream);
 }
 
+static_assert(LocalBPlanB<128, 128>::bytes <= 232448 && PrepPlanB<128, 128>::bytes <= 232448, "shared memory per CTA");
 static_assert(prep_smem<128, 128>() <= 232448 && local_a_smem<128, 128>() <= 232448 &&
                   local_b_smem<128, 128>() <= 232448 && pass_smem<128, 128, 64>() <= 232448,
               "shared memory per CTA");
