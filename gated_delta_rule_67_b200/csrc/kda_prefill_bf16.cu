@@ -30,13 +30,14 @@
 //     blocks by forward substitution, the others with warp-level tf32
 //     products), and W^T, U^T with two more MMAs.  It writes, per chunk, a
 //     record of ready-to-use operand images (already in the swizzled
-//     shared-memory layout the MMAs read): [-W ; Q+] (128 x 128), A_qk^T
-//     (64 x 64), Kbar (64 x 128), U^T (128 x 64) and gamma = exp(G_C)
-//     (128 fp32).
+//     shared-memory layout the MMAs read): -W^T (128 key-channel rows x 64
+//     tokens), Q+ (64 token rows x 128), A_qk (64 x 64), Kbar (64 x 128),
+//     U^T (128 x 64) and gamma = exp(G_C) (128 fp32).  In its backward mode
+//     it writes the backward's per-chunk operands instead.
 //  2. kda_state_pass: walks chunks in order with the state S^T (d_v x d_k,
 //     fp32) resident in tensor memory.  Per chunk: S0^T -> bf16 operand;
 //     P = S0^T (-W)^T; V'^T = U^T + P while S^T is decayed by gamma and
-//     O^T = S0^T Q+^T is formed; then [O^T | S^T] += V'^T [A_qk^T | Kbar].
+//     O^T = S0^T Q+^T is formed; then O^T += V'^T A_qk^T and S^T += V'^T Kbar.
 //     The next chunk's record is prefetched with bulk copies while the
 //     current one is processed.  One CTA per (sequence, head), or, when few
 //     chains cover many chunks, the chunk-parallel scan: one CTA per group
@@ -84,7 +85,7 @@ constexpr uint32_t kRecBytes = 74240;
 // staging tile; rows 64-127 ([8K,16K) and [24K,32K)) hold q, then Q+_r.
 // Once the score MMA is done, the v tile takes [8K,16K) and [24K,32K) (a
 // 64-row tile whose channel halves lie 16 KiB apart); its second half comes
-// after the A_qk^T staging tile at [24K,32K) has been bulk-stored.
+// after the A_qk staging tile at [24K,32K) has been bulk-stored.
 // Region B (16 KiB): the k tile, turned in place into K-_r (score B operand);
 // then the 10 A_kk blocks [0,10K) and six T blocks [10K,16K); after the
 // solve the (T diag beta)^T operand [0,8K); finally the U^T staging tile.
@@ -370,7 +371,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       const int i = tg + 16 * t;
       const uint32_t oK = kmajor_off(i, c8, kC);        // 64-row tiles: k, K-_r, Kbar
       const uint32_t oA = kmajor_off(i, c8, 128);       // row i of region A
-      const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A and of the [-W;Q+] image
+      const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A (q, then Q+_r)
       float k8[8], q8[8], Gt[8];
       tmem_ld8(g_tm + 8 * t, Gt);
       ld8(sm + kP1B + oK, k8);
@@ -433,7 +434,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     wait_or_flag(&bar_mma, 0, hdr, 2);
     tc_fence_after();
 
-    // ---- rows 0-63 -> A_kk blocks (times beta_i, strictly lower); rows 64-127 -> A_qk^T staging
+    // ---- rows 0-63 -> A_kk blocks (times beta_i, strictly lower); rows 64-127 -> A_qk staging
     {
       const int row = (warp & 3) * 32 + lane;
       const int col0 = (warp >> 2) * 32;
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
       st8(rec + oRecQ + oK, qp);
       st8(rec + oRecKbar + oK, kb);
     }
-    __syncthreads();  // k and q are read: region B takes the A_kk blocks, [24K,32K) of region A the A_qk^T staging
+    __syncthreads();  // k and q are read: region B takes the A_kk blocks, [24K,32K) of region A the A_qk staging
 #pragma unroll 1
     for (int t = 0; t < 9; ++t) {
       const int p = tid + t * kP1Threads;
@@ -601,7 +602,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     bulk_store(rec + oRecAqk, sm + kP1QT, 8192);
     bulk_commit();
     // Q+_r is dead: bring v while the triangle is inverted, its first
-    // channel half now, the second once the A_qk^T store has read its bytes
+    // channel half now, the second once the A_qk store has read its bytes
     mbar_expect_tx(&bar_v, 16384);
     tma_load_4d(sm + kP1V, &tm_v, &bar_v, 0, h, t0, b);
   }
@@ -771,12 +772,13 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
 // Tensor memory (fp32 unless noted):
 //   [P | O^T | S^T] at [0,64) [64,128) [128,256)
 //   S0^T as bf16 A operand [256,320), V'^T as bf16 A operand [320,352)
-// Three MMA groups per chunk, all A operands read from tensor memory:
-//   P           = S0^T (-W)^T               (N = 64,  K = 128: 8 instructions, committed alone)
-//   O^T         = S0^T Q+^T                 (N = 64,  K = 128: 8 instructions, while V' is formed)
-//   [O^T | S^T] += V'^T [A_qk^T | Kbar]      (N = 192, K = 64:  4 instructions)
+// Four MMA groups per chunk, all A operands read from tensor memory:
+//   P    = S0^T (-W)^T     (N = 64,  K = 128: 8 instructions, committed alone; B = -W^T, MN-major)
+//   O^T  = S0^T Q+^T       (N = 64,  K = 128: 8 instructions, while V' is formed; B = Q+, K-major)
+//   O^T += V'^T A_qk^T     (N = 64,  K = 64:  4 instructions; B = A_qk, K-major)
+//   S^T += V'^T Kbar       (N = 128, K = 64:  4 instructions; B = Kbar, MN-major)
 // with P = -(W S0)^T and V'^T = U^T + P formed on the CUDA cores.  Only P
-// and the last group are on the chain's critical path; the O^T group waits
+// and the S^T update are on the chain's critical path; the O^T groups wait
 // for the output warps to release the previous chunk's O^T off that path.
 constexpr int kSPThreads = 288;
 constexpr uint32_t kTmP = 0, kTmO = 64, kTmS = 128, kTmAS = 256, kTmAV = 320;
@@ -785,8 +787,8 @@ constexpr uint32_t kTmP = 0, kTmO = 64, kTmS = 128, kTmAS = 256, kTmAV = 320;
 // a lighter instance of the same kernel, two CTAs per SM: 192 threads (state
 // warps 0-3, warp 4 streams the records, warp 5 issues the MMAs), 256 columns
 // of tensor memory ([P | S^T | S0^T bf16], V'^T in bf16 written over the P
-// columns it was formed from), compact stages holding only -W (its two
-// 64-channel halves 8 KiB apart), Kbar, U and gamma, and the start state
+// columns it was formed from), compact stages holding only -W^T, Kbar, U
+// and gamma, and the start state
 // read straight from global memory.
 constexpr int kSPThreadsNoOut = 192;
 constexpr uint32_t kTmSNo = 64, kTmASNo = 192;  // P at 0, V'^T bf16 over P's first 32 columns
@@ -796,11 +798,10 @@ constexpr uint32_t kP2BytesNoOut = 2 * kStageNoOut;
 static_assert(kCGamma + 512 <= kStageNoOut, "compact stage");
 
 // Brings the record of one chunk into a stage.  A pass that writes outputs
-// needs all of it; a pass without outputs reads only -W (the first 64 rows
-// of each 64-column block of [-W; Q+]), Kbar, U and gamma; the transition
-// pass (U = 0) not even U.
-constexpr uint32_t kRecNoOutBytes = 2 * 8192 + (kRecBytes - kRecKbar);
-constexpr uint32_t kRecTransBytes = 2 * 8192 + (kRecU - kRecKbar) + (kRecBytes - kRecGamma);
+// needs all of it; a pass without outputs reads only -W^T, Kbar, U and
+// gamma; the transition pass (U = 0) not even U.
+constexpr uint32_t kRecNoOutBytes = (kRecQ - kRecW) + (kRecBytes - kRecKbar);
+constexpr uint32_t kRecTransBytes = (kRecQ - kRecW) + (kRecU - kRecKbar) + (kRecBytes - kRecGamma);
 __device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, uint64_t* bar, bool out,
                                             bool zero_u) {
   if (out) {
@@ -818,9 +819,9 @@ __device__ __forceinline__ void load_record(uint8_t* stage, const uint8_t* rec, 
   }
 }
 
-// The same parts into a compact stage: -W's halves (rows 0-63 of each
-// 64-column block) to [0, 16K), then Kbar, U and gamma, contiguous in the
-// record, to [16K, 48.5K) (U skipped for the transition pass).
+// The same parts into a compact stage: -W^T to [0, 16K), then Kbar, U and
+// gamma, contiguous in the record, to [16K, 48.5K) (U skipped for the
+// transition pass).
 __device__ __forceinline__ void load_record_compact(uint8_t* stage, const uint8_t* rec, uint64_t* bar, bool zero_u) {
   mbar_expect_tx(bar, zero_u ? kRecTransBytes : kRecNoOutBytes);
   bulk_load(stage + kCW, rec + kRecW, kRecQ - kRecW, bar);
