@@ -287,3 +287,22 @@ def test_backward_tensor_core_passes_exact_path():
     ref = oracle.kda_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d ** -0.5, x["initial_state"], d_o, d_s)
     for name in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
         assert rel_err(got[name], ref[name]) < TOL[torch.bfloat16], name
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_backward_empty_sequence(dtype):
+    """T = 0: the token gradients are empty and dL/dS_0 = dL/dS_T (zeros
+    when no final-state gradient is given)."""
+    dev = cuda_or_skip()
+    B, T, H, d = 2, 0, 2, 128
+    x = make_prefill_inputs(B, T, H, d, d, dtype, 0.1, seed=171, device=dev)
+    d_o, d_s = make_cotangents(B, T, H, d, d, dtype, seed=172, device=dev)
+    args = (x["q"], x["k"], x["v"], x["g"], x["beta"], d_o, None, x["initial_state"])
+    got = kda_backward(*args, d_s)
+    torch.cuda.synchronize()
+    for name in ("dq", "dk", "dv", "dg", "dbeta"):
+        assert got[name].numel() == 0, name
+    assert torch.equal(got["dS0"], d_s)
+    got = kda_backward(*args, None)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(got["dS0"]) == 0

@@ -258,3 +258,19 @@ def test_long_chains_light_offset_passes(d, in_place):
     torch.cuda.synchronize()
     assert rel_err(o, ref_o) < TOLB
     assert rel_err(state if in_place else sT, ref_s) < TOLB
+
+
+@pytest.mark.parametrize("B,T", [(2, 0), (0, 64)], ids=["no-tokens", "no-sequences"])
+def test_empty_inputs(B, T):
+    """Nothing to run: the call succeeds without a workspace, o is empty, and
+    the final state is the initial state (or zeros without one)."""
+    dev = cuda_or_skip()
+    H, d = 2, 128
+    x = make_prefill_inputs(B, T, H, d, d, torch.bfloat16, 0.1, seed=170, device=dev)
+    o, sT = kda_chunk_fwd(*(x[n] for n in NAMES), None, x["initial_state"])
+    torch.cuda.synchronize()
+    assert o.shape == (B, T, H, d)
+    assert torch.equal(sT, x["initial_state"])
+    o, sT = kda_chunk_fwd(*(x[n] for n in NAMES), None, None)
+    torch.cuda.synchronize()
+    assert sT.shape == (B, H, d, d) and torch.count_nonzero(sT) == 0
