@@ -376,6 +376,17 @@ def run_ours(args, cfg):
                             "kda_state_pass+scan": {"ms": mean_state,
                                                     "share": mean_state / (mean_prep + mean_state)}},
                 "dominant": dom}
+    # the prep kernel on its own: its algorithmic bytes are its inputs (q, k, v,
+    # the per-channel g and beta); the record it writes is an intermediate
+    prep_bytes = cfg.B * cfg.T * cfg.H * (3 * cfg.dk + cfg.dv + 1) * 2
+    prep_gbs = prep_bytes / (mean_prep / 1e3) / 1e9
+    roofline["dominant_kernel"] = {
+        "name": "kda_chunk_prep", "ms": mean_prep, "algorithmic_bytes": prep_bytes, "achieved": prep_gbs,
+        **hbm_fracs(prep_gbs, peaks),
+        "traffic": None if prof is None else prof.get("prep_bytes_per_launch", {}).get(cfg.name),
+        "scope": "one prep launch: q, k, v, g, beta read (1026 B per token-head at d = 128); CUDA events "
+                 "around it in separate calls; traffic = ncu DRAM bytes of the launch (reads its inputs, "
+                 "writes the 74 KB record per 64-token tile)"}
     tflops = flops / call_s / 1e12
 
     # ---- end to end through the public API: every step copies its inputs from
