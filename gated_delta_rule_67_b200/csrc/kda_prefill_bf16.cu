@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   __shared__ float sbeta[kC];
   __shared__ float sgh[kScalarGate ? kC : 1];  // per-head log-gates of the chunk (zeros without a gate)
   __shared__ float snq[kPrep ? kC : 1], snk[kPrep ? kC : 1];  // per-token sums of q^2, k^2 (fused L2 norm)
-  __shared__ float segr[kD];  // per channel: exp(G_r) (factored form) or 1 (exact path); scales W in its extraction
+  __shared__ __align__(16) float segr[kD];  // per channel: exp(G_r) (factored form) or 1 (exact path); scales W in its extraction
   const bool l2n = kPrep && (prep & KDA_PREP_L2NORM_QK);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -275,123 +275,184 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
   const uint32_t tm = tmem_base;
   wait_or_flag(&bar_in, 0, hdr, 1);
 
-  // ---- pass 1: in-chunk cumulative log-gate.  Thread = (8-channel group cg,
-  // token lane tg) owning tokens tg, tg+16, tg+32, tg+48: the 8 lanes of a
-  // quarter-warp then touch rows of 8 different swizzle phases (no bank
-  // conflicts).  Inclusive scans over the 16 lanes of each token stride,
-  // then the stride totals are added in order.
+  // Thread = (8-channel group cg, token lane tg) in the shuffle-scan form of
+  // pass 1 and the passes after it; thread = (token mi, 16 channels of each
+  // 64-channel half at 16 q4) in the tensor-core form (per-channel gates given
+  // as bf16 log-gates, the KDA case), whose G comes from one product.
+  constexpr bool kMmaScan = !kScalarGate && !kPrep;
   const int cg = 2 * warp + (lane >> 4);
   const int tg = lane & 15;
   const int c8 = 8 * cg;
-  float G[4][8], gref[8], gend[8];
-  if (l2n) {  // per-token sums of squares of q and k over the 128 channels
+  const int mi = 32 * (warp & 1) + lane;
+  const int q4 = 2 * ((warp >> 1) & 1) + (warp >> 2);
+  const uint32_t lane_tm = tm + ((uint32_t)((warp & 3) * 32) << 16);
+  // shuffle-scan form: G parked at columns (warp / 4) * 32 + 8t + e of this lane
+  const uint32_t g_tm = lane_tm + (warp >> 2) * 32;
+  // tensor-core form: accumulator [0,64), the ones operand [64,96), the parked first half [96,128)
+  constexpr uint32_t kTmL = 64, kTmG0 = 96;
+  float* sgref = reinterpret_cast<float*>(sm + kP1T);  // region T, idle until the solve:
+  float* sgend = sgref + kD;                            // G at tokens 31 and 63, exp(G_C - G_r)
+  float* segb = sgref + 2 * kD;
+  float gref[8], gend[8];
+  int slow;
+  if constexpr (kMmaScan) {
+    // ---- pass 1 (tensor cores): G = L g with L the 64 x 64 lower-triangular
+    // matrix of ones as the A operand in tensor memory (rows 64-127 repeat
+    // rows 0-63, so that the lanes of every warp hold tokens) and the g tile
+    // as the MN-major B operand, one 64-channel half at a time.  The products
+    // are exact (g is bf16, L is 0 or 1) and the sums fp32.
+    if (warp < 4) {
+      uint32_t lw[32];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int i = tg + 16 * t;
-      float q8[8], k8[8];
-      ld8(sm + kP1A + kmajor_off(kC + i, c8, 128), q8);
-      ld8(sm + kP1B + kmajor_off(i, c8, kC), k8);
-      float sq2 = 0.f, sk2 = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        sq2 = fmaf(q8[e], q8[e], sq2);
-        sk2 = fmaf(k8[e], k8[e], sk2);
-      }
-      atomicAdd(&snq[i], sq2);
-      atomicAdd(&snk[i], sk2);
+      for (int e = 0; e < 32; ++e)
+        lw[e] = (2 * e <= mi ? 0x3F80u : 0u) | (2 * e + 1 <= mi ? 0x3F800000u : 0u);  // bf16 1.0 pairs
+      tmem_st32u(lane_tm + kTmL, lw);
+      tmem_wait_st();
     }
-  }
-  if (!kScalarGate) {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+#pragma unroll 1
+    for (int hf = 0; hf < 2; ++hf) {
+      if (tid == 0) {
+        const uint32_t idesc = idesc_bf16_f32(128, 64, 0, 1);
+        const uint64_t b0 = desc_sw128(smem_u32(sm + kP1A + hf * 16384), 16384, 1024);
 #pragma unroll
-    for (int t = 0; t < 4; ++t) ld8(sm + kP1A + kmajor_off(tg + 16 * t, c8, 128), G[t]);
-    if (kPrep && (prep & KDA_PREP_GATE_LOGSIGMOID)) {
+        for (int k = 0; k < kC / 16; ++k)
+          mma_bf16_ts(tm, tm + kTmL + k * 8, b0 + (uint64_t)((k * 2048) >> 4), idesc, k > 0);
+        mma_commit(&bar_mma);
+      }
+      wait_or_flag(&bar_mma, hf, hdr, 5 + hf);
+      tc_fence_after();
+      float Gq[16];
+      tmem_ld16(lane_tm + 16 * q4, Gq);
+      if (lane == 31) {  // tokens 31 (the reference) and 63 (the chunk end)
+        float4* dst = reinterpret_cast<float4*>(((warp & 1) ? sgend : sgref) + 64 * hf + 16 * q4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = make_float4(Gq[4 * e], Gq[4 * e + 1], Gq[4 * e + 2], Gq[4 * e + 3]);
+      }
+      if (hf == 0) {  // the first half waits in this lane's spare columns; the accumulator takes the second
+        tmem_st16(lane_tm + kTmG0 + 16 * (warp >> 2), Gq);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+      }
+    }
+    __syncthreads();  // G at tokens 31 and 63 is in shared memory
+    if (tid < kC) sbeta[tid] = beta_x;
+    bool unsafe = false;
+    if (tid < kD) {
+      const float gr = sgref[tid], ge = sgend[tid];
+      unsafe = ge < -kSafeSpan;
+      segr[tid] = __expf(gr);
+      segb[tid] = __expf(ge - gr);
+      (kBwd ? bo.gam + ri * kD : reinterpret_cast<float*>(rec + kRecGamma))[tid] = expf(ge);
+    }
+    slow = __syncthreads_or(unsafe);  // the g tile is dead from here on
+  } else {
+    // ---- pass 1: in-chunk cumulative log-gate.  Thread = (8-channel group cg,
+    // token lane tg) owning tokens tg, tg+16, tg+32, tg+48: the 8 lanes of a
+    // quarter-warp then touch rows of 8 different swizzle phases (no bank
+    // conflicts).  Inclusive scans over the 16 lanes of each token stride,
+    // then the stride totals are added in order.
+    float G[4][8];
+    if (l2n) {  // per-token sums of squares of q and k over the 128 channels
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int i = tg + 16 * t;
+        float q8[8], k8[8];
+        ld8(sm + kP1A + kmajor_off(kC + i, c8, 128), q8);
+        ld8(sm + kP1B + kmajor_off(i, c8, kC), k8);
+        float sq2 = 0.f, sk2 = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          sq2 = fmaf(q8[e], q8[e], sq2);
+          sk2 = fmaf(k8[e], k8[e], sk2);
+        }
+        atomicAdd(&snq[i], sq2);
+        atomicAdd(&snk[i], sk2);
+      }
+    }
+    if (!kScalarGate) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) ld8(sm + kP1A + kmajor_off(tg + 16 * t, c8, 128), G[t]);
+      if (kPrep && (prep & KDA_PREP_GATE_LOGSIGMOID)) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) G[t][e] = tg + 16 * t < L ? log_sigmoid_fast(G[t][e]) : 0.f;  // padding: no decay
+      }
+    } else {  // one log-gate per token for every channel (zero without a gate)
 #pragma unroll
       for (int t = 0; t < 4; ++t)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) G[t][e] = tg + 16 * t < L ? log_sigmoid_fast(G[t][e]) : 0.f;  // padding: no decay
+        for (int e = 0; e < 8; ++e) G[t][e] = sgh[tg + 16 * t];
     }
-  } else {  // one log-gate per token for every channel (zero without a gate)
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) G[t][e] = sgh[tg + 16 * t];
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    float tot[4];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      float x = G[t][e];
-#pragma unroll
-      for (int d = 1; d < 16; d <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, d, 16);
-        if (tg >= d) x += y;
-      }
-      G[t][e] = x;
-      tot[t] = __shfl_sync(0xffffffffu, x, 15, 16);
-    }
-    G[1][e] += tot[0];
-    G[2][e] += tot[0] + tot[1];
-    G[3][e] += (tot[0] + tot[1]) + tot[2];
-    gref[e] = tot[0] + tot[1];                 // G at token 31
-    gend[e] = ((tot[0] + tot[1]) + tot[2]) + tot[3];  // G at token 63 (= G_C; padding has g = 0)
-  }
-  // G goes to tensor memory until the decayed operands are formed (held in
-  // registers across that stretch it would spill to local memory): thread
-  // (warp, lane) keeps its 32 values in its own lane (warp % 4) * 32 + lane,
-  // columns (warp / 4) * 32 + 8t + e.  The score MMA overwrites them later.
-  const uint32_t g_tm = tm + ((uint32_t)((warp & 3) * 32) << 16) + (warp >> 2) * 32;
-  tmem_st32(g_tm, &G[0][0]);
-  tmem_wait_st();
-  if (tid < kC) sbeta[tid] = (kPrep && tid < L) ? prep_beta(prep, beta_x) : beta_x;
-  bool unsafe = false;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) unsafe |= gend[e] < -kSafeSpan;
-  if (tg == 0) {
-    float* gam = (kBwd ? bo.gam + ri * kD : reinterpret_cast<float*>(rec + kRecGamma)) + c8;
-    *reinterpret_cast<float4*>(gam) = make_float4(expf(gend[0]), expf(gend[1]), expf(gend[2]), expf(gend[3]));
-    *reinterpret_cast<float4*>(gam + 4) = make_float4(expf(gend[4]), expf(gend[5]), expf(gend[6]), expf(gend[7]));
-  }
-  const int slow = __syncthreads_or(unsafe);  // the g tile is dead from here on
-
-  if (!slow) {
-    // ---- pass 2 (factored form): decayed operands relative to token kRefTok
-    float egr[8], egb[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      egr[e] = __expf(gref[e]);
-      egb[e] = __expf(gend[e] - gref[e]);
-    }
-    if (tg == 0) {
+      float tot[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) segr[c8 + e] = egr[e];
-    }
+      for (int t = 0; t < 4; ++t) {
+        float x = G[t][e];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int i = tg + 16 * t;
-      const uint32_t oK = kmajor_off(i, c8, kC);        // 64-row tiles: k, K-_r, Kbar
-      const uint32_t oA = kmajor_off(i, c8, 128);       // row i of region A
-      const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A (q, then Q+_r)
-      float k8[8], q8[8], Gt[8];
-      tmem_ld8(g_tm + 8 * t, Gt);
-      ld8(sm + kP1B + oK, k8);
-      ld8(sm + kP1A + oQ, q8);
-      if (l2n) {
-        const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          k8[e] *= rk;
-          q8[e] *= rq;
+        for (int d = 1; d < 16; d <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, x, d, 16);
+          if (tg >= d) x += y;
         }
+        G[t][e] = x;
+        tot[t] = __shfl_sync(0xffffffffu, x, 15, 16);
       }
-      // the start-decayed operands first, then the end-decayed ones, so that
-      // fewer values are live at once (64 registers at 4 CTAs per SM)
-      float w[8];
-      {
-        float ex[8];
+      G[1][e] += tot[0];
+      G[2][e] += tot[0] + tot[1];
+      G[3][e] += (tot[0] + tot[1]) + tot[2];
+      gref[e] = tot[0] + tot[1];                 // G at token 31
+      gend[e] = ((tot[0] + tot[1]) + tot[2]) + tot[3];  // G at token 63 (= G_C; padding has g = 0)
+    }
+    // G goes to tensor memory until the decayed operands are formed (held in
+    // registers across that stretch it would spill to local memory): thread
+    // (warp, lane) keeps its 32 values in its own lane (warp % 4) * 32 + lane,
+    // columns (warp / 4) * 32 + 8t + e.  The score MMA overwrites them later.
+    tmem_st32(g_tm, &G[0][0]);
+    tmem_wait_st();
+    if (tid < kC) sbeta[tid] = (kPrep && tid < L) ? prep_beta(prep, beta_x) : beta_x;
+    bool unsafe = false;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) unsafe |= gend[e] < -kSafeSpan;
+    if (tg == 0) {
+      float* gam = (kBwd ? bo.gam + ri * kD : reinterpret_cast<float*>(rec + kRecGamma)) + c8;
+      *reinterpret_cast<float4*>(gam) = make_float4(expf(gend[0]), expf(gend[1]), expf(gend[2]), expf(gend[3]));
+      *reinterpret_cast<float4*>(gam + 4) = make_float4(expf(gend[4]), expf(gend[5]), expf(gend[6]), expf(gend[7]));
+    }
+    slow = __syncthreads_or(unsafe);  // the g tile is dead from here on
+
+  }
+
+  if (!slow) {
+    if constexpr (kMmaScan) {
+      // ---- pass 2 (factored form), token mi and four 8-channel pieces: the
+      // decayed operands relative to token kRefTok.  Each (token, piece) slot
+      // of the k, q and g tiles belongs to one thread, read before it is
+      // overwritten; the per-channel factors come from shared memory.
+#pragma unroll 1
+      for (int p = 0; p < 4; ++p) {
+        const int hf = p >> 1, c = 64 * hf + 16 * q4 + 8 * (p & 1);
+        float Gt[8], f8[8], k8[8], q8[8], w[8], ex[8];
+        tmem_ld8(hf == 0 ? lane_tm + kTmG0 + 16 * (warp >> 2) + 8 * (p & 1) : lane_tm + 16 * q4 + 8 * (p & 1), Gt);
+        const uint32_t oK = kmajor_off(mi, c, kC);        // 64-row tiles: k, K-_r, Kbar, the Q+ image
+        const uint32_t oA = kmajor_off(mi, c, 128);       // row mi of region A
+        const uint32_t oQ = kmajor_off(kC + mi, c, 128);  // row 64+mi of region A (q, then Q+_r)
+        ld8(sm + kP1B + oK, k8);
+        ld8(sm + kP1A + oQ, q8);
+        auto ld8f = [](const float* src, float* f) {  // 8 per-channel factors, two 16-byte loads
+          const float4 a0 = *reinterpret_cast<const float4*>(src), a1 = *reinterpret_cast<const float4*>(src + 4);
+          f[0] = a0.x, f[1] = a0.y, f[2] = a0.z, f[3] = a0.w, f[4] = a1.x, f[5] = a1.y, f[6] = a1.z, f[7] = a1.w;
+        };
+        ld8f(sgref + c, f8);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          ex[e] = __expf(Gt[e] - gref[e]);
+          Gt[e] -= f8[e];  // G - G_r
+          ex[e] = __expf(Gt[e]);
           q8[e] *= scale;
         }
 #pragma unroll
@@ -400,20 +461,81 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = q8[e] * ex[e];
         st8(sm + kP1A + oQ, w);               // Q+_r (in place of q)
+        ld8f(segr + c, f8);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * egr[e]);
-        st8(rec + oRecQ + oK, w);             // Q+ image (64 token rows, the layout of the k tile)
-      }
-      {
-        float ei[8];
+        for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * f8[e]);
+        st8(rec + oRecQ + oK, w);             // Q+ image
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ei[e] = __expf(gref[e] - Gt[e]);
+        for (int e = 0; e < 8; ++e) ex[e] = __expf(-Gt[e]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) w[e] = k8[e] * ei[e];
+        for (int e = 0; e < 8; ++e) w[e] = k8[e] * ex[e];
         st8(sm + kP1B + oK, w);               // K-_r, in place of k
+        ld8f(segb + c, f8);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ei[e] * egb[e]);
+        for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ex[e] * f8[e]);
         st8(rec + oRecKbar + oK, w);          // Kbar image = k exp(G_C - G_i)
+      }
+    } else {
+      // ---- pass 2 (factored form): decayed operands relative to token kRefTok
+      float egr[8], egb[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        egr[e] = __expf(gref[e]);
+        egb[e] = __expf(gend[e] - gref[e]);
+      }
+      if (tg == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) segr[c8 + e] = egr[e];
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int i = tg + 16 * t;
+        const uint32_t oK = kmajor_off(i, c8, kC);        // 64-row tiles: k, K-_r, Kbar
+        const uint32_t oA = kmajor_off(i, c8, 128);       // row i of region A
+        const uint32_t oQ = kmajor_off(kC + i, c8, 128);  // row 64+i of region A (q, then Q+_r)
+        float k8[8], q8[8], Gt[8];
+        tmem_ld8(g_tm + 8 * t, Gt);
+        ld8(sm + kP1B + oK, k8);
+        ld8(sm + kP1A + oQ, q8);
+        if (l2n) {
+          const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            k8[e] *= rk;
+            q8[e] *= rq;
+          }
+        }
+        // the start-decayed operands first, then the end-decayed ones, so that
+        // fewer values are live at once (64 registers at 4 CTAs per SM)
+        float w[8];
+        {
+          float ex[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            ex[e] = __expf(Gt[e] - gref[e]);
+            q8[e] *= scale;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = k8[e] * ex[e];
+          st8(sm + kP1A + oA, w);               // K+_r (over the dead g rows)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = q8[e] * ex[e];
+          st8(sm + kP1A + oQ, w);               // Q+_r (in place of q)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = q8[e] * (ex[e] * egr[e]);
+          st8(rec + oRecQ + oK, w);             // Q+ image (64 token rows, the layout of the k tile)
+        }
+        {
+          float ei[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ei[e] = __expf(gref[e] - Gt[e]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = k8[e] * ei[e];
+          st8(sm + kP1B + oK, w);               // K-_r, in place of k
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = k8[e] * (ei[e] * egb[e]);
+          st8(rec + oRecKbar + oK, w);          // Kbar image = k exp(G_C - G_i)
+        }
       }
     }
     fence_async_smem();
@@ -496,7 +618,12 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     for (int t = 0; t < 9; ++t) akk[t] = aqk[t] = 0.f;
 #pragma unroll 1
     for (int hf = 0; hf < 2; ++hf) {
-      if ((c8 >> 6) == hf) {
+      if constexpr (kMmaScan) {
+        float Gq[16];
+        tmem_ld16(hf == 0 ? lane_tm + kTmG0 + 16 * (warp >> 2) : lane_tm + 16 * q4, Gq);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) *gp(mi, 16 * q4 + e) = Gq[e];
+      } else if ((c8 >> 6) == hf) {
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           float Gt[8];
@@ -534,37 +661,64 @@ __global__ void __launch_bounds__(kP1Threads, kP1Blocks)
     // pass 2 (exact): start- and end-decayed operands, factors <= 1; K+ goes
     // over the dead g rows of region A (where the factored form keeps K+_r),
     // with a unit W scale
-    if (tg == 0) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) segr[c8 + e] = 1.f;
-    }
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int i = tg + 16 * t;
-      const uint32_t oK = kmajor_off(i, c8, kC);
-      const uint32_t oQ = kmajor_off(kC + i, c8, 128);
-      float k8[8], q8[8], kp[8], qp[8], kb[8], Gt[8];
-      tmem_ld8(g_tm + 8 * t, Gt);
-      ld8(sm + kP1B + oK, k8);
-      ld8(sm + kP1A + oQ, q8);
-      if (l2n) {
-        const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
+    if constexpr (kMmaScan) {
+      if (tid < kD) segr[tid] = 1.f;
+#pragma unroll 1
+      for (int p = 0; p < 4; ++p) {
+        const int hf = p >> 1, c = 64 * hf + 16 * q4 + 8 * (p & 1);
+        float Gt[8], ge[8], k8[8], q8[8], kp[8], qp[8], kb[8];
+        tmem_ld8(hf == 0 ? lane_tm + kTmG0 + 16 * (warp >> 2) + 8 * (p & 1) : lane_tm + 16 * q4 + 8 * (p & 1), Gt);
+        const uint32_t oK = kmajor_off(mi, c, kC);
+        ld8(sm + kP1B + oK, k8);
+        ld8(sm + kP1A + kmajor_off(kC + mi, c, 128), q8);
+        {
+          const float4 a0 = *reinterpret_cast<const float4*>(sgend + c), a1 = *reinterpret_cast<const float4*>(sgend + c + 4);
+          ge[0] = a0.x, ge[1] = a0.y, ge[2] = a0.z, ge[3] = a0.w, ge[4] = a1.x, ge[5] = a1.y, ge[6] = a1.z, ge[7] = a1.w;
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          k8[e] *= rk;
-          q8[e] *= rq;
+          const float e0 = __expf(Gt[e]);
+          kp[e] = k8[e] * e0;
+          qp[e] = scale * q8[e] * e0;
+          kb[e] = k8[e] * __expf(ge[e] - Gt[e]);
         }
+        st8(sm + kP1A + kmajor_off(mi, c, 128), kp);
+        st8(rec + oRecQ + oK, qp);
+        st8(rec + oRecKbar + oK, kb);
+      }
+    } else {
+      if (tg == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) segr[c8 + e] = 1.f;
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float e0 = __expf(Gt[e]);
-        kp[e] = k8[e] * e0;
-        qp[e] = scale * q8[e] * e0;
-        kb[e] = k8[e] * __expf(gend[e] - Gt[e]);
+      for (int t = 0; t < 4; ++t) {
+        const int i = tg + 16 * t;
+        const uint32_t oK = kmajor_off(i, c8, kC);
+        const uint32_t oQ = kmajor_off(kC + i, c8, 128);
+        float k8[8], q8[8], kp[8], qp[8], kb[8], Gt[8];
+        tmem_ld8(g_tm + 8 * t, Gt);
+        ld8(sm + kP1B + oK, k8);
+        ld8(sm + kP1A + oQ, q8);
+        if (l2n) {
+          const float rk = rsqrtf(snk[i] + kL2Eps), rq = rsqrtf(snq[i] + kL2Eps);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            k8[e] *= rk;
+            q8[e] *= rq;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float e0 = __expf(Gt[e]);
+          kp[e] = k8[e] * e0;
+          qp[e] = scale * q8[e] * e0;
+          kb[e] = k8[e] * __expf(gend[e] - Gt[e]);
+        }
+        st8(sm + kP1A + kmajor_off(i, c8, 128), kp);
+        st8(rec + oRecQ + oK, qp);
+        st8(rec + oRecKbar + oK, kb);
       }
-      st8(sm + kP1A + kmajor_off(i, c8, 128), kp);
-      st8(rec + oRecQ + oK, qp);
-      st8(rec + oRecKbar + oK, kb);
     }
     __syncthreads();  // k and q are read: region B takes the A_kk blocks, [24K,32K) of region A the A_qk staging
 #pragma unroll 1
