@@ -29,15 +29,20 @@
 // Four launches per group of (sequence, head) pairs (as many as the workspace
 // holds), the last three chained to the one before by programmatic dependent
 // launch:
-//   1. bwd_prep    (chunk, seq x head): W, U, Q+, Kbar, Aqk, P, T, gamma per chunk
+//   1. bwd_prep    (chunk, seq x head): W, U, Q+, Kbar, Aqk, P, T, gamma per
+//      chunk; for bf16 at d_k = d_v = 128 from 16 (sequence, head) pairs on,
+//      the prefill's tcgen05 preparation kernel in its backward mode
 //   2. bwd_pass    (seq x head x column slice, 2 roles): the forward state
 //      replay (checkpoints S0 and V' per chunk) and the reverse dS sweep
 //      (dS and dV' per chunk, dL/dS_0); the columns of the state evolve
-//      independently in both
+//      independently in both; with the tcgen05 preparation, one CTA per
+//      (sequence, head) and role on the tcgen05 tensor cores, the state in
+//      tensor memory
 //   3. bwd_local_a (chunk, seq x head): the products contracting over d_v:
 //      dAqk, dT (first part), dv, dbeta (first part), dO S0^T, dW, dKbar, dgamma
 //   4. bwd_local_b (chunk, seq x head): the rest, and dq, dk, dg, dbeta
-// Arithmetic: warp-level tensor-core products (mma.sync), fp32 accumulation.
+// Arithmetic of the per-chunk kernels here: warp-level tensor-core products
+// (mma.sync), fp32 accumulation.
 // fp32 inputs: fp32 shared tiles, m16n8k8 with tf32 operands in the
 // three-term split (a_hi b_hi + a_hi b_lo + a_lo b_hi), which keeps fp32-level
 // accuracy; fp32 workspace.  bf16 inputs: bf16 operand images (ldmatrix, with
