@@ -207,8 +207,10 @@ KDA_API size_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, 
  * alignment); outputs must not overlap any input, each other or the
  * workspace.  Every sum runs in a fixed order (no atomics), so results are
  * bit-reproducible.  T = 0 or B = 0 is valid
- * (grad_initial_state = grad_final_state).  For bf16 at dk = dv = 128 the
- * state passes run on the tcgen05 tensor cores with bounded mbarrier waits;
+ * (grad_initial_state = grad_final_state).  For bf16 at dk = dv = 128 with
+ * at least 16 (sequence, head) pairs in a group, the per-chunk operands come
+ * from the prefill's preparation kernel and the state passes run on the
+ * tcgen05 tensor cores, both with bounded mbarrier waits;
  * kda_chunk_fwd_check(workspace, ...) afterwards returns KDA_ERR_TIMEOUT if
  * one gave up (the gradients are then not valid), KDA_OK otherwise.
  */
