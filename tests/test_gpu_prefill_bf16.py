@@ -274,3 +274,20 @@ def test_empty_inputs(B, T):
     o, sT = kda_chunk_fwd(*(x[n] for n in NAMES), None, None)
     torch.cuda.synchronize()
     assert sT.shape == (B, H, d, d) and torch.count_nonzero(sT) == 0
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 200, 2), (1, 64 * 13 + 5, 2)], ids=["one-pass", "scan"])
+def test_no_writes_pure_decay(B, T, H):
+    """beta = 0: nothing is written, the state only decays channel by channel,
+    S_T = Diag(exp(sum_t g_t)) S0 and o_t = scale (Diag(exp(sum_{s<=t} g_s)) S0)^T q_t;
+    against the oracle and against that closed form for the final state."""
+    dev = cuda_or_skip()
+    x = make_prefill_inputs(B, T, H, 128, 128, torch.bfloat16, 0.1, seed=173 + T, device="cpu")
+    x["beta"] = torch.zeros_like(x["beta"])
+    o, sT = _run(x, dev)
+    ref_o, ref_s = _oracle(x)
+    assert rel_err(o, ref_o) < TOLB
+    assert rel_err(sT, ref_s) < TOLB
+    decay = torch.exp(x["g"].double().sum(dim=1))             # [B, H, dk]
+    closed = decay.unsqueeze(-1) * x["initial_state"].double()  # Diag(alpha) S0, per key channel
+    assert rel_err(sT, closed) < TOLB
