@@ -1011,6 +1011,11 @@ struct StatePassArgs {
   float* mbuf;      // transition matrices: [B*H][G] slots of 64 KiB, each the 32 KiB bf16 K-major image of M_g
   float* sbuf;
   int T, H, NC, G, L, phase, dk, dv;
+  // phase 3 launches may cover groups [g_first, g_first + g_count) only (0: all);
+  // s0_direct: group 0 reads the caller's initial state itself; dep_wait = 0:
+  // no wait for the previous grid (its inputs were complete before that grid
+  // could be scheduled); trigger: let the next grid be scheduled early
+  int g_first, g_count, s0_direct, dep_wait, trigger;
 };
 
 template <bool kOut>
@@ -1067,14 +1072,20 @@ __global__ void __launch_bounds__(kOut ? kSPThreads : kSPThreadsNoOut, kOut ? 1 
     cb = g * L;
     ce = min(NC, cb + L);
   } else {
-    bh = blockIdx.x / G;
-    const int g = blockIdx.x % G;
+    const int gn = args.g_count > 0 ? args.g_count : G;
+    bh = blockIdx.x / gn;
+    const int g = args.g_first + blockIdx.x % gn;
     cb = g * L;
     ce = min(NC, cb + L);
-    // group 0 starts from the initial state (its copy in sbuf slot 0), group 1
-    // from R_0; later ones from the combination kernel's output
-    init = g == 0 ? (args.s0 ? args.sbuf + (size_t)bh * G * kSt : nullptr)
-                  : g == 1 ? args.rbuf + (size_t)bh * G * kSt : args.sbuf + ((size_t)bh * G + g) * kSt;
+    // group 0 starts from the initial state (the caller's, or its copy in sbuf
+    // slot 0), group 1 from R_0; later ones from the combination kernel's output
+    if (g == 0 && args.s0_direct) {
+      init = args.s0 ? args.s0 + bh * kUserSt : nullptr;
+      init_user = true;
+    } else {
+      init = g == 0 ? (args.s0 ? args.sbuf + (size_t)bh * G * kSt : nullptr)
+                    : g == 1 ? args.rbuf + (size_t)bh * G * kSt : args.sbuf + ((size_t)bh * G + g) * kSt;
+    }
     fin = (g == G - 1 && args.sT) ? args.sT + bh * kUserSt : nullptr;
     fin_user = true;
   }
@@ -1086,7 +1097,7 @@ __global__ void __launch_bounds__(kOut ? kSPThreads : kSPThreadsNoOut, kOut ? 1 
   // (and no tensor memory, which that kernel's CTAs may still be allocating)
   // is touched before it has finished.
   if (tid == 0) prefetch_tensormap(&tm_o);
-  grid_dep_wait();
+  if (args.dep_wait) grid_dep_wait();
   if (tid == 0) {
     mbar_init(&bar_full[0], 1);
     mbar_init(&bar_full[1], 1);
@@ -1109,7 +1120,7 @@ __global__ void __launch_bounds__(kOut ? kSPThreads : kSPThreadsNoOut, kOut ? 1 
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
-  if (args.phase == 1) grid_dep_launch();  // the combination kernel may be scheduled
+  if (args.phase == 1 || args.trigger) grid_dep_launch();  // the next kernel may be scheduled
 
   if (warp == kMmaWarp) {
     // ------------------------------------------------------------ mma
@@ -1556,13 +1567,19 @@ constexpr int kScanMinChunks = 4;
 // steps and launches (measured: 134 vs 77 us of state passes at B1 H16
 // T4096 with 8 groups of 8 chunks instead of 6 of 11).
 constexpr int kScanLongChunks = 256;
-void scan_groups(int BH, int NC, int* G_out, int* L_out, bool* light = nullptr) {
+// Long chains whose final state does not overwrite the initial state also run
+// the output pass of group 0 (which needs nothing from the scan) beside the
+// light offset/transition passes, on the SMs those leave free: one more group
+// then fits, with the other G - 1 output passes still one wave.
+void scan_groups(int BH, int NC, int* G_out, int* L_out, bool* light = nullptr, bool early0 = false) {
   int G = 1;
   bool lt = false;
   if (BH > 0 && 3 * BH <= kScanSMs) {
     G = std::min((kScanSMs / BH + 3) / 2, NC / kScanMinChunks);
     if (G >= 3 && NC / G >= kScanLongChunks) {
-      G = std::min(std::min(kScanSMs / BH, (2 * kScanSMs / BH + 3) / 2), NC / kScanMinChunks);
+      G = early0 ? std::min(kScanSMs / BH + 1, (2 * (kScanSMs - BH) / BH + 3) / 2)
+                 : std::min(kScanSMs / BH, (2 * kScanSMs / BH + 3) / 2);
+      G = std::min(G, NC / kScanMinChunks);
       lt = true;
     }
   }
@@ -1604,6 +1621,9 @@ size_t prefill_bf16_workspace_bytes(int B, int T, int H, int dk, int dv, int chu
   const int NC = (int)(((size_t)T + kC - 1) / kC);
   int G, L;
   scan_groups(B * H, NC, &G, &L);
+  int G2, L2;
+  scan_groups(B * H, NC, &G2, &L2, nullptr, true);  // the schedule with group 0's outputs early
+  G = std::max(G, G2);
   const size_t scan = G > 1 ? 3 * (size_t)B * H * G * kD * kD * sizeof(float) : 0;
   return sizeof(WorkspaceHeader) + (size_t)B * H * NC * kRecBytes + scan;
 }
@@ -1647,8 +1667,13 @@ cudaError_t launch_prep_for_backward(const bf16* q, const bf16* k, const bf16* v
 int prefill_bf16_launches(int B, int T, int H) {
   const int NC = (int)(((size_t)T + kC - 1) / kC);
   int G, L;
-  scan_groups(B * H, NC, &G, &L);
-  return G > 1 ? 4 : 2;
+  bool light = false;
+  scan_groups(B * H, NC, &G, &L, &light, true);
+  if (G == 1) return 2;
+  // long chains: prep, group 0's output pass, offset/transition passes,
+  // combination, the other output passes (4 launches when the final state
+  // overwrites the initial state: group 0's outputs then follow the scan)
+  return light ? 5 : 4;
 }
 
 cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, const bf16* g, const bf16* beta,
@@ -1709,11 +1734,13 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
   e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 1, stream);
   if (e != cudaSuccess) return e;
-  StatePassArgs a{records, hdr, s0, sT, nullptr, nullptr, nullptr, T, H, NC, 1, NC, 0, dk, dv};
+  StatePassArgs a{records, hdr, s0, sT, nullptr, nullptr, nullptr, T, H, NC, 1, NC, 0, dk, dv, 0, 0, 0, 1, 0};
   const int BH = B * H;
   int G, L;
   bool light = false;
-  scan_groups(BH, NC, &G, &L, &light);
+  const bool in_place = s0 != nullptr && (const void*)s0 == (const void*)sT;
+  scan_groups(BH, NC, &G, &L, &light, !in_place);
+  const bool early0 = light && !in_place && G > 1;
   if (G == 1) {
     e = launch_dependent(kda_state_pass_kernel<true>, (unsigned)BH, kSPThreads, kP2Bytes + 1024, stream, mo, a);
   } else {
@@ -1724,17 +1751,30 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     a.sbuf = scan + 2 * per;
     a.G = G;
     a.L = L;
+    if (early0) {
+      // group 0's output pass first: it waits for the prep, then lets the
+      // offset/transition passes be scheduled beside it; those need no wait
+      // (the prep had finished before any CTA of this grid passed its wait)
+      a.phase = 3;
+      a.g_first = 0, a.g_count = 1, a.s0_direct = 1, a.trigger = 1;
+      e = launch_dependent(kda_state_pass_kernel<true>, (unsigned)BH, kSPThreads, kP2Bytes + 1024, stream, mo, a);
+      if (e != cudaSuccess) return e;
+      a.g_count = 0, a.s0_direct = 0, a.trigger = 0, a.dep_wait = 0;
+    }
     a.phase = 1;
     e = light ? launch_dependent(kda_state_pass_kernel<false>, (unsigned)(BH * (2 * G - 3)), kSPThreadsNoOut,
                                  kP2BytesNoOut + 1024, stream, mo, a)
               : launch_dependent(kda_state_pass_kernel<true>, (unsigned)(BH * (2 * G - 3)), kSPThreads,
                                  kP2Bytes + 1024, stream, mo, a);
     if (e != cudaSuccess) return e;
+    a.dep_wait = 1;
     e = launch_dependent(kda_scan_combine_kernel, (unsigned)BH, kCbThreads, kCbSmem, stream, scan + 2 * per,
                          (const float*)scan, (const float*)(scan + per), G, hdr);
     if (e != cudaSuccess) return e;
     a.phase = 3;
-    e = launch_dependent(kda_state_pass_kernel<true>, (unsigned)(BH * G), kSPThreads, kP2Bytes + 1024, stream, mo, a);
+    if (early0) a.g_first = 1, a.g_count = G - 1;
+    e = launch_dependent(kda_state_pass_kernel<true>, (unsigned)(BH * (early0 ? G - 1 : G)), kSPThreads,
+                         kP2Bytes + 1024, stream, mo, a);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e == cudaSuccess) e = mark(events, 2, stream);
