@@ -1752,12 +1752,15 @@ cudaError_t launch_prefill_bf16(const bf16* q, const bf16* k, const bf16* v, con
     a.G = G;
     a.L = L;
     if (early0) {
-      // group 0's output pass first: it waits for the prep, then lets the
-      // offset/transition passes be scheduled beside it; those need no wait
-      // (the prep had finished before any CTA of this grid passed its wait)
+      // group 0's output pass first, launched in plain stream order (with a
+      // programmatic launch its CTAs took SMs in the prep's last wave and
+      // waited there: 31.8 vs 30.9 ms per call at T = 1,048,576); it lets the
+      // offset/transition passes be scheduled beside it, and those need no
+      // wait (the prep had finished before this grid started)
       a.phase = 3;
       a.g_first = 0, a.g_count = 1, a.s0_direct = 1, a.trigger = 1;
-      e = launch_dependent(kda_state_pass_kernel<true>, (unsigned)BH, kSPThreads, kP2Bytes + 1024, stream, mo, a);
+      kda_state_pass_kernel<true><<<(unsigned)BH, kSPThreads, kP2Bytes + 1024, stream>>>(mo, a);
+      e = cudaGetLastError();
       if (e != cudaSuccess) return e;
       a.g_count = 0, a.s0_direct = 0, a.trigger = 0, a.dep_wait = 0;
     }
