@@ -104,8 +104,11 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
  * (the workspace-header clear, a memset, is not counted): 1 for the fp32
  * path; for bf16 the chunk preparation plus either one state pass or, when
  * few (sequence, head) chains cover many chunks, the three launches of the
- * chunk-parallel scan.  0 when there is nothing to run (B or T zero), -1 for
- * arguments kda_chunk_fwd would reject.  Pure host arithmetic.
+ * chunk-parallel scan, or four for long chains (group 0's output pass runs
+ * as its own launch beside the scan; three again when final_state is the
+ * initial state's buffer, which this query does not see).  0 when there is
+ * nothing to run (B or T zero), -1 for arguments kda_chunk_fwd would reject.
+ * Pure host arithmetic.
  */
 KDA_API int kda_chunk_fwd_launch_count(int B, int T, int H, int dk, int dv, int chunk, int dtype);
 

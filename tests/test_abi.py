@@ -123,6 +123,7 @@ def test_launch_count(lib):
     assert f(1, 64, 1, 128, 128, 64, 1) == 2        # prep + one state pass
     assert f(1, 4096, 16, 128, 128, 64, 1) == 4     # few chains, many chunks: chunk-parallel scan
     assert f(8, 8192, 32, 128, 128, 64, 1) == 2     # many chains: one state pass
+    assert f(1, 1 << 20, 32, 128, 128, 64, 1) == 5  # long chains: group 0's outputs as a launch of their own
     assert f(1, 256, 2, 64, 64, 64, 0) == 1         # fp32 path
     assert f(0, 64, 1, 128, 128, 64, 1) == 0
     assert f(1, 64, 1, 96, 96, 64, 1) == -1
