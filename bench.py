@@ -63,6 +63,12 @@ def prefill_bytes(B, T, H, dk, dv, elem=2, state_in=True, state_out=True) -> flo
     return B * T * H * per_tok + st * (int(state_in) + int(state_out))
 
 
+def prep_input_bytes(B, T, H, dk, dv, elem=2) -> float:
+    """Algorithmic bytes of the prep kernel alone: its inputs q, k, the
+    per-channel g, v and beta (the record it writes is an intermediate)."""
+    return B * T * H * (3 * dk + dv + 1) * elem
+
+
 def backward_bytes(B, T, H, dk, dv, elem=2) -> float:
     """Algorithmic HBM bytes of one backward call: q, k, g, v, beta, dL/do read;
     dq, dk, dg, dv, dbeta written; S0 and dL/dS_T read, dL/dS0 written (fp32)."""
@@ -378,7 +384,7 @@ def run_ours(args, cfg):
                 "dominant": dom}
     # the prep kernel on its own: its algorithmic bytes are its inputs (q, k, v,
     # the per-channel g and beta); the record it writes is an intermediate
-    prep_bytes = cfg.B * cfg.T * cfg.H * (3 * cfg.dk + cfg.dv + 1) * 2
+    prep_bytes = prep_input_bytes(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv)
     prep_gbs = prep_bytes / (mean_prep / 1e3) / 1e9
     roofline["dominant_kernel"] = {
         "name": "kda_chunk_prep", "ms": mean_prep, "algorithmic_bytes": prep_bytes, "achieved": prep_gbs,

@@ -22,6 +22,8 @@ def test_accounting_matches_hand_count():
     assert bench.prefill_bytes(1, 1, 1, 128, 128, 2, False, False) == 1282
     assert bench.prefill_bytes(1, 0, 1, 128, 128, 2, True, True) == 2 * 128 * 128 * 4
     assert bench.decode_bytes(256, 32, 128, 128) == 256 * 32 * (2 * 65536 + 1282)
+    # the prep kernel alone reads q, k, g, v and beta: 1282 B less the 256 B of o
+    assert bench.prep_input_bytes(1, 1, 1, 128, 128) == 1026
 
 
 def _free_port():
